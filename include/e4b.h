@@ -1,0 +1,240 @@
+/*
+ * e4b.h -- C ABI of libe4b: the routed Mixture-of-Experts expert layer run
+ * directly on NF4-packed fused expert stacks, on one NVIDIA B200 (sm_100a).
+ *
+ * The operations follow the pages this library is written from:
+ *   - fused stacks gate_up_proj [E, 2I, H] and down_proj [E, H, I]
+ *     ("Why does load_in_4bit still OOM on a Mixture-of-Experts model?",
+ *     section "Why it happens");
+ *   - 4-bit NF4 storage with blocks of 64 that never cross an expert boundary
+ *     (same page, "Which project solves it"; experts4bit-qlora 0.22.0,
+ *     "Install": the fast path takes NF4 with blocksize 64 only);
+ *   - sorting token/expert pairs into per-expert groups (experts4bit-qlora
+ *     0.22.0, "Which training path?");
+ *   - one grouped GEMM launch that decodes the nibbles in registers with fp32
+ *     accumulation and materialises no bf16 expert tensor (Solutions -- one
+ *     page per problem, the grouped-nf4-gemm row on gemm_4bit_grouped);
+ *   - the SwiGLU expert MLP ("Scope") and the per-expert LoRA delta added
+ *     before the activation (Solutions page, the ExpertsLoRA row; r=8,
+ *     alpha=16 in "Quickstart").
+ *
+ * Conventions for every call
+ *   - Pointers to tensors are DEVICE pointers unless a comment says otherwise.
+ *     The caller allocates and owns every buffer, workspaces included; the
+ *     library never allocates, frees or synchronises on these calls.
+ *   - Tensors are contiguous, row-major and 16-byte aligned (base address),
+ *     except where a leading dimension is passed.
+ *   - bf16 data is passed as raw 16-bit patterns (uint16_t).
+ *   - Calls are stream-ordered on `stream` (a cudaStream_t; NULL is the legacy
+ *     default stream).  No call reads device data back to the host, so every
+ *     call can be captured in a CUDA graph.
+ *   - Arguments are checked on the host before anything is launched.  A bad
+ *     argument returns E4B_ERR_INVALID_ARGUMENT, a shape or device the kernels
+ *     do not support returns E4B_ERR_UNSUPPORTED, a workspace that is too small
+ *     returns E4B_ERR_WORKSPACE, and a failed launch returns E4B_ERR_CUDA.
+ *     e4b_last_error() then names the argument or the CUDA error.  Nothing
+ *     falls back silently to another path: the path that ran is reported by
+ *     e4b_last_path().
+ *   - Device data that breaks a documented invariant (offsets that are not
+ *     non-decreasing, indices out of range) cannot be checked on the host; the
+ *     kernels clamp such values so that no access leaves the buffers, and the
+ *     affected outputs are unspecified.
+ */
+#ifndef E4B_H_
+#define E4B_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define E4B_VERSION 1
+
+#if defined(__GNUC__)
+#define E4B_API __attribute__((visibility("default")))
+#else
+#define E4B_API
+#endif
+
+typedef enum {
+  E4B_OK = 0,
+  E4B_ERR_INVALID_ARGUMENT = 1,
+  E4B_ERR_UNSUPPORTED = 2, /* shape, dtype or device (not sm_100) */
+  E4B_ERR_WORKSPACE = 3,   /* workspace smaller than the size query returns */
+  E4B_ERR_CUDA = 4         /* a CUDA runtime call or a launch failed */
+} e4b_status;
+
+typedef enum { E4B_F32 = 0, E4B_BF16 = 1 } e4b_dtype;
+
+typedef enum {
+  E4B_EPI_NONE = 0,  /* out = A_rows . W^T                                  */
+  E4B_EPI_SWIGLU = 1 /* y = A_rows . W^T (+ LoRA); out = SiLU(y[:, :N/2]) * y[:, N/2:] */
+} e4b_epilogue;
+
+/* Which implementation e4b_moe_expert_forward_path() runs. */
+typedef enum {
+  E4B_PATH_AUTO = 0,    /* small token counts -> DECODE, otherwise GROUPED */
+  E4B_PATH_DECODE = 1,  /* fused split-row GEMV over the touched experts only */
+  E4B_PATH_GROUPED = 2  /* grouped tensor-core GEMMs + combine */
+} e4b_path;
+
+typedef struct CUstream_st* e4b_stream; /* identical to cudaStream_t */
+
+/* Human-readable name of a status code (static string). */
+E4B_API const char* e4b_status_string(e4b_status s);
+
+/* Detail of the last failing call on this host thread ("" if none). */
+E4B_API const char* e4b_last_error(void);
+
+/* Name of the kernel path the last successful call on this host thread
+ * launched, e.g. "quantize", "route.small", "gemm.tc", "forward.decode". */
+E4B_API const char* e4b_last_path(void);
+
+/* E4B_VERSION of the built library. */
+E4B_API int e4b_version(void);
+
+/* Number of kernels the last call on this host thread launched. */
+E4B_API int e4b_last_launches(void);
+
+/*
+ * Kernel timing for benchmarks and profiling (host thread local).
+ * e4b_timing_enable(1) clears earlier records and, until e4b_timing_enable(0),
+ * brackets every kernel the library launches on this thread with a pair of
+ * CUDA events recorded on the launch stream (events are created on first use
+ * and reused).  e4b_timing_kernels() counts the distinct kernel names
+ * recorded; e4b_timing_get(i, ...) waits for the events of kernel name i and
+ * returns its total elapsed milliseconds and launch count.  Not for use inside
+ * a CUDA graph capture.
+ */
+E4B_API e4b_status e4b_timing_enable(int on);
+E4B_API int e4b_timing_kernels(void);
+E4B_API e4b_status e4b_timing_get(int i, const char** name, double* total_ms, int* launches);
+
+/*
+ * a1 -- NF4 quantisation of a fused expert stack.
+ * Source: "Why does load_in_4bit still OOM on a Mixture-of-Experts model?",
+ * "Which project solves it" (blocks never cross an expert boundary).
+ *
+ * W        [E, N, K] row-major, fp32 (w_dtype E4B_F32) or bf16 (E4B_BF16).
+ * packed   [E, N*K/2] uint8 out.  Each expert is flattened row-major and cut
+ *          into blocks of 64 consecutive elements; byte j holds the codes of
+ *          elements 2j (high nibble) and 2j+1 (low nibble).
+ * absmax   [E, N*K/64] fp32 out: the largest |w| of each block.
+ * Each code is the nearest entry of the 16-entry NF4 codebook (QLoRA table,
+ * ascending, entry 7 = 0) to s = w / absmax computed as one IEEE fp32
+ * division; a value exactly between two entries takes the lower index; an
+ * all-zero block stores absmax 0 and code 7.  Bit-exact by construction.
+ * Requires blocksize == 64, E >= 1, N >= 1, K >= 1, (N*K) % 64 == 0.
+ * Non-finite inputs give unspecified codes (no fault).
+ */
+E4B_API e4b_status e4b_nf4_quantize_stack(const void* W, e4b_dtype w_dtype, int64_t E, int64_t N,
+                                  int64_t K, int blocksize, uint8_t* packed, float* absmax,
+                                  e4b_stream stream);
+
+/*
+ * a2 + a3 -- router top-k and the token/expert permutation.
+ * Source: experts4bit-qlora 0.22.0, "Which training path?" (sort the
+ * token/expert pairs, run the groups); routing "softmax top-k renormalised".
+ *
+ * logits          [M, E] fp32.
+ * topk_ids        [M, k] int32 out: per token, experts ordered by (logit
+ *                 descending, index ascending); slot j = the j-th.
+ * topk_w          [M, k] fp32 out: renormalize != 0: softmax over the k
+ *                 selected logits; renormalize == 0: the full softmax over E
+ *                 evaluated at the selected experts.
+ * expert_offsets  [E+1] int32 out: first permuted position of each expert;
+ *                 expert_offsets[E] = M*k.
+ * perm            [M*k] int32 out: flat slots f = t*k + j in a stable sort
+ *                 by expert id.
+ * inv_perm        [M*k] int32 out: inv_perm[perm[p]] = p.
+ * workspace       device scratch of e4b_moe_route_permute_workspace_size()
+ *                 bytes (may be NULL when that size is 0).
+ * Requires M >= 0, 1 <= E <= 1024, 1 <= k <= min(E, 32).  M == 0 writes only
+ * expert_offsets (all zero).  ids and perm are bit-exact; weights use expf.
+ * NaN logits give unspecified (in-range) ids.
+ */
+E4B_API size_t e4b_moe_route_permute_workspace_size(int64_t M, int64_t E, int k);
+E4B_API e4b_status e4b_moe_route_permute(const float* logits, int64_t M, int64_t E, int k,
+                                 int renormalize, int32_t* topk_ids, float* topk_w,
+                                 int32_t* expert_offsets, int32_t* perm, int32_t* inv_perm,
+                                 void* workspace, size_t workspace_bytes, e4b_stream stream);
+
+/*
+ * a4..a7 -- one grouped GEMM over E expert groups on NF4-packed weights.
+ * Source: Solutions -- one page per problem, the grouped-nf4-gemm row
+ * (gemm_4bit_grouped: one launch, nibbles decoded in registers, fp32
+ * accumulation).
+ *
+ * Row p (0 <= p < total_rows) belongs to the group e with
+ * expert_offsets[e] <= p < expert_offsets[e+1] and computes
+ *     y[p, :] = A[row_index[p], :] . W_e^T                      (N values)
+ *     y[p, :] += lora_scale * (A[row_index[p], :] . lora_A[e]^T) . lora_B[e]^T
+ * where W_e = codebook[q] * absmax is expert e's [N, K] NF4 matrix.
+ *
+ * A               [a_rows, lda] bf16 (lda >= K, in elements, lda % 8 == 0).
+ * row_index       [total_rows] int32 indices into A, or NULL for p itself.
+ * expert_offsets  [E+1] int32, non-decreasing, expert_offsets[E] == total_rows.
+ * packed, absmax  [E, N*K/2] uint8 and [E, N*K/64] fp32 (e4b_nf4_quantize_stack).
+ * lora_A, lora_B  [E, r, K] and [E, N, r] bf16, or both NULL (no adapter).
+ * epi             E4B_EPI_NONE: out[p, n] = y[p, n], n < N.
+ *                 E4B_EPI_SWIGLU: out[p, n] = SiLU(y[p, n]) * y[p, N/2 + n],
+ *                 n < N/2 (gate = first half of the rows, up = second half).
+ * out             [total_rows, N or N/2] of out_dtype.
+ * Requires K % 64 == 0, N % 64 == 0, 0 <= r <= 16, total_rows < 2^31.
+ * workspace       e4b_grouped_nf4_gemm_workspace_size() bytes.
+ * Groups with no rows cost nothing and write nothing.
+ */
+E4B_API size_t e4b_grouped_nf4_gemm_workspace_size(int64_t total_rows, int64_t N, int64_t K, int r);
+E4B_API e4b_status e4b_grouped_nf4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda,
+                                const int32_t* row_index, const int32_t* expert_offsets,
+                                int64_t E, int64_t total_rows, const uint8_t* packed,
+                                const float* absmax, int64_t N, int64_t K,
+                                const uint16_t* lora_A, const uint16_t* lora_B, int r,
+                                float lora_scale, e4b_epilogue epi, void* out,
+                                e4b_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                                e4b_stream stream);
+
+/* The two packed stacks of one MoE layer (device pointers), plus its adapter. */
+typedef struct {
+  const uint8_t* gu_packed; /* [E, 2I*H/2]  gate_up_proj, NF4 */
+  const float* gu_absmax;   /* [E, 2I*H/64] */
+  const uint8_t* dn_packed; /* [E, H*I/2]   down_proj, NF4 */
+  const float* dn_absmax;   /* [E, H*I/64] */
+  const uint16_t* lora_A;   /* [E, r, H] bf16 or NULL */
+  const uint16_t* lora_B;   /* [E, 2I, r] bf16 or NULL */
+  int lora_r;               /* 0 without an adapter */
+  float lora_alpha;         /* scale = lora_alpha / lora_r */
+  int64_t E, H, I;
+} e4b_expert_stack;
+
+/*
+ * a2..a8 -- the routed expert layer end to end:
+ *     out[t] = sum_j w[t,j] * ( SiLU(g) * u ) . Wd_e^T,  [g | u] = x_t . Wgu_e^T (+ LoRA)
+ * with (e, w[t,j]) from the top-k routing of router_logits[t].
+ * Sources: as for the three calls above; the weighted sum over a token's
+ * experts is the combine of experts4bit-qlora 0.22.0, "Which training path?".
+ *
+ * x [M, H] bf16, router_logits [M, E] fp32, out [M, H] bf16.
+ * Requires H % 64 == 0, I % 64 == 0, 1 <= k <= min(E, 32), E <= 1024.
+ * workspace  e4b_moe_expert_forward_workspace_size() bytes (covers both paths).
+ * The sum over a token's k experts is taken in a fixed order for a given path,
+ * so results are deterministic run to run.
+ */
+E4B_API size_t e4b_moe_expert_forward_workspace_size(int64_t M, const e4b_expert_stack* w, int k);
+E4B_API e4b_status e4b_moe_expert_forward(const uint16_t* x, int64_t M, const float* router_logits,
+                                  int k, int renormalize, const e4b_expert_stack* w,
+                                  uint16_t* out, void* workspace, size_t workspace_bytes,
+                                  e4b_stream stream);
+/* Same, with the implementation chosen explicitly (tests and benchmarks). */
+E4B_API e4b_status e4b_moe_expert_forward_path(const uint16_t* x, int64_t M, const float* router_logits,
+                                       int k, int renormalize, const e4b_expert_stack* w,
+                                       uint16_t* out, void* workspace, size_t workspace_bytes,
+                                       e4b_path path, e4b_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* E4B_H_ */

@@ -1,0 +1,456 @@
+// The extern "C" boundary of libe4b: argument checks, workspace layout, launches.
+//
+// Every call validates its arguments on the host before launching anything
+// and reports failures through a status code plus a per-thread message; no
+// call allocates, frees or synchronises.  See include/e4b.h for the contract.
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "e4b_internal.h"
+
+namespace e4b {
+
+namespace {
+thread_local std::string g_error;
+thread_local const char* g_path = "";
+thread_local int g_launches = 0;
+
+struct TimingRec {
+  const char* name;
+  cudaEvent_t start, stop;
+};
+struct TimingState {
+  bool on = false;
+  std::vector<TimingRec> recs;
+  std::vector<cudaEvent_t> pool;  // events reused across enable cycles
+  size_t pool_used = 0;
+  cudaEvent_t take() {
+    if (pool_used == pool.size()) {
+      cudaEvent_t ev;
+      if (cudaEventCreate(&ev) != cudaSuccess) return nullptr;
+      pool.push_back(ev);
+    }
+    return pool[pool_used++];
+  }
+};
+thread_local TimingState g_timing;
+
+constexpr size_t kAlign = 256;
+
+struct Carve {
+  size_t off = 0;
+  size_t take(size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, kAlign);
+    return o;
+  }
+};
+
+// Workspace of the grouped forward path.
+struct GroupedLayout {
+  size_t ids, w, offsets, perm, inv, row_token, route_ws, xa, h, z, total;
+};
+
+GroupedLayout grouped_layout(int64_t M, int64_t E, int64_t H, int64_t I, int k, int r) {
+  const int64_t S = M * k;
+  Carve c;
+  GroupedLayout L;
+  L.ids = c.take(S * sizeof(int32_t));
+  L.w = c.take(S * sizeof(float));
+  L.offsets = c.take((E + 1) * sizeof(int32_t));
+  L.perm = c.take(S * sizeof(int32_t));
+  L.inv = c.take(S * sizeof(int32_t));
+  L.row_token = c.take(S * sizeof(int32_t));
+  L.route_ws = c.take(route_workspace_bytes(M, E, k));
+  L.xa = c.take(r > 0 ? S * r * sizeof(float) : 0);
+  L.h = c.take(S * I * sizeof(uint16_t));
+  L.z = c.take(S * H * sizeof(float));
+  L.total = c.off;
+  return L;
+}
+
+template <typename T>
+T* at(void* base, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(base) + off);
+}
+
+e4b_status fail(e4b_status s, const std::string& msg) {
+  g_error = msg;
+  return s;
+}
+
+e4b_status cuda_fail(cudaError_t err, const char* where) {
+  g_error = std::string(where) + ": " + cudaGetErrorName(err) + " (" + cudaGetErrorString(err) + ")";
+  return E4B_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+e4b_status check_device() {
+  DeviceInfo di;
+  const cudaError_t err = device_info(&di);
+  if (err != cudaSuccess) return cuda_fail(err, "device query");
+  if (di.major != 10 || di.minor != 0)
+    return fail(E4B_ERR_UNSUPPORTED, "libe4b is built for sm_100a (B200); current device is sm_" +
+                                         std::to_string(di.major) + std::to_string(di.minor));
+  return E4B_OK;
+}
+
+std::string shape_str(const char* name, int64_t v) { return std::string(name) + "=" + std::to_string(v); }
+
+}  // namespace
+
+void set_error(const std::string& msg) { g_error = msg; }
+void set_path(const char* path) { g_path = path; }
+void begin_call() {
+  g_launches = 0;
+  g_error.clear();
+}
+
+LaunchScope::LaunchScope(const char* name, cudaStream_t stream) : rec_(-1), stream_(stream) {
+  ++g_launches;
+  if (!g_timing.on) return;
+  TimingRec r{name, g_timing.take(), g_timing.take()};
+  if (!r.start || !r.stop) return;
+  if (cudaEventRecord(r.start, stream) != cudaSuccess) return;
+  g_timing.recs.push_back(r);
+  rec_ = static_cast<int>(g_timing.recs.size()) - 1;
+}
+
+LaunchScope::~LaunchScope() {
+  if (rec_ >= 0) cudaEventRecord(g_timing.recs[rec_].stop, stream_);
+}
+
+cudaError_t device_info(DeviceInfo* out) {
+  static std::mutex mu;
+  static std::vector<DeviceInfo> cache;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    for (const auto& d : cache)
+      if (d.device == dev) {
+        *out = d;
+        return cudaSuccess;
+      }
+  }
+  DeviceInfo d{};
+  d.device = dev;
+  int v = 0;
+  if ((err = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
+  d.sm_count = v;
+  if ((err = cudaDeviceGetAttribute(&v, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess) return err;
+  d.major = v;
+  if ((err = cudaDeviceGetAttribute(&v, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess) return err;
+  d.minor = v;
+  if ((err = cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return err;
+  d.smem_optin = static_cast<size_t>(v);
+  std::lock_guard<std::mutex> lk(mu);
+  cache.push_back(d);
+  *out = d;
+  return cudaSuccess;
+}
+
+cudaError_t launch_lora_xa(const GemmArgs& a, cudaStream_t stream);
+
+}  // namespace e4b
+
+using namespace e4b;
+
+extern "C" {
+
+const char* e4b_status_string(e4b_status s) {
+  switch (s) {
+    case E4B_OK: return "E4B_OK";
+    case E4B_ERR_INVALID_ARGUMENT: return "E4B_ERR_INVALID_ARGUMENT";
+    case E4B_ERR_UNSUPPORTED: return "E4B_ERR_UNSUPPORTED";
+    case E4B_ERR_WORKSPACE: return "E4B_ERR_WORKSPACE";
+    case E4B_ERR_CUDA: return "E4B_ERR_CUDA";
+  }
+  return "E4B_ERR_UNKNOWN";
+}
+
+const char* e4b_last_error(void) { return g_error.c_str(); }
+const char* e4b_last_path(void) { return g_path; }
+int e4b_version(void) { return E4B_VERSION; }
+int e4b_last_launches(void) { return g_launches; }
+
+e4b_status e4b_timing_enable(int on) {
+  g_timing.on = on != 0;
+  g_timing.recs.clear();
+  g_timing.pool_used = 0;
+  return E4B_OK;
+}
+
+int e4b_timing_kernels(void) {
+  std::vector<const char*> names;
+  for (const auto& r : g_timing.recs)
+    if (std::find_if(names.begin(), names.end(), [&](const char* n) { return std::strcmp(n, r.name) == 0; }) ==
+        names.end())
+      names.push_back(r.name);
+  return static_cast<int>(names.size());
+}
+
+e4b_status e4b_timing_get(int i, const char** name, double* total_ms, int* launches) {
+  std::vector<const char*> names;
+  for (const auto& r : g_timing.recs)
+    if (std::find_if(names.begin(), names.end(), [&](const char* n) { return std::strcmp(n, r.name) == 0; }) ==
+        names.end())
+      names.push_back(r.name);
+  if (i < 0 || i >= static_cast<int>(names.size()) || !name || !total_ms || !launches)
+    return fail(E4B_ERR_INVALID_ARGUMENT, "timing index out of range or null output");
+  double ms = 0.0;
+  int n = 0;
+  for (const auto& r : g_timing.recs) {
+    if (std::strcmp(r.name, names[i]) != 0) continue;
+    cudaError_t err = cudaEventSynchronize(r.stop);
+    if (err != cudaSuccess) return cuda_fail(err, "timing event sync");
+    float t = 0.f;
+    err = cudaEventElapsedTime(&t, r.start, r.stop);
+    if (err != cudaSuccess) return cuda_fail(err, "timing elapsed");
+    ms += t;
+    ++n;
+  }
+  *name = names[i];
+  *total_ms = ms;
+  *launches = n;
+  return E4B_OK;
+}
+
+e4b_status e4b_nf4_quantize_stack(const void* W, e4b_dtype w_dtype, int64_t E, int64_t N, int64_t K,
+                                  int blocksize, uint8_t* packed, float* absmax, e4b_stream stream) {
+  begin_call();
+  if (blocksize != 64) return fail(E4B_ERR_UNSUPPORTED, "blocksize must be 64, got " + std::to_string(blocksize));
+  if (w_dtype != E4B_F32 && w_dtype != E4B_BF16) return fail(E4B_ERR_INVALID_ARGUMENT, "w_dtype must be F32 or BF16");
+  if (E < 1 || N < 1 || K < 1)
+    return fail(E4B_ERR_INVALID_ARGUMENT, "E, N, K must be >= 1 (" + shape_str("E", E) + ", " + shape_str("N", N) +
+                                              ", " + shape_str("K", K) + ")");
+  if ((N * K) % 64 != 0) return fail(E4B_ERR_UNSUPPORTED, "N*K must be a multiple of 64 (blocks stay inside an expert)");
+  if (!W || !packed || !absmax) return fail(E4B_ERR_INVALID_ARGUMENT, "null pointer (W, packed or absmax)");
+  if (!aligned16(W) || !aligned16(packed) || !aligned16(absmax))
+    return fail(E4B_ERR_INVALID_ARGUMENT, "W, packed and absmax must be 16-byte aligned");
+  if (e4b_status s = check_device(); s != E4B_OK) return s;
+  const int64_t nblocks = E * N * K / 64;
+  cudaError_t err = launch_quantize(W, w_dtype == E4B_BF16, nblocks, packed, absmax, stream);
+  if (err != cudaSuccess) return cuda_fail(err, "quantize launch");
+  set_path("quantize");
+  return E4B_OK;
+}
+
+size_t e4b_moe_route_permute_workspace_size(int64_t M, int64_t E, int k) {
+  if (M < 0 || E < 1 || k < 1) return 0;
+  return route_workspace_bytes(M, E, k);
+}
+
+e4b_status e4b_moe_route_permute(const float* logits, int64_t M, int64_t E, int k, int renormalize,
+                                 int32_t* topk_ids, float* topk_w, int32_t* expert_offsets, int32_t* perm,
+                                 int32_t* inv_perm, void* workspace, size_t workspace_bytes, e4b_stream stream) {
+  begin_call();
+  if (M < 0) return fail(E4B_ERR_INVALID_ARGUMENT, "M must be >= 0");
+  if (E < 1 || E > 1024) return fail(E4B_ERR_UNSUPPORTED, "E must be in [1, 1024], got " + std::to_string(E));
+  if (k < 1 || k > E || k > 32) return fail(E4B_ERR_INVALID_ARGUMENT, "k must be in [1, min(E, 32)]");
+  if (M * k > INT32_MAX) return fail(E4B_ERR_UNSUPPORTED, "M*k exceeds int32 slot indices");
+  if (!expert_offsets) return fail(E4B_ERR_INVALID_ARGUMENT, "null expert_offsets");
+  if (M > 0 && (!logits || !topk_ids || !topk_w || !perm || !inv_perm))
+    return fail(E4B_ERR_INVALID_ARGUMENT, "null pointer (logits, topk_ids, topk_w, perm or inv_perm)");
+  const size_t need = route_workspace_bytes(M, E, k);
+  if (workspace_bytes < need || (need > 0 && !workspace))
+    return fail(E4B_ERR_WORKSPACE, "route workspace needs " + std::to_string(need) + " bytes");
+  if (e4b_status s = check_device(); s != E4B_OK) return s;
+  RouteOut o{topk_ids, topk_w, expert_offsets, perm, inv_perm, nullptr};
+  cudaError_t err = launch_route(logits, M, static_cast<int>(E), k, renormalize != 0, o, workspace, stream);
+  if (err != cudaSuccess) return cuda_fail(err, "route launch");
+  if (M == 0) set_path("route.empty");
+  return E4B_OK;
+}
+
+size_t e4b_grouped_nf4_gemm_workspace_size(int64_t total_rows, int64_t N, int64_t K, int r) {
+  (void)N;
+  (void)K;
+  if (total_rows < 0 || r < 0) return 0;
+  return gemm_workspace_bytes(total_rows, r);
+}
+
+e4b_status e4b_grouped_nf4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda, const int32_t* row_index,
+                                const int32_t* expert_offsets, int64_t E, int64_t total_rows, const uint8_t* packed,
+                                const float* absmax, int64_t N, int64_t K, const uint16_t* lora_A,
+                                const uint16_t* lora_B, int r, float lora_scale, e4b_epilogue epi, void* out,
+                                e4b_dtype out_dtype, void* workspace, size_t workspace_bytes, e4b_stream stream) {
+  begin_call();
+  if (E < 1 || E > 65536) return fail(E4B_ERR_INVALID_ARGUMENT, "E must be in [1, 65536]");
+  if (total_rows < 0 || a_rows < 0) return fail(E4B_ERR_INVALID_ARGUMENT, "total_rows and a_rows must be >= 0");
+  if (total_rows > 0 && a_rows < 1) return fail(E4B_ERR_INVALID_ARGUMENT, "a_rows must be >= 1 when rows exist");
+  if (K < 64 || K % 64 != 0) return fail(E4B_ERR_UNSUPPORTED, "K must be a positive multiple of 64");
+  if (N < 64 || N % 64 != 0) return fail(E4B_ERR_UNSUPPORTED, "N must be a positive multiple of 64");
+  if (lda < K || lda % 8 != 0) return fail(E4B_ERR_INVALID_ARGUMENT, "lda must be >= K and a multiple of 8");
+  if (epi != E4B_EPI_NONE && epi != E4B_EPI_SWIGLU) return fail(E4B_ERR_INVALID_ARGUMENT, "unknown epilogue");
+  if (out_dtype != E4B_F32 && out_dtype != E4B_BF16) return fail(E4B_ERR_INVALID_ARGUMENT, "out_dtype must be F32 or BF16");
+  if ((lora_A == nullptr) != (lora_B == nullptr))
+    return fail(E4B_ERR_INVALID_ARGUMENT, "lora_A and lora_B must be both set or both NULL");
+  if (lora_A && (r < 1 || r > 16)) return fail(E4B_ERR_UNSUPPORTED, "LoRA rank must be in [1, 16]");
+  if (!lora_A) r = 0;
+  if (!expert_offsets || !packed || !absmax) return fail(E4B_ERR_INVALID_ARGUMENT, "null expert_offsets, packed or absmax");
+  if (total_rows > 0 && (!A || !out)) return fail(E4B_ERR_INVALID_ARGUMENT, "null A or out");
+  if (total_rows > INT32_MAX) return fail(E4B_ERR_UNSUPPORTED, "total_rows exceeds int32");
+  if ((A && !aligned16(A)) || !aligned16(packed) || (out && !aligned16(out)))
+    return fail(E4B_ERR_INVALID_ARGUMENT, "A, packed and out must be 16-byte aligned");
+  const size_t need = gemm_workspace_bytes(total_rows, r);
+  if (workspace_bytes < need || (need > 0 && !workspace))
+    return fail(E4B_ERR_WORKSPACE, "gemm workspace needs " + std::to_string(need) + " bytes");
+  if (e4b_status s = check_device(); s != E4B_OK) return s;
+  if (total_rows == 0) {
+    set_path("gemm.empty");
+    return E4B_OK;
+  }
+  GemmArgs g{};
+  g.A = A;
+  g.a_rows = a_rows;
+  g.lda = lda;
+  g.row_index = row_index;
+  g.offsets = expert_offsets;
+  g.E = static_cast<int>(E);
+  g.total_rows = total_rows;
+  g.packed = packed;
+  g.absmax = absmax;
+  g.N = static_cast<int>(N);
+  g.K = static_cast<int>(K);
+  g.lora_A = lora_A;
+  g.lora_B = lora_B;
+  g.r = r;
+  g.lora_scale = lora_scale;
+  g.xa = r > 0 ? static_cast<float*>(workspace) : nullptr;
+  g.epi = epi;
+  g.out = out;
+  g.out_bf16 = out_dtype == E4B_BF16;
+  const char* path = "";
+  cudaError_t err = launch_grouped_gemm(g, stream, &path);
+  if (err != cudaSuccess) return cuda_fail(err, "grouped gemm launch");
+  set_path(path);
+  return E4B_OK;
+}
+
+static e4b_status check_stack(const e4b_expert_stack* w, int k) {
+  if (!w) return fail(E4B_ERR_INVALID_ARGUMENT, "null expert stack");
+  if (w->E < 1 || w->E > 1024) return fail(E4B_ERR_UNSUPPORTED, "E must be in [1, 1024]");
+  if (w->H < 64 || w->H % 64 != 0) return fail(E4B_ERR_UNSUPPORTED, "H must be a positive multiple of 64");
+  if (w->I < 64 || w->I % 64 != 0) return fail(E4B_ERR_UNSUPPORTED, "I must be a positive multiple of 64");
+  if (k < 1 || k > w->E || k > 32) return fail(E4B_ERR_INVALID_ARGUMENT, "k must be in [1, min(E, 32)]");
+  if (!w->gu_packed || !w->gu_absmax || !w->dn_packed || !w->dn_absmax)
+    return fail(E4B_ERR_INVALID_ARGUMENT, "null packed stack pointer");
+  if ((w->lora_A == nullptr) != (w->lora_B == nullptr))
+    return fail(E4B_ERR_INVALID_ARGUMENT, "lora_A and lora_B must be both set or both NULL");
+  if (w->lora_A && (w->lora_r < 1 || w->lora_r > 16)) return fail(E4B_ERR_UNSUPPORTED, "LoRA rank must be in [1, 16]");
+  if (!aligned16(w->gu_packed) || !aligned16(w->dn_packed) || !aligned16(w->gu_absmax) || !aligned16(w->dn_absmax))
+    return fail(E4B_ERR_INVALID_ARGUMENT, "packed stacks and absmax must be 16-byte aligned");
+  return E4B_OK;
+}
+
+static int stack_r(const e4b_expert_stack* w) { return w->lora_A ? w->lora_r : 0; }
+
+size_t e4b_moe_expert_forward_workspace_size(int64_t M, const e4b_expert_stack* w, int k) {
+  if (!w || M <= 0 || k < 1) return 0;
+  const size_t g = grouped_layout(M, w->E, w->H, w->I, k, stack_r(w)).total;
+  const size_t d = decode_workspace_bytes(M, w->E, k, w->H, w->I, stack_r(w));
+  return g > d ? g : d;
+}
+
+static e4b_status forward_grouped(const uint16_t* x, int64_t M, const float* logits, int k, int renormalize,
+                                  const e4b_expert_stack* w, uint16_t* out, void* ws, cudaStream_t stream) {
+  const int r = stack_r(w);
+  const GroupedLayout L = grouped_layout(M, w->E, w->H, w->I, k, r);
+  RouteOut o{at<int32_t>(ws, L.ids), at<float>(ws, L.w), at<int32_t>(ws, L.offsets),
+             at<int32_t>(ws, L.perm), at<int32_t>(ws, L.inv), at<int32_t>(ws, L.row_token)};
+  cudaError_t err = launch_route(logits, M, static_cast<int>(w->E), k, renormalize != 0, o,
+                                 at<void>(ws, L.route_ws), stream);
+  if (err != cudaSuccess) return cuda_fail(err, "route launch");
+  const int64_t S = M * k;
+  GemmArgs g{};
+  g.A = x;
+  g.a_rows = M;
+  g.lda = w->H;
+  g.row_index = o.row_token;
+  g.offsets = o.offsets;
+  g.E = static_cast<int>(w->E);
+  g.total_rows = S;
+  g.packed = w->gu_packed;
+  g.absmax = w->gu_absmax;
+  g.N = static_cast<int>(2 * w->I);
+  g.K = static_cast<int>(w->H);
+  g.lora_A = r ? w->lora_A : nullptr;
+  g.lora_B = r ? w->lora_B : nullptr;
+  g.r = r;
+  g.lora_scale = r ? w->lora_alpha / static_cast<float>(r) : 0.0f;
+  g.xa = r ? at<float>(ws, L.xa) : nullptr;
+  g.epi = E4B_EPI_SWIGLU;
+  g.out = at<uint16_t>(ws, L.h);
+  g.out_bf16 = true;
+  const char* p1 = "";
+  if ((err = launch_grouped_gemm(g, stream, &p1)) != cudaSuccess) return cuda_fail(err, "gate_up gemm launch");
+  GemmArgs d{};
+  d.A = at<uint16_t>(ws, L.h);
+  d.a_rows = S;
+  d.lda = w->I;
+  d.row_index = nullptr;
+  d.offsets = o.offsets;
+  d.E = static_cast<int>(w->E);
+  d.total_rows = S;
+  d.packed = w->dn_packed;
+  d.absmax = w->dn_absmax;
+  d.N = static_cast<int>(w->H);
+  d.K = static_cast<int>(w->I);
+  d.epi = E4B_EPI_NONE;
+  d.out = at<float>(ws, L.z);
+  d.out_bf16 = false;
+  const char* p2 = "";
+  if ((err = launch_grouped_gemm(d, stream, &p2)) != cudaSuccess) return cuda_fail(err, "down gemm launch");
+  if ((err = launch_combine(at<float>(ws, L.z), o.inv, o.w, M, k, static_cast<int>(w->H), out, stream)) != cudaSuccess)
+    return cuda_fail(err, "combine launch");
+  set_path("forward.grouped");
+  return E4B_OK;
+}
+
+e4b_status e4b_moe_expert_forward_path(const uint16_t* x, int64_t M, const float* router_logits, int k,
+                                       int renormalize, const e4b_expert_stack* w, uint16_t* out, void* workspace,
+                                       size_t workspace_bytes, e4b_path path, e4b_stream stream) {
+  begin_call();
+  if (e4b_status s = check_stack(w, k); s != E4B_OK) return s;
+  if (M < 0) return fail(E4B_ERR_INVALID_ARGUMENT, "M must be >= 0");
+  if (M * k > INT32_MAX) return fail(E4B_ERR_UNSUPPORTED, "M*k exceeds int32 slot indices");
+  if (M > 0 && (!x || !router_logits || !out)) return fail(E4B_ERR_INVALID_ARGUMENT, "null x, router_logits or out");
+  if (M > 0 && (!aligned16(x) || !aligned16(out))) return fail(E4B_ERR_INVALID_ARGUMENT, "x and out must be 16-byte aligned");
+  if (path != E4B_PATH_AUTO && path != E4B_PATH_DECODE && path != E4B_PATH_GROUPED)
+    return fail(E4B_ERR_INVALID_ARGUMENT, "unknown path");
+  const size_t need = e4b_moe_expert_forward_workspace_size(M, w, k);
+  if (workspace_bytes < need || (need > 0 && !workspace))
+    return fail(E4B_ERR_WORKSPACE, "forward workspace needs " + std::to_string(need) + " bytes");
+  if (e4b_status s = check_device(); s != E4B_OK) return s;
+  if (M == 0) {
+    set_path("forward.empty");
+    return E4B_OK;
+  }
+  const bool dec_ok = decode_supported(M, w->E, k, w->H, w->I);
+  if (path == E4B_PATH_DECODE && !dec_ok)
+    return fail(E4B_ERR_UNSUPPORTED, "the decode path takes at most 8 tokens (M=" + std::to_string(M) + ")");
+  if (path == E4B_PATH_DECODE || (path == E4B_PATH_AUTO && dec_ok)) {
+    DecodeArgs a{x, M, router_logits, k, renormalize != 0, w, out, workspace};
+    cudaError_t err = launch_decode_forward(a, stream);
+    if (err != cudaSuccess) return cuda_fail(err, "decode forward launch");
+    set_path("forward.decode");
+    return E4B_OK;
+  }
+  return forward_grouped(x, M, router_logits, k, renormalize, w, out, workspace, stream);
+}
+
+e4b_status e4b_moe_expert_forward(const uint16_t* x, int64_t M, const float* router_logits, int k, int renormalize,
+                                  const e4b_expert_stack* w, uint16_t* out, void* workspace, size_t workspace_bytes,
+                                  e4b_stream stream) {
+  return e4b_moe_expert_forward_path(x, M, router_logits, k, renormalize, w, out, workspace, workspace_bytes,
+                                     E4B_PATH_AUTO, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,116 @@
+// Internal declarations shared by the translation units of libe4b.
+// Host-side launchers only; each kernel lives in its own .cu file.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "../../include/e4b.h"
+
+namespace e4b {
+
+// Per-thread error / path reporting (set by the C-ABI layer).
+void set_error(const std::string& msg);
+void set_path(const char* path);
+
+// Every kernel launch of the library is wrapped in a LaunchScope: it counts the
+// launches of the current call and, while kernel timing is enabled on this
+// thread, brackets the launch with CUDA events recorded on its stream.
+class LaunchScope {
+ public:
+  LaunchScope(const char* name, cudaStream_t stream);
+  ~LaunchScope();
+  LaunchScope(const LaunchScope&) = delete;
+  LaunchScope& operator=(const LaunchScope&) = delete;
+
+ private:
+  int rec_;
+  cudaStream_t stream_;
+};
+void begin_call();  // resets the per-call launch counter
+
+// The NF4 codebook as the library holds it (QLoRA table, ascending).
+extern const float kNf4Codebook[16];
+
+// Quantiser decision thresholds: T[c] is the smallest float strictly above
+// the exact midpoint (cb[c] + cb[c+1]) / 2, so that for any float s,
+// s > midpoint  <=>  s >= T[c].  T[15] = +inf.
+struct Nf4Thresholds {
+  float t[16];
+};
+Nf4Thresholds nf4_thresholds();
+
+cudaError_t launch_quantize(const void* W, bool bf16, int64_t nblocks, uint8_t* packed,
+                            float* absmax, cudaStream_t stream);
+
+// ---- routing -------------------------------------------------------------
+struct RouteOut {
+  int32_t* ids;        // [M, k]
+  float* w;            // [M, k]
+  int32_t* offsets;    // [E+1]
+  int32_t* perm;       // [S]
+  int32_t* inv;        // [S]
+  int32_t* row_token;  // [S] perm[p] / k, or nullptr
+};
+size_t route_workspace_bytes(int64_t M, int64_t E, int k);
+bool route_uses_small_kernel(int64_t M, int64_t E, int k);
+cudaError_t launch_route(const float* logits, int64_t M, int E, int k, bool renormalize,
+                         const RouteOut& o, void* workspace, cudaStream_t stream);
+
+// ---- grouped GEMM --------------------------------------------------------
+struct GemmArgs {
+  const uint16_t* A;
+  int64_t a_rows, lda;
+  const int32_t* row_index;  // nullable
+  const int32_t* offsets;    // [E+1]
+  int E;
+  int64_t total_rows;
+  const uint8_t* packed;
+  const float* absmax;
+  int N, K;
+  const uint16_t* lora_A;  // [E, r, K] or nullptr
+  const uint16_t* lora_B;  // [E, N, r] or nullptr
+  int r;
+  float lora_scale;
+  float* xa;  // workspace [total_rows, r] (LoRA only)
+  int epi;    // e4b_epilogue
+  void* out;
+  bool out_bf16;
+};
+size_t gemm_workspace_bytes(int64_t total_rows, int r);
+// Picks the implementation; reports the path name through set_path.
+cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const char** path);
+
+// ---- combine ---------------------------------------------------------------
+cudaError_t launch_combine(const float* z, const int32_t* inv, const float* w, int64_t M, int k,
+                           int H, uint16_t* out, cudaStream_t stream);
+
+// ---- fused small-M forward ---------------------------------------------------
+struct DecodeArgs {
+  const uint16_t* x;
+  int64_t M;
+  const float* logits;
+  int k;
+  bool renormalize;
+  const e4b_expert_stack* w;
+  uint16_t* out;
+  void* workspace;
+};
+bool decode_supported(int64_t M, int64_t E, int k, int64_t H, int64_t I);
+size_t decode_workspace_bytes(int64_t M, int64_t E, int k, int64_t H, int64_t I, int r);
+cudaError_t launch_decode_forward(const DecodeArgs& a, cudaStream_t stream);
+
+// Device properties cached per device.
+struct DeviceInfo {
+  int device;
+  int sm_count;
+  int major, minor;
+  size_t smem_optin;
+};
+cudaError_t device_info(DeviceInfo* out);
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace e4b

@@ -1,0 +1,141 @@
+// NF4 blockwise quantisation of a fused expert stack (load time).
+//
+// Follows "Why does load_in_4bit still OOM on a Mixture-of-Experts model?",
+// section "Which project solves it": the stack is quantised expert by expert
+// with blocks that never cross an expert boundary.  Because every expert holds
+// N*K elements with (N*K) % 64 == 0, cutting the flattened [E, N*K] stack into
+// consecutive blocks of 64 gives exactly the per-expert blocks.
+//
+// Per block: absmax a = max |w| (exact in fp32); s = w / a as one IEEE fp32
+// division; code = number of decision thresholds T[c] <= s, where T[c] is the
+// smallest float above the exact midpoint of codebook entries c and c+1 (so a
+// value exactly on a midpoint takes the lower code); a = 0 gives code 7.
+//
+// HBM-bound: 4 B (fp32) or 2 B (bf16) read + 0.5625 B written per weight.  One
+// warp handles 8 blocks (512 weights) per step with 16-byte loads; each block
+// is reduced by a 16-lane shuffle tree.
+#include <cmath>
+#include <limits>
+
+#include "common.cuh"
+#include "e4b_internal.h"
+
+namespace e4b {
+
+const float kNf4Codebook[16] = {E4B_NF4_CODEBOOK_VALUES};
+
+Nf4Thresholds nf4_thresholds() {
+  Nf4Thresholds th;
+  for (int c = 0; c < 15; ++c) {
+    // Exact in double: sum of two floats, then an exact halving.
+    const double mid = (static_cast<double>(kNf4Codebook[c]) + static_cast<double>(kNf4Codebook[c + 1])) * 0.5;
+    float f = static_cast<float>(mid);
+    if (static_cast<double>(f) <= mid) f = std::nextafter(f, std::numeric_limits<float>::infinity());
+    th.t[c] = f;
+  }
+  th.t[15] = std::numeric_limits<float>::infinity();
+  return th;
+}
+
+namespace {
+
+// Code of s: count of thresholds <= s, by a 4-step branchless binary search
+// over the ascending table in shared memory.
+__device__ __forceinline__ uint32_t code_of(float s, const float* t) {
+  uint32_t q = (s >= t[7]) ? 8u : 0u;
+  q += (s >= t[q + 3]) ? 4u : 0u;
+  q += (s >= t[q + 1]) ? 2u : 0u;
+  q += (s >= t[q]) ? 1u : 0u;
+  return q;
+}
+
+template <bool kBf16>
+__device__ __forceinline__ void load4(const void* W, int64_t elem, float v[4]) {
+  if constexpr (kBf16) {
+    const uint2 raw = __ldcs(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(W) + elem));
+    v[0] = __uint_as_float(raw.x << 16);
+    v[1] = __uint_as_float(raw.x & 0xffff0000u);
+    v[2] = __uint_as_float(raw.y << 16);
+    v[3] = __uint_as_float(raw.y & 0xffff0000u);
+  } else {
+    const float4 f = __ldcs(reinterpret_cast<const float4*>(static_cast<const float*>(W) + elem));
+    v[0] = f.x;
+    v[1] = f.y;
+    v[2] = f.z;
+    v[3] = f.w;
+  }
+}
+
+template <bool kBf16>
+__global__ void __launch_bounds__(256) nf4_quantize_kernel(const void* __restrict__ W, int64_t nblocks,
+                                                           uint8_t* __restrict__ packed,
+                                                           float* __restrict__ absmax, Nf4Thresholds th) {
+  __shared__ float t_s[16];
+  if (threadIdx.x < 16) t_s[threadIdx.x] = th.t[threadIdx.x];
+  __syncthreads();
+
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int64_t ngroups = (nblocks + 7) / 8;  // 8 blocks = 512 weights per warp step
+
+  for (int64_t g = warp; g < ngroups; g += nwarps) {
+    float v[4][4];
+    bool valid[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      // Step i covers blocks 2i (lanes 0-15) and 2i+1 (lanes 16-31).
+      const int64_t blk = g * 8 + 2 * i + (lane >> 4);
+      valid[i] = blk < nblocks;
+      const int64_t elem = g * 512 + 128 * i + 4 * lane;
+      if (valid[i]) {
+        load4<kBf16>(W, elem, v[i]);
+      } else {
+        v[i][0] = v[i][1] = v[i][2] = v[i][3] = 0.0f;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float m = fmaxf(fmaxf(fabsf(v[i][0]), fabsf(v[i][1])), fmaxf(fabsf(v[i][2]), fabsf(v[i][3])));
+#pragma unroll
+      for (int o = 8; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      uint32_t q[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        // IEEE division (no fast-math in this file): bit-exact fl32(w / a).
+        q[j] = (m > 0.0f) ? code_of(__fdiv_rn(v[i][j], m), t_s) : 7u;
+      }
+      const int64_t blk = g * 8 + 2 * i + (lane >> 4);
+      const int64_t elem = g * 512 + 128 * i + 4 * lane;
+      if (valid[i]) {
+        const uint16_t two = static_cast<uint16_t>(((q[0] << 4) | q[1]) | (((q[2] << 4) | q[3]) << 8));
+        *reinterpret_cast<uint16_t*>(packed + elem / 2) = two;
+        if ((lane & 15) == 0) absmax[blk] = m;
+      }
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(const void* W, bool bf16, int64_t nblocks, uint8_t* packed, float* absmax,
+                            cudaStream_t stream) {
+  if (nblocks == 0) return cudaSuccess;
+  DeviceInfo di;
+  cudaError_t err = device_info(&di);
+  if (err != cudaSuccess) return err;
+  const int64_t ngroups = (nblocks + 7) / 8;
+  const int threads = 256;
+  const int64_t want = (ngroups + (threads / 32) - 1) / (threads / 32);
+  const int64_t cap = static_cast<int64_t>(di.sm_count) * 8;
+  const int grid = static_cast<int>(want < cap ? want : cap);
+  const Nf4Thresholds th = nf4_thresholds();
+  LaunchScope ls("quantize", stream);
+  if (bf16)
+    nf4_quantize_kernel<true><<<grid, threads, 0, stream>>>(W, nblocks, packed, absmax, th);
+  else
+    nf4_quantize_kernel<false><<<grid, threads, 0, stream>>>(W, nblocks, packed, absmax, th);
+  return cudaGetLastError();
+}
+
+}  // namespace e4b

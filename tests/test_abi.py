@@ -1,0 +1,76 @@
+"""The C ABI library loads and exports every symbol include/e4b.h declares.
+
+CPU only: no call here launches GPU work.  Argument checks that fail before
+any device query are exercised directly.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from quantized_moe_expert_nf4_b200 import e4b
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "e4b.h")
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"\b(e4b_[a-z0-9_]+)\s*\(", src)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(e4b.LIB_PATH):
+        from quantized_moe_expert_nf4_b200 import build
+        build.build()
+    return e4b.load_library()
+
+
+def test_header_declares_the_four_calls():
+    names = _declared_functions()
+    for n in ("e4b_nf4_quantize_stack", "e4b_moe_route_permute", "e4b_grouped_nf4_gemm",
+              "e4b_moe_expert_forward"):
+        assert n in names
+    assert sorted(e4b.EXPORTED) == names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in _declared_functions():
+        assert hasattr(lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", e4b.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (e4b_[a-z0-9_]+)", out))
+    assert exported == set(_declared_functions())
+
+
+def test_status_strings_and_version(lib):
+    assert lib.e4b_version() == 1
+    assert lib.e4b_status_string(0) == b"E4B_OK"
+    assert lib.e4b_status_string(3) == b"E4B_ERR_WORKSPACE"
+
+
+def test_host_side_rejections_without_gpu(lib):
+    # blocksize is checked before any device query
+    st = lib.e4b_nf4_quantize_stack(None, 0, 2, 64, 64, 32, None, None, None)
+    assert st == 2 and b"blocksize" in lib.e4b_last_error()
+    st = lib.e4b_nf4_quantize_stack(None, 0, 2, 3, 5, 64, None, None, None)
+    assert st == 2 and b"multiple of 64" in lib.e4b_last_error()
+    st = lib.e4b_moe_route_permute(None, 4, 8, 9, 1, None, None, None, None, None, None, 0, None)
+    assert st == 1 and b"k must be" in lib.e4b_last_error()
+    st = lib.e4b_grouped_nf4_gemm(None, 1, 64, None, None, 2, 1, None, None, 64, 96, None, None, 0, 0.0, 0,
+                                  None, 0, None, 0, None)
+    assert st == 2 and b"K must be" in lib.e4b_last_error()
+
+
+def test_workspace_queries_are_host_only(lib):
+    assert e4b.e4b_moe_route_permute_workspace_size(1, 64, 8) == 0
+    assert e4b.e4b_moe_route_permute_workspace_size(4096, 128, 8) > 4096 * 8 * 4
+    assert e4b.e4b_grouped_nf4_gemm_workspace_size(100, 128, 64, 0) == 0
+    assert e4b.e4b_grouped_nf4_gemm_workspace_size(100, 128, 64, 8) == 100 * 8 * 4
+    st = e4b.ExpertStackC(1, 1, 1, 1, None, None, 0, 0.0, 64, 2048, 1024)
+    n = lib.e4b_moe_expert_forward_workspace_size(2048, ctypes.byref(st), 8)
+    assert n >= 2048 * 8 * (1024 * 2 + 2048 * 4)

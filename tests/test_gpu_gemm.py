@@ -1,0 +1,119 @@
+"""GPU grouped NF4 GEMM vs the float64 oracle (every epilogue and output type)."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe, nf4
+from quantized_moe_expert_nf4_b200 import e4b, workloads
+from gpu_util import bf16_to_f64, rel_errors, require_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(E, N, K, counts, a_rows, seed, lora_r=0):
+    rng = np.random.default_rng(seed)
+    W = (rng.standard_normal((E, N, K)) * 0.02).astype(np.float32)
+    packed, absmax = nf4.quantize_stack(W)
+    A32 = rng.standard_normal((a_rows, K)).astype(np.float32)
+    Abits = workloads.to_bf16_bits(A32)
+    offs = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    rows = int(offs[-1])
+    ridx = rng.integers(0, a_rows, size=rows).astype(np.int32)
+    la = lb = None
+    if lora_r:
+        la = workloads.to_bf16_bits((rng.standard_normal((E, lora_r, K)) * 0.05).astype(np.float32))
+        lb = workloads.to_bf16_bits((rng.standard_normal((E, N, lora_r)) * 0.05).astype(np.float32))
+    return dict(E=E, N=N, K=K, packed=packed, absmax=absmax, Abits=Abits, offs=offs, rows=rows, ridx=ridx,
+                la=la, lb=lb, r=lora_r)
+
+
+def _t_bf16(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def _run_gpu(c, epi, out_dtype, use_ridx=True, scale=2.0):
+    ncols = c["N"] // 2 if epi == e4b.E4B_EPI_SWIGLU else c["N"]
+    out = torch.full((c["rows"] + 1, ncols), float("nan"), dtype=out_dtype, device="cuda")   # +1 guard row
+    ws = e4b.workspace(e4b.e4b_grouped_nf4_gemm_workspace_size(c["rows"], c["N"], c["K"], c["r"]))
+    e4b.e4b_grouped_nf4_gemm(
+        _t_bf16(c["Abits"]), torch.from_numpy(c["ridx"]).cuda() if use_ridx else None,
+        torch.from_numpy(c["offs"]).cuda(), c["rows"], torch.from_numpy(c["packed"]).cuda(),
+        torch.from_numpy(c["absmax"]).cuda(), c["N"], c["K"], out, epi,
+        _t_bf16(c["la"]) if c["r"] else None, _t_bf16(c["lb"]) if c["r"] else None, scale, ws)
+    torch.cuda.synchronize()
+    res = out.float().cpu().numpy().astype(np.float64)
+    assert np.all(np.isnan(res[c["rows"]])), "guard row written"
+    return res[:c["rows"]], e4b.last_path()
+
+
+def _oracle(c, epi, use_ridx=True, scale=2.0):
+    A = workloads.bf16_bits_to_f32(c["Abits"]).astype(np.float64)
+    la = workloads.bf16_bits_to_f32(c["la"]).astype(np.float64) if c["r"] else None
+    lb = workloads.bf16_bits_to_f32(c["lb"]).astype(np.float64) if c["r"] else None
+    return moe.grouped_nf4_gemm(A, c["ridx"] if use_ridx else None, c["offs"], c["packed"], c["absmax"],
+                                c["N"], c["K"], la, lb, scale, swiglu=(epi == e4b.E4B_EPI_SWIGLU))
+
+
+CASES = [
+    # E, N, K, counts (ragged, with empty groups), a_rows
+    (3, 128, 256, [5, 0, 70], 40),
+    (4, 192, 128, [1, 130, 0, 64], 200),
+    (2, 64, 64, [0, 1], 3),
+    (8, 256, 192, [17, 3, 0, 0, 65, 1, 33, 128], 100),
+]
+
+
+@pytest.mark.parametrize("ci", range(len(CASES)))
+@pytest.mark.parametrize("epi", [e4b.E4B_EPI_NONE, e4b.E4B_EPI_SWIGLU])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_grouped_gemm_matches_oracle(ci, epi, out_dtype):
+    require_gpu()
+    E, N, K, counts, a_rows = CASES[ci]
+    c = _case(E, N, K, counts, a_rows, seed=ci)
+    got, path = _run_gpu(c, epi, out_dtype)
+    ref = _oracle(c, epi)
+    fro, mx = rel_errors(got, ref)
+    # fp32 output: the only rounding is the codebook entry to bf16 (relative
+    # error <= 2^-9 per weight); SwiGLU multiplies two such results, so its
+    # bound doubles (<= 2 * 2^-9 ~ 3.9e-3).  bf16 output adds one more rounding.
+    tol = (2e-3 if epi == e4b.E4B_EPI_NONE else 4e-3) if out_dtype == torch.float32 else 1e-2
+    print(f"[parity] gemm case {ci} epi {epi} {out_dtype} path {path}: rel_fro={fro:.2e} max={mx:.2e}")
+    assert fro <= tol and mx <= 2 * tol
+
+
+@pytest.mark.parametrize("epi", [e4b.E4B_EPI_NONE, e4b.E4B_EPI_SWIGLU])
+def test_grouped_gemm_lora(epi):
+    require_gpu()
+    c = _case(4, 256, 128, [3, 0, 80, 20], 64, seed=11, lora_r=8)
+    got, _ = _run_gpu(c, epi, torch.float32)
+    ref = _oracle(c, epi)
+    fro, mx = rel_errors(got, ref)
+    assert fro <= 2e-3 and mx <= 4e-3
+    # the delta matters: without it the result is off
+    ref0 = _oracle(dict(c, r=0), epi)
+    assert rel_errors(ref0, ref)[0] > 1e-2
+
+
+def test_grouped_gemm_identity_rows_and_all_ones():
+    require_gpu()
+    c = _case(3, 64, 128, [10, 0, 6], 16, seed=3)
+    got, _ = _run_gpu(c, e4b.E4B_EPI_NONE, torch.float32, use_ridx=False)
+    assert rel_errors(got, _oracle(c, e4b.E4B_EPI_NONE, use_ridx=False))[0] <= 2e-3
+    # all codes 15, absmax 1 -> every output is the row sum of A (exact for small integers)
+    c["packed"][:] = 0xFF
+    c["absmax"][:] = 1.0
+    c["Abits"] = workloads.to_bf16_bits(np.random.default_rng(4).integers(-3, 4, size=(16, 128)).astype(np.float32))
+    got, _ = _run_gpu(c, e4b.E4B_EPI_NONE, torch.float32)
+    A = workloads.bf16_bits_to_f32(c["Abits"]).astype(np.float64)
+    want = A[c["ridx"]].sum(axis=1)[:, None] * np.ones((1, 64))
+    assert np.array_equal(got, want)
+
+
+def test_grouped_gemm_positive_control_flipped_nibble():
+    require_gpu()
+    c = _case(2, 64, 128, [8, 8], 16, seed=5)
+    ref = _oracle(c, e4b.E4B_EPI_NONE)
+    c["packed"][1, 0] ^= 0x88        # flip one byte of the second expert
+    got, _ = _run_gpu(c, e4b.E4B_EPI_NONE, torch.float32)
+    rows = slice(8, 16)
+    assert np.max(np.abs(got[rows, 0] - ref[rows, 0])) > 1e-4
