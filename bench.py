@@ -425,13 +425,29 @@ def dominant_roofline(cfg, M, kt, touched_avg, peaks, long_region):
                   "peak_source": peaks["source"] + " " + key}
 
 
+def reduce_over_ranks(value, dist, device, op="max"):
+    """Max (or min) of a per-rank float over all ranks; identity without a process group."""
+    if dist is None:
+        return float(value)
+    import torch
+
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.MIN)
+    return float(t.item())
+
+
+def job_throughput(per_rank_units, steps, world, max_seconds):
+    """Whole-job units/s: every rank processes `per_rank_units` per step (weak scaling)."""
+    return world * per_rank_units * steps / max_seconds
+
+
 def measure(args, name, rank, world, dist, peaks, primary):
     import torch
 
     cfgname, M = WORKLOADS[name]
     cfg = workloads.CONFIGS[cfgname]
     dev = f"cuda:{torch.cuda.current_device()}"
-    R = replicas_for(cfg, M)
+    R = args.replicas if args.replicas > 0 else replicas_for(cfg, M)
     b = Bench(cfg, M, dev, R, seed_base=rank)
     b.capture()
     b.run_steps(args.warmup)
@@ -439,19 +455,19 @@ def measure(args, name, rank, world, dist, peaks, primary):
     sampler = ClockSampler(torch.cuda.current_device())
     with sampler:
         t = b.time_steps(args.steps, dist)
-    if dist is not None:
-        tt = torch.tensor([t], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t = float(tt.item())
+    t = reduce_over_ranks(t, dist, dev, "max")
     S = M * cfg.k
-    value = world * S * args.steps / t
+    value = job_throughput(S, args.steps, world, t)
     ms = 1e3 * t / args.steps
     touched_avg = float(np.mean([b.touched[i % R] for i in range(args.steps)]))
     flops, nbytes = step_work(cfg, M, touched_avg)
     t_star = max(nbytes / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12))
     step_bound = "hbm" if nbytes / (peaks["hbm_gbs"] * 1e9) >= flops / (peaks["bf16_tflops"] * 1e12) else "tensor"
-    kt = b.kernel_timing(min(max(args.steps, 20), 400))
-    kname, roof = dominant_roofline(cfg, M, kt, touched_avg, peaks, long_region=t > 1.0)
+    if args.no_kernel_timing:
+        kt, roof = {}, None
+    else:
+        kt = b.kernel_timing(min(max(args.steps, 20), 400))
+        kname, roof = dominant_roofline(cfg, M, kt, touched_avg, peaks, long_region=t > 1.0)
     res = {
         "value": value, "ms_per_step": ms, "tflops": world * flops / (ms * 1e-3) / 1e12 if ms else None,
         "path": b.path, "launches_per_step": b.launches_per_step, "touched_experts_avg": touched_avg,
@@ -463,12 +479,10 @@ def measure(args, name, rank, world, dist, peaks, primary):
         "kernels_us": {k: v[0] * 1e3 for k, v in kt.items()},
         "clocks": sampler.summary(),
     }
-    if primary:
+    res["e2e"] = None
+    if primary and not args.no_e2e:
         ev, h2d, d2h = b.e2e(min(args.steps, 2000))
-        if dist is not None:
-            et = torch.tensor([ev], device=dev, dtype=torch.float64)
-            dist.all_reduce(et, op=dist.ReduceOp.MIN)
-            ev = float(et.item()) * world
+        ev = reduce_over_ranks(ev, dist, dev, "min") * world
         res["e2e"] = {"value": ev, "unit": "routed_tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     res["cfg"] = cfg
     res["M"] = M
@@ -486,6 +500,9 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end host-buffer pass")
+    ap.add_argument("--no-kernel-timing", action="store_true", help="skip the per-kernel event pass")
+    ap.add_argument("--replicas", type=int, default=0, help="layer replicas (0: enough to exceed L2 4x)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -524,8 +541,10 @@ def main():
             r = measure(args, name, rank, world, dist, peaks, primary=False)
             sweep.append({"workload": name, "value": r["value"], "ms_per_step": r["ms_per_step"],
                           "tflops": r["tflops"], "path": r["path"], "touched_experts_avg": r["touched_experts_avg"],
-                          "roofline_frac": r["roofline"]["frac"], "roofline_bound": r["roofline"]["bound"],
-                          "roofline_kernel": r["roofline"]["kernel"], "step_roofline_frac": r["step_roofline"]["frac"],
+                          "roofline_frac": r["roofline"]["frac"] if r["roofline"] else None,
+                          "roofline_bound": r["roofline"]["bound"] if r["roofline"] else None,
+                          "roofline_kernel": r["roofline"]["kernel"] if r["roofline"] else None,
+                          "step_roofline_frac": r["step_roofline"]["frac"],
                           "clocks": r["clocks"]})
     if rank == 0:
         cb = None
