@@ -26,8 +26,9 @@
  *     except where a leading dimension is passed.
  *   - bf16 data is passed as raw 16-bit patterns (uint16_t).
  *   - Calls are stream-ordered on `stream` (a cudaStream_t; NULL is the legacy
- *     default stream).  No call reads device data back to the host, so every
- *     call can be captured in a CUDA graph.
+ *     default stream).  The four calls of the layer (quantise, route/permute,
+ *     grouped GEMM, forward) read no device data back to the host and can be
+ *     captured in a CUDA graph.
  *   - Arguments are checked on the host before anything is launched.  A bad
  *     argument returns E4B_ERR_INVALID_ARGUMENT, a shape or device the kernels
  *     do not support returns E4B_ERR_UNSUPPORTED, a workspace that is too small
@@ -232,6 +233,34 @@ E4B_API e4b_status e4b_moe_expert_forward_path(const uint16_t* x, int64_t M, con
                                        int k, int renormalize, const e4b_expert_stack* w,
                                        uint16_t* out, void* workspace, size_t workspace_bytes,
                                        e4b_path path, e4b_stream stream);
+
+/*
+ * Allocation-free small-batch forward.  The pages have no counterpart of this
+ * call; it exists for hosts that cannot give the library device memory:
+ * serving engines that plan every byte of device memory into a fixed pool at
+ * start-up, and runtimes that allow no allocator call (cudaMalloc or any
+ * other) once their decode loop is running.
+ *
+ * Computes exactly what e4b_moe_expert_forward() computes for 1 <= M <= 8
+ * tokens, with the decode kernels, but takes no workspace: its scratch (the
+ * SwiGLU activations of the routed slots, M*k*I bf16 values, plus an error
+ * word) lives in one statically sized device array of the library,
+ * 512 KiB + 256 B, which every GPU that loads the library holds until the
+ * process exits.  Requires M*k*I <= 262144 (for example M = 8, k = 8,
+ * I <= 4096); larger shapes return E4B_ERR_UNSUPPORTED with a message.  The
+ * caller still owns x, router_logits, the stacks and out; nothing here calls
+ * cudaMalloc, cudaFree or any allocating routine.
+ *
+ * The first call on each device looks up the device address of the array
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls share the one array and it keeps the
+ * last call's contents, so calls whose kernels overlap on the GPU (different
+ * streams without ordering between them) race and give wrong results.
+ */
+E4B_API e4b_status e4b_moe_expert_forward_decode_noalloc(const uint16_t* x, int64_t M,
+                                                         const float* router_logits, int k,
+                                                         int renormalize, const e4b_expert_stack* w,
+                                                         uint16_t* out, e4b_stream stream);
 
 #ifdef __cplusplus
 }

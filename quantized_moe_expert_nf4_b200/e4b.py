@@ -35,7 +35,7 @@ EXPORTED = (
     "e4b_moe_route_permute_workspace_size", "e4b_moe_route_permute",
     "e4b_grouped_nf4_gemm_workspace_size", "e4b_grouped_nf4_gemm",
     "e4b_moe_expert_forward_workspace_size", "e4b_moe_expert_forward",
-    "e4b_moe_expert_forward_path",
+    "e4b_moe_expert_forward_path", "e4b_moe_expert_forward_decode_noalloc",
 )
 
 
@@ -99,6 +99,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.e4b_moe_expert_forward_workspace_size.argtypes = [i64, ctypes.POINTER(ExpertStackC), i32]
     lib.e4b_moe_expert_forward.restype = i32
     lib.e4b_moe_expert_forward.argtypes = [vp, i64, vp, i32, i32, ctypes.POINTER(ExpertStackC), vp, vp, sz, vp]
+    lib.e4b_moe_expert_forward_decode_noalloc.restype = i32
+    lib.e4b_moe_expert_forward_decode_noalloc.argtypes = [vp, i64, vp, i32, i32, ctypes.POINTER(ExpertStackC), vp,
+                                                          vp]
     lib.e4b_moe_expert_forward_path.restype = i32
     lib.e4b_moe_expert_forward_path.argtypes = [vp, i64, vp, i32, i32, ctypes.POINTER(ExpertStackC), vp, vp,
                                                 sz, i32, vp]
@@ -274,6 +277,20 @@ def e4b_moe_expert_forward(x: torch.Tensor, router_logits: torch.Tensor, k: int,
     _check(load_library().e4b_moe_expert_forward_path(
         x.data_ptr(), M, router_logits.data_ptr(), k, int(bool(renormalize)), ctypes.byref(stack.c),
         out.data_ptr(), _ptr(workspace), ws, path, _stream(stream)), "e4b_moe_expert_forward")
+
+
+def e4b_moe_expert_forward_decode_noalloc(x: torch.Tensor, router_logits: torch.Tensor, k: int, renormalize: bool,
+                                          stack: ExpertStack, out: torch.Tensor, stream=None) -> None:
+    """The layer forward for 1..8 tokens without a workspace (see include/e4b.h)."""
+    _dev(x, "x", torch.bfloat16)
+    _dev(router_logits, "router_logits", torch.float32)
+    _dev(out, "out", torch.bfloat16)
+    M = x.shape[0]
+    if x.shape[1] != stack.H or router_logits.shape != (M, stack.E) or out.shape != (M, stack.H):
+        raise ValueError("x [M, H], router_logits [M, E] and out [M, H] required")
+    _check(load_library().e4b_moe_expert_forward_decode_noalloc(
+        x.data_ptr(), M, router_logits.data_ptr(), k, int(bool(renormalize)), ctypes.byref(stack.c),
+        out.data_ptr(), _stream(stream)), "e4b_moe_expert_forward_decode_noalloc")
 
 
 def workspace(nbytes: int, device="cuda") -> torch.Tensor:
