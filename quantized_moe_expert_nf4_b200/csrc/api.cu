@@ -52,13 +52,14 @@ struct Carve {
 
 // Workspace of the grouped forward path.
 struct GroupedLayout {
-  size_t ids, w, offsets, perm, inv, row_token, route_ws, xa, h, z, total;
+  size_t err, ids, w, offsets, perm, inv, row_token, route_ws, xa, h, z, total;
 };
 
 GroupedLayout grouped_layout(int64_t M, int64_t E, int64_t H, int64_t I, int k, int r) {
   const int64_t S = M * k;
   Carve c;
   GroupedLayout L;
+  L.err = c.take(sizeof(int32_t));
   L.ids = c.take(S * sizeof(int32_t));
   L.w = c.take(S * sizeof(float));
   L.offsets = c.take((E + 1) * sizeof(int32_t));
@@ -323,7 +324,8 @@ e4b_status e4b_grouped_nf4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda, 
   g.lora_B = lora_B;
   g.r = r;
   g.lora_scale = lora_scale;
-  g.xa = r > 0 ? static_cast<float*>(workspace) : nullptr;
+  g.err = static_cast<int*>(workspace);
+  g.xa = r > 0 ? reinterpret_cast<float*>(static_cast<char*>(workspace) + 256) : nullptr;
   g.epi = epi;
   g.out = out;
   g.out_bf16 = out_dtype == E4B_BF16;
@@ -386,6 +388,7 @@ static e4b_status forward_grouped(const uint16_t* x, int64_t M, const float* log
   g.r = r;
   g.lora_scale = r ? w->lora_alpha / static_cast<float>(r) : 0.0f;
   g.xa = r ? at<float>(ws, L.xa) : nullptr;
+  g.err = at<int>(ws, L.err);
   g.epi = E4B_EPI_SWIGLU;
   g.out = at<uint16_t>(ws, L.h);
   g.out_bf16 = true;
@@ -403,6 +406,7 @@ static e4b_status forward_grouped(const uint16_t* x, int64_t M, const float* log
   d.absmax = w->dn_absmax;
   d.N = static_cast<int>(w->H);
   d.K = static_cast<int>(w->I);
+  d.err = at<int>(ws, L.err);
   d.epi = E4B_EPI_NONE;
   d.out = at<float>(ws, L.z);
   d.out_bf16 = false;

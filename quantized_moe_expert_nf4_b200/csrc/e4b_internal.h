@@ -7,7 +7,7 @@
 
 #include <string>
 
-#include "../../include/e4b.h"
+#include "e4b.h"
 
 namespace e4b {
 
@@ -75,11 +75,14 @@ struct GemmArgs {
   int r;
   float lora_scale;
   float* xa;  // workspace [total_rows, r] (LoRA only)
+  int* err;   // workspace error word of the tensor-core kernel's bounded waits
   int epi;    // e4b_epilogue
   void* out;
   bool out_bf16;
 };
 size_t gemm_workspace_bytes(int64_t total_rows, int r);
+bool tc_supported(const GemmArgs& a);
+cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int* err_word, cudaStream_t stream);
 // Picks the implementation; reports the path name through set_path.
 cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const char** path);
 

@@ -22,6 +22,9 @@
 // K order inside a 32-wide chunk is permuted consistently for both operands:
 // lane t of a quad owns physical k in [8t, 8t+8), which is one 32-bit word of
 // packed nibbles for A and one 16-byte vector of bf16 activations for B.
+#include <cstdlib>
+#include <cstring>
+
 #include "common.cuh"
 #include "e4b_internal.h"
 
@@ -275,16 +278,40 @@ cudaError_t launch_grouped_gemm_mma(const GemmArgs& a, cudaStream_t stream) {
 
 namespace e4b {
 
+// Workspace: [error word, 256 B][LoRA x.A^T, total_rows * r fp32].
 size_t gemm_workspace_bytes(int64_t total_rows, int r) {
-  return r > 0 ? static_cast<size_t>(total_rows) * r * sizeof(float) : 0;
+  return 256 + (r > 0 ? static_cast<size_t>(total_rows) * r * sizeof(float) : 0);
 }
 
+namespace {
+// Which grouped GEMM kernel runs: the tensor-core (tcgen05) kernel for large
+// row counts, the warp-MMA kernel otherwise.  E4B_GEMM=mma|tc forces one (tests,
+// benchmarks); a forced kernel that cannot take the call is an error, never a
+// silent switch.
+int gemm_override() {
+  const char* v = getenv("E4B_GEMM");
+  if (!v) return 0;
+  if (!strcmp(v, "mma")) return 1;
+  if (!strcmp(v, "tc")) return 2;
+  return 0;
+}
+constexpr int64_t kTcMinRows = 512;
+}  // namespace
+
 cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const char** path) {
+  const int ov = gemm_override();
+  const bool tc_ok = tc_supported(a);
+  const bool use_tc = ov == 2 || (ov == 0 && tc_ok && a.total_rows >= kTcMinRows);
+  if (use_tc) {
+    if (!tc_ok) return cudaErrorNotSupported;
+    *path = a.epi == E4B_EPI_SWIGLU ? "gemm.tc.swiglu" : "gemm.tc";
+    return launch_grouped_gemm_tc(a, a.err, stream);
+  }
   if (a.lora_B && a.r > 0) {
     cudaError_t err = launch_lora_xa(a, stream);
     if (err != cudaSuccess) return err;
   }
-  *path = "gemm.mma";
+  *path = a.epi == E4B_EPI_SWIGLU ? "gemm.mma.swiglu" : "gemm.mma";
   return launch_grouped_gemm_mma(a, stream);
 }
 

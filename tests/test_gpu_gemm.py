@@ -54,12 +54,33 @@ def _oracle(c, epi, use_ridx=True, scale=2.0):
                                 c["N"], c["K"], la, lb, scale, swiglu=(epi == e4b.E4B_EPI_SWIGLU))
 
 
+def gemm_tolerance(path, epi, out_dtype):
+    """Relative Frobenius tolerance of one grouped GEMM against the float64 oracle.
+
+    Warp-MMA path: the only rounding of a weight is its codebook entry to bf16
+    (relative error <= 2^-9; absmax is applied in fp32 per 64-block), so a plain
+    fp32 output stays within 2e-3 and SwiGLU, the product of two such results,
+    within 4e-3.  Tensor-core path: the decoded weight is rounded three times
+    (codebook entry, absmax and their product, each <= 2^-9 relative, rms about
+    2^-9 together), so 4e-3 plain and 6e-3 for SwiGLU.  bf16 outputs add one
+    rounding of 2^-9: 1e-2 for both paths.
+    """
+    if out_dtype == torch.bfloat16:
+        return 1e-2
+    tc = path.startswith("gemm.tc")
+    if epi == e4b.E4B_EPI_NONE:
+        return 4e-3 if tc else 2e-3
+    return 6e-3 if tc else 4e-3
+
+
 CASES = [
     # E, N, K, counts (ragged, with empty groups), a_rows
     (3, 128, 256, [5, 0, 70], 40),
     (4, 192, 128, [1, 130, 0, 64], 200),
     (2, 64, 64, [0, 1], 3),
     (8, 256, 192, [17, 3, 0, 0, 65, 1, 33, 128], 100),
+    # several n tiles with a ragged last one, several token tiles per group
+    (4, 640, 320, [300, 0, 129, 77], 256),
 ]
 
 
@@ -73,10 +94,7 @@ def test_grouped_gemm_matches_oracle(ci, epi, out_dtype):
     got, path = _run_gpu(c, epi, out_dtype)
     ref = _oracle(c, epi)
     fro, mx = rel_errors(got, ref)
-    # fp32 output: the only rounding is the codebook entry to bf16 (relative
-    # error <= 2^-9 per weight); SwiGLU multiplies two such results, so its
-    # bound doubles (<= 2 * 2^-9 ~ 3.9e-3).  bf16 output adds one more rounding.
-    tol = (2e-3 if epi == e4b.E4B_EPI_NONE else 4e-3) if out_dtype == torch.float32 else 1e-2
+    tol = gemm_tolerance(path, epi, out_dtype)
     print(f"[parity] gemm case {ci} epi {epi} {out_dtype} path {path}: rel_fro={fro:.2e} max={mx:.2e}")
     assert fro <= tol and mx <= 2 * tol
 
@@ -85,10 +103,11 @@ def test_grouped_gemm_matches_oracle(ci, epi, out_dtype):
 def test_grouped_gemm_lora(epi):
     require_gpu()
     c = _case(4, 256, 128, [3, 0, 80, 20], 64, seed=11, lora_r=8)
-    got, _ = _run_gpu(c, epi, torch.float32)
+    got, path = _run_gpu(c, epi, torch.float32)
     ref = _oracle(c, epi)
     fro, mx = rel_errors(got, ref)
-    assert fro <= 2e-3 and mx <= 4e-3
+    tol = gemm_tolerance(path, epi, torch.float32)
+    assert fro <= tol and mx <= 2 * tol
     # the delta matters: without it the result is off
     ref0 = _oracle(dict(c, r=0), epi)
     assert rel_errors(ref0, ref)[0] > 1e-2
@@ -97,8 +116,9 @@ def test_grouped_gemm_lora(epi):
 def test_grouped_gemm_identity_rows_and_all_ones():
     require_gpu()
     c = _case(3, 64, 128, [10, 0, 6], 16, seed=3)
-    got, _ = _run_gpu(c, e4b.E4B_EPI_NONE, torch.float32, use_ridx=False)
-    assert rel_errors(got, _oracle(c, e4b.E4B_EPI_NONE, use_ridx=False))[0] <= 2e-3
+    got, path = _run_gpu(c, e4b.E4B_EPI_NONE, torch.float32, use_ridx=False)
+    assert rel_errors(got, _oracle(c, e4b.E4B_EPI_NONE, use_ridx=False))[0] <= gemm_tolerance(
+        path, e4b.E4B_EPI_NONE, torch.float32)
     # all codes 15, absmax 1 -> every output is the row sum of A (exact for small integers)
     c["packed"][:] = 0xFF
     c["absmax"][:] = 1.0
