@@ -52,7 +52,7 @@ struct Carve {
 
 // Workspace of the grouped forward path.
 struct GroupedLayout {
-  size_t err, ids, w, offsets, perm, inv, row_token, route_ws, xa, h, z, total;
+  size_t err, ids, w, offsets, perm, inv, row_token, route_ws, xa, xg, h, z, total;
 };
 
 GroupedLayout grouped_layout(int64_t M, int64_t E, int64_t H, int64_t I, int k, int r) {
@@ -68,6 +68,7 @@ GroupedLayout grouped_layout(int64_t M, int64_t E, int64_t H, int64_t I, int k, 
   L.row_token = c.take(S * sizeof(int32_t));
   L.route_ws = c.take(route_workspace_bytes(M, E, k));
   L.xa = c.take(r > 0 ? S * r * sizeof(float) : 0);
+  L.xg = c.take(S * H * sizeof(uint16_t));
   L.h = c.take(S * I * sizeof(uint16_t));
   L.z = c.take(S * H * sizeof(float));
   L.total = c.off;
@@ -272,9 +273,8 @@ e4b_status e4b_moe_route_permute(const float* logits, int64_t M, int64_t E, int 
 
 size_t e4b_grouped_nf4_gemm_workspace_size(int64_t total_rows, int64_t N, int64_t K, int r) {
   (void)N;
-  (void)K;
-  if (total_rows < 0 || r < 0) return 0;
-  return gemm_workspace_bytes(total_rows, r);
+  if (total_rows < 0 || r < 0 || K < 0) return 0;
+  return gemm_workspace_bytes(total_rows, K, r);
 }
 
 e4b_status e4b_grouped_nf4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda, const int32_t* row_index,
@@ -300,7 +300,7 @@ e4b_status e4b_grouped_nf4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda, 
   if (total_rows > INT32_MAX) return fail(E4B_ERR_UNSUPPORTED, "total_rows exceeds int32");
   if ((A && !aligned16(A)) || !aligned16(packed) || (out && !aligned16(out)))
     return fail(E4B_ERR_INVALID_ARGUMENT, "A, packed and out must be 16-byte aligned");
-  const size_t need = gemm_workspace_bytes(total_rows, r);
+  const size_t need = gemm_workspace_bytes(total_rows, K, r);
   if (workspace_bytes < need || (need > 0 && !workspace))
     return fail(E4B_ERR_WORKSPACE, "gemm workspace needs " + std::to_string(need) + " bytes");
   if (e4b_status s = check_device(); s != E4B_OK) return s;
@@ -325,7 +325,10 @@ e4b_status e4b_grouped_nf4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda, 
   g.r = r;
   g.lora_scale = lora_scale;
   g.err = static_cast<int*>(workspace);
-  g.xa = r > 0 ? reinterpret_cast<float*>(static_cast<char*>(workspace) + 256) : nullptr;
+  g.xa = r > 0 ? reinterpret_cast<float*>(static_cast<char*>(workspace) + gemm_workspace_xa_offset()) : nullptr;
+  g.a_gathered = row_index ? reinterpret_cast<uint16_t*>(static_cast<char*>(workspace) +
+                                                         gemm_workspace_gather_offset(total_rows, r))
+                           : nullptr;
   g.epi = epi;
   g.out = out;
   g.out_bf16 = out_dtype == E4B_BF16;
@@ -388,6 +391,7 @@ static e4b_status forward_grouped(const uint16_t* x, int64_t M, const float* log
   g.r = r;
   g.lora_scale = r ? w->lora_alpha / static_cast<float>(r) : 0.0f;
   g.xa = r ? at<float>(ws, L.xa) : nullptr;
+  g.a_gathered = at<uint16_t>(ws, L.xg);
   g.err = at<int>(ws, L.err);
   g.epi = E4B_EPI_SWIGLU;
   g.out = at<uint16_t>(ws, L.h);

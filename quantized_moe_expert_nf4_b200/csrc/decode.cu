@@ -6,24 +6,28 @@
 // layer step ("CUDA-graph decode capture").  Here the whole layer is two
 // kernels chained with programmatic dependent launch:
 //
-//   kernel A  routing (every CTA, redundantly: M <= 8 tokens), then for every
-//             touched expert and block of 8 output columns, the gate and up
-//             rows (8 + 8 weight rows, all of K = H) -> SiLU(gate) * up -> h
-//             (bf16, [M*k, I], slot order); also prefetches the down rows of
-//             the touched experts into L2 so HBM never idles between kernels.
-//   kernel B  routing again, then for every block of 16 output rows of H, the
-//             down rows of every touched expert in ascending expert order,
-//             accumulated with the routing weights folded in -> out (bf16).
-//             The sum over a token's experts happens inside one CTA in a fixed
-//             order, so the result is deterministic.
+//   kernel A  routing (every CTA, redundantly: M <= 8 tokens), then the gate
+//             and up rows of every touched expert in items of 8 gate + 8 up
+//             rows over all of K = H -> SiLU(gate) * up (+ LoRA delta) -> h
+//             (bf16, [M*k, I], slot order).  It also prefetches the touched
+//             experts' down rows into L2, so that HBM keeps streaming while the
+//             second kernel starts.
+//   kernel B  routing again (before it waits on kernel A), then for every block
+//             of 16 output rows of H the down rows of every touched expert, with
+//             the routing weights folded into the per-block scale, so the
+//             combine happens inside the CTA in a fixed order (deterministic).
 //
-// Only the experts that some token selected are read.  Weight rows stream
-// through a shared-memory ring filled by 1-D bulk copies (TMA engine) from one
-// producer thread; 16 consumer warps split K, decode nibbles through a
-// per-lane-replicated byte -> bf16x2 codebook table (conflict-free) into
-// mma.sync m16n8k16 fragments (weight rows = M dimension, tokens = the 8
-// columns), and fold each 64-block's absmax into the fp32 accumulator once.
+// Only experts that some token selected are read.  Both kernels are split-K
+// GEMVs on warp tensor cores: each CTA owns a contiguous run of items, its 16
+// warps split K, and each warp loads its 8-byte slices of the packed rows
+// straight from HBM into the registers of an mma.sync m16n8k16 fragment
+// (weight rows = MMA rows, the <= 8 tokens = the 8 MMA columns), several
+// items ahead, so ~100 KB per SM are in flight.  Nibbles become bf16 through a
+// per-lane replicated byte -> bf16x2 codebook table in shared memory (lane l
+// reads only bank l), and each 64-block's absmax is applied to the fp32 partial
+// product once.  One block barrier per batch gathers the 16 warps' partials.
 #include <algorithm>
+#include <mutex>
 
 #include "async.cuh"
 #include "common.cuh"
@@ -34,9 +38,11 @@ namespace e4b {
 namespace {
 
 constexpr int kMaxM = 8;
-constexpr int kCW = 16;                   // consumer warps
-constexpr int kThreads = (kCW + 1) * 32;  // + one producer warp
-constexpr uint32_t kRingBytes = 96 * 1024;
+constexpr int kWarps = 16;
+constexpr int kThreads = kWarps * 32;
+constexpr int kSlots = 8;                  // (item, k-block) load slots per warp per batch in kernel A
+constexpr int kPairSlots = 4;              // (expert, k-block) load slots per warp per batch in kernel B
+constexpr int kMaxKBW = 4;                 // k-blocks per warp per item: H <= 64 * 16 * 4 = 4096
 constexpr unsigned long long kPrefetchLimit = 64ull << 20;
 constexpr uint32_t kPrefetchChunk = 32 * 1024;
 
@@ -55,64 +61,27 @@ struct DecodeParams {
   float lora_scale;
   uint16_t* h;    // [S, I] bf16 (slot order)
   uint16_t* out;  // [M, H] bf16
-  int* err;
 };
-
-// Stage geometry for 16 weight rows of length K (bytes, with bank padding).
-struct StageGeom {
-  uint32_t row_stride;    // packed row stride in smem (bytes)
-  uint32_t am_stride;     // absmax row stride in smem (floats)
-  bool per_row_absmax;    // absmax copied row by row (padded) or 8 rows at a time
-  uint32_t packed_bytes;  // 16 * row_stride
-  uint32_t bytes;         // whole stage (packed + absmax), multiple of 128
-  uint32_t tx_bytes;      // bytes the bulk copies deliver
-};
-
-__host__ __device__ inline StageGeom stage_geom(int K) {
-  StageGeom g;
-  const uint32_t rb = static_cast<uint32_t>(K / 2);
-  // row stride = 32 (mod 128): the 8 rows a warp reads at once fall in distinct banks
-  g.row_stride = rb + ((32u - (rb % 128u)) + 128u) % 128u;
-  const uint32_t kb = static_cast<uint32_t>(K / 64);
-  if (kb % 4 == 0) {
-    g.per_row_absmax = true;
-    g.am_stride = kb + (((kb / 4) % 2 == 0) ? 4u : 8u);  // 4 * odd words: distinct banks
-  } else {
-    g.per_row_absmax = false;  // kb odd or 2 mod 4: unpadded rows are conflict-free
-    g.am_stride = kb;
-  }
-  g.packed_bytes = 16 * g.row_stride;
-  const uint32_t am_bytes = 16 * g.am_stride * 4;
-  g.bytes = (g.packed_bytes + am_bytes + 127u) / 128u * 128u;
-  g.tx_bytes = 16 * rb + 16 * kb * 4;
-  return g;
-}
 
 struct Layout {
-  uint32_t ring, bars, lut, xs, red, ids, w, uidx, touched, slotmap, xa, total;
-  int stages;
-  StageGeom geom;
+  uint32_t lut, xs, red, ids, w, uidx, touched, slotmap, xa, total;
 };
 
 __host__ __device__ inline uint32_t al(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
+__host__ __device__ inline int kbw_of(int H) { return (H / 64 + kWarps - 1) / kWarps; }
+
 // Shared-memory carve of kernel A (gate_up) or B (down).
-__host__ __device__ inline Layout make_layout(bool is_a, int M, int k, int E, int H, int I, int r) {
+__host__ __device__ inline Layout make_layout(bool is_a, int M, int k, int E, int H, int r) {
   Layout L;
-  L.geom = stage_geom(is_a ? H : I);
-  int st = static_cast<int>(kRingBytes / L.geom.bytes);
-  L.stages = st < 2 ? 2 : (st > 12 ? 12 : st);
   uint32_t o = 0;
-  L.ring = o;
-  o = al(o + L.stages * L.geom.bytes, 128);
-  L.bars = o;
-  o = al(o + 2 * L.stages * 8, 16);
   L.lut = o;
   o = al(o + 256 * 32 * 4, 16);
   L.xs = o;
   if (is_a) o = al(o + M * (2 * H + 16), 16);
   L.red = o;
-  o = al(o + 2 * kCW * 32 * 16, 16);
+  const int items = is_a ? kSlots : 1;  // partial sums of up to 8 items per batch (A), 1 row block (B)
+  o = al(o + items * kWarps * 32 * 16, 16);
   const int S = M * k;
   L.ids = o;
   o = al(o + S * 4, 16);
@@ -139,7 +108,7 @@ __device__ __forceinline__ void mma_16816(float c[4], uint32_t a0, uint32_t a1, 
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// One 64-block of a 16-row stage: rows g (A rows 0..7) and g+8, thread t owns
+// One 64-block of a 16-row tile: rows g (MMA rows 0..7) and g+8, thread t owns
 // physical k in [16t, 16t+16) = 8 byte pairs; MMA j takes pairs 2j and 2j+1.
 __device__ __forceinline__ void block_mma(const uint32_t* __restrict__ lut_lane, uint2 r0, uint2 r1, uint4 x0, uint4 x1,
                                           float tmp[4]) {
@@ -151,16 +120,55 @@ __device__ __forceinline__ void block_mma(const uint32_t* __restrict__ lut_lane,
   mma_16816(tmp, L(r0.y, 2), L(r1.y, 2), L(r0.y, 3), L(r1.y, 3), x1.z, x1.w);
 }
 
-// Routing of all M tokens into shared memory (every CTA does it; M <= 8).
-// Builds: ids/w per slot, the touched experts in ascending id order, and
-// slotmap[u][t] = slot of token t in expert touched[u] (or -1).
-template <int MAXJ>
-__device__ void decode_route(const DecodeParams& p, int* ids_s, float* w_s, int* uidx, int* touched, int* slotmap,
-                             int* nU_out) {
+__device__ __forceinline__ uint2 ld_stream_u2(const uint8_t* p) {
+  return __ldcs(reinterpret_cast<const uint2*>(p));
+}
+
+// Top-k of token `t` by the calling warp, with the key array sized for E.
+__device__ __forceinline__ void route_one(const DecodeParams& p, int t, int* ids_s, float* w_s) {
+  const int maxj = (p.E + 31) / 32;
+  if (maxj <= 1) route_token<1>(p.logits, t, p.E, p.k, p.renorm != 0, ids_s, w_s);
+  else if (maxj <= 2) route_token<2>(p.logits, t, p.E, p.k, p.renorm != 0, ids_s, w_s);
+  else if (maxj <= 4) route_token<4>(p.logits, t, p.E, p.k, p.renorm != 0, ids_s, w_s);
+  else if (maxj <= 8) route_token<8>(p.logits, t, p.E, p.k, p.renorm != 0, ids_s, w_s);
+  else route_token<16>(p.logits, t, p.E, p.k, p.renorm != 0, ids_s, w_s);
+}
+
+// Byte -> bf16x2 codebook pairs, replicated per lane (entry b of lane l at
+// b * 32 + l), written by the warps [w0, kWarps) of the block.
+__device__ __forceinline__ void fill_lut_warps(uint32_t* lut, int w0) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (warp < w0) return;
+  const float cbl = kNf4CodebookDev[lane & 15];
+  for (int b = warp - w0; b < 256; b += kWarps - w0) {
+    const float hi = __shfl_sync(0xffffffffu, cbl, b >> 4);
+    const float lo = __shfl_sync(0xffffffffu, cbl, b & 15);
+    lut[b * 32 + lane] = pack_bf16x2(hi, lo);
+  }
+}
+
+// Prologue shared by both kernels: warps < M route one token each while the
+// other warps build the codebook table (and, in kernel A, stage x).  Then the
+// touched experts (ascending id) and slotmap[u][t] = slot of token t in expert
+// touched[u] (or -1) are built.
+__device__ void decode_prologue(const DecodeParams& p, uint32_t* lut, uint16_t* xs, int xstride, int* ids_s,
+                                float* w_s, int* uidx, int* touched, int* slotmap, int* nU_out) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int S = p.M * p.k;
   for (int e = tid; e < p.E; e += blockDim.x) uidx[e] = -1;
-  if (warp < p.M) route_token<MAXJ>(p.logits, warp, p.E, p.k, p.renorm != 0, ids_s, w_s);
+  if (warp < p.M) {
+    route_one(p, warp, ids_s, w_s);
+  } else {
+    fill_lut_warps(lut, p.M);
+    if (xs) {
+      const int nthr = (kWarps - p.M) * 32, me = tid - p.M * 32;
+      for (int i = me; i < p.M * (p.H / 8); i += nthr) {
+        const int t = i / (p.H / 8), c = i % (p.H / 8);
+        reinterpret_cast<uint4*>(xs + t * xstride)[c] =
+            reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(t) * p.H)[c];
+      }
+    }
+  }
   __syncthreads();
   for (int s = tid; s < S; s += blockDim.x) uidx[ids_s[s]] = 0;  // flag
   __syncthreads();
@@ -169,13 +177,13 @@ __device__ void decode_route(const DecodeParams& p, int* ids_s, float* w_s, int*
     for (int base = 0; base < p.E; base += 32) {
       const int e = base + lane;
       const bool f = (e < p.E) && uidx[e] == 0;
-      const uint32_t b = __ballot_sync(0xffffffffu, f);
+      const uint32_t bal = __ballot_sync(0xffffffffu, f);
       if (f) {
-        const int u = count + __popc(b & lanemask_lt());
+        const int u = count + __popc(bal & lanemask_lt());
         touched[u] = e;
         uidx[e] = u;
       }
-      count += __popc(b);
+      count += __popc(bal);
     }
     if (lane == 0) *nU_out = count;
   }
@@ -187,45 +195,28 @@ __device__ void decode_route(const DecodeParams& p, int* ids_s, float* w_s, int*
   __syncthreads();
 }
 
-__device__ __forceinline__ void fill_lut(uint32_t* lut) {
-  for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) {
-    const int b = i >> 5;
-    lut[i] = pack_bf16x2(kNf4CodebookDev[b >> 4], kNf4CodebookDev[b & 15]);
-  }
-}
-
-// Producer: issue the bulk copies of one 16-row stage (rows row0[0..7], row1[0..7]
-// as two runs of 8 consecutive rows) into `dst`.
-__device__ __forceinline__ void issue_stage(const StageGeom& g, unsigned char* dst, uint64_t* full, const uint8_t* packed,
-                                            const float* absmax, int K, int64_t run0, int64_t run1) {
-  const uint32_t rb = K / 2, kb = K / 64;
-  mbar_arrive_expect_tx(full, g.tx_bytes);
-  const int64_t runs[2] = {run0, run1};
-  float* am = reinterpret_cast<float*>(dst + g.packed_bytes);
-  for (int h = 0; h < 2; ++h) {
-    const int64_t r0 = runs[h];
-    if (g.row_stride == rb) {
-      bulk_g2s(dst + h * 8 * g.row_stride, packed + r0 * rb, 8 * rb, full);
-    } else {
-      for (int i = 0; i < 8; ++i) bulk_g2s(dst + (h * 8 + i) * g.row_stride, packed + (r0 + i) * rb, rb, full);
-    }
-    if (g.per_row_absmax) {
-      for (int i = 0; i < 8; ++i) bulk_g2s(am + (h * 8 + i) * g.am_stride, absmax + (r0 + i) * kb, kb * 4, full);
-    } else {
-      bulk_g2s(am + h * 8 * g.am_stride, absmax + r0 * kb, 8 * kb * 4, full);
-    }
-  }
+// L2 prefetch of the gate and up rows (and their absmax) of items [a, b),
+// one thread per item.
+__device__ __forceinline__ void prefetch_items(const DecodeParams& p, const int* touched, int a, int b) {
+  const int i = a + static_cast<int>(threadIdx.x);
+  if (i >= b) return;
+  const int ipe = p.I / 8;
+  const int u = i / ipe, rb = i % ipe;
+  const int64_t grow = static_cast<int64_t>(touched[u]) * 2 * p.I + rb * 8;
+  const int64_t row_bytes = p.H / 2, kb = p.H / 64;
+  prefetch_l2(p.gu_packed + grow * row_bytes, static_cast<uint32_t>(8 * row_bytes));
+  prefetch_l2(p.gu_packed + (grow + p.I) * row_bytes, static_cast<uint32_t>(8 * row_bytes));
+  prefetch_l2(p.gu_absmax + grow * kb, static_cast<uint32_t>(8 * kb * 4));
+  prefetch_l2(p.gu_absmax + (grow + p.I) * kb, static_cast<uint32_t>(8 * kb * 4));
 }
 
 // ---------------------------------------------------------------------------
-// Kernel A: gate_up + SwiGLU (+ LoRA delta) -> h
-template <int MAXJ>
+// Kernel A: gate_up + SwiGLU (+ LoRA delta) -> h.  KBW = k-blocks per warp per item.
+template <int KBW>
 __global__ void __launch_bounds__(kThreads, 1) decode_gate_up_kernel(DecodeParams p) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  const Layout L = make_layout(true, p.M, p.k, p.E, p.H, p.I, p.r);
-  const StageGeom& G = L.geom;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
-  uint64_t* empty = full + L.stages;
+  constexpr int IB = kSlots / KBW;  // items per batch
+  extern __shared__ __align__(16) unsigned char smem[];
+  const Layout L = make_layout(true, p.M, p.k, p.E, p.H, p.r);
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L.lut);
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem + L.xs);
   float4* red = reinterpret_cast<float4*>(smem + L.red);
@@ -238,145 +229,152 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gate_up_kernel(DecodeParam
   __shared__ int nU_s;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int H = p.H, I = p.I;
-  const int xstride = H + 8;  // bf16 elements (2H + 16 bytes)
+  const int H = p.H, I = p.I, KB = H / 64;
+  const int xstride = H + 8;  // bf16 elements (2H + 16 bytes: conflict-free 16-byte reads)
 
-  if (tid == 0) {
-    for (int s = 0; s < L.stages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kCW);
-    }
-    fence_mbar_init();
-  }
-  pdl_wait();               // inputs of this call are final
-  if (blockIdx.x == 0 && tid == 0) *p.err = kErrNone;
+  pdl_wait();               // the inputs of this call are final
   pdl_launch_dependents();  // the down kernel may launch and run its prologue
-  fill_lut(lut);
-  for (int i = tid; i < p.M * (H / 8); i += blockDim.x) {
-    const int t = i / (H / 8), c = i % (H / 8);
-    reinterpret_cast<uint4*>(xs + t * xstride)[c] = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(t) * H)[c];
-  }
-  decode_route<MAXJ>(p, ids_s, w_s, uidx, touched, slotmap, &nU_s);
+  decode_prologue(p, lut, xs, xstride, ids_s, w_s, uidx, touched, slotmap, &nU_s);
   const int nU = nU_s;
-  const int items_per_expert = I / 8;
-  const int nitems = nU * items_per_expert;
+  const int ipe = I / 8;  // items per expert
+  const int nitems = nU * ipe;
+  // A contiguous run of items per CTA: consecutive items are consecutive rows.
+  const int q = nitems / gridDim.x, rem = nitems % gridDim.x;
+  const int i0 = blockIdx.x * q + min(static_cast<int>(blockIdx.x), rem);
+  const int i1 = i0 + q + (static_cast<int>(blockIdx.x) < rem ? 1 : 0);
 
-  if (warp == kCW) {
-    // ---------------- producer warp ----------------
-    if (lane == 0) {
-      int j = 0;
-      for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++j) {
-        const int s = j % L.stages;
-        if (j >= L.stages && !mbar_wait(&empty[s], ((j / L.stages) - 1) & 1)) {
-          record_error(p.err, kErrWaitEmpty);
-          break;
-        }
-        const int u = it / items_per_expert, rb = it % items_per_expert;
-        const int64_t e = touched[u];
-        const int64_t gate0 = e * 2 * I + rb * 8, up0 = gate0 + I;
-        issue_stage(G, smem + L.ring + s * G.bytes, &full[s], p.gu_packed, p.gu_absmax, H, gate0, up0);
-      }
-    } else {
-      // Lanes 1..31: prefetch this CTA's share of the touched experts' down rows into L2.
-      const uint64_t per_expert = static_cast<uint64_t>(H) * I / 2;
-      const uint64_t per_expert_am = static_cast<uint64_t>(H) * (I / 64) * 4;
-      const uint64_t chunks_pk = (per_expert + kPrefetchChunk - 1) / kPrefetchChunk;
-      const uint64_t chunks_am = (per_expert_am + kPrefetchChunk - 1) / kPrefetchChunk;
-      const uint64_t per_u = chunks_pk + chunks_am;
-      uint64_t total = static_cast<uint64_t>(nU) * per_u;
-      const uint64_t cap = kPrefetchLimit / kPrefetchChunk;
-      if (total > cap) total = cap;
-      for (uint64_t c = static_cast<uint64_t>(blockIdx.x) * 31 + (lane - 1); c < total;
-           c += static_cast<uint64_t>(gridDim.x) * 31) {
-        const uint64_t u = c / per_u, q = c % per_u;
-        const int64_t e = touched[u];
-        if (q < chunks_pk) {
-          const uint64_t off = q * kPrefetchChunk;
-          const uint64_t n = min(static_cast<uint64_t>(kPrefetchChunk), per_expert - off);
-          prefetch_l2(p.dn_packed + e * per_expert + off, static_cast<uint32_t>(n));
-        } else {
-          const uint64_t off = (q - chunks_pk) * kPrefetchChunk;
-          const uint64_t n = min(static_cast<uint64_t>(kPrefetchChunk), per_expert_am - off);
-          prefetch_l2(reinterpret_cast<const unsigned char*>(p.dn_absmax) + e * per_expert_am + off,
-                      static_cast<uint32_t>(n));
-        }
+  if (warp == kWarps - 1) {
+    // Prefetch this CTA's share of the touched experts' down rows into L2.
+    const uint64_t per_expert = static_cast<uint64_t>(H) * I / 2;
+    const uint64_t per_expert_am = static_cast<uint64_t>(H) * (I / 64) * 4;
+    const uint64_t chunks_pk = (per_expert + kPrefetchChunk - 1) / kPrefetchChunk;
+    const uint64_t chunks_am = (per_expert_am + kPrefetchChunk - 1) / kPrefetchChunk;
+    const uint64_t per_u = chunks_pk + chunks_am;
+    uint64_t total = static_cast<uint64_t>(nU) * per_u;
+    const uint64_t cap = kPrefetchLimit / kPrefetchChunk;
+    if (total > cap) total = cap;
+    for (uint64_t c = static_cast<uint64_t>(blockIdx.x) * 32 + lane; c < total; c += static_cast<uint64_t>(gridDim.x) * 32) {
+      const uint64_t u = c / per_u, qq = c % per_u;
+      const int64_t e = touched[u];
+      if (qq < chunks_pk) {
+        const uint64_t off = qq * kPrefetchChunk;
+        const uint64_t n = min(static_cast<uint64_t>(kPrefetchChunk), per_expert - off);
+        prefetch_l2(p.dn_packed + e * per_expert + off, static_cast<uint32_t>(n));
+      } else {
+        const uint64_t off = (qq - chunks_pk) * kPrefetchChunk;
+        const uint64_t n = min(static_cast<uint64_t>(kPrefetchChunk), per_expert_am - off);
+        prefetch_l2(reinterpret_cast<const unsigned char*>(p.dn_absmax) + e * per_expert_am + off,
+                    static_cast<uint32_t>(n));
       }
     }
-    return;
   }
 
-  // ---------------- consumer warps ----------------
   const int g = lane >> 2, t = lane & 3;
   const int S = p.M * p.k;
   if (p.r > 0) {
     // LoRA first factor per slot: xa[s, rho] = x[token(s)] . lora_A[e(s), rho]
-    for (int q = warp; q < S * p.r; q += kCW) {
-      const int s = q / p.r, rho = q % p.r;
+    for (int qd = warp; qd < S * p.r; qd += kWarps) {
+      const int s = qd / p.r, rho = qd % p.r;
       const int tok = s / p.k;
       const uint16_t* la = p.lora_A + (static_cast<int64_t>(ids_s[s]) * p.r + rho) * H;
       float acc = 0.f;
-      for (int kk = lane; kk < H; kk += 32)
-        acc = fmaf(bf16_bits_to_float(xs[tok * xstride + kk]), bf16_bits_to_float(la[kk]), acc);
+      for (int kk = lane * 8; kk < H; kk += 256) {
+        const uint4 xv = *reinterpret_cast<const uint4*>(xs + tok * xstride + kk);
+        const uint4 av = *reinterpret_cast<const uint4*>(la + kk);
+        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, aw[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc = fmaf(__uint_as_float(xw[i] << 16), __uint_as_float(aw[i] << 16), acc);
+          acc = fmaf(__uint_as_float(xw[i] & 0xffff0000u), __uint_as_float(aw[i] & 0xffff0000u), acc);
+        }
+      }
 #pragma unroll
       for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) xa[q] = acc;
+      if (lane == 0) xa[qd] = acc;
     }
-    named_barrier(1, kCW * 32);
+    __syncthreads();
   }
   const uint32_t* lut_lane = lut + lane;
-  const int KB = H / 64;
-  int j = 0;
-  for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++j) {
-    const int s = j % L.stages;
-    const int u = it / items_per_expert, rb = it % items_per_expert;
-    const int slot_g = (g < p.M) ? slotmap[u * kMaxM + g] : -1;
-    const uint16_t* xrow = xs + g * xstride + 16 * t;
-    if (!mbar_wait(&full[s], (j / L.stages) & 1)) {
-      record_error(p.err, kErrWaitFull);
-      break;
-    }
-    const unsigned char* st = smem + L.ring + s * G.bytes;
-    const float* am = reinterpret_cast<const float*>(st + G.packed_bytes);
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int kb = warp; kb < KB; kb += kCW) {
-      const uint2 r0 = *reinterpret_cast<const uint2*>(st + g * G.row_stride + kb * 32 + 8 * t);
-      const uint2 r1 = *reinterpret_cast<const uint2*>(st + (g + 8) * G.row_stride + kb * 32 + 8 * t);
-      const float a0 = am[g * G.am_stride + kb], a1 = am[(g + 8) * G.am_stride + kb];
-      uint4 x0 = make_uint4(0, 0, 0, 0), x1 = make_uint4(0, 0, 0, 0);
-      if (slot_g >= 0) {
-        x0 = *reinterpret_cast<const uint4*>(xrow + kb * 64);
-        x1 = *reinterpret_cast<const uint4*>(xrow + kb * 64 + 8);
+  const int64_t row_bytes = H / 2;
+  // Batches after the first read L2: keep the bulk prefetch two batches ahead.
+  if (tid < 2 * IB) prefetch_items(p, touched, min(i0 + IB, i1), min(i0 + 3 * IB, i1));
+  for (int b0 = i0; b0 < i1; b0 += IB) {
+    const int nb = min(IB, i1 - b0);
+    if (b0 > i0 && tid < IB) prefetch_items(p, touched, min(b0 + 2 * IB, i1), min(b0 + 3 * IB, i1));
+    // Issue every load of the batch first (HBM latency is hidden by the batch).
+    uint2 pk[IB][KBW][2];
+    float am[IB][KBW][2];
+#pragma unroll
+    for (int ii = 0; ii < IB; ++ii) {
+      const int it = b0 + (ii < nb ? ii : 0);
+      const int u = it / ipe, rb = it % ipe;
+      const int64_t grow = static_cast<int64_t>(touched[u]) * 2 * I + rb * 8 + g;  // gate row of lane's MMA row g
+      const uint8_t* gp = p.gu_packed + grow * row_bytes + 8 * t;
+      const uint8_t* up = gp + static_cast<int64_t>(I) * row_bytes;
+      const float* ga = p.gu_absmax + grow * KB;
+      const float* ua = ga + static_cast<int64_t>(I) * KB;
+#pragma unroll
+      for (int q2 = 0; q2 < KBW; ++q2) {
+        const int kb = warp + kWarps * q2;
+        if (ii < nb && kb < KB) {
+          pk[ii][q2][0] = ld_stream_u2(gp + kb * 32);
+          pk[ii][q2][1] = ld_stream_u2(up + kb * 32);
+          am[ii][q2][0] = __ldg(ga + kb);
+          am[ii][q2][1] = __ldg(ua + kb);
+        } else {
+          pk[ii][q2][0] = pk[ii][q2][1] = make_uint2(0, 0);
+          am[ii][q2][0] = am[ii][q2][1] = 0.f;
+        }
       }
-      float tmp[4];
-      block_mma(lut_lane, r0, r1, x0, x1, tmp);
-      acc[0] = fmaf(tmp[0], a0, acc[0]);
-      acc[1] = fmaf(tmp[1], a0, acc[1]);
-      acc[2] = fmaf(tmp[2], a1, acc[2]);
-      acc[3] = fmaf(tmp[3], a1, acc[3]);
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
-    red[((j & 1) * kCW + warp) * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    named_barrier(1, kCW * 32);
-    if (warp == 0) {
+#pragma unroll
+    for (int ii = 0; ii < IB; ++ii) {
+      if (ii >= nb) break;
+      const int u = (b0 + ii) / ipe;
+      const bool has_g = (g < p.M) && slotmap[u * kMaxM + g] >= 0;  // token g routes to this expert
+      const uint16_t* xrow = xs + g * xstride + 16 * t;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int q2 = 0; q2 < KBW; ++q2) {
+        const int kb = warp + kWarps * q2;
+        if (kb >= KB) break;
+        uint4 x0 = make_uint4(0, 0, 0, 0), x1 = make_uint4(0, 0, 0, 0);
+        if (has_g) {
+          x0 = *reinterpret_cast<const uint4*>(xrow + kb * 64);
+          x1 = *reinterpret_cast<const uint4*>(xrow + kb * 64 + 8);
+        }
+        float tmp[4];
+        block_mma(lut_lane, pk[ii][q2][0], pk[ii][q2][1], x0, x1, tmp);
+        acc[0] = fmaf(tmp[0], am[ii][q2][0], acc[0]);
+        acc[1] = fmaf(tmp[1], am[ii][q2][0], acc[1]);
+        acc[2] = fmaf(tmp[2], am[ii][q2][1], acc[2]);
+        acc[3] = fmaf(tmp[3], am[ii][q2][1], acc[3]);
+      }
+      red[(ii * kWarps + warp) * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    }
+    __syncthreads();
+    if (warp < nb) {
+      // Warp `warp` finishes item b0 + warp: sum the 16 partials in warp order.
       float4 c = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int w = 0; w < kCW; ++w) {
-        const float4 v = red[((j & 1) * kCW + w) * 32 + lane];
+      for (int w = 0; w < kWarps; ++w) {
+        const float4 v = red[(warp * kWarps + w) * 32 + lane];
         c.x += v.x;
         c.y += v.y;
         c.z += v.z;
         c.w += v.w;
       }
+      const int it = b0 + warp;
+      const int u = it / ipe, rb = it % ipe;
       const int e = touched[u];
       const int col = rb * 8 + g;  // h column == gate row index
       const float gate_v[2] = {c.x, c.y}, up_v[2] = {c.z, c.w};
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const int tok = 2 * t + q;
+      for (int qq = 0; qq < 2; ++qq) {
+        const int tok = 2 * t + qq;
         if (tok >= p.M) continue;
         const int slot = slotmap[u * kMaxM + tok];
         if (slot < 0) continue;
-        float gv = gate_v[q], uv = up_v[q];
+        float gv = gate_v[qq], uv = up_v[qq];
         if (p.r > 0) {
           const uint16_t* bg = p.lora_B + (static_cast<int64_t>(e) * 2 * I + col) * p.r;
           const uint16_t* bu = p.lora_B + (static_cast<int64_t>(e) * 2 * I + I + col) * p.r;
@@ -392,18 +390,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gate_up_kernel(DecodeParam
         p.h[static_cast<int64_t>(slot) * I + col] = float_to_bf16_bits(silu_f32(gv) * uv);
       }
     }
+    __syncthreads();
   }
 }
 
 // ---------------------------------------------------------------------------
-// Kernel B: down rows of every touched expert, weighted combine -> out
-template <int MAXJ>
+// Kernel B: down rows of every touched expert, weighted combine -> out.
 __global__ void __launch_bounds__(kThreads, 1) decode_down_kernel(DecodeParams p) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  const Layout L = make_layout(false, p.M, p.k, p.E, p.H, p.I, 0);
-  const StageGeom& G = L.geom;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
-  uint64_t* empty = full + L.stages;
+  extern __shared__ __align__(16) unsigned char smem[];
+  const Layout L = make_layout(false, p.M, p.k, p.E, p.H, 0);
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L.lut);
   float4* red = reinterpret_cast<float4*>(smem + L.red);
   int* ids_s = reinterpret_cast<int*>(smem + L.ids);
@@ -414,108 +409,73 @@ __global__ void __launch_bounds__(kThreads, 1) decode_down_kernel(DecodeParams p
   __shared__ int nU_s;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int H = p.H, I = p.I;
-  if (tid == 0) {
-    for (int s = 0; s < L.stages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kCW);
-    }
-    fence_mbar_init();
-  }
-  // The prologue only reads inputs the gate_up kernel does not write.
-  fill_lut(lut);
-  decode_route<MAXJ>(p, ids_s, w_s, uidx, touched, slotmap, &nU_s);
+  const int H = p.H, I = p.I, KB = I / 64;
+  // The prologue reads only inputs the gate_up kernel does not write.
+  decode_prologue(p, lut, nullptr, 0, ids_s, w_s, uidx, touched, slotmap, &nU_s);
   const int nU = nU_s;
-  const int nrb = H / 16;
-
-  if (warp == kCW) {
-    if (lane == 0) {
-      // Weights do not depend on the gate_up kernel: start streaming at once.
-      int j = 0;
-      for (int rb = blockIdx.x; rb < nrb; rb += gridDim.x) {
-        bool ok = true;
-        for (int u = 0; u < nU; ++u, ++j) {
-          const int s = j % L.stages;
-          if (j >= L.stages && !mbar_wait(&empty[s], ((j / L.stages) - 1) & 1)) {
-            record_error(p.err, kErrWaitEmpty);
-            ok = false;
-            break;
-          }
-          const int64_t row0 = static_cast<int64_t>(touched[u]) * H + rb * 16;
-          issue_stage(G, smem + L.ring + s * G.bytes, &full[s], p.dn_packed, p.dn_absmax, I, row0, row0 + 8);
-        }
-        if (!ok) break;
-      }
-    }
-    return;
-  }
-
-  pdl_wait();  // h written by the gate_up kernel is visible from here on
+  const int npairs = nU * KB;  // (expert, k-block) pairs of one row block
   const int g = lane >> 2, t = lane & 3;
   const uint32_t* lut_lane = lut + lane;
-  const int KB = I / 64;
-  int j = 0, item = 0;
-  bool ok = true;
-  for (int rb = blockIdx.x; rb < nrb && ok; rb += gridDim.x, ++item) {
+  const int64_t row_bytes = I / 2;
+  // L2 prefetch of this CTA's first row block of every touched expert (weights
+  // do not depend on the gate_up kernel, so this runs before the wait).
+  for (int u = tid; u < nU && static_cast<int>(blockIdx.x) < H / 16; u += blockDim.x) {
+    const int64_t row = static_cast<int64_t>(touched[u]) * H + blockIdx.x * 16;
+    prefetch_l2(p.dn_packed + row * row_bytes, static_cast<uint32_t>(16 * row_bytes));
+    prefetch_l2(p.dn_absmax + row * KB, static_cast<uint32_t>(16 * KB * 4));
+  }
+  pdl_wait();  // h written by the gate_up kernel is visible from here on
+  for (int rb = blockIdx.x; rb < H / 16; rb += gridDim.x) {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int u = 0; u < nU; ++u, ++j) {
-      const int s = j % L.stages;
-      // token columns g (B operand) and 2t, 2t+1 (accumulator columns)
-      const int slot_g = (g < p.M) ? slotmap[u * kMaxM + g] : -1;
-      const int sc0 = (2 * t < p.M) ? slotmap[u * kMaxM + 2 * t] : -1;
-      const int sc1 = (2 * t + 1 < p.M) ? slotmap[u * kMaxM + 2 * t + 1] : -1;
-      const float wc0 = sc0 >= 0 ? w_s[sc0] : 0.f, wc1 = sc1 >= 0 ? w_s[sc1] : 0.f;
-      const uint16_t* hrow = p.h + static_cast<int64_t>(slot_g < 0 ? 0 : slot_g) * I + 16 * t;
-      // Issue the h loads of this stage before waiting for its weights.
-      uint4 hx[2][2];
-      int nkb = 0;
-      for (int kb = warp; kb < KB && nkb < 2; kb += kCW, ++nkb) {
-        hx[nkb][0] = hx[nkb][1] = make_uint4(0, 0, 0, 0);
-        if (slot_g >= 0) {
-          hx[nkb][0] = *reinterpret_cast<const uint4*>(hrow + kb * 64);
-          hx[nkb][1] = *reinterpret_cast<const uint4*>(hrow + kb * 64 + 8);
-        }
-      }
-      if (!mbar_wait(&full[s], (j / L.stages) & 1)) {
-        record_error(p.err, kErrWaitFull);
-        ok = false;
-        break;
-      }
-      const unsigned char* st = smem + L.ring + s * G.bytes;
-      const float* am = reinterpret_cast<const float*>(st + G.packed_bytes);
-      int q = 0;
-      for (int kb = warp; kb < KB; kb += kCW, ++q) {
-        uint4 x0, x1;
-        if (q < 2) {
-          x0 = hx[q][0];
-          x1 = hx[q][1];
-        } else {
-          x0 = x1 = make_uint4(0, 0, 0, 0);
+    for (int pb = warp; pb < npairs; pb += kWarps * kPairSlots) {
+      uint2 pk[kPairSlots][2];
+      float am[kPairSlots][2];
+      uint4 hx[kPairSlots][2];
+      float wc[kPairSlots][2];
+#pragma unroll
+      for (int sl = 0; sl < kPairSlots; ++sl) {
+        const int pi = pb + kWarps * sl;
+        pk[sl][0] = pk[sl][1] = make_uint2(0, 0);
+        am[sl][0] = am[sl][1] = 0.f;
+        hx[sl][0] = hx[sl][1] = make_uint4(0, 0, 0, 0);
+        wc[sl][0] = wc[sl][1] = 0.f;
+        if (pi < npairs) {
+          const int u = pi / KB, kb = pi % KB;
+          const int64_t row = static_cast<int64_t>(touched[u]) * H + rb * 16 + g;
+          const uint8_t* rp = p.dn_packed + row * row_bytes + kb * 32 + 8 * t;
+          pk[sl][0] = ld_stream_u2(rp);
+          pk[sl][1] = ld_stream_u2(rp + 8 * row_bytes);
+          am[sl][0] = __ldg(p.dn_absmax + row * KB + kb);
+          am[sl][1] = __ldg(p.dn_absmax + (row + 8) * KB + kb);
+          const int slot_g = (g < p.M) ? slotmap[u * kMaxM + g] : -1;
           if (slot_g >= 0) {
-            x0 = *reinterpret_cast<const uint4*>(hrow + kb * 64);
-            x1 = *reinterpret_cast<const uint4*>(hrow + kb * 64 + 8);
+            const uint16_t* hr = p.h + static_cast<int64_t>(slot_g) * I + kb * 64 + 16 * t;
+            hx[sl][0] = *reinterpret_cast<const uint4*>(hr);
+            hx[sl][1] = *reinterpret_cast<const uint4*>(hr + 8);
           }
+          const int s0 = (2 * t < p.M) ? slotmap[u * kMaxM + 2 * t] : -1;
+          const int s1 = (2 * t + 1 < p.M) ? slotmap[u * kMaxM + 2 * t + 1] : -1;
+          wc[sl][0] = s0 >= 0 ? w_s[s0] : 0.f;
+          wc[sl][1] = s1 >= 0 ? w_s[s1] : 0.f;
         }
-        const uint2 r0 = *reinterpret_cast<const uint2*>(st + g * G.row_stride + kb * 32 + 8 * t);
-        const uint2 r1 = *reinterpret_cast<const uint2*>(st + (g + 8) * G.row_stride + kb * 32 + 8 * t);
-        const float a0 = am[g * G.am_stride + kb], a1 = am[(g + 8) * G.am_stride + kb];
-        float tmp[4];
-        block_mma(lut_lane, r0, r1, x0, x1, tmp);
-        acc[0] = fmaf(tmp[0], a0 * wc0, acc[0]);
-        acc[1] = fmaf(tmp[1], a0 * wc1, acc[1]);
-        acc[2] = fmaf(tmp[2], a1 * wc0, acc[2]);
-        acc[3] = fmaf(tmp[3], a1 * wc1, acc[3]);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
+#pragma unroll
+      for (int sl = 0; sl < kPairSlots; ++sl) {
+        if (pb + kWarps * sl >= npairs) break;
+        float tmp[4];
+        block_mma(lut_lane, pk[sl][0], pk[sl][1], hx[sl][0], hx[sl][1], tmp);
+        acc[0] = fmaf(tmp[0], am[sl][0] * wc[sl][0], acc[0]);
+        acc[1] = fmaf(tmp[1], am[sl][0] * wc[sl][1], acc[1]);
+        acc[2] = fmaf(tmp[2], am[sl][1] * wc[sl][0], acc[2]);
+        acc[3] = fmaf(tmp[3], am[sl][1] * wc[sl][1], acc[3]);
+      }
     }
-    if (!ok) break;
-    red[((item & 1) * kCW + warp) * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    named_barrier(1, kCW * 32);
+    red[warp * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    __syncthreads();
     if (warp == 0) {
       float4 c = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int w = 0; w < kCW; ++w) {
-        const float4 v = red[((item & 1) * kCW + w) * 32 + lane];
+      for (int w = 0; w < kWarps; ++w) {
+        const float4 v = red[w * 32 + lane];
         c.x += v.x;
         c.y += v.y;
         c.z += v.z;
@@ -530,26 +490,39 @@ __global__ void __launch_bounds__(kThreads, 1) decode_down_kernel(DecodeParams p
         if (tok < p.M) p.out[static_cast<int64_t>(tok) * H + row] = float_to_bf16_bits(v[q2]);
       }
     }
+    __syncthreads();
   }
 }
 
-template <int MAXJ>
-cudaError_t launch_pair(const DecodeParams& p, int sm_count, size_t smem_a, size_t smem_b, cudaStream_t stream) {
-  // The dynamic shared-memory limit is a per-function attribute: raise it to
-  // what this call needs (kept per instantiation; raising is idempotent).
-  static size_t configured_a = 0, configured_b = 0;
+// The dynamic shared-memory limit is a per-function attribute.  Each kernel
+// function keeps one high-water mark and the limit is only ever raised, so a
+// call with a smaller need never lowers the limit another call relies on.
+std::mutex g_attr_mu;
+size_t g_down_configured = 0;
+
+template <int KBW>
+cudaError_t raise_smem_limits(size_t smem_a, size_t smem_b) {
+  static size_t configured_a = 0;  // one per decode_gate_up_kernel<KBW>
+  std::lock_guard<std::mutex> lk(g_attr_mu);
   if (smem_a > configured_a) {
-    cudaError_t e1 = cudaFuncSetAttribute(decode_gate_up_kernel<MAXJ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e1 = cudaFuncSetAttribute(decode_gate_up_kernel<KBW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           static_cast<int>(smem_a));
     if (e1 != cudaSuccess) return e1;
     configured_a = smem_a;
   }
-  if (smem_b > configured_b) {
-    cudaError_t e1 = cudaFuncSetAttribute(decode_down_kernel<MAXJ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (smem_b > g_down_configured) {
+    cudaError_t e1 = cudaFuncSetAttribute(decode_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           static_cast<int>(smem_b));
     if (e1 != cudaSuccess) return e1;
-    configured_b = smem_b;
+    g_down_configured = smem_b;
   }
+  return cudaSuccess;
+}
+
+template <int KBW>
+cudaError_t launch_pair(const DecodeParams& p, int sm_count, size_t smem_a, size_t smem_b, cudaStream_t stream) {
+  cudaError_t aerr = raise_smem_limits<KBW>(smem_a, smem_b);
+  if (aerr != cudaSuccess) return aerr;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -563,37 +536,36 @@ cudaError_t launch_pair(const DecodeParams& p, int sm_count, size_t smem_a, size
   cfg.dynamicSmemBytes = smem_a;
   {
     LaunchScope ls("decode.gate_up", stream);
-    cudaError_t err = cudaLaunchKernelEx(&cfg, decode_gate_up_kernel<MAXJ>, p);
+    cudaError_t err = cudaLaunchKernelEx(&cfg, decode_gate_up_kernel<KBW>, p);
     if (err != cudaSuccess) return err;
   }
   cfg.gridDim = dim3(std::max(1, std::min(sm_count, p.H / 16)));
   cfg.dynamicSmemBytes = smem_b;
   LaunchScope ls("decode.down", stream);
-  return cudaLaunchKernelEx(&cfg, decode_down_kernel<MAXJ>, p);
+  return cudaLaunchKernelEx(&cfg, decode_down_kernel, p);
 }
 
 struct DecodeWs {
-  size_t h, err, total;
+  size_t h, total;
 };
 
+// Workspace: h [M*k, I] bf16, then 256 bytes kept for the layout (unused).
 DecodeWs decode_ws(int64_t M, int k, int64_t I) {
   DecodeWs w;
   w.h = 0;
-  w.err = align_up(static_cast<size_t>(M * k * I * 2), 256);
-  w.total = w.err + 256;
+  w.total = align_up(static_cast<size_t>(M * k * I * 2), 256) + 256;
   return w;
 }
 
 }  // namespace
 
 bool decode_supported(int64_t M, int64_t E, int k, int64_t H, int64_t I) {
-  if (M < 1 || M > kMaxM || k > 32 || E > 512) return false;
+  if (M < 1 || M > kMaxM || k > 32 || E > 512 || H > 64 * kWarps * kMaxKBW) return false;
+  (void)I;
   DeviceInfo di;
   if (device_info(&di) != cudaSuccess) return false;
-  const Layout a = make_layout(true, static_cast<int>(M), k, static_cast<int>(E), static_cast<int>(H),
-                               static_cast<int>(I), 16);
-  const Layout b = make_layout(false, static_cast<int>(M), k, static_cast<int>(E), static_cast<int>(H),
-                               static_cast<int>(I), 0);
+  const Layout a = make_layout(true, static_cast<int>(M), k, static_cast<int>(E), static_cast<int>(H), 16);
+  const Layout b = make_layout(false, static_cast<int>(M), k, static_cast<int>(E), static_cast<int>(H), 0);
   const size_t lim = di.smem_optin - 1024;  // leave room for the kernels' static shared memory
   return a.total <= lim && b.total <= lim;
 }
@@ -632,14 +604,14 @@ cudaError_t launch_decode_forward(const DecodeArgs& a, cudaStream_t stream) {
   p.lora_scale = r ? w->lora_alpha / static_cast<float>(r) : 0.f;
   p.h = reinterpret_cast<uint16_t*>(static_cast<char*>(a.workspace) + ws.h);
   p.out = a.out;
-  p.err = reinterpret_cast<int*>(static_cast<char*>(a.workspace) + ws.err);
-  const size_t smem_a = make_layout(true, p.M, p.k, p.E, p.H, p.I, r).total;
-  const size_t smem_b = make_layout(false, p.M, p.k, p.E, p.H, p.I, 0).total;
-  if (p.E <= 32) return launch_pair<1>(p, di.sm_count, smem_a, smem_b, stream);
-  if (p.E <= 64) return launch_pair<2>(p, di.sm_count, smem_a, smem_b, stream);
-  if (p.E <= 128) return launch_pair<4>(p, di.sm_count, smem_a, smem_b, stream);
-  if (p.E <= 256) return launch_pair<8>(p, di.sm_count, smem_a, smem_b, stream);
-  return launch_pair<16>(p, di.sm_count, smem_a, smem_b, stream);  // E <= 512 (decode_supported)
+  const size_t smem_a = make_layout(true, p.M, p.k, p.E, p.H, r).total;
+  const size_t smem_b = make_layout(false, p.M, p.k, p.E, p.H, 0).total;
+  switch (kbw_of(p.H)) {
+    case 1: return launch_pair<1>(p, di.sm_count, smem_a, smem_b, stream);
+    case 2: return launch_pair<2>(p, di.sm_count, smem_a, smem_b, stream);
+    case 3: return launch_pair<3>(p, di.sm_count, smem_a, smem_b, stream);
+    default: return launch_pair<4>(p, di.sm_count, smem_a, smem_b, stream);
+  }
 }
 
 }  // namespace e4b

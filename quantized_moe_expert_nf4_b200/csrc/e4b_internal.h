@@ -58,6 +58,9 @@ size_t route_workspace_bytes(int64_t M, int64_t E, int k);
 bool route_uses_small_kernel(int64_t M, int64_t E, int k);
 cudaError_t launch_route(const float* logits, int64_t M, int E, int k, bool renormalize,
                          const RouteOut& o, void* workspace, cudaStream_t stream);
+// out[p, :] = A[row_index[p], :K] for p < S (the routed rows, contiguous).
+cudaError_t launch_gather_rows(const uint16_t* A, int64_t a_rows, int64_t lda, const int32_t* row_index, int64_t S,
+                               int K, uint16_t* out, cudaStream_t stream);
 
 // ---- grouped GEMM --------------------------------------------------------
 struct GemmArgs {
@@ -75,12 +78,17 @@ struct GemmArgs {
   int r;
   float lora_scale;
   float* xa;  // workspace [total_rows, r] (LoRA only)
+  uint16_t* a_gathered;  // workspace [total_rows, K]: routed rows gathered for the tensor-core kernel
   int* err;   // workspace error word of the tensor-core kernel's bounded waits
   int epi;    // e4b_epilogue
   void* out;
   bool out_bf16;
 };
-size_t gemm_workspace_bytes(int64_t total_rows, int r);
+// Workspace: [error word, 256 B][LoRA x.A^T, total_rows * r fp32, 256-B aligned]
+// [gathered rows, total_rows * K bf16].
+size_t gemm_workspace_bytes(int64_t total_rows, int64_t K, int r);
+size_t gemm_workspace_xa_offset();
+size_t gemm_workspace_gather_offset(int64_t total_rows, int r);
 bool tc_supported(const GemmArgs& a);
 cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int* err_word, cudaStream_t stream);
 // Picks the implementation; reports the path name through set_path.

@@ -223,8 +223,11 @@ __global__ void __launch_bounds__(kThreads) grouped_nf4_mma_kernel(GemmArgs a) {
   }
 }
 
-// LoRA first factor: xa[p, :] = A[row(p)] . lora_A[e]^T (fp32), one warp per row.
+// LoRA first factor: xa[p, :] = A[row(p)] . lora_A[e]^T (fp32), one warp per row:
+// lanes stream 8 consecutive k (16-byte loads of the activation row and of each
+// of the r adapter rows), then each of the r sums is reduced across the warp.
 __global__ void __launch_bounds__(256) lora_xa_kernel(GemmArgs a) {
+  constexpr int kMaxR = 16;
   const int lane = threadIdx.x & 31;
   const int64_t p = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   if (p >= a.total_rows) return;
@@ -240,13 +243,31 @@ __global__ void __launch_bounds__(256) lora_xa_kernel(GemmArgs a) {
   src = clampv<int64_t>(src, 0, a.a_rows - 1);
   const uint16_t* x = a.A + src * a.lda;
   const uint16_t* la = a.lora_A + static_cast<int64_t>(e) * a.r * a.K;
-  for (int rr = 0; rr < a.r; ++rr) {
-    float s = 0.f;
-    for (int kk = lane; kk < a.K; kk += 32)
-      s = fmaf(bf16_bits_to_float(x[kk]), bf16_bits_to_float(la[static_cast<int64_t>(rr) * a.K + kk]), s);
+  float acc[kMaxR];
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) a.xa[p * a.r + rr] = s;
+  for (int rr = 0; rr < kMaxR; ++rr) acc[rr] = 0.f;
+  for (int kk = lane * 8; kk < a.K; kk += 256) {
+    const uint4 xv = *reinterpret_cast<const uint4*>(x + kk);
+    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+    for (int rr = 0; rr < kMaxR; ++rr) {
+      if (rr >= a.r) break;
+      const uint4 av = *reinterpret_cast<const uint4*>(la + static_cast<int64_t>(rr) * a.K + kk);
+      const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[rr] = fmaf(__uint_as_float(xw[i] << 16), __uint_as_float(aw[i] << 16), acc[rr]);
+        acc[rr] = fmaf(__uint_as_float(xw[i] & 0xffff0000u), __uint_as_float(aw[i] & 0xffff0000u), acc[rr]);
+      }
+    }
+  }
+#pragma unroll
+  for (int rr = 0; rr < kMaxR; ++rr) {
+    if (rr >= a.r) break;
+    float v = acc[rr];
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) a.xa[p * a.r + rr] = v;
   }
 }
 
@@ -278,9 +299,12 @@ cudaError_t launch_grouped_gemm_mma(const GemmArgs& a, cudaStream_t stream) {
 
 namespace e4b {
 
-// Workspace: [error word, 256 B][LoRA x.A^T, total_rows * r fp32].
-size_t gemm_workspace_bytes(int64_t total_rows, int r) {
-  return 256 + (r > 0 ? static_cast<size_t>(total_rows) * r * sizeof(float) : 0);
+size_t gemm_workspace_xa_offset() { return 256; }
+size_t gemm_workspace_gather_offset(int64_t total_rows, int r) {
+  return 256 + align_up(r > 0 ? static_cast<size_t>(total_rows) * r * sizeof(float) : 0, 256);
+}
+size_t gemm_workspace_bytes(int64_t total_rows, int64_t K, int r) {
+  return gemm_workspace_gather_offset(total_rows, r) + static_cast<size_t>(total_rows) * K * sizeof(uint16_t);
 }
 
 namespace {
@@ -300,12 +324,25 @@ constexpr int64_t kTcMinRows = 512;
 
 cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const char** path) {
   const int ov = gemm_override();
-  const bool tc_ok = tc_supported(a);
+  // The tensor-core kernel reads contiguous operand rows: a row_index call
+  // gathers them into the workspace first.
+  GemmArgs c = a;
+  if (c.row_index && c.a_gathered) {
+    c.A = c.a_gathered;
+    c.a_rows = c.total_rows;
+    c.lda = c.K;
+    c.row_index = nullptr;
+  }
+  const bool tc_ok = tc_supported(c);
   const bool use_tc = ov == 2 || (ov == 0 && tc_ok && a.total_rows >= kTcMinRows);
   if (use_tc) {
     if (!tc_ok) return cudaErrorNotSupported;
+    if (a.row_index) {
+      cudaError_t err = launch_gather_rows(a.A, a.a_rows, a.lda, a.row_index, a.total_rows, a.K, a.a_gathered, stream);
+      if (err != cudaSuccess) return err;
+    }
     *path = a.epi == E4B_EPI_SWIGLU ? "gemm.tc.swiglu" : "gemm.tc";
-    return launch_grouped_gemm_tc(a, a.err, stream);
+    return launch_grouped_gemm_tc(c, c.err, stream);
   }
   if (a.lora_B && a.r > 0) {
     cudaError_t err = launch_lora_xa(a, stream);

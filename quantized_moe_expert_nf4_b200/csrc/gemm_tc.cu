@@ -5,25 +5,34 @@
 // (gemm_4bit_grouped: nibbles decoded inside the mainloop, fp32 accumulation, no
 // bf16 expert tensor in memory), laid out for sm_100a.
 //
-// Tile: 2 x 128 weight rows (the MMA's M; for SwiGLU the gate rows and the
-// matching up rows, so the activation is computed in the epilogue from two
-// accumulators of the same TMEM lanes) x 128 routed rows (the MMA's N) x K.
-// One K step is one absmax block (64).  Warp roles, one persistent CTA per SM:
-//   warp 12      TMA producer: packed nibbles (2-D tiled box 32 B x 128 rows per
-//                half) and the 128 B operand rows -- a 2-D tiled box when the rows
-//                are contiguous, four-row gathers (tile::gather4) through
-//                row_index otherwise -- into a 4-stage ring;
-//   warps 4-11   decoders: one weight row per thread; nibbles -> bf16 through a
-//                per-lane-replicated byte -> bf16x2 codebook table, times the
-//                block's absmax (bf16x2 multiply), stored in the canonical
-//                128-byte-swizzled K-major layout the MMA reads (2-stage ring);
-//   warp 13      TMEM allocator and MMA issuer (one thread): 4 x 2 MMAs
-//                (M=128, N=128, K=16) per K step into a double-buffered pair of
-//                accumulators (4 x 128 of the 512 TMEM columns);
-//   warps 0-3    epilogue: TMEM -> registers (32 lanes x 32 columns at a time),
-//                SwiGLU or plain store, overlapped with the next tile's mainloop.
+// The routed activation rows of a group are contiguous here (the caller gathers
+// them once, in routed order, before the launch): each K step loads them as one
+// 2-D tiled TMA box, which the TMA engine moves far faster than per-row
+// gathers of the same bytes.
+//
+// Tile: HALVES x 128 weight rows (the MMA's M, per half; for SwiGLU the gate
+// rows and the matching up rows, so the activation is computed in the epilogue
+// from two accumulators of the same TMEM lanes) x BN routed rows (the MMA's N,
+// cut to the rows present in a group's last tile) x K, with NACC accumulator
+// sets so that the epilogue of one tile can overlap the mainloop of the next
+// (HALVES x BN x NACC <= the 512 TMEM columns).  One K step is one absmax
+// block (64).  Warp roles, one persistent CTA per SM:
+//   warp 20      TMA producer: packed nibbles (2-D tiled box 32 B x 128 rows per
+//                half) and the 128 B x BN operand rows into a KS-stage ring;
+//   warps 4-19   decoders: one weight row and 1/2 or 1/4 of a k block per thread;
+//                nibbles -> bf16 through a per-lane-replicated byte -> bf16x2
+//                codebook table, times the block's absmax (bf16x2 multiply),
+//                stored in the canonical 128-byte-swizzled K-major layout the
+//                MMA reads (2-stage ring);
+//   warp 21      TMEM allocator and MMA issuer (one thread): 4 x HALVES MMAs
+//                (M=128, N<=BN, K=16) per K step;
+//   warps 0-3    epilogue: TMEM -> registers (32 lanes x 16 columns at a time),
+//                SwiGLU or plain store.
 // Every wait is bounded; TMEM is freed on every exit path.
 #include <cuda.h>
+
+#include <cstdlib>
+#include <cstring>
 
 #include "async.cuh"
 #include "common.cuh"
@@ -34,38 +43,51 @@ namespace e4b {
 namespace {
 
 constexpr int kBM = 128;           // weight rows per MMA (per half)
-constexpr int kBN = 128;           // routed rows per tile
-constexpr int kKS = 4;             // TMA ring stages
-constexpr int kAS = 2;             // decoded-A ring stages
-constexpr int kWarpDec = 4;        // warps 4..11
-constexpr int kNumDecWarps = 8;
-constexpr int kWarpTma = 12;
-constexpr int kWarpMma = 13;
-constexpr int kThreadsTc = 14 * 32;
-
-constexpr uint32_t kPackedHalfBytes = kBM * 32;           // 128 rows x 32 B
-constexpr uint32_t kPackedBytes = 2 * kPackedHalfBytes;   // 8 KB
-constexpr uint32_t kBBytes = kBN * 128;                   // 16 KB
-constexpr uint32_t kTmaStageBytes = kPackedBytes + kBBytes;
-constexpr uint32_t kAHalfBytes = kBM * 128;               // 16 KB
-constexpr uint32_t kAStageBytes = 2 * kAHalfBytes;
+constexpr int kWarpDec = 4;        // warps 4..19
+constexpr int kNumDecWarps = 16;
+constexpr int kDecThreads = kNumDecWarps * 32;
+constexpr int kWarpTma = 20;
+constexpr int kWarpMma = 21;
+constexpr int kThreadsTc = 22 * 32;
+constexpr uint32_t kPackedHalfBytes = kBM * 32;  // 128 rows x 32 B
+constexpr uint32_t kAHalfBytes = kBM * 128;      // 128 rows x 64 bf16
 constexpr uint32_t kLutBytes = 256 * 32 * 4;
+constexpr uint32_t kSmemLimit = 227 * 1024;
+constexpr uint32_t kSmemMisc = 1024 + 512;       // alignment slack, barriers, TMEM slot
 
-constexpr uint32_t kOffTma = 0;
-constexpr uint32_t kOffA = kOffTma + kKS * kTmaStageBytes;
-constexpr uint32_t kOffLut = kOffA + kAS * kAStageBytes;
-constexpr uint32_t kOffBar = kOffLut + kLutBytes;
-constexpr uint32_t kNumBars = 2 * kKS + 2 * kAS + 4;
-constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
-constexpr uint32_t kOffRows = kOffTmemSlot + 16;
-constexpr uint32_t kSmemBytes = kOffRows + kBN * 4 + 1024;  // + slack for 1024-B alignment
+template <int BN_, int HALVES_, int NACC_>
+struct TcShape {
+  static constexpr int BN = BN_, HALVES = HALVES_, NACC = NACC_;
+  static constexpr int kRows = HALVES * kBM;        // weight rows per tile
+  static constexpr int kTpr = kDecThreads / kRows;  // decoder threads per weight row
+  static constexpr int kChunks = 8 / kTpr;          // 16-byte decoded chunks per thread per k block
+  static constexpr uint32_t kPackedBytes = HALVES * kPackedHalfBytes;
+  static constexpr uint32_t kBBytes = BN * 128;
+  static constexpr uint32_t kTmaStageBytes = kPackedBytes + kBBytes;
+  static constexpr int kAS = 2;
+  static constexpr uint32_t kAStageBytes = HALVES * kAHalfBytes;
+  static constexpr int kKSFit =
+      static_cast<int>((kSmemLimit - kSmemMisc - kLutBytes - kAS * kAStageBytes) / kTmaStageBytes);
+  static constexpr int kKS = kKSFit < 6 ? kKSFit : 6;
+  static constexpr uint32_t kCols = HALVES * BN;    // TMEM columns of one accumulator set
+  static constexpr uint32_t kOffTma = 0;
+  static constexpr uint32_t kOffA = kOffTma + kKS * kTmaStageBytes;
+  static constexpr uint32_t kOffLut = kOffA + kAS * kAStageBytes;
+  static constexpr uint32_t kOffBar = kOffLut + kLutBytes;
+  static constexpr uint32_t kNumBars = 2 * kKS + 2 * kAS + 2 * NACC;
+  static constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
+  static constexpr uint32_t kSmemBytes = kOffTmemSlot + 16 + 1024;
+  static_assert(kTpr == 2 || kTpr == 4, "decoder split");
+  static_assert(kKS >= 2, "ring depth");
+  static_assert(kCols * NACC <= 512, "TMEM columns");
+  static_assert(BN % 16 == 0 && BN <= 256, "MMA N");
+  static_assert(kSmemBytes <= kSmemLimit, "shared memory");
+};
 
 struct TcParams {
   const int32_t* offsets;
   int E;
   int64_t total_rows;
-  const int32_t* row_index;  // gather rows of A (nullable: contiguous rows)
-  int64_t a_rows;
   const float* absmax;
   int N, K;
   int swiglu;
@@ -75,24 +97,26 @@ struct TcParams {
   int* err;
 };
 
+// Weight rows of the tile's halves.
+template <int HALVES>
 __device__ __forceinline__ void tile_rows(const TcParams& p, int n_tile, int* r0, int* r1) {
   if (p.swiglu) {
     *r0 = n_tile * kBM;
     *r1 = p.N / 2 + n_tile * kBM;
   } else {
-    *r0 = n_tile * 2 * kBM;
-    *r1 = n_tile * 2 * kBM + kBM;
+    *r0 = n_tile * HALVES * kBM;
+    *r1 = *r0 + kBM;
   }
 }
 
-// Tile t -> (group, routed-row range, n tile); warp-collective.
-__device__ __forceinline__ bool locate(const TcParams& p, int64_t t, int* e, int64_t* rb, int64_t* re, int* n_tile) {
-  const int64_t tok_tile_span = static_cast<int64_t>(kBN);
+// Tile t -> (group, routed-row range, n tile); warp-collective.  Each group owns
+// ceil(rows / BN) * n_tiles tiles, the n tile running fastest.
+template <int BN>
+__device__ __forceinline__ bool locate(const TcParams& p, int64_t t, int* e, int64_t* rb, int64_t* re,
+                                       int* n_tile) {
   int g;
   int64_t b0, b1;
-  // Each group owns ceil(cnt / kBN) * n_tiles tiles: locate by (token tile, n tile).
-  const int64_t q = t / p.n_tiles;
-  if (!find_group_tile(p.offsets, p.E, p.total_rows, static_cast<int>(tok_tile_span), q, &g, &b0, &b1)) return false;
+  if (!find_group_tile(p.offsets, p.E, p.total_rows, BN, t / p.n_tiles, &g, &b0, &b1)) return false;
   *e = g;
   *rb = b0;
   *re = b1;
@@ -100,40 +124,42 @@ __device__ __forceinline__ bool locate(const TcParams& p, int64_t t, int* e, int
   return true;
 }
 
+template <class S>
 __global__ void __launch_bounds__(kThreadsTc, 1)
     grouped_nf4_tc_kernel(const __grid_constant__ CUtensorMap tm_packed, const __grid_constant__ CUtensorMap tm_b,
                           TcParams p) {
+  constexpr int BN = S::BN, HALVES = S::HALVES, NACC = S::NACC, KS = S::kKS, AS = S::kAS;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kOffBar);
   uint64_t* tma_full = bars;
-  uint64_t* tma_empty = bars + kKS;
-  uint64_t* a_full = bars + 2 * kKS;
-  uint64_t* a_empty = a_full + kAS;
-  uint64_t* acc_full = a_empty + kAS;
-  uint64_t* acc_empty = acc_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffTmemSlot);
-  int32_t* rows_s = reinterpret_cast<int32_t*>(smem + kOffRows);
-  uint32_t* lut = reinterpret_cast<uint32_t*>(smem + kOffLut);
+  uint64_t* tma_empty = bars + KS;
+  uint64_t* a_full = bars + 2 * KS;
+  uint64_t* a_empty = a_full + AS;
+  uint64_t* acc_full = a_empty + AS;
+  uint64_t* acc_empty = acc_full + NACC;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kOffTmemSlot);
+  uint32_t* lut = reinterpret_cast<uint32_t*>(smem + S::kOffLut);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int KB = p.K / 64;
 
   if (tid == 0) {
-    for (int s = 0; s < kKS; ++s) {
+    for (int s = 0; s < KS; ++s) {
       mbar_init(&tma_full[s], 1);
       mbar_init(&tma_empty[s], 1);
     }
-    for (int s = 0; s < kAS; ++s) {
+    for (int s = 0; s < AS; ++s) {
       mbar_init(&a_full[s], kNumDecWarps);
       mbar_init(&a_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < NACC; ++s) {
       mbar_init(&acc_full[s], 1);
       mbar_init(&acc_empty[s], 4);
     }
     fence_mbar_init();
   }
+  // byte b = (code of the even element << 4) | code of the odd element, 32 copies
   for (int i = tid; i < 256 * 32; i += blockDim.x) {
     const int b = i >> 5;
     lut[i] = pack_bf16x2(kNf4CodebookDev[b >> 4], kNf4CodebookDev[b & 15]);
@@ -147,8 +173,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  // Total tiles: every CTA walks the same global list with a stride of gridDim.x.
-  // A tile past the last group ends the walk (locate() returns false).
+  // Every role walks the same tile list (stride gridDim.x); a tile past the
+  // last group ends the walk.
   if (warp == kWarpTma) {
     // ------------------------------------------------------------- producer
     uint32_t kbg = 0;
@@ -156,82 +182,64 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     for (int64_t t = blockIdx.x; ok; t += gridDim.x) {
       int e, n_tile;
       int64_t rb, re;
-      if (!locate(p, t, &e, &rb, &re, &n_tile)) break;
+      if (!locate<BN>(p, t, &e, &rb, &re, &n_tile)) break;
       int r0, r1;
-      tile_rows(p, n_tile, &r0, &r1);
+      tile_rows<HALVES>(p, n_tile, &r0, &r1);
       const int32_t y0 = e * p.N + r0, y1 = e * p.N + r1;
-      if (p.row_index) {
-        // Row indices of this tile (rows past the group repeat a valid row).
-        for (int i = lane; i < kBN; i += 32) {
-          int64_t q = rb + i;
-          if (q >= re) q = rb;
-          int64_t src = p.row_index[q];
-          src = src < 0 ? 0 : (src >= p.a_rows ? p.a_rows - 1 : src);
-          rows_s[i] = static_cast<int32_t>(src);
-        }
-      }
-      __syncwarp();
-      int32_t rowv[kBN / 32];
-      if (p.row_index) {
-#pragma unroll
-        for (int i = 0; i < kBN / 32; ++i) rowv[i] = rows_s[lane * (kBN / 32) + i];
-      }
       for (int kb = 0; kb < KB; ++kb, ++kbg) {
-        const int s = kbg % kKS;
-        if (kbg >= kKS && !mbar_wait(&tma_empty[s], ((kbg / kKS) - 1) & 1)) {
+        const int s = kbg % KS;
+        if (kbg >= KS && !mbar_wait(&tma_empty[s], ((kbg / KS) - 1) & 1)) {
           record_error(p.err, kErrWaitEmpty);
           ok = false;
           break;
         }
-        unsigned char* st = smem + kOffTma + s * kTmaStageBytes;
+        unsigned char* st = smem + S::kOffTma + s * S::kTmaStageBytes;
         if (lane == 0) {
-          mbar_arrive_expect_tx(&tma_full[s], kTmaStageBytes);
+          mbar_arrive_expect_tx(&tma_full[s], S::kTmaStageBytes);
           tma_load_2d(st, &tm_packed, kb * 32, y0, &tma_full[s]);
-          tma_load_2d(st + kPackedHalfBytes, &tm_packed, kb * 32, y1, &tma_full[s]);
-          if (!p.row_index) tma_load_2d(st + kPackedBytes, &tm_b, kb * 64, static_cast<int32_t>(rb), &tma_full[s]);
-        }
-        __syncwarp();
-        if (p.row_index) {
-          // 32 gathers of 4 rows; lane l issues the gathers of rows 4l .. 4l+3.
-          tma_gather4(st + kPackedBytes + lane * 4 * 128, &tm_b, kb * 64, rowv[0], rowv[1], rowv[2], rowv[3],
-                      &tma_full[s]);
+          if (HALVES == 2) tma_load_2d(st + kPackedHalfBytes, &tm_packed, kb * 32, y1, &tma_full[s]);
+          tma_load_2d(st + S::kPackedBytes, &tm_b, kb * 64, static_cast<int32_t>(rb), &tma_full[s]);
         }
         __syncwarp();
       }
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------- MMA issuer
-    const uint32_t idesc = idesc_bf16_f32(kBM, kBN);
     uint32_t kbg = 0, j = 0;
     bool ok = true;
     for (int64_t t = blockIdx.x; ok; t += gridDim.x, ++j) {
       int e, n_tile;
       int64_t rb, re;
-      if (!locate(p, t, &e, &rb, &re, &n_tile)) break;
-      const int b = j & 1;
-      if (j >= 2 && !mbar_wait(&acc_empty[b], ((j >> 1) - 1) & 1)) {
+      if (!locate<BN>(p, t, &e, &rb, &re, &n_tile)) break;
+      // N of this tile: the routed rows present, rounded up to the MMA's step of 16.
+      const int nrows = static_cast<int>(re - rb);
+      const int n_mma = min(BN, (nrows + 15) & ~15);
+      const uint32_t idesc = idesc_bf16_f32(kBM, n_mma);
+      const uint32_t slot = j % NACC;
+      if (j >= NACC && !mbar_wait(&acc_empty[slot], ((j / NACC) - 1) & 1)) {
         record_error(p.err, kErrWaitEmpty);
         break;
       }
       tc_fence_after();
-      const uint32_t d0 = tmem_base + (2 * b + 0) * kBN, d1 = tmem_base + (2 * b + 1) * kBN;
+      const uint32_t d = tmem_base + slot * S::kCols;
       for (int kb = 0; kb < KB; ++kb, ++kbg) {
-        const int s = kbg % kKS, a = kbg % kAS;
-        if (!mbar_wait(&a_full[a], (kbg / kAS) & 1) || !mbar_wait(&tma_full[s], (kbg / kKS) & 1)) {
+        const int s = kbg % KS, a = kbg % AS;
+        if (!mbar_wait(&a_full[a], (kbg / AS) & 1) || !mbar_wait(&tma_full[s], (kbg / KS) & 1)) {
           record_error(p.err, kErrWaitFull);
           ok = false;
           break;
         }
         tc_fence_after();
         if (lane == 0) {
-          const uint32_t a_addr = smem_u32(smem + kOffA + a * kAStageBytes);
-          const uint32_t b_addr = smem_u32(smem + kOffTma + s * kTmaStageBytes + kPackedBytes);
+          const uint32_t a_addr = smem_u32(smem + S::kOffA + a * S::kAStageBytes);
+          const uint32_t b_addr = smem_u32(smem + S::kOffTma + s * S::kTmaStageBytes + S::kPackedBytes);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint32_t acc = (kb | kk) ? 1u : 0u;
             const uint64_t bd = smem_desc_sw128(b_addr + kk * 32);
-            umma_bf16(d0, smem_desc_sw128(a_addr + kk * 32), bd, idesc, acc);
-            umma_bf16(d1, smem_desc_sw128(a_addr + kAHalfBytes + kk * 32), bd, idesc, acc);
+#pragma unroll
+            for (int h = 0; h < HALVES; ++h)
+              umma_bf16(d + h * BN, smem_desc_sw128(a_addr + h * kAHalfBytes + kk * 32), bd, idesc, acc);
           }
           umma_commit(&tma_empty[s]);
           umma_commit(&a_empty[a]);
@@ -239,12 +247,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         __syncwarp();
       }
       if (!ok) break;
-      if (lane == 0) umma_commit(&acc_full[b]);
+      if (lane == 0) umma_commit(&acc_full[slot]);
       __syncwarp();
     }
   } else if (warp >= kWarpDec && warp < kWarpDec + kNumDecWarps) {
     // ------------------------------------------------------------- decoders
-    const int r = tid - kWarpDec * 32;  // 0..255: weight row of the tile
+    const int dt = tid - kWarpDec * 32;            // 0..511
+    const int r = dt / S::kTpr, kq = dt % S::kTpr;  // weight row of the tile, part of the k block
     const int half = r >> 7, ri = r & 127;
     const uint32_t* lut_lane = lut + lane;
     uint32_t kbg = 0;
@@ -252,45 +261,67 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     for (int64_t t = blockIdx.x; ok; t += gridDim.x) {
       int e, n_tile;
       int64_t rb, re;
-      if (!locate(p, t, &e, &rb, &re, &n_tile)) break;
+      if (!locate<BN>(p, t, &e, &rb, &re, &n_tile)) break;
       int r0, r1;
-      tile_rows(p, n_tile, &r0, &r1);
+      tile_rows<HALVES>(p, n_tile, &r0, &r1);
       const int n = (half ? r1 : r0) + ri;
       const bool valid = n < p.N;
       const float* am = p.absmax + (static_cast<int64_t>(e) * p.N + (valid ? n : 0)) * KB;
-      float sc_next = valid ? __ldg(am) : 0.0f;
-      for (int kb = 0; kb < KB; ++kb, ++kbg) {
-        const int s = kbg % kKS, a = kbg % kAS;
-        const float sc = sc_next;
-        if (kb + 1 < KB) sc_next = valid ? __ldg(am + kb + 1) : 0.0f;
-        if (!mbar_wait(&tma_full[s], (kbg / kKS) & 1) ||
-            (kbg >= kAS && !mbar_wait(&a_empty[a], ((kbg / kAS) - 1) & 1))) {
-          record_error(p.err, kErrWaitFull);
-          ok = false;
-          break;
-        }
-        const unsigned char* pk = smem + kOffTma + s * kTmaStageBytes + half * kPackedHalfBytes + ri * 32;
-        const uint4 q0 = *reinterpret_cast<const uint4*>(pk);
-        const uint4 q1 = *reinterpret_cast<const uint4*>(pk + 16);
-        const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-        const __nv_bfloat162 s2 = __float2bfloat162_rn(sc);
-        unsigned char* arow = smem + kOffA + a * kAStageBytes + half * kAHalfBytes + (ri >> 3) * 1024 + (ri & 7) * 128;
+      // absmax of the next 4 k blocks in flight (an L2 round trip outlasts one k block)
+      float sc_ring[4];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {  // chunk c = k [8c, 8c+8) = one packed word
-          const uint32_t w = words[c];
-          uint32_t v[4];
+      for (int i = 0; i < 4; ++i) sc_ring[i] = (valid && i < KB) ? __ldg(am + i) : 0.0f;
+      for (int kb0 = 0; kb0 < KB && ok; kb0 += 4) {
 #pragma unroll
-          for (int by = 0; by < 4; ++by) {
-            uint32_t pair = lut_lane[((w >> (8 * by)) & 0xffu) << 5];
-            __nv_bfloat162 h2 = *reinterpret_cast<__nv_bfloat162*>(&pair);
-            h2 = __hmul2(h2, s2);
-            v[by] = *reinterpret_cast<uint32_t*>(&h2);
+        for (int i = 0; i < 4; ++i) {
+          const int kb = kb0 + i;
+          if (kb >= KB) break;
+          const float sc = sc_ring[i];
+          sc_ring[i] = (valid && kb + 4 < KB) ? __ldg(am + kb + 4) : 0.0f;
+          const int s = kbg % KS, a = kbg % AS;
+          if (!mbar_wait(&tma_full[s], (kbg / KS) & 1) ||
+              (kbg >= AS && !mbar_wait(&a_empty[a], ((kbg / AS) - 1) & 1))) {
+            record_error(p.err, kErrWaitFull);
+            ok = false;
+            break;
           }
-          *reinterpret_cast<uint4*>(arow + ((c ^ (ri & 7)) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
+          // packed words of k [64 kq / kTpr, +64 / kTpr): one word = 8 elements = one chunk
+          const unsigned char* src =
+              smem + S::kOffTma + s * S::kTmaStageBytes + half * kPackedHalfBytes + ri * 32 + kq * (32 / S::kTpr);
+          uint32_t words[S::kChunks];
+          if constexpr (S::kChunks == 4) {
+            const uint4 q = *reinterpret_cast<const uint4*>(src);
+            words[0] = q.x;
+            words[1] = q.y;
+            words[2] = q.z;
+            words[3] = q.w;
+          } else {
+            const uint2 q = *reinterpret_cast<const uint2*>(src);
+            words[0] = q.x;
+            words[1] = q.y;
+          }
+          const __nv_bfloat162 s2 = __float2bfloat162_rn(sc);
+          unsigned char* arow =
+              smem + S::kOffA + a * S::kAStageBytes + half * kAHalfBytes + (ri >> 3) * 1024 + (ri & 7) * 128;
+#pragma unroll
+          for (int c = 0; c < S::kChunks; ++c) {
+            const uint32_t w = words[c];
+            uint32_t v[4];
+#pragma unroll
+            for (int by = 0; by < 4; ++by) {
+              uint32_t pair = lut_lane[((w >> (8 * by)) & 0xffu) << 5];
+              __nv_bfloat162 h2 = *reinterpret_cast<__nv_bfloat162*>(&pair);
+              h2 = __hmul2(h2, s2);
+              v[by] = *reinterpret_cast<uint32_t*>(&h2);
+            }
+            const int chunk = kq * S::kChunks + c;
+            *reinterpret_cast<uint4*>(arow + ((chunk ^ (ri & 7)) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&a_full[a]);
+          ++kbg;
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&a_full[a]);
       }
     }
   } else if (warp < 4) {
@@ -301,30 +332,30 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     for (int64_t t = blockIdx.x;; t += gridDim.x, ++j) {
       int e, n_tile;
       int64_t rb, re;
-      if (!locate(p, t, &e, &rb, &re, &n_tile)) break;
-      const int b = j & 1;
-      if (!mbar_wait(&acc_full[b], (j >> 1) & 1)) {
+      if (!locate<BN>(p, t, &e, &rb, &re, &n_tile)) break;
+      const uint32_t slot = j % NACC;
+      if (!mbar_wait(&acc_full[slot], (j / NACC) & 1)) {
         record_error(p.err, kErrWaitFull);
         break;
       }
       tc_fence_after();
       int r0, r1;
-      tile_rows(p, n_tile, &r0, &r1);
+      tile_rows<HALVES>(p, n_tile, &r0, &r1);
       const int nrows = static_cast<int>(re - rb);
-      const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-      const uint32_t c0 = tmem_base + lane_off + (2 * b) * kBN, c1 = tmem_base + lane_off + (2 * b + 1) * kBN;
+      const uint32_t c0 = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + slot * S::kCols;
+      const int ncols = min(BN, (nrows + 15) & ~15);
       if (p.swiglu) {
         const int n = r0 + ri;  // output column
         const int outN = p.N / 2;
         const bool valid = n < outN;
-        for (int cc = 0; cc < kBN; cc += 32) {
-          float g[32], u[32];
-          tmem_ld_32x32b_x32(c0 + cc, g);
-          tmem_ld_32x32b_x32(c1 + cc, u);
+        for (int cc = 0; cc < ncols; cc += 16) {
+          float g[16], u[16];
+          tmem_ld_32x32b_x16(c0 + cc, g);
+          tmem_ld_32x32b_x16(c0 + BN + cc, u);
           tmem_ld_wait();
           if (valid) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
+            for (int i = 0; i < 16; ++i) {
               const int tok = cc + i;
               if (tok < nrows) {
                 const float hv = silu_f32(g[i]) * u[i];
@@ -338,17 +369,18 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           }
         }
       } else {
-        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int h = 0; h < HALVES; ++h) {
           const int n = (h ? r1 : r0) + ri;
           const bool valid = n < p.N;
-          const uint32_t cb = h ? c1 : c0;
-          for (int cc = 0; cc < kBN; cc += 32) {
-            float v[32];
-            tmem_ld_32x32b_x32(cb + cc, v);
+          const uint32_t cb = c0 + h * BN;
+          for (int cc = 0; cc < ncols; cc += 16) {
+            float v[16];
+            tmem_ld_32x32b_x16(cb + cc, v);
             tmem_ld_wait();
             if (valid) {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) {
+              for (int i = 0; i < 16; ++i) {
                 const int tok = cc + i;
                 if (tok < nrows) {
                   const int64_t o = (rb + tok) * p.N + n;
@@ -364,7 +396,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[b]);
+      if (lane == 0) mbar_arrive(&acc_empty[slot]);
     }
   }
   // All roles are done (every MMA was waited on through acc_full): free TMEM.
@@ -406,21 +438,15 @@ bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint6
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
-
-bool tc_supported(const GemmArgs& a) {
-  // No LoRA epilogue in the tensor-core kernel yet; K % 64 and N % 64 hold by contract.
-  return a.lora_B == nullptr && a.lda % 8 == 0 && encode_fn() != nullptr;
-}
-
-cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int* err_word, cudaStream_t stream) {
+template <class S>
+cudaError_t launch_shape(const GemmArgs& a, int* err_word, cudaStream_t stream) {
   DeviceInfo di;
   cudaError_t err = device_info(&di);
   if (err != cudaSuccess) return err;
-  static bool configured = false;
+  static bool configured = false;  // one flag per shape: each instantiation has its own kernel
   if (!configured) {
-    err = cudaFuncSetAttribute(grouped_nf4_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kSmemBytes));
+    err = cudaFuncSetAttribute(grouped_nf4_tc_kernel<S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(S::kSmemBytes));
     if (err != cudaSuccess) return err;
     configured = true;
   }
@@ -429,30 +455,66 @@ cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int* err_word, cudaStream_
   if (!make_map_2d(&tm_packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.packed, a.K / 2, total_w_rows, a.K / 2, 32, kBM,
                    CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
-  const uint32_t box_rows = a.row_index ? 1u : static_cast<uint32_t>(kBN);
-  if (!make_map_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.A, a.K, a.a_rows, a.lda * 2, 64, box_rows,
+  if (!make_map_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.A, a.K, a.a_rows, a.lda * 2, 64, S::BN,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   TcParams p{};
   p.offsets = a.offsets;
   p.E = a.E;
   p.total_rows = a.total_rows;
-  p.row_index = a.row_index;
-  p.a_rows = a.a_rows;
   p.absmax = a.absmax;
   p.N = a.N;
   p.K = a.K;
   p.swiglu = a.epi == E4B_EPI_SWIGLU;
   p.out = a.out;
   p.out_bf16 = a.out_bf16;
-  p.n_tiles = p.swiglu ? (a.N / 2 + kBM - 1) / kBM : (a.N + 2 * kBM - 1) / (2 * kBM);
+  const int wrows = p.swiglu ? kBM : S::HALVES * kBM;  // output columns (weight rows) per tile
+  p.n_tiles = ((p.swiglu ? a.N / 2 : a.N) + wrows - 1) / wrows;
   p.err = err_word;
   // Upper bound of the tile count: (ceil(rows / BN) + groups) * n_tiles.
-  const int64_t tiles = ((a.total_rows + kBN - 1) / kBN + (a.E < a.total_rows ? a.E : a.total_rows)) * p.n_tiles;
+  const int64_t tiles =
+      ((a.total_rows + S::BN - 1) / S::BN + (a.E < a.total_rows ? a.E : a.total_rows)) * p.n_tiles;
   const int grid = static_cast<int>(tiles < di.sm_count ? tiles : di.sm_count);
   LaunchScope ls(p.swiglu ? "gemm.tc.swiglu" : "gemm.tc", stream);
-  grouped_nf4_tc_kernel<<<grid, kThreadsTc, kSmemBytes, stream>>>(tm_packed, tm_b, p);
+  grouped_nf4_tc_kernel<S><<<grid, kThreadsTc, S::kSmemBytes, stream>>>(tm_packed, tm_b, p);
   return cudaGetLastError();
+}
+
+using ShapeWide = TcShape<256, 2, 1>;    // 2 x 128 weight rows x 256 routed rows, one accumulator set
+using ShapeDouble = TcShape<128, 2, 2>;  // 2 x 128 x 128, two accumulator sets
+using ShapeNarrow = TcShape<256, 1, 2>;  // 128 x 256, two accumulator sets (no SwiGLU)
+
+int shape_override() {
+  const char* v = getenv("E4B_TC_SHAPE");
+  if (!v) return 0;
+  if (!strcmp(v, "wide")) return 1;
+  if (!strcmp(v, "double")) return 2;
+  if (!strcmp(v, "narrow")) return 3;
+  return 0;
+}
+
+}  // namespace
+
+bool tc_supported(const GemmArgs& a) {
+  // No LoRA epilogue in the tensor-core kernel yet; the operand rows must be
+  // contiguous (row_index already applied); K % 64 and N % 64 hold by contract.
+  return a.lora_B == nullptr && a.row_index == nullptr && a.lda % 8 == 0 && encode_fn() != nullptr;
+}
+
+cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int* err_word, cudaStream_t stream) {
+  const bool swiglu = a.epi == E4B_EPI_SWIGLU;
+  int s = shape_override();
+  if (s == 3 && swiglu) s = 0;
+  if (s == 0) {
+    // Measured on B200: the plain (down-projection) GEMM runs best 128 x 256
+    // with two accumulator sets.  SwiGLU tiles take 256 routed rows when groups
+    // are large (few partial tiles), else 128 with the epilogue overlapped.
+    const int64_t rows_per_group = a.total_rows / (a.E > 0 ? a.E : 1);
+    s = !swiglu ? 3 : (rows_per_group >= 512 ? 1 : 2);
+  }
+  if (s == 1) return launch_shape<ShapeWide>(a, err_word, stream);
+  if (s == 2) return launch_shape<ShapeDouble>(a, err_word, stream);
+  return launch_shape<ShapeNarrow>(a, err_word, stream);
 }
 
 }  // namespace e4b

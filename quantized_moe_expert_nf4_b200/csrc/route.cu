@@ -22,7 +22,7 @@ namespace e4b {
 namespace {
 
 constexpr int kSmallMaxSlots = 4096;
-constexpr int kTileTokens = 64;  // tokens per tile of the large path
+constexpr int kTileTokens = 16;  // tokens per tile of the large path
 
 // Ranks slots [0, n) of `ids_s` within their expert in slot order, by one warp.
 // counts[e] must be zero on entry; on exit it holds the per-expert totals.
@@ -197,7 +197,39 @@ cudaError_t launch_route_t(const float* logits, int64_t M, int E, int k, bool re
   return cudaGetLastError();
 }
 
+// Token gather: out[p, :] = A[row_index[p], :K], one warp per routed row,
+// 16-byte vectors (K % 8 == 0, lda % 8 == 0, 16-byte aligned bases).  Indices
+// out of range are clamped.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ A, int64_t a_rows,
+                                                          int64_t lda, const int32_t* __restrict__ row_index,
+                                                          int64_t S, int K, uint16_t* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int vecs = K / 8;
+  for (int64_t p = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; p < S; p += nwarps) {
+    const int64_t src = clampv<int64_t>(row_index[p], 0, a_rows - 1);
+    const uint4* s = reinterpret_cast<const uint4*>(A + src * lda);
+    uint4* d = reinterpret_cast<uint4*>(out + p * K);
+#pragma unroll 4
+    for (int i = lane; i < vecs; i += 32) d[i] = __ldg(s + i);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_gather_rows(const uint16_t* A, int64_t a_rows, int64_t lda, const int32_t* row_index, int64_t S,
+                               int K, uint16_t* out, cudaStream_t stream) {
+  if (S == 0) return cudaSuccess;
+  DeviceInfo di;
+  cudaError_t err = device_info(&di);
+  if (err != cudaSuccess) return err;
+  const int64_t want = (S + 7) / 8;
+  const int64_t cap = static_cast<int64_t>(di.sm_count) * 16;
+  LaunchScope ls("gather", stream);
+  gather_rows_kernel<<<static_cast<int>(want < cap ? want : cap), 256, 0, stream>>>(A, a_rows, lda, row_index, S, K,
+                                                                                   out);
+  return cudaGetLastError();
+}
 
 bool route_uses_small_kernel(int64_t M, int64_t E, int k) { return M * k <= kSmallMaxSlots; }
 

@@ -15,67 +15,68 @@ __device__ __forceinline__ uint32_t ordered_bits(float v) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+__device__ __forceinline__ float from_ordered_bits(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
 // One warp selects the top k of row `logits[0..E)`; lane j < k receives the
-// j-th expert id and its logit.  MAXJ = ceil(E / 32) values held per lane.
+// j-th expert id and its logit.  Each lane holds MAXJ = ceil(E / 32) logits as
+// order-preserving 32-bit keys.  Per selection: the warp maximum of the keys
+// (__reduce_max_sync), then the lowest expert index holding that key
+// (__reduce_min_sync) -- the (value descending, index ascending) order exactly.
 template <int MAXJ>
 __device__ __forceinline__ void warp_topk(const float* __restrict__ row, int E, int k, int* my_id,
                                           float* my_logit, float* full_max, float* full_sum,
                                           bool need_full) {
   const int lane = threadIdx.x & 31;
-  float v[MAXJ];
-  uint64_t key[MAXJ];
+  uint32_t key[MAXJ];
+  uint32_t live = 0;  // bit q: entry lane + 32q is a valid, not yet selected expert
 #pragma unroll
-  for (int j = 0; j < MAXJ; ++j) {
-    const int e = lane + 32 * j;
-    v[j] = (e < E) ? row[e] : 0.0f;
-    key[j] = (e < E) ? ((static_cast<uint64_t>(ordered_bits(v[j])) << 32) | static_cast<uint32_t>(~e)) : 0ull;
+  for (int q = 0; q < MAXJ; ++q) {
+    const int e = lane + 32 * q;
+    key[q] = (e < E) ? ordered_bits(row[e]) : 0u;
+    if (e < E) live |= 1u << q;
   }
   int sel_id = 0;
   float sel_v = 0.0f;
   for (int j = 0; j < k; ++j) {
-    uint64_t best = 0;
-    float bv = 0.0f;
-#pragma unroll
-    for (int q = 0; q < MAXJ; ++q) {
-      if (key[q] > best) {
-        best = key[q];
-        bv = v[q];
-      }
-    }
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-      const uint64_t ob = __shfl_xor_sync(0xffffffffu, best, o);
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      if (ob > best) {
-        best = ob;
-        bv = ov;
-      }
-    }
-    const int id = static_cast<int>(~static_cast<uint32_t>(best & 0xffffffffu));
+    uint32_t m = 0;
 #pragma unroll
     for (int q = 0; q < MAXJ; ++q)
-      if (key[q] == best) key[q] = 0;  // taken
+      if (((live >> q) & 1u) && key[q] > m) m = key[q];
+    // A live entry can have key 0 only for a NaN pattern; it still takes part
+    // through the index step below.
+    const uint32_t wm = __reduce_max_sync(0xffffffffu, m);
+    uint32_t idx = 0xffffffffu;
+#pragma unroll
+    for (int q = 0; q < MAXJ; ++q)
+      if (((live >> q) & 1u) && key[q] == wm) {
+        idx = static_cast<uint32_t>(lane + 32 * q);
+        break;
+      }
+    const uint32_t wi = __reduce_min_sync(0xffffffffu, idx);
+    if (static_cast<int>(wi & 31u) == lane) live &= ~(1u << (wi >> 5));
     if (lane == j) {
-      sel_id = id;
-      sel_v = bv;
+      sel_id = static_cast<int>(wi);
+      sel_v = from_ordered_bits(wm);
     }
   }
   *my_id = sel_id;
   *my_logit = sel_v;
   if (need_full) {
-    float m = -INFINITY;
+    float mx = -INFINITY;
 #pragma unroll
     for (int q = 0; q < MAXJ; ++q)
-      if (lane + 32 * q < E) m = fmaxf(m, v[q]);
+      if (lane + 32 * q < E) mx = fmaxf(mx, from_ordered_bits(key[q]));
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     float s = 0.0f;
 #pragma unroll
     for (int q = 0; q < MAXJ; ++q)
-      if (lane + 32 * q < E) s += expf(v[q] - m);
+      if (lane + 32 * q < E) s += expf(from_ordered_bits(key[q]) - mx);
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    *full_max = m;
+    *full_max = mx;
     *full_sum = s;
   }
 }

@@ -137,3 +137,57 @@ def test_grouped_gemm_positive_control_flipped_nibble():
     got, _ = _run_gpu(c, e4b.E4B_EPI_NONE, torch.float32)
     rows = slice(8, 16)
     assert np.max(np.abs(got[rows, 0] - ref[rows, 0])) > 1e-4
+
+
+# The tensor-core kernel in each of its tile shapes (forced through the
+# E4B_GEMM / E4B_TC_SHAPE switches, which apply to every call of the process):
+# wide = 2 x 128 weight rows x 256 routed rows, double = 2 x 128 x 128 with two
+# accumulator sets, narrow = 128 x 256 with two accumulator sets (plain
+# epilogue only; a SwiGLU call takes the wide shape).
+TC_SHAPES = ["wide", "double", "narrow"]
+TC_CASES = CASES + [
+    # several 256-row token tiles per group and a one-row group
+    (3, 256, 512, [700, 1, 300], 500),
+]
+
+
+@pytest.mark.parametrize("shape", TC_SHAPES)
+@pytest.mark.parametrize("ci", range(len(TC_CASES)))
+@pytest.mark.parametrize("epi", [e4b.E4B_EPI_NONE, e4b.E4B_EPI_SWIGLU])
+def test_grouped_gemm_tensor_core_shapes(monkeypatch, shape, ci, epi):
+    require_gpu()
+    monkeypatch.setenv("E4B_GEMM", "tc")
+    monkeypatch.setenv("E4B_TC_SHAPE", shape)
+    E, N, K, counts, a_rows = TC_CASES[ci]
+    c = _case(E, N, K, counts, a_rows, seed=100 + ci)
+    for use_ridx in (True, False):
+        if not use_ridx:
+            c["Abits"] = np.resize(c["Abits"], (max(1, c["rows"]), K))  # one A row per routed row
+        got, path = _run_gpu(c, epi, torch.float32, use_ridx=use_ridx)
+        assert path.startswith("gemm.tc"), path
+        ref = _oracle(c, epi, use_ridx=use_ridx)
+        fro, mx = rel_errors(got, ref)
+        tol = gemm_tolerance(path, epi, torch.float32)
+        print(f"[parity] tc {shape} case {ci} epi {epi} ridx {use_ridx}: rel_fro={fro:.2e} max={mx:.2e}")
+        assert fro <= tol and mx <= 2 * tol
+
+
+@pytest.mark.parametrize("shape", TC_SHAPES)
+def test_grouped_gemm_tensor_core_bf16_and_exact_sums(monkeypatch, shape):
+    require_gpu()
+    monkeypatch.setenv("E4B_GEMM", "tc")
+    monkeypatch.setenv("E4B_TC_SHAPE", shape)
+    c = _case(4, 640, 320, [300, 0, 129, 77], 256, seed=7)
+    for epi in (e4b.E4B_EPI_NONE, e4b.E4B_EPI_SWIGLU):
+        got, path = _run_gpu(c, epi, torch.bfloat16)
+        assert path.startswith("gemm.tc"), path
+        fro, mx = rel_errors(got, _oracle(c, epi))
+        assert fro <= 1e-2 and mx <= 2e-2
+    # all codes 15, absmax 1: every output is the row sum of A, exact for small integers
+    c["packed"][:] = 0xFF
+    c["absmax"][:] = 1.0
+    c["Abits"] = workloads.to_bf16_bits(np.random.default_rng(8).integers(-3, 4, size=(256, 320)).astype(np.float32))
+    got, _ = _run_gpu(c, e4b.E4B_EPI_NONE, torch.float32)
+    A = workloads.bf16_bits_to_f32(c["Abits"]).astype(np.float64)
+    want = A[c["ridx"]].sum(axis=1)[:, None] * np.ones((1, 640))
+    assert np.array_equal(got, want)
