@@ -20,14 +20,17 @@
 //   warp 20      TMA producer: packed nibbles (2-D tiled box 32 B x 128 rows per
 //                half) and the 128 B x BN operand rows into a KS-stage ring;
 //   warps 4-19   decoders: one weight row and 1/2 or 1/4 of a k block per thread;
-//                nibbles -> bf16 through a per-lane-replicated byte -> bf16x2
-//                codebook table, times the block's absmax (bf16x2 multiply),
-//                stored in the canonical 128-byte-swizzled K-major layout the
-//                MMA reads (2-stage ring);
+//                nibbles -> bf16 in registers (byte permutes over the codebook's
+//                low and high bytes, no table in shared memory), times the
+//                block's absmax (bf16x2 multiply), stored in the canonical
+//                128-byte-swizzled K-major layout the MMA reads (2-stage ring);
 //   warp 21      TMEM allocator and MMA issuer (one thread): 4 x HALVES MMAs
 //                (M=128, N<=BN, K=16) per K step;
 //   warps 0-3    epilogue: TMEM -> registers (32 lanes x 16 columns at a time),
-//                SwiGLU or plain store.
+//                SwiGLU or plain, staged 32 routed rows at a time in shared
+//                memory (double-buffered) and written by TMA tensor stores; a
+//                group's ragged last rows are copied out with plain stores so
+//                that no store reaches the next group's rows.
 // Every wait is bounded; TMEM is freed on every exit path.
 #include <cuda.h>
 
@@ -51,7 +54,9 @@ constexpr int kWarpMma = 21;
 constexpr int kThreadsTc = 22 * 32;
 constexpr uint32_t kPackedHalfBytes = kBM * 32;  // 128 rows x 32 B
 constexpr uint32_t kAHalfBytes = kBM * 128;      // 128 rows x 64 bf16
-constexpr uint32_t kLutBytes = 256 * 32 * 4;
+constexpr int kChunk = 32;                         // routed rows per staged output chunk
+constexpr uint32_t kOutChunkBytes = kChunk * kBM * 4;  // 32 rows x 128 columns x fp32
+constexpr uint32_t kOutBytes = 2 * kOutChunkBytes;     // double-buffered
 constexpr uint32_t kSmemLimit = 227 * 1024;
 constexpr uint32_t kSmemMisc = 1024 + 512;       // alignment slack, barriers, TMEM slot
 
@@ -67,14 +72,14 @@ struct TcShape {
   static constexpr int kAS = 2;
   static constexpr uint32_t kAStageBytes = HALVES * kAHalfBytes;
   static constexpr int kKSFit =
-      static_cast<int>((kSmemLimit - kSmemMisc - kLutBytes - kAS * kAStageBytes) / kTmaStageBytes);
+      static_cast<int>((kSmemLimit - kSmemMisc - kOutBytes - kAS * kAStageBytes) / kTmaStageBytes);
   static constexpr int kKS = kKSFit < 6 ? kKSFit : 6;
   static constexpr uint32_t kCols = HALVES * BN;    // TMEM columns of one accumulator set
   static constexpr uint32_t kOffTma = 0;
   static constexpr uint32_t kOffA = kOffTma + kKS * kTmaStageBytes;
-  static constexpr uint32_t kOffLut = kOffA + kAS * kAStageBytes;
-  static constexpr uint32_t kOffBar = kOffLut + kLutBytes;
-  static constexpr uint32_t kNumBars = 2 * kKS + 2 * kAS + 2 * NACC;
+  static constexpr uint32_t kOffOut = kOffA + kAS * kAStageBytes;
+  static constexpr uint32_t kOffBar = kOffOut + kOutBytes;
+  static constexpr uint32_t kNumBars = 2 * kKS + 2 * kAS + 2 * NACC + 1;
   static constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
   static constexpr uint32_t kSmemBytes = kOffTmemSlot + 16 + 1024;
   static_assert(kTpr == 2 || kTpr == 4, "decoder split");
@@ -93,9 +98,42 @@ struct TcParams {
   int swiglu;
   void* out;
   int out_bf16;
+  int out_cols;  // columns of out: N, or N / 2 for SwiGLU
   int n_tiles;
   int* err;
 };
+
+// The codebook's bf16 patterns split into low and high bytes, four entries per
+// word: lo[j / 4] byte (j % 4) = low byte of bf16(codebook[j]).
+struct CodebookBytes {
+  uint32_t lo[4], hi[4];
+};
+
+__device__ __forceinline__ CodebookBytes codebook_bytes() {
+  CodebookBytes t{};
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const uint32_t b = float_to_bf16_bits(kNf4CodebookDev[j]);
+    t.lo[j >> 2] |= (b & 0xffu) << (8 * (j & 3));
+    t.hi[j >> 2] |= (b >> 8) << (8 * (j & 3));
+  }
+  return t;
+}
+
+// Four nibbles (bits 0-15 of g: the low then the high nibble of two packed
+// bytes, i.e. elements 2i+1, 2i, 2i+3, 2i+2) -> two bf16x2 words in element
+// order.  A byte permute looks up entries 0-7 and 8-15 for all four nibbles at
+// once (its selector takes the nibbles' low three bits); a second permute
+// keeps, per nibble, the half its top bit names; a third interleaves the low
+// and high bytes.
+__device__ __forceinline__ void decode4(uint32_t g, const CodebookBytes& t, uint32_t* w0, uint32_t* w1) {
+  const uint32_t s = g & 0x7777u;
+  const uint32_t pick = ((g >> 1) & 0x4444u) | 0x3210u;  // field i: i, or i + 4 when nibble i >= 8
+  const uint32_t lo = __byte_perm(__byte_perm(t.lo[0], t.lo[1], s), __byte_perm(t.lo[2], t.lo[3], s), pick);
+  const uint32_t hi = __byte_perm(__byte_perm(t.hi[0], t.hi[1], s), __byte_perm(t.hi[2], t.hi[3], s), pick);
+  *w0 = __byte_perm(lo, hi, 0x4051u);  // (element 2i, element 2i+1)
+  *w1 = __byte_perm(lo, hi, 0x6273u);  // (element 2i+2, element 2i+3)
+}
 
 // Weight rows of the tile's halves.
 template <int HALVES>
@@ -127,7 +165,7 @@ __device__ __forceinline__ bool locate(const TcParams& p, int64_t t, int* e, int
 template <class S>
 __global__ void __launch_bounds__(kThreadsTc, 1)
     grouped_nf4_tc_kernel(const __grid_constant__ CUtensorMap tm_packed, const __grid_constant__ CUtensorMap tm_b,
-                          TcParams p) {
+                          const __grid_constant__ CUtensorMap tm_out, TcParams p) {
   constexpr int BN = S::BN, HALVES = S::HALVES, NACC = S::NACC, KS = S::kKS, AS = S::kAS;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -138,8 +176,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   uint64_t* a_empty = a_full + AS;
   uint64_t* acc_full = a_empty + AS;
   uint64_t* acc_empty = acc_full + NACC;
+  uint64_t* epi_bar = acc_empty + NACC;  // barrier of the four epilogue warps (bounded waits)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kOffTmemSlot);
-  uint32_t* lut = reinterpret_cast<uint32_t*>(smem + S::kOffLut);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int KB = p.K / 64;
@@ -157,12 +195,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       mbar_init(&acc_full[s], 1);
       mbar_init(&acc_empty[s], 4);
     }
+    mbar_init(epi_bar, 4);
     fence_mbar_init();
-  }
-  // byte b = (code of the even element << 4) | code of the odd element, 32 copies
-  for (int i = tid; i < 256 * 32; i += blockDim.x) {
-    const int b = i >> 5;
-    lut[i] = pack_bf16x2(kNf4CodebookDev[b >> 4], kNf4CodebookDev[b & 15]);
   }
   if (warp == kWarpMma) {
     tmem_alloc(tmem_slot, 512);
@@ -255,7 +289,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     const int dt = tid - kWarpDec * 32;            // 0..511
     const int r = dt / S::kTpr, kq = dt % S::kTpr;  // weight row of the tile, part of the k block
     const int half = r >> 7, ri = r & 127;
-    const uint32_t* lut_lane = lut + lane;
+    const CodebookBytes cbt = codebook_bytes();
     uint32_t kbg = 0;
     bool ok = true;
     for (int64_t t = blockIdx.x; ok; t += gridDim.x) {
@@ -307,10 +341,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           for (int c = 0; c < S::kChunks; ++c) {
             const uint32_t w = words[c];
             uint32_t v[4];
+            decode4(w, cbt, &v[0], &v[1]);
+            decode4(w >> 16, cbt, &v[2], &v[3]);
 #pragma unroll
             for (int by = 0; by < 4; ++by) {
-              uint32_t pair = lut_lane[((w >> (8 * by)) & 0xffu) << 5];
-              __nv_bfloat162 h2 = *reinterpret_cast<__nv_bfloat162*>(&pair);
+              __nv_bfloat162 h2 = *reinterpret_cast<__nv_bfloat162*>(&v[by]);
               h2 = __hmul2(h2, s2);
               v[by] = *reinterpret_cast<uint32_t*>(&h2);
             }
@@ -326,10 +361,23 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------- epilogue
-    const int q = warp;  // TMEM lane quadrant
+    const int q = warp;  // TMEM lane quadrant = output columns 32q .. 32q + 31 of a part
     const int ri = q * 32 + lane;
-    uint32_t j = 0;
-    for (int64_t t = blockIdx.x;; t += gridDim.x, ++j) {
+    const int esize = p.out_bf16 ? 2 : 4;
+    const uint32_t row_bytes = kBM * esize;
+    unsigned char* stage0 = smem + S::kOffOut;
+    uint32_t j = 0, chunk_no = 0, epi_phase = 0;
+    bool ok = true;
+    // All four warps meet here; false (error recorded) if one never arrives.
+    auto epi_sync = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(epi_bar);
+      const bool w = mbar_wait(epi_bar, epi_phase & 1);
+      ++epi_phase;
+      if (!w) record_error(p.err, kErrWaitFull);
+      return w;
+    };
+    for (int64_t t = blockIdx.x; ok; t += gridDim.x, ++j) {
       int e, n_tile;
       int64_t rb, re;
       if (!locate<BN>(p, t, &e, &rb, &re, &n_tile)) break;
@@ -343,61 +391,69 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       tile_rows<HALVES>(p, n_tile, &r0, &r1);
       const int nrows = static_cast<int>(re - rb);
       const uint32_t c0 = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + slot * S::kCols;
-      const int ncols = min(BN, (nrows + 15) & ~15);
-      if (p.swiglu) {
-        const int n = r0 + ri;  // output column
-        const int outN = p.N / 2;
-        const bool valid = n < outN;
-        for (int cc = 0; cc < ncols; cc += 16) {
-          float g[16], u[16];
-          tmem_ld_32x32b_x16(c0 + cc, g);
-          tmem_ld_32x32b_x16(c0 + BN + cc, u);
-          tmem_ld_wait();
-          if (valid) {
+      const int parts = p.swiglu ? 1 : HALVES;
+      for (int part = 0; part < parts && ok; ++part) {
+        const int col0 = (part ? r1 : r0);  // first output column of this part
+        if (col0 >= p.out_cols) continue;   // a half past the last weight row
+        for (int cr = 0; cr < nrows; cr += kChunk, ++chunk_no) {
+          unsigned char* stage = stage0 + (chunk_no & 1) * kOutChunkBytes;
+          // The store that last read this buffer (two chunks ago) must be done reading.
+          if (tid == 0) bulk_wait_group_read<1>();
+          if (!(ok = epi_sync())) break;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int tok = cc + i;
-              if (tok < nrows) {
-                const float hv = silu_f32(g[i]) * u[i];
-                const int64_t o = (rb + tok) * outN + n;
-                if (p.out_bf16)
-                  static_cast<uint16_t*>(p.out)[o] = float_to_bf16_bits(hv);
-                else
-                  static_cast<float*>(p.out)[o] = hv;
-              }
-            }
-          }
-        }
-      } else {
-#pragma unroll
-        for (int h = 0; h < HALVES; ++h) {
-          const int n = (h ? r1 : r0) + ri;
-          const bool valid = n < p.N;
-          const uint32_t cb = c0 + h * BN;
-          for (int cc = 0; cc < ncols; cc += 16) {
+          for (int hs = 0; hs < kChunk; hs += 16) {
             float v[16];
-            tmem_ld_32x32b_x16(cb + cc, v);
-            tmem_ld_wait();
-            if (valid) {
+            if (p.swiglu) {
+              float u[16];
+              tmem_ld_32x32b_x16(c0 + cr + hs, v);
+              tmem_ld_32x32b_x16(c0 + BN + cr + hs, u);
+              tmem_ld_wait();
 #pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const int tok = cc + i;
-                if (tok < nrows) {
-                  const int64_t o = (rb + tok) * p.N + n;
-                  if (p.out_bf16)
-                    static_cast<uint16_t*>(p.out)[o] = float_to_bf16_bits(v[i]);
-                  else
-                    static_cast<float*>(p.out)[o] = v[i];
-                }
+              for (int i = 0; i < 16; ++i) v[i] = __fdividef(v[i], 1.0f + __expf(-v[i])) * u[i];
+            } else {
+              tmem_ld_32x32b_x16(c0 + part * BN + cr + hs, v);
+              tmem_ld_wait();
+            }
+            if (p.out_bf16) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                *reinterpret_cast<uint16_t*>(stage + (hs + i) * row_bytes + ri * 2) = float_to_bf16_bits(v[i]);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) *reinterpret_cast<float*>(stage + (hs + i) * row_bytes + ri * 4) = v[i];
+            }
+          }
+          fence_proxy_async_smem();
+          if (!(ok = epi_sync())) break;
+          const int rows_here = min(kChunk, nrows - cr);
+          if (rows_here == kChunk) {
+            if (tid == 0) tma_store_2d(&tm_out, stage, col0, static_cast<int32_t>(rb + cr));
+          } else {
+            // Ragged end of the group: plain 16-byte (fp32) or 8-byte (bf16) stores, row by row.
+            const int ncol = min(kBM, p.out_cols - col0);
+            for (int rr = q; rr < rows_here; rr += 4) {
+              const int c = lane * 4;  // four columns per lane
+              if (c < ncol) {
+                const unsigned char* src = stage + rr * row_bytes + c * esize;
+                unsigned char* dst = static_cast<unsigned char*>(p.out) +
+                                     ((rb + cr + rr) * p.out_cols + col0 + c) * static_cast<int64_t>(esize);
+                if (p.out_bf16)
+                  *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(src);
+                else
+                  *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
               }
             }
           }
+          // One bulk group per chunk (empty for a ragged chunk) keeps the
+          // read-wait above tied to the buffer two chunks back.
+          if (tid == 0) bulk_commit_group();
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[slot]);
     }
+    if (tid == 0) bulk_wait_group_all();
   }
   // All roles are done (every MMA was waited on through acc_full): free TMEM.
   tc_fence_before();
@@ -458,6 +514,13 @@ cudaError_t launch_shape(const GemmArgs& a, int* err_word, cudaStream_t stream) 
   if (!make_map_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.A, a.K, a.a_rows, a.lda * 2, 64, S::BN,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
+  const int out_cols = a.epi == E4B_EPI_SWIGLU ? a.N / 2 : a.N;
+  const int esize = a.out_bf16 ? 2 : 4;
+  CUtensorMap tm_out;
+  if (!make_map_2d(&tm_out, a.out_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.out,
+                   out_cols, a.total_rows, static_cast<uint64_t>(out_cols) * esize, kBM, kChunk,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
   TcParams p{};
   p.offsets = a.offsets;
   p.E = a.E;
@@ -468,6 +531,7 @@ cudaError_t launch_shape(const GemmArgs& a, int* err_word, cudaStream_t stream) 
   p.swiglu = a.epi == E4B_EPI_SWIGLU;
   p.out = a.out;
   p.out_bf16 = a.out_bf16;
+  p.out_cols = out_cols;
   const int wrows = p.swiglu ? kBM : S::HALVES * kBM;  // output columns (weight rows) per tile
   p.n_tiles = ((p.swiglu ? a.N / 2 : a.N) + wrows - 1) / wrows;
   p.err = err_word;
@@ -476,7 +540,7 @@ cudaError_t launch_shape(const GemmArgs& a, int* err_word, cudaStream_t stream) 
       ((a.total_rows + S::BN - 1) / S::BN + (a.E < a.total_rows ? a.E : a.total_rows)) * p.n_tiles;
   const int grid = static_cast<int>(tiles < di.sm_count ? tiles : di.sm_count);
   LaunchScope ls(p.swiglu ? "gemm.tc.swiglu" : "gemm.tc", stream);
-  grouped_nf4_tc_kernel<S><<<grid, kThreadsTc, S::kSmemBytes, stream>>>(tm_packed, tm_b, p);
+  grouped_nf4_tc_kernel<S><<<grid, kThreadsTc, S::kSmemBytes, stream>>>(tm_packed, tm_b, tm_out, p);
   return cudaGetLastError();
 }
 
@@ -506,11 +570,11 @@ cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int* err_word, cudaStream_
   int s = shape_override();
   if (s == 3 && swiglu) s = 0;
   if (s == 0) {
-    // Measured on B200: the plain (down-projection) GEMM runs best 128 x 256
-    // with two accumulator sets.  SwiGLU tiles take 256 routed rows when groups
-    // are large (few partial tiles), else 128 with the epilogue overlapped.
+    // Measured on B200 (OLMoE-, Qwen3- and gpt-oss-shaped prefill): SwiGLU
+    // runs best on the 2 x 128 x 256 tile; the plain GEMM on 128 x 256 with two
+    // accumulator sets unless the groups are large.
     const int64_t rows_per_group = a.total_rows / (a.E > 0 ? a.E : 1);
-    s = !swiglu ? 3 : (rows_per_group >= 512 ? 1 : 2);
+    s = swiglu ? 1 : (rows_per_group >= 512 ? 1 : 3);
   }
   if (s == 1) return launch_shape<ShapeWide>(a, err_word, stream);
   if (s == 2) return launch_shape<ShapeDouble>(a, err_word, stream);
