@@ -67,7 +67,7 @@ GroupedLayout grouped_layout(int64_t M, int64_t E, int64_t H, int64_t I, int k, 
   L.inv = c.take(S * sizeof(int32_t));
   L.row_token = c.take(S * sizeof(int32_t));
   L.route_ws = c.take(route_workspace_bytes(M, E, k));
-  L.xa = c.take(r > 0 ? S * r * sizeof(float) : 0);
+  L.xa = c.take(r > 0 ? S * 128 : 0);  // LoRA products, either layout (r <= 16)
   L.xg = c.take(S * H * sizeof(uint16_t));
   L.h = c.take(S * I * sizeof(uint16_t));
   L.z = c.take(S * H * sizeof(float));

@@ -77,20 +77,24 @@ struct GemmArgs {
   const uint16_t* lora_B;  // [E, N, r] or nullptr
   int r;
   float lora_scale;
-  float* xa;  // workspace [total_rows, r] (LoRA only)
+  float* xa;  // workspace LoRA products: [total_rows, r] fp32 (warp-MMA path) or [total_rows, 64] bf16 (tensor cores)
   uint16_t* a_gathered;  // workspace [total_rows, K]: routed rows gathered for the tensor-core kernel
   int* err;   // workspace error word of the tensor-core kernel's bounded waits
   int epi;    // e4b_epilogue
   void* out;
   bool out_bf16;
 };
-// Workspace: [error word, 256 B][LoRA x.A^T, total_rows * r fp32, 256-B aligned]
+// Workspace: [error word, 256 B][LoRA x.A^T, 128 B per row, 256-B aligned]
 // [gathered rows, total_rows * K bf16].
 size_t gemm_workspace_bytes(int64_t total_rows, int64_t K, int r);
 size_t gemm_workspace_xa_offset();
 size_t gemm_workspace_gather_offset(int64_t total_rows, int r);
 bool tc_supported(const GemmArgs& a);
 cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int* err_word, cudaStream_t stream);
+// Gathers the routed rows (when a.row_index is set) and writes the LoRA
+// products the tensor-core kernel reads: xa as [total_rows, 64] bf16,
+// scale * x . lora_A^T, zero past r.
+cudaError_t launch_tc_lora_prep(const GemmArgs& a, cudaStream_t stream);
 // Picks the implementation; reports the path name through set_path.
 cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const char** path);
 

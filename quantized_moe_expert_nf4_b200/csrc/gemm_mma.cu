@@ -301,7 +301,8 @@ namespace e4b {
 
 size_t gemm_workspace_xa_offset() { return 256; }
 size_t gemm_workspace_gather_offset(int64_t total_rows, int r) {
-  return 256 + align_up(r > 0 ? static_cast<size_t>(total_rows) * r * sizeof(float) : 0, 256);
+  // 128 bytes per row hold either layout of the LoRA products (r <= 16).
+  return 256 + align_up(r > 0 ? static_cast<size_t>(total_rows) * 128 : 0, 256);
 }
 size_t gemm_workspace_bytes(int64_t total_rows, int64_t K, int r) {
   return gemm_workspace_gather_offset(total_rows, r) + static_cast<size_t>(total_rows) * K * sizeof(uint16_t);
@@ -337,7 +338,10 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const ch
   const bool use_tc = ov == 2 || (ov == 0 && tc_ok && a.total_rows >= kTcMinRows);
   if (use_tc) {
     if (!tc_ok) return cudaErrorNotSupported;
-    if (a.row_index) {
+    if (a.lora_B && a.r > 0) {
+      cudaError_t err = launch_tc_lora_prep(a, stream);  // gathers too
+      if (err != cudaSuccess) return err;
+    } else if (a.row_index) {
       cudaError_t err = launch_gather_rows(a.A, a.a_rows, a.lda, a.row_index, a.total_rows, a.K, a.a_gathered, stream);
       if (err != cudaSuccess) return err;
     }

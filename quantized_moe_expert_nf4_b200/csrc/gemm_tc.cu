@@ -36,6 +36,7 @@
 
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 
 #include "async.cuh"
 #include "common.cuh"
@@ -59,6 +60,8 @@ constexpr uint32_t kOutChunkBytes = kChunk * kBM * 4;  // 32 rows x 128 columns 
 constexpr uint32_t kOutBytes = 2 * kOutChunkBytes;     // double-buffered
 constexpr uint32_t kSmemLimit = 227 * 1024;
 constexpr uint32_t kSmemMisc = 1024 + 512;       // alignment slack, barriers, TMEM slot
+constexpr int kLoraCols = 64;                    // width of a row of scale * x . lora_A^T (bf16, zero past r)
+constexpr size_t kLoraPrepSmemMax = 192 * 1024;  // lora_A[e] staged by the prep kernel
 
 template <int BN_, int HALVES_, int NACC_>
 struct TcShape {
@@ -101,6 +104,8 @@ struct TcParams {
   int out_cols;  // columns of out: N, or N / 2 for SwiGLU
   int n_tiles;
   int* err;
+  const uint16_t* lora_B;  // [E, N, r] bf16, or null (no LoRA step)
+  int r;
 };
 
 // The codebook's bf16 patterns split into low and high bytes, four entries per
@@ -165,7 +170,8 @@ __device__ __forceinline__ bool locate(const TcParams& p, int64_t t, int* e, int
 template <class S>
 __global__ void __launch_bounds__(kThreadsTc, 1)
     grouped_nf4_tc_kernel(const __grid_constant__ CUtensorMap tm_packed, const __grid_constant__ CUtensorMap tm_b,
-                          const __grid_constant__ CUtensorMap tm_out, TcParams p) {
+                          const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ CUtensorMap tm_xa,
+                          TcParams p) {
   constexpr int BN = S::BN, HALVES = S::HALVES, NACC = S::NACC, KS = S::kKS, AS = S::kAS;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -236,6 +242,22 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         }
         __syncwarp();
       }
+      if (ok && p.lora_B) {
+        // LoRA step: the tile's rows of scale * x . lora_A^T (bf16, 64 wide, zero past r)
+        const int s = kbg % KS;
+        if (kbg >= KS && !mbar_wait(&tma_empty[s], ((kbg / KS) - 1) & 1)) {
+          record_error(p.err, kErrWaitEmpty);
+          ok = false;
+          break;
+        }
+        unsigned char* st = smem + S::kOffTma + s * S::kTmaStageBytes;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&tma_full[s], S::kBBytes);
+          tma_load_2d(st + S::kPackedBytes, &tm_xa, 0, static_cast<int32_t>(rb), &tma_full[s]);
+        }
+        __syncwarp();
+        ++kbg;
+      }
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------- MMA issuer
@@ -279,6 +301,27 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           umma_commit(&a_empty[a]);
         }
         __syncwarp();
+      }
+      if (ok && p.lora_B) {
+        // LoRA step: D += lora_B[rows, 0:16] . (scale x . lora_A^T)[tokens, 0:16]^T, one K=16 MMA per half
+        const int s = kbg % KS, a = kbg % AS;
+        if (!mbar_wait(&a_full[a], (kbg / AS) & 1) || !mbar_wait(&tma_full[s], (kbg / KS) & 1)) {
+          record_error(p.err, kErrWaitFull);
+          ok = false;
+        } else {
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t a_addr = smem_u32(smem + S::kOffA + a * S::kAStageBytes);
+            const uint64_t bd = smem_desc_sw128(smem_u32(smem + S::kOffTma + s * S::kTmaStageBytes + S::kPackedBytes));
+#pragma unroll
+            for (int h = 0; h < HALVES; ++h)
+              umma_bf16(d + h * BN, smem_desc_sw128(a_addr + h * kAHalfBytes), bd, idesc, 1u);
+            umma_commit(&tma_empty[s]);
+            umma_commit(&a_empty[a]);
+          }
+          __syncwarp();
+          ++kbg;
+        }
       }
       if (!ok) break;
       if (lane == 0) umma_commit(&acc_full[slot]);
@@ -357,6 +400,35 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           if (lane == 0) mbar_arrive(&a_full[a]);
           ++kbg;
         }
+      }
+      if (ok && p.lora_B) {
+        // LoRA step: row n's lora_B[e, n, 0:r] as the first 16 k of an A row (chunks 0 and 1).
+        const int s = kbg % KS, a = kbg % AS;
+        if (!mbar_wait(&tma_full[s], (kbg / KS) & 1) ||
+            (kbg >= AS && !mbar_wait(&a_empty[a], ((kbg / AS) - 1) & 1))) {
+          record_error(p.err, kErrWaitFull);
+          ok = false;
+          break;
+        }
+        if (kq < 2) {
+          uint32_t v[4] = {0u, 0u, 0u, 0u};
+          if (valid) {
+            const uint16_t* lb = p.lora_B + (static_cast<int64_t>(e) * p.N + n) * p.r;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int j = kq * 8 + i;
+              const uint32_t b = j < p.r ? lb[j] : 0u;
+              v[i >> 1] |= b << (16 * (i & 1));
+            }
+          }
+          unsigned char* arow =
+              smem + S::kOffA + a * S::kAStageBytes + half * kAHalfBytes + (ri >> 3) * 1024 + (ri & 7) * 128;
+          *reinterpret_cast<uint4*>(arow + ((kq ^ (ri & 7)) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_full[a]);
+        ++kbg;
       }
     }
   } else if (warp < 4) {
@@ -499,6 +571,11 @@ cudaError_t launch_shape(const GemmArgs& a, int* err_word, cudaStream_t stream) 
                    out_cols, a.total_rows, static_cast<uint64_t>(out_cols) * esize, kBM, kChunk,
                    CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
+  const bool lora = a.lora_B != nullptr && a.r > 0;
+  CUtensorMap tm_xa = tm_b;  // unused without LoRA
+  if (lora && !make_map_2d(&tm_xa, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.xa, kLoraCols, a.total_rows, kLoraCols * 2, 64,
+                           S::BN, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
   TcParams p{};
   p.offsets = a.offsets;
   p.E = a.E;
@@ -510,6 +587,8 @@ cudaError_t launch_shape(const GemmArgs& a, int* err_word, cudaStream_t stream) 
   p.out = a.out;
   p.out_bf16 = a.out_bf16;
   p.out_cols = out_cols;
+  p.lora_B = lora ? a.lora_B : nullptr;
+  p.r = lora ? a.r : 0;
   const int wrows = p.swiglu ? kBM : S::HALVES * kBM;  // output columns (weight rows) per tile
   p.n_tiles = ((p.swiglu ? a.N / 2 : a.N) + wrows - 1) / wrows;
   p.err = err_word;
@@ -518,8 +597,90 @@ cudaError_t launch_shape(const GemmArgs& a, int* err_word, cudaStream_t stream) 
       ((a.total_rows + S::BN - 1) / S::BN + (a.E < a.total_rows ? a.E : a.total_rows)) * p.n_tiles;
   const int grid = static_cast<int>(tiles < di.sm_count ? tiles : di.sm_count);
   LaunchScope ls(p.swiglu ? "gemm.tc.swiglu" : "gemm.tc", stream);
-  grouped_nf4_tc_kernel<S><<<grid, kThreadsTc, S::kSmemBytes, stream>>>(tm_packed, tm_b, tm_out, p);
+  grouped_nf4_tc_kernel<S><<<grid, kThreadsTc, S::kSmemBytes, stream>>>(tm_packed, tm_b, tm_out, tm_xa, p);
   return cudaGetLastError();
+}
+
+// LoRA prep for the tensor-core kernel: one CTA per (group, 64-row tile),
+// lora_A[e] (r x K bf16) staged in shared memory, one warp per routed row.
+// The warp copies the row into `gathered` (when a row index is given) and
+// writes xa[p, 0:64] = bf16(scale * A_row . lora_A[e, j]) for j < r, zeros
+// after -- the B operand of the kernel's extra K=16 MMA step.
+struct PrepParams {
+  const uint16_t* A;
+  int64_t a_rows, lda;
+  const int32_t* row_index;  // nullable
+  const int32_t* offsets;
+  int E;
+  int64_t total_rows;
+  int K;
+  uint16_t* gathered;  // [total_rows, K] or null
+  const uint16_t* lora_A;
+  int r;
+  float scale;
+  uint16_t* xa;  // [total_rows, 64]
+};
+
+constexpr int kPrepRows = 64;
+
+__global__ void __launch_bounds__(256) lora_prep_kernel(PrepParams q) {
+  extern __shared__ __align__(16) uint16_t la_s[];  // [r, K]
+  __shared__ int64_t tile_s[3];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (warp == 0) {
+    int g;
+    int64_t b0, b1;
+    const bool found = find_group_tile(q.offsets, q.E, q.total_rows, kPrepRows, blockIdx.x, &g, &b0, &b1);
+    if (lane == 0) {
+      tile_s[0] = found ? g : -1;
+      tile_s[1] = b0;
+      tile_s[2] = b1;
+    }
+  }
+  __syncthreads();
+  const int e = static_cast<int>(tile_s[0]);
+  if (e < 0) return;
+  const int64_t rb = tile_s[1], re = tile_s[2];
+  const int K = q.K, kv = K / 8;
+  const uint4* src_a = reinterpret_cast<const uint4*>(q.lora_A + static_cast<int64_t>(e) * q.r * K);
+  for (int i = threadIdx.x; i < q.r * kv; i += blockDim.x) reinterpret_cast<uint4*>(la_s)[i] = src_a[i];
+  __syncthreads();
+  for (int64_t pr = rb + warp; pr < re; pr += blockDim.x / 32) {
+    int64_t src = q.row_index ? q.row_index[pr] : pr;
+    src = clampv<int64_t>(src, 0, q.a_rows - 1);
+    const uint4* xrow = reinterpret_cast<const uint4*>(q.A + src * q.lda);
+    uint4* grow = q.gathered ? reinterpret_cast<uint4*>(q.gathered + pr * K) : nullptr;
+    float acc[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) acc[j] = 0.f;
+    for (int c = lane; c < kv; c += 32) {
+      const uint4 xv = __ldg(xrow + c);
+      if (grow) grow[c] = xv;
+      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        if (j >= q.r) break;
+        const uint4 av = reinterpret_cast<const uint4*>(la_s + j * K)[c];
+        const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[j] = fmaf(__uint_as_float(xw[i] << 16), __uint_as_float(aw[i] << 16), acc[j]);
+          acc[j] = fmaf(__uint_as_float(xw[i] & 0xffff0000u), __uint_as_float(aw[i] & 0xffff0000u), acc[j]);
+        }
+      }
+    }
+    float v0 = 0.f, v1 = 0.f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (j >= q.r) break;
+      float v = acc[j];
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (j == 2 * lane) v0 = v;
+      if (j == 2 * lane + 1) v1 = v;
+    }
+    reinterpret_cast<uint32_t*>(q.xa + pr * kLoraCols)[lane] = pack_bf16x2(q.scale * v0, q.scale * v1);
+  }
 }
 
 using ShapeWide = TcShape<256, 2, 1>;    // 2 x 128 weight rows x 256 routed rows, one accumulator set
@@ -577,9 +738,14 @@ bool encode_tensor_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const v
 }
 
 bool tc_supported(const GemmArgs& a) {
-  // No LoRA epilogue in the tensor-core kernel yet; the operand rows must be
-  // contiguous (row_index already applied); K % 64 and N % 64 hold by contract.
-  return a.lora_B == nullptr && a.row_index == nullptr && a.lda % 8 == 0 && tensor_maps_available();
+  // The operand rows must be contiguous (row_index already applied); K % 64
+  // and N % 64 hold by contract.  With LoRA, lora_A[e] must fit the prep
+  // kernel's shared memory and the products need their workspace rows.
+  if (a.row_index != nullptr || a.lda % 8 != 0 || !tensor_maps_available()) return false;
+  if (a.lora_B && a.r > 0)
+    return a.r <= 16 && a.xa != nullptr && static_cast<size_t>(a.r) * a.K * 2 <= kLoraPrepSmemMax &&
+           (reinterpret_cast<uintptr_t>(a.lora_A) & 15u) == 0;
+  return true;
 }
 
 cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int* err_word, cudaStream_t stream) {
@@ -596,6 +762,40 @@ cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int* err_word, cudaStream_
   if (s == 1) return launch_shape<ShapeWide>(a, err_word, stream);
   if (s == 2) return launch_shape<ShapeDouble>(a, err_word, stream);
   return launch_shape<ShapeNarrow>(a, err_word, stream);
+}
+
+cudaError_t launch_tc_lora_prep(const GemmArgs& a, cudaStream_t stream) {
+  if (a.total_rows == 0) return cudaSuccess;
+  PrepParams q{};
+  q.A = a.A;
+  q.a_rows = a.a_rows;
+  q.lda = a.lda;
+  q.row_index = a.row_index;
+  q.offsets = a.offsets;
+  q.E = a.E;
+  q.total_rows = a.total_rows;
+  q.K = a.K;
+  q.gathered = a.row_index ? a.a_gathered : nullptr;
+  q.lora_A = a.lora_A;
+  q.r = a.r;
+  q.scale = a.lora_scale;
+  q.xa = reinterpret_cast<uint16_t*>(a.xa);
+  const size_t smem = static_cast<size_t>(a.r) * a.K * 2;
+  static size_t configured = 0;
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (smem > configured) {
+      cudaError_t err = cudaFuncSetAttribute(lora_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kLoraPrepSmemMax));
+      if (err != cudaSuccess) return err;
+      configured = kLoraPrepSmemMax;
+    }
+  }
+  const int64_t tiles = (a.total_rows + kPrepRows - 1) / kPrepRows + (a.E < a.total_rows ? a.E : a.total_rows);
+  LaunchScope ls("gemm.tc.lora_prep", stream);
+  lora_prep_kernel<<<static_cast<unsigned>(tiles), 256, smem, stream>>>(q);
+  return cudaGetLastError();
 }
 
 }  // namespace e4b

@@ -71,7 +71,7 @@ def test_workspace_queries_are_host_only(lib):
     assert e4b.e4b_moe_route_permute_workspace_size(4096, 128, 8) > 4096 * 8 * 4
     # error word, LoRA products (256-byte aligned), gathered rows
     assert e4b.e4b_grouped_nf4_gemm_workspace_size(100, 128, 64, 0) == 256 + 100 * 64 * 2
-    xa = (100 * 8 * 4 + 255) // 256 * 256
+    xa = (100 * 128 + 255) // 256 * 256   # LoRA products: 128 bytes per row
     assert e4b.e4b_grouped_nf4_gemm_workspace_size(100, 128, 64, 8) == 256 + xa + 100 * 64 * 2
     st = e4b.ExpertStackC(1, 1, 1, 1, None, None, 0, 0.0, 64, 2048, 1024)
     n = lib.e4b_moe_expert_forward_workspace_size(2048, ctypes.byref(st), 8)

@@ -191,3 +191,28 @@ def test_grouped_gemm_tensor_core_bf16_and_exact_sums(monkeypatch, shape):
     A = workloads.bf16_bits_to_f32(c["Abits"]).astype(np.float64)
     want = A[c["ridx"]].sum(axis=1)[:, None] * np.ones((1, 640))
     assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("shape", TC_SHAPES)
+@pytest.mark.parametrize("r", [3, 8, 16])
+@pytest.mark.parametrize("epi", [e4b.E4B_EPI_NONE, e4b.E4B_EPI_SWIGLU])
+def test_grouped_gemm_tensor_core_lora(monkeypatch, shape, r, epi):
+    """The tensor-core kernel's LoRA step (one K=16 MMA per tile on lora_B rows
+    and bf16(scale * x . lora_A^T)): the extra rounding of the products to bf16
+    is 2^-9 of the delta, inside the path's tolerance."""
+    require_gpu()
+    monkeypatch.setenv("E4B_GEMM", "tc")
+    monkeypatch.setenv("E4B_TC_SHAPE", shape)
+    c = _case(4, 640, 320, [300, 0, 129, 77], 256, seed=40 + r, lora_r=r)
+    for use_ridx in (True, False):
+        if not use_ridx:
+            c["Abits"] = np.resize(c["Abits"], (c["rows"], c["K"]))
+        got, path = _run_gpu(c, epi, torch.float32, use_ridx=use_ridx)
+        assert path.startswith("gemm.tc"), path
+        ref = _oracle(c, epi, use_ridx=use_ridx)
+        fro, mx = rel_errors(got, ref)
+        tol = gemm_tolerance(path, epi, torch.float32)
+        print(f"[parity] tc lora {shape} r={r} epi {epi} ridx {use_ridx}: rel_fro={fro:.2e} max={mx:.2e}")
+        assert fro <= tol and mx <= 2 * tol
+        # the delta matters
+        assert rel_errors(_oracle(dict(c, r=0), epi, use_ridx=use_ridx), ref)[0] > 1e-2
