@@ -70,7 +70,7 @@ GroupedLayout grouped_layout(int64_t M, int64_t E, int64_t H, int64_t I, int k, 
   L.xa = c.take(r > 0 ? S * 128 : 0);  // LoRA products, either layout (r <= 16)
   L.xg = c.take(S * H * sizeof(uint16_t));
   L.h = c.take(S * I * sizeof(uint16_t));
-  L.z = c.take(S * H * sizeof(float));
+  L.z = c.take(S * H * sizeof(uint16_t));
   L.total = c.off;
   return L;
 }
@@ -412,11 +412,11 @@ static e4b_status forward_grouped(const uint16_t* x, int64_t M, const float* log
   d.K = static_cast<int>(w->I);
   d.err = at<int>(ws, L.err);
   d.epi = E4B_EPI_NONE;
-  d.out = at<float>(ws, L.z);
-  d.out_bf16 = false;
+  d.out = at<uint16_t>(ws, L.z);
+  d.out_bf16 = true;  // per-slot expert outputs in bf16 (the combine sums them in fp32)
   const char* p2 = "";
   if ((err = launch_grouped_gemm(d, stream, &p2)) != cudaSuccess) return cuda_fail(err, "down gemm launch");
-  if ((err = launch_combine(at<float>(ws, L.z), o.inv, o.w, M, k, static_cast<int>(w->H), out, stream)) != cudaSuccess)
+  if ((err = launch_combine(at<uint16_t>(ws, L.z), o.inv, o.w, M, k, static_cast<int>(w->H), out, stream)) != cudaSuccess)
     return cuda_fail(err, "combine launch");
   set_path("forward.grouped");
   return E4B_OK;

@@ -99,7 +99,7 @@ cudaError_t launch_tc_lora_prep(const GemmArgs& a, cudaStream_t stream);
 cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const char** path);
 
 // ---- combine ---------------------------------------------------------------
-cudaError_t launch_combine(const float* z, const int32_t* inv, const float* w, int64_t M, int k,
+cudaError_t launch_combine(const uint16_t* z, const int32_t* inv, const float* w, int64_t M, int k,
                            int H, uint16_t* out, cudaStream_t stream);
 
 // ---- fused small-M forward ---------------------------------------------------

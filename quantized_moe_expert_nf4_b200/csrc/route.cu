@@ -12,8 +12,11 @@
 //     warp with __match_any_sync (peers share an expert; rank = peers below);
 //   * positions = offsets[e] + (slots of e in earlier tiles) + local rank.
 // Small calls (<= 4096 slots) run all of it in one CTA, one launch.  Larger
-// calls use a tile kernel (top-k, local ranks, per-tile counts) and a scatter
-// kernel whose CTAs each rebuild the offsets from the per-tile counts.
+// calls use a tile kernel (top-k, local ranks, per-tile counts), a column scan
+// per expert over the tiles, and a scatter kernel whose CTAs each scan the
+// expert totals into the offsets.
+#include <algorithm>
+
 #include "common.cuh"
 #include "e4b_internal.h"
 #include "topk.cuh"
@@ -130,31 +133,53 @@ __global__ void __launch_bounds__(256) route_tile_kernel(const float* __restrict
   for (int e = tid; e < E; e += blockDim.x) tile_counts[static_cast<int64_t>(blockIdx.x) * E + e] = counts[e];
 }
 
-// Large path, kernel 2: every CTA rebuilds the offsets and its tile's bases.
-__global__ void __launch_bounds__(1024) route_scatter_kernel(int M, int E, int k, int ntiles, RouteOut o,
+// Large path, kernel 2: one CTA per expert scans that expert's per-tile counts
+// over the tiles, in place (tile_counts[t][e] becomes the slots of e in tiles
+// before t), and writes the expert's total.
+__global__ void __launch_bounds__(1024) route_colscan_kernel(int ntiles, int E, int* __restrict__ tile_counts,
+                                                             int* __restrict__ totals) {
+  __shared__ int warp_sums[33];
+  const int e = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int nwarps = blockDim.x >> 5;
+  int carry = 0;
+  for (int base = 0; base < ntiles; base += blockDim.x) {
+    const int t = base + tid;
+    int* cell = tile_counts + static_cast<int64_t>(t) * E + e;
+    const int v = (t < ntiles) ? *cell : 0;
+    const int incl = warp_inclusive_scan(v);
+    if (lane == 31) warp_sums[wid] = incl;
+    __syncthreads();
+    if (wid == 0) {
+      const int ws = (lane < nwarps) ? warp_sums[lane] : 0;
+      const int wi = warp_inclusive_scan(ws);
+      if (lane < nwarps) warp_sums[lane] = wi - ws;
+      if (lane == 31) warp_sums[32] = wi;  // block total
+    }
+    __syncthreads();
+    if (t < ntiles) *cell = carry + warp_sums[wid] + incl - v;
+    const int total = warp_sums[32];
+    __syncthreads();
+    carry += total;
+  }
+  if (tid == 0) totals[e] = carry;
+}
+
+// Large path, kernel 3: every CTA scans the expert totals into the offsets and
+// places its tile's slots.
+__global__ void __launch_bounds__(1024) route_scatter_kernel(int M, int E, int k, RouteOut o,
                                                              const int* __restrict__ local_rank,
-                                                             const int* __restrict__ tile_counts) {
+                                                             const int* __restrict__ tile_before,
+                                                             const int* __restrict__ totals) {
   extern __shared__ int smem[];
-  int* totals = smem;             // [E]
-  int* before = totals + E;       // [E]
-  int* offs = before + E;         // [E+1]
+  int* offs = smem;               // [E+1]
   int* warp_sums = offs + E + 1;  // [33]
   const int tid = threadIdx.x;
   const int tile = blockIdx.x;
-  for (int e = tid; e < E; e += blockDim.x) {
-    int tot = 0, bef = 0;
-    for (int t = 0; t < ntiles; ++t) {
-      const int c = tile_counts[static_cast<int64_t>(t) * E + e];
-      tot += c;
-      if (t < tile) bef += c;
-    }
-    totals[e] = tot;
-    before[e] = bef;
-  }
-  __syncthreads();
   block_exclusive_scan(totals, E, offs, warp_sums);
   if (tile == 0)
     for (int e = tid; e <= E; e += blockDim.x) o.offsets[e] = offs[e];
+  const int* before = tile_before + static_cast<int64_t>(tile) * E;
   const int f0 = tile * kTileTokens * k;
   const int nslots = min(kTileTokens, M - tile * kTileTokens) * k;
   for (int i = tid; i < nslots; i += blockDim.x) {
@@ -189,10 +214,18 @@ cudaError_t launch_route_t(const float* logits, int64_t M, int E, int k, bool re
   }
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  const size_t smem2 = (3 * E + 1 + 33) * sizeof(int);
+  int* totals = tile_counts + static_cast<int64_t>(ntiles) * E;
+  {
+    const int threads = std::min(1024, (ntiles + 31) / 32 * 32);
+    LaunchScope ls("route.colscan", stream);
+    route_colscan_kernel<<<E, threads, 0, stream>>>(ntiles, E, tile_counts, totals);
+  }
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  const size_t smem2 = (E + 1 + 33) * sizeof(int);
   LaunchScope ls("route.scatter", stream);
-  route_scatter_kernel<<<ntiles, 1024, smem2, stream>>>(static_cast<int>(M), E, k, ntiles, o, local_rank,
-                                                        tile_counts);
+  route_scatter_kernel<<<ntiles, 1024, smem2, stream>>>(static_cast<int>(M), E, k, o, local_rank, tile_counts,
+                                                        totals);
   set_path("route.tiled");
   return cudaGetLastError();
 }
@@ -237,7 +270,7 @@ size_t route_workspace_bytes(int64_t M, int64_t E, int k) {
   const int64_t S = M * k;
   if (S <= kSmallMaxSlots) return 0;
   const int64_t ntiles = (M + kTileTokens - 1) / kTileTokens;
-  return (align_up(S, 64) + ntiles * E) * sizeof(int);
+  return (align_up(S, 64) + ntiles * E + align_up(E, 64)) * sizeof(int);
 }
 
 cudaError_t launch_route(const float* logits, int64_t M, int E, int k, bool renormalize, const RouteOut& o,
