@@ -400,6 +400,14 @@ def replicas_for(cfg, M):
     return int(min(32, max(2, math.ceil(4 * L2_BYTES / per_step))))
 
 
+# DRAM bytes (read + write) per launch from one ncu capture of the kernel as it
+# is now, keyed by (layer config, M, kernel); a kernel changed since its capture
+# has no entry.  Source: profiles/decode_gate_up_traffic_olmoe_m1.md.
+MEASURED_TRAFFIC = {
+    ("olmoe", 1, "decode.gate_up"): 28410368,
+}
+
+
 def dominant_roofline(cfg, M, kt, touched_avg, peaks, long_region):
     name, (avg_ms, n) = max(kt.items(), key=lambda kv: kv[1][0] * kv[1][1])
     S = M * cfg.k
@@ -410,7 +418,7 @@ def dominant_roofline(cfg, M, kt, touched_avg, peaks, long_region):
         achieved = alg / (avg_ms * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
         return name, {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                      "traffic": None, "kernel": name, "avg_us": avg_ms * 1e3,
+                      "traffic": MEASURED_TRAFFIC.get((cfg.name, M, name)), "kernel": name, "avg_us": avg_ms * 1e3,
                       "algorithmic_bytes_per_launch": alg, "peak_source": peaks["source"] + " hbm_gbs"}
     # tensor-bound GEMM of the grouped path
     if "swiglu" in name:
@@ -421,7 +429,8 @@ def dominant_roofline(cfg, M, kt, touched_avg, peaks, long_region):
     key = "bf16_tflops_sustained" if long_region else "bf16_tflops"
     peak = peaks[key]
     return name, {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                  "traffic": None, "kernel": name, "avg_us": avg_ms * 1e3, "algorithmic_flops_per_launch": flops,
+                  "traffic": MEASURED_TRAFFIC.get((cfg.name, M, name)), "kernel": name, "avg_us": avg_ms * 1e3,
+                  "algorithmic_flops_per_launch": flops,
                   "peak_source": peaks["source"] + " " + key}
 
 

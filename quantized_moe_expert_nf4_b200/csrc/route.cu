@@ -243,8 +243,19 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
     const int64_t src = clampv<int64_t>(row_index[p], 0, a_rows - 1);
     const uint4* s = reinterpret_cast<const uint4*>(A + src * lda);
     uint4* d = reinterpret_cast<uint4*>(out + p * K);
-#pragma unroll 4
-    for (int i = lane; i < vecs; i += 32) d[i] = __ldg(s + i);
+    for (int i0 = 0; i0 < vecs; i0 += 8 * 32) {  // eight 16-byte loads per lane in flight
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * 32 + lane;
+        if (i < vecs) v[u] = __ldg(s + i);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * 32 + lane;
+        if (i < vecs) d[i] = v[u];
+      }
+    }
   }
 }
 
