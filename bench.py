@@ -472,6 +472,7 @@ def measure(args, name, rank, world, dist, peaks, primary):
     flops, nbytes = step_work(cfg, M, touched_avg)
     t_star = max(nbytes / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12))
     step_bound = "hbm" if nbytes / (peaks["hbm_gbs"] * 1e9) >= flops / (peaks["bf16_tflops"] * 1e12) else "tensor"
+    t_star_nom = max(nbytes / (NOMINAL_PEAKS["hbm_gbs"] * 1e9), flops / (NOMINAL_PEAKS["bf16_tflops"] * 1e12))
     if args.no_kernel_timing:
         kt, roof = {}, None
     else:
@@ -484,7 +485,9 @@ def measure(args, name, rank, world, dist, peaks, primary):
         "step_roofline": {"bound": step_bound, "t_star_us": t_star * 1e6, "frac": t_star / (ms * 1e-3),
                           "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
                           "peaks": {"hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"],
-                                    "source": peaks["source"]}},
+                                    "source": peaks["source"]},
+                          "nominal": {"peaks": NOMINAL_PEAKS, "source": "nominal B200 figures",
+                                      "t_star_us": t_star_nom * 1e6, "frac": t_star_nom / (ms * 1e-3)}},
         "kernels_us": {k: v[0] * 1e3 for k, v in kt.items()},
         "clocks": sampler.summary(),
     }
@@ -498,6 +501,38 @@ def measure(args, name, rank, world, dist, peaks, primary):
     del b
     torch.cuda.empty_cache()
     return res
+
+
+# Nominal B200 figures (HBM3e 8 TB/s, dense bf16 2.25 PFLOP/s), reported beside the measured peaks.
+NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
+
+
+def time_quantize(cfg, dev, reps=3):
+    """Load-time step, timed apart from the forward: e4b_nf4_quantize_stack on the
+    layer's whole gate_up stack from fp32 ([E, 2I, H]); HBM-bound (4 B read +
+    0.5 + 4/64 B written per weight)."""
+    import torch
+
+    from quantized_moe_expert_nf4_b200 import e4b
+
+    W = torch.randn((cfg.E, 2 * cfg.I, cfg.H), device=dev, dtype=torch.float32)
+    n = W.numel()
+    packed = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+    absmax = torch.empty(n // 64, dtype=torch.float32, device=dev)
+    e4b.e4b_nf4_quantize_stack(W, packed, absmax)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        e4b.e4b_nf4_quantize_stack(W, packed, absmax)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    nbytes = n * (4 + 0.5 + 4.0 / 64)
+    del W, packed, absmax
+    torch.cuda.empty_cache()
+    return {"stack": f"gate_up [{cfg.E}, {2 * cfg.I}, {cfg.H}] fp32", "ms": ms, "bytes": nbytes,
+            "GB_per_s": nbytes / (ms * 1e-3) / 1e9}
 
 
 def main():
@@ -555,6 +590,10 @@ def main():
                           "roofline_kernel": r["roofline"]["kernel"] if r["roofline"] else None,
                           "step_roofline_frac": r["step_roofline"]["frac"],
                           "clocks": r["clocks"]})
+    quant = None
+    if rank == 0 and world == 1:
+        quant = time_quantize(cfg, f"cuda:{local}")
+        quant["frac_hbm"] = quant["GB_per_s"] / peaks["hbm_gbs"]
     if rank == 0:
         cb = None
         if world == 1 and not args.no_cpu_baseline:
@@ -577,6 +616,7 @@ def main():
             "kernels_us": main_res["kernels_us"],
             "cpu_baseline": cb, "e2e": main_res["e2e"], "clocks": main_res["clocks"],
             "gpu_launches": main_res["launches_per_step"] * args.steps,
+            "quantize": quant,
             "sweep": sweep,
         }
         print(json.dumps(line), flush=True)

@@ -1,6 +1,5 @@
 // Asynchronous-copy and synchronisation primitives for sm_100a (inline PTX):
-// mbarriers, 1-D bulk copies (TMA engine) into shared memory, L2 prefetch,
-// programmatic dependent launch, named barriers.  Every wait is bounded: it
+// mbarriers, L2 prefetch, programmatic dependent launch.  Every wait is bounded: it
 // gives up after a time limit, records an error code and returns false, so a
 // kernel never spins forever.
 #pragma once
@@ -63,40 +62,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
-__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Spinning wait (non-blocking test_wait) for latency-critical hand-offs: a
-// suspended try_wait can take a few hundred nanoseconds to resume after the
-// phase completes.  Bounded like mbar_wait; false after the time limit.
-__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity) {
-  if (mbar_test_wait(bar, parity)) return true;
-  const unsigned long long t0 = global_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_test_wait(bar, parity)) return true;
-    if ((i & 1023u) == 0 && global_ns() - t0 > kWaitLimitNs) return false;
-  }
-}
-
-// 1-D bulk copy global -> shared, completion counted on `bar` (bytes % 16 == 0,
-// both addresses 16-byte aligned).
-__device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(smem_dst)),
-      "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
 __device__ __forceinline__ void prefetch_l2(const void* gmem, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gmem), "r"(bytes) : "memory");
 }
@@ -105,11 +70,6 @@ __device__ __forceinline__ void prefetch_l2(const void* gmem, uint32_t bytes) {
 // prologue / wait until the previous kernel's results are visible.
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-
-// Barrier over a subset of warps (ids 1..15; 0 is __syncthreads).
-__device__ __forceinline__ void named_barrier(int id, int threads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
 
 __device__ __forceinline__ void record_error(int* err, int code) {
   if (err) atomicCAS(err, kErrNone, code);

@@ -55,7 +55,6 @@ struct RouteOut {
   int32_t* row_token;  // [S] perm[p] / k, or nullptr
 };
 size_t route_workspace_bytes(int64_t M, int64_t E, int k);
-bool route_uses_small_kernel(int64_t M, int64_t E, int k);
 cudaError_t launch_route(const float* logits, int64_t M, int E, int k, bool renormalize,
                          const RouteOut& o, void* workspace, cudaStream_t stream);
 // out[p, :] = A[row_index[p], :K] for p < S (the routed rows, contiguous).

@@ -275,8 +275,6 @@ cudaError_t launch_gather_rows(const uint16_t* A, int64_t a_rows, int64_t lda, c
   return cudaGetLastError();
 }
 
-bool route_uses_small_kernel(int64_t M, int64_t E, int k) { return M * k <= kSmallMaxSlots; }
-
 size_t route_workspace_bytes(int64_t M, int64_t E, int k) {
   const int64_t S = M * k;
   if (S <= kSmallMaxSlots) return 0;

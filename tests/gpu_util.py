@@ -5,7 +5,7 @@ import torch
 
 from quantized_moe_expert_nf4_b200 import e4b
 
-# Tolerances of the layer output against the float64 oracle (spec bar).
+# Tolerances of the layer output against the float64 oracle (relative Frobenius and max-abs bars).
 REL_FRO_TOL = 1e-2
 MAX_ABS_TOL = 2e-2
 
