@@ -19,13 +19,13 @@
 //
 // Only experts that some token selected are read.  Both kernels are split-K
 // GEMVs on warp tensor cores: each CTA owns a contiguous run of items, its 16
-// warps split K, and each warp loads its 8-byte slices of the packed rows
-// straight from HBM into the registers of an mma.sync m16n8k16 fragment
-// (weight rows = MMA rows, the <= 8 tokens = the 8 MMA columns), several
-// items ahead, so ~100 KB per SM are in flight.  Nibbles become bf16 through a
-// per-lane replicated byte -> bf16x2 codebook table in shared memory (lane l
-// reads only bank l), and each 64-block's absmax is applied to the fp32 partial
-// product once.  One block barrier per batch gathers the 16 warps' partials.
+// warps split K in spans of two absmax blocks (128 k), and each lane loads its
+// 16-byte slice of a span of the packed rows straight from HBM into the
+// registers of an mma.sync m16n8k16 fragment (weight rows = MMA rows, the <= 8
+// tokens = the 8 MMA columns), several items ahead.  Nibbles become bf16
+// through a per-lane replicated byte -> bf16x2 codebook table in shared memory
+// (lane l reads only bank l), scaled by the block's bf16 absmax before the
+// MMA.  One block barrier per batch gathers the 16 warps' partials.
 #include <algorithm>
 #include <mutex>
 
@@ -40,9 +40,9 @@ namespace {
 constexpr int kMaxM = 8;
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
-constexpr int kSlots = 8;                  // (item, k-block) load slots per warp per batch in kernel A
-constexpr int kPairSlots = 4;              // (expert, k-block) load slots per warp per batch in kernel B
-constexpr int kMaxKBW = 4;                 // k-blocks per warp per item: H <= 64 * 16 * 4 = 4096
+constexpr int kSlots = 4;                  // (item, span) load slots per warp per batch in kernel A
+constexpr int kPairSlots = 2;              // (expert, span) load slots per warp per batch in kernel B
+constexpr int kMaxKBW = 2;                 // spans (2 k-blocks) per warp per item: H <= 128 * 16 * 2 = 4096
 constexpr unsigned long long kPrefetchLimit = 64ull << 20;
 constexpr uint32_t kPrefetchChunk = 32 * 1024;
 
@@ -69,7 +69,8 @@ struct Layout {
 
 __host__ __device__ inline uint32_t al(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
-__host__ __device__ inline int kbw_of(int H) { return (H / 64 + kWarps - 1) / kWarps; }
+// Spans of 128 k (2 absmax blocks, 64 packed bytes of a row) per warp per item.
+__host__ __device__ inline int kbw_of(int H) { return ((H / 64 + 1) / 2 + kWarps - 1) / kWarps; }
 
 // Shared-memory carve of kernel A (gate_up) or B (down).
 __host__ __device__ inline Layout make_layout(bool is_a, int M, int k, int E, int H, int r) {
@@ -80,7 +81,7 @@ __host__ __device__ inline Layout make_layout(bool is_a, int M, int k, int E, in
   L.xs = o;
   if (is_a) o = al(o + M * (2 * H + 16), 16);
   L.red = o;
-  const int items = is_a ? kSlots : 1;  // partial sums of up to 8 items per batch (A), 1 row block (B)
+  const int items = is_a ? kSlots : 1;  // partial sums of up to kSlots items per batch (A), 1 row block (B)
   o = al(o + items * kWarps * 32 * 16, 16);
   const int S = M * k;
   L.ids = o;
@@ -108,20 +109,35 @@ __device__ __forceinline__ void mma_16816(float c[4], uint32_t a0, uint32_t a1, 
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// One 64-block of a 16-row tile: rows g (MMA rows 0..7) and g+8, thread t owns
-// physical k in [16t, 16t+16) = 8 byte pairs; MMA j takes pairs 2j and 2j+1.
-__device__ __forceinline__ void block_mma(const uint32_t* __restrict__ lut_lane, uint2 r0, uint2 r1, uint4 x0, uint4 x1,
-                                          float tmp[4]) {
-  auto L = [&](uint32_t word, int byte) { return lut_lane[((word >> (8 * byte)) & 0xffu) << 5]; };
-  tmp[0] = tmp[1] = tmp[2] = tmp[3] = 0.0f;
-  mma_16816(tmp, L(r0.x, 0), L(r1.x, 0), L(r0.x, 1), L(r1.x, 1), x0.x, x0.y);
-  mma_16816(tmp, L(r0.x, 2), L(r1.x, 2), L(r0.x, 3), L(r1.x, 3), x0.z, x0.w);
-  mma_16816(tmp, L(r0.y, 0), L(r1.y, 0), L(r0.y, 1), L(r1.y, 1), x1.x, x1.y);
-  mma_16816(tmp, L(r0.y, 2), L(r1.y, 2), L(r0.y, 3), L(r1.y, 3), x1.z, x1.w);
+__device__ __forceinline__ uint4 ld_stream_u4(const uint8_t* p) {
+  return __ldcs(reinterpret_cast<const uint4*>(p));
 }
 
-__device__ __forceinline__ uint2 ld_stream_u2(const uint8_t* p) {
-  return __ldcs(reinterpret_cast<const uint2*>(p));
+// One span (128 k = 2 absmax blocks) of a 16-row tile, accumulated into c.
+// Thread (g, t) owns physical k [32t, 32t+32) of the span -- 16 packed bytes of
+// row g (r0) and of row g+8 (r1), all inside k-block t/2 -- and the matching 32
+// bf16 of its token column g (x).  Each byte's codebook pair is scaled by its
+// row's bf16(absmax) before the MMA (the block scale differs between threads of
+// one MMA, so it cannot be applied to the product).  MMA j takes bytes 2j and
+// 2j+1 of each row; K is permuted identically on both operands.
+__device__ __forceinline__ void span_mma(const uint32_t* __restrict__ lut_lane, uint4 r0, uint4 r1, float a0,
+                                         float a1, const uint4 x[4], float c[4]) {
+  const __nv_bfloat162 s0 = __float2bfloat162_rn(a0), s1 = __float2bfloat162_rn(a1);
+  const uint32_t w0[4] = {r0.x, r0.y, r0.z, r0.w}, w1[4] = {r1.x, r1.y, r1.z, r1.w};
+  const uint32_t xw[16] = {x[0].x, x[0].y, x[0].z, x[0].w, x[1].x, x[1].y, x[1].z, x[1].w,
+                           x[2].x, x[2].y, x[2].z, x[2].w, x[3].x, x[3].y, x[3].z, x[3].w};
+  auto pair = [&](uint32_t word, int byte, __nv_bfloat162 sc) {
+    uint32_t v = lut_lane[((word >> (8 * byte)) & 0xffu) << 5];
+    __nv_bfloat162 h2 = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&v), sc);
+    return *reinterpret_cast<uint32_t*>(&h2);
+  };
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int b = 2 * (j & 1);
+    const uint32_t wa = w0[j >> 1], wb = w1[j >> 1];
+    mma_16816(c, pair(wa, b, s0), pair(wb, b, s1), pair(wa, b + 1, s0), pair(wb, b + 1, s1), xw[2 * j],
+              xw[2 * j + 1]);
+  }
 }
 
 // Top-k of token `t` by the calling warp, with the key array sized for E.
@@ -302,27 +318,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gate_up_kernel(DecodeParam
     const int nb = min(IB, i1 - b0);
     if (b0 > i0 && tid < IB) prefetch_items(p, touched, min(b0 + 2 * IB, i1), min(b0 + 3 * IB, i1));
     // Issue every load of the batch first (HBM latency is hidden by the batch).
-    uint2 pk[IB][KBW][2];
+    // 16-byte loads: a lane's 32 k of a span lie in k-block 2 * span + t / 2.
+    uint4 pk[IB][KBW][2];
     float am[IB][KBW][2];
 #pragma unroll
     for (int ii = 0; ii < IB; ++ii) {
       const int it = b0 + (ii < nb ? ii : 0);
       const int u = it / ipe, rb = it % ipe;
       const int64_t grow = static_cast<int64_t>(touched[u]) * 2 * I + rb * 8 + g;  // gate row of lane's MMA row g
-      const uint8_t* gp = p.gu_packed + grow * row_bytes + 8 * t;
+      const uint8_t* gp = p.gu_packed + grow * row_bytes + 16 * t;
       const uint8_t* up = gp + static_cast<int64_t>(I) * row_bytes;
       const float* ga = p.gu_absmax + grow * KB;
       const float* ua = ga + static_cast<int64_t>(I) * KB;
 #pragma unroll
       for (int q2 = 0; q2 < KBW; ++q2) {
-        const int kb = warp + kWarps * q2;
+        const int sp = warp + kWarps * q2;
+        const int kb = 2 * sp + (t >> 1);
         if (ii < nb && kb < KB) {
-          pk[ii][q2][0] = ld_stream_u2(gp + kb * 32);
-          pk[ii][q2][1] = ld_stream_u2(up + kb * 32);
+          pk[ii][q2][0] = ld_stream_u4(gp + sp * 64);
+          pk[ii][q2][1] = ld_stream_u4(up + sp * 64);
           am[ii][q2][0] = __ldg(ga + kb);
           am[ii][q2][1] = __ldg(ua + kb);
         } else {
-          pk[ii][q2][0] = pk[ii][q2][1] = make_uint2(0, 0);
+          pk[ii][q2][0] = pk[ii][q2][1] = make_uint4(0, 0, 0, 0);
           am[ii][q2][0] = am[ii][q2][1] = 0.f;
         }
       }
@@ -332,23 +350,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gate_up_kernel(DecodeParam
       if (ii >= nb) break;
       const int u = (b0 + ii) / ipe;
       const bool has_g = (g < p.M) && slotmap[u * kMaxM + g] >= 0;  // token g routes to this expert
-      const uint16_t* xrow = xs + g * xstride + 16 * t;
+      const uint16_t* xrow = xs + g * xstride + 32 * t;
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int q2 = 0; q2 < KBW; ++q2) {
-        const int kb = warp + kWarps * q2;
-        if (kb >= KB) break;
-        uint4 x0 = make_uint4(0, 0, 0, 0), x1 = make_uint4(0, 0, 0, 0);
-        if (has_g) {
-          x0 = *reinterpret_cast<const uint4*>(xrow + kb * 64);
-          x1 = *reinterpret_cast<const uint4*>(xrow + kb * 64 + 8);
+        const int sp = warp + kWarps * q2;
+        if (2 * sp >= KB) break;
+        uint4 xv[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+        if (has_g && 2 * sp + (t >> 1) < KB) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) xv[i] = *reinterpret_cast<const uint4*>(xrow + sp * 128 + 8 * i);
         }
-        float tmp[4];
-        block_mma(lut_lane, pk[ii][q2][0], pk[ii][q2][1], x0, x1, tmp);
-        acc[0] = fmaf(tmp[0], am[ii][q2][0], acc[0]);
-        acc[1] = fmaf(tmp[1], am[ii][q2][0], acc[1]);
-        acc[2] = fmaf(tmp[2], am[ii][q2][1], acc[2]);
-        acc[3] = fmaf(tmp[3], am[ii][q2][1], acc[3]);
+        span_mma(lut_lane, pk[ii][q2][0], pk[ii][q2][1], am[ii][q2][0], am[ii][q2][1], xv, acc);
       }
       red[(ii * kWarps + warp) * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
     }
@@ -413,7 +426,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_down_kernel(DecodeParams p
   // The prologue reads only inputs the gate_up kernel does not write.
   decode_prologue(p, lut, nullptr, 0, ids_s, w_s, uidx, touched, slotmap, &nU_s);
   const int nU = nU_s;
-  const int npairs = nU * KB;  // (expert, k-block) pairs of one row block
+  const int NSP = (KB + 1) / 2;  // spans of 128 k (two absmax blocks) in a down row
+  const int npairs = nU * NSP;   // (expert, span) pairs of one row block
   const int g = lane >> 2, t = lane & 3;
   const uint32_t* lut_lane = lut + lane;
   const int64_t row_bytes = I / 2;
@@ -428,30 +442,34 @@ __global__ void __launch_bounds__(kThreads, 1) decode_down_kernel(DecodeParams p
   for (int rb = blockIdx.x; rb < H / 16; rb += gridDim.x) {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     for (int pb = warp; pb < npairs; pb += kWarps * kPairSlots) {
-      uint2 pk[kPairSlots][2];
+      uint4 pk[kPairSlots][2];
       float am[kPairSlots][2];
-      uint4 hx[kPairSlots][2];
+      uint4 hx[kPairSlots][4];
       float wc[kPairSlots][2];
 #pragma unroll
       for (int sl = 0; sl < kPairSlots; ++sl) {
         const int pi = pb + kWarps * sl;
-        pk[sl][0] = pk[sl][1] = make_uint2(0, 0);
+        pk[sl][0] = pk[sl][1] = make_uint4(0, 0, 0, 0);
         am[sl][0] = am[sl][1] = 0.f;
-        hx[sl][0] = hx[sl][1] = make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) hx[sl][i] = make_uint4(0, 0, 0, 0);
         wc[sl][0] = wc[sl][1] = 0.f;
         if (pi < npairs) {
-          const int u = pi / KB, kb = pi % KB;
+          const int u = pi / NSP, sp = pi % NSP;
+          const int kb = 2 * sp + (t >> 1);  // this lane's 32 k of the span lie in k-block kb
           const int64_t row = static_cast<int64_t>(touched[u]) * H + rb * 16 + g;
-          const uint8_t* rp = p.dn_packed + row * row_bytes + kb * 32 + 8 * t;
-          pk[sl][0] = ld_stream_u2(rp);
-          pk[sl][1] = ld_stream_u2(rp + 8 * row_bytes);
-          am[sl][0] = __ldg(p.dn_absmax + row * KB + kb);
-          am[sl][1] = __ldg(p.dn_absmax + (row + 8) * KB + kb);
-          const int slot_g = (g < p.M) ? slotmap[u * kMaxM + g] : -1;
-          if (slot_g >= 0) {
-            const uint16_t* hr = p.h + static_cast<int64_t>(slot_g) * I + kb * 64 + 16 * t;
-            hx[sl][0] = *reinterpret_cast<const uint4*>(hr);
-            hx[sl][1] = *reinterpret_cast<const uint4*>(hr + 8);
+          if (kb < KB) {
+            const uint8_t* rp = p.dn_packed + row * row_bytes + sp * 64 + 16 * t;
+            pk[sl][0] = ld_stream_u4(rp);
+            pk[sl][1] = ld_stream_u4(rp + 8 * row_bytes);
+            am[sl][0] = __ldg(p.dn_absmax + row * KB + kb);
+            am[sl][1] = __ldg(p.dn_absmax + (row + 8) * KB + kb);
+            const int slot_g = (g < p.M) ? slotmap[u * kMaxM + g] : -1;
+            if (slot_g >= 0) {
+              const uint16_t* hr = p.h + static_cast<int64_t>(slot_g) * I + sp * 128 + 32 * t;
+#pragma unroll
+              for (int i = 0; i < 4; ++i) hx[sl][i] = *reinterpret_cast<const uint4*>(hr + 8 * i);
+            }
           }
           const int s0 = (2 * t < p.M) ? slotmap[u * kMaxM + 2 * t] : -1;
           const int s1 = (2 * t + 1 < p.M) ? slotmap[u * kMaxM + 2 * t + 1] : -1;
@@ -462,12 +480,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_down_kernel(DecodeParams p
 #pragma unroll
       for (int sl = 0; sl < kPairSlots; ++sl) {
         if (pb + kWarps * sl >= npairs) break;
-        float tmp[4];
-        block_mma(lut_lane, pk[sl][0], pk[sl][1], hx[sl][0], hx[sl][1], tmp);
-        acc[0] = fmaf(tmp[0], am[sl][0] * wc[sl][0], acc[0]);
-        acc[1] = fmaf(tmp[1], am[sl][0] * wc[sl][1], acc[1]);
-        acc[2] = fmaf(tmp[2], am[sl][1] * wc[sl][0], acc[2]);
-        acc[3] = fmaf(tmp[3], am[sl][1] * wc[sl][1], acc[3]);
+        float tmp[4] = {0.f, 0.f, 0.f, 0.f};
+        span_mma(lut_lane, pk[sl][0], pk[sl][1], am[sl][0], am[sl][1], hx[sl], tmp);
+        acc[0] = fmaf(tmp[0], wc[sl][0], acc[0]);
+        acc[1] = fmaf(tmp[1], wc[sl][1], acc[1]);
+        acc[2] = fmaf(tmp[2], wc[sl][0], acc[2]);
+        acc[3] = fmaf(tmp[3], wc[sl][1], acc[3]);
       }
     }
     red[warp * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
@@ -560,7 +578,7 @@ DecodeWs decode_ws(int64_t M, int k, int64_t I) {
 }  // namespace
 
 bool decode_supported(int64_t M, int64_t E, int k, int64_t H, int64_t I) {
-  if (M < 1 || M > kMaxM || k > 32 || E > 512 || H > 64 * kWarps * kMaxKBW) return false;
+  if (M < 1 || M > kMaxM || k > 32 || E > 512 || H > 128 * kWarps * kMaxKBW) return false;
   (void)I;
   DeviceInfo di;
   if (device_info(&di) != cudaSuccess) return false;
@@ -608,9 +626,7 @@ cudaError_t launch_decode_forward(const DecodeArgs& a, cudaStream_t stream) {
   const size_t smem_b = make_layout(false, p.M, p.k, p.E, p.H, 0).total;
   switch (kbw_of(p.H)) {
     case 1: return launch_pair<1>(p, di.sm_count, smem_a, smem_b, stream);
-    case 2: return launch_pair<2>(p, di.sm_count, smem_a, smem_b, stream);
-    case 3: return launch_pair<3>(p, di.sm_count, smem_a, smem_b, stream);
-    default: return launch_pair<4>(p, di.sm_count, smem_a, smem_b, stream);
+    default: return launch_pair<2>(p, di.sm_count, smem_a, smem_b, stream);
   }
 }
 
