@@ -403,7 +403,9 @@ def replicas_for(cfg, M):
 # DRAM bytes (read + write) per launch from one ncu capture of the kernel as it
 # is now, keyed by (layer config, M, kernel); a kernel changed since its capture
 # has no entry.  Source: profiles/decode_gate_up_traffic_olmoe_m1.md.
-MEASURED_TRAFFIC = {}
+MEASURED_TRAFFIC = {
+    ("olmoe", 1, "decode.gate_up"): 28410368,
+}
 
 
 def dominant_roofline(cfg, M, kt, touched_avg, peaks, long_region):
