@@ -402,10 +402,8 @@ def replicas_for(cfg, M):
 
 # DRAM bytes (read + write) per launch from one ncu capture of the kernel as it
 # is now, keyed by (layer config, M, kernel); a kernel changed since its capture
-# has no entry.  Source: profiles/decode_gate_up_traffic_olmoe_m1.md.
-MEASURED_TRAFFIC = {
-    ("olmoe", 1, "decode.gate_up"): 28410368,
-}
+# has no entry (profiles/decode_gate_up_traffic_olmoe_m1.md holds the last capture).
+MEASURED_TRAFFIC = {}
 
 
 def dominant_roofline(cfg, M, kt, touched_avg, peaks, long_region):

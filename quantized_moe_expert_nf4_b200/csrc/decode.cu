@@ -12,7 +12,7 @@
 //             (bf16, [M*k, I], slot order).  It also prefetches the touched
 //             experts' down rows into L2, so that HBM keeps streaming while the
 //             second kernel starts.
-//   kernel B  routing again (before it waits on kernel A), then for every block
+//   kernel B  the routing kernel A published, then for every block
 //             of 16 output rows of H the down rows of every touched expert, with
 //             the routing weights folded into the per-block scale, so the
 //             combine happens inside the CTA in a fixed order (deterministic).
@@ -61,6 +61,9 @@ struct DecodeParams {
   float lora_scale;
   uint16_t* h;    // [S, I] bf16 (slot order)
   uint16_t* out;  // [M, H] bf16
+  // Routing result of the gate_up kernel for the down kernel: [nU, pad x3],
+  // touched [S], slotmap [S * kMaxM], weights [S] (as float bits).
+  int* meta;
 };
 
 struct Layout {
@@ -252,6 +255,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gate_up_kernel(DecodeParam
   pdl_launch_dependents();  // the down kernel may launch and run its prologue
   decode_prologue(p, lut, xs, xstride, ids_s, w_s, uidx, touched, slotmap, &nU_s);
   const int nU = nU_s;
+  if (blockIdx.x == 0) {
+    // Every CTA routed identically; one publishes the result for the down kernel.
+    const int S = p.M * p.k;
+    int* m_touched = p.meta + 4;
+    int* m_slotmap = m_touched + S;
+    float* m_w = reinterpret_cast<float*>(m_slotmap + S * kMaxM);
+    if (tid == 0) p.meta[0] = nU;
+    for (int i = tid; i < nU; i += blockDim.x) m_touched[i] = touched[i];
+    for (int i = tid; i < nU * kMaxM; i += blockDim.x) m_slotmap[i] = slotmap[i];
+    for (int i = tid; i < S; i += blockDim.x) m_w[i] = w_s[i];
+  }
   const int ipe = I / 8;  // items per expert
   const int nitems = nU * ipe;
   // A contiguous run of items per CTA: consecutive items are consecutive rows.
@@ -414,31 +428,36 @@ __global__ void __launch_bounds__(kThreads, 1) decode_down_kernel(DecodeParams p
   const Layout L = make_layout(false, p.M, p.k, p.E, p.H, 0);
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L.lut);
   float4* red = reinterpret_cast<float4*>(smem + L.red);
-  int* ids_s = reinterpret_cast<int*>(smem + L.ids);
   float* w_s = reinterpret_cast<float*>(smem + L.w);
-  int* uidx = reinterpret_cast<int*>(smem + L.uidx);
   int* touched = reinterpret_cast<int*>(smem + L.touched);
   int* slotmap = reinterpret_cast<int*>(smem + L.slotmap);
   __shared__ int nU_s;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int H = p.H, I = p.I, KB = I / 64;
-  // The prologue reads only inputs the gate_up kernel does not write.
-  decode_prologue(p, lut, nullptr, 0, ids_s, w_s, uidx, touched, slotmap, &nU_s);
+  // The down kernel starts once the gate_up kernel's CTAs leave the SMs; it
+  // builds its codebook table, waits for that kernel's results (h and the
+  // routing it published) and reads the routing instead of recomputing it.
+  fill_lut_warps(lut, 0);
+  pdl_wait();  // h and the routing written by the gate_up kernel are visible from here on
+  {
+    const int S = p.M * p.k;
+    const int* m_touched = p.meta + 4;
+    const int* m_slotmap = m_touched + S;
+    const float* m_w = reinterpret_cast<const float*>(m_slotmap + S * kMaxM);
+    const int n = __ldcg(p.meta);
+    if (tid == 0) nU_s = n;
+    for (int i = tid; i < n; i += blockDim.x) touched[i] = __ldcg(m_touched + i);
+    for (int i = tid; i < n * kMaxM; i += blockDim.x) slotmap[i] = __ldcg(m_slotmap + i);
+    for (int i = tid; i < S; i += blockDim.x) w_s[i] = __ldcg(m_w + i);
+  }
+  __syncthreads();
   const int nU = nU_s;
   const int NSP = (KB + 1) / 2;  // spans of 128 k (two absmax blocks) in a down row
   const int npairs = nU * NSP;   // (expert, span) pairs of one row block
   const int g = lane >> 2, t = lane & 3;
   const uint32_t* lut_lane = lut + lane;
   const int64_t row_bytes = I / 2;
-  // L2 prefetch of this CTA's first row block of every touched expert (weights
-  // do not depend on the gate_up kernel, so this runs before the wait).
-  for (int u = tid; u < nU && static_cast<int>(blockIdx.x) < H / 16; u += blockDim.x) {
-    const int64_t row = static_cast<int64_t>(touched[u]) * H + blockIdx.x * 16;
-    prefetch_l2(p.dn_packed + row * row_bytes, static_cast<uint32_t>(16 * row_bytes));
-    prefetch_l2(p.dn_absmax + row * KB, static_cast<uint32_t>(16 * KB * 4));
-  }
-  pdl_wait();  // h written by the gate_up kernel is visible from here on
   for (int rb = blockIdx.x; rb < H / 16; rb += gridDim.x) {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     for (int pb = warp; pb < npairs; pb += kWarps * kPairSlots) {
@@ -564,14 +583,16 @@ cudaError_t launch_pair(const DecodeParams& p, int sm_count, size_t smem_a, size
 }
 
 struct DecodeWs {
-  size_t h, total;
+  size_t h, meta, total;
 };
 
-// Workspace: h [M*k, I] bf16, then 256 bytes kept for the layout (unused).
+// Workspace: h [M*k, I] bf16, then the published routing (4 + S * (2 + kMaxM) ints).
 DecodeWs decode_ws(int64_t M, int k, int64_t I) {
   DecodeWs w;
+  const int64_t S = M * k;
   w.h = 0;
-  w.total = align_up(static_cast<size_t>(M * k * I * 2), 256) + 256;
+  w.meta = align_up(static_cast<size_t>(S * I * 2), 256);
+  w.total = w.meta + align_up(static_cast<size_t>(4 + S * (2 + kMaxM)) * 4, 256);
   return w;
 }
 
@@ -621,6 +642,7 @@ cudaError_t launch_decode_forward(const DecodeArgs& a, cudaStream_t stream) {
   p.r = r;
   p.lora_scale = r ? w->lora_alpha / static_cast<float>(r) : 0.f;
   p.h = reinterpret_cast<uint16_t*>(static_cast<char*>(a.workspace) + ws.h);
+  p.meta = reinterpret_cast<int*>(static_cast<char*>(a.workspace) + ws.meta);
   p.out = a.out;
   const size_t smem_a = make_layout(true, p.M, p.k, p.E, p.H, r).total;
   const size_t smem_b = make_layout(false, p.M, p.k, p.E, p.H, 0).total;
