@@ -6,6 +6,7 @@
 #include <algorithm>
 #include <cstdio>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -125,6 +126,21 @@ LaunchScope::LaunchScope(const char* name, cudaStream_t stream) : rec_(-1), stre
 
 LaunchScope::~LaunchScope() {
   if (rec_ >= 0) cudaEventRecord(g_timing.recs[rec_].stop, stream_);
+}
+
+cudaError_t ensure_smem_limit(const void* func, size_t bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<int, const void*>, size_t> raised;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  std::lock_guard<std::mutex> lk(mu);
+  size_t& cur = raised[{dev, func}];
+  if (bytes <= cur) return cudaSuccess;
+  err = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (err != cudaSuccess) return err;
+  cur = bytes;
+  return cudaSuccess;
 }
 
 cudaError_t device_info(DeviceInfo* out) {

@@ -27,7 +27,6 @@
 // (lane l reads only bank l), scaled by the block's bf16 absmax before the
 // MMA.  One block barrier per batch gathers the 16 warps' partials.
 #include <algorithm>
-#include <mutex>
 
 #include "async.cuh"
 #include "common.cuh"
@@ -531,29 +530,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_down_kernel(DecodeParams p
   }
 }
 
-// The dynamic shared-memory limit is a per-function attribute.  Each kernel
-// function keeps one high-water mark and the limit is only ever raised, so a
-// call with a smaller need never lowers the limit another call relies on.
-std::mutex g_attr_mu;
-size_t g_down_configured = 0;
-
 template <int KBW>
 cudaError_t raise_smem_limits(size_t smem_a, size_t smem_b) {
-  static size_t configured_a = 0;  // one per decode_gate_up_kernel<KBW>
-  std::lock_guard<std::mutex> lk(g_attr_mu);
-  if (smem_a > configured_a) {
-    cudaError_t e1 = cudaFuncSetAttribute(decode_gate_up_kernel<KBW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          static_cast<int>(smem_a));
-    if (e1 != cudaSuccess) return e1;
-    configured_a = smem_a;
-  }
-  if (smem_b > g_down_configured) {
-    cudaError_t e1 = cudaFuncSetAttribute(decode_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          static_cast<int>(smem_b));
-    if (e1 != cudaSuccess) return e1;
-    g_down_configured = smem_b;
-  }
-  return cudaSuccess;
+  cudaError_t err = ensure_smem_limit(reinterpret_cast<const void*>(decode_gate_up_kernel<KBW>), smem_a);
+  if (err != cudaSuccess) return err;
+  return ensure_smem_limit(reinterpret_cast<const void*>(decode_down_kernel), smem_b);
 }
 
 template <int KBW>

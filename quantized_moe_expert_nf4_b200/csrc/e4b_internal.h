@@ -125,6 +125,11 @@ struct DeviceInfo {
 };
 cudaError_t device_info(DeviceInfo* out);
 
+// Raises `func`'s dynamic shared-memory limit on the current device to at least
+// `bytes`.  The attribute belongs to one function on one device; it is only ever
+// raised, under a lock, so a call needing less never lowers what another relies on.
+cudaError_t ensure_smem_limit(const void* func, size_t bytes);
+
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 }  // namespace e4b

@@ -36,7 +36,6 @@
 
 #include <cstdlib>
 #include <cstring>
-#include <mutex>
 
 #include "async.cuh"
 #include "common.cuh"
@@ -549,13 +548,8 @@ cudaError_t launch_shape(const GemmArgs& a, int* err_word, cudaStream_t stream) 
   DeviceInfo di;
   cudaError_t err = device_info(&di);
   if (err != cudaSuccess) return err;
-  static bool configured = false;  // one flag per shape: each instantiation has its own kernel
-  if (!configured) {
-    err = cudaFuncSetAttribute(grouped_nf4_tc_kernel<S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(S::kSmemBytes));
-    if (err != cudaSuccess) return err;
-    configured = true;
-  }
+  err = ensure_smem_limit(reinterpret_cast<const void*>(grouped_nf4_tc_kernel<S>), S::kSmemBytes);
+  if (err != cudaSuccess) return err;
   CUtensorMap tm_packed, tm_b;
   const uint64_t total_w_rows = static_cast<uint64_t>(a.E) * a.N;
   if (!make_map_2d(&tm_packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.packed, a.K / 2, total_w_rows, a.K / 2, 32, kBM,
@@ -781,17 +775,8 @@ cudaError_t launch_tc_lora_prep(const GemmArgs& a, cudaStream_t stream) {
   q.scale = a.lora_scale;
   q.xa = reinterpret_cast<uint16_t*>(a.xa);
   const size_t smem = static_cast<size_t>(a.r) * a.K * 2;
-  static size_t configured = 0;
-  static std::mutex mu;
-  {
-    std::lock_guard<std::mutex> lk(mu);
-    if (smem > configured) {
-      cudaError_t err = cudaFuncSetAttribute(lora_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(kLoraPrepSmemMax));
-      if (err != cudaSuccess) return err;
-      configured = kLoraPrepSmemMax;
-    }
-  }
+  cudaError_t err = ensure_smem_limit(reinterpret_cast<const void*>(lora_prep_kernel), smem);
+  if (err != cudaSuccess) return err;
   const int64_t tiles = (a.total_rows + kPrepRows - 1) / kPrepRows + (a.E < a.total_rows ? a.E : a.total_rows);
   LaunchScope ls("gemm.tc.lora_prep", stream);
   lora_prep_kernel<<<static_cast<unsigned>(tiles), 256, smem, stream>>>(q);
