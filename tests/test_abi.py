@@ -76,3 +76,27 @@ def test_workspace_queries_are_host_only(lib):
     st = e4b.ExpertStackC(1, 1, 1, 1, None, None, 0, 0.0, 64, 2048, 1024)
     n = lib.e4b_moe_expert_forward_workspace_size(2048, ctypes.byref(st), 8)
     assert n >= 2048 * 8 * (1024 * 2 + 2048 * 4)
+
+
+def test_gemm_workspace_too_small_is_rejected_on_the_host(lib):
+    """The workspace check runs before any device query: a call with one byte
+    too few returns E4B_ERR_WORKSPACE and names the size it needs."""
+    rows, N, K = 300, 128, 256
+    need = e4b.e4b_grouped_nf4_gemm_workspace_size(rows, N, K, 0)
+    assert need == 256 + rows * K * 2          # error word + the gathered routed rows
+    fake = ctypes.c_void_p(1 << 20)            # never dereferenced: rejected before launch
+    offs = ctypes.c_void_p(1 << 21)
+    st = lib.e4b_grouped_nf4_gemm(fake, rows, K, None, offs, 2, rows, fake, fake, N, K, None, None, 0, 0.0, 0,
+                                  fake, 0, fake, need - 1, None)
+    assert st == 3 and str(need).encode() in lib.e4b_last_error()
+
+
+def test_forward_workspace_covers_both_paths(lib):
+    """The forward workspace is the larger of the grouped and decode layouts,
+    and grows with M."""
+    st = e4b.ExpertStackC(1, 1, 1, 1, None, None, 0, 0.0, 64, 2048, 1024)
+    sizes = [lib.e4b_moe_expert_forward_workspace_size(M, ctypes.byref(st), 8) for M in (1, 8, 9, 64, 2048)]
+    assert all(a <= b for a, b in zip(sizes, sizes[1:]))
+    # grouped layout at M=9: per slot at least h (2I) + gathered x (2H) + Z (2H) bytes
+    assert sizes[2] >= 9 * 8 * (1024 * 2 + 2048 * 2 + 2048 * 2)
+    assert lib.e4b_moe_expert_forward_workspace_size(0, ctypes.byref(st), 8) == 0
