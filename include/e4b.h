@@ -178,7 +178,8 @@ E4B_API e4b_status e4b_moe_route_permute(const float* logits, int64_t M, int64_t
  * row_index       [total_rows] int32 indices into A, or NULL for p itself.
  * expert_offsets  [E+1] int32, non-decreasing, expert_offsets[E] == total_rows.
  * packed, absmax  [E, N*K/2] uint8 and [E, N*K/64] fp32 (e4b_nf4_quantize_stack).
- * lora_A, lora_B  [E, r, K] and [E, N, r] bf16, or both NULL (no adapter).
+ * lora_A, lora_B  [E, r, K] and [E, N, r] bf16, or both NULL (no adapter);
+ *                 16-byte aligned like every other tensor.
  * epi             E4B_EPI_NONE: out[p, n] = y[p, n], n < N.
  *                 E4B_EPI_SWIGLU: out[p, n] = SiLU(y[p, n]) * y[p, N/2 + n],
  *                 n < N/2 (gate = first half of the rows, up = second half).

@@ -316,6 +316,8 @@ e4b_status e4b_grouped_nf4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda, 
   if (total_rows > INT32_MAX) return fail(E4B_ERR_UNSUPPORTED, "total_rows exceeds int32");
   if ((A && !aligned16(A)) || !aligned16(packed) || (out && !aligned16(out)))
     return fail(E4B_ERR_INVALID_ARGUMENT, "A, packed and out must be 16-byte aligned");
+  if (lora_A && (!aligned16(lora_A) || !aligned16(lora_B)))
+    return fail(E4B_ERR_INVALID_ARGUMENT, "lora_A and lora_B must be 16-byte aligned");
   const size_t need = gemm_workspace_bytes(total_rows, K, r);
   if (workspace_bytes < need || (need > 0 && !workspace))
     return fail(E4B_ERR_WORKSPACE, "gemm workspace needs " + std::to_string(need) + " bytes");
@@ -366,6 +368,8 @@ static e4b_status check_stack(const e4b_expert_stack* w, int k) {
   if ((w->lora_A == nullptr) != (w->lora_B == nullptr))
     return fail(E4B_ERR_INVALID_ARGUMENT, "lora_A and lora_B must be both set or both NULL");
   if (w->lora_A && (w->lora_r < 1 || w->lora_r > 16)) return fail(E4B_ERR_UNSUPPORTED, "LoRA rank must be in [1, 16]");
+  if (w->lora_A && (!aligned16(w->lora_A) || !aligned16(w->lora_B)))
+    return fail(E4B_ERR_INVALID_ARGUMENT, "lora_A and lora_B must be 16-byte aligned");
   if (!aligned16(w->gu_packed) || !aligned16(w->dn_packed) || !aligned16(w->gu_absmax) || !aligned16(w->dn_absmax))
     return fail(E4B_ERR_INVALID_ARGUMENT, "packed stacks and absmax must be 16-byte aligned");
   return E4B_OK;

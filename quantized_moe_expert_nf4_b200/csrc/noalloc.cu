@@ -77,6 +77,8 @@ extern "C" e4b_status e4b_moe_expert_forward_decode_noalloc(const uint16_t* x, i
   auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
   if (!a16(x) || !a16(out) || !a16(w->gu_packed) || !a16(w->dn_packed) || !a16(w->gu_absmax) || !a16(w->dn_absmax))
     return nofail(E4B_ERR_INVALID_ARGUMENT, "x, out, packed stacks and absmax must be 16-byte aligned");
+  if (w->lora_A && (!a16(w->lora_A) || !a16(w->lora_B)))
+    return nofail(E4B_ERR_INVALID_ARGUMENT, "lora_A and lora_B must be 16-byte aligned");
   DeviceInfo di;
   cudaError_t err = device_info(&di);
   if (err != cudaSuccess) return nofail(E4B_ERR_CUDA, std::string("device query: ") + cudaGetErrorString(err));

@@ -100,3 +100,18 @@ def test_forward_workspace_covers_both_paths(lib):
     # grouped layout at M=9: per slot at least h (2I) + gathered x (2H) + Z (2H) bytes
     assert sizes[2] >= 9 * 8 * (1024 * 2 + 2048 * 2 + 2048 * 2)
     assert lib.e4b_moe_expert_forward_workspace_size(0, ctypes.byref(st), 8) == 0
+
+
+def test_misaligned_lora_adapter_is_rejected_on_the_host(lib):
+    """Kernels read lora_A with 16-byte loads: a misaligned adapter is an
+    argument error, never a launch."""
+    rows, N, K, r = 64, 128, 128, 8
+    need = e4b.e4b_grouped_nf4_gemm_workspace_size(rows, N, K, r)
+    p = ctypes.c_void_p(1 << 20)
+    bad = ctypes.c_void_p((1 << 20) + 2)
+    st = lib.e4b_grouped_nf4_gemm(p, rows, K, None, p, 2, rows, p, p, N, K, bad, p, r, 2.0, 0,
+                                  p, 0, p, need, None)
+    assert st == 1 and b"lora_A and lora_B" in lib.e4b_last_error()
+    stk = e4b.ExpertStackC(1 << 20, 1 << 20, 1 << 20, 1 << 20, (1 << 20) + 2, 1 << 20, 8, 16.0, 8, 256, 128)
+    st = lib.e4b_moe_expert_forward(p, 4, p, 2, 1, ctypes.byref(stk), p, p, 1 << 30, None)
+    assert st == 1 and b"lora_A and lora_B" in lib.e4b_last_error()
