@@ -567,12 +567,14 @@ struct DecodeWs {
   size_t h, meta, total;
 };
 
-// Workspace: h [M*k, I] bf16, then the published routing (4 + S * (2 + kMaxM) ints).
+// Workspace: the error word every workspace begins with (no decode kernel
+// waits, so it stays untouched), h [M*k, I] bf16, then the published routing
+// (4 + S * (2 + kMaxM) ints).
 DecodeWs decode_ws(int64_t M, int k, int64_t I) {
   DecodeWs w;
   const int64_t S = M * k;
-  w.h = 0;
-  w.meta = align_up(static_cast<size_t>(S * I * 2), 256);
+  w.h = 256;
+  w.meta = w.h + align_up(static_cast<size_t>(S * I * 2), 256);
   w.total = w.meta + align_up(static_cast<size_t>(4 + S * (2 + kMaxM)) * 4, 256);
   return w;
 }
