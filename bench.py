@@ -584,7 +584,12 @@ def main():
     sweep = []
     if not args.no_sweep and args.workload == DEFAULT_WORKLOAD:
         for name in DEFAULT_SWEEP:
-            r = measure(args, name, rank, world, dist, peaks, primary=False)
+            try:
+                r = measure(args, name, rank, world, dist, peaks, primary=False)
+            except Exception as exc:  # a failing sweep row is reported, the headline line still prints
+                sweep.append({"workload": name, "error": f"{type(exc).__name__}: {exc}"})
+                torch.cuda.empty_cache()
+                continue
             sweep.append({"workload": name, "value": r["value"], "ms_per_step": r["ms_per_step"],
                           "tflops": r["tflops"], "path": r["path"], "touched_experts_avg": r["touched_experts_avg"],
                           "roofline_frac": r["roofline"]["frac"] if r["roofline"] else None,
