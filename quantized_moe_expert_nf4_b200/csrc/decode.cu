@@ -27,6 +27,7 @@
 // (lane l reads only bank l), scaled by the block's bf16 absmax before the
 // MMA.  One block barrier per batch gathers the 16 warps' partials.
 #include <algorithm>
+#include <string>
 
 #include "async.cuh"
 #include "common.cuh"
@@ -588,15 +589,24 @@ DecodeWs decode_ws(int64_t M, int k, int64_t I) {
 
 }  // namespace
 
-bool decode_supported(int64_t M, int64_t E, int k, int64_t H, int64_t I) {
-  if (M < 1 || M > kMaxM || k > 32 || E > 512 || H > 128 * kWarps * kMaxKBW) return false;
+std::string decode_unsupported_reason(int64_t M, int64_t E, int k, int64_t H, int64_t I) {
   (void)I;
+  if (M < 1 || M > kMaxM) return "the decode path takes 1 to " + std::to_string(kMaxM) + " tokens (M=" + std::to_string(M) + ")";
+  if (k > 32) return "the decode path takes k <= 32 (k=" + std::to_string(k) + ")";
+  if (E > 512) return "the decode path takes at most 512 experts (E=" + std::to_string(E) + ")";
+  if (H > 128 * kWarps * kMaxKBW)
+    return "the decode path takes H <= " + std::to_string(128 * kWarps * kMaxKBW) + " (H=" + std::to_string(H) + ")";
   DeviceInfo di;
-  if (device_info(&di) != cudaSuccess) return false;
+  if (device_info(&di) != cudaSuccess) return "device query failed";
   const Layout a = make_layout(true, static_cast<int>(M), k, static_cast<int>(E), static_cast<int>(H), 16);
   const Layout b = make_layout(false, static_cast<int>(M), k, static_cast<int>(E), static_cast<int>(H), 0);
   const size_t lim = di.smem_optin - 1024;  // leave room for the kernels' static shared memory
-  return a.total <= lim && b.total <= lim;
+  if (a.total > lim || b.total > lim) return "the decode kernels' shared-memory plan does not fit this shape";
+  return "";
+}
+
+bool decode_supported(int64_t M, int64_t E, int k, int64_t H, int64_t I) {
+  return decode_unsupported_reason(M, E, k, H, I).empty();
 }
 
 size_t decode_workspace_bytes(int64_t M, int64_t E, int k, int64_t H, int64_t I, int r) {
