@@ -444,7 +444,7 @@ def replicas_for(cfg, M):
 
 # DRAM bytes (read + write) per launch from one ncu capture of the kernel as it
 # is now, keyed by (layer config, M, kernel); a kernel changed since its capture
-# has no entry (profiles/decode_gate_up_traffic_olmoe_m1.md holds the last capture).
+# has no entry.
 MEASURED_TRAFFIC = {}
 
 

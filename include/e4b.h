@@ -282,11 +282,19 @@ E4B_API e4b_status e4b_moe_expert_forward_path(const uint16_t* x, int64_t M, con
  * caller still owns x, router_logits, the stacks and out; nothing here calls
  * cudaMalloc, cudaFree or any allocating routine.
  *
- * The first call on each device looks up the device address of the array
- * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  All calls share the one array and it keeps the
- * last call's contents, so calls whose kernels overlap on the GPU (different
- * streams without ordering between them) race and give wrong results.
+ * The first call in each CUDA context looks up the device address of the
+ * array (cudaGetSymbolAddress) with that context current, and caches it under
+ * the context's unique id, so a context created after cudaDeviceReset gets a
+ * fresh lookup.  With lazy module loading (CUDA_MODULE_LOADING=LAZY, the
+ * default) the driver only materialises the library's module, and this
+ * static array with it, at that first lookup or at the first launch of any
+ * libe4b kernel: that is a device allocation made by the driver.  The promise
+ * of no allocation therefore holds from the second call on: make one eager
+ * call on each device (or context) during start-up, before any stream capture
+ * and outside the decode loop.  All calls share the one array and it keeps
+ * the last call's contents, so calls whose kernels overlap on the GPU
+ * (different streams without ordering between them) race and give wrong
+ * results.
  */
 E4B_API e4b_status e4b_moe_expert_forward_decode_noalloc(const uint16_t* x, int64_t M,
                                                          const float* router_logits, int k,

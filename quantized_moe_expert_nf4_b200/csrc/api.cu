@@ -191,6 +191,26 @@ cudaError_t device_info(DeviceInfo* out) {
 
 cudaError_t launch_lora_xa(const GemmArgs& a, cudaStream_t stream);
 
+e4b_status check_stack(const e4b_expert_stack* w, int k) {
+  if (!w) return fail(E4B_ERR_INVALID_ARGUMENT, "null expert stack");
+  if (w->E < 1 || w->E > 1024) return fail(E4B_ERR_UNSUPPORTED, "E must be in [1, 1024]");
+  if (w->H < 64 || w->H % 64 != 0) return fail(E4B_ERR_UNSUPPORTED, "H must be a positive multiple of 64");
+  if (w->I < 64 || w->I % 64 != 0) return fail(E4B_ERR_UNSUPPORTED, "I must be a positive multiple of 64");
+  if (k < 1 || k > w->E || k > 32) return fail(E4B_ERR_INVALID_ARGUMENT, "k must be in [1, min(E, 32)]");
+  if (!w->gu_packed || !w->gu_absmax || !w->dn_packed || !w->dn_absmax)
+    return fail(E4B_ERR_INVALID_ARGUMENT, "null packed stack pointer");
+  if ((w->lora_A == nullptr) != (w->lora_B == nullptr))
+    return fail(E4B_ERR_INVALID_ARGUMENT, "lora_A and lora_B must be both set or both NULL");
+  if (w->lora_A && (w->lora_r < 1 || w->lora_r > 16)) return fail(E4B_ERR_UNSUPPORTED, "LoRA rank must be in [1, 16]");
+  if (w->lora_A && (!aligned16(w->lora_A) || !aligned16(w->lora_B)))
+    return fail(E4B_ERR_INVALID_ARGUMENT, "lora_A and lora_B must be 16-byte aligned");
+  if (!aligned16(w->gu_packed) || !aligned16(w->dn_packed) || !aligned16(w->gu_absmax) || !aligned16(w->dn_absmax))
+    return fail(E4B_ERR_INVALID_ARGUMENT, "packed stacks and absmax must be 16-byte aligned");
+  return E4B_OK;
+}
+
+e4b_status check_sm100() { return check_device(); }
+
 }  // namespace e4b
 
 using namespace e4b;
@@ -391,24 +411,6 @@ e4b_status e4b_grouped_nf4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda, 
   cudaError_t err = launch_grouped_gemm(g, stream, &path);
   if (err != cudaSuccess) return cuda_fail(err, "grouped gemm launch");
   set_path(path);
-  return E4B_OK;
-}
-
-static e4b_status check_stack(const e4b_expert_stack* w, int k) {
-  if (!w) return fail(E4B_ERR_INVALID_ARGUMENT, "null expert stack");
-  if (w->E < 1 || w->E > 1024) return fail(E4B_ERR_UNSUPPORTED, "E must be in [1, 1024]");
-  if (w->H < 64 || w->H % 64 != 0) return fail(E4B_ERR_UNSUPPORTED, "H must be a positive multiple of 64");
-  if (w->I < 64 || w->I % 64 != 0) return fail(E4B_ERR_UNSUPPORTED, "I must be a positive multiple of 64");
-  if (k < 1 || k > w->E || k > 32) return fail(E4B_ERR_INVALID_ARGUMENT, "k must be in [1, min(E, 32)]");
-  if (!w->gu_packed || !w->gu_absmax || !w->dn_packed || !w->dn_absmax)
-    return fail(E4B_ERR_INVALID_ARGUMENT, "null packed stack pointer");
-  if ((w->lora_A == nullptr) != (w->lora_B == nullptr))
-    return fail(E4B_ERR_INVALID_ARGUMENT, "lora_A and lora_B must be both set or both NULL");
-  if (w->lora_A && (w->lora_r < 1 || w->lora_r > 16)) return fail(E4B_ERR_UNSUPPORTED, "LoRA rank must be in [1, 16]");
-  if (w->lora_A && (!aligned16(w->lora_A) || !aligned16(w->lora_B)))
-    return fail(E4B_ERR_INVALID_ARGUMENT, "lora_A and lora_B must be 16-byte aligned");
-  if (!aligned16(w->gu_packed) || !aligned16(w->dn_packed) || !aligned16(w->gu_absmax) || !aligned16(w->dn_absmax))
-    return fail(E4B_ERR_INVALID_ARGUMENT, "packed stacks and absmax must be 16-byte aligned");
   return E4B_OK;
 }
 

@@ -31,6 +31,11 @@ class LaunchScope {
 };
 void begin_call();  // resets the per-call launch counter
 
+// Host-side argument checks shared by the C-ABI entry points; on failure they
+// record the message (e4b_last_error) and return the status.
+e4b_status check_stack(const e4b_expert_stack* w, int k);  // stack pointers, shapes, alignment, LoRA rank, k
+e4b_status check_sm100();                                 // the current device is sm_100
+
 // The NF4 codebook as the library holds it (QLoRA table, ascending).
 extern const float kNf4Codebook[16];
 

@@ -9,8 +9,11 @@
 // statically sized device array that exists from the moment the library is
 // loaded on a GPU until the process exits.  The caller still passes x, the
 // router logits, the packed stacks and the output buffer.
+#include <cuda.h>
+
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include "e4b_internal.h"
 
@@ -24,25 +27,60 @@ constexpr size_t kNoAllocBytes = kNoAllocHBytes + 16 * 1024;  // + the error wor
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices] = {};
+// Device address of the scratch array in the current context.  The host-side
+// name of the array is not a device address.  The address belongs to the
+// module instance of one CUDA context: after cudaDeviceReset, or with another
+// context current on the same device, the module is loaded again and the
+// array may sit elsewhere, so the cache is keyed by the context's unique id
+// (cuCtxGetId), never by the device index alone.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
 
-// Device address of the scratch array on the current device, looked up once per
-// device.  The host-side name of the array is not a device address.
+struct ScratchEntry {
+  unsigned long long ctx_id;
+  void* addr;
+};
+
+std::mutex g_mu;
+std::vector<ScratchEntry> g_scratch;
+
+template <class Fn>
+Fn driver_fn(const char* name) {
+  void* ptr = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPointByVersion(name, &ptr, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(ptr);
+}
+
 cudaError_t scratch_address(void** out) {
-  int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
-  if (err != cudaSuccess) return err;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
+  static const CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  if (!get_current || !get_id) return cudaErrorNotSupported;
+  cudaError_t err = cudaSuccess;
+  void* p = nullptr;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+  if (!ctx) {
+    // No context on this thread yet: the runtime's symbol lookup makes the
+    // device's primary context current (and loads the module).
     err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (err != cudaSuccess) return err;
-    g_scratch_addr[dev] = p;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return cudaErrorDeviceUninitialized;
   }
-  *out = g_scratch_addr[dev];
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (const ScratchEntry& e : g_scratch)
+    if (e.ctx_id == id) {
+      *out = e.addr;
+      return cudaSuccess;
+    }
+  err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (err != cudaSuccess) return err;
+  g_scratch.push_back({id, p});
+  *out = p;
   return cudaSuccess;
 }
 
@@ -60,35 +98,22 @@ extern "C" e4b_status e4b_moe_expert_forward_decode_noalloc(const uint16_t* x, i
                                                             int k, int renormalize, const e4b_expert_stack* w,
                                                             uint16_t* out, e4b_stream stream) {
   begin_call();
-  if (!w) return nofail(E4B_ERR_INVALID_ARGUMENT, "null expert stack");
+  if (e4b_status st = check_stack(w, k); st != E4B_OK) return st;
   if (M < 1 || M > 8) return nofail(E4B_ERR_UNSUPPORTED, "the allocation-free forward takes 1 to 8 tokens");
-  if (k < 1 || k > 32 || k > w->E) return nofail(E4B_ERR_INVALID_ARGUMENT, "k must be in [1, min(E, 32)]");
-  if (w->E < 1 || w->H < 64 || w->H % 64 != 0 || w->I < 64 || w->I % 64 != 0)
-    return nofail(E4B_ERR_UNSUPPORTED, "E >= 1 and H, I positive multiples of 64 required");
   if (M * k * w->I > kNoAllocMaxHElems)
     return nofail(E4B_ERR_UNSUPPORTED, "M*k*I = " + std::to_string(M * k * w->I) +
                                            " exceeds the static scratch of the allocation-free forward (" +
                                            std::to_string(kNoAllocMaxHElems) + " activations)");
-  if (!x || !router_logits || !out || !w->gu_packed || !w->gu_absmax || !w->dn_packed || !w->dn_absmax)
-    return nofail(E4B_ERR_INVALID_ARGUMENT, "null pointer argument");
-  if ((w->lora_A == nullptr) != (w->lora_B == nullptr))
-    return nofail(E4B_ERR_INVALID_ARGUMENT, "lora_A and lora_B must be both set or both NULL");
-  if (w->lora_A && (w->lora_r < 1 || w->lora_r > 16)) return nofail(E4B_ERR_UNSUPPORTED, "LoRA rank must be in [1, 16]");
+  if (!x || !router_logits || !out) return nofail(E4B_ERR_INVALID_ARGUMENT, "null x, router_logits or out");
   auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
-  if (!a16(x) || !a16(out) || !a16(w->gu_packed) || !a16(w->dn_packed) || !a16(w->gu_absmax) || !a16(w->dn_absmax))
-    return nofail(E4B_ERR_INVALID_ARGUMENT, "x, out, packed stacks and absmax must be 16-byte aligned");
-  if (w->lora_A && (!a16(w->lora_A) || !a16(w->lora_B)))
-    return nofail(E4B_ERR_INVALID_ARGUMENT, "lora_A and lora_B must be 16-byte aligned");
-  DeviceInfo di;
-  cudaError_t err = device_info(&di);
-  if (err != cudaSuccess) return nofail(E4B_ERR_CUDA, std::string("device query: ") + cudaGetErrorString(err));
-  if (di.major != 10 || di.minor != 0) return nofail(E4B_ERR_UNSUPPORTED, "libe4b is built for sm_100a (B200)");
+  if (!a16(x) || !a16(out)) return nofail(E4B_ERR_INVALID_ARGUMENT, "x and out must be 16-byte aligned");
+  if (e4b_status st = check_sm100(); st != E4B_OK) return st;
   if (const std::string why = decode_unsupported_reason(M, w->E, k, w->H, w->I); !why.empty())
     return nofail(E4B_ERR_UNSUPPORTED, why);
   if (decode_workspace_bytes(M, w->E, k, w->H, w->I, w->lora_A ? w->lora_r : 0) > kNoAllocBytes)
     return nofail(E4B_ERR_UNSUPPORTED, "decode scratch layout exceeds the static array");
   void* scratch = nullptr;
-  err = scratch_address(&scratch);
+  cudaError_t err = scratch_address(&scratch);
   if (err != cudaSuccess)
     return nofail(E4B_ERR_CUDA, std::string("cudaGetSymbolAddress of the static scratch: ") + cudaGetErrorString(err));
   DecodeArgs a{x, M, router_logits, k, renormalize != 0, w, out, scratch};

@@ -156,3 +156,25 @@ def test_zero_row_gemm_needs_no_workspace(lib):
     st = lib.e4b_grouped_nf4_gemm(p, 1, 128, None, p, 2, 0, p, p, 128, 128, None, None, 0, 0.0, 0, p, 0, None, 0,
                                   None)
     assert st != 3 and b"workspace" not in lib.e4b_last_error()
+
+
+def test_noalloc_forward_rejections_on_the_host(lib):
+    """The allocation-free forward checks its arguments with the regular
+    forward's stack check, then its own token range, scratch limit, null and
+    alignment rules, all before any device query."""
+    p = ctypes.c_void_p(1 << 20)
+    bad = ctypes.c_void_p((1 << 20) + 2)
+    stk = e4b.ExpertStackC(1 << 20, 1 << 20, 1 << 20, 1 << 20, None, None, 0, 0.0, 8, 256, 128)
+    fn = lib.e4b_moe_expert_forward_decode_noalloc
+    assert fn(p, 1, p, 2, 1, None, p, None) == 1 and b"null expert stack" in lib.e4b_last_error()
+    assert fn(p, 0, p, 2, 1, ctypes.byref(stk), p, None) == 2 and b"1 to 8 tokens" in lib.e4b_last_error()
+    assert fn(p, 9, p, 2, 1, ctypes.byref(stk), p, None) == 2 and b"1 to 8 tokens" in lib.e4b_last_error()
+    assert fn(p, 1, p, 9, 1, ctypes.byref(stk), p, None) == 1 and b"k must be" in lib.e4b_last_error()
+    assert fn(None, 1, p, 2, 1, ctypes.byref(stk), p, None) == 1 and b"null x" in lib.e4b_last_error()
+    assert fn(p, 1, p, 2, 1, ctypes.byref(stk), bad, None) == 1 and b"16-byte aligned" in lib.e4b_last_error()
+    big = e4b.ExpertStackC(1 << 20, 1 << 20, 1 << 20, 1 << 20, None, None, 0, 0.0, 32, 128, 8192)
+    assert fn(p, 2, p, 32, 1, ctypes.byref(big), p, None) == 2 and b"static scratch" in lib.e4b_last_error()
+    lora = e4b.ExpertStackC(1 << 20, 1 << 20, 1 << 20, 1 << 20, (1 << 20) + 2, 1 << 20, 8, 16.0, 8, 256, 128)
+    assert fn(p, 1, p, 2, 1, ctypes.byref(lora), p, None) == 1 and b"lora_A and lora_B" in lib.e4b_last_error()
+    rank = e4b.ExpertStackC(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 17, 16.0, 8, 256, 128)
+    assert fn(p, 1, p, 2, 1, ctypes.byref(rank), p, None) == 2 and b"LoRA rank" in lib.e4b_last_error()

@@ -52,7 +52,12 @@ def _oracle_tokens(cfg, x, logits, tokens, check_gpu_layer=None, renormalize=Tru
         lb = workloads.bf16_bits_to_f32(workloads.lora_B(cfg)).astype(np.float64)
     st = moe.ExpertStack(gp, ga, dp, da, E, H, I, la, lb, workloads.lora_scale(cfg))
     xs = bf16_to_f64(x[torch.as_tensor(tokens, device=x.device)])
-    return moe.moe_forward_per_token(xs, ids, w, st)
+    if len(tokens) <= 16:
+        return moe.moe_forward_per_token(xs, ids, w, st)
+    # many tokens: the permuted form (equal to the per-token form to 1e-12, and it
+    # dequantises one expert at a time instead of caching every touched expert)
+    offsets, perm, inv = routing.permute(ids, E)
+    return moe.moe_forward_grouped(xs, ids, w, offsets, perm, inv, st)
 
 
 SMALL = [
@@ -89,11 +94,31 @@ def test_forward_full_size_sampled_tokens(name, M):
     layer = synthetic.make_device_layer(cfg)
     x, logits = synthetic.inputs(cfg, M)
     out, p = _forward(layer, x, logits)
-    tokens = np.unique(np.array([0, M - 1, M // 2, M // 3]))[:4]
+    # every token of a decode batch; four spread tokens of a prefill batch
+    tokens = np.arange(M) if M <= 8 else np.unique(np.array([0, M - 1, M // 2, M // 3]))[:4]
     ref = _oracle_tokens(cfg, x, logits, tokens, check_gpu_layer=layer)
     got = bf16_to_f64(out[torch.as_tensor(tokens, device="cuda")])
     assert_close_layer(got, ref, f"{name} M={M} {p} tokens {tokens.tolist()}")
     assert torch.isfinite(out.float()).all()
+
+
+def test_forward_prefill_many_tokens_across_the_batch():
+    """256 tokens spread over an OLMoE-shaped prefill batch of 2048 (16384
+    routed rows, every expert touched): the tensor-core GEMMs' late tiles,
+    each group's ragged tail and the combine of tokens far apart in the
+    batch all reach the comparison."""
+    require_gpu()
+    cfg = workloads.CONFIGS["olmoe"]
+    M = 2048
+    layer = synthetic.make_device_layer(cfg)
+    x, logits = synthetic.inputs(cfg, M)
+    out, p = _forward(layer, x, logits)
+    assert p == "forward.grouped"
+    tokens = np.unique(np.linspace(0, M - 1, 256).round().astype(np.int64))
+    assert tokens.size == 256
+    ref = _oracle_tokens(cfg, x, logits, tokens)
+    got = bf16_to_f64(out[torch.as_tensor(tokens, device="cuda")])
+    assert_close_layer(got, ref, f"olmoe M={M} {p} 256 tokens")
 
 
 DECODE = [

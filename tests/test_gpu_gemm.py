@@ -217,3 +217,75 @@ def test_grouped_gemm_tensor_core_lora(monkeypatch, shape, r, epi):
         assert fro <= tol and mx <= 2 * tol
         # the delta matters
         assert rel_errors(_oracle(dict(c, r=0), epi, use_ridx=use_ridx), ref)[0] > 1e-2
+
+
+# The persistent regime of the tensor-core kernel: more than two tiles per CTA
+# (the grid is min(tiles, SMs) and each CTA walks tiles with a stride of the
+# grid), so accumulator hand-offs, barrier phases and ring slots carry over
+# from tile to tile.  Group sizes are Zipf-like with empty groups, one-row
+# groups and groups one row short of / past a 256-row tile; every output
+# element is compared with the float64 oracle.
+MULTI_COUNTS = [2900, 1500, 0, 1, 1000, 700, 0, 513, 256, 255, 1, 600, 300, 0, 900, 75]
+MULTI_N, MULTI_K = 2048, 1024
+_multi_cache = {}
+
+
+def _multi_case(lora_r=0):
+    key = ("case", lora_r)
+    if key not in _multi_cache:
+        _multi_cache[key] = _case(len(MULTI_COUNTS), MULTI_N, MULTI_K, MULTI_COUNTS, 4096, seed=77 + lora_r,
+                                  lora_r=lora_r)
+    return _multi_cache[key]
+
+
+def _multi_oracle(c, epi, lora_r):
+    key = ("ref", lora_r, epi)
+    if key not in _multi_cache:
+        _multi_cache[key] = _oracle(c, epi)
+    return _multi_cache[key]
+
+
+def _tc_tile_count(counts, n_out_cols, wrows, bn):
+    n_tiles = -(-n_out_cols // wrows)
+    return sum(-(-c // bn) for c in counts) * n_tiles
+
+
+@pytest.mark.parametrize("shape", TC_SHAPES)
+@pytest.mark.parametrize("epi", [e4b.E4B_EPI_NONE, e4b.E4B_EPI_SWIGLU])
+def test_grouped_gemm_tensor_core_persistent_full_output(monkeypatch, shape, epi):
+    require_gpu()
+    monkeypatch.setenv("E4B_GEMM", "tc")
+    monkeypatch.setenv("E4B_TC_SHAPE", shape)
+    swiglu = epi == e4b.E4B_EPI_SWIGLU
+    eff_shape = "wide" if (shape == "narrow" and swiglu) else shape
+    bn = 128 if eff_shape == "double" else 256
+    wrows = 128 if (swiglu or eff_shape == "narrow") else 256
+    tiles = _tc_tile_count(MULTI_COUNTS, MULTI_N // 2 if swiglu else MULTI_N, wrows, bn)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert tiles > 2 * sms, f"{tiles} tiles do not give every CTA a third tile"
+    c = _multi_case()
+    got, path = _run_gpu(c, epi, torch.float32)
+    assert path.startswith("gemm.tc"), path
+    ref = _multi_oracle(c, epi, 0)
+    fro, mx = rel_errors(got, ref)
+    tol = gemm_tolerance(path, epi, torch.float32)
+    print(f"[parity] tc persistent {shape} epi {epi} tiles {tiles}: rel_fro={fro:.2e} max={mx:.2e}")
+    assert fro <= tol and mx <= 2 * tol
+    # and per routed row: a fault confined to a few late tiles must not hide in the norm
+    row_err = np.linalg.norm(got - ref, axis=1) / np.maximum(np.linalg.norm(ref, axis=1), 1e-30)
+    assert float(row_err.max()) <= 4 * tol, f"worst row {int(row_err.argmax())}: {row_err.max():.2e}"
+
+
+def test_grouped_gemm_tensor_core_persistent_lora(monkeypatch):
+    require_gpu()
+    monkeypatch.setenv("E4B_GEMM", "tc")
+    c = _multi_case(lora_r=8)
+    got, path = _run_gpu(c, e4b.E4B_EPI_SWIGLU, torch.float32)
+    assert path.startswith("gemm.tc"), path
+    ref = _multi_oracle(c, e4b.E4B_EPI_SWIGLU, 8)
+    fro, mx = rel_errors(got, ref)
+    tol = gemm_tolerance(path, e4b.E4B_EPI_SWIGLU, torch.float32)
+    print(f"[parity] tc persistent lora: rel_fro={fro:.2e} max={mx:.2e}")
+    assert fro <= tol and mx <= 2 * tol
+    row_err = np.linalg.norm(got - ref, axis=1) / np.maximum(np.linalg.norm(ref, axis=1), 1e-30)
+    assert float(row_err.max()) <= 4 * tol
