@@ -451,6 +451,15 @@ MEASURED_TRAFFIC = {}
 def dominant_roofline(cfg, M, kt, touched_avg, peaks, long_region):
     name, (avg_ms, n) = max(kt.items(), key=lambda kv: kv[1][0] * kv[1][1])
     S = M * cfg.k
+    if name.startswith("decode.fused"):
+        # HBM-bound: the whole layer in one launch, so its algorithmic bytes are
+        # the step's (both stacks of the touched experts, x, out, the router logits)
+        alg = step_work(cfg, M, touched_avg)[1]
+        achieved = alg / (avg_ms * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        return name, {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                      "traffic": MEASURED_TRAFFIC.get((cfg.name, M, name)), "kernel": name, "avg_us": avg_ms * 1e3,
+                      "algorithmic_bytes_per_launch": alg, "peak_source": peaks["source"] + " hbm_gbs"}
     if name.startswith("decode.gate_up") or name.startswith("decode.down"):
         # HBM-bound: the projection's packed bytes + absmax of the touched experts
         per_expert = gate_up_expert_bytes(cfg) if "gate_up" in name else cfg.H * cfg.I * (0.5 + 4.0 / 64)

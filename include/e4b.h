@@ -105,6 +105,7 @@ E4B_API const char* e4b_last_path(void);
 #define E4B_KERNEL_ERR_WAIT_FULL 1  /* a consumer waited in vain for its input tile */
 #define E4B_KERNEL_ERR_WAIT_EMPTY 2 /* a producer waited in vain for a free stage */
 #define E4B_KERNEL_ERR_WAIT_DRAIN 3 /* a CTA gave up waiting for its own copies */
+#define E4B_KERNEL_ERR_GRID_BARRIER 4 /* a CTA of the decode kernel gave up waiting for the others */
 
 /* Reads the error word of `workspace` into *code.  Synchronises the device
  * first (a diagnostic call, not for the hot path or a graph capture).  This
@@ -256,10 +257,16 @@ E4B_API e4b_status e4b_moe_expert_forward(const uint16_t* x, int64_t M, const fl
                                   uint16_t* out, void* workspace, size_t workspace_bytes,
                                   e4b_stream stream);
 /* Same, with the implementation chosen explicitly (tests and benchmarks).
- * E4B_PATH_AUTO takes the decode kernels when they can run the shape -- 1 <= M <= 8,
- * k <= 32, E <= 512, H <= 4096 and their shared-memory plan fits -- and the grouped
- * path otherwise.  E4B_PATH_DECODE on any other shape returns E4B_ERR_UNSUPPORTED
- * and e4b_last_error() names the limit. */
+ * E4B_PATH_AUTO takes the decode kernel when it can run the shape -- 1 <= M <= 8,
+ * k <= 32, E <= 512, H <= 4096, I <= 4096 and its shared-memory plan fits -- and
+ * the grouped path otherwise.  E4B_PATH_DECODE on any other shape returns
+ * E4B_ERR_UNSUPPORTED and e4b_last_error() names the limit.
+ * The decode path is one cooperative launch of one CTA per SM (at most 1024
+ * CTAs): it needs the whole grid resident at once, so a launch that cannot get
+ * every SM it asks for fails with E4B_ERR_CUDA instead of waiting.  Its CTAs
+ * meet at a grid barrier whose slots live in the workspace and are tagged with
+ * the launch's grid id: a workspace needs no initialisation for it, and the
+ * barrier keeps no state from one call to the next. */
 E4B_API e4b_status e4b_moe_expert_forward_path(const uint16_t* x, int64_t M, const float* router_logits,
                                        int k, int renormalize, const e4b_expert_stack* w,
                                        uint16_t* out, void* workspace, size_t workspace_bytes,
@@ -273,9 +280,9 @@ E4B_API e4b_status e4b_moe_expert_forward_path(const uint16_t* x, int64_t M, con
  * other) once their decode loop is running.
  *
  * Computes exactly what e4b_moe_expert_forward() computes for 1 <= M <= 8
- * tokens, with the decode kernels, but takes no workspace: its scratch (the
- * SwiGLU activations of the routed slots, M*k*I bf16 values, plus the routing
- * result the first decode kernel hands to the second) lives in one statically
+ * tokens, with the decode kernel, but takes no workspace: its scratch (the
+ * SwiGLU activations of the routed slots, M*k*I bf16 values, plus one 64-bit
+ * slot per CTA for the kernel's grid barrier) lives in one statically
  * sized device array of the library, 528 KiB, which every GPU that loads the
  * library holds until the process exits.  Requires M*k*I <= 262144 (for example M = 8, k = 8,
  * I <= 4096); larger shapes return E4B_ERR_UNSUPPORTED with a message.  The

@@ -105,7 +105,8 @@ e4b_status check_workspace(const char* what, size_t need, const void* workspace,
 }
 
 static_assert(kErrNone == E4B_KERNEL_ERR_NONE && kErrWaitFull == E4B_KERNEL_ERR_WAIT_FULL &&
-                  kErrWaitEmpty == E4B_KERNEL_ERR_WAIT_EMPTY && kErrWaitDrain == E4B_KERNEL_ERR_WAIT_DRAIN,
+                  kErrWaitEmpty == E4B_KERNEL_ERR_WAIT_EMPTY && kErrWaitDrain == E4B_KERNEL_ERR_WAIT_DRAIN &&
+                  kErrGridBarrier == E4B_KERNEL_ERR_GRID_BARRIER,
               "device error codes match the header");
 
 e4b_status check_device() {

@@ -9,7 +9,7 @@
 namespace e4b {
 
 // Error codes written to the workspace error word when a bounded wait gives up.
-enum : int { kErrNone = 0, kErrWaitFull = 1, kErrWaitEmpty = 2, kErrWaitDrain = 3 };
+enum : int { kErrNone = 0, kErrWaitFull = 1, kErrWaitEmpty = 2, kErrWaitDrain = 3, kErrGridBarrier = 4 };
 
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 

@@ -1,31 +1,43 @@
-// Fused small-M (decode) forward of the NF4 expert layer: two kernels, no host sync.
+// Fused small-M (decode) forward of the NF4 expert layer: one kernel, no host sync.
 //
 // The pages' inference fast path for single-token decode is a fused 4-bit GEMV
 // over the routed experts (experts4bit-qlora 0.22.0, "Inference: serve the
 // fine-tune you just made"), and decode is launch-bound at ~89 launches per
-// layer step ("CUDA-graph decode capture").  Here the whole layer is two
-// kernels chained with programmatic dependent launch:
+// layer step ("CUDA-graph decode capture").  Here the whole layer is ONE
+// cooperative launch of one CTA per SM:
 //
-//   kernel A  routing (every CTA, redundantly: M <= 8 tokens), then the gate
-//             and up rows of every touched expert in items of 8 gate + 8 up
-//             rows over all of K = H -> SiLU(gate) * up (+ LoRA delta) -> h
-//             (bf16, [M*k, I], slot order).  It also prefetches the touched
-//             experts' down rows into L2, so that HBM keeps streaming while the
-//             second kernel starts.
-//   kernel B  the routing kernel A published, then for every block
-//             of 16 output rows of H the down rows of every touched expert, with
-//             the routing weights folded into the per-block scale, so the
-//             combine happens inside the CTA in a fixed order (deterministic).
+//   prologue  every CTA routes the M <= 8 tokens (top-k + weights) and lists
+//             the touched experts (ascending id); only those are read.
+//   phase 1   gate_up: the CTA's contiguous run of items (8 gate + 8 up rows
+//             of one touched expert over all of K = H) -> SiLU(gate) * up
+//             (+ LoRA delta) -> h (bf16, [M*k, I], slot order) in the workspace.
+//   barrier   grid-wide: every CTA's h is written.
+//   phase 2   down: for each block of 16 output rows the CTA owns, the down
+//             rows of every touched expert times h, the routing weights
+//             folded in per token column -> out (bf16).  The combine over the
+//             experts of a token happens inside the CTA in a fixed order, so
+//             the result is deterministic and needs no extra kernel.
 //
-// Only experts that some token selected are read.  Both kernels are split-K
-// GEMVs on warp tensor cores: each CTA owns a contiguous run of items, its 16
-// warps split K in spans of two absmax blocks (128 k), and each lane loads its
-// 16-byte slice of a span of the packed rows straight from HBM into the
-// registers of an mma.sync m16n8k16 fragment (weight rows = MMA rows, the <= 8
-// tokens = the 8 MMA columns), several items ahead.  Nibbles become bf16
-// through a per-lane replicated byte -> bf16x2 codebook table in shared memory
-// (lane l reads only bank l), scaled by the block's bf16 absmax before the
-// MMA.  One block barrier per batch gathers the 16 warps' partials.
+// One producer warp streams the packed rows and their fp32 absmax with bulk
+// asynchronous copies (one per row, mbarrier transaction counts) through a
+// ring of shared-memory stages: first phase 1's items, then -- without waiting
+// for the barrier, since weights do not depend on h -- phase 2's stages, so
+// HBM keeps streaming the down rows while phase 1 computes and the barrier
+// resolves.  Sixteen math warps decode and multiply: nibbles become bf16 pairs
+// through a per-lane replicated byte -> bf16x2 codebook table (lane l reads
+// only bank l) and feed mma.sync m16n8k16 with the weight rows as MMA rows and
+// the <= 8 tokens as the 8 MMA columns.  Each MMA stays inside one 64-element
+// absmax block, so the block's fp32 absmax scales the products (no rounding of
+// the scale).  Rows are staged with a stride of 32 mod 128 bytes so that the
+// fragment loads are conflict-free.
+//
+// The grid barrier is stateless: each CTA publishes the launch's %gridid (a
+// number the hardware gives every grid launch in a context) in its own slot of
+// the workspace, and waits until every slot holds that number, so a workspace
+// needs no initialisation and no reset.  Every wait is bounded; a wait that
+// gives up records an error code in the workspace's error word, marks the CTA
+// aborted (later waits return at once, the results are unspecified) and the
+// kernel still runs to its end.
 #include <algorithm>
 #include <string>
 
@@ -38,15 +50,23 @@ namespace e4b {
 namespace {
 
 constexpr int kMaxM = 8;
-constexpr int kWarps = 16;
+constexpr int kMath = 16;               // math warps
+constexpr int kProducer = kMath;        // warp issuing the bulk copies
+constexpr int kWarps = kMath + 1;
 constexpr int kThreads = kWarps * 32;
-constexpr int kMaxSlots = 8;               // (item, span) load slots per warp per batch in kernel A
-constexpr int kPairSlots = 2;              // (expert, span) load slots per warp per batch in kernel B
-constexpr int kMaxKBW = 2;                 // spans (2 k-blocks) per warp per item: H <= 128 * 16 * 2 = 4096
-constexpr unsigned long long kPrefetchLimit = 64ull << 20;
-constexpr uint32_t kPrefetchChunk = 32 * 1024;
+constexpr int kGroups = 2;              // phase 1: items alternate between two groups of math warps
+constexpr int kGW = kMath / kGroups;    // warps per group
+constexpr int kMaxSPW = 4;              // spans (128 k) per warp of an item: H <= 8 * 4 * 128 = 4096
+constexpr int kMaxPPW = 4;              // (expert, k-block) pairs per warp of a down stage
+constexpr int kMaxKBI = kMath * kMaxPPW;  // k-blocks of a down row: I <= 4096
+constexpr int kMaxGrid = 1024;          // barrier slots in the workspace
+constexpr int kMaxStages = 32;
+constexpr uint32_t kLutBytes = 256 * 32 * 4;
+constexpr uint32_t kRedBytes = kGroups * 2 * kGW * 32 * 16;  // phase 1: [group][parity][warp][lane] float4
+constexpr int kBarGroup0 = 1;           // named barriers: 1, 2 (groups), 3 (all math warps)
+constexpr int kBarMath = 3;
 
-struct DecodeParams {
+struct FusedParams {
   const uint16_t* x;
   const float* logits;
   int M, k, E, H, I;
@@ -59,40 +79,50 @@ struct DecodeParams {
   const uint16_t* lora_B;
   int r;
   float lora_scale;
-  uint16_t* h;    // [S, I] bf16 (slot order)
-  uint16_t* out;  // [M, H] bf16
-  // Routing result of the gate_up kernel for the down kernel: [nU, pad x3],
-  // touched [S], slotmap [S * kMaxM], weights [S] (as float bits).
-  int* meta;
-};
-
-struct Layout {
-  uint32_t lut, xs, red, ids, w, uidx, touched, slotmap, xa, total;
+  uint16_t* h;                 // [S, I] bf16 (slot order)
+  uint16_t* out;               // [M, H] bf16
+  int* err;                    // error word
+  unsigned long long* flags;   // [gridDim.x] barrier slots
+  int stages;                  // ring depth (even)
+  int dpe;                     // down experts per phase-2 stage
 };
 
 __host__ __device__ inline uint32_t al(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
-// Spans of 128 k (2 absmax blocks, 64 packed bytes of a row) per warp per item.
-__host__ __device__ inline int kbw_of(int H) { return ((H / 64 + 1) / 2 + kWarps - 1) / kWarps; }
+// Shared-memory stride of a staged packed row of K elements: K/2 bytes padded
+// to 32 mod 128, so the 8 rows of a fragment load fall on distinct banks.
+__host__ __device__ inline uint32_t row_stride(int K) {
+  const uint32_t b = static_cast<uint32_t>(K / 2);
+  return b + (160u - b % 128u) % 128u;
+}
 
-// (item, span) load slots per warp per batch of kernel A: eight for one token
-// with one span per warp (a CTA's whole share in one batch; measured faster at
-// M = 1), four otherwise (more tokens need the registers for x; measured
-// faster at M = 4 and 8).
-__host__ __device__ inline int slots_for(int M, int H) { return (M == 1 && kbw_of(H) == 1) ? 8 : 4; }
+// absmax rows: copied one by one when a row is a 16-byte multiple (KB % 4 ==
+// 0), with a stride of 4 mod 8 floats; otherwise as chunks of 8 contiguous
+// rows (stride KB, odd or 2 mod 4: still distinct banks for 8 rows).
+__host__ __device__ inline bool am_by_rows(int KB) { return KB % 4 == 0; }
+__host__ __device__ inline uint32_t am_stride(int KB) {
+  return static_cast<uint32_t>(am_by_rows(KB) ? (KB % 8 == 4 ? KB : KB + 4) : KB);
+}
 
-// Shared-memory carve of kernel A (gate_up) or B (down).
-__host__ __device__ inline Layout make_layout(bool is_a, int M, int k, int E, int H, int r) {
-  Layout L;
+// A block of 16 staged rows of K elements with their absmax: bytes and the
+// absmax offset inside it.
+__host__ __device__ inline uint32_t rows16_am_off(int K) { return 16 * row_stride(K); }
+__host__ __device__ inline uint32_t rows16_bytes(int K) {
+  return rows16_am_off(K) + al(16 * am_stride(K / 64) * 4, 16);
+}
+
+struct Smem {
+  uint32_t lut, red, ids, w, uidx, touched, slotmap, xa, bars, ring, total;
+};
+
+__host__ __device__ inline Smem make_smem(int M, int k, int E, int r, int stages, uint32_t slot) {
+  Smem L;
+  const int S = M * k;
   uint32_t o = 0;
   L.lut = o;
-  o = al(o + 256 * 32 * 4, 16);
-  L.xs = o;
-  if (is_a) o = al(o + M * (2 * H + 16), 16);
+  o += kLutBytes;
   L.red = o;
-  const int items = is_a ? slots_for(M, H) : 1;  // partial sums of the items of a batch (A), 1 row block (B)
-  o = al(o + items * kWarps * 32 * 16, 16);
-  const int S = M * k;
+  o += kRedBytes;
   L.ids = o;
   o = al(o + S * 4, 16);
   L.w = o;
@@ -104,8 +134,11 @@ __host__ __device__ inline Layout make_layout(bool is_a, int M, int k, int E, in
   L.slotmap = o;
   o = al(o + S * kMaxM * 4, 16);
   L.xa = o;
-  if (is_a && r > 0) o = al(o + S * r * 4, 16);
-  L.total = o;
+  if (r > 0) o = al(o + S * r * 4, 16);
+  L.bars = o;
+  o = al(o + 2 * stages * 8, 16);
+  L.ring = al(o, 128);
+  L.total = L.ring + static_cast<uint32_t>(stages) * slot;
   return L;
 }
 
@@ -118,39 +151,78 @@ __device__ __forceinline__ void mma_16816(float c[4], uint32_t a0, uint32_t a1, 
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint4 ld_stream_u4(const uint8_t* p) {
-  return __ldcs(reinterpret_cast<const uint4*>(p));
+__device__ __forceinline__ void named_bar(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// One span (128 k = 2 absmax blocks) of a 16-row tile, accumulated into c.
-// Thread (g, t) owns physical k [32t, 32t+32) of the span -- 16 packed bytes of
-// row g (r0) and of row g+8 (r1), all inside k-block t/2 -- and the matching 32
-// bf16 of its token column g (x).  Each byte's codebook pair is scaled by its
-// row's bf16(absmax) before the MMA (the block scale differs between threads of
-// one MMA, so it cannot be applied to the product).  MMA j takes bytes 2j and
-// 2j+1 of each row; K is permuted identically on both operands.
-__device__ __forceinline__ void span_mma(const uint32_t* __restrict__ lut_lane, uint4 r0, uint4 r1, float a0,
-                                         float a1, const uint4 x[4], float c[4]) {
-  const __nv_bfloat162 s0 = __float2bfloat162_rn(a0), s1 = __float2bfloat162_rn(a1);
-  const uint32_t w0[4] = {r0.x, r0.y, r0.z, r0.w}, w1[4] = {r1.x, r1.y, r1.z, r1.w};
-  const uint32_t xw[16] = {x[0].x, x[0].y, x[0].z, x[0].w, x[1].x, x[1].y, x[1].z, x[1].w,
-                           x[2].x, x[2].y, x[2].z, x[2].w, x[3].x, x[3].y, x[3].z, x[3].w};
-  auto pair = [&](uint32_t word, int byte, __nv_bfloat162 sc) {
-    uint32_t v = lut_lane[((word >> (8 * byte)) & 0xffu) << 5];
-    __nv_bfloat162 h2 = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&v), sc);
-    return *reinterpret_cast<uint32_t*>(&h2);
-  };
+__device__ __forceinline__ void mbar_arrive_cnt(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+// Bulk asynchronous copy global -> this CTA's shared memory, completing on `bar`
+// (both addresses 16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(smem_dst)),
+               "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ uint2 lds64(const unsigned char* p) { return *reinterpret_cast<const uint2*>(p); }
+
+__device__ __forceinline__ unsigned long long grid_id() {
+  unsigned long long v;
+  asm volatile("mov.u64 %0, %%gridid;" : "=l"(v));
+  return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Bounded wait on a ring barrier.  Once any wait of the CTA has given up
+// (*abort set), every later wait returns false at once.
+__device__ __forceinline__ bool ring_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* err, int code) {
+  if (mbar_try_wait(bar, parity)) return true;
+  if (*abort) return false;
+  const unsigned long long t0 = global_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort) return false;
+    if (global_ns() - t0 > kWaitLimitNs) {
+      *abort = 1;
+      record_error(err, code);
+      return false;
+    }
+  }
+  return true;
+}
+
+// The four MMAs of one 64-element k-block of a 16-row tile, into d (zeroed by
+// the caller).  Thread (g, t) holds packed bytes [8t, 8t+8) of the block for
+// row g (w0) and row g+8 (w1) -- elements 16t .. 16t+15 -- and the matching 16
+// bf16 of its token column g (xw, 8 words).  MMA j takes bytes 2j, 2j+1: their
+// bf16 pairs are the A fragment (row g / g+8, k slots 2t..2t+1 and 2t+8..2t+9)
+// and x words 2j, 2j+1 the B fragment, so both operands see the same physical
+// k for every slot.
+__device__ __forceinline__ void block_mma(const uint32_t* __restrict__ lut_lane, uint2 w0, uint2 w1,
+                                          const uint32_t* xw, float d[4]) {
+  auto pair = [&](uint32_t word, int byte) { return lut_lane[((word >> (8 * byte)) & 0xffu) << 5]; };
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t wa = (j < 2) ? w0.x : w0.y, wb = (j < 2) ? w1.x : w1.y;
     const int b = 2 * (j & 1);
-    const uint32_t wa = w0[j >> 1], wb = w1[j >> 1];
-    mma_16816(c, pair(wa, b, s0), pair(wb, b, s1), pair(wa, b + 1, s0), pair(wb, b + 1, s1), xw[2 * j],
-              xw[2 * j + 1]);
+    mma_16816(d, pair(wa, b), pair(wb, b), pair(wa, b + 1), pair(wb, b + 1), xw[2 * j], xw[2 * j + 1]);
   }
 }
 
 // Top-k of token `t` by the calling warp, with the key array sized for E.
-__device__ __forceinline__ void route_one(const DecodeParams& p, int t, int* ids_s, float* w_s) {
+__device__ __forceinline__ void route_one(const FusedParams& p, int t, int* ids_s, float* w_s) {
   const int maxj = (p.E + 31) / 32;
   if (maxj <= 1) route_token<1>(p.logits, t, p.E, p.k, p.renorm != 0, ids_s, w_s);
   else if (maxj <= 2) route_token<2>(p.logits, t, p.E, p.k, p.renorm != 0, ids_s, w_s);
@@ -159,39 +231,24 @@ __device__ __forceinline__ void route_one(const DecodeParams& p, int t, int* ids
   else route_token<16>(p.logits, t, p.E, p.k, p.renorm != 0, ids_s, w_s);
 }
 
-// Byte -> bf16x2 codebook pairs, replicated per lane (entry b of lane l at
-// b * 32 + l), written by the warps [w0, kWarps) of the block.
-__device__ __forceinline__ void fill_lut_warps(uint32_t* lut, int w0) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (warp < w0) return;
-  const float cbl = kNf4CodebookDev[lane & 15];
-  for (int b = warp - w0; b < 256; b += kWarps - w0) {
-    const float hi = __shfl_sync(0xffffffffu, cbl, b >> 4);
-    const float lo = __shfl_sync(0xffffffffu, cbl, b & 15);
-    lut[b * 32 + lane] = pack_bf16x2(hi, lo);
-  }
-}
-
-// Prologue shared by both kernels: warps < M route one token each while the
-// other warps build the codebook table (and, in kernel A, stage x).  Then the
+// Prologue: warps < M route one token each while the other warps build the
+// byte -> bf16x2 codebook table (entry b of lane l at b * 32 + l: low half the
+// high nibble's value, i.e. element 2i, high half element 2i+1).  Then the
 // touched experts (ascending id) and slotmap[u][t] = slot of token t in expert
-// touched[u] (or -1) are built.
-__device__ void decode_prologue(const DecodeParams& p, uint32_t* lut, uint16_t* xs, int xstride, int* ids_s,
-                                float* w_s, int* uidx, int* touched, int* slotmap, int* nU_out) {
+// touched[u] (or -1).
+__device__ void prologue(const FusedParams& p, uint32_t* lut, int* ids_s, float* w_s, int* uidx, int* touched,
+                         int* slotmap, int* nU_out) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int S = p.M * p.k;
   for (int e = tid; e < p.E; e += blockDim.x) uidx[e] = -1;
   if (warp < p.M) {
     route_one(p, warp, ids_s, w_s);
   } else {
-    fill_lut_warps(lut, p.M);
-    if (xs) {
-      const int nthr = (kWarps - p.M) * 32, me = tid - p.M * 32;
-      for (int i = me; i < p.M * (p.H / 8); i += nthr) {
-        const int t = i / (p.H / 8), c = i % (p.H / 8);
-        reinterpret_cast<uint4*>(xs + t * xstride)[c] =
-            reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(t) * p.H)[c];
-      }
+    const float cbl = kNf4CodebookDev[lane & 15];
+    for (int b = warp - p.M; b < 256; b += kWarps - p.M) {
+      const float hi = __shfl_sync(0xffffffffu, cbl, b >> 4);
+      const float lo = __shfl_sync(0xffffffffu, cbl, b & 15);
+      lut[b * 32 + lane] = pack_bf16x2(hi, lo);
     }
   }
   __syncthreads();
@@ -220,31 +277,42 @@ __device__ void decode_prologue(const DecodeParams& p, uint32_t* lut, uint16_t* 
   __syncthreads();
 }
 
-// L2 prefetch of the gate and up rows (and their absmax) of items [a, b),
-// one thread per item.
-__device__ __forceinline__ void prefetch_items(const DecodeParams& p, const int* touched, int a, int b) {
-  const int i = a + static_cast<int>(threadIdx.x);
-  if (i >= b) return;
-  const int ipe = p.I / 8;
-  const int u = i / ipe, rb = i % ipe;
-  const int64_t grow = static_cast<int64_t>(touched[u]) * 2 * p.I + rb * 8;
-  const int64_t row_bytes = p.H / 2, kb = p.H / 64;
-  prefetch_l2(p.gu_packed + grow * row_bytes, static_cast<uint32_t>(8 * row_bytes));
-  prefetch_l2(p.gu_packed + (grow + p.I) * row_bytes, static_cast<uint32_t>(8 * row_bytes));
-  prefetch_l2(p.gu_absmax + grow * kb, static_cast<uint32_t>(8 * kb * 4));
-  prefetch_l2(p.gu_absmax + (grow + p.I) * kb, static_cast<uint32_t>(8 * kb * 4));
+// Copies of 16 rows (rows [0, 8) from row_a, [8, 16) from row_b) of a packed
+// matrix with K columns, and their absmax, into a staged block.  Run by the
+// whole producer warp.
+__device__ __forceinline__ void copy_rows16(unsigned char* dst, uint64_t* full, const uint8_t* packed,
+                                            const float* absmax, int K, int64_t row_a, int64_t row_b) {
+  const int lane = threadIdx.x & 31;
+  const int KB = K / 64;
+  const uint32_t rowb = static_cast<uint32_t>(K / 2), ps = row_stride(K), sa = am_stride(KB);
+  unsigned char* am = dst + rows16_am_off(K);
+  if (lane < 16) {
+    const int64_t row = (lane < 8 ? row_a : row_b) + (lane & 7);
+    bulk_g2s(dst + lane * ps, packed + row * rowb, rowb, full);
+  } else if (am_by_rows(KB)) {
+    const int i = lane - 16;
+    const int64_t row = (i < 8 ? row_a : row_b) + (i & 7);
+    bulk_g2s(am + i * sa * 4, absmax + row * KB, static_cast<uint32_t>(KB * 4), full);
+  } else if (lane < 18) {
+    const int i = lane - 16;
+    bulk_g2s(am + i * 8 * sa * 4, absmax + (i == 0 ? row_a : row_b) * KB, static_cast<uint32_t>(8 * KB * 4), full);
+  }
 }
 
 // ---------------------------------------------------------------------------
-// Kernel A: gate_up + SwiGLU (+ LoRA delta) -> h.  KBW = k-blocks per warp per item.
-template <int KBW, int SLOTS>
-__global__ void __launch_bounds__(kThreads, 1) decode_gate_up_kernel(DecodeParams p) {
-  static_assert(SLOTS <= kMaxSlots, "load slots");
-  constexpr int IB = SLOTS / KBW;  // items per batch
-  extern __shared__ __align__(16) unsigned char smem[];
-  const Layout L = make_layout(true, p.M, p.k, p.E, p.H, p.r);
+// SPW: spans (two k-blocks) per math warp of a phase-1 item; PPW: (expert,
+// k-block) pairs per math warp of a phase-2 stage.
+template <int SPW, int PPW>
+__global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int H = p.H, I = p.I, KB = H / 64, KBI = I / 64;
+  const int RS = p.stages, DPE = p.dpe;
+  const uint32_t ps_gu = row_stride(H), sa_gu = am_stride(KB), am_gu = rows16_am_off(H);
+  const uint32_t ps_dn = row_stride(I), sa_dn = am_stride(KBI), am_dn = rows16_am_off(I);
+  const uint32_t exp_dn = rows16_bytes(I);
+  const uint32_t slot = al(max(rows16_bytes(H), static_cast<uint32_t>(DPE) * exp_dn), 128);
+  const Smem L = make_smem(p.M, p.k, p.E, p.r, RS, slot);
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L.lut);
-  uint16_t* xs = reinterpret_cast<uint16_t*>(smem + L.xs);
   float4* red = reinterpret_cast<float4*>(smem + L.red);
   int* ids_s = reinterpret_cast<int*>(smem + L.ids);
   float* w_s = reinterpret_cast<float*>(smem + L.w);
@@ -252,71 +320,93 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gate_up_kernel(DecodeParam
   int* touched = reinterpret_cast<int*>(smem + L.touched);
   int* slotmap = reinterpret_cast<int*>(smem + L.slotmap);
   float* xa = reinterpret_cast<float*>(smem + L.xa);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);  // stage landed
+  uint64_t* empty = full + RS;                                   // stage consumed (16 arrivals)
+  unsigned char* ring = smem + L.ring;
   __shared__ int nU_s;
+  __shared__ volatile int abort_s;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int H = p.H, I = p.I, KB = H / 64;
-  const int xstride = H + 8;  // bf16 elements (2H + 16 bytes: conflict-free 16-byte reads)
-
-  pdl_wait();               // the inputs of this call are final
-  pdl_launch_dependents();  // the down kernel may launch and run its prologue
-  decode_prologue(p, lut, xs, xstride, ids_s, w_s, uidx, touched, slotmap, &nU_s);
-  const int nU = nU_s;
-  if (blockIdx.x == 0) {
-    // Every CTA routed identically; one publishes the result for the down kernel.
-    const int S = p.M * p.k;
-    int* m_touched = p.meta + 4;
-    int* m_slotmap = m_touched + S;
-    float* m_w = reinterpret_cast<float*>(m_slotmap + S * kMaxM);
-    if (tid == 0) p.meta[0] = nU;
-    for (int i = tid; i < nU; i += blockDim.x) m_touched[i] = touched[i];
-    for (int i = tid; i < nU * kMaxM; i += blockDim.x) m_slotmap[i] = slotmap[i];
-    for (int i = tid; i < S; i += blockDim.x) m_w[i] = w_s[i];
-  }
-  const int ipe = I / 8;  // items per expert
-  const int nitems = nU * ipe;
-  // A contiguous run of items per CTA: consecutive items are consecutive rows.
-  const int q = nitems / gridDim.x, rem = nitems % gridDim.x;
-  const int i0 = blockIdx.x * q + min(static_cast<int>(blockIdx.x), rem);
-  const int i1 = i0 + q + (static_cast<int>(blockIdx.x) < rem ? 1 : 0);
-
-  if (warp == kWarps - 1) {
-    // Prefetch this CTA's share of the touched experts' down rows into L2.
-    const uint64_t per_expert = static_cast<uint64_t>(H) * I / 2;
-    const uint64_t per_expert_am = static_cast<uint64_t>(H) * (I / 64) * 4;
-    const uint64_t chunks_pk = (per_expert + kPrefetchChunk - 1) / kPrefetchChunk;
-    const uint64_t chunks_am = (per_expert_am + kPrefetchChunk - 1) / kPrefetchChunk;
-    const uint64_t per_u = chunks_pk + chunks_am;
-    uint64_t total = static_cast<uint64_t>(nU) * per_u;
-    const uint64_t cap = kPrefetchLimit / kPrefetchChunk;
-    if (total > cap) total = cap;
-    for (uint64_t c = static_cast<uint64_t>(blockIdx.x) * 32 + lane; c < total; c += static_cast<uint64_t>(gridDim.x) * 32) {
-      const uint64_t u = c / per_u, qq = c % per_u;
-      const int64_t e = touched[u];
-      if (qq < chunks_pk) {
-        const uint64_t off = qq * kPrefetchChunk;
-        const uint64_t n = min(static_cast<uint64_t>(kPrefetchChunk), per_expert - off);
-        prefetch_l2(p.dn_packed + e * per_expert + off, static_cast<uint32_t>(n));
-      } else {
-        const uint64_t off = (qq - chunks_pk) * kPrefetchChunk;
-        const uint64_t n = min(static_cast<uint64_t>(kPrefetchChunk), per_expert_am - off);
-        prefetch_l2(reinterpret_cast<const unsigned char*>(p.dn_absmax) + e * per_expert_am + off,
-                    static_cast<uint32_t>(n));
-      }
-    }
-  }
-
   const int g = lane >> 2, t = lane & 3;
+  if (tid == 0) {
+    abort_s = 0;
+    for (int s = 0; s < RS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kMath);
+    }
+    fence_mbar_init();
+  }
+  prologue(p, lut, ids_s, w_s, uidx, touched, slotmap, &nU_s);
+  const int nU = nU_s;
+  const int G = static_cast<int>(gridDim.x), bid = static_cast<int>(blockIdx.x);
+
+  // Phase-1 items: a contiguous run per CTA (consecutive items = consecutive rows).
+  const int ipe = I / 8;
+  const int nitems = nU * ipe;
+  const int q_it = nitems / G, rem_it = nitems % G;
+  const int i0 = bid * q_it + min(bid, rem_it);
+  const int n_gu = q_it + (bid < rem_it ? 1 : 0);
+  // Phase-2 stages: row blocks bid, bid + G, ...; per row block ceil(nU / DPE) stages.
+  const int nrb_all = H / 16;
+  const int nrb = bid < nrb_all ? (nrb_all - bid + G - 1) / G : 0;
+  const int nch = (nU + DPE - 1) / DPE;
+  const int n_dn = nrb * nch;
+  const int T = n_gu + n_dn;
+
+  if (warp == kProducer) {
+    // ------------------------------------------------------------ producer
+    int issued = 0;
+    for (int j = 0; j < T; ++j) {
+      const int s = j % RS;
+      if (j >= RS && !ring_wait(&empty[s], ((j / RS) - 1) & 1, &abort_s, p.err, kErrWaitEmpty)) break;
+      unsigned char* st = ring + static_cast<uint32_t>(s) * slot;
+      if (j < n_gu) {
+        const int it = i0 + j, u = it / ipe, rb = it % ipe;
+        const int64_t grow = static_cast<int64_t>(touched[u]) * 2 * I + rb * 8;
+        if (lane == 0) mbar_arrive_expect_tx(&full[s], 16u * (H / 2) + 16u * KB * 4);
+        __syncwarp();
+        copy_rows16(st, &full[s], p.gu_packed, p.gu_absmax, H, grow, grow + I);
+      } else {
+        const int jd = j - n_gu, ch = jd % nch, rb = bid + (jd / nch) * G;
+        const int u0 = ch * DPE, ne = min(DPE, nU - u0);
+        if (lane == 0) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(ne) * (16u * (I / 2) + 16u * KBI * 4));
+        __syncwarp();
+        for (int ei = 0; ei < ne; ++ei) {
+          const int64_t row0 = static_cast<int64_t>(touched[u0 + ei]) * H + rb * 16;
+          copy_rows16(st + ei * exp_dn, &full[s], p.dn_packed, p.dn_absmax, I, row0, row0 + 8);
+        }
+      }
+      ++issued;
+    }
+    // Every copy in flight lands before the CTA may exit.
+    for (int j = max(0, issued - RS); j < issued; ++j) {
+      if (mbar_try_wait(&full[j % RS], (j / RS) & 1)) continue;
+      const unsigned long long t0 = global_ns();
+      while (!mbar_try_wait(&full[j % RS], (j / RS) & 1))
+        if (global_ns() - t0 > kWaitLimitNs) {
+          record_error(p.err, kErrWaitDrain);
+          break;
+        }
+    }
+    return;
+  }
+
+  // ---------------------------------------------------------------- math warps
+  const uint32_t* lut_lane = lut + lane;
   const int S = p.M * p.k;
-  if (p.r > 0) {
-    // LoRA first factor per slot: xa[s, rho] = x[token(s)] . lora_A[e(s), rho]
-    for (int qd = warp; qd < S * p.r; qd += kWarps) {
+  if (p.r > 0 && n_gu > 0) {
+    // LoRA first factor of the slots whose expert has items in this CTA:
+    // xa[s, rho] = x[token(s)] . lora_A[e(s), rho]
+    const int u_lo = i0 / ipe, u_hi = (i0 + n_gu - 1) / ipe;
+    for (int qd = warp; qd < S * p.r; qd += kMath) {
       const int s = qd / p.r, rho = qd % p.r;
-      const int tok = s / p.k;
+      const int u = uidx[ids_s[s]];
+      if (u < u_lo || u > u_hi) continue;
+      const uint16_t* xr = p.x + static_cast<int64_t>(s / p.k) * H;
       const uint16_t* la = p.lora_A + (static_cast<int64_t>(ids_s[s]) * p.r + rho) * H;
       float acc = 0.f;
       for (int kk = lane * 8; kk < H; kk += 256) {
-        const uint4 xv = *reinterpret_cast<const uint4*>(xs + tok * xstride + kk);
+        const uint4 xv = *reinterpret_cast<const uint4*>(xr + kk);
         const uint4 av = *reinterpret_cast<const uint4*>(la + kk);
         const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, aw[4] = {av.x, av.y, av.z, av.w};
 #pragma unroll
@@ -329,280 +419,296 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gate_up_kernel(DecodeParam
       for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
       if (lane == 0) xa[qd] = acc;
     }
-    __syncthreads();
+    named_bar(kBarMath, kMath * 32);
   }
-  const uint32_t* lut_lane = lut + lane;
-  const int64_t row_bytes = H / 2;
-  // Batches after the first read L2: keep the bulk prefetch two batches ahead.
-  if (tid < 2 * IB) prefetch_items(p, touched, min(i0 + IB, i1), min(i0 + 3 * IB, i1));
-  for (int b0 = i0; b0 < i1; b0 += IB) {
-    const int nb = min(IB, i1 - b0);
-    if (b0 > i0 && tid < IB) prefetch_items(p, touched, min(b0 + 2 * IB, i1), min(b0 + 3 * IB, i1));
-    // Issue every load of the batch first (HBM latency is hidden by the batch).
-    // 16-byte loads: a lane's 32 k of a span lie in k-block 2 * span + t / 2.
-    uint4 pk[IB][KBW][2];
-    float am[IB][KBW][2];
-#pragma unroll
-    for (int ii = 0; ii < IB; ++ii) {
-      const int it = b0 + (ii < nb ? ii : 0);
-      const int u = it / ipe, rb = it % ipe;
-      const int64_t grow = static_cast<int64_t>(touched[u]) * 2 * I + rb * 8 + g;  // gate row of lane's MMA row g
-      const uint8_t* gp = p.gu_packed + grow * row_bytes + 16 * t;
-      const uint8_t* up = gp + static_cast<int64_t>(I) * row_bytes;
-      const float* ga = p.gu_absmax + grow * KB;
-      const float* ua = ga + static_cast<int64_t>(I) * KB;
-#pragma unroll
-      for (int q2 = 0; q2 < KBW; ++q2) {
-        const int sp = warp + kWarps * q2;
-        const int kb = 2 * sp + (t >> 1);
-        if (ii < nb && kb < KB) {
-          pk[ii][q2][0] = ld_stream_u4(gp + sp * 64);
-          pk[ii][q2][1] = ld_stream_u4(up + sp * 64);
-          am[ii][q2][0] = __ldg(ga + kb);
-          am[ii][q2][1] = __ldg(ua + kb);
-        } else {
-          pk[ii][q2][0] = pk[ii][q2][1] = make_uint4(0, 0, 0, 0);
-          am[ii][q2][0] = am[ii][q2][1] = 0.f;
-        }
-      }
-    }
-#pragma unroll
-    for (int ii = 0; ii < IB; ++ii) {
-      if (ii >= nb) break;
-      const int u = (b0 + ii) / ipe;
-      const bool has_g = (g < p.M) && slotmap[u * kMaxM + g] >= 0;  // token g routes to this expert
-      const uint16_t* xrow = xs + g * xstride + 32 * t;
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int q2 = 0; q2 < KBW; ++q2) {
-        const int sp = warp + kWarps * q2;
-        if (2 * sp >= KB) break;
-        uint4 xv[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
-        if (has_g && 2 * sp + (t >> 1) < KB) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) xv[i] = *reinterpret_cast<const uint4*>(xrow + sp * 128 + 8 * i);
-        }
-        span_mma(lut_lane, pk[ii][q2][0], pk[ii][q2][1], am[ii][q2][0], am[ii][q2][1], xv, acc);
-      }
-      red[(ii * kWarps + warp) * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    }
-    __syncthreads();
-    if (warp < nb) {
-      // Warp `warp` finishes item b0 + warp: sum the 16 partials in warp order.
-      float4 c = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int w = 0; w < kWarps; ++w) {
-        const float4 v = red[(warp * kWarps + w) * 32 + lane];
-        c.x += v.x;
-        c.y += v.y;
-        c.z += v.z;
-        c.w += v.w;
-      }
-      const int it = b0 + warp;
-      const int u = it / ipe, rb = it % ipe;
-      const int e = touched[u];
-      const int col = rb * 8 + g;  // h column == gate row index
-      const float gate_v[2] = {c.x, c.y}, up_v[2] = {c.z, c.w};
-#pragma unroll
-      for (int qq = 0; qq < 2; ++qq) {
-        const int tok = 2 * t + qq;
-        if (tok >= p.M) continue;
-        const int slot = slotmap[u * kMaxM + tok];
-        if (slot < 0) continue;
-        float gv = gate_v[qq], uv = up_v[qq];
-        if (p.r > 0) {
-          const uint16_t* bg = p.lora_B + (static_cast<int64_t>(e) * 2 * I + col) * p.r;
-          const uint16_t* bu = p.lora_B + (static_cast<int64_t>(e) * 2 * I + I + col) * p.r;
-          float dg = 0.f, du = 0.f;
-          for (int rho = 0; rho < p.r; ++rho) {
-            const float xv = xa[slot * p.r + rho];
-            dg = fmaf(xv, bf16_bits_to_float(bg[rho]), dg);
-            du = fmaf(xv, bf16_bits_to_float(bu[rho]), du);
-          }
-          gv = fmaf(p.lora_scale, dg, gv);
-          uv = fmaf(p.lora_scale, du, uv);
-        }
-        p.h[static_cast<int64_t>(slot) * I + col] = float_to_bf16_bits(silu_f32(gv) * uv);
-      }
-    }
-    __syncthreads();
-  }
-}
 
-// ---------------------------------------------------------------------------
-// Kernel B: down rows of every touched expert, weighted combine -> out.
-__global__ void __launch_bounds__(kThreads, 1) decode_down_kernel(DecodeParams p) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  const Layout L = make_layout(false, p.M, p.k, p.E, p.H, 0);
-  uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L.lut);
-  float4* red = reinterpret_cast<float4*>(smem + L.red);
-  float* w_s = reinterpret_cast<float*>(smem + L.w);
-  int* touched = reinterpret_cast<int*>(smem + L.touched);
-  int* slotmap = reinterpret_cast<int*>(smem + L.slotmap);
-  __shared__ int nU_s;
-
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int H = p.H, I = p.I, KB = I / 64;
-  // The down kernel starts once the gate_up kernel's CTAs leave the SMs; it
-  // builds its codebook table, waits for that kernel's results (h and the
-  // routing it published) and reads the routing instead of recomputing it.
-  fill_lut_warps(lut, 0);
-  pdl_wait();  // h and the routing written by the gate_up kernel are visible from here on
+  // -------------------------------------------------------------- phase 1
   {
-    const int S = p.M * p.k;
-    const int* m_touched = p.meta + 4;
-    const int* m_slotmap = m_touched + S;
-    const float* m_w = reinterpret_cast<const float*>(m_slotmap + S * kMaxM);
-    const int n = __ldcg(p.meta);
-    if (tid == 0) nU_s = n;
-    for (int i = tid; i < n; i += blockDim.x) touched[i] = __ldcg(m_touched + i);
-    for (int i = tid; i < n * kMaxM; i += blockDim.x) slotmap[i] = __ldcg(m_slotmap + i);
-    for (int i = tid; i < S; i += blockDim.x) w_s[i] = __ldcg(m_w + i);
-  }
-  __syncthreads();
-  const int nU = nU_s;
-  const int NSP = (KB + 1) / 2;  // spans of 128 k (two absmax blocks) in a down row
-  const int npairs = nU * NSP;   // (expert, span) pairs of one row block
-  const int g = lane >> 2, t = lane & 3;
-  const uint32_t* lut_lane = lut + lane;
-  const int64_t row_bytes = I / 2;
-  for (int rb = blockIdx.x; rb < H / 16; rb += gridDim.x) {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int pb = warp; pb < npairs; pb += kWarps * kPairSlots) {
-      uint4 pk[kPairSlots][2];
-      float am[kPairSlots][2];
-      uint4 hx[kPairSlots][4];
-      float wc[kPairSlots][2];
+    const int gi = warp / kGW, wi = warp % kGW;
+    // The warp's k-blocks are the same in every item: its slice of x (token g
+    // of the MMA column) stays in registers.  Columns of tokens that do not
+    // route to an item's expert compute values that are never stored.
+    uint32_t xr[SPW][2][8];
 #pragma unroll
-      for (int sl = 0; sl < kPairSlots; ++sl) {
-        const int pi = pb + kWarps * sl;
-        pk[sl][0] = pk[sl][1] = make_uint4(0, 0, 0, 0);
-        am[sl][0] = am[sl][1] = 0.f;
+    for (int q = 0; q < SPW; ++q) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) hx[sl][i] = make_uint4(0, 0, 0, 0);
-        wc[sl][0] = wc[sl][1] = 0.f;
-        if (pi < npairs) {
-          const int u = pi / NSP, sp = pi % NSP;
-          const int kb = 2 * sp + (t >> 1);  // this lane's 32 k of the span lie in k-block kb
-          const int64_t row = static_cast<int64_t>(touched[u]) * H + rb * 16 + g;
+      for (int hh = 0; hh < 2; ++hh) {
+        const int kb = 2 * (wi + kGW * q) + hh;
+        uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+        if (g < p.M && kb < KB) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(g) * H + kb * 64 + 16 * t);
+          a = src[0];
+          b = src[1];
+        }
+        xr[q][hh][0] = a.x; xr[q][hh][1] = a.y; xr[q][hh][2] = a.z; xr[q][hh][3] = a.w;
+        xr[q][hh][4] = b.x; xr[q][hh][5] = b.y; xr[q][hh][6] = b.z; xr[q][hh][7] = b.w;
+      }
+    }
+    for (int jj = gi; jj < n_gu; jj += kGroups) {
+      const int s = jj % RS;
+      ring_wait(&full[s], (jj / RS) & 1, &abort_s, p.err, kErrWaitFull);
+      const unsigned char* st = ring + static_cast<uint32_t>(s) * slot;
+      const float* am = reinterpret_cast<const float*>(st + am_gu);
+      float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int q = 0; q < SPW; ++q) {
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int kb = 2 * (wi + kGW * q) + hh;
           if (kb < KB) {
-            const uint8_t* rp = p.dn_packed + row * row_bytes + sp * 64 + 16 * t;
-            pk[sl][0] = ld_stream_u4(rp);
-            pk[sl][1] = ld_stream_u4(rp + 8 * row_bytes);
-            am[sl][0] = __ldg(p.dn_absmax + row * KB + kb);
-            am[sl][1] = __ldg(p.dn_absmax + (row + 8) * KB + kb);
-            const int slot_g = (g < p.M) ? slotmap[u * kMaxM + g] : -1;
-            if (slot_g >= 0) {
-              const uint16_t* hr = p.h + static_cast<int64_t>(slot_g) * I + sp * 128 + 32 * t;
-#pragma unroll
-              for (int i = 0; i < 4; ++i) hx[sl][i] = *reinterpret_cast<const uint4*>(hr + 8 * i);
-            }
+            const uint2 w0 = lds64(st + g * ps_gu + kb * 32 + 8 * t);
+            const uint2 w1 = lds64(st + (g + 8) * ps_gu + kb * 32 + 8 * t);
+            const float a0 = am[g * sa_gu + kb], a1 = am[(g + 8) * sa_gu + kb];
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            block_mma(lut_lane, w0, w1, xr[q][hh], d);
+            c[0] = fmaf(a0, d[0], c[0]);
+            c[1] = fmaf(a0, d[1], c[1]);
+            c[2] = fmaf(a1, d[2], c[2]);
+            c[3] = fmaf(a1, d[3], c[3]);
           }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cnt(&empty[s], kMath / kGW);
+      const int par = (jj / kGroups) & 1;
+      red[((gi * 2 + par) * kGW + wi) * 32 + lane] = make_float4(c[0], c[1], c[2], c[3]);
+      named_bar(kBarGroup0 + gi, kGW * 32);
+      if (wi == (jj / kGroups) % kGW) {
+        // This warp finishes the item: the group's partials in warp order,
+        // then SwiGLU (+ LoRA delta) for the tokens routed to the expert.
+        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int w = 0; w < kGW; ++w) {
+          const float4 v = red[((gi * 2 + par) * kGW + w) * 32 + lane];
+          sum.x += v.x;
+          sum.y += v.y;
+          sum.z += v.z;
+          sum.w += v.w;
+        }
+        const int it = i0 + jj, u = it / ipe, rb = it % ipe;
+        const int e = touched[u];
+        const int col = rb * 8 + g;  // h column == gate row index
+        const float gate_v[2] = {sum.x, sum.y}, up_v[2] = {sum.z, sum.w};
+#pragma unroll
+        for (int qq = 0; qq < 2; ++qq) {
+          const int tok = 2 * t + qq;
+          if (tok >= p.M) continue;
+          const int sl = slotmap[u * kMaxM + tok];
+          if (sl < 0) continue;
+          float gv = gate_v[qq], uv = up_v[qq];
+          if (p.r > 0) {
+            const uint16_t* bg = p.lora_B + (static_cast<int64_t>(e) * 2 * I + col) * p.r;
+            const uint16_t* bu = p.lora_B + (static_cast<int64_t>(e) * 2 * I + I + col) * p.r;
+            float dg = 0.f, du = 0.f;
+            for (int rho = 0; rho < p.r; ++rho) {
+              const float xv = xa[sl * p.r + rho];
+              dg = fmaf(xv, bf16_bits_to_float(bg[rho]), dg);
+              du = fmaf(xv, bf16_bits_to_float(bu[rho]), du);
+            }
+            gv = fmaf(p.lora_scale, dg, gv);
+            uv = fmaf(p.lora_scale, du, uv);
+          }
+          p.h[static_cast<int64_t>(sl) * I + col] = float_to_bf16_bits(silu_f32(gv) * uv);
+        }
+      }
+    }
+  }
+
+  // --------------------------------------------------------- grid barrier
+  named_bar(kBarMath, kMath * 32);  // every h store of this CTA is issued
+  if (warp == 0) {
+    const unsigned long long gid = grid_id();
+    if (lane == 0) {
+      __threadfence();
+      st_release_gpu(p.flags + bid, gid);
+    }
+    __syncwarp();
+    const unsigned long long t0 = global_ns();
+    while (true) {
+      bool ready = true;
+      for (int c = lane; c < G; c += 32) ready = ready && ld_acquire_gpu(p.flags + c) == gid;
+      if (__all_sync(0xffffffffu, ready)) break;
+      if (abort_s) break;
+      if (global_ns() - t0 > kWaitLimitNs) {
+        if (lane == 0) {
+          abort_s = 1;
+          record_error(p.err, kErrGridBarrier);
+        }
+        break;
+      }
+    }
+    __threadfence();
+  }
+  named_bar(kBarMath, kMath * 32);
+
+  // -------------------------------------------------------------- phase 2
+  {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    uint4 hA[PPW][2], hB[PPW][2];
+    // h fragments of stage jd for this warp's pairs (zeros where token g does
+    // not route to the pair's expert), loaded one stage ahead of their use.
+    auto load_h = [&](int jd, uint4 (&hb)[PPW][2]) {
+#pragma unroll
+      for (int q = 0; q < PPW; ++q) hb[q][0] = hb[q][1] = make_uint4(0, 0, 0, 0);
+      if (jd >= n_dn) return;
+      const int u0 = (jd % nch) * DPE, np = min(DPE, nU - u0) * KBI;
+#pragma unroll
+      for (int q = 0; q < PPW; ++q) {
+        const int pi = warp + kMath * q;
+        if (pi < np) {
+          const int u = u0 + pi / KBI, kb = pi % KBI;
+          const int sg = g < p.M ? slotmap[u * kMaxM + g] : -1;
+          if (sg >= 0) {
+            const uint4* src = reinterpret_cast<const uint4*>(p.h + static_cast<int64_t>(sg) * I + kb * 64 + 16 * t);
+            hb[q][0] = __ldcg(src);
+            hb[q][1] = __ldcg(src + 1);
+          }
+        }
+      }
+    };
+    auto compute = [&](int jd, const uint4 (&hb)[PPW][2]) {
+      const int j = n_gu + jd, s = j % RS;
+      ring_wait(&full[s], (j / RS) & 1, &abort_s, p.err, kErrWaitFull);
+      const unsigned char* st = ring + static_cast<uint32_t>(s) * slot;
+      const int ch = jd % nch, u0 = ch * DPE, np = min(DPE, nU - u0) * KBI;
+#pragma unroll
+      for (int q = 0; q < PPW; ++q) {
+        const int pi = warp + kMath * q;
+        if (pi < np) {
+          const int ei = pi / KBI, kb = pi % KBI, u = u0 + ei;
+          const unsigned char* base = st + ei * exp_dn;
+          const float* am = reinterpret_cast<const float*>(base + am_dn);
+          const uint2 w0 = lds64(base + g * ps_dn + kb * 32 + 8 * t);
+          const uint2 w1 = lds64(base + (g + 8) * ps_dn + kb * 32 + 8 * t);
+          const float a0 = am[g * sa_dn + kb], a1 = am[(g + 8) * sa_dn + kb];
+          float d[4] = {0.f, 0.f, 0.f, 0.f};
+          block_mma(lut_lane, w0, w1, reinterpret_cast<const uint32_t*>(hb[q]), d);
           const int s0 = (2 * t < p.M) ? slotmap[u * kMaxM + 2 * t] : -1;
           const int s1 = (2 * t + 1 < p.M) ? slotmap[u * kMaxM + 2 * t + 1] : -1;
-          wc[sl][0] = s0 >= 0 ? w_s[s0] : 0.f;
-          wc[sl][1] = s1 >= 0 ? w_s[s1] : 0.f;
+          const float wc0 = s0 >= 0 ? w_s[s0] : 0.f, wc1 = s1 >= 0 ? w_s[s1] : 0.f;
+          acc[0] = fmaf(a0 * wc0, d[0], acc[0]);
+          acc[1] = fmaf(a0 * wc1, d[1], acc[1]);
+          acc[2] = fmaf(a1 * wc0, d[2], acc[2]);
+          acc[3] = fmaf(a1 * wc1, d[3], acc[3]);
         }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      if (ch == nch - 1) {
+        // End of a row block: the 16 warps' sums in warp order -> out.
+        const int rbq = jd / nch, par = rbq & 1;
+        red[(par * kMath + warp) * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+        named_bar(kBarMath, kMath * 32);
+        if (warp == rbq % kMath) {
+          float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int w = 0; w < kMath; ++w) {
+            const float4 v = red[(par * kMath + w) * 32 + lane];
+            sum.x += v.x;
+            sum.y += v.y;
+            sum.z += v.z;
+            sum.w += v.w;
+          }
+          const int row0 = (bid + rbq * G) * 16 + g;
+          const float v[4] = {sum.x, sum.y, sum.z, sum.w};
 #pragma unroll
-      for (int sl = 0; sl < kPairSlots; ++sl) {
-        if (pb + kWarps * sl >= npairs) break;
-        float tmp[4] = {0.f, 0.f, 0.f, 0.f};
-        span_mma(lut_lane, pk[sl][0], pk[sl][1], am[sl][0], am[sl][1], hx[sl], tmp);
-        acc[0] = fmaf(tmp[0], wc[sl][0], acc[0]);
-        acc[1] = fmaf(tmp[1], wc[sl][1], acc[1]);
-        acc[2] = fmaf(tmp[2], wc[sl][0], acc[2]);
-        acc[3] = fmaf(tmp[3], wc[sl][1], acc[3]);
+          for (int q2 = 0; q2 < 4; ++q2) {
+            const int tok = 2 * t + (q2 & 1);
+            const int row = row0 + ((q2 >> 1) ? 8 : 0);
+            if (tok < p.M) p.out[static_cast<int64_t>(tok) * H + row] = float_to_bf16_bits(v[q2]);
+          }
+        }
+      }
+    };
+    load_h(0, hA);
+    for (int jd = 0; jd < n_dn; jd += 2) {
+      load_h(jd + 1, hB);
+      compute(jd, hA);
+      if (jd + 1 < n_dn) {
+        load_h(jd + 2, hA);
+        compute(jd + 1, hB);
       }
     }
-    red[warp * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    __syncthreads();
-    if (warp == 0) {
-      float4 c = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int w = 0; w < kWarps; ++w) {
-        const float4 v = red[w * 32 + lane];
-        c.x += v.x;
-        c.y += v.y;
-        c.z += v.z;
-        c.w += v.w;
-      }
-      const int row0 = rb * 16 + g;
-      const float v[4] = {c.x, c.y, c.z, c.w};
-#pragma unroll
-      for (int q2 = 0; q2 < 4; ++q2) {
-        const int tok = 2 * t + (q2 & 1);
-        const int row = row0 + ((q2 >> 1) ? 8 : 0);
-        if (tok < p.M) p.out[static_cast<int64_t>(tok) * H + row] = float_to_bf16_bits(v[q2]);
-      }
-    }
-    __syncthreads();
   }
 }
 
-template <int KBW, int SLOTS>
-cudaError_t raise_smem_limits(size_t smem_a, size_t smem_b) {
-  cudaError_t err = ensure_smem_limit(reinterpret_cast<const void*>(decode_gate_up_kernel<KBW, SLOTS>), smem_a);
-  if (err != cudaSuccess) return err;
-  return ensure_smem_limit(reinterpret_cast<const void*>(decode_down_kernel), smem_b);
+using KernelFn = void (*)(FusedParams);
+
+template <int SPW>
+KernelFn pick_ppw(int ppw) {
+  switch (ppw) {
+    case 1: return decode_fused_kernel<SPW, 1>;
+    case 2: return decode_fused_kernel<SPW, 2>;
+    case 3: return decode_fused_kernel<SPW, 3>;
+    default: return decode_fused_kernel<SPW, 4>;
+  }
 }
 
-template <int KBW, int SLOTS>
-cudaError_t launch_pair(const DecodeParams& p, int sm_count, size_t smem_a, size_t smem_b, cudaStream_t stream) {
-  cudaError_t aerr = raise_smem_limits<KBW, SLOTS>(smem_a, smem_b);
-  if (aerr != cudaSuccess) return aerr;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(kThreads);
-  cfg.stream = stream;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const int nitems_upper = std::min(p.M * p.k, p.E) * (p.I / 8);
-  cfg.gridDim = dim3(std::max(1, std::min(sm_count, nitems_upper)));
-  cfg.dynamicSmemBytes = smem_a;
-  {
-    LaunchScope ls("decode.gate_up", stream);
-    cudaError_t err = cudaLaunchKernelEx(&cfg, decode_gate_up_kernel<KBW, SLOTS>, p);
-    if (err != cudaSuccess) return err;
+KernelFn pick_kernel(int spw, int ppw) {
+  switch (spw) {
+    case 1: return pick_ppw<1>(ppw);
+    case 2: return pick_ppw<2>(ppw);
+    case 3: return pick_ppw<3>(ppw);
+    default: return pick_ppw<4>(ppw);
   }
-  cfg.gridDim = dim3(std::max(1, std::min(sm_count, p.H / 16)));
-  cfg.dynamicSmemBytes = smem_b;
-  LaunchScope ls("decode.down", stream);
-  return cudaLaunchKernelEx(&cfg, decode_down_kernel, p);
+}
+
+// Launch plan of one shape.
+struct Plan {
+  int spw, ppw, dpe, stages, grid;
+  uint32_t slot;
+  size_t smem;
+};
+
+// Fills *pl; returns "" or why the shape does not fit the kernel.
+std::string make_plan(int M, int k, int E, int H, int I, int r, size_t smem_limit, int sm_count, Plan* pl) {
+  const int KB = H / 64, KBI = I / 64, nsp = (KB + 1) / 2;
+  pl->spw = (nsp + kGW - 1) / kGW;
+  if (pl->spw > kMaxSPW) return "the decode path takes H <= " + std::to_string(kGW * kMaxSPW * 128);
+  if (KBI > kMaxKBI) return "the decode path takes I <= " + std::to_string(kMaxKBI * 64);
+  const uint32_t gu = rows16_bytes(H), dn = rows16_bytes(I);
+  pl->dpe = std::max(1, std::min(static_cast<int>(gu / dn), kMaxKBI / KBI));
+  pl->ppw = (pl->dpe * KBI + kMath - 1) / kMath;
+  pl->slot = al(std::max(gu, static_cast<uint32_t>(pl->dpe) * dn), 128);
+  const size_t fixed = make_smem(M, k, E, r, 0, pl->slot).ring + 2 * kMaxStages * 8;
+  if (fixed >= smem_limit) return "the decode kernel's shared-memory plan does not fit this shape";
+  int st = static_cast<int>((smem_limit - fixed) / pl->slot);
+  st = std::min(st, kMaxStages) & ~1;
+  if (st < 2) return "the decode kernel's shared-memory ring does not fit this shape";
+  pl->stages = st;
+  pl->smem = make_smem(M, k, E, r, st, pl->slot).total;
+  const int items_upper = std::min(M * k, E) * (I / 8);
+  pl->grid = std::max(1, std::min({sm_count, kMaxGrid, std::max(items_upper, H / 16)}));
+  return "";
 }
 
 struct DecodeWs {
-  size_t h, meta, total;
+  size_t flags, h, total;
 };
 
-// Workspace: the error word every workspace begins with (no decode kernel
-// waits, so it stays untouched), h [M*k, I] bf16, then the published routing
-// (4 + S * (2 + kMaxM) ints).
+// Workspace: the error word every workspace begins with (256-byte slot), the
+// grid barrier's slots (one 64-bit word per CTA), h [M*k, I] bf16.
 DecodeWs decode_ws(int64_t M, int k, int64_t I) {
   DecodeWs w;
-  const int64_t S = M * k;
-  w.h = 256;
-  w.meta = w.h + align_up(static_cast<size_t>(S * I * 2), 256);
-  w.total = w.meta + align_up(static_cast<size_t>(4 + S * (2 + kMaxM)) * 4, 256);
+  w.flags = 256;
+  w.h = w.flags + static_cast<size_t>(kMaxGrid) * 8;
+  w.total = w.h + align_up(static_cast<size_t>(M * k * I * 2), 256);
   return w;
 }
 
 }  // namespace
 
 std::string decode_unsupported_reason(int64_t M, int64_t E, int k, int64_t H, int64_t I) {
-  (void)I;
   if (M < 1 || M > kMaxM) return "the decode path takes 1 to " + std::to_string(kMaxM) + " tokens (M=" + std::to_string(M) + ")";
   if (k > 32) return "the decode path takes k <= 32 (k=" + std::to_string(k) + ")";
   if (E > 512) return "the decode path takes at most 512 experts (E=" + std::to_string(E) + ")";
-  if (H > 128 * kWarps * kMaxKBW)
-    return "the decode path takes H <= " + std::to_string(128 * kWarps * kMaxKBW) + " (H=" + std::to_string(H) + ")";
+  if (H > kGW * kMaxSPW * 128)
+    return "the decode path takes H <= " + std::to_string(kGW * kMaxSPW * 128) + " (H=" + std::to_string(H) + ")";
+  if (I > kMaxKBI * 64) return "the decode path takes I <= " + std::to_string(kMaxKBI * 64) + " (I=" + std::to_string(I) + ")";
   DeviceInfo di;
   if (device_info(&di) != cudaSuccess) return "device query failed";
-  const Layout a = make_layout(true, static_cast<int>(M), k, static_cast<int>(E), static_cast<int>(H), 16);
-  const Layout b = make_layout(false, static_cast<int>(M), k, static_cast<int>(E), static_cast<int>(H), 0);
-  const size_t lim = di.smem_optin - 1024;  // leave room for the kernels' static shared memory
-  if (a.total > lim || b.total > lim) return "the decode kernels' shared-memory plan does not fit this shape";
-  return "";
+  Plan pl;
+  return make_plan(static_cast<int>(M), k, static_cast<int>(E), static_cast<int>(H), static_cast<int>(I), 16,
+                   di.smem_optin - 1024, di.sm_count, &pl);
 }
 
 bool decode_supported(int64_t M, int64_t E, int k, int64_t H, int64_t I) {
@@ -624,7 +730,7 @@ cudaError_t launch_decode_forward(const DecodeArgs& a, cudaStream_t stream) {
   const e4b_expert_stack* w = a.w;
   const int r = w->lora_A ? w->lora_r : 0;
   const DecodeWs ws = decode_ws(a.M, a.k, w->I);
-  DecodeParams p{};
+  FusedParams p{};
   p.x = a.x;
   p.logits = a.logits;
   p.M = static_cast<int>(a.M);
@@ -641,16 +747,30 @@ cudaError_t launch_decode_forward(const DecodeArgs& a, cudaStream_t stream) {
   p.lora_B = r ? w->lora_B : nullptr;
   p.r = r;
   p.lora_scale = r ? w->lora_alpha / static_cast<float>(r) : 0.f;
+  p.err = static_cast<int*>(a.workspace);
+  p.flags = reinterpret_cast<unsigned long long*>(static_cast<char*>(a.workspace) + ws.flags);
   p.h = reinterpret_cast<uint16_t*>(static_cast<char*>(a.workspace) + ws.h);
-  p.meta = reinterpret_cast<int*>(static_cast<char*>(a.workspace) + ws.meta);
   p.out = a.out;
-  const size_t smem_a = make_layout(true, p.M, p.k, p.E, p.H, r).total;
-  const size_t smem_b = make_layout(false, p.M, p.k, p.E, p.H, 0).total;
-  if (kbw_of(p.H) == 1) {
-    if (slots_for(p.M, p.H) == 8) return launch_pair<1, 8>(p, di.sm_count, smem_a, smem_b, stream);
-    return launch_pair<1, 4>(p, di.sm_count, smem_a, smem_b, stream);
-  }
-  return launch_pair<2, 4>(p, di.sm_count, smem_a, smem_b, stream);
+  Plan pl;
+  if (!make_plan(p.M, p.k, p.E, p.H, p.I, r, di.smem_optin - 1024, di.sm_count, &pl).empty())
+    return cudaErrorInvalidConfiguration;
+  p.stages = pl.stages;
+  p.dpe = pl.dpe;
+  const KernelFn fn = pick_kernel(pl.spw, pl.ppw);
+  err = ensure_smem_limit(reinterpret_cast<const void*>(fn), pl.smem);
+  if (err != cudaSuccess) return err;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pl.grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = pl.smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  LaunchScope ls("decode.fused", stream);
+  return cudaLaunchKernelEx(&cfg, fn, p);
 }
 
 }  // namespace e4b

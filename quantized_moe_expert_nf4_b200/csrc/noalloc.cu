@@ -4,10 +4,9 @@
 // carve every byte of device memory out of a fixed pool planned at start-up,
 // and runtimes that forbid any allocator call (cudaMalloc included) once the
 // decode loop is running.  For them this file keeps the decode path's scratch
-// -- the SwiGLU activations h of the routed slots and the routing result the
-// gate_up kernel hands to the down kernel -- in a
-// statically sized device array that exists from the moment the library is
-// loaded on a GPU until the process exits.  The caller still passes x, the
+// -- the SwiGLU activations h of the routed slots and the slots of the decode
+// kernel's grid barrier -- in a statically sized device array that exists from
+// the moment the library is loaded on a GPU until the process exits.  The caller still passes x, the
 // router logits, the packed stacks and the output buffer.
 #include <cuda.h>
 
@@ -23,7 +22,7 @@ namespace {
 // h holds M*k*I bf16 values; the limit below allows e.g. M=8, k=8, I=4096.
 constexpr int64_t kNoAllocMaxHElems = 256 * 1024;
 constexpr size_t kNoAllocHBytes = static_cast<size_t>(kNoAllocMaxHElems) * 2;
-constexpr size_t kNoAllocBytes = kNoAllocHBytes + 16 * 1024;  // + the error word and the routing the kernels share
+constexpr size_t kNoAllocBytes = kNoAllocHBytes + 16 * 1024;  // + the error word and the grid-barrier slots
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 

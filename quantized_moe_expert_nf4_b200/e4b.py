@@ -305,6 +305,7 @@ def workspace(nbytes: int, device="cuda") -> torch.Tensor:
 
 
 E4B_KERNEL_ERR_NONE, E4B_KERNEL_ERR_WAIT_FULL, E4B_KERNEL_ERR_WAIT_EMPTY, E4B_KERNEL_ERR_WAIT_DRAIN = 0, 1, 2, 3
+E4B_KERNEL_ERR_GRID_BARRIER = 4
 
 
 def workspace_error(ws: torch.Tensor) -> int:

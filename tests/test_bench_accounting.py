@@ -48,6 +48,18 @@ def test_decode_roofline_arithmetic():
     assert r["frac"] == pytest.approx(r["achieved"] / 6541.5)
 
 
+def test_fused_decode_roofline_counts_the_whole_step():
+    """The fused decode kernel is the whole layer: its algorithmic bytes are the step's."""
+    cfg = workloads.CONFIGS["olmoe"]
+    peaks = {"hbm_gbs": 6541.5, "bf16_tflops": 1617.9, "bf16_tflops_sustained": 1374.1, "source": "measured"}
+    name, r = bench.dominant_roofline(cfg, 1, {"decode.fused": (0.008, 100)}, 8.0, peaks, long_region=False)
+    step_bytes = bench.step_work(cfg, 1, 8.0)[1]
+    assert name == "decode.fused" and r["bound"] == "hbm"
+    assert r["algorithmic_bytes_per_launch"] == pytest.approx(step_bytes)
+    assert 28.0e6 < step_bytes < 28.7e6        # 8 experts x 3.54 MB + x, out, logits
+    assert r["frac"] == pytest.approx(step_bytes / 8e-6 / 1e9 / 6541.5)
+
+
 def test_grouped_roofline_uses_the_sustained_peak_in_a_long_region():
     cfg = workloads.CONFIGS["qwen3"]
     peaks = {"hbm_gbs": 6541.5, "bf16_tflops": 1617.9, "bf16_tflops_sustained": 1374.1, "source": "measured"}

@@ -138,13 +138,55 @@ def test_forward_decode_path_all_tokens(name, cfg, M):
     layer = synthetic.make_device_layer(cfg)
     x, logits = synthetic.inputs(cfg, M)
     out, p = _forward(layer, x, logits, e4b.E4B_PATH_DECODE)
-    assert p == "forward.decode" and e4b.last_launches() == 2
+    assert p == "forward.decode" and e4b.last_launches() == 1
     ref = _oracle_tokens(cfg, x, logits, np.arange(M))
     assert_close_layer(bf16_to_f64(out), ref, f"{name} M={M} {p}")
     out2, _ = _forward(layer, x, logits, e4b.E4B_PATH_DECODE)
     assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
     outg, _ = _forward(layer, x, logits, e4b.E4B_PATH_GROUPED)
     assert_close_layer(bf16_to_f64(outg), ref, f"{name} M={M} grouped")
+
+
+@pytest.mark.parametrize("name,M", [("olmoe", 1), ("olmoe", 8), ("gptoss", 3)])
+def test_forward_decode_reuses_one_workspace_across_changing_inputs(name, M):
+    """The decode kernel's grid barrier keeps no state between calls: one
+    workspace (filled with garbage first) serves consecutive calls on new
+    inputs, eagerly and as replays of one captured graph whose input buffers
+    are refilled between replays; every result equals a fresh grouped-path
+    forward of the same inputs to the layer tolerance, and eager and replayed
+    calls agree bit for bit."""
+    require_gpu()
+    cfg = workloads.CONFIGS[name]
+    layer = synthetic.make_device_layer(cfg)
+    ws = e4b.workspace(e4b.e4b_moe_expert_forward_workspace_size(M, layer.stack, cfg.k))
+    ws.random_(0, 255)
+    ws[:16].zero_()                       # the error word stays meaningful
+    x_buf, lg_buf = synthetic.inputs(cfg, M)
+    out = torch.empty((M, cfg.H), dtype=torch.bfloat16, device="cuda")
+    eager = []
+    for rep in range(3):
+        x, lg = synthetic.inputs(cfg, M, replica=rep + 1)
+        x_buf.copy_(x)
+        lg_buf.copy_(lg)
+        e4b.e4b_moe_expert_forward(x_buf, lg_buf, cfg.k, True, layer.stack, out, ws, path=e4b.E4B_PATH_DECODE)
+        torch.cuda.synchronize()
+        eager.append(out.clone())
+        ref, _ = _forward(layer, x, lg, e4b.E4B_PATH_GROUPED)
+        assert_close_layer(bf16_to_f64(out), bf16_to_f64(ref), f"{name} M={M} call {rep} vs grouped")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        e4b.e4b_moe_expert_forward(x_buf, lg_buf, cfg.k, True, layer.stack, out, ws, path=e4b.E4B_PATH_DECODE)
+    for rep in range(3):
+        x, lg = synthetic.inputs(cfg, M, replica=rep + 1)
+        x_buf.copy_(x)
+        lg_buf.copy_(lg)
+        out.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out.view(torch.int16), eager[rep].view(torch.int16)), f"replay {rep}"
+    assert e4b.workspace_error(ws) == e4b.E4B_KERNEL_ERR_NONE
 
 
 def test_forward_decode_rejects_large_batches():

@@ -49,40 +49,185 @@ def _layer_rows(seed, rows, K):
 
 
 @pytest.mark.parametrize("K", [128, 192, 2880])
-def test_decode_span_fragment_mapping(K):
-    """csrc/decode.cu span_mma: thread (g, t) of a span (128 k) holds 16 packed
-    bytes of rows g and g+8 at byte 16t (all inside k-block 2 span + t/2), the
-    block's absmax multiplied into each decoded pair, MMA j taking bytes 2j and
-    2j+1 and x words 2j, 2j+1 of the thread's 32 k."""
+def test_decode_block_fragment_mapping(K):
+    """csrc/decode.cu block_mma: in each 64-element k-block thread (g, t) holds
+    packed bytes [8t, 8t+8) of rows g and g+8 (elements 16t .. 16t+15) and the
+    16 matching x values of token column g; MMA j takes bytes 2j and 2j+1 and
+    x words 2j, 2j+1; the four MMAs of a block go into a zeroed partial that
+    the block's fp32 absmax of each row scales afterwards."""
     packed, absmax, W = _layer_rows(1, 16, K)
     rng = np.random.default_rng(2)
     x = rng.standard_normal((8, K))
     KB = K // 64
     acc = np.zeros((32, 4))
-    for sp in range((KB + 1) // 2):
-        A = [[None] * 32 for _ in range(8)]
-        B = [[None] * 32 for _ in range(8)]
+    for kb in range(KB):
+        d = np.zeros((32, 4))
+        for j in range(4):
+            A = [None] * 32
+            B = [None] * 32
+            for lane in range(32):
+                g, t = lane >> 2, lane & 3
+                r0 = packed[g, kb * 32 + 8 * t: kb * 32 + 8 * t + 8]
+                r1 = packed[g + 8, kb * 32 + 8 * t: kb * 32 + 8 * t + 8]
+                xs = x[g, kb * 64 + 16 * t: kb * 64 + 16 * t + 16]
+                A[lane] = (_pair(r0[2 * j]), _pair(r1[2 * j]), _pair(r0[2 * j + 1]), _pair(r1[2 * j + 1]))
+                B[lane] = ((xs[4 * j], xs[4 * j + 1]), (xs[4 * j + 2], xs[4 * j + 3]))
+            _mma(d, A, B)
         for lane in range(32):
-            g, t = lane >> 2, lane & 3
-            kb = 2 * sp + (t >> 1)
-            live = kb < KB
-            r0 = packed[g, sp * 64 + 16 * t: sp * 64 + 16 * t + 16] if live else np.zeros(16, np.uint8)
-            r1 = packed[g + 8, sp * 64 + 16 * t: sp * 64 + 16 * t + 16] if live else np.zeros(16, np.uint8)
-            a0 = absmax[g, kb] if live else 0.0
-            a1 = absmax[g + 8, kb] if live else 0.0
-            xs = x[g, sp * 128 + 32 * t: sp * 128 + 32 * t + 32] if live else np.zeros(32)
-            for j in range(8):
-                p = lambda r, i, a: tuple(v * a for v in _pair(r[i]))
-                A[j][lane] = (p(r0, 2 * j, a0), p(r1, 2 * j, a1), p(r0, 2 * j + 1, a0), p(r1, 2 * j + 1, a1))
-                B[j][lane] = ((xs[4 * j], xs[4 * j + 1]), (xs[4 * j + 2], xs[4 * j + 3]))
-        for j in range(8):
-            _mma(acc, A[j], B[j])
+            g = lane >> 2
+            acc[lane] += d[lane] * np.array([absmax[g, kb], absmax[g, kb], absmax[g + 8, kb], absmax[g + 8, kb]])
     got = np.zeros((16, 8))
     for lane in range(32):
         g, t = lane >> 2, lane & 3
         got[g, 2 * t], got[g, 2 * t + 1], got[g + 8, 2 * t], got[g + 8, 2 * t + 1] = acc[lane]
     ref = W @ x.T
     assert np.abs(got - ref).max() <= 1e-12 * np.abs(ref).max()
+
+
+# ---- csrc/decode.cu: the fused kernel's shared-memory plan and copies -------------
+SMEM_LIMIT = 227 * 1024 - 1024   # opt-in dynamic shared memory minus the kernel's reserve
+SMS = 148
+
+
+def _al(v, a):
+    return (v + a - 1) // a * a
+
+
+def _row_stride(K):
+    b = K // 2
+    return b + (160 - b % 128) % 128
+
+
+def _am_by_rows(KB):
+    return KB % 4 == 0
+
+
+def _am_stride(KB):
+    return (KB if KB % 8 == 4 else KB + 4) if _am_by_rows(KB) else KB
+
+
+def _rows16_bytes(K):
+    return 16 * _row_stride(K) + _al(16 * _am_stride(K // 64) * 4, 16)
+
+
+def _plan(M, k, E, H, I, r):
+    KB, KBI = H // 64, I // 64
+    spw = -(-((KB + 1) // 2) // 8)
+    gu, dn = _rows16_bytes(H), _rows16_bytes(I)
+    dpe = max(1, min(gu // dn, 64 // KBI))
+    ppw = -(-(dpe * KBI) // 16)
+    slot = _al(max(gu, dpe * dn), 128)
+    S = M * k
+    o = 256 * 32 * 4 + 2 * 2 * 8 * 32 * 16
+    for n in (S * 4, S * 4, E * 4, S * 4, S * 8 * 4):
+        o = _al(o + n, 16)
+    if r:
+        o = _al(o + S * r * 4, 16)
+    fixed = _al(o, 128) + 2 * 32 * 8
+    stages = min((SMEM_LIMIT - fixed) // slot, 32) & ~1
+    ring = _al(_al(o + 2 * stages * 8, 16), 128)
+    return dict(spw=spw, ppw=ppw, dpe=dpe, slot=slot, stages=stages, ring=ring, total=ring + stages * slot)
+
+
+def _copies_rows16(K, row_a, row_b):
+    """(dst offset, src byte offset in packed, src byte offset in absmax, bytes) of one block of 16 rows."""
+    KB = K // 64
+    ps, sa = _row_stride(K), _am_stride(KB)
+    am = 16 * ps
+    pk, ab = [], []
+    for lane in range(16):
+        row = (row_a if lane < 8 else row_b) + (lane & 7)
+        pk.append((lane * ps, row * (K // 2), K // 2))
+    if _am_by_rows(KB):
+        for i in range(16):
+            row = (row_a if i < 8 else row_b) + (i & 7)
+            ab.append((am + i * sa * 4, row * KB * 4, KB * 4))
+    else:
+        for i in range(2):
+            ab.append((am + i * 8 * sa * 4, (row_a if i == 0 else row_b) * KB * 4, 8 * KB * 4))
+    return pk, ab
+
+
+DECODE_SHAPES = [
+    # (M, k, E, H, I, r): the decode rows of the bench and every decode shape the GPU tests run
+    (1, 8, 64, 2048, 1024, 0), (4, 8, 64, 2048, 1024, 0), (8, 8, 64, 2048, 1024, 0),
+    (1, 4, 32, 2880, 2880, 0), (8, 4, 32, 2880, 2880, 0), (8, 8, 128, 2048, 768, 8), (3, 8, 128, 2048, 768, 8),
+    (1, 2, 8, 256, 128, 0), (8, 2, 8, 256, 128, 0), (5, 3, 12, 192, 320, 0), (3, 2, 6, 128, 192, 8),
+    (2, 6, 40, 448, 128, 0), (7, 32, 33, 128, 64, 0), (8, 2, 8, 2880, 704, 0), (8, 2, 8, 4096, 128, 0),
+    (8, 8, 512, 128, 64, 0), (6, 1, 8, 256, 192, 0), (7, 4, 4, 256, 192, 0), (5, 3, 12, 192, 320, 0),
+    (4, 2, 4, 4096, 4096, 16),
+]
+
+
+@pytest.mark.parametrize("shape", DECODE_SHAPES)
+def test_decode_fused_plan_copies_and_reads_stay_in_bounds(shape):
+    """Every bulk copy of a stage is 16-byte aligned at both ends, a multiple of
+    16 bytes, inside its slot and inside the source stack; the transaction
+    count equals the bytes copied; every fragment and absmax read of the math
+    warps stays inside the bytes the copies wrote; the plan fits the shared
+    memory and holds an even number of stages."""
+    M, k, E, H, I, r = shape
+    pl = _plan(M, k, E, H, I, r)
+    assert pl["total"] <= SMEM_LIMIT and pl["stages"] >= 2 and pl["stages"] % 2 == 0
+    assert pl["spw"] <= 4 and pl["ppw"] <= 4 and pl["ring"] % 128 == 0 and pl["slot"] % 128 == 0
+    KB, KBI = H // 64, I // 64
+    # phase 1: every item of the largest expert id (the last rows of the stack)
+    gu_rows, gu_bytes = 2 * I * E, None
+    for rb in (0, I // 8 - 1):
+        grow = (E - 1) * 2 * I + rb * 8
+        pk, ab = _copies_rows16(H, grow, grow + I)
+        written = set()
+        for dst, src, n in pk:
+            assert dst % 16 == 0 and src % 16 == 0 and n % 16 == 0 and dst + n <= pl["slot"]
+            assert src + n <= gu_rows * (H // 2)
+            written.update(range(dst, dst + n))
+        for dst, src, n in ab:
+            assert dst % 16 == 0 and src % 16 == 0 and n % 16 == 0 and dst + n <= pl["slot"]
+            assert src + n <= gu_rows * KB * 4
+            written.update(range(dst, dst + n))
+        assert sum(n for _, _, n in pk + ab) == 16 * (H // 2) + 16 * KB * 4
+        ps, sa, am = _row_stride(H), _am_stride(KB), 16 * _row_stride(H)
+        for g in range(8):
+            for t in range(4):
+                for kb in range(KB):
+                    for row in (g, g + 8):
+                        off = row * ps + kb * 32 + 8 * t
+                        assert set(range(off, off + 8)) <= written
+                        a = am + (row * sa + kb) * 4
+                        assert set(range(a, a + 4)) <= written
+    # phase 2: the last row block of the last experts
+    dn = _rows16_bytes(I)
+    for ne in range(1, pl["dpe"] + 1):
+        total = 0
+        for ei in range(ne):
+            row0 = (E - 1 - ei) * H + (H // 16 - 1) * 16
+            pk, ab = _copies_rows16(I, row0, row0 + 8)
+            for dst, src, n in pk + ab:
+                dst += ei * dn
+                assert dst % 16 == 0 and src % 16 == 0 and n % 16 == 0 and dst + n <= pl["slot"]
+                total += n
+            assert max(src + n for _, src, n in pk) <= E * H * (I // 2)
+            assert max(src + n for _, src, n in ab) <= E * H * KBI * 4
+        assert total == ne * (16 * (I // 2) + 16 * KBI * 4)
+        assert ne * KBI <= 16 * pl["ppw"]
+
+
+@pytest.mark.parametrize("K", [128, 192, 320, 448, 704, 768, 1024, 2048, 2880, 4096])
+def test_decode_fused_fragment_reads_are_conflict_free(K):
+    """Rows staged 32 mod 128 bytes apart: the 8-byte fragment loads of each
+    half-warp (rows g = 4h .. 4h+3, t = 0..3) hit 32 distinct banks, and the
+    absmax loads of the 8 rows g fall on 8 distinct banks."""
+    ps, sa = _row_stride(K), _am_stride(K // 64)
+    assert ps % 128 == 32 and ps >= K // 2
+    for kb in range(K // 64):
+        for half in range(2):
+            banks = []
+            for g in range(4 * half, 4 * half + 4):
+                for t in range(4):
+                    w = (g * ps + kb * 32 + 8 * t) // 4
+                    banks += [w % 32, (w + 1) % 32]
+            assert len(set(banks)) == 32
+        assert len({(g * sa + kb) % 32 for g in range(8)}) == 8
 
 
 def test_warp_mma_gemm_fragment_mapping():
