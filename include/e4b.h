@@ -224,6 +224,37 @@ E4B_API e4b_status e4b_grouped_nf4_gemm(const uint16_t* A, int64_t a_rows, int64
                                 e4b_dtype out_dtype, void* workspace, size_t workspace_bytes,
                                 e4b_stream stream);
 
+/*
+ * Backward through the frozen base -- the input gradient of the grouped NF4
+ * GEMM above, in one launch over all groups.
+ * Source: experts4bit-qlora 0.22.0, "Which training path?" (the backward's
+ * dgrad runs as one launch instead of a per-expert decode loop; the frozen
+ * base is decoded again from the packed bytes, never kept dequantised).
+ *
+ * Row p (0 <= p < total_rows) of group e computes
+ *     dx[p, :] = dY[row_index[p], :] . W_e                       (K values)
+ *     dx[p, :] += lora_scale * (dY[row_index[p], :] . lora_B[e]) . lora_A[e]
+ * with W_e expert e's [N, K] NF4 matrix as in e4b_grouped_nf4_gemm(): for a
+ * forward y = a . W_e^T (+ adapter), dx is the gradient of <dY, y> by a.
+ *
+ * dY              [dy_rows, lddy] bf16 (lddy >= N, lddy % 8 == 0).
+ * row_index       [total_rows] int32 indices into dY, or NULL for p itself.
+ * expert_offsets, packed, absmax, lora_A, lora_B: as in e4b_grouped_nf4_gemm().
+ * out             [total_rows, K] of out_dtype.
+ * Requires K % 64 == 0, N % 64 == 0, 0 <= r <= 16, total_rows < 2^31.
+ * workspace       e4b_grouped_nf4_gemm_dgrad_workspace_size() bytes: an error
+ *                 word and the products dY . lora_B (total_rows x r fp32).
+ * Groups with no rows cost nothing and write nothing.
+ */
+E4B_API size_t e4b_grouped_nf4_gemm_dgrad_workspace_size(int64_t total_rows, int64_t N, int64_t K, int r);
+E4B_API e4b_status e4b_grouped_nf4_gemm_dgrad(const uint16_t* dY, int64_t dy_rows, int64_t lddy,
+                                      const int32_t* row_index, const int32_t* expert_offsets,
+                                      int64_t E, int64_t total_rows, const uint8_t* packed,
+                                      const float* absmax, int64_t N, int64_t K,
+                                      const uint16_t* lora_A, const uint16_t* lora_B, int r,
+                                      float lora_scale, void* out, e4b_dtype out_dtype,
+                                      void* workspace, size_t workspace_bytes, e4b_stream stream);
+
 /* The two packed stacks of one MoE layer (device pointers), plus its adapter. */
 typedef struct {
   const uint8_t* gu_packed; /* [E, 2I*H/2]  gate_up_proj, NF4 */

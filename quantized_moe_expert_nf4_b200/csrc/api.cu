@@ -393,6 +393,71 @@ e4b_status e4b_grouped_nf4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda, 
   return E4B_OK;
 }
 
+size_t e4b_grouped_nf4_gemm_dgrad_workspace_size(int64_t total_rows, int64_t N, int64_t K, int r) {
+  (void)N;
+  (void)K;
+  if (total_rows < 0 || r < 0) return 0;
+  return dgrad_workspace_bytes(total_rows, r);
+}
+
+e4b_status e4b_grouped_nf4_gemm_dgrad(const uint16_t* dY, int64_t dy_rows, int64_t lddy, const int32_t* row_index,
+                                      const int32_t* expert_offsets, int64_t E, int64_t total_rows,
+                                      const uint8_t* packed, const float* absmax, int64_t N, int64_t K,
+                                      const uint16_t* lora_A, const uint16_t* lora_B, int r, float lora_scale,
+                                      void* out, e4b_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                                      e4b_stream stream) {
+  begin_call();
+  if (E < 1 || E > 65536) return fail(E4B_ERR_INVALID_ARGUMENT, "E must be in [1, 65536]");
+  if (total_rows < 0 || dy_rows < 0) return fail(E4B_ERR_INVALID_ARGUMENT, "total_rows and dy_rows must be >= 0");
+  if (total_rows > 0 && dy_rows < 1) return fail(E4B_ERR_INVALID_ARGUMENT, "dy_rows must be >= 1 when rows exist");
+  if (K < 64 || K % 64 != 0) return fail(E4B_ERR_UNSUPPORTED, "K must be a positive multiple of 64");
+  if (N < 64 || N % 64 != 0) return fail(E4B_ERR_UNSUPPORTED, "N must be a positive multiple of 64");
+  if (lddy < N || lddy % 8 != 0) return fail(E4B_ERR_INVALID_ARGUMENT, "lddy must be >= N and a multiple of 8");
+  if (out_dtype != E4B_F32 && out_dtype != E4B_BF16) return fail(E4B_ERR_INVALID_ARGUMENT, "out_dtype must be F32 or BF16");
+  if ((lora_A == nullptr) != (lora_B == nullptr))
+    return fail(E4B_ERR_INVALID_ARGUMENT, "lora_A and lora_B must be both set or both NULL");
+  if (lora_A && (r < 1 || r > 16)) return fail(E4B_ERR_UNSUPPORTED, "LoRA rank must be in [1, 16]");
+  if (!lora_A) r = 0;
+  if (!expert_offsets || !packed || !absmax) return fail(E4B_ERR_INVALID_ARGUMENT, "null expert_offsets, packed or absmax");
+  if (total_rows > 0 && (!dY || !out)) return fail(E4B_ERR_INVALID_ARGUMENT, "null dY or out");
+  if (total_rows > INT32_MAX) return fail(E4B_ERR_UNSUPPORTED, "total_rows exceeds int32");
+  if ((dY && !aligned16(dY)) || !aligned16(packed) || !aligned16(absmax) || (out && !aligned16(out)))
+    return fail(E4B_ERR_INVALID_ARGUMENT, "dY, packed, absmax and out must be 16-byte aligned");
+  if (lora_A && (!aligned16(lora_A) || !aligned16(lora_B)))
+    return fail(E4B_ERR_INVALID_ARGUMENT, "lora_A and lora_B must be 16-byte aligned");
+  if (e4b_status s = check_workspace("dgrad", dgrad_workspace_bytes(total_rows, r), workspace, workspace_bytes);
+      s != E4B_OK)
+    return s;
+  if (e4b_status s = check_device(); s != E4B_OK) return s;
+  if (total_rows == 0) {
+    set_path("dgrad.empty");
+    return E4B_OK;
+  }
+  DgradArgs d{};
+  d.dY = dY;
+  d.dy_rows = dy_rows;
+  d.lddy = lddy;
+  d.row_index = row_index;
+  d.offsets = expert_offsets;
+  d.E = static_cast<int>(E);
+  d.total_rows = total_rows;
+  d.packed = packed;
+  d.absmax = absmax;
+  d.N = static_cast<int>(N);
+  d.K = static_cast<int>(K);
+  d.lora_A = r ? lora_A : nullptr;
+  d.lora_B = r ? lora_B : nullptr;
+  d.r = r;
+  d.lora_scale = lora_scale;
+  d.yb = r ? reinterpret_cast<float*>(static_cast<char*>(workspace) + dgrad_workspace_yb_offset()) : nullptr;
+  d.out = out;
+  d.out_bf16 = out_dtype == E4B_BF16;
+  cudaError_t err = launch_grouped_dgrad(d, reinterpret_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "grouped dgrad launch");
+  set_path("dgrad.mma");
+  return E4B_OK;
+}
+
 static e4b_status check_stack(const e4b_expert_stack* w, int k) {
   if (!w) return fail(E4B_ERR_INVALID_ARGUMENT, "null expert stack");
   if (w->E < 1 || w->E > 1024) return fail(E4B_ERR_UNSUPPORTED, "E must be in [1, 1024]");

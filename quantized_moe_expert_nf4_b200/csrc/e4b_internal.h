@@ -97,6 +97,30 @@ cudaError_t launch_tc_lora_prep(const GemmArgs& a, cudaStream_t stream);
 // Picks the implementation; reports the path name through set_path.
 cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const char** path);
 
+// ---- grouped dgrad ---------------------------------------------------------
+struct DgradArgs {
+  const uint16_t* dY;
+  int64_t dy_rows, lddy;
+  const int32_t* row_index;  // nullable
+  const int32_t* offsets;    // [E+1]
+  int E;
+  int64_t total_rows;
+  const uint8_t* packed;
+  const float* absmax;
+  int N, K;
+  const uint16_t* lora_A;  // [E, r, K] or nullptr
+  const uint16_t* lora_B;  // [E, N, r] or nullptr
+  int r;
+  float lora_scale;
+  float* yb;  // workspace [total_rows, r] fp32: dY . lora_B
+  void* out;  // [total_rows, K]
+  bool out_bf16;
+};
+// Workspace: [error word, 256 B][dY . lora_B, total_rows * r fp32, 256-B aligned].
+size_t dgrad_workspace_bytes(int64_t total_rows, int r);
+size_t dgrad_workspace_yb_offset();
+cudaError_t launch_grouped_dgrad(const DgradArgs& a, cudaStream_t stream);
+
 // ---- combine ---------------------------------------------------------------
 cudaError_t launch_combine(const uint16_t* z, const int32_t* inv, const float* w, int64_t M, int k,
                            int H, uint16_t* out, cudaStream_t stream);

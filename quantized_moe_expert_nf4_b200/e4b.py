@@ -35,6 +35,7 @@ EXPORTED = (
     "e4b_nf4_quantize_stack",
     "e4b_moe_route_permute_workspace_size", "e4b_moe_route_permute",
     "e4b_grouped_nf4_gemm_workspace_size", "e4b_grouped_nf4_gemm",
+    "e4b_grouped_nf4_gemm_dgrad_workspace_size", "e4b_grouped_nf4_gemm_dgrad",
     "e4b_moe_expert_forward_workspace_size", "e4b_moe_expert_forward",
     "e4b_moe_expert_forward_path", "e4b_moe_expert_forward_decode_noalloc",
 )
@@ -96,6 +97,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.e4b_grouped_nf4_gemm.restype = i32
     lib.e4b_grouped_nf4_gemm.argtypes = [vp, i64, i64, vp, vp, i64, i64, vp, vp, i64, i64, vp, vp, i32,
                                          ctypes.c_float, i32, vp, i32, vp, sz, vp]
+    lib.e4b_grouped_nf4_gemm_dgrad_workspace_size.restype = sz
+    lib.e4b_grouped_nf4_gemm_dgrad_workspace_size.argtypes = [i64, i64, i64, i32]
+    lib.e4b_grouped_nf4_gemm_dgrad.restype = i32
+    lib.e4b_grouped_nf4_gemm_dgrad.argtypes = [vp, i64, i64, vp, vp, i64, i64, vp, vp, i64, i64, vp, vp, i32,
+                                               ctypes.c_float, vp, i32, vp, sz, vp]
     lib.e4b_moe_expert_forward_workspace_size.restype = sz
     lib.e4b_moe_expert_forward_workspace_size.argtypes = [i64, ctypes.POINTER(ExpertStackC), i32]
     lib.e4b_moe_expert_forward.restype = i32
@@ -238,6 +244,42 @@ def e4b_grouped_nf4_gemm(A: torch.Tensor, row_index: Optional[torch.Tensor], exp
         A.data_ptr(), A.shape[0], A.stride(0), _ptr(row_index), expert_offsets.data_ptr(), E, total_rows,
         packed.data_ptr(), absmax.data_ptr(), N, K, _ptr(lora_A), _ptr(lora_B), r, float(lora_scale), epi,
         out.data_ptr(), od, _ptr(workspace), ws, _stream(stream)), "e4b_grouped_nf4_gemm")
+
+
+def e4b_grouped_nf4_gemm_dgrad_workspace_size(total_rows: int, N: int, K: int, r: int = 0) -> int:
+    return int(load_library().e4b_grouped_nf4_gemm_dgrad_workspace_size(total_rows, N, K, r))
+
+
+def e4b_grouped_nf4_gemm_dgrad(dY: torch.Tensor, row_index: Optional[torch.Tensor], expert_offsets: torch.Tensor,
+                               total_rows: int, packed: torch.Tensor, absmax: torch.Tensor, N: int, K: int,
+                               out: torch.Tensor, lora_A: Optional[torch.Tensor] = None,
+                               lora_B: Optional[torch.Tensor] = None, lora_scale: float = 0.0,
+                               workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """out[p] = dY[row_index[p]] . W_e (+ lora_scale * (dY . lora_B[e]) . lora_A[e]), [total_rows, K]."""
+    if dY.dim() != 2 or dY.dtype != torch.bfloat16 or not dY.is_cuda or dY.stride(1) != 1:
+        raise ValueError("dY must be a 2-D bf16 CUDA tensor with unit column stride")
+    _dev(expert_offsets, "expert_offsets", torch.int32)
+    _dev(packed, "packed", torch.uint8)
+    _dev(absmax, "absmax", torch.float32)
+    _dev(out, "out")
+    if row_index is not None:
+        _dev(row_index, "row_index", torch.int32)
+    E = expert_offsets.numel() - 1
+    r = 0
+    if lora_A is not None:
+        _dev(lora_A, "lora_A", torch.bfloat16)
+        _dev(lora_B, "lora_B", torch.bfloat16)
+        r = lora_A.shape[1]
+    od = {torch.float32: E4B_F32, torch.bfloat16: E4B_BF16}.get(out.dtype)
+    if od is None:
+        raise ValueError("out must be float32 or bfloat16")
+    if out.numel() < total_rows * K:
+        raise ValueError("out too small")
+    ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load_library().e4b_grouped_nf4_gemm_dgrad(
+        dY.data_ptr(), dY.shape[0], dY.stride(0), _ptr(row_index), expert_offsets.data_ptr(), E, total_rows,
+        packed.data_ptr(), absmax.data_ptr(), N, K, _ptr(lora_A), _ptr(lora_B), r, float(lora_scale),
+        out.data_ptr(), od, _ptr(workspace), ws, _stream(stream)), "e4b_grouped_nf4_gemm_dgrad")
 
 
 class ExpertStack:

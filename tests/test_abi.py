@@ -144,3 +144,30 @@ def test_error_word_calls_check_their_arguments_on_the_host(lib):
     assert lib.e4b_workspace_clear_error(None, None) == 1
     assert code.value == 7   # untouched on a rejected call
 
+
+
+def test_dgrad_host_side_rejections(lib):
+    """The grouped dgrad checks its arguments before any device query."""
+    p = ctypes.c_void_p(1 << 20)
+    rows, N, K = 64, 128, 192
+    need = e4b.e4b_grouped_nf4_gemm_dgrad_workspace_size(rows, N, K, 0)
+    assert need == 256                                   # error word only without an adapter
+    assert e4b.e4b_grouped_nf4_gemm_dgrad_workspace_size(rows, N, K, 8) == 256 + (rows * 8 * 4 + 255) // 256 * 256
+
+    def call(**kw):
+        a = dict(dY=p, dy_rows=rows, lddy=N, ridx=None, offs=p, E=2, rows=rows, packed=p, absmax=p, N=N, K=K,
+                 la=None, lb=None, r=0, scale=0.0, out=p, od=0, ws=p, wsb=need)
+        a.update(kw)
+        return lib.e4b_grouped_nf4_gemm_dgrad(a["dY"], a["dy_rows"], a["lddy"], a["ridx"], a["offs"], a["E"],
+                                              a["rows"], a["packed"], a["absmax"], a["N"], a["K"], a["la"],
+                                              a["lb"], a["r"], a["scale"], a["out"], a["od"], a["ws"], a["wsb"],
+                                              None)
+    assert call(K=96) == 2 and b"K must be" in lib.e4b_last_error()
+    assert call(N=100) == 2 and b"N must be" in lib.e4b_last_error()
+    assert call(lddy=N - 8) == 1 and b"lddy" in lib.e4b_last_error()
+    assert call(lddy=N + 4) == 1 and b"lddy" in lib.e4b_last_error()
+    assert call(la=p) == 1 and b"both set" in lib.e4b_last_error()
+    assert call(la=p, lb=p, r=17) == 2 and b"rank" in lib.e4b_last_error()
+    assert call(absmax=ctypes.c_void_p((1 << 20) + 4)) == 1 and b"16-byte aligned" in lib.e4b_last_error()
+    assert call(wsb=need - 1) == 3 and str(need).encode() in lib.e4b_last_error()
+    assert call(ws=ctypes.c_void_p((1 << 20) + 8)) == 1 and b"dgrad workspace must be" in lib.e4b_last_error()
