@@ -255,6 +255,34 @@ E4B_API e4b_status e4b_grouped_nf4_gemm_dgrad(const uint16_t* dY, int64_t dy_row
                                       float lora_scale, void* out, e4b_dtype out_dtype,
                                       void* workspace, size_t workspace_bytes, e4b_stream stream);
 
+/*
+ * The adapter's gradients of one grouped projection (backward of the
+ * per-expert LoRA delta over the frozen NF4 base).
+ * Source: Solutions -- one page per problem, the ExpertsLoRA row (a per-expert
+ * low-rank delta before each routed expert's activation, trained over the
+ * frozen stack); experts4bit-qlora 0.22.0, "Which training path?".
+ *
+ * For the forward y_p = x_p . W_e^T + s (x_p . A_e^T) . B_e^T of
+ * e4b_grouped_nf4_gemm() (x_p = x[row_index[p]]) and the gradient da of its
+ * output rows (group order, [total_rows, ldda]):
+ *     dB_e = s * sum_{p in e} da_p^T (x_p . A_e^T)          [N, r] fp32
+ *     dA_e = s * sum_{p in e} (da_p . B_e)^T x_p            [r, K] fp32
+ * summed over each group's rows in order (deterministic); experts without rows
+ * get zeros.  x [x_rows, ldx] bf16 (ldx >= K, ldx % 8 == 0), da bf16,
+ * lora_A [E, r, K], lora_B [E, N, r] bf16, dA [E, r, K], dB [E, N, r] fp32.
+ * Requires K % 64 == 0, N % 64 == 0, 1 <= r <= 16.
+ * workspace       e4b_grouped_lora_grads_workspace_size() bytes: an error
+ *                 word and the products x . A^T and da . B (total_rows x r fp32 each).
+ */
+E4B_API size_t e4b_grouped_lora_grads_workspace_size(int64_t total_rows, int r);
+E4B_API e4b_status e4b_grouped_lora_grads(const uint16_t* x, int64_t x_rows, int64_t ldx,
+                                  const int32_t* row_index, const int32_t* expert_offsets,
+                                  int64_t E, int64_t total_rows, const uint16_t* da, int64_t ldda,
+                                  int64_t N, int64_t K, const uint16_t* lora_A,
+                                  const uint16_t* lora_B, int r, float lora_scale, float* dA,
+                                  float* dB, void* workspace, size_t workspace_bytes,
+                                  e4b_stream stream);
+
 /* The two packed stacks of one MoE layer (device pointers), plus its adapter. */
 typedef struct {
   const uint8_t* gu_packed; /* [E, 2I*H/2]  gate_up_proj, NF4 */

@@ -458,6 +458,96 @@ e4b_status e4b_grouped_nf4_gemm_dgrad(const uint16_t* dY, int64_t dy_rows, int64
   return E4B_OK;
 }
 
+size_t e4b_grouped_lora_grads_workspace_size(int64_t total_rows, int r) {
+  if (total_rows < 0 || r < 1 || r > 16) return 0;
+  return lora_grads_workspace_bytes(total_rows, r);
+}
+
+e4b_status e4b_grouped_lora_grads(const uint16_t* x, int64_t x_rows, int64_t ldx, const int32_t* row_index,
+                                  const int32_t* expert_offsets, int64_t E, int64_t total_rows, const uint16_t* da,
+                                  int64_t ldda, int64_t N, int64_t K, const uint16_t* lora_A,
+                                  const uint16_t* lora_B, int r, float lora_scale, float* dA, float* dB,
+                                  void* workspace, size_t workspace_bytes, e4b_stream stream) {
+  begin_call();
+  if (E < 1 || E > 65536) return fail(E4B_ERR_INVALID_ARGUMENT, "E must be in [1, 65536]");
+  if (total_rows < 0 || x_rows < 0) return fail(E4B_ERR_INVALID_ARGUMENT, "total_rows and x_rows must be >= 0");
+  if (total_rows > 0 && x_rows < 1) return fail(E4B_ERR_INVALID_ARGUMENT, "x_rows must be >= 1 when rows exist");
+  if (K < 64 || K % 64 != 0) return fail(E4B_ERR_UNSUPPORTED, "K must be a positive multiple of 64");
+  if (N < 64 || N % 64 != 0) return fail(E4B_ERR_UNSUPPORTED, "N must be a positive multiple of 64");
+  if (r < 1 || r > 16) return fail(E4B_ERR_UNSUPPORTED, "LoRA rank must be in [1, 16]");
+  if (ldx < K || ldx % 8 != 0) return fail(E4B_ERR_INVALID_ARGUMENT, "ldx must be >= K and a multiple of 8");
+  if (ldda < N) return fail(E4B_ERR_INVALID_ARGUMENT, "ldda must be >= N");
+  if (!expert_offsets || !lora_A || !lora_B || !dA || !dB)
+    return fail(E4B_ERR_INVALID_ARGUMENT, "null expert_offsets, lora_A, lora_B, dA or dB");
+  if (total_rows > 0 && (!x || !da)) return fail(E4B_ERR_INVALID_ARGUMENT, "null x or da");
+  if (total_rows > INT32_MAX) return fail(E4B_ERR_UNSUPPORTED, "total_rows exceeds int32");
+  if ((x && !aligned16(x)) || !aligned16(lora_A) || !aligned16(lora_B) || !aligned16(dA) || !aligned16(dB) ||
+      (da && !aligned16(da)))
+    return fail(E4B_ERR_INVALID_ARGUMENT, "x, da, lora_A, lora_B, dA and dB must be 16-byte aligned");
+  if (e4b_status s = check_workspace("lora grads", lora_grads_workspace_bytes(total_rows, r), workspace,
+                                     workspace_bytes);
+      s != E4B_OK)
+    return s;
+  if (e4b_status s = check_device(); s != E4B_OK) return s;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  float* xa = reinterpret_cast<float*>(static_cast<char*>(workspace) + 256);
+  float* yb = reinterpret_cast<float*>(static_cast<char*>(workspace) + lora_grads_workspace_yb_offset(total_rows, r));
+  if (total_rows > 0) {
+    GemmArgs g{};
+    g.A = x;
+    g.a_rows = x_rows;
+    g.lda = ldx;
+    g.row_index = row_index;
+    g.offsets = expert_offsets;
+    g.E = static_cast<int>(E);
+    g.total_rows = total_rows;
+    g.N = static_cast<int>(N);
+    g.K = static_cast<int>(K);
+    g.lora_A = lora_A;
+    g.lora_B = lora_B;
+    g.r = r;
+    g.xa = xa;
+    cudaError_t err = launch_lora_xa(g, st);
+    if (err != cudaSuccess) return cuda_fail(err, "lora grads: x . A^T");
+    DgradArgs d{};
+    d.dY = da;
+    d.dy_rows = total_rows;
+    d.lddy = ldda;
+    d.offsets = expert_offsets;
+    d.E = static_cast<int>(E);
+    d.total_rows = total_rows;
+    d.N = static_cast<int>(N);
+    d.K = static_cast<int>(K);
+    d.lora_B = lora_B;
+    d.r = r;
+    d.yb = yb;
+    err = launch_dgrad_lora_yb(d, st);
+    if (err != cudaSuccess) return cuda_fail(err, "lora grads: da . B");
+  }
+  LoraGradArgs a{};
+  a.x = x;
+  a.x_rows = x_rows;
+  a.ldx = ldx;
+  a.row_index = row_index;
+  a.offsets = expert_offsets;
+  a.E = static_cast<int>(E);
+  a.total_rows = total_rows;
+  a.da = da;
+  a.ldda = ldda;
+  a.N = static_cast<int>(N);
+  a.K = static_cast<int>(K);
+  a.r = r;
+  a.lora_scale = lora_scale;
+  a.xa = xa;
+  a.yb = yb;
+  a.dA = dA;
+  a.dB = dB;
+  cudaError_t err = launch_lora_grads(a, st);
+  if (err != cudaSuccess) return cuda_fail(err, "lora grads launch");
+  set_path("lora_grads");
+  return E4B_OK;
+}
+
 static e4b_status check_stack(const e4b_expert_stack* w, int k) {
   if (!w) return fail(E4B_ERR_INVALID_ARGUMENT, "null expert stack");
   if (w->E < 1 || w->E > 1024) return fail(E4B_ERR_UNSUPPORTED, "E must be in [1, 1024]");

@@ -234,20 +234,105 @@ __global__ void __launch_bounds__(256) dgrad_lora_yb_kernel(DgradArgs a) {
   }
 }
 
+// Adapter gradients of one grouped projection, from xa = x . A_e^T and
+// yb = da . B_e (both [total_rows, r] fp32), summed over each group's rows in
+// row order (deterministic).  One thread per output row n (dB) or column k
+// (dA), r accumulators each; experts without rows write zeros.
+__global__ void __launch_bounds__(128) lora_grad_b_kernel(LoraGradArgs a) {
+  constexpr int kMaxR = 16;
+  const int e = blockIdx.x;
+  const int n = blockIdx.y * 128 + threadIdx.x;
+  const int64_t lo = clampv<int64_t>(a.offsets[e], 0, a.total_rows);
+  const int64_t hi = max(lo, clampv<int64_t>(a.offsets[e + 1], 0, a.total_rows));
+  float acc[kMaxR];
+#pragma unroll
+  for (int rr = 0; rr < kMaxR; ++rr) acc[rr] = 0.f;
+  if (n < a.N) {
+    for (int64_t p = lo; p < hi; ++p) {
+      const float d = bf16_bits_to_float(a.da[p * a.ldda + n]);
+#pragma unroll
+      for (int rr = 0; rr < kMaxR; ++rr) {
+        if (rr >= a.r) break;
+        acc[rr] = fmaf(d, a.xa[p * a.r + rr], acc[rr]);
+      }
+    }
+    float* out = a.dB + (static_cast<int64_t>(e) * a.N + n) * a.r;
+#pragma unroll
+    for (int rr = 0; rr < kMaxR; ++rr) {
+      if (rr >= a.r) break;
+      out[rr] = a.lora_scale * acc[rr];
+    }
+  }
+}
+
+__global__ void __launch_bounds__(128) lora_grad_a_kernel(LoraGradArgs a) {
+  constexpr int kMaxR = 16;
+  const int e = blockIdx.x;
+  const int k = blockIdx.y * 128 + threadIdx.x;
+  const int64_t lo = clampv<int64_t>(a.offsets[e], 0, a.total_rows);
+  const int64_t hi = max(lo, clampv<int64_t>(a.offsets[e + 1], 0, a.total_rows));
+  float acc[kMaxR];
+#pragma unroll
+  for (int rr = 0; rr < kMaxR; ++rr) acc[rr] = 0.f;
+  if (k < a.K) {
+    for (int64_t p = lo; p < hi; ++p) {
+      int64_t src = a.row_index ? a.row_index[p] : p;
+      src = clampv<int64_t>(src, 0, a.x_rows - 1);
+      const float xv = bf16_bits_to_float(a.x[src * a.ldx + k]);
+#pragma unroll
+      for (int rr = 0; rr < kMaxR; ++rr) {
+        if (rr >= a.r) break;
+        acc[rr] = fmaf(a.yb[p * a.r + rr], xv, acc[rr]);
+      }
+    }
+#pragma unroll
+    for (int rr = 0; rr < kMaxR; ++rr) {
+      if (rr >= a.r) break;
+      a.dA[(static_cast<int64_t>(e) * a.r + rr) * a.K + k] = a.lora_scale * acc[rr];
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_dgrad_lora_yb(const DgradArgs& a, cudaStream_t stream) {
+  if (a.total_rows == 0) return cudaSuccess;
+  const int grid = static_cast<int>((a.total_rows * 32 + 255) / 256);
+  LaunchScope ls("dgrad.lora_yb", stream);
+  dgrad_lora_yb_kernel<<<grid, 256, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lora_grads(const LoraGradArgs& a, cudaStream_t stream) {
+  {
+    dim3 grid(static_cast<unsigned>(a.E), static_cast<unsigned>((a.N + 127) / 128));
+    LaunchScope ls("lora_grad.b", stream);
+    lora_grad_b_kernel<<<grid, 128, 0, stream>>>(a);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
+  dim3 grid(static_cast<unsigned>(a.E), static_cast<unsigned>((a.K + 127) / 128));
+  LaunchScope ls("lora_grad.a", stream);
+  lora_grad_a_kernel<<<grid, 128, 0, stream>>>(a);
+  return cudaGetLastError();
+}
 
 size_t dgrad_workspace_yb_offset() { return 256; }
 size_t dgrad_workspace_bytes(int64_t total_rows, int r) {
   return 256 + align_up(r > 0 ? static_cast<size_t>(total_rows) * r * sizeof(float) : 0, 256);
 }
 
+size_t lora_grads_workspace_yb_offset(int64_t total_rows, int r) {
+  return 256 + align_up(static_cast<size_t>(total_rows) * r * sizeof(float), 256);
+}
+size_t lora_grads_workspace_bytes(int64_t total_rows, int r) {
+  return lora_grads_workspace_yb_offset(total_rows, r) + align_up(static_cast<size_t>(total_rows) * r * sizeof(float), 256);
+}
+
 cudaError_t launch_grouped_dgrad(const DgradArgs& a, cudaStream_t stream) {
   if (a.total_rows == 0) return cudaSuccess;
   if (a.lora_A && a.r > 0) {
-    const int grid = static_cast<int>((a.total_rows * 32 + 255) / 256);
-    LaunchScope ls("dgrad.lora_yb", stream);
-    dgrad_lora_yb_kernel<<<grid, 256, 0, stream>>>(a);
-    cudaError_t err = cudaGetLastError();
+    cudaError_t err = launch_dgrad_lora_yb(a, stream);
     if (err != cudaSuccess) return err;
   }
   // Upper bound on routed-row tiles: ceil(total/64) + number of non-empty groups.

@@ -120,6 +120,30 @@ struct DgradArgs {
 size_t dgrad_workspace_bytes(int64_t total_rows, int r);
 size_t dgrad_workspace_yb_offset();
 cudaError_t launch_grouped_dgrad(const DgradArgs& a, cudaStream_t stream);
+// yb = dY . lora_B per routed row (into a.yb); a.lora_B, a.r, a.N, a.dY, a.lddy used.
+cudaError_t launch_dgrad_lora_yb(const DgradArgs& a, cudaStream_t stream);
+
+// ---- grouped LoRA gradients ---------------------------------------------------
+struct LoraGradArgs {
+  const uint16_t* x;  // input rows of the projection (gathered by row_index)
+  int64_t x_rows, ldx;
+  const int32_t* row_index;  // nullable
+  const int32_t* offsets;    // [E+1]
+  int E;
+  int64_t total_rows;
+  const uint16_t* da;  // [total_rows, ldda] gradient of the projection's output rows
+  int64_t ldda;
+  int N, K, r;
+  float lora_scale;
+  const float* xa;  // [total_rows, r] x . A_e^T
+  const float* yb;  // [total_rows, r] da . B_e
+  float* dA;        // [E, r, K]
+  float* dB;        // [E, N, r]
+};
+// Workspace: [error word, 256 B][xa, total_rows * r fp32][yb, total_rows * r fp32], 256-B aligned parts.
+size_t lora_grads_workspace_bytes(int64_t total_rows, int r);
+size_t lora_grads_workspace_yb_offset(int64_t total_rows, int r);
+cudaError_t launch_lora_grads(const LoraGradArgs& a, cudaStream_t stream);
 
 // ---- combine ---------------------------------------------------------------
 cudaError_t launch_combine(const uint16_t* z, const int32_t* inv, const float* w, int64_t M, int k,

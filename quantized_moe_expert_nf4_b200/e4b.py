@@ -36,6 +36,7 @@ EXPORTED = (
     "e4b_moe_route_permute_workspace_size", "e4b_moe_route_permute",
     "e4b_grouped_nf4_gemm_workspace_size", "e4b_grouped_nf4_gemm",
     "e4b_grouped_nf4_gemm_dgrad_workspace_size", "e4b_grouped_nf4_gemm_dgrad",
+    "e4b_grouped_lora_grads_workspace_size", "e4b_grouped_lora_grads",
     "e4b_moe_expert_forward_workspace_size", "e4b_moe_expert_forward",
     "e4b_moe_expert_forward_path", "e4b_moe_expert_forward_decode_noalloc",
 )
@@ -102,6 +103,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.e4b_grouped_nf4_gemm_dgrad.restype = i32
     lib.e4b_grouped_nf4_gemm_dgrad.argtypes = [vp, i64, i64, vp, vp, i64, i64, vp, vp, i64, i64, vp, vp, i32,
                                                ctypes.c_float, vp, i32, vp, sz, vp]
+    lib.e4b_grouped_lora_grads_workspace_size.restype = sz
+    lib.e4b_grouped_lora_grads_workspace_size.argtypes = [i64, i32]
+    lib.e4b_grouped_lora_grads.restype = i32
+    lib.e4b_grouped_lora_grads.argtypes = [vp, i64, i64, vp, vp, i64, i64, vp, i64, i64, i64, vp, vp, i32,
+                                           ctypes.c_float, vp, vp, vp, sz, vp]
     lib.e4b_moe_expert_forward_workspace_size.restype = sz
     lib.e4b_moe_expert_forward_workspace_size.argtypes = [i64, ctypes.POINTER(ExpertStackC), i32]
     lib.e4b_moe_expert_forward.restype = i32
@@ -280,6 +286,36 @@ def e4b_grouped_nf4_gemm_dgrad(dY: torch.Tensor, row_index: Optional[torch.Tenso
         dY.data_ptr(), dY.shape[0], dY.stride(0), _ptr(row_index), expert_offsets.data_ptr(), E, total_rows,
         packed.data_ptr(), absmax.data_ptr(), N, K, _ptr(lora_A), _ptr(lora_B), r, float(lora_scale),
         out.data_ptr(), od, _ptr(workspace), ws, _stream(stream)), "e4b_grouped_nf4_gemm_dgrad")
+
+
+def e4b_grouped_lora_grads_workspace_size(total_rows: int, r: int) -> int:
+    return int(load_library().e4b_grouped_lora_grads_workspace_size(total_rows, r))
+
+
+def e4b_grouped_lora_grads(x: torch.Tensor, row_index: Optional[torch.Tensor], expert_offsets: torch.Tensor,
+                           total_rows: int, da: torch.Tensor, N: int, K: int, lora_A: torch.Tensor,
+                           lora_B: torch.Tensor, lora_scale: float, dA: torch.Tensor, dB: torch.Tensor,
+                           workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """dA [E, r, K], dB [E, N, r] (fp32) of one grouped projection's adapter."""
+    for t, n in ((x, "x"), (da, "da")):
+        if t.dim() != 2 or t.dtype != torch.bfloat16 or not t.is_cuda or t.stride(1) != 1:
+            raise ValueError(f"{n} must be a 2-D bf16 CUDA tensor with unit column stride")
+    _dev(expert_offsets, "expert_offsets", torch.int32)
+    _dev(lora_A, "lora_A", torch.bfloat16)
+    _dev(lora_B, "lora_B", torch.bfloat16)
+    _dev(dA, "dA", torch.float32)
+    _dev(dB, "dB", torch.float32)
+    if row_index is not None:
+        _dev(row_index, "row_index", torch.int32)
+    E = expert_offsets.numel() - 1
+    r = lora_A.shape[1]
+    if dA.numel() < E * r * K or dB.numel() < E * N * r:
+        raise ValueError("dA/dB too small")
+    ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load_library().e4b_grouped_lora_grads(
+        x.data_ptr(), x.shape[0], x.stride(0), _ptr(row_index), expert_offsets.data_ptr(), E, total_rows,
+        da.data_ptr(), da.stride(0), N, K, lora_A.data_ptr(), lora_B.data_ptr(), r, float(lora_scale),
+        dA.data_ptr(), dB.data_ptr(), _ptr(workspace), ws, _stream(stream)), "e4b_grouped_lora_grads")
 
 
 class ExpertStack:

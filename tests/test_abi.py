@@ -171,3 +171,25 @@ def test_dgrad_host_side_rejections(lib):
     assert call(absmax=ctypes.c_void_p((1 << 20) + 4)) == 1 and b"16-byte aligned" in lib.e4b_last_error()
     assert call(wsb=need - 1) == 3 and str(need).encode() in lib.e4b_last_error()
     assert call(ws=ctypes.c_void_p((1 << 20) + 8)) == 1 and b"dgrad workspace must be" in lib.e4b_last_error()
+
+
+def test_lora_grads_host_side_rejections(lib):
+    p = ctypes.c_void_p(1 << 20)
+    rows, N, K, r = 64, 128, 192, 8
+    need = e4b.e4b_grouped_lora_grads_workspace_size(rows, r)
+    assert need == 256 + 2 * ((rows * r * 4 + 255) // 256 * 256)
+    assert e4b.e4b_grouped_lora_grads_workspace_size(rows, 0) == 0
+
+    def call(**kw):
+        a = dict(x=p, x_rows=rows, ldx=K, ridx=None, offs=p, E=2, rows=rows, da=p, ldda=N, N=N, K=K, la=p, lb=p,
+                 r=r, scale=1.0, dA=p, dB=p, ws=p, wsb=need)
+        a.update(kw)
+        return lib.e4b_grouped_lora_grads(a["x"], a["x_rows"], a["ldx"], a["ridx"], a["offs"], a["E"], a["rows"],
+                                          a["da"], a["ldda"], a["N"], a["K"], a["la"], a["lb"], a["r"], a["scale"],
+                                          a["dA"], a["dB"], a["ws"], a["wsb"], None)
+    assert call(r=0) == 2 and b"rank" in lib.e4b_last_error()
+    assert call(K=100) == 2 and b"K must be" in lib.e4b_last_error()
+    assert call(ldx=K + 4) == 1 and b"ldx" in lib.e4b_last_error()
+    assert call(ldda=N - 1) == 1 and b"ldda" in lib.e4b_last_error()
+    assert call(dB=None) == 1 and b"null" in lib.e4b_last_error()
+    assert call(wsb=need - 1) == 3 and str(need).encode() in lib.e4b_last_error()

@@ -158,3 +158,36 @@ def test_grouped_dgrad_empty_and_errors():
         e4b.e4b_grouped_nf4_gemm_dgrad(_t_bf16(c["dYbits"]), None, torch.from_numpy(c["offs"]).cuda(), 0,
                                        torch.from_numpy(c["packed"]).cuda(), torch.from_numpy(c["absmax"]).cuda(),
                                        96, 64, out)
+
+
+@pytest.mark.parametrize("r", [1, 8, 16])
+def test_grouped_lora_grads_match_oracle(r):
+    """dA, dB of one grouped projection: ragged and empty groups, a row gather."""
+    require_gpu()
+    rng = np.random.default_rng(40 + r)
+    E, N, K = 4, 192, 256
+    counts = [70, 0, 3, 200]
+    offs = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    rows = int(offs[-1])
+    x_rows = 300
+    xbits = workloads.to_bf16_bits(rng.standard_normal((x_rows, K)).astype(np.float32))
+    dabits = workloads.to_bf16_bits(rng.standard_normal((rows, N)).astype(np.float32))
+    ridx = rng.integers(0, x_rows, size=rows).astype(np.int32)
+    la = workloads.to_bf16_bits((rng.standard_normal((E, r, K)) * 0.05).astype(np.float32))
+    lb = workloads.to_bf16_bits((rng.standard_normal((E, N, r)) * 0.05).astype(np.float32))
+    scale = 16.0 / r
+    dA = torch.full((E, r, K), float("nan"), dtype=torch.float32, device="cuda")
+    dB = torch.full((E, N, r), float("nan"), dtype=torch.float32, device="cuda")
+    ws = e4b.workspace(e4b.e4b_grouped_lora_grads_workspace_size(rows, r))
+    e4b.e4b_grouped_lora_grads(_t_bf16(xbits), torch.from_numpy(ridx).cuda(), torch.from_numpy(offs).cuda(), rows,
+                               _t_bf16(dabits), N, K, _t_bf16(la), _t_bf16(lb), scale, dA, dB, ws)
+    torch.cuda.synchronize()
+    assert e4b.last_path() == "lora_grads"
+    f = lambda b: workloads.bf16_bits_to_f32(b).astype(np.float64)
+    rA, rB = backward.grouped_lora_grads(f(xbits), ridx, offs, f(dabits), f(la), f(lb), scale)
+    gA, gB = dA.cpu().numpy().astype(np.float64), dB.cpu().numpy().astype(np.float64)
+    assert np.all(gA[1] == 0) and np.all(gB[1] == 0)   # the empty group
+    # inputs are exact bf16 values; fp32 accumulation over <= 200 rows and <= 256 terms
+    for got, ref in ((gA, rA), (gB, rB)):
+        fro, mx = rel_errors(got, ref)
+        assert fro <= 1e-4 and mx <= 1e-3
