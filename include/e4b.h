@@ -321,6 +321,33 @@ E4B_API e4b_status e4b_moe_expert_forward_path(const uint16_t* x, int64_t M, con
                                        e4b_path path, e4b_stream stream);
 
 /*
+ * Backward of the layer through the frozen NF4 experts, routing ids held fixed
+ * (top-k selection is piecewise constant in the logits).
+ * Source: experts4bit-qlora 0.22.0, "Which training path?" (per-expert LoRA
+ * over a frozen NF4 stack; the base is decoded again in backward, one dgrad
+ * launch per projection); Solutions -- one page per problem, the ExpertsLoRA row.
+ *
+ * For out = e4b_moe_expert_forward(x, router_logits, ...) and an upstream
+ * gradient dout [M, H] bf16, writes the gradients of sum(dout * out):
+ *   dx       [M, H] fp32    through gate_up and the adapter's delta
+ *   dlogits  [M, E] fp32    through the routing weights (zero on unselected
+ *                           experts with renormalisation)
+ *   dA, dB   [E, r, H], [E, 2I, r] fp32, the adapter's gradients (required
+ *            when the stack has an adapter, ignored otherwise)
+ * The frozen stacks get no gradient.  It routes again, recomputes the gate_up
+ * output (fp32) and the per-slot expert outputs (fp32), and runs the two
+ * grouped dgrad products of e4b_grouped_nf4_gemm_dgrad() with the SwiGLU
+ * derivative between them; every sum runs in a fixed order (deterministic).
+ * workspace  e4b_moe_expert_backward_workspace_size() bytes (error word first).
+ */
+E4B_API size_t e4b_moe_expert_backward_workspace_size(int64_t M, const e4b_expert_stack* w, int k);
+E4B_API e4b_status e4b_moe_expert_backward(const uint16_t* x, int64_t M, const float* router_logits,
+                                   int k, int renormalize, const e4b_expert_stack* w,
+                                   const uint16_t* dout, float* dx, float* dlogits, float* dA,
+                                   float* dB, void* workspace, size_t workspace_bytes,
+                                   e4b_stream stream);
+
+/*
  * Allocation-free small-batch forward.  The pages have no counterpart of this
  * call; it exists for hosts that cannot give the library device memory:
  * serving engines that plan every byte of device memory into a fixed pool at

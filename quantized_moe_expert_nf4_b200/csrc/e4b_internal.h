@@ -145,6 +145,17 @@ size_t lora_grads_workspace_bytes(int64_t total_rows, int r);
 size_t lora_grads_workspace_yb_offset(int64_t total_rows, int r);
 cudaError_t launch_lora_grads(const LoraGradArgs& a, cudaStream_t stream);
 
+// ---- layer backward steps (csrc/backward.cu) -------------------------------------
+cudaError_t launch_swiglu_h(const float* a, int64_t S, int I, uint16_t* h, cudaStream_t stream);
+cudaError_t launch_slot_grads(const uint16_t* dout, const float* z, const int32_t* perm, const int32_t* row_token,
+                              const float* w, int64_t S, int64_t M, int H, uint16_t* dz, float* dw,
+                              cudaStream_t stream);
+cudaError_t launch_swiglu_bwd(const float* a, const float* dh, int64_t S, int I, uint16_t* da, cudaStream_t stream);
+cudaError_t launch_token_sum(const float* dxg, const int32_t* inv, int64_t M, int k, int H, float* dx,
+                             cudaStream_t stream);
+cudaError_t launch_router_grad(const float* logits, const int32_t* ids, const float* w, const float* dw, int64_t M,
+                               int E, int k, bool renormalize, float* dlogits, cudaStream_t stream);
+
 // ---- combine ---------------------------------------------------------------
 cudaError_t launch_combine(const uint16_t* z, const int32_t* inv, const float* w, int64_t M, int k,
                            int H, uint16_t* out, cudaStream_t stream);

@@ -39,6 +39,7 @@ EXPORTED = (
     "e4b_grouped_lora_grads_workspace_size", "e4b_grouped_lora_grads",
     "e4b_moe_expert_forward_workspace_size", "e4b_moe_expert_forward",
     "e4b_moe_expert_forward_path", "e4b_moe_expert_forward_decode_noalloc",
+    "e4b_moe_expert_backward_workspace_size", "e4b_moe_expert_backward",
 )
 
 
@@ -119,6 +120,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.e4b_workspace_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
     lib.e4b_workspace_clear_error.restype = i32
     lib.e4b_workspace_clear_error.argtypes = [vp, vp]
+    lib.e4b_moe_expert_backward_workspace_size.restype = sz
+    lib.e4b_moe_expert_backward_workspace_size.argtypes = [i64, ctypes.POINTER(ExpertStackC), i32]
+    lib.e4b_moe_expert_backward.restype = i32
+    lib.e4b_moe_expert_backward.argtypes = [vp, i64, vp, i32, i32, ctypes.POINTER(ExpertStackC), vp, vp, vp, vp,
+                                            vp, vp, sz, vp]
     lib.e4b_moe_expert_forward_path.restype = i32
     lib.e4b_moe_expert_forward_path.argtypes = [vp, i64, vp, i32, i32, ctypes.POINTER(ExpertStackC), vp, vp,
                                                 sz, i32, vp]
@@ -360,6 +366,35 @@ def e4b_moe_expert_forward(x: torch.Tensor, router_logits: torch.Tensor, k: int,
     _check(load_library().e4b_moe_expert_forward_path(
         x.data_ptr(), M, router_logits.data_ptr(), k, int(bool(renormalize)), ctypes.byref(stack.c),
         out.data_ptr(), _ptr(workspace), ws, path, _stream(stream)), "e4b_moe_expert_forward")
+
+
+def e4b_moe_expert_backward_workspace_size(M: int, stack: "ExpertStack", k: int) -> int:
+    return int(load_library().e4b_moe_expert_backward_workspace_size(M, ctypes.byref(stack.c), k))
+
+
+def e4b_moe_expert_backward(x: torch.Tensor, router_logits: torch.Tensor, k: int, renormalize: bool,
+                            stack: "ExpertStack", dout: torch.Tensor, dx: torch.Tensor, dlogits: torch.Tensor,
+                            dA: Optional[torch.Tensor], dB: Optional[torch.Tensor], workspace: Optional[torch.Tensor],
+                            stream=None) -> None:
+    """Gradients of sum(dout * forward(x, router_logits)): dx [M, H], dlogits [M, E] and, with an
+    adapter, dA [E, r, H], dB [E, 2I, r] (all fp32); routing ids held fixed (see include/e4b.h)."""
+    _dev(x, "x", torch.bfloat16)
+    _dev(router_logits, "router_logits", torch.float32)
+    _dev(dout, "dout", torch.bfloat16)
+    _dev(dx, "dx", torch.float32)
+    _dev(dlogits, "dlogits", torch.float32)
+    M = x.shape[0]
+    if (x.shape[1] != stack.H or router_logits.shape != (M, stack.E) or dout.shape != (M, stack.H)
+            or dx.shape != (M, stack.H) or dlogits.shape != (M, stack.E)):
+        raise ValueError("x, dout, dx [M, H] and router_logits, dlogits [M, E] required")
+    for t, n in ((dA, "dA"), (dB, "dB")):
+        if t is not None:
+            _dev(t, n, torch.float32)
+    ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load_library().e4b_moe_expert_backward(
+        x.data_ptr(), M, router_logits.data_ptr(), k, int(bool(renormalize)), ctypes.byref(stack.c),
+        dout.data_ptr(), dx.data_ptr(), dlogits.data_ptr(), _ptr(dA), _ptr(dB), _ptr(workspace), ws,
+        _stream(stream)), "e4b_moe_expert_backward")
 
 
 def e4b_moe_expert_forward_decode_noalloc(x: torch.Tensor, router_logits: torch.Tensor, k: int, renormalize: bool,

@@ -193,3 +193,22 @@ def test_lora_grads_host_side_rejections(lib):
     assert call(ldda=N - 1) == 1 and b"ldda" in lib.e4b_last_error()
     assert call(dB=None) == 1 and b"null" in lib.e4b_last_error()
     assert call(wsb=need - 1) == 3 and str(need).encode() in lib.e4b_last_error()
+
+
+def test_backward_host_side_checks(lib):
+    p = 1 << 20
+    st = e4b.ExpertStackC(p, p, p, p, None, None, 0, 0.0, 8, 256, 128)
+    sizes = [lib.e4b_moe_expert_backward_workspace_size(M, ctypes.byref(st), 2) for M in (1, 64, 300)]
+    assert sizes[0] < sizes[1] < sizes[2]
+    # per routed row at least a (fp32 2I), z and dxg (fp32 H each), dz (bf16 H), dh (fp32 I), da (bf16 2I)
+    assert sizes[2] >= 600 * (8 * 128 + 4 * 256 * 2 + 2 * 256 + 4 * 128 + 4 * 128)
+    assert lib.e4b_moe_expert_backward_workspace_size(0, ctypes.byref(st), 2) == 0
+    vp = ctypes.c_void_p(p)
+    need = sizes[1]
+    status = lib.e4b_moe_expert_backward(vp, 64, vp, 2, 1, ctypes.byref(st), vp, vp, vp, None, None, vp, need - 1,
+                                         None)
+    assert status == 3 and str(need).encode() in lib.e4b_last_error()
+    stl = e4b.ExpertStackC(p, p, p, p, p, p, 8, 16.0, 8, 256, 128)
+    status = lib.e4b_moe_expert_backward(vp, 64, vp, 2, 1, ctypes.byref(stl), vp, vp, vp, None, None, vp, 1 << 40,
+                                         None)
+    assert status == 1 and b"needs dA and dB" in lib.e4b_last_error()
