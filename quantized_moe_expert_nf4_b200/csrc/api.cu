@@ -429,8 +429,8 @@ e4b_status e4b_grouped_nf4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda, 
 size_t e4b_grouped_nf4_gemm_dgrad_workspace_size(int64_t total_rows, int64_t N, int64_t K, int r) {
   (void)N;
   (void)K;
-  if (total_rows < 0 || r < 0) return 0;
-  return dgrad_workspace_bytes(total_rows, r);
+  if (total_rows < 0 || r < 0 || N < 0) return 0;
+  return dgrad_workspace_bytes(total_rows, N, r);
 }
 
 e4b_status e4b_grouped_nf4_gemm_dgrad(const uint16_t* dY, int64_t dy_rows, int64_t lddy, const int32_t* row_index,
@@ -458,7 +458,7 @@ e4b_status e4b_grouped_nf4_gemm_dgrad(const uint16_t* dY, int64_t dy_rows, int64
     return fail(E4B_ERR_INVALID_ARGUMENT, "dY, packed, absmax and out must be 16-byte aligned");
   if (lora_A && (!aligned16(lora_A) || !aligned16(lora_B)))
     return fail(E4B_ERR_INVALID_ARGUMENT, "lora_A and lora_B must be 16-byte aligned");
-  if (e4b_status s = check_workspace("dgrad", dgrad_workspace_bytes(total_rows, r), workspace, workspace_bytes);
+  if (e4b_status s = check_workspace("dgrad", dgrad_workspace_bytes(total_rows, N, r), workspace, workspace_bytes);
       s != E4B_OK)
     return s;
   if (e4b_status s = check_device(); s != E4B_OK) return s;
@@ -483,11 +483,14 @@ e4b_status e4b_grouped_nf4_gemm_dgrad(const uint16_t* dY, int64_t dy_rows, int64
   d.r = r;
   d.lora_scale = lora_scale;
   d.yb = r ? reinterpret_cast<float*>(static_cast<char*>(workspace) + dgrad_workspace_yb_offset()) : nullptr;
+  d.gathered = reinterpret_cast<uint16_t*>(static_cast<char*>(workspace) + dgrad_workspace_gather_offset(total_rows, r));
+  d.err = static_cast<int*>(workspace);
   d.out = out;
   d.out_bf16 = out_dtype == E4B_BF16;
-  cudaError_t err = launch_grouped_dgrad(d, reinterpret_cast<cudaStream_t>(stream));
+  const char* path = "";
+  cudaError_t err = launch_grouped_dgrad(d, reinterpret_cast<cudaStream_t>(stream), &path);
   if (err != cudaSuccess) return cuda_fail(err, "grouped dgrad launch");
-  set_path("dgrad.mma");
+  set_path(path);
   return E4B_OK;
 }
 
@@ -812,7 +815,8 @@ e4b_status e4b_moe_expert_backward(const uint16_t* x, int64_t M, const float* ro
   dd.K = I;
   dd.out = at<float>(ws, L.dh);
   dd.out_bf16 = false;
-  if ((err = launch_grouped_dgrad(dd, stream_)) != cudaSuccess) return cuda_fail(err, "backward: dgrad down");
+  dd.err = at<int>(ws, L.err);
+  if ((err = launch_grouped_dgrad(dd, stream_, &path)) != cudaSuccess) return cuda_fail(err, "backward: dgrad down");
   if ((err = launch_swiglu_bwd(at<float>(ws, L.a), at<float>(ws, L.dh), S, I, at<uint16_t>(ws, L.da), stream_)) !=
       cudaSuccess)
     return cuda_fail(err, "backward: swiglu derivative");
@@ -835,7 +839,8 @@ e4b_status e4b_moe_expert_backward(const uint16_t* x, int64_t M, const float* ro
   dg.yb = r ? at<float>(ws, L.yb) : nullptr;
   dg.out = at<float>(ws, L.dxg);
   dg.out_bf16 = false;
-  if ((err = launch_grouped_dgrad(dg, stream_)) != cudaSuccess) return cuda_fail(err, "backward: dgrad gate_up");
+  dg.err = at<int>(ws, L.err);
+  if ((err = launch_grouped_dgrad(dg, stream_, &path)) != cudaSuccess) return cuda_fail(err, "backward: dgrad gate_up");
   if ((err = launch_token_sum(at<float>(ws, L.dxg), o.inv, M, k, H, dx, stream_)) != cudaSuccess)
     return cuda_fail(err, "backward: token sum");
   if ((err = launch_router_grad(router_logits, o.ids, o.w, at<float>(ws, L.dw), M, E, k, renormalize != 0, dlogits,

@@ -21,6 +21,9 @@
 // scales it by (absmax[n], absmax[n+1]) and stores 8 rows n of one column k as
 // one 16-byte run of W^T.  The contraction order inside a 32-wide chunk is
 // permuted identically on both operands: lane t of a quad owns n in [8t, 8t+8).
+#include <cstdlib>
+#include <cstring>
+
 #include "common.cuh"
 #include "e4b_internal.h"
 
@@ -318,8 +321,8 @@ cudaError_t launch_lora_grads(const LoraGradArgs& a, cudaStream_t stream) {
 }
 
 size_t dgrad_workspace_yb_offset() { return 256; }
-size_t dgrad_workspace_bytes(int64_t total_rows, int r) {
-  return 256 + align_up(r > 0 ? static_cast<size_t>(total_rows) * r * sizeof(float) : 0, 256);
+size_t dgrad_workspace_bytes(int64_t total_rows, int64_t N, int r) {
+  return dgrad_workspace_gather_offset(total_rows, r) + static_cast<size_t>(total_rows) * N * sizeof(uint16_t);
 }
 
 size_t lora_grads_workspace_yb_offset(int64_t total_rows, int r) {
@@ -329,17 +332,86 @@ size_t lora_grads_workspace_bytes(int64_t total_rows, int r) {
   return lora_grads_workspace_yb_offset(total_rows, r) + align_up(static_cast<size_t>(total_rows) * r * sizeof(float), 256);
 }
 
-cudaError_t launch_grouped_dgrad(const DgradArgs& a, cudaStream_t stream) {
+namespace {
+int dgrad_override() {
+  const char* v = getenv("E4B_DGRAD");
+  if (!v) return 0;
+  if (!strcmp(v, "mma")) return 1;
+  if (!strcmp(v, "tc")) return 2;
+  return 0;
+}
+constexpr int64_t kTcMinRows = 512;
+
+// The adapter's share after the tensor-core product (fp32 output):
+// out[p, k] += scale * sum_rho yb[p, rho] * lora_A[e, rho, k].
+__global__ void __launch_bounds__(256) dgrad_lora_add_kernel(DgradArgs a) {
+  __shared__ float yb_s[16];
+  __shared__ int e_s;
+  const int64_t p = blockIdx.x;
+  if (threadIdx.x == 0) {
+    int lo = 0, hi = a.E - 1;  // group of p: last e with offsets[e] <= p
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (a.offsets[mid] <= p) lo = mid;
+      else hi = mid - 1;
+    }
+    e_s = lo;
+  }
+  if (threadIdx.x < a.r) yb_s[threadIdx.x] = a.yb[p * a.r + threadIdx.x];
+  __syncthreads();
+  const int k = blockIdx.y * blockDim.x + threadIdx.x;
+  if (k >= a.K) return;
+  const uint16_t* la = a.lora_A + static_cast<int64_t>(e_s) * a.r * a.K + k;
+  float d = 0.f;
+  for (int rr = 0; rr < a.r; ++rr) d = fmaf(yb_s[rr], bf16_bits_to_float(la[static_cast<int64_t>(rr) * a.K]), d);
+  float* o = static_cast<float*>(a.out) + p * a.K + k;
+  *o = fmaf(a.lora_scale, d, *o);
+}
+}  // namespace
+
+size_t dgrad_workspace_gather_offset(int64_t total_rows, int r) {
+  return 256 + align_up(r > 0 ? static_cast<size_t>(total_rows) * r * sizeof(float) : 0, 256);
+}
+
+cudaError_t launch_grouped_dgrad(const DgradArgs& a, cudaStream_t stream, const char** path) {
   if (a.total_rows == 0) return cudaSuccess;
-  if (a.lora_A && a.r > 0) {
+  const bool lora = a.lora_A && a.r > 0;
+  if (lora) {
     cudaError_t err = launch_dgrad_lora_yb(a, stream);
     if (err != cudaSuccess) return err;
+  }
+  const int ov = dgrad_override();
+  const bool tc_ok = dgrad_tc_supported(a, a.row_index ? a.N : a.lddy);
+  const bool use_tc = ov == 2 || (ov == 0 && tc_ok && a.total_rows >= kTcMinRows);
+  if (use_tc) {
+    if (!tc_ok) return cudaErrorNotSupported;
+    const uint16_t* dy = a.dY;
+    int64_t rows = a.dy_rows, ld = a.lddy;
+    if (a.row_index) {  // the tensor-core kernel reads dY rows as contiguous tiles
+      cudaError_t err = launch_gather_rows(a.dY, a.dy_rows, a.lddy, a.row_index, a.total_rows, a.N, a.gathered, stream);
+      if (err != cudaSuccess) return err;
+      dy = a.gathered;
+      rows = a.total_rows;
+      ld = a.N;
+    }
+    cudaError_t err = launch_grouped_dgrad_tc(a, dy, rows, ld, a.err, stream);
+    if (err != cudaSuccess) return err;
+    if (lora) {
+      dim3 grid(static_cast<unsigned>(a.total_rows), static_cast<unsigned>((a.K + 255) / 256));
+      LaunchScope ls("dgrad.lora_add", stream);
+      dgrad_lora_add_kernel<<<grid, 256, 0, stream>>>(a);
+      err = cudaGetLastError();
+      if (err != cudaSuccess) return err;
+    }
+    *path = "dgrad.tc";
+    return cudaSuccess;
   }
   // Upper bound on routed-row tiles: ceil(total/64) + number of non-empty groups.
   const int64_t gx = (a.total_rows + kTileT - 1) / kTileT + (a.E < a.total_rows ? a.E : a.total_rows);
   dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(a.K / kTileK));
   LaunchScope ls("dgrad.mma", stream);
   grouped_nf4_dgrad_kernel<<<grid, kThreads, 0, stream>>>(a);
+  *path = "dgrad.mma";
   return cudaGetLastError();
 }
 

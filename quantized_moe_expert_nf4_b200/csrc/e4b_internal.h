@@ -113,13 +113,22 @@ struct DgradArgs {
   int r;
   float lora_scale;
   float* yb;  // workspace [total_rows, r] fp32: dY . lora_B
+  uint16_t* gathered;  // workspace [total_rows, N] bf16: dY rows in group order (tensor-core path)
+  int* err;            // workspace error word
   void* out;  // [total_rows, K]
   bool out_bf16;
 };
-// Workspace: [error word, 256 B][dY . lora_B, total_rows * r fp32, 256-B aligned].
-size_t dgrad_workspace_bytes(int64_t total_rows, int r);
+// Workspace: [error word, 256 B][dY . lora_B, total_rows * r fp32][dY rows gathered,
+// total_rows * N bf16], parts 256-B aligned.
+size_t dgrad_workspace_bytes(int64_t total_rows, int64_t N, int r);
 size_t dgrad_workspace_yb_offset();
-cudaError_t launch_grouped_dgrad(const DgradArgs& a, cudaStream_t stream);
+size_t dgrad_workspace_gather_offset(int64_t total_rows, int r);
+// Warp-MMA kernel below 512 routed rows (and with an adapter and bf16 output),
+// the tensor-core kernel otherwise; E4B_DGRAD=mma|tc forces one.
+cudaError_t launch_grouped_dgrad(const DgradArgs& a, cudaStream_t stream, const char** path);
+bool dgrad_tc_supported(const DgradArgs& a, int64_t lddy);
+cudaError_t launch_grouped_dgrad_tc(const DgradArgs& a, const uint16_t* dy, int64_t dy_rows, int64_t lddy,
+                                    int* err_word, cudaStream_t stream);
 // yb = dY . lora_B per routed row (into a.yb); a.lora_B, a.r, a.N, a.dY, a.lddy used.
 cudaError_t launch_dgrad_lora_yb(const DgradArgs& a, cudaStream_t stream);
 

@@ -151,8 +151,10 @@ def test_dgrad_host_side_rejections(lib):
     p = ctypes.c_void_p(1 << 20)
     rows, N, K = 64, 128, 192
     need = e4b.e4b_grouped_nf4_gemm_dgrad_workspace_size(rows, N, K, 0)
-    assert need == 256                                   # error word only without an adapter
-    assert e4b.e4b_grouped_nf4_gemm_dgrad_workspace_size(rows, N, K, 8) == 256 + (rows * 8 * 4 + 255) // 256 * 256
+    # error word, then (with an adapter) dY . lora_B, then room for the dY rows gathered in group order
+    assert need == 256 + rows * N * 2
+    assert e4b.e4b_grouped_nf4_gemm_dgrad_workspace_size(rows, N, K, 8) == \
+        256 + (rows * 8 * 4 + 255) // 256 * 256 + rows * N * 2
 
     def call(**kw):
         a = dict(dY=p, dy_rows=rows, lddy=N, ridx=None, offs=p, E=2, rows=rows, packed=p, absmax=p, N=N, K=K,

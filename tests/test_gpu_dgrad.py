@@ -75,22 +75,40 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("kernel", ["mma", "tc"])
 @pytest.mark.parametrize("ci", range(len(CASES)))
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
-def test_grouped_dgrad_matches_oracle(ci, out_dtype):
+def test_grouped_dgrad_matches_oracle(monkeypatch, kernel, ci, out_dtype):
+    """Both kernels (warp MMA; tcgen05 with the transposing decoders), forced."""
     require_gpu()
+    monkeypatch.setenv("E4B_DGRAD", kernel)
     c = _case(*CASES[ci], seed=ci)
     got, path = _run_gpu(c, out_dtype)
     ref = _oracle(c)
     fro, mx = rel_errors(got, ref)
     print(f"[parity] dgrad case {ci} {out_dtype} path {path}: rel_fro={fro:.2e} max={mx:.2e}")
-    assert path == "dgrad.mma"
+    assert path == f"dgrad.{kernel}"
     assert fro <= _tol(out_dtype) and mx <= 2 * _tol(out_dtype)
 
 
-@pytest.mark.parametrize("r", [3, 8, 16])
-def test_grouped_dgrad_lora(r):
+@pytest.mark.parametrize("shape", ["wide", "double"])
+def test_grouped_dgrad_tensor_core_shapes_and_size_choice(monkeypatch, shape):
+    """Both tile shapes of the tensor-core dgrad, a column count that is not a
+    multiple of the 256-column tile, and the automatic choice for >= 512 rows."""
     require_gpu()
+    monkeypatch.setenv("E4B_TC_SHAPE", shape)
+    c = _case(3, 320, 704, [600, 0, 45], 700, seed=21)
+    got, path = _run_gpu(c, torch.float32)
+    assert path == "dgrad.tc"
+    fro, mx = rel_errors(got, _oracle(c))
+    assert fro <= 4e-3 and mx <= 8e-3
+
+
+@pytest.mark.parametrize("kernel", ["mma", "tc"])
+@pytest.mark.parametrize("r", [3, 8, 16])
+def test_grouped_dgrad_lora(monkeypatch, kernel, r):
+    require_gpu()
+    monkeypatch.setenv("E4B_DGRAD", kernel)
     c = _case(4, 192, 256, [33, 0, 100, 7], 90, seed=10 + r, lora_r=r)
     got, _ = _run_gpu(c, torch.float32, scale=16.0 / r)
     ref = _oracle(c, scale=16.0 / r)
