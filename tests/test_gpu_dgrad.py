@@ -1,10 +1,11 @@
 """GPU grouped NF4 dgrad (input gradient through the frozen base) vs the float64 oracle.
 
-Tolerance: the kernel rounds each decoded weight three times (codebook entry,
-absmax and their product, each <= 2^-9 relative, about 2^-9 rms together) and
-accumulates in fp32, so a plain fp32 result stays within 4e-3 relative
+Tolerance: the kernels round each decoded weight three times (codebook entry,
+absmax and their product, each <= 2^-9 relative, so <= 3 * 2^-9 ~ 5.9e-3 per
+weight) and accumulate in fp32, so an fp32 result stays within 6e-3 relative
 Frobenius (max-abs within twice that of max|ref|); a bf16 result adds one
-rounding of 2^-9: 1e-2.
+rounding of 2^-9: 1e-2.  (A numpy model with exactly these roundings gives
+2.5e-3 to 2.8e-3 on the cases below.)
 """
 import numpy as np
 import pytest
@@ -62,7 +63,7 @@ def _oracle(c, use_ridx=True, scale=2.0):
 
 
 def _tol(out_dtype):
-    return 1e-2 if out_dtype == torch.bfloat16 else 4e-3
+    return 1e-2 if out_dtype == torch.bfloat16 else 6e-3
 
 
 CASES = [
@@ -101,7 +102,7 @@ def test_grouped_dgrad_tensor_core_shapes_and_size_choice(monkeypatch, shape):
     got, path = _run_gpu(c, torch.float32)
     assert path == "dgrad.tc"
     fro, mx = rel_errors(got, _oracle(c))
-    assert fro <= 4e-3 and mx <= 8e-3
+    assert fro <= 6e-3 and mx <= 1.2e-2
 
 
 @pytest.mark.parametrize("kernel", ["mma", "tc"])
@@ -113,7 +114,7 @@ def test_grouped_dgrad_lora(monkeypatch, kernel, r):
     got, _ = _run_gpu(c, torch.float32, scale=16.0 / r)
     ref = _oracle(c, scale=16.0 / r)
     fro, mx = rel_errors(got, ref)
-    assert fro <= 4e-3 and mx <= 8e-3
+    assert fro <= 6e-3 and mx <= 1.2e-2
     # the adapter's share is not negligible here, so the check covers it
     base = _oracle(dict(c, r=0, la=None, lb=None))
     assert rel_errors(base, ref)[0] > 5e-2
@@ -124,7 +125,7 @@ def test_grouped_dgrad_identity_rows():
     c = _case(3, 128, 128, [40, 24, 0], 64, seed=3)
     got, _ = _run_gpu(c, torch.float32, use_ridx=False)
     ref = _oracle(c, use_ridx=False)
-    assert rel_errors(got, ref)[0] <= 4e-3
+    assert rel_errors(got, ref)[0] <= 6e-3
 
 
 def test_grouped_dgrad_positive_control_flipped_nibble():
