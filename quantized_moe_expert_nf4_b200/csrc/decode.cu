@@ -39,7 +39,7 @@ namespace {
 constexpr int kMaxM = 8;
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
-constexpr int kSlots = 4;                  // (item, span) load slots per warp per batch in kernel A
+constexpr int kMaxSlots = 8;               // (item, span) load slots per warp per batch in kernel A
 constexpr int kPairSlots = 2;              // (expert, span) load slots per warp per batch in kernel B
 constexpr int kMaxKBW = 2;                 // spans (2 k-blocks) per warp per item: H <= 128 * 16 * 2 = 4096
 constexpr unsigned long long kPrefetchLimit = 64ull << 20;
@@ -74,6 +74,12 @@ __host__ __device__ inline uint32_t al(uint32_t v, uint32_t a) { return (v + a -
 // Spans of 128 k (2 absmax blocks, 64 packed bytes of a row) per warp per item.
 __host__ __device__ inline int kbw_of(int H) { return ((H / 64 + 1) / 2 + kWarps - 1) / kWarps; }
 
+// (item, span) load slots per warp per batch of kernel A: eight for one token
+// with one span per warp (a CTA's whole share in one batch; measured faster at
+// M = 1), four otherwise (more tokens need the registers for x; measured
+// faster at M = 4 and 8).
+__host__ __device__ inline int slots_for(int M, int H) { return (M == 1 && kbw_of(H) == 1) ? 8 : 4; }
+
 // Shared-memory carve of kernel A (gate_up) or B (down).
 __host__ __device__ inline Layout make_layout(bool is_a, int M, int k, int E, int H, int r) {
   Layout L;
@@ -83,7 +89,7 @@ __host__ __device__ inline Layout make_layout(bool is_a, int M, int k, int E, in
   L.xs = o;
   if (is_a) o = al(o + M * (2 * H + 16), 16);
   L.red = o;
-  const int items = is_a ? kSlots : 1;  // partial sums of up to kSlots items per batch (A), 1 row block (B)
+  const int items = is_a ? slots_for(M, H) : 1;  // partial sums of the items of a batch (A), 1 row block (B)
   o = al(o + items * kWarps * 32 * 16, 16);
   const int S = M * k;
   L.ids = o;
@@ -230,9 +236,10 @@ __device__ __forceinline__ void prefetch_items(const DecodeParams& p, const int*
 
 // ---------------------------------------------------------------------------
 // Kernel A: gate_up + SwiGLU (+ LoRA delta) -> h.  KBW = k-blocks per warp per item.
-template <int KBW>
+template <int KBW, int SLOTS>
 __global__ void __launch_bounds__(kThreads, 1) decode_gate_up_kernel(DecodeParams p) {
-  constexpr int IB = kSlots / KBW;  // items per batch
+  static_assert(SLOTS <= kMaxSlots, "load slots");
+  constexpr int IB = SLOTS / KBW;  // items per batch
   extern __shared__ __align__(16) unsigned char smem[];
   const Layout L = make_layout(true, p.M, p.k, p.E, p.H, p.r);
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L.lut);
@@ -530,16 +537,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_down_kernel(DecodeParams p
   }
 }
 
-template <int KBW>
+template <int KBW, int SLOTS>
 cudaError_t raise_smem_limits(size_t smem_a, size_t smem_b) {
-  cudaError_t err = ensure_smem_limit(reinterpret_cast<const void*>(decode_gate_up_kernel<KBW>), smem_a);
+  cudaError_t err = ensure_smem_limit(reinterpret_cast<const void*>(decode_gate_up_kernel<KBW, SLOTS>), smem_a);
   if (err != cudaSuccess) return err;
   return ensure_smem_limit(reinterpret_cast<const void*>(decode_down_kernel), smem_b);
 }
 
-template <int KBW>
+template <int KBW, int SLOTS>
 cudaError_t launch_pair(const DecodeParams& p, int sm_count, size_t smem_a, size_t smem_b, cudaStream_t stream) {
-  cudaError_t aerr = raise_smem_limits<KBW>(smem_a, smem_b);
+  cudaError_t aerr = raise_smem_limits<KBW, SLOTS>(smem_a, smem_b);
   if (aerr != cudaSuccess) return aerr;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -554,7 +561,7 @@ cudaError_t launch_pair(const DecodeParams& p, int sm_count, size_t smem_a, size
   cfg.dynamicSmemBytes = smem_a;
   {
     LaunchScope ls("decode.gate_up", stream);
-    cudaError_t err = cudaLaunchKernelEx(&cfg, decode_gate_up_kernel<KBW>, p);
+    cudaError_t err = cudaLaunchKernelEx(&cfg, decode_gate_up_kernel<KBW, SLOTS>, p);
     if (err != cudaSuccess) return err;
   }
   cfg.gridDim = dim3(std::max(1, std::min(sm_count, p.H / 16)));
@@ -629,10 +636,11 @@ cudaError_t launch_decode_forward(const DecodeArgs& a, cudaStream_t stream) {
   p.out = a.out;
   const size_t smem_a = make_layout(true, p.M, p.k, p.E, p.H, r).total;
   const size_t smem_b = make_layout(false, p.M, p.k, p.E, p.H, 0).total;
-  switch (kbw_of(p.H)) {
-    case 1: return launch_pair<1>(p, di.sm_count, smem_a, smem_b, stream);
-    default: return launch_pair<2>(p, di.sm_count, smem_a, smem_b, stream);
+  if (kbw_of(p.H) == 1) {
+    if (slots_for(p.M, p.H) == 8) return launch_pair<1, 8>(p, di.sm_count, smem_a, smem_b, stream);
+    return launch_pair<1, 4>(p, di.sm_count, smem_a, smem_b, stream);
   }
+  return launch_pair<2, 4>(p, di.sm_count, smem_a, smem_b, stream);
 }
 
 }  // namespace e4b
