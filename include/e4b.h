@@ -317,15 +317,17 @@ E4B_API e4b_status e4b_moe_expert_forward(const uint16_t* x, int64_t M, const fl
                                   e4b_stream stream);
 /* Same, with the implementation chosen explicitly (tests and benchmarks).
  * E4B_PATH_AUTO takes the decode kernel when it can run the shape -- 1 <= M <= 8,
- * k <= 32, E <= 512, H <= 4096, I <= 4096 and its shared-memory plan fits -- and
+ * k <= 32, E <= 512, H <= 4096, I <= 3072 and its shared-memory plan fits -- and
  * the grouped path otherwise.  E4B_PATH_DECODE on any other shape returns
  * E4B_ERR_UNSUPPORTED and e4b_last_error() names the limit.
  * The decode path is one cooperative launch of one CTA per SM (at most 1024
  * CTAs): it needs the whole grid resident at once, so a launch that cannot get
  * every SM it asks for fails with E4B_ERR_CUDA instead of waiting.  Its CTAs
- * meet at a grid barrier whose slots live in the workspace and are tagged with
- * the launch's grid id: a workspace needs no initialisation for it, and the
- * barrier keeps no state from one call to the next. */
+ * meet at a grid barrier whose slots and epoch word live in the workspace:
+ * each call tags its slots with the epoch + 1 and advances the epoch, so a
+ * workspace needs no initialisation for it (garbage, or the grouped path's
+ * data, is fine) and graph replays work; two calls that share a workspace
+ * must not overlap on the GPU. */
 E4B_API e4b_status e4b_moe_expert_forward_path(const uint16_t* x, int64_t M, const float* router_logits,
                                        int k, int renormalize, const e4b_expert_stack* w,
                                        uint16_t* out, void* workspace, size_t workspace_bytes,
@@ -367,8 +369,8 @@ E4B_API e4b_status e4b_moe_expert_backward(const uint16_t* x, int64_t M, const f
  *
  * Computes exactly what e4b_moe_expert_forward() computes for 1 <= M <= 8
  * tokens, with the decode kernel, but takes no workspace: its scratch (the
- * SwiGLU activations of the routed slots, M*k*I bf16 values, plus one 64-bit
- * slot per CTA for the kernel's grid barrier) lives in one statically
+ * SwiGLU activations of the routed slots, M*k*I bf16 values, plus the slots
+ * and epoch word of the kernel's grid barrier) lives in one statically
  * sized device array of the library, 528 KiB, which every GPU that loads the
  * library holds until the process exits.  Requires M*k*I <= 262144 (for example M = 8, k = 8,
  * I <= 4096); larger shapes return E4B_ERR_UNSUPPORTED with a message.  The

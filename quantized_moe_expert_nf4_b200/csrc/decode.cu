@@ -8,7 +8,7 @@
 //
 //   prologue  every CTA routes the M <= 8 tokens (top-k + weights) and lists
 //             the touched experts (ascending id); only those are read.
-//   phase 1   gate_up: the CTA's contiguous run of items (8 gate + 8 up rows
+//   phase 1   gate_up: the CTA's contiguous run of items (16 gate + 16 up rows
 //             of one touched expert over all of K = H) -> SiLU(gate) * up
 //             (+ LoRA delta) -> h (bf16, [M*k, I], slot order) in the workspace.
 //   barrier   grid-wide: every CTA's h is written.
@@ -19,22 +19,32 @@
 //             the result is deterministic and needs no extra kernel.
 //
 // One producer warp streams the packed rows and their fp32 absmax with bulk
-// asynchronous copies (one per row, mbarrier transaction counts) through a
-// ring of shared-memory stages: first phase 1's items, then -- without waiting
-// for the barrier, since weights do not depend on h -- phase 2's stages, so
-// HBM keeps streaming the down rows while phase 1 computes and the barrier
-// resolves.  Sixteen math warps decode and multiply: nibbles become bf16 pairs
+// asynchronous copies (mbarrier transaction counts) through a ring of
+// shared-memory stages: first phase 1's items, then -- without waiting for the
+// barrier, since weights do not depend on h -- phase 2's stages, so HBM keeps
+// streaming the down rows while phase 1 computes and the barrier resolves.
+// A copy engine pays a fixed cost per copy (measured on B200: 1 KB copies
+// stream at about half the rate of 4 KB ones), so rows travel four at a time:
+// a block of 16 rows is four copies of 4 consecutive rows, each copy 32 bytes
+// (mod 128) past the previous one.  MMA row g (and g + 8) reads row
+// 4 (g % 4) + g / 4 (+ 2) of its block, so the four rows a half-warp's
+// fragment loads touch lie in four different copies, on four different bank
+// groups.  Sixteen math warps decode and multiply: nibbles become bf16 pairs
 // through a per-lane replicated byte -> bf16x2 codebook table (lane l reads
 // only bank l) and feed mma.sync m16n8k16 with the weight rows as MMA rows and
 // the <= 8 tokens as the 8 MMA columns.  Each MMA stays inside one 64-element
 // absmax block, so the block's fp32 absmax scales the products (no rounding of
-// the scale).  Rows are staged with a stride of 32 mod 128 bytes so that the
-// fragment loads are conflict-free.
+// the scale).
 //
-// The grid barrier is stateless: each CTA publishes the launch's %gridid (a
-// number the hardware gives every grid launch in a context) in its own slot of
-// the workspace, and waits until every slot holds that number, so a workspace
-// needs no initialisation and no reset.  Every wait is bounded; a wait that
+// The grid barrier needs no initialised workspace: a 64-bit epoch word sits
+// beside one slot per CTA.  Every CTA reads the epoch e at its start, publishes
+// e + 1 in its own slot once its h is written, and waits until every slot
+// holds e + 1; CTA 0 then stores e + 1 as the new epoch (every CTA read e
+// before it published, so none reads the new value in this launch).  Stale
+// slots of earlier calls hold smaller tags and garbage matches a 64-bit tag
+// only by chance, so a fresh workspace works, as does one the grouped path
+// wrote in between, and graph replays (which repeat the grid launch's own
+// identifiers) still get a new tag each time.  Every wait is bounded; a wait that
 // gives up records an error code in the workspace's error word, marks the CTA
 // aborted (later waits return at once, the results are unspecified) and the
 // kernel still runs to its end.
@@ -57,12 +67,13 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kGroups = 2;              // phase 1: items alternate between two groups of math warps
 constexpr int kGW = kMath / kGroups;    // warps per group
 constexpr int kMaxSPW = 4;              // spans (128 k) per warp of an item: H <= 8 * 4 * 128 = 4096
-constexpr int kMaxPPW = 4;              // (expert, k-block) pairs per warp of a down stage
-constexpr int kMaxKBI = kMath * kMaxPPW;  // k-blocks of a down row: I <= 4096
+constexpr int kMaxPPW = 3;              // (expert, k-block) pairs per warp of a down stage
+constexpr int kMaxDPE = 4;              // down experts per stage (8 copies each: one producer lane per copy)
+constexpr int kMaxKBI = kMath * kMaxPPW;  // k-blocks of a down row: I <= 3072
 constexpr int kMaxGrid = 1024;          // barrier slots in the workspace
 constexpr int kMaxStages = 32;
 constexpr uint32_t kLutBytes = 256 * 32 * 4;
-constexpr uint32_t kRedBytes = kGroups * 2 * kGW * 32 * 16;  // phase 1: [group][parity][warp][lane] float4
+constexpr uint32_t kRedBytes = kGroups * 2 * kGW * 2 * 32 * 16;  // phase 1: [group][parity][warp][tile][lane] float4
 constexpr int kBarGroup0 = 1;           // named barriers: 1, 2 (groups), 3 (all math warps)
 constexpr int kBarMath = 3;
 
@@ -82,34 +93,26 @@ struct FusedParams {
   uint16_t* h;                 // [S, I] bf16 (slot order)
   uint16_t* out;               // [M, H] bf16
   int* err;                    // error word
-  unsigned long long* flags;   // [gridDim.x] barrier slots
+  unsigned long long* flags;   // [kMaxGrid] barrier slots, then the epoch word
   int stages;                  // ring depth (even)
   int dpe;                     // down experts per phase-2 stage
 };
 
 __host__ __device__ inline uint32_t al(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
-// Shared-memory stride of a staged packed row of K elements: K/2 bytes padded
-// to 32 mod 128, so the 8 rows of a fragment load fall on distinct banks.
-__host__ __device__ inline uint32_t row_stride(int K) {
-  const uint32_t b = static_cast<uint32_t>(K / 2);
-  return b + (160u - b % 128u) % 128u;
-}
-
-// absmax rows: copied one by one when a row is a 16-byte multiple (KB % 4 ==
-// 0), with a stride of 4 mod 8 floats; otherwise as chunks of 8 contiguous
-// rows (stride KB, odd or 2 mod 4: still distinct banks for 8 rows).
-__host__ __device__ inline bool am_by_rows(int KB) { return KB % 4 == 0; }
+// A staged block of 16 rows of K elements: packed copy c (rows 4c .. 4c+3,
+// dense, K/2 bytes apart) at c * copy_stride(K) = c * (2K + 32) bytes, which is
+// 32 mod 128, then the absmax copies (4 rows x KB floats each) at
+// am_stride(KB) = 16 KB + pad bytes, 16 mod 128.  A gate_up stage holds two
+// such blocks side by side (gate copies 0-3, up copies 4-7, then their
+// absmax copies 0-7); a down stage holds one block per expert.
+__host__ __device__ inline uint32_t copy_stride(int K) { return static_cast<uint32_t>(2 * K + 32); }
 __host__ __device__ inline uint32_t am_stride(int KB) {
-  return static_cast<uint32_t>(am_by_rows(KB) ? (KB % 8 == 4 ? KB : KB + 4) : KB);
+  const uint32_t b = static_cast<uint32_t>(16 * KB);
+  return b + (144u - b % 128u) % 128u;
 }
-
-// A block of 16 staged rows of K elements with their absmax: bytes and the
-// absmax offset inside it.
-__host__ __device__ inline uint32_t rows16_am_off(int K) { return 16 * row_stride(K); }
-__host__ __device__ inline uint32_t rows16_bytes(int K) {
-  return rows16_am_off(K) + al(16 * am_stride(K / 64) * 4, 16);
-}
+__host__ __device__ inline uint32_t gu_stage_bytes(int H) { return 8 * copy_stride(H) + 8 * am_stride(H / 64); }
+__host__ __device__ inline uint32_t dn_block_bytes(int I) { return 4 * copy_stride(I) + 4 * am_stride(I / 64); }
 
 struct Smem {
   uint32_t lut, red, ids, w, uidx, touched, slotmap, xa, bars, ring, total;
@@ -170,14 +173,14 @@ __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, u
 
 __device__ __forceinline__ uint2 lds64(const unsigned char* p) { return *reinterpret_cast<const uint2*>(p); }
 
-__device__ __forceinline__ unsigned long long grid_id() {
-  unsigned long long v;
-  asm volatile("mov.u64 %0, %%gridid;" : "=l"(v));
-  return v;
-}
-
 __device__ __forceinline__ void st_release_gpu(unsigned long long* p, unsigned long long v) {
   asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long ld_relaxed_gpu(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
 }
 
 __device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long long* p) {
@@ -277,26 +280,19 @@ __device__ void prologue(const FusedParams& p, uint32_t* lut, int* ids_s, float*
   __syncthreads();
 }
 
-// Copies of 16 rows (rows [0, 8) from row_a, [8, 16) from row_b) of a packed
-// matrix with K columns, and their absmax, into a staged block.  Run by the
-// whole producer warp.
-__device__ __forceinline__ void copy_rows16(unsigned char* dst, uint64_t* full, const uint8_t* packed,
-                                            const float* absmax, int K, int64_t row_a, int64_t row_b) {
-  const int lane = threadIdx.x & 31;
+// Copy `lane_c` (0-3 packed, 4-7 absmax) of a block of 16 rows starting at
+// global row `row0` of a packed matrix with K columns into the block at `dst`
+// (packed copies at dst + c * copy_stride, absmax copies at am_dst + c * am_stride).
+__device__ __forceinline__ void copy_block_part(int lane_c, unsigned char* dst, unsigned char* am_dst,
+                                                uint64_t* full, const uint8_t* packed, const float* absmax, int K,
+                                                int64_t row0) {
   const int KB = K / 64;
-  const uint32_t rowb = static_cast<uint32_t>(K / 2), ps = row_stride(K), sa = am_stride(KB);
-  unsigned char* am = dst + rows16_am_off(K);
-  if (lane < 16) {
-    const int64_t row = (lane < 8 ? row_a : row_b) + (lane & 7);
-    bulk_g2s(dst + lane * ps, packed + row * rowb, rowb, full);
-  } else if (am_by_rows(KB)) {
-    const int i = lane - 16;
-    const int64_t row = (i < 8 ? row_a : row_b) + (i & 7);
-    bulk_g2s(am + i * sa * 4, absmax + row * KB, static_cast<uint32_t>(KB * 4), full);
-  } else if (lane < 18) {
-    const int i = lane - 16;
-    bulk_g2s(am + i * 8 * sa * 4, absmax + (i == 0 ? row_a : row_b) * KB, static_cast<uint32_t>(8 * KB * 4), full);
-  }
+  const int c = lane_c & 3;
+  const int64_t row = row0 + 4 * c;
+  if (lane_c < 4)
+    bulk_g2s(dst + c * copy_stride(K), packed + row * (K / 2), static_cast<uint32_t>(2 * K), full);
+  else
+    bulk_g2s(am_dst + c * am_stride(KB), absmax + row * KB, static_cast<uint32_t>(16 * KB), full);
 }
 
 // ---------------------------------------------------------------------------
@@ -307,10 +303,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
   extern __shared__ __align__(128) unsigned char smem[];
   const int H = p.H, I = p.I, KB = H / 64, KBI = I / 64;
   const int RS = p.stages, DPE = p.dpe;
-  const uint32_t ps_gu = row_stride(H), sa_gu = am_stride(KB), am_gu = rows16_am_off(H);
-  const uint32_t ps_dn = row_stride(I), sa_dn = am_stride(KBI), am_dn = rows16_am_off(I);
-  const uint32_t exp_dn = rows16_bytes(I);
-  const uint32_t slot = al(max(rows16_bytes(H), static_cast<uint32_t>(DPE) * exp_dn), 128);
+  const uint32_t cs_gu = copy_stride(H), as_gu = am_stride(KB) / 4, am_gu = 8 * cs_gu;
+  const uint32_t cs_dn = copy_stride(I), as_dn = am_stride(KBI) / 4, am_dn = 4 * cs_dn;
+  const uint32_t exp_dn = dn_block_bytes(I);
+  const uint32_t slot = al(max(gu_stage_bytes(H), static_cast<uint32_t>(DPE) * exp_dn), 128);
   const Smem L = make_smem(p.M, p.k, p.E, p.r, RS, slot);
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L.lut);
   float4* red = reinterpret_cast<float4*>(smem + L.red);
@@ -328,6 +324,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
+  // This launch's barrier tag: the workspace's epoch + 1 (read before this
+  // CTA publishes anything; see the barrier below).
+  const unsigned long long tag = (warp == 0) ? ld_relaxed_gpu(p.flags + kMaxGrid) + 1 : 0;
   if (tid == 0) {
     abort_s = 0;
     for (int s = 0; s < RS; ++s) {
@@ -341,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
   const int G = static_cast<int>(gridDim.x), bid = static_cast<int>(blockIdx.x);
 
   // Phase-1 items: a contiguous run per CTA (consecutive items = consecutive rows).
-  const int ipe = I / 8;
+  const int ipe = I / 16;
   const int nitems = nU * ipe;
   const int q_it = nitems / G, rem_it = nitems % G;
   const int i0 = bid * q_it + min(bid, rem_it);
@@ -361,19 +360,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
       if (j >= RS && !ring_wait(&empty[s], ((j / RS) - 1) & 1, &abort_s, p.err, kErrWaitEmpty)) break;
       unsigned char* st = ring + static_cast<uint32_t>(s) * slot;
       if (j < n_gu) {
+        // 16 gate rows (block 0) and the matching 16 up rows (block 1): lanes
+        // 0-3 / 8-11 the gate / up packed copies, 4-7 / 12-15 their absmax.
         const int it = i0 + j, u = it / ipe, rb = it % ipe;
-        const int64_t grow = static_cast<int64_t>(touched[u]) * 2 * I + rb * 8;
-        if (lane == 0) mbar_arrive_expect_tx(&full[s], 16u * (H / 2) + 16u * KB * 4);
+        const int64_t grow = static_cast<int64_t>(touched[u]) * 2 * I + rb * 16;
+        if (lane == 0) mbar_arrive_expect_tx(&full[s], 32u * (H / 2) + 32u * KB * 4);
         __syncwarp();
-        copy_rows16(st, &full[s], p.gu_packed, p.gu_absmax, H, grow, grow + I);
+        if (lane < 16) {
+          const int blk = lane >> 3;
+          copy_block_part(lane & 7, st + blk * 4 * cs_gu, st + am_gu + blk * 16 * as_gu, &full[s], p.gu_packed,
+                          p.gu_absmax, H, grow + blk * I);
+        }
       } else {
+        // One block of 16 down rows per expert: lane 8 ei + c issues copy c of expert ei.
         const int jd = j - n_gu, ch = jd % nch, rb = bid + (jd / nch) * G;
         const int u0 = ch * DPE, ne = min(DPE, nU - u0);
         if (lane == 0) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(ne) * (16u * (I / 2) + 16u * KBI * 4));
         __syncwarp();
-        for (int ei = 0; ei < ne; ++ei) {
+        if (lane < 8 * ne) {
+          const int ei = lane >> 3;
           const int64_t row0 = static_cast<int64_t>(touched[u0 + ei]) * H + rb * 16;
-          copy_rows16(st + ei * exp_dn, &full[s], p.dn_packed, p.dn_absmax, I, row0, row0 + 8);
+          copy_block_part(lane & 7, st + ei * exp_dn, st + ei * exp_dn + am_dn, &full[s], p.dn_packed, p.dn_absmax, I,
+                          row0);
         }
       }
       ++issued;
@@ -449,65 +457,78 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
       ring_wait(&full[s], (jj / RS) & 1, &abort_s, p.err, kErrWaitFull);
       const unsigned char* st = ring + static_cast<uint32_t>(s) * slot;
       const float* am = reinterpret_cast<const float*>(st + am_gu);
-      float c[4] = {0.f, 0.f, 0.f, 0.f};
+      // Tile T: MMA row g = gate column 4 (g % 4) + 2T + g / 4 of the item
+      // (copy g % 4 of the gate block, row 2T + g / 4 in it); row g + 8 = the
+      // same column's up row (copy 4 + g % 4).
+      float c[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
       for (int q = 0; q < SPW; ++q) {
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const int kb = 2 * (wi + kGW * q) + hh;
           if (kb < KB) {
-            const uint2 w0 = lds64(st + g * ps_gu + kb * 32 + 8 * t);
-            const uint2 w1 = lds64(st + (g + 8) * ps_gu + kb * 32 + 8 * t);
-            const float a0 = am[g * sa_gu + kb], a1 = am[(g + 8) * sa_gu + kb];
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
-            block_mma(lut_lane, w0, w1, xr[q][hh], d);
-            c[0] = fmaf(a0, d[0], c[0]);
-            c[1] = fmaf(a0, d[1], c[1]);
-            c[2] = fmaf(a1, d[2], c[2]);
-            c[3] = fmaf(a1, d[3], c[3]);
+#pragma unroll
+            for (int T = 0; T < 2; ++T) {
+              const int r = 2 * T + (g >> 2), cg = g & 3;
+              const uint32_t off = r * (H / 2) + kb * 32 + 8 * t;
+              const uint2 w0 = lds64(st + cg * cs_gu + off);
+              const uint2 w1 = lds64(st + (4 + cg) * cs_gu + off);
+              const float a0 = am[cg * as_gu + r * KB + kb], a1 = am[(4 + cg) * as_gu + r * KB + kb];
+              float d[4] = {0.f, 0.f, 0.f, 0.f};
+              block_mma(lut_lane, w0, w1, xr[q][hh], d);
+              c[T][0] = fmaf(a0, d[0], c[T][0]);
+              c[T][1] = fmaf(a0, d[1], c[T][1]);
+              c[T][2] = fmaf(a1, d[2], c[T][2]);
+              c[T][3] = fmaf(a1, d[3], c[T][3]);
+            }
           }
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive_cnt(&empty[s], kMath / kGW);
       const int par = (jj / kGroups) & 1;
-      red[((gi * 2 + par) * kGW + wi) * 32 + lane] = make_float4(c[0], c[1], c[2], c[3]);
+      float4* rp = red + (((gi * 2 + par) * kGW + wi) * 2) * 32 + lane;
+      rp[0] = make_float4(c[0][0], c[0][1], c[0][2], c[0][3]);
+      rp[32] = make_float4(c[1][0], c[1][1], c[1][2], c[1][3]);
       named_bar(kBarGroup0 + gi, kGW * 32);
       if (wi == (jj / kGroups) % kGW) {
         // This warp finishes the item: the group's partials in warp order,
         // then SwiGLU (+ LoRA delta) for the tokens routed to the expert.
-        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int w = 0; w < kGW; ++w) {
-          const float4 v = red[((gi * 2 + par) * kGW + w) * 32 + lane];
-          sum.x += v.x;
-          sum.y += v.y;
-          sum.z += v.z;
-          sum.w += v.w;
-        }
         const int it = i0 + jj, u = it / ipe, rb = it % ipe;
         const int e = touched[u];
-        const int col = rb * 8 + g;  // h column == gate row index
-        const float gate_v[2] = {sum.x, sum.y}, up_v[2] = {sum.z, sum.w};
 #pragma unroll
-        for (int qq = 0; qq < 2; ++qq) {
-          const int tok = 2 * t + qq;
-          if (tok >= p.M) continue;
-          const int sl = slotmap[u * kMaxM + tok];
-          if (sl < 0) continue;
-          float gv = gate_v[qq], uv = up_v[qq];
-          if (p.r > 0) {
-            const uint16_t* bg = p.lora_B + (static_cast<int64_t>(e) * 2 * I + col) * p.r;
-            const uint16_t* bu = p.lora_B + (static_cast<int64_t>(e) * 2 * I + I + col) * p.r;
-            float dg = 0.f, du = 0.f;
-            for (int rho = 0; rho < p.r; ++rho) {
-              const float xv = xa[sl * p.r + rho];
-              dg = fmaf(xv, bf16_bits_to_float(bg[rho]), dg);
-              du = fmaf(xv, bf16_bits_to_float(bu[rho]), du);
-            }
-            gv = fmaf(p.lora_scale, dg, gv);
-            uv = fmaf(p.lora_scale, du, uv);
+        for (int T = 0; T < 2; ++T) {
+          float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int w = 0; w < kGW; ++w) {
+            const float4 v = red[(((gi * 2 + par) * kGW + w) * 2 + T) * 32 + lane];
+            sum.x += v.x;
+            sum.y += v.y;
+            sum.z += v.z;
+            sum.w += v.w;
           }
-          p.h[static_cast<int64_t>(sl) * I + col] = float_to_bf16_bits(silu_f32(gv) * uv);
+          const int col = rb * 16 + 4 * (g & 3) + 2 * T + (g >> 2);  // h column == gate row index
+          const float gate_v[2] = {sum.x, sum.y}, up_v[2] = {sum.z, sum.w};
+#pragma unroll
+          for (int qq = 0; qq < 2; ++qq) {
+            const int tok = 2 * t + qq;
+            if (tok >= p.M) continue;
+            const int sl = slotmap[u * kMaxM + tok];
+            if (sl < 0) continue;
+            float gv = gate_v[qq], uv = up_v[qq];
+            if (p.r > 0) {
+              const uint16_t* bg = p.lora_B + (static_cast<int64_t>(e) * 2 * I + col) * p.r;
+              const uint16_t* bu = p.lora_B + (static_cast<int64_t>(e) * 2 * I + I + col) * p.r;
+              float dg = 0.f, du = 0.f;
+              for (int rho = 0; rho < p.r; ++rho) {
+                const float xv = xa[sl * p.r + rho];
+                dg = fmaf(xv, bf16_bits_to_float(bg[rho]), dg);
+                du = fmaf(xv, bf16_bits_to_float(bu[rho]), du);
+              }
+              gv = fmaf(p.lora_scale, dg, gv);
+              uv = fmaf(p.lora_scale, du, uv);
+            }
+            p.h[static_cast<int64_t>(sl) * I + col] = float_to_bf16_bits(silu_f32(gv) * uv);
+          }
         }
       }
     }
@@ -516,17 +537,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
   // --------------------------------------------------------- grid barrier
   named_bar(kBarMath, kMath * 32);  // every h store of this CTA is issued
   if (warp == 0) {
-    const unsigned long long gid = grid_id();
     if (lane == 0) {
       __threadfence();
-      st_release_gpu(p.flags + bid, gid);
+      st_release_gpu(p.flags + bid, tag);
     }
     __syncwarp();
     const unsigned long long t0 = global_ns();
     while (true) {
       bool ready = true;
-      for (int c = lane; c < G; c += 32) ready = ready && ld_acquire_gpu(p.flags + c) == gid;
-      if (__all_sync(0xffffffffu, ready)) break;
+      for (int c = lane; c < G; c += 32) ready = ready && ld_acquire_gpu(p.flags + c) == tag;
+      if (__all_sync(0xffffffffu, ready)) {
+        // Every CTA has read the old epoch: advance it for the next launch.
+        if (bid == 0 && lane == 0) st_release_gpu(p.flags + kMaxGrid, tag);
+        break;
+      }
       if (abort_s) break;
       if (global_ns() - t0 > kWaitLimitNs) {
         if (lane == 0) {
@@ -575,11 +599,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
         const int pi = warp + kMath * q;
         if (pi < np) {
           const int ei = pi / KBI, kb = pi % KBI, u = u0 + ei;
+          // MMA row g = block row 4 (g % 4) + g / 4, row g + 8 = that + 2.
           const unsigned char* base = st + ei * exp_dn;
           const float* am = reinterpret_cast<const float*>(base + am_dn);
-          const uint2 w0 = lds64(base + g * ps_dn + kb * 32 + 8 * t);
-          const uint2 w1 = lds64(base + (g + 8) * ps_dn + kb * 32 + 8 * t);
-          const float a0 = am[g * sa_dn + kb], a1 = am[(g + 8) * sa_dn + kb];
+          const int cg = g & 3, r = g >> 2;
+          const uint32_t off = cg * cs_dn + r * (I / 2) + kb * 32 + 8 * t;
+          const uint2 w0 = lds64(base + off);
+          const uint2 w1 = lds64(base + off + I);  // two rows further
+          const float a0 = am[cg * as_dn + r * KBI + kb], a1 = am[cg * as_dn + (r + 2) * KBI + kb];
           float d[4] = {0.f, 0.f, 0.f, 0.f};
           block_mma(lut_lane, w0, w1, reinterpret_cast<const uint32_t*>(hb[q]), d);
           const int s0 = (2 * t < p.M) ? slotmap[u * kMaxM + 2 * t] : -1;
@@ -608,12 +635,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
             sum.z += v.z;
             sum.w += v.w;
           }
-          const int row0 = (bid + rbq * G) * 16 + g;
+          const int row0 = (bid + rbq * G) * 16 + 4 * (g & 3) + (g >> 2);
           const float v[4] = {sum.x, sum.y, sum.z, sum.w};
 #pragma unroll
           for (int q2 = 0; q2 < 4; ++q2) {
             const int tok = 2 * t + (q2 & 1);
-            const int row = row0 + ((q2 >> 1) ? 8 : 0);
+            const int row = row0 + ((q2 >> 1) ? 2 : 0);
             if (tok < p.M) p.out[static_cast<int64_t>(tok) * H + row] = float_to_bf16_bits(v[q2]);
           }
         }
@@ -638,8 +665,7 @@ KernelFn pick_ppw(int ppw) {
   switch (ppw) {
     case 1: return decode_fused_kernel<SPW, 1>;
     case 2: return decode_fused_kernel<SPW, 2>;
-    case 3: return decode_fused_kernel<SPW, 3>;
-    default: return decode_fused_kernel<SPW, 4>;
+    default: return decode_fused_kernel<SPW, 3>;
   }
 }
 
@@ -665,8 +691,8 @@ std::string make_plan(int M, int k, int E, int H, int I, int r, size_t smem_limi
   pl->spw = (nsp + kGW - 1) / kGW;
   if (pl->spw > kMaxSPW) return "the decode path takes H <= " + std::to_string(kGW * kMaxSPW * 128);
   if (KBI > kMaxKBI) return "the decode path takes I <= " + std::to_string(kMaxKBI * 64);
-  const uint32_t gu = rows16_bytes(H), dn = rows16_bytes(I);
-  pl->dpe = std::max(1, std::min(static_cast<int>(gu / dn), kMaxKBI / KBI));
+  const uint32_t gu = gu_stage_bytes(H), dn = dn_block_bytes(I);
+  pl->dpe = std::max(1, std::min({static_cast<int>(gu / dn), kMaxDPE, kMaxKBI / KBI}));
   pl->ppw = (pl->dpe * KBI + kMath - 1) / kMath;
   pl->slot = al(std::max(gu, static_cast<uint32_t>(pl->dpe) * dn), 128);
   const size_t fixed = make_smem(M, k, E, r, 0, pl->slot).ring + 2 * kMaxStages * 8;
@@ -676,7 +702,7 @@ std::string make_plan(int M, int k, int E, int H, int I, int r, size_t smem_limi
   if (st < 2) return "the decode kernel's shared-memory ring does not fit this shape";
   pl->stages = st;
   pl->smem = make_smem(M, k, E, r, st, pl->slot).total;
-  const int items_upper = std::min(M * k, E) * (I / 8);
+  const int items_upper = std::min(M * k, E) * (I / 16);
   pl->grid = std::max(1, std::min({sm_count, kMaxGrid, std::max(items_upper, H / 16)}));
   return "";
 }
@@ -686,11 +712,11 @@ struct DecodeWs {
 };
 
 // Workspace: the error word every workspace begins with (256-byte slot), the
-// grid barrier's slots (one 64-bit word per CTA), h [M*k, I] bf16.
+// grid barrier's slots (one 64-bit word per CTA) and its epoch word, h [M*k, I] bf16.
 DecodeWs decode_ws(int64_t M, int k, int64_t I) {
   DecodeWs w;
   w.flags = 256;
-  w.h = w.flags + static_cast<size_t>(kMaxGrid) * 8;
+  w.h = w.flags + align_up(static_cast<size_t>(kMaxGrid + 1) * 8, 256);
   w.total = w.h + align_up(static_cast<size_t>(M * k * I * 2), 256);
   return w;
 }

@@ -149,8 +149,9 @@ def test_forward_decode_path_all_tokens(name, cfg, M):
 
 @pytest.mark.parametrize("name,M", [("olmoe", 1), ("olmoe", 8), ("gptoss", 3)])
 def test_forward_decode_reuses_one_workspace_across_changing_inputs(name, M):
-    """The decode kernel's grid barrier keeps no state between calls: one
-    workspace (filled with garbage first) serves consecutive calls on new
+    """The decode kernel's grid barrier needs no initialised workspace and
+    tags every call anew (graph replays repeat the launch's own identifiers):
+    one workspace, filled with garbage first, serves consecutive calls on new
     inputs, eagerly and as replays of one captured graph whose input buffers
     are refilled between replays; every result equals a fresh grouped-path
     forward of the same inputs to the layer tolerance, and eager and replayed

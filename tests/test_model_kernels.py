@@ -86,39 +86,38 @@ def test_decode_block_fragment_mapping(K):
 
 # ---- csrc/decode.cu: the fused kernel's shared-memory plan and copies -------------
 SMEM_LIMIT = 227 * 1024 - 1024   # opt-in dynamic shared memory minus the kernel's reserve
-SMS = 148
 
 
 def _al(v, a):
     return (v + a - 1) // a * a
 
 
-def _row_stride(K):
-    b = K // 2
-    return b + (160 - b % 128) % 128
-
-
-def _am_by_rows(KB):
-    return KB % 4 == 0
+def _copy_stride(K):
+    return 2 * K + 32
 
 
 def _am_stride(KB):
-    return (KB if KB % 8 == 4 else KB + 4) if _am_by_rows(KB) else KB
+    b = 16 * KB
+    return b + (144 - b % 128) % 128
 
 
-def _rows16_bytes(K):
-    return 16 * _row_stride(K) + _al(16 * _am_stride(K // 64) * 4, 16)
+def _gu_stage(H):
+    return 8 * _copy_stride(H) + 8 * _am_stride(H // 64)
+
+
+def _dn_block(I):
+    return 4 * _copy_stride(I) + 4 * _am_stride(I // 64)
 
 
 def _plan(M, k, E, H, I, r):
     KB, KBI = H // 64, I // 64
     spw = -(-((KB + 1) // 2) // 8)
-    gu, dn = _rows16_bytes(H), _rows16_bytes(I)
-    dpe = max(1, min(gu // dn, 64 // KBI))
+    gu, dn = _gu_stage(H), _dn_block(I)
+    dpe = max(1, min(gu // dn, 4, 48 // KBI))
     ppw = -(-(dpe * KBI) // 16)
     slot = _al(max(gu, dpe * dn), 128)
     S = M * k
-    o = 256 * 32 * 4 + 2 * 2 * 8 * 32 * 16
+    o = 256 * 32 * 4 + 2 * 2 * 8 * 2 * 32 * 16
     for n in (S * 4, S * 4, E * 4, S * 4, S * 8 * 4):
         o = _al(o + n, 16)
     if r:
@@ -129,23 +128,28 @@ def _plan(M, k, E, H, I, r):
     return dict(spw=spw, ppw=ppw, dpe=dpe, slot=slot, stages=stages, ring=ring, total=ring + stages * slot)
 
 
-def _copies_rows16(K, row_a, row_b):
-    """(dst offset, src byte offset in packed, src byte offset in absmax, bytes) of one block of 16 rows."""
+def _block_copies(K, row0, dst, am_dst):
+    """(lane_c, dst, src byte offset in packed / absmax, bytes, is_absmax) of one staged block of 16 rows."""
     KB = K // 64
-    ps, sa = _row_stride(K), _am_stride(KB)
-    am = 16 * ps
-    pk, ab = [], []
-    for lane in range(16):
-        row = (row_a if lane < 8 else row_b) + (lane & 7)
-        pk.append((lane * ps, row * (K // 2), K // 2))
-    if _am_by_rows(KB):
-        for i in range(16):
-            row = (row_a if i < 8 else row_b) + (i & 7)
-            ab.append((am + i * sa * 4, row * KB * 4, KB * 4))
-    else:
-        for i in range(2):
-            ab.append((am + i * 8 * sa * 4, (row_a if i == 0 else row_b) * KB * 4, 8 * KB * 4))
-    return pk, ab
+    out = []
+    for lc in range(8):
+        c = lc & 3
+        row = row0 + 4 * c
+        if lc < 4:
+            out.append((dst + c * _copy_stride(K), row * (K // 2), 2 * K, False))
+        else:
+            out.append((am_dst + c * _am_stride(KB), row * KB * 4, 16 * KB, True))
+    return out
+
+
+def _check_copies(copies, slot, packed_bytes, absmax_bytes):
+    written = set()
+    for dst, src, n, is_am in copies:
+        assert dst % 16 == 0 and src % 16 == 0 and n % 16 == 0 and dst + n <= slot
+        assert src + n <= (absmax_bytes if is_am else packed_bytes)
+        assert not (set(range(dst, dst + n)) & written), "copies overlap"
+        written.update(range(dst, dst + n))
+    return written
 
 
 DECODE_SHAPES = [
@@ -154,80 +158,90 @@ DECODE_SHAPES = [
     (1, 4, 32, 2880, 2880, 0), (8, 4, 32, 2880, 2880, 0), (8, 8, 128, 2048, 768, 8), (3, 8, 128, 2048, 768, 8),
     (1, 2, 8, 256, 128, 0), (8, 2, 8, 256, 128, 0), (5, 3, 12, 192, 320, 0), (3, 2, 6, 128, 192, 8),
     (2, 6, 40, 448, 128, 0), (7, 32, 33, 128, 64, 0), (8, 2, 8, 2880, 704, 0), (8, 2, 8, 4096, 128, 0),
-    (8, 8, 512, 128, 64, 0), (6, 1, 8, 256, 192, 0), (7, 4, 4, 256, 192, 0), (5, 3, 12, 192, 320, 0),
-    (4, 2, 4, 4096, 4096, 16),
+    (8, 8, 512, 128, 64, 0), (6, 1, 8, 256, 192, 0), (7, 4, 4, 256, 192, 0), (4, 2, 4, 3072, 3072, 16),
 ]
 
 
 @pytest.mark.parametrize("shape", DECODE_SHAPES)
 def test_decode_fused_plan_copies_and_reads_stay_in_bounds(shape):
     """Every bulk copy of a stage is 16-byte aligned at both ends, a multiple of
-    16 bytes, inside its slot and inside the source stack; the transaction
-    count equals the bytes copied; every fragment and absmax read of the math
-    warps stays inside the bytes the copies wrote; the plan fits the shared
-    memory and holds an even number of stages."""
+    16 bytes, inside its slot, disjoint from the others and inside the source
+    stack; the transaction count equals the bytes copied; every fragment and
+    absmax read of the math warps lies in bytes the copies wrote; the plan
+    fits the shared memory and holds an even number of stages."""
     M, k, E, H, I, r = shape
     pl = _plan(M, k, E, H, I, r)
     assert pl["total"] <= SMEM_LIMIT and pl["stages"] >= 2 and pl["stages"] % 2 == 0
-    assert pl["spw"] <= 4 and pl["ppw"] <= 4 and pl["ring"] % 128 == 0 and pl["slot"] % 128 == 0
+    assert pl["spw"] <= 4 and pl["ppw"] <= 3 and pl["dpe"] <= 4 and pl["ring"] % 128 == 0 and pl["slot"] % 128 == 0
     KB, KBI = H // 64, I // 64
-    # phase 1: every item of the largest expert id (the last rows of the stack)
-    gu_rows, gu_bytes = 2 * I * E, None
-    for rb in (0, I // 8 - 1):
-        grow = (E - 1) * 2 * I + rb * 8
-        pk, ab = _copies_rows16(H, grow, grow + I)
-        written = set()
-        for dst, src, n in pk:
-            assert dst % 16 == 0 and src % 16 == 0 and n % 16 == 0 and dst + n <= pl["slot"]
-            assert src + n <= gu_rows * (H // 2)
-            written.update(range(dst, dst + n))
-        for dst, src, n in ab:
-            assert dst % 16 == 0 and src % 16 == 0 and n % 16 == 0 and dst + n <= pl["slot"]
-            assert src + n <= gu_rows * KB * 4
-            written.update(range(dst, dst + n))
-        assert sum(n for _, _, n in pk + ab) == 16 * (H // 2) + 16 * KB * 4
-        ps, sa, am = _row_stride(H), _am_stride(KB), 16 * _row_stride(H)
+    cs, am0 = _copy_stride(H), 8 * _copy_stride(H)
+    # phase 1: the first and the last item of the last expert
+    for rb in (0, I // 16 - 1):
+        grow = (E - 1) * 2 * I + rb * 16
+        copies = []
+        for blk in range(2):
+            copies += _block_copies(H, grow + blk * I, blk * 4 * cs, am0 + blk * 4 * _am_stride(KB))
+        written = _check_copies(copies, pl["slot"], E * 2 * I * (H // 2), E * 2 * I * KB * 4)
+        assert sum(n for _, _, n, _ in copies) == 32 * (H // 2) + 32 * KB * 4
         for g in range(8):
             for t in range(4):
-                for kb in range(KB):
-                    for row in (g, g + 8):
-                        off = row * ps + kb * 32 + 8 * t
-                        assert set(range(off, off + 8)) <= written
-                        a = am + (row * sa + kb) * 4
-                        assert set(range(a, a + 4)) <= written
-    # phase 2: the last row block of the last experts
-    dn = _rows16_bytes(I)
+                for T in range(2):
+                    rr, cg = 2 * T + (g >> 2), g & 3
+                    for kb in range(KB):
+                        off = rr * (H // 2) + kb * 32 + 8 * t
+                        for base in (cg * cs, (4 + cg) * cs):
+                            assert set(range(base + off, base + off + 8)) <= written
+                        for ci in (cg, 4 + cg):
+                            a = am0 + ci * _am_stride(KB) + (rr * KB + kb) * 4
+                            assert set(range(a, a + 4)) <= written
+                        # the row read is column 4 (g % 4) + 2T + g / 4 of the item, in its copy
+                        assert 4 * cg + rr == 4 * (g & 3) + 2 * T + (g >> 2)
+    # phase 2: the last row block of the last experts, every expert count of a stage
+    exp, csd, amd = _dn_block(I), _copy_stride(I), 4 * _copy_stride(I)
     for ne in range(1, pl["dpe"] + 1):
-        total = 0
+        copies = []
         for ei in range(ne):
             row0 = (E - 1 - ei) * H + (H // 16 - 1) * 16
-            pk, ab = _copies_rows16(I, row0, row0 + 8)
-            for dst, src, n in pk + ab:
-                dst += ei * dn
-                assert dst % 16 == 0 and src % 16 == 0 and n % 16 == 0 and dst + n <= pl["slot"]
-                total += n
-            assert max(src + n for _, src, n in pk) <= E * H * (I // 2)
-            assert max(src + n for _, src, n in ab) <= E * H * KBI * 4
-        assert total == ne * (16 * (I // 2) + 16 * KBI * 4)
+            copies += _block_copies(I, row0, ei * exp, ei * exp + amd)
+        written = _check_copies(copies, pl["slot"], E * H * (I // 2), E * H * KBI * 4)
+        assert sum(n for _, _, n, _ in copies) == ne * (16 * (I // 2) + 16 * KBI * 4)
         assert ne * KBI <= 16 * pl["ppw"]
-
-
-@pytest.mark.parametrize("K", [128, 192, 320, 448, 704, 768, 1024, 2048, 2880, 4096])
-def test_decode_fused_fragment_reads_are_conflict_free(K):
-    """Rows staged 32 mod 128 bytes apart: the 8-byte fragment loads of each
-    half-warp (rows g = 4h .. 4h+3, t = 0..3) hit 32 distinct banks, and the
-    absmax loads of the 8 rows g fall on 8 distinct banks."""
-    ps, sa = _row_stride(K), _am_stride(K // 64)
-    assert ps % 128 == 32 and ps >= K // 2
-    for kb in range(K // 64):
-        for half in range(2):
-            banks = []
-            for g in range(4 * half, 4 * half + 4):
+        for ei in range(ne):
+            for g in range(8):
                 for t in range(4):
-                    w = (g * ps + kb * 32 + 8 * t) // 4
-                    banks += [w % 32, (w + 1) % 32]
-            assert len(set(banks)) == 32
-        assert len({(g * sa + kb) % 32 for g in range(8)}) == 8
+                    cg, rr = g & 3, g >> 2
+                    for kb in range(KBI):
+                        off = ei * exp + cg * csd + rr * (I // 2) + kb * 32 + 8 * t
+                        for o in (off, off + I):
+                            assert set(range(o, o + 8)) <= written
+                        for row in (rr, rr + 2):
+                            a = ei * exp + amd + cg * _am_stride(KBI) + (row * KBI + kb) * 4
+                            assert set(range(a, a + 4)) <= written
+
+
+@pytest.mark.parametrize("K", [128, 192, 320, 448, 704, 768, 1024, 2048, 2880, 3072, 4096])
+def test_decode_fused_fragment_reads_are_conflict_free(K):
+    """Copies 32 mod 128 bytes apart: the 8-byte fragment loads of each
+    half-warp (MMA rows g = 4h .. 4h+3 -> copies 0-3, one row each; t = 0..3)
+    hit 32 distinct banks; the absmax loads of the 8 rows g touch at most two
+    addresses per bank."""
+    cs, asz = _copy_stride(K), _am_stride(K // 64)
+    assert cs % 128 == 32 and asz % 128 == 16
+    KB = K // 64
+    for kb in range(KB):
+        for half in range(2):
+            for r2 in (0, 2):
+                banks = []
+                for g in range(4 * half, 4 * half + 4):
+                    for t in range(4):
+                        w = ((g & 3) * cs + ((g >> 2) + r2) * (K // 2) + kb * 32 + 8 * t) // 4
+                        banks += [w % 32, (w + 1) % 32]
+                assert len(set(banks)) == 32
+        words = [((g & 3) * asz + ((g >> 2) * KB + kb) * 4) // 4 for g in range(8)]
+        per_bank = {}
+        for w in words:
+            per_bank.setdefault(w % 32, set()).add(w)
+        assert max(len(v) for v in per_bank.values()) <= 2
 
 
 def test_warp_mma_gemm_fragment_mapping():
