@@ -52,14 +52,36 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase with the given parity to complete; false after the time limit.
+// try_wait with a suspend-time hint: the thread sleeps in the barrier unit
+// until the phase completes or the hint (ns) elapses, instead of spinning.
+constexpr uint32_t kSuspendHintNs = 20000;
+
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for the phase with the given parity to complete; false after the time
+// limit.  The clock is read once every 64 attempts: reading %globaltimer in a
+// tight loop from many warps saturates the SM's special-function pipe.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = global_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_ns() - t0 > kWaitLimitNs) return false;
+  unsigned long long t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      const unsigned long long now = global_ns();
+      if (it == 0) t0 = now;
+      else if (now - t0 > kWaitLimitNs) return false;
+    }
   }
-  return true;
 }
 
 __device__ __forceinline__ void prefetch_l2(const void* gmem, uint32_t bytes) {

@@ -114,11 +114,19 @@ __host__ __device__ inline uint32_t am_stride(int KB) {
 __host__ __device__ inline uint32_t gu_stage_bytes(int H) { return 8 * copy_stride(H) + 8 * am_stride(H / 64); }
 __host__ __device__ inline uint32_t dn_block_bytes(int I) { return 4 * copy_stride(I) + 4 * am_stride(I / 64); }
 
+// Bytes of h staged in shared memory for phase 2 (all of it when it fits the
+// budget, else 0: the fragments then come from L2 into registers).
+constexpr uint32_t kHStageMax = 32 * 1024;
+__host__ __device__ inline uint32_t h_stage_bytes(int M, int k, int I) {
+  const uint32_t b = static_cast<uint32_t>(M * k) * static_cast<uint32_t>(I) * 2;
+  return b <= kHStageMax ? b : 0;
+}
+
 struct Smem {
-  uint32_t lut, red, ids, w, uidx, touched, slotmap, xa, bars, ring, total;
+  uint32_t lut, red, ids, w, uidx, touched, slotmap, xa, hs, bars, ring, total;
 };
 
-__host__ __device__ inline Smem make_smem(int M, int k, int E, int r, int stages, uint32_t slot) {
+__host__ __device__ inline Smem make_smem(int M, int k, int E, int r, int I, int stages, uint32_t slot) {
   Smem L;
   const int S = M * k;
   uint32_t o = 0;
@@ -138,8 +146,10 @@ __host__ __device__ inline Smem make_smem(int M, int k, int E, int r, int stages
   o = al(o + S * kMaxM * 4, 16);
   L.xa = o;
   if (r > 0) o = al(o + S * r * 4, 16);
+  L.hs = o;
+  o = al(o + h_stage_bytes(M, k, I), 128);
   L.bars = o;
-  o = al(o + 2 * stages * 8, 16);
+  o = al(o + (2 * stages + 1) * 8, 16);
   L.ring = al(o, 128);
   L.total = L.ring + static_cast<uint32_t>(stages) * slot;
   return L;
@@ -193,17 +203,21 @@ __device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long
 // (*abort set), every later wait returns false at once.
 __device__ __forceinline__ bool ring_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* err, int code) {
   if (mbar_try_wait(bar, parity)) return true;
-  if (*abort) return false;
-  const unsigned long long t0 = global_ns();
-  while (!mbar_try_wait(bar, parity)) {
+  unsigned long long t0 = 0;
+  for (uint32_t it = 0;; ++it) {
     if (*abort) return false;
-    if (global_ns() - t0 > kWaitLimitNs) {
-      *abort = 1;
-      record_error(err, code);
-      return false;
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    if ((it & 63u) == 0) {  // the clock only now and then: see mbar_wait
+      const unsigned long long now = global_ns();
+      if (it == 0) {
+        t0 = now;
+      } else if (now - t0 > kWaitLimitNs) {
+        *abort = 1;
+        record_error(err, code);
+        return false;
+      }
     }
   }
-  return true;
 }
 
 // The four MMAs of one 64-element k-block of a 16-row tile, into d (zeroed by
@@ -212,10 +226,15 @@ __device__ __forceinline__ bool ring_wait(uint64_t* bar, uint32_t parity, volati
 // bf16 of its token column g (xw, 8 words).  MMA j takes bytes 2j, 2j+1: their
 // bf16 pairs are the A fragment (row g / g+8, k slots 2t..2t+1 and 2t+8..2t+9)
 // and x words 2j, 2j+1 the B fragment, so both operands see the same physical
-// k for every slot.
-__device__ __forceinline__ void block_mma(const uint32_t* __restrict__ lut_lane, uint2 w0, uint2 w1,
+// k for every slot.  The table entry of byte b for lane l is at byte
+// b * 128 + 4 l of the table, i.e. at (b << 7) | lane4: one shift and one
+// three-input logic op per lookup.
+__device__ __forceinline__ void block_mma(const unsigned char* __restrict__ lut, uint32_t lane4, uint2 w0, uint2 w1,
                                           const uint32_t* xw, float d[4]) {
-  auto pair = [&](uint32_t word, int byte) { return lut_lane[((word >> (8 * byte)) & 0xffu) << 5]; };
+  auto pair = [&](uint32_t word, int byte) {
+    const uint32_t sh = byte == 0 ? (word << 7) : (word >> (8 * byte - 7));
+    return *reinterpret_cast<const uint32_t*>(lut + ((sh & 0x7f80u) | lane4));
+  };
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const uint32_t wa = (j < 2) ? w0.x : w0.y, wb = (j < 2) ? w1.x : w1.y;
@@ -307,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
   const uint32_t cs_dn = copy_stride(I), as_dn = am_stride(KBI) / 4, am_dn = 4 * cs_dn;
   const uint32_t exp_dn = dn_block_bytes(I);
   const uint32_t slot = al(max(gu_stage_bytes(H), static_cast<uint32_t>(DPE) * exp_dn), 128);
-  const Smem L = make_smem(p.M, p.k, p.E, p.r, RS, slot);
+  const Smem L = make_smem(p.M, p.k, p.E, p.r, p.I, RS, slot);
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L.lut);
   float4* red = reinterpret_cast<float4*>(smem + L.red);
   int* ids_s = reinterpret_cast<int*>(smem + L.ids);
@@ -318,6 +337,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
   float* xa = reinterpret_cast<float*>(smem + L.xa);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);  // stage landed
   uint64_t* empty = full + RS;                                   // stage consumed (16 arrivals)
+  uint64_t* hbar = empty + RS;                                   // h staged for phase 2
+  const uint32_t HSB = h_stage_bytes(p.M, p.k, I);
   unsigned char* ring = smem + L.ring;
   __shared__ int nU_s;
   __shared__ volatile int abort_s;
@@ -333,6 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kMath);
     }
+    mbar_init(hbar, 1);
     fence_mbar_init();
   }
   prologue(p, lut, ids_s, w_s, uidx, touched, slotmap, &nU_s);
@@ -387,20 +409,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
       ++issued;
     }
     // Every copy in flight lands before the CTA may exit.
-    for (int j = max(0, issued - RS); j < issued; ++j) {
-      if (mbar_try_wait(&full[j % RS], (j / RS) & 1)) continue;
-      const unsigned long long t0 = global_ns();
-      while (!mbar_try_wait(&full[j % RS], (j / RS) & 1))
-        if (global_ns() - t0 > kWaitLimitNs) {
-          record_error(p.err, kErrWaitDrain);
-          break;
-        }
-    }
+    for (int j = max(0, issued - RS); j < issued; ++j)
+      if (!mbar_wait(&full[j % RS], (j / RS) & 1)) record_error(p.err, kErrWaitDrain);
     return;
   }
 
   // ---------------------------------------------------------------- math warps
-  const uint32_t* lut_lane = lut + lane;
+  const unsigned char* lut_b = smem + L.lut;
+  const uint32_t lane4 = static_cast<uint32_t>(lane) * 4;
   const int S = p.M * p.k;
   if (p.r > 0 && n_gu > 0) {
     // LoRA first factor of the slots whose expert has items in this CTA:
@@ -475,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
               const uint2 w1 = lds64(st + (4 + cg) * cs_gu + off);
               const float a0 = am[cg * as_gu + r * KB + kb], a1 = am[(4 + cg) * as_gu + r * KB + kb];
               float d[4] = {0.f, 0.f, 0.f, 0.f};
-              block_mma(lut_lane, w0, w1, xr[q][hh], d);
+              block_mma(lut_b, lane4, w0, w1, xr[q][hh], d);
               c[T][0] = fmaf(a0, d[0], c[T][0]);
               c[T][1] = fmaf(a0, d[1], c[T][1]);
               c[T][2] = fmaf(a1, d[2], c[T][2]);
@@ -542,25 +558,48 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
       st_release_gpu(p.flags + bid, tag);
     }
     __syncwarp();
-    const unsigned long long t0 = global_ns();
-    while (true) {
+    unsigned long long t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+      // Independent relaxed loads of every slot (one round trip per poll),
+      // then one fence once all are seen.
       bool ready = true;
-      for (int c = lane; c < G; c += 32) ready = ready && ld_acquire_gpu(p.flags + c) == tag;
+      for (int base = 0; base < G; base += 256) {
+        unsigned long long v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int c = base + lane + 32 * i;
+          v[i] = c < G ? ld_relaxed_gpu(p.flags + c) : tag;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ready = ready && v[i] == tag;
+      }
       if (__all_sync(0xffffffffu, ready)) {
+        __threadfence();
         // Every CTA has read the old epoch: advance it for the next launch.
         if (bid == 0 && lane == 0) st_release_gpu(p.flags + kMaxGrid, tag);
         break;
       }
       if (abort_s) break;
-      if (global_ns() - t0 > kWaitLimitNs) {
-        if (lane == 0) {
-          abort_s = 1;
-          record_error(p.err, kErrGridBarrier);
+      if ((it & 63u) == 0) {  // the clock only now and then: see mbar_wait
+        const unsigned long long now = global_ns();
+        if (it == 0) {
+          t0 = now;
+        } else if (now - t0 > kWaitLimitNs) {
+          if (lane == 0) {
+            abort_s = 1;
+            record_error(p.err, kErrGridBarrier);
+          }
+          break;
         }
-        break;
       }
     }
-    __threadfence();
+    if (HSB > 0 && n_dn > 0 && lane == 0) {
+      // Small h: all of it into shared memory with one bulk copy (the async
+      // proxy reads what the generic proxy of the other CTAs wrote).
+      asm volatile("fence.proxy.async;" ::: "memory");
+      mbar_arrive_expect_tx(hbar, HSB);
+      bulk_g2s(smem + L.hs, p.h, HSB, hbar);
+    }
   }
   named_bar(kBarMath, kMath * 32);
 
@@ -570,6 +609,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
     uint4 hA[PPW][2], hB[PPW][2];
     // h fragments of stage jd for this warp's pairs (zeros where token g does
     // not route to the pair's expert), loaded one stage ahead of their use.
+    if (HSB > 0 && n_dn > 0) ring_wait(hbar, 0, &abort_s, p.err, kErrWaitFull);
+    const uint16_t* hsrc = HSB > 0 ? reinterpret_cast<const uint16_t*>(smem + L.hs) : p.h;
     auto load_h = [&](int jd, uint4 (&hb)[PPW][2]) {
 #pragma unroll
       for (int q = 0; q < PPW; ++q) hb[q][0] = hb[q][1] = make_uint4(0, 0, 0, 0);
@@ -582,9 +623,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
           const int u = u0 + pi / KBI, kb = pi % KBI;
           const int sg = g < p.M ? slotmap[u * kMaxM + g] : -1;
           if (sg >= 0) {
-            const uint4* src = reinterpret_cast<const uint4*>(p.h + static_cast<int64_t>(sg) * I + kb * 64 + 16 * t);
-            hb[q][0] = __ldcg(src);
-            hb[q][1] = __ldcg(src + 1);
+            const uint4* src = reinterpret_cast<const uint4*>(hsrc + static_cast<int64_t>(sg) * I + kb * 64 + 16 * t);
+            if (HSB > 0) {
+              hb[q][0] = src[0];
+              hb[q][1] = src[1];
+            } else {
+              hb[q][0] = __ldcg(src);
+              hb[q][1] = __ldcg(src + 1);
+            }
           }
         }
       }
@@ -608,7 +654,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
           const uint2 w1 = lds64(base + off + I);  // two rows further
           const float a0 = am[cg * as_dn + r * KBI + kb], a1 = am[cg * as_dn + (r + 2) * KBI + kb];
           float d[4] = {0.f, 0.f, 0.f, 0.f};
-          block_mma(lut_lane, w0, w1, reinterpret_cast<const uint32_t*>(hb[q]), d);
+          block_mma(lut_b, lane4, w0, w1, reinterpret_cast<const uint32_t*>(hb[q]), d);
           const int s0 = (2 * t < p.M) ? slotmap[u * kMaxM + 2 * t] : -1;
           const int s1 = (2 * t + 1 < p.M) ? slotmap[u * kMaxM + 2 * t + 1] : -1;
           const float wc0 = s0 >= 0 ? w_s[s0] : 0.f, wc1 = s1 >= 0 ? w_s[s1] : 0.f;
@@ -695,13 +741,13 @@ std::string make_plan(int M, int k, int E, int H, int I, int r, size_t smem_limi
   pl->dpe = std::max(1, std::min({static_cast<int>(gu / dn), kMaxDPE, kMaxKBI / KBI}));
   pl->ppw = (pl->dpe * KBI + kMath - 1) / kMath;
   pl->slot = al(std::max(gu, static_cast<uint32_t>(pl->dpe) * dn), 128);
-  const size_t fixed = make_smem(M, k, E, r, 0, pl->slot).ring + 2 * kMaxStages * 8;
+  const size_t fixed = make_smem(M, k, E, r, I, 0, pl->slot).ring + 2 * kMaxStages * 8;
   if (fixed >= smem_limit) return "the decode kernel's shared-memory plan does not fit this shape";
   int st = static_cast<int>((smem_limit - fixed) / pl->slot);
   st = std::min(st, kMaxStages) & ~1;
   if (st < 2) return "the decode kernel's shared-memory ring does not fit this shape";
   pl->stages = st;
-  pl->smem = make_smem(M, k, E, r, st, pl->slot).total;
+  pl->smem = make_smem(M, k, E, r, I, st, pl->slot).total;
   const int items_upper = std::min(M * k, E) * (I / 16);
   pl->grid = std::max(1, std::min({sm_count, kMaxGrid, std::max(items_upper, H / 16)}));
   return "";
