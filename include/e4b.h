@@ -248,8 +248,8 @@ E4B_API e4b_status e4b_moe_expert_forward_path(const uint16_t* x, int64_t M, con
  *
  * Computes exactly what e4b_moe_expert_forward() computes for 1 <= M <= 8
  * tokens, with the decode kernels, but takes no workspace: its scratch (the
- * SwiGLU activations of the routed slots, M*k*I bf16 values, plus the routing
- * result the first decode kernel hands to the second) lives in one statically
+ * SwiGLU activations of the routed slots, M*k*I bf16 values, plus the decode
+ * kernels' error word) lives in one statically
  * sized device array of the library, 528 KiB, which every GPU that loads the
  * library holds until the process exits.  Requires M*k*I <= 262144 (for example M = 8, k = 8,
  * I <= 4096); larger shapes return E4B_ERR_UNSUPPORTED with a message.  The

@@ -9,23 +9,23 @@
 //   kernel A  routing (every CTA, redundantly: M <= 8 tokens), then the gate
 //             and up rows of every touched expert in items of 8 gate + 8 up
 //             rows over all of K = H -> SiLU(gate) * up (+ LoRA delta) -> h
-//             (bf16, [M*k, I], slot order).  It also prefetches the touched
-//             experts' down rows into L2, so that HBM keeps streaming while the
-//             second kernel starts.
-//   kernel B  the routing kernel A published, then for every block
-//             of 16 output rows of H the down rows of every touched expert, with
-//             the routing weights folded into the per-block scale, so the
-//             combine happens inside the CTA in a fixed order (deterministic).
+//             (bf16, [M*k, I], slot order).
+//   kernel B  the same routing, then for every block of 16 output rows of H
+//             the down rows of every touched expert, with the routing weights
+//             folded in, so the combine happens inside the CTA in a fixed
+//             order (deterministic).  Its weight stream starts before kernel A
+//             has finished; only the h rows wait for it.
 //
-// Only experts that some token selected are read.  Both kernels are split-K
-// GEMVs on warp tensor cores: each CTA owns a contiguous run of items, its 16
-// warps split K in spans of two absmax blocks (128 k), and each lane loads its
-// 16-byte slice of a span of the packed rows straight from HBM into the
-// registers of an mma.sync m16n8k16 fragment (weight rows = MMA rows, the <= 8
-// tokens = the 8 MMA columns), several items ahead.  Nibbles become bf16
-// through a per-lane replicated byte -> bf16x2 codebook table in shared memory
-// (lane l reads only bank l), scaled by the block's bf16 absmax before the
-// MMA.  One block barrier per batch gathers the 16 warps' partials.
+// Only experts that some token selected are read.  Each CTA streams its share
+// of the packed rows and their absmax through a ring of shared-memory stages
+// filled by bulk asynchronous copies (one producer warp, one copy per row,
+// mbarrier transaction counts), so HBM keeps streaming while the math warps
+// decode.  The 16 math warps split K in spans of two absmax blocks (128 k) and
+// run mma.sync m16n8k16 with the weight rows as MMA rows and the <= 8 tokens as
+// the 8 MMA columns.  Nibbles become bf16 through a per-lane replicated byte ->
+// bf16x2 codebook table in shared memory (lane l reads only bank l), scaled by
+// the block's bf16 absmax before the MMA.  Rows are staged 16 bytes apart from
+// the next row's bank so that the fragment loads are conflict-free.
 #include <algorithm>
 
 #include "async.cuh"
@@ -37,13 +37,15 @@ namespace e4b {
 namespace {
 
 constexpr int kMaxM = 8;
-constexpr int kWarps = 16;
+constexpr int kMath = 16;                  // math warps: split K in spans of 128
+constexpr int kProducer = kMath;           // warp issuing the bulk copies
+constexpr int kEpilogue = kMath + 1;       // warp summing the math warps' partials
+constexpr int kWarps = kMath + 2;
 constexpr int kThreads = kWarps * 32;
-constexpr int kSlots = 4;                  // (item, span) load slots per warp per batch in kernel A
-constexpr int kPairSlots = 2;              // (expert, span) load slots per warp per batch in kernel B
-constexpr int kMaxKBW = 2;                 // spans (2 k-blocks) per warp per item: H <= 128 * 16 * 2 = 4096
-constexpr unsigned long long kPrefetchLimit = 64ull << 20;
-constexpr uint32_t kPrefetchChunk = 32 * 1024;
+constexpr int kMaxKBW = 2;                 // spans per math warp per row: K <= 128 * 16 * 2 = 4096
+constexpr int kMaxStages = 12;
+constexpr int kMinStages = 2;
+constexpr uint32_t kRedBytes = kMath * 32 * 16;  // one float4 per lane of every math warp
 
 struct DecodeParams {
   const uint16_t* x;
@@ -60,32 +62,56 @@ struct DecodeParams {
   float lora_scale;
   uint16_t* h;    // [S, I] bf16 (slot order)
   uint16_t* out;  // [M, H] bf16
-  // Routing result of the gate_up kernel for the down kernel: [nU, pad x3],
-  // touched [S], slotmap [S * kMaxM], weights [S] (as float bits).
-  int* meta;
-};
-
-struct Layout {
-  uint32_t lut, xs, red, ids, w, uidx, touched, slotmap, xa, total;
+  int* err;       // error word (a bounded wait gave up)
+  int stages_a, stages_b;
 };
 
 __host__ __device__ inline uint32_t al(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
-// Spans of 128 k (2 absmax blocks, 64 packed bytes of a row) per warp per item.
-__host__ __device__ inline int kbw_of(int H) { return ((H / 64 + 1) / 2 + kWarps - 1) / kWarps; }
+// One ring stage: 16 rows of K/2 packed bytes, their absmax, optionally the h
+// rows of the stage's tokens (kernel B) and the math warps' partials (kernel A).
+struct RingGeom {
+  uint32_t ps;       // shared-memory stride of a packed row, bytes (K/2 + 16)
+  uint32_t sa;       // stride of an absmax row, floats
+  bool am_rows;      // absmax copied row by row (strided) or as two 8-row chunks
+  uint32_t am_off;   // offsets inside the stage, bytes
+  uint32_t h_off;
+  uint32_t hs;       // stride of an h row, bytes (2 K + 16)
+  uint32_t red_off;
+  uint32_t bytes;    // stage size (128-byte multiple)
+};
 
-// Shared-memory carve of kernel A (gate_up) or B (down).
-__host__ __device__ inline Layout make_layout(bool is_a, int M, int k, int E, int H, int r) {
+// K = row length of the streamed matrix; h_rows = token rows of h per stage.
+__host__ __device__ inline RingGeom ring_geom(int K, int h_rows, bool with_red) {
+  RingGeom g;
+  const int KB = K / 64;
+  g.ps = static_cast<uint32_t>(K / 2 + 16);
+  // A row's absmax can be copied on its own only if it is a 16-byte multiple;
+  // then the stride is KB rounded up to 4 (mod 8), which puts the 8 rows of a
+  // fragment on 8 distinct groups of 4 banks.  Otherwise the rows of a chunk
+  // stay contiguous (KB is not a multiple of 4: at most 2-way conflicts).
+  g.am_rows = (KB % 4) == 0;
+  g.sa = static_cast<uint32_t>(g.am_rows ? (KB % 8 == 4 ? KB : KB + 4) : KB);
+  g.am_off = 16 * g.ps;
+  g.h_off = g.am_off + al(16 * g.sa * 4, 16);
+  g.hs = static_cast<uint32_t>(2 * K + 16);
+  g.red_off = g.h_off + static_cast<uint32_t>(h_rows) * g.hs;
+  g.bytes = al(g.red_off + (with_red ? kRedBytes : 0u), 128);
+  return g;
+}
+
+struct Layout {
+  uint32_t lut, ids, w, uidx, touched, slotmap, xa, bars, red, ring, total;
+};
+
+// Shared-memory carve of kernel A (gate_up) or B (down) with `stages` ring stages.
+__host__ __device__ inline Layout make_layout(bool is_a, int M, int k, int E, int r, const RingGeom& g,
+                                              int stages) {
   Layout L;
   uint32_t o = 0;
-  L.lut = o;
-  o = al(o + 256 * 32 * 4, 16);
-  L.xs = o;
-  if (is_a) o = al(o + M * (2 * H + 16), 16);
-  L.red = o;
-  const int items = is_a ? kSlots : 1;  // partial sums of up to kSlots items per batch (A), 1 row block (B)
-  o = al(o + items * kWarps * 32 * 16, 16);
   const int S = M * k;
+  L.lut = o;
+  o += 256 * 32 * 4;
   L.ids = o;
   o = al(o + S * 4, 16);
   L.w = o;
@@ -98,8 +124,20 @@ __host__ __device__ inline Layout make_layout(bool is_a, int M, int k, int E, in
   o = al(o + S * kMaxM * 4, 16);
   L.xa = o;
   if (is_a && r > 0) o = al(o + S * r * 4, 16);
-  L.total = o;
+  L.bars = o;
+  o = al(o + (is_a ? 3 * stages : 2 * stages + 4) * 8, 16);
+  L.red = o;
+  if (!is_a) o += 2 * kRedBytes;  // partials of two row blocks
+  L.ring = al(o, 128);
+  L.total = L.ring + static_cast<uint32_t>(stages) * g.bytes;
   return L;
+}
+
+// Deepest ring that fits `limit` bytes, or 0.
+inline int pick_stages(bool is_a, int M, int k, int E, int r, const RingGeom& g, size_t limit) {
+  for (int s = kMaxStages; s >= kMinStages; --s)
+    if (make_layout(is_a, M, k, E, r, g, s).total <= limit) return s;
+  return 0;
 }
 
 __device__ __forceinline__ void mma_16816(float c[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
@@ -111,8 +149,13 @@ __device__ __forceinline__ void mma_16816(float c[4], uint32_t a0, uint32_t a1, 
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint4 ld_stream_u4(const uint8_t* p) {
-  return __ldcs(reinterpret_cast<const uint4*>(p));
+// Bulk asynchronous copy global -> this CTA's shared memory, completing on `bar`
+// (both addresses 16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(smem_dst)),
+               "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
 }
 
 // One span (128 k = 2 absmax blocks) of a 16-row tile, accumulated into c.
@@ -153,40 +196,28 @@ __device__ __forceinline__ void route_one(const DecodeParams& p, int t, int* ids
 }
 
 // Byte -> bf16x2 codebook pairs, replicated per lane (entry b of lane l at
-// b * 32 + l), written by the warps [w0, kWarps) of the block.
-__device__ __forceinline__ void fill_lut_warps(uint32_t* lut, int w0) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (warp < w0) return;
+// b * 32 + l), entries first, first + step, ... written by the calling warp.
+__device__ __forceinline__ void fill_lut(uint32_t* lut, int first, int step) {
+  const int lane = threadIdx.x & 31;
   const float cbl = kNf4CodebookDev[lane & 15];
-  for (int b = warp - w0; b < 256; b += kWarps - w0) {
+  for (int b = first; b < 256; b += step) {
     const float hi = __shfl_sync(0xffffffffu, cbl, b >> 4);
     const float lo = __shfl_sync(0xffffffffu, cbl, b & 15);
     lut[b * 32 + lane] = pack_bf16x2(hi, lo);
   }
 }
 
-// Prologue shared by both kernels: warps < M route one token each while the
-// other warps build the codebook table (and, in kernel A, stage x).  Then the
-// touched experts (ascending id) and slotmap[u][t] = slot of token t in expert
-// touched[u] (or -1) are built.
-__device__ void decode_prologue(const DecodeParams& p, uint32_t* lut, uint16_t* xs, int xstride, int* ids_s,
-                                float* w_s, int* uidx, int* touched, int* slotmap, int* nU_out) {
+// Prologue of both kernels: warps < M route one token each while the other
+// warps build the codebook table.  Then the touched experts (ascending id) and
+// slotmap[u][t] = slot of token t in expert touched[u] (or -1) are built.  Ends
+// with a block barrier (which also publishes the mbarrier initialisation).
+__device__ void route_prologue(const DecodeParams& p, uint32_t* lut, int* ids_s, float* w_s, int* uidx,
+                               int* touched, int* slotmap, int* nU_out) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int S = p.M * p.k;
   for (int e = tid; e < p.E; e += blockDim.x) uidx[e] = -1;
-  if (warp < p.M) {
-    route_one(p, warp, ids_s, w_s);
-  } else {
-    fill_lut_warps(lut, p.M);
-    if (xs) {
-      const int nthr = (kWarps - p.M) * 32, me = tid - p.M * 32;
-      for (int i = me; i < p.M * (p.H / 8); i += nthr) {
-        const int t = i / (p.H / 8), c = i % (p.H / 8);
-        reinterpret_cast<uint4*>(xs + t * xstride)[c] =
-            reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(t) * p.H)[c];
-      }
-    }
-  }
+  if (warp < p.M) route_one(p, warp, ids_s, w_s);
+  else fill_lut(lut, warp - p.M, kWarps - p.M);
   __syncthreads();
   for (int s = tid; s < S; s += blockDim.x) uidx[ids_s[s]] = 0;  // flag
   __syncthreads();
@@ -213,183 +244,140 @@ __device__ void decode_prologue(const DecodeParams& p, uint32_t* lut, uint16_t* 
   __syncthreads();
 }
 
-// L2 prefetch of the gate and up rows (and their absmax) of items [a, b),
-// one thread per item.
-__device__ __forceinline__ void prefetch_items(const DecodeParams& p, const int* touched, int a, int b) {
-  const int i = a + static_cast<int>(threadIdx.x);
-  if (i >= b) return;
-  const int ipe = p.I / 8;
-  const int u = i / ipe, rb = i % ipe;
-  const int64_t grow = static_cast<int64_t>(touched[u]) * 2 * p.I + rb * 8;
-  const int64_t row_bytes = p.H / 2, kb = p.H / 64;
-  prefetch_l2(p.gu_packed + grow * row_bytes, static_cast<uint32_t>(8 * row_bytes));
-  prefetch_l2(p.gu_packed + (grow + p.I) * row_bytes, static_cast<uint32_t>(8 * row_bytes));
-  prefetch_l2(p.gu_absmax + grow * kb, static_cast<uint32_t>(8 * kb * 4));
-  prefetch_l2(p.gu_absmax + (grow + p.I) * kb, static_cast<uint32_t>(8 * kb * 4));
+// Issues the copies of one stage: 16 packed rows (rows [0, 8) from `row_a`,
+// [8, 16) from `row_b`) and their absmax, announcing `extra` more bytes that
+// the caller copies itself.  Called by the whole producer warp.
+__device__ __forceinline__ void issue_rows(const RingGeom& G, unsigned char* st, uint64_t* full,
+                                           const uint8_t* packed, const float* absmax, int K, int64_t row_a,
+                                           int64_t row_b, uint32_t extra) {
+  const int lane = threadIdx.x & 31;
+  const int KB = K / 64;
+  const uint32_t rowb = static_cast<uint32_t>(K / 2);
+  if (lane == 0) mbar_arrive_expect_tx(full, 16 * rowb + 16 * KB * 4 + extra);
+  __syncwarp();
+  if (lane < 16) {
+    const int64_t row = (lane < 8 ? row_a : row_b) + (lane & 7);
+    bulk_g2s(st + lane * G.ps, packed + row * rowb, rowb, full);
+  } else if (G.am_rows) {
+    const int i = lane - 16;
+    const int64_t row = (i < 8 ? row_a : row_b) + (i & 7);
+    bulk_g2s(st + G.am_off + i * G.sa * 4, absmax + row * KB, KB * 4, full);
+  } else if (lane < 18) {
+    const int i = lane - 16;
+    bulk_g2s(st + G.am_off + i * 8 * G.sa * 4, absmax + (i == 0 ? row_a : row_b) * KB, 8 * KB * 4, full);
+  }
+}
+
+// Drains the producer's copies in flight (bounded) before the CTA exits.
+__device__ __forceinline__ void drain_ring(uint64_t* full, int issued, int stages) {
+  for (int j = max(0, issued - stages); j < issued; ++j) mbar_wait(&full[j % stages], (j / stages) & 1);
 }
 
 // ---------------------------------------------------------------------------
-// Kernel A: gate_up + SwiGLU (+ LoRA delta) -> h.  KBW = k-blocks per warp per item.
+// Kernel A: gate_up + SwiGLU (+ LoRA delta) -> h.  KBW = spans per math warp.
 template <int KBW>
 __global__ void __launch_bounds__(kThreads, 1) decode_gate_up_kernel(DecodeParams p) {
-  constexpr int IB = kSlots / KBW;  // items per batch
-  extern __shared__ __align__(16) unsigned char smem[];
-  const Layout L = make_layout(true, p.M, p.k, p.E, p.H, p.r);
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int RS = p.stages_a;
+  const RingGeom G = ring_geom(p.H, 0, true);
+  const Layout L = make_layout(true, p.M, p.k, p.E, p.r, G, RS);
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L.lut);
-  uint16_t* xs = reinterpret_cast<uint16_t*>(smem + L.xs);
-  float4* red = reinterpret_cast<float4*>(smem + L.red);
   int* ids_s = reinterpret_cast<int*>(smem + L.ids);
   float* w_s = reinterpret_cast<float*>(smem + L.w);
   int* uidx = reinterpret_cast<int*>(smem + L.uidx);
   int* touched = reinterpret_cast<int*>(smem + L.touched);
   int* slotmap = reinterpret_cast<int*>(smem + L.slotmap);
   float* xa = reinterpret_cast<float*>(smem + L.xa);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);  // stage landed
+  uint64_t* done = full + RS;                                    // math warps' partials written
+  uint64_t* empty = done + RS;                                   // stage free again
+  unsigned char* ring = smem + L.ring;
   __shared__ int nU_s;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int H = p.H, I = p.I, KB = H / 64;
-  const int xstride = H + 8;  // bf16 elements (2H + 16 bytes: conflict-free 16-byte reads)
-
-  pdl_wait();               // the inputs of this call are final
-  pdl_launch_dependents();  // the down kernel may launch and run its prologue
-  decode_prologue(p, lut, xs, xstride, ids_s, w_s, uidx, touched, slotmap, &nU_s);
-  const int nU = nU_s;
-  if (blockIdx.x == 0) {
-    // Every CTA routed identically; one publishes the result for the down kernel.
-    const int S = p.M * p.k;
-    int* m_touched = p.meta + 4;
-    int* m_slotmap = m_touched + S;
-    float* m_w = reinterpret_cast<float*>(m_slotmap + S * kMaxM);
-    if (tid == 0) p.meta[0] = nU;
-    for (int i = tid; i < nU; i += blockDim.x) m_touched[i] = touched[i];
-    for (int i = tid; i < nU * kMaxM; i += blockDim.x) m_slotmap[i] = slotmap[i];
-    for (int i = tid; i < S; i += blockDim.x) m_w[i] = w_s[i];
+  const int H = p.H, I = p.I, KB = H / 64, NSP = (KB + 1) / 2;
+  const int nact = min(kMath, NSP);  // math warps with a span
+  if (tid == 0) {
+    for (int s = 0; s < RS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&done[s], nact);
+      mbar_init(&empty[s], 1);
+    }
+    fence_mbar_init();
   }
+  pdl_wait();               // the inputs of this call are final
+  pdl_launch_dependents();  // the down kernel may launch and start its weight stream
+  route_prologue(p, lut, ids_s, w_s, uidx, touched, slotmap, &nU_s);
+  const int nU = nU_s;
   const int ipe = I / 8;  // items per expert
   const int nitems = nU * ipe;
   // A contiguous run of items per CTA: consecutive items are consecutive rows.
   const int q = nitems / gridDim.x, rem = nitems % gridDim.x;
   const int i0 = blockIdx.x * q + min(static_cast<int>(blockIdx.x), rem);
-  const int i1 = i0 + q + (static_cast<int>(blockIdx.x) < rem ? 1 : 0);
-
-  if (warp == kWarps - 1) {
-    // Prefetch this CTA's share of the touched experts' down rows into L2.
-    const uint64_t per_expert = static_cast<uint64_t>(H) * I / 2;
-    const uint64_t per_expert_am = static_cast<uint64_t>(H) * (I / 64) * 4;
-    const uint64_t chunks_pk = (per_expert + kPrefetchChunk - 1) / kPrefetchChunk;
-    const uint64_t chunks_am = (per_expert_am + kPrefetchChunk - 1) / kPrefetchChunk;
-    const uint64_t per_u = chunks_pk + chunks_am;
-    uint64_t total = static_cast<uint64_t>(nU) * per_u;
-    const uint64_t cap = kPrefetchLimit / kPrefetchChunk;
-    if (total > cap) total = cap;
-    for (uint64_t c = static_cast<uint64_t>(blockIdx.x) * 32 + lane; c < total; c += static_cast<uint64_t>(gridDim.x) * 32) {
-      const uint64_t u = c / per_u, qq = c % per_u;
-      const int64_t e = touched[u];
-      if (qq < chunks_pk) {
-        const uint64_t off = qq * kPrefetchChunk;
-        const uint64_t n = min(static_cast<uint64_t>(kPrefetchChunk), per_expert - off);
-        prefetch_l2(p.dn_packed + e * per_expert + off, static_cast<uint32_t>(n));
-      } else {
-        const uint64_t off = (qq - chunks_pk) * kPrefetchChunk;
-        const uint64_t n = min(static_cast<uint64_t>(kPrefetchChunk), per_expert_am - off);
-        prefetch_l2(reinterpret_cast<const unsigned char*>(p.dn_absmax) + e * per_expert_am + off,
-                    static_cast<uint32_t>(n));
-      }
-    }
-  }
+  const int n = q + (static_cast<int>(blockIdx.x) < rem ? 1 : 0);
 
   const int g = lane >> 2, t = lane & 3;
   const int S = p.M * p.k;
   if (p.r > 0) {
     // LoRA first factor per slot: xa[s, rho] = x[token(s)] . lora_A[e(s), rho]
-    for (int qd = warp; qd < S * p.r; qd += kWarps) {
-      const int s = qd / p.r, rho = qd % p.r;
-      const int tok = s / p.k;
-      const uint16_t* la = p.lora_A + (static_cast<int64_t>(ids_s[s]) * p.r + rho) * H;
-      float acc = 0.f;
-      for (int kk = lane * 8; kk < H; kk += 256) {
-        const uint4 xv = *reinterpret_cast<const uint4*>(xs + tok * xstride + kk);
-        const uint4 av = *reinterpret_cast<const uint4*>(la + kk);
-        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, aw[4] = {av.x, av.y, av.z, av.w};
+    if (warp < kMath) {
+      for (int qd = warp; qd < S * p.r; qd += kMath) {
+        const int s = qd / p.r, rho = qd % p.r;
+        const uint16_t* xr = p.x + static_cast<int64_t>(s / p.k) * H;
+        const uint16_t* la = p.lora_A + (static_cast<int64_t>(ids_s[s]) * p.r + rho) * H;
+        float acc = 0.f;
+        for (int kk = lane * 8; kk < H; kk += 256) {
+          const uint4 xv = *reinterpret_cast<const uint4*>(xr + kk);
+          const uint4 av = *reinterpret_cast<const uint4*>(la + kk);
+          const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, aw[4] = {av.x, av.y, av.z, av.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          acc = fmaf(__uint_as_float(xw[i] << 16), __uint_as_float(aw[i] << 16), acc);
-          acc = fmaf(__uint_as_float(xw[i] & 0xffff0000u), __uint_as_float(aw[i] & 0xffff0000u), acc);
+          for (int i = 0; i < 4; ++i) {
+            acc = fmaf(__uint_as_float(xw[i] << 16), __uint_as_float(aw[i] << 16), acc);
+            acc = fmaf(__uint_as_float(xw[i] & 0xffff0000u), __uint_as_float(aw[i] & 0xffff0000u), acc);
+          }
         }
-      }
 #pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) xa[qd] = acc;
+        for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) xa[qd] = acc;
+      }
     }
     __syncthreads();
   }
-  const uint32_t* lut_lane = lut + lane;
-  const int64_t row_bytes = H / 2;
-  // Batches after the first read L2: keep the bulk prefetch two batches ahead.
-  if (tid < 2 * IB) prefetch_items(p, touched, min(i0 + IB, i1), min(i0 + 3 * IB, i1));
-  for (int b0 = i0; b0 < i1; b0 += IB) {
-    const int nb = min(IB, i1 - b0);
-    if (b0 > i0 && tid < IB) prefetch_items(p, touched, min(b0 + 2 * IB, i1), min(b0 + 3 * IB, i1));
-    // Issue every load of the batch first (HBM latency is hidden by the batch).
-    // 16-byte loads: a lane's 32 k of a span lie in k-block 2 * span + t / 2.
-    uint4 pk[IB][KBW][2];
-    float am[IB][KBW][2];
-#pragma unroll
-    for (int ii = 0; ii < IB; ++ii) {
-      const int it = b0 + (ii < nb ? ii : 0);
-      const int u = it / ipe, rb = it % ipe;
-      const int64_t grow = static_cast<int64_t>(touched[u]) * 2 * I + rb * 8 + g;  // gate row of lane's MMA row g
-      const uint8_t* gp = p.gu_packed + grow * row_bytes + 16 * t;
-      const uint8_t* up = gp + static_cast<int64_t>(I) * row_bytes;
-      const float* ga = p.gu_absmax + grow * KB;
-      const float* ua = ga + static_cast<int64_t>(I) * KB;
-#pragma unroll
-      for (int q2 = 0; q2 < KBW; ++q2) {
-        const int sp = warp + kWarps * q2;
-        const int kb = 2 * sp + (t >> 1);
-        if (ii < nb && kb < KB) {
-          pk[ii][q2][0] = ld_stream_u4(gp + sp * 64);
-          pk[ii][q2][1] = ld_stream_u4(up + sp * 64);
-          am[ii][q2][0] = __ldg(ga + kb);
-          am[ii][q2][1] = __ldg(ua + kb);
-        } else {
-          pk[ii][q2][0] = pk[ii][q2][1] = make_uint4(0, 0, 0, 0);
-          am[ii][q2][0] = am[ii][q2][1] = 0.f;
-        }
+
+  if (warp == kProducer) {
+    int issued = 0;
+    for (int j = 0; j < n; ++j) {
+      const int s = j % RS;
+      if (j >= RS && !mbar_wait(&empty[s], ((j / RS) - 1) & 1)) {
+        record_error(p.err, kErrWaitEmpty);
+        break;
       }
+      const int it = i0 + j, u = it / ipe, rb = it % ipe;
+      const int64_t grow = static_cast<int64_t>(touched[u]) * 2 * I + rb * 8;
+      issue_rows(G, ring + s * G.bytes, &full[s], p.gu_packed, p.gu_absmax, H, grow, grow + I, 0);
+      ++issued;
     }
-#pragma unroll
-    for (int ii = 0; ii < IB; ++ii) {
-      if (ii >= nb) break;
-      const int u = (b0 + ii) / ipe;
-      const bool has_g = (g < p.M) && slotmap[u * kMaxM + g] >= 0;  // token g routes to this expert
-      const uint16_t* xrow = xs + g * xstride + 32 * t;
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int q2 = 0; q2 < KBW; ++q2) {
-        const int sp = warp + kWarps * q2;
-        if (2 * sp >= KB) break;
-        uint4 xv[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
-        if (has_g && 2 * sp + (t >> 1) < KB) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) xv[i] = *reinterpret_cast<const uint4*>(xrow + sp * 128 + 8 * i);
-        }
-        span_mma(lut_lane, pk[ii][q2][0], pk[ii][q2][1], am[ii][q2][0], am[ii][q2][1], xv, acc);
+    drain_ring(full, issued, RS);
+  } else if (warp == kEpilogue) {
+    for (int j = 0; j < n; ++j) {
+      const int s = j % RS;
+      if (!mbar_wait(&done[s], (j / RS) & 1)) {
+        record_error(p.err, kErrWaitFull);
+        break;
       }
-      red[(ii * kWarps + warp) * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    }
-    __syncthreads();
-    if (warp < nb) {
-      // Warp `warp` finishes item b0 + warp: sum the 16 partials in warp order.
+      // Sum the partials in warp order, then hand the stage back.
+      const float4* red = reinterpret_cast<const float4*>(ring + s * G.bytes + G.red_off);
       float4 c = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int w = 0; w < kWarps; ++w) {
-        const float4 v = red[(warp * kWarps + w) * 32 + lane];
+      for (int w = 0; w < nact; ++w) {
+        const float4 v = red[w * 32 + lane];
         c.x += v.x;
         c.y += v.y;
         c.z += v.z;
         c.w += v.w;
       }
-      const int it = b0 + warp;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      const int it = i0 + j;
       const int u = it / ipe, rb = it % ipe;
       const int e = touched[u];
       const int col = rb * 8 + g;  // h column == gate row index
@@ -416,107 +404,154 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gate_up_kernel(DecodeParam
         p.h[static_cast<int64_t>(slot) * I + col] = float_to_bf16_bits(silu_f32(gv) * uv);
       }
     }
-    __syncthreads();
+  } else if (warp < nact) {
+    // The warp's spans are the same in every item: its slice of x (token g of
+    // the MMA column) stays in registers.  Columns of tokens that do not route
+    // to an item's expert compute values that the epilogue never stores.
+    uint4 xv[KBW][4];
+#pragma unroll
+    for (int q2 = 0; q2 < KBW; ++q2) {
+      const int sp = warp + kMath * q2;
+      const bool live = g < p.M && sp < NSP && 2 * sp + (t >> 1) < KB;
+      const uint16_t* xr = p.x + static_cast<int64_t>(g) * H + sp * 128 + 32 * t;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        xv[q2][i] = live ? *reinterpret_cast<const uint4*>(xr + 8 * i) : make_uint4(0, 0, 0, 0);
+    }
+    const uint32_t* lut_lane = lut + lane;
+    for (int j = 0; j < n; ++j) {
+      const int s = j % RS;
+      if (!mbar_wait(&full[s], (j / RS) & 1)) {
+        record_error(p.err, kErrWaitFull);
+        break;
+      }
+      const unsigned char* st = ring + s * G.bytes;
+      const float* am = reinterpret_cast<const float*>(st + G.am_off);
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int q2 = 0; q2 < KBW; ++q2) {
+        const int sp = warp + kMath * q2;
+        if (sp >= NSP) break;
+        const int kb = 2 * sp + (t >> 1);  // this lane's 32 k of the span lie in k-block kb
+        uint4 r0 = make_uint4(0, 0, 0, 0), r1 = make_uint4(0, 0, 0, 0);
+        float a0 = 0.f, a1 = 0.f;
+        if (kb < KB) {
+          r0 = *reinterpret_cast<const uint4*>(st + g * G.ps + sp * 64 + 16 * t);
+          r1 = *reinterpret_cast<const uint4*>(st + (g + 8) * G.ps + sp * 64 + 16 * t);
+          a0 = am[g * G.sa + kb];
+          a1 = am[(g + 8) * G.sa + kb];
+        }
+        span_mma(lut_lane, r0, r1, a0, a1, xv[q2], acc);
+      }
+      float4* red = reinterpret_cast<float4*>(ring + s * G.bytes + G.red_off);
+      red[warp * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&done[s]);
+    }
   }
 }
 
 // ---------------------------------------------------------------------------
 // Kernel B: down rows of every touched expert, weighted combine -> out.
+// Stage j of a CTA = (row block blockIdx.x + (j / nU) * gridDim.x, expert
+// touched[j % nU]): 16 down rows over all of K = I plus the h rows of the
+// tokens routed to that expert.  The math warps take the (stage, span) pairs
+// of a row block in turn; each keeps one running sum per row block.
 __global__ void __launch_bounds__(kThreads, 1) decode_down_kernel(DecodeParams p) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  const Layout L = make_layout(false, p.M, p.k, p.E, p.H, 0);
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int RS = p.stages_b;
+  const RingGeom G = ring_geom(p.I, p.M, false);
+  const Layout L = make_layout(false, p.M, p.k, p.E, 0, G, RS);
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L.lut);
-  float4* red = reinterpret_cast<float4*>(smem + L.red);
+  int* ids_s = reinterpret_cast<int*>(smem + L.ids);
   float* w_s = reinterpret_cast<float*>(smem + L.w);
+  int* uidx = reinterpret_cast<int*>(smem + L.uidx);
   int* touched = reinterpret_cast<int*>(smem + L.touched);
   int* slotmap = reinterpret_cast<int*>(smem + L.slotmap);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);  // stage landed
+  uint64_t* empty = full + RS;                                   // every span of the stage consumed
+  uint64_t* rdone = empty + RS;                                  // [2] partials of a row block written
+  uint64_t* rfree = rdone + 2;                                   // [2] partials of a row block summed
+  float4* red = reinterpret_cast<float4*>(smem + L.red);         // [2][kMath][32]
+  unsigned char* ring = smem + L.ring;
   __shared__ int nU_s;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int H = p.H, I = p.I, KB = I / 64;
-  // The down kernel starts once the gate_up kernel's CTAs leave the SMs; it
-  // builds its codebook table, waits for that kernel's results (h and the
-  // routing it published) and reads the routing instead of recomputing it.
-  fill_lut_warps(lut, 0);
-  pdl_wait();  // h and the routing written by the gate_up kernel are visible from here on
-  {
-    const int S = p.M * p.k;
-    const int* m_touched = p.meta + 4;
-    const int* m_slotmap = m_touched + S;
-    const float* m_w = reinterpret_cast<const float*>(m_slotmap + S * kMaxM);
-    const int n = __ldcg(p.meta);
-    if (tid == 0) nU_s = n;
-    for (int i = tid; i < n; i += blockDim.x) touched[i] = __ldcg(m_touched + i);
-    for (int i = tid; i < n * kMaxM; i += blockDim.x) slotmap[i] = __ldcg(m_slotmap + i);
-    for (int i = tid; i < S; i += blockDim.x) w_s[i] = __ldcg(m_w + i);
-  }
-  __syncthreads();
-  const int nU = nU_s;
-  const int NSP = (KB + 1) / 2;  // spans of 128 k (two absmax blocks) in a down row
-  const int npairs = nU * NSP;   // (expert, span) pairs of one row block
-  const int g = lane >> 2, t = lane & 3;
-  const uint32_t* lut_lane = lut + lane;
-  const int64_t row_bytes = I / 2;
-  for (int rb = blockIdx.x; rb < H / 16; rb += gridDim.x) {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int pb = warp; pb < npairs; pb += kWarps * kPairSlots) {
-      uint4 pk[kPairSlots][2];
-      float am[kPairSlots][2];
-      uint4 hx[kPairSlots][4];
-      float wc[kPairSlots][2];
-#pragma unroll
-      for (int sl = 0; sl < kPairSlots; ++sl) {
-        const int pi = pb + kWarps * sl;
-        pk[sl][0] = pk[sl][1] = make_uint4(0, 0, 0, 0);
-        am[sl][0] = am[sl][1] = 0.f;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) hx[sl][i] = make_uint4(0, 0, 0, 0);
-        wc[sl][0] = wc[sl][1] = 0.f;
-        if (pi < npairs) {
-          const int u = pi / NSP, sp = pi % NSP;
-          const int kb = 2 * sp + (t >> 1);  // this lane's 32 k of the span lie in k-block kb
-          const int64_t row = static_cast<int64_t>(touched[u]) * H + rb * 16 + g;
-          if (kb < KB) {
-            const uint8_t* rp = p.dn_packed + row * row_bytes + sp * 64 + 16 * t;
-            pk[sl][0] = ld_stream_u4(rp);
-            pk[sl][1] = ld_stream_u4(rp + 8 * row_bytes);
-            am[sl][0] = __ldg(p.dn_absmax + row * KB + kb);
-            am[sl][1] = __ldg(p.dn_absmax + (row + 8) * KB + kb);
-            const int slot_g = (g < p.M) ? slotmap[u * kMaxM + g] : -1;
-            if (slot_g >= 0) {
-              const uint16_t* hr = p.h + static_cast<int64_t>(slot_g) * I + sp * 128 + 32 * t;
-#pragma unroll
-              for (int i = 0; i < 4; ++i) hx[sl][i] = *reinterpret_cast<const uint4*>(hr + 8 * i);
-            }
-          }
-          const int s0 = (2 * t < p.M) ? slotmap[u * kMaxM + 2 * t] : -1;
-          const int s1 = (2 * t + 1 < p.M) ? slotmap[u * kMaxM + 2 * t + 1] : -1;
-          wc[sl][0] = s0 >= 0 ? w_s[s0] : 0.f;
-          wc[sl][1] = s1 >= 0 ? w_s[s1] : 0.f;
-        }
-      }
-#pragma unroll
-      for (int sl = 0; sl < kPairSlots; ++sl) {
-        if (pb + kWarps * sl >= npairs) break;
-        float tmp[4] = {0.f, 0.f, 0.f, 0.f};
-        span_mma(lut_lane, pk[sl][0], pk[sl][1], am[sl][0], am[sl][1], hx[sl], tmp);
-        acc[0] = fmaf(tmp[0], wc[sl][0], acc[0]);
-        acc[1] = fmaf(tmp[1], wc[sl][1], acc[1]);
-        acc[2] = fmaf(tmp[2], wc[sl][0], acc[2]);
-        acc[3] = fmaf(tmp[3], wc[sl][1], acc[3]);
-      }
+  const int H = p.H, I = p.I, KB = I / 64, NSP = (KB + 1) / 2;
+  if (tid == 0) {
+    for (int s = 0; s < RS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], NSP);
     }
-    red[warp * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    __syncthreads();
-    if (warp == 0) {
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&rdone[b], kMath);
+      mbar_init(&rfree[b], 1);
+    }
+    fence_mbar_init();
+  }
+  // Routing again (it reads only this call's logits, final before the gate_up
+  // kernel let this one launch); h is waited for by the producer alone.
+  route_prologue(p, lut, ids_s, w_s, uidx, touched, slotmap, &nU_s);
+  const int nU = nU_s;
+  const int nrb_all = H / 16;
+  const int nrb = (nrb_all - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                  static_cast<int>(gridDim.x);  // row blocks of this CTA
+  const int T = nrb * nU;                       // stages of this CTA
+  const int g = lane >> 2, t = lane & 3;
+
+  if (warp == kProducer) {
+    const uint32_t hrow = static_cast<uint32_t>(I) * 2;
+    auto issue_w = [&](int j) {
+      const int s = j % RS, u = j % nU;
+      const int rb = static_cast<int>(blockIdx.x) + (j / nU) * static_cast<int>(gridDim.x);
+      const bool has = lane < p.M && slotmap[u * kMaxM + lane] >= 0;
+      const int nh = __popc(__ballot_sync(0xffffffffu, has));
+      const int64_t row0 = static_cast<int64_t>(touched[u]) * H + rb * 16;
+      issue_rows(G, ring + s * G.bytes, &full[s], p.dn_packed, p.dn_absmax, I, row0, row0 + 8, nh * hrow);
+    };
+    auto issue_h = [&](int j) {
+      const int s = j % RS, u = j % nU;
+      if (lane < p.M) {
+        const int slot = slotmap[u * kMaxM + lane];
+        if (slot >= 0)
+          bulk_g2s(ring + s * G.bytes + G.h_off + lane * G.hs, p.h + static_cast<int64_t>(slot) * I, hrow, &full[s]);
+      }
+    };
+    // The first stages' weights stream while the gate_up kernel finishes.
+    const int pre = min(RS, T);
+    for (int j = 0; j < pre; ++j) issue_w(j);
+    pdl_wait();  // h written by the gate_up kernel is visible from here on
+    for (int j = 0; j < pre; ++j) issue_h(j);
+    int issued = pre;
+    for (int j = pre; j < T; ++j) {
+      const int s = j % RS;
+      if (!mbar_wait(&empty[s], ((j / RS) - 1) & 1)) {
+        record_error(p.err, kErrWaitEmpty);
+        break;
+      }
+      issue_w(j);
+      issue_h(j);
+      ++issued;
+    }
+    drain_ring(full, issued, RS);
+  } else if (warp == kEpilogue) {
+    for (int rbi = 0; rbi < nrb; ++rbi) {
+      const int par = rbi & 1;
+      if (!mbar_wait(&rdone[par], (rbi >> 1) & 1)) {
+        record_error(p.err, kErrWaitFull);
+        break;
+      }
       float4 c = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int w = 0; w < kWarps; ++w) {
-        const float4 v = red[w * 32 + lane];
+      for (int w = 0; w < kMath; ++w) {
+        const float4 v = red[(par * kMath + w) * 32 + lane];
         c.x += v.x;
         c.y += v.y;
         c.z += v.z;
         c.w += v.w;
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&rfree[par]);
+      const int rb = static_cast<int>(blockIdx.x) + rbi * static_cast<int>(gridDim.x);
       const int row0 = rb * 16 + g;
       const float v[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
@@ -526,21 +561,71 @@ __global__ void __launch_bounds__(kThreads, 1) decode_down_kernel(DecodeParams p
         if (tok < p.M) p.out[static_cast<int64_t>(tok) * H + row] = float_to_bf16_bits(v[q2]);
       }
     }
-    __syncthreads();
+  } else {
+    const uint32_t* lut_lane = lut + lane;
+    const int npr = nU * NSP;  // (expert, span) pairs of one row block
+    bool ok = true;
+    for (int rbi = 0; rbi < nrb && ok; ++rbi) {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int qp = warp; qp < npr; qp += kMath) {
+        const int u = qp / NSP, sp = qp % NSP;
+        const int j = rbi * nU + u, s = j % RS;
+        if (!mbar_wait(&full[s], (j / RS) & 1)) {
+          record_error(p.err, kErrWaitFull);
+          ok = false;
+          break;
+        }
+        const unsigned char* st = ring + s * G.bytes;
+        const float* am = reinterpret_cast<const float*>(st + G.am_off);
+        const int kb = 2 * sp + (t >> 1);  // this lane's 32 k of the span lie in k-block kb
+        uint4 r0 = make_uint4(0, 0, 0, 0), r1 = make_uint4(0, 0, 0, 0);
+        float a0 = 0.f, a1 = 0.f;
+        uint4 hx[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0),
+                       make_uint4(0, 0, 0, 0)};
+        if (kb < KB) {
+          r0 = *reinterpret_cast<const uint4*>(st + g * G.ps + sp * 64 + 16 * t);
+          r1 = *reinterpret_cast<const uint4*>(st + (g + 8) * G.ps + sp * 64 + 16 * t);
+          a0 = am[g * G.sa + kb];
+          a1 = am[(g + 8) * G.sa + kb];
+          const int slot_g = (g < p.M) ? slotmap[u * kMaxM + g] : -1;  // h row of token g landed
+          if (slot_g >= 0) {
+            const unsigned char* hr = st + G.h_off + g * G.hs + sp * 256 + 64 * t;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) hx[i] = *reinterpret_cast<const uint4*>(hr + 16 * i);
+          }
+        }
+        const int s0 = (2 * t < p.M) ? slotmap[u * kMaxM + 2 * t] : -1;
+        const int s1 = (2 * t + 1 < p.M) ? slotmap[u * kMaxM + 2 * t + 1] : -1;
+        const float wc0 = s0 >= 0 ? w_s[s0] : 0.f, wc1 = s1 >= 0 ? w_s[s1] : 0.f;
+        float tmp[4] = {0.f, 0.f, 0.f, 0.f};
+        span_mma(lut_lane, r0, r1, a0, a1, hx, tmp);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        acc[0] = fmaf(tmp[0], wc0, acc[0]);
+        acc[1] = fmaf(tmp[1], wc1, acc[1]);
+        acc[2] = fmaf(tmp[2], wc0, acc[2]);
+        acc[3] = fmaf(tmp[3], wc1, acc[3]);
+      }
+      if (!ok) break;
+      // Publish this warp's sum for the row block (every warp, work or not).
+      const int par = rbi & 1;
+      if (rbi >= 2 && !mbar_wait(&rfree[par], ((rbi >> 1) - 1) & 1)) {
+        record_error(p.err, kErrWaitEmpty);
+        break;
+      }
+      red[(par * kMath + warp) * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&rdone[par]);
+    }
   }
 }
 
 template <int KBW>
-cudaError_t raise_smem_limits(size_t smem_a, size_t smem_b) {
+cudaError_t launch_pair(const DecodeParams& p, int sm_count, size_t smem_a, size_t smem_b, cudaStream_t stream) {
   cudaError_t err = ensure_smem_limit(reinterpret_cast<const void*>(decode_gate_up_kernel<KBW>), smem_a);
   if (err != cudaSuccess) return err;
-  return ensure_smem_limit(reinterpret_cast<const void*>(decode_down_kernel), smem_b);
-}
-
-template <int KBW>
-cudaError_t launch_pair(const DecodeParams& p, int sm_count, size_t smem_a, size_t smem_b, cudaStream_t stream) {
-  cudaError_t aerr = raise_smem_limits<KBW>(smem_a, smem_b);
-  if (aerr != cudaSuccess) return aerr;
+  err = ensure_smem_limit(reinterpret_cast<const void*>(decode_down_kernel), smem_b);
+  if (err != cudaSuccess) return err;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -554,7 +639,7 @@ cudaError_t launch_pair(const DecodeParams& p, int sm_count, size_t smem_a, size
   cfg.dynamicSmemBytes = smem_a;
   {
     LaunchScope ls("decode.gate_up", stream);
-    cudaError_t err = cudaLaunchKernelEx(&cfg, decode_gate_up_kernel<KBW>, p);
+    err = cudaLaunchKernelEx(&cfg, decode_gate_up_kernel<KBW>, p);
     if (err != cudaSuccess) return err;
   }
   cfg.gridDim = dim3(std::max(1, std::min(sm_count, p.H / 16)));
@@ -567,7 +652,8 @@ struct DecodeWs {
   size_t h, meta, total;
 };
 
-// Workspace: h [M*k, I] bf16, then the published routing (4 + S * (2 + kMaxM) ints).
+// Workspace: h [M*k, I] bf16, then 4 + S * (2 + kMaxM) ints whose first is the
+// error word.
 DecodeWs decode_ws(int64_t M, int k, int64_t I) {
   DecodeWs w;
   const int64_t S = M * k;
@@ -577,17 +663,31 @@ DecodeWs decode_ws(int64_t M, int k, int64_t I) {
   return w;
 }
 
+struct Stages {
+  int a, b;
+  size_t smem_a, smem_b;
+};
+
+Stages plan_stages(int M, int k, int E, int H, int I, int r, size_t limit) {
+  Stages st{};
+  const RingGeom ga = ring_geom(H, 0, true), gb = ring_geom(I, M, false);
+  st.a = pick_stages(true, M, k, E, r, ga, limit);
+  st.b = pick_stages(false, M, k, E, 0, gb, limit);
+  if (st.a) st.smem_a = make_layout(true, M, k, E, r, ga, st.a).total;
+  if (st.b) st.smem_b = make_layout(false, M, k, E, 0, gb, st.b).total;
+  return st;
+}
+
 }  // namespace
 
 bool decode_supported(int64_t M, int64_t E, int k, int64_t H, int64_t I) {
-  if (M < 1 || M > kMaxM || k > 32 || E > 512 || H > 128 * kWarps * kMaxKBW) return false;
-  (void)I;
+  if (M < 1 || M > kMaxM || k > 32 || E > 512 || H > 128 * kMath * kMaxKBW) return false;
   DeviceInfo di;
   if (device_info(&di) != cudaSuccess) return false;
-  const Layout a = make_layout(true, static_cast<int>(M), k, static_cast<int>(E), static_cast<int>(H), 16);
-  const Layout b = make_layout(false, static_cast<int>(M), k, static_cast<int>(E), static_cast<int>(H), 0);
   const size_t lim = di.smem_optin - 1024;  // leave room for the kernels' static shared memory
-  return a.total <= lim && b.total <= lim;
+  const Stages st = plan_stages(static_cast<int>(M), k, static_cast<int>(E), static_cast<int>(H),
+                                static_cast<int>(I), 16, lim);
+  return st.a >= kMinStages && st.b >= kMinStages;
 }
 
 size_t decode_workspace_bytes(int64_t M, int64_t E, int k, int64_t H, int64_t I, int r) {
@@ -623,14 +723,15 @@ cudaError_t launch_decode_forward(const DecodeArgs& a, cudaStream_t stream) {
   p.r = r;
   p.lora_scale = r ? w->lora_alpha / static_cast<float>(r) : 0.f;
   p.h = reinterpret_cast<uint16_t*>(static_cast<char*>(a.workspace) + ws.h);
-  p.meta = reinterpret_cast<int*>(static_cast<char*>(a.workspace) + ws.meta);
+  p.err = reinterpret_cast<int*>(static_cast<char*>(a.workspace) + ws.meta);
   p.out = a.out;
-  const size_t smem_a = make_layout(true, p.M, p.k, p.E, p.H, r).total;
-  const size_t smem_b = make_layout(false, p.M, p.k, p.E, p.H, 0).total;
-  switch (kbw_of(p.H)) {
-    case 1: return launch_pair<1>(p, di.sm_count, smem_a, smem_b, stream);
-    default: return launch_pair<2>(p, di.sm_count, smem_a, smem_b, stream);
-  }
+  const Stages st = plan_stages(p.M, p.k, p.E, p.H, p.I, r, di.smem_optin - 1024);
+  if (st.a < kMinStages || st.b < kMinStages) return cudaErrorInvalidConfiguration;
+  p.stages_a = st.a;
+  p.stages_b = st.b;
+  const int nsp = (p.H / 64 + 1) / 2;
+  if (nsp <= kMath) return launch_pair<1>(p, di.sm_count, st.smem_a, st.smem_b, stream);
+  return launch_pair<2>(p, di.sm_count, st.smem_a, st.smem_b, stream);
 }
 
 }  // namespace e4b

@@ -4,8 +4,8 @@
 // carve every byte of device memory out of a fixed pool planned at start-up,
 // and runtimes that forbid any allocator call (cudaMalloc included) once the
 // decode loop is running.  For them this file keeps the decode path's scratch
-// -- the SwiGLU activations h of the routed slots and the routing result the
-// gate_up kernel hands to the down kernel -- in a
+// -- the SwiGLU activations h of the routed slots and the kernels' error word
+// -- in a
 // statically sized device array that exists from the moment the library is
 // loaded on a GPU until the process exits.  The caller still passes x, the
 // router logits, the packed stacks and the output buffer.
