@@ -23,9 +23,10 @@
 // decode.  The 16 math warps split K in spans of two absmax blocks (128 k) and
 // run mma.sync m16n8k16 with the weight rows as MMA rows and the <= 8 tokens as
 // the 8 MMA columns.  Nibbles become bf16 through a per-lane replicated byte ->
-// bf16x2 codebook table in shared memory (lane l reads only bank l), scaled by
-// the block's bf16 absmax before the MMA.  Rows are staged 16 bytes apart from
-// the next row's bank so that the fragment loads are conflict-free.
+// bf16x2 codebook table in shared memory (lane l reads only bank l); every MMA
+// stays inside one absmax block, so the fp32 absmax scales its products.  Rows
+// are staged 16 bytes apart from the next row's bank so that the fragment loads
+// are conflict-free.
 #include <algorithm>
 
 #include "async.cuh"
@@ -159,29 +160,56 @@ __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, u
 }
 
 // One span (128 k = 2 absmax blocks) of a 16-row tile, accumulated into c.
-// Thread (g, t) owns physical k [32t, 32t+32) of the span -- 16 packed bytes of
-// row g (r0) and of row g+8 (r1), all inside k-block t/2 -- and the matching 32
-// bf16 of its token column g (x).  Each byte's codebook pair is scaled by its
-// row's bf16(absmax) before the MMA (the block scale differs between threads of
-// one MMA, so it cannot be applied to the product).  MMA j takes bytes 2j and
-// 2j+1 of each row; K is permuted identically on both operands.
-__device__ __forceinline__ void span_mma(const uint32_t* __restrict__ lut_lane, uint4 r0, uint4 r1, float a0,
-                                         float a1, const uint4 x[4], float c[4]) {
-  const __nv_bfloat162 s0 = __float2bfloat162_rn(a0), s1 = __float2bfloat162_rn(a1);
-  const uint32_t w0[4] = {r0.x, r0.y, r0.z, r0.w}, w1[4] = {r1.x, r1.y, r1.z, r1.w};
-  const uint32_t xw[16] = {x[0].x, x[0].y, x[0].z, x[0].w, x[1].x, x[1].y, x[1].z, x[1].w,
-                           x[2].x, x[2].y, x[2].z, x[2].w, x[3].x, x[3].y, x[3].z, x[3].w};
-  auto pair = [&](uint32_t word, int byte, __nv_bfloat162 sc) {
-    uint32_t v = lut_lane[((word >> (8 * byte)) & 0xffu) << 5];
-    __nv_bfloat162 h2 = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&v), sc);
-    return *reinterpret_cast<uint32_t*>(&h2);
-  };
+// In each k-block h of the span, thread (g, t) owns physical k [16t, 16t+16):
+// 8 packed bytes of row g (w0[2h], w0[2h+1]) and of row g+8 (w1[2h], w1[2h+1])
+// and the matching 16 bf16 of its token column g (x[2h], x[2h+1]).  MMAs 0-3
+// cover the first k-block and 4-7 the second, so every MMA sees one absmax per
+// row: the products of a k-block are scaled in fp32 afterwards (a0 = row g,
+// a1 = row g+8), with no rounding of the scale.  MMA j of a k-block takes bytes
+// 2j and 2j+1 of the thread's 8 bytes; K is permuted identically on both
+// operands.  A k-block past the end of the row must come with zero x and scale.
+__device__ __forceinline__ void span_mma(const uint32_t* __restrict__ lut_lane, const uint32_t w0[4],
+                                         const uint32_t w1[4], const float a0[2], const float a1[2],
+                                         const uint4 x[4], float c[4]) {
+  auto pair = [&](uint32_t word, int byte) { return lut_lane[((word >> (8 * byte)) & 0xffu) << 5]; };
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int b = 2 * (j & 1);
-    const uint32_t wa = w0[j >> 1], wb = w1[j >> 1];
-    mma_16816(c, pair(wa, b, s0), pair(wb, b, s1), pair(wa, b + 1, s0), pair(wb, b + 1, s1), xw[2 * j],
-              xw[2 * j + 1]);
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t xw[8] = {x[2 * h].x,     x[2 * h].y,     x[2 * h].z,     x[2 * h].w,
+                            x[2 * h + 1].x, x[2 * h + 1].y, x[2 * h + 1].z, x[2 * h + 1].w};
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int b = 2 * (j & 1);
+      const uint32_t wa = w0[2 * h + (j >> 1)], wb = w1[2 * h + (j >> 1)];
+      mma_16816(d, pair(wa, b), pair(wb, b), pair(wa, b + 1), pair(wb, b + 1), xw[2 * j], xw[2 * j + 1]);
+    }
+    c[0] = fmaf(a0[h], d[0], c[0]);
+    c[1] = fmaf(a0[h], d[1], c[1]);
+    c[2] = fmaf(a1[h], d[2], c[2]);
+    c[3] = fmaf(a1[h], d[3], c[3]);
+  }
+}
+
+// Loads the span's fragment of rows g and g+8 of a stage (two 8-byte pieces
+// per row, one per k-block) and their absmax; zeros past the row's end.
+__device__ __forceinline__ void load_span(const RingGeom& G, const unsigned char* st, int g, int t, int sp, int KB,
+                                          uint32_t w0[4], uint32_t w1[4], float a0[2], float a1[2]) {
+  const float* am = reinterpret_cast<const float*>(st + G.am_off);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int kb = 2 * sp + h;
+    uint2 v0 = make_uint2(0u, 0u), v1 = make_uint2(0u, 0u);
+    a0[h] = a1[h] = 0.f;
+    if (kb < KB) {
+      v0 = *reinterpret_cast<const uint2*>(st + g * G.ps + sp * 64 + 32 * h + 8 * t);
+      v1 = *reinterpret_cast<const uint2*>(st + (g + 8) * G.ps + sp * 64 + 32 * h + 8 * t);
+      a0[h] = am[g * G.sa + kb];
+      a1[h] = am[(g + 8) * G.sa + kb];
+    }
+    w0[2 * h] = v0.x;
+    w0[2 * h + 1] = v0.y;
+    w1[2 * h] = v1.x;
+    w1[2 * h + 1] = v1.y;
   }
 }
 
@@ -412,11 +440,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gate_up_kernel(DecodeParam
 #pragma unroll
     for (int q2 = 0; q2 < KBW; ++q2) {
       const int sp = warp + kMath * q2;
-      const bool live = g < p.M && sp < NSP && 2 * sp + (t >> 1) < KB;
-      const uint16_t* xr = p.x + static_cast<int64_t>(g) * H + sp * 128 + 32 * t;
+      const uint16_t* xr = p.x + static_cast<int64_t>(g) * H + sp * 128 + 16 * t;
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        xv[q2][i] = live ? *reinterpret_cast<const uint4*>(xr + 8 * i) : make_uint4(0, 0, 0, 0);
+      for (int i = 0; i < 4; ++i) {
+        const bool live = g < p.M && sp < NSP && 2 * sp + (i >> 1) < KB;  // k-block i / 2 of the span
+        xv[q2][i] = live ? *reinterpret_cast<const uint4*>(xr + 64 * (i >> 1) + 8 * (i & 1)) : make_uint4(0, 0, 0, 0);
+      }
     }
     const uint32_t* lut_lane = lut + lane;
     for (int j = 0; j < n; ++j) {
@@ -426,22 +455,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gate_up_kernel(DecodeParam
         break;
       }
       const unsigned char* st = ring + s * G.bytes;
-      const float* am = reinterpret_cast<const float*>(st + G.am_off);
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int q2 = 0; q2 < KBW; ++q2) {
         const int sp = warp + kMath * q2;
         if (sp >= NSP) break;
-        const int kb = 2 * sp + (t >> 1);  // this lane's 32 k of the span lie in k-block kb
-        uint4 r0 = make_uint4(0, 0, 0, 0), r1 = make_uint4(0, 0, 0, 0);
-        float a0 = 0.f, a1 = 0.f;
-        if (kb < KB) {
-          r0 = *reinterpret_cast<const uint4*>(st + g * G.ps + sp * 64 + 16 * t);
-          r1 = *reinterpret_cast<const uint4*>(st + (g + 8) * G.ps + sp * 64 + 16 * t);
-          a0 = am[g * G.sa + kb];
-          a1 = am[(g + 8) * G.sa + kb];
-        }
-        span_mma(lut_lane, r0, r1, a0, a1, xv[q2], acc);
+        uint32_t w0[4], w1[4];
+        float a0[2], a1[2];
+        load_span(G, st, g, t, sp, KB, w0, w1, a0, a1);
+        span_mma(lut_lane, w0, w1, a0, a1, xv[q2], acc);
       }
       float4* red = reinterpret_cast<float4*>(ring + s * G.bytes + G.red_off);
       red[warp * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
@@ -576,29 +598,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_down_kernel(DecodeParams p
           break;
         }
         const unsigned char* st = ring + s * G.bytes;
-        const float* am = reinterpret_cast<const float*>(st + G.am_off);
-        const int kb = 2 * sp + (t >> 1);  // this lane's 32 k of the span lie in k-block kb
-        uint4 r0 = make_uint4(0, 0, 0, 0), r1 = make_uint4(0, 0, 0, 0);
-        float a0 = 0.f, a1 = 0.f;
-        uint4 hx[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0),
-                       make_uint4(0, 0, 0, 0)};
-        if (kb < KB) {
-          r0 = *reinterpret_cast<const uint4*>(st + g * G.ps + sp * 64 + 16 * t);
-          r1 = *reinterpret_cast<const uint4*>(st + (g + 8) * G.ps + sp * 64 + 16 * t);
-          a0 = am[g * G.sa + kb];
-          a1 = am[(g + 8) * G.sa + kb];
-          const int slot_g = (g < p.M) ? slotmap[u * kMaxM + g] : -1;  // h row of token g landed
-          if (slot_g >= 0) {
-            const unsigned char* hr = st + G.h_off + g * G.hs + sp * 256 + 64 * t;
+        uint32_t w0[4], w1[4];
+        float a0[2], a1[2];
+        load_span(G, st, g, t, sp, KB, w0, w1, a0, a1);
+        uint4 hx[4];
+        const int slot_g = (g < p.M) ? slotmap[u * kMaxM + g] : -1;  // h row of token g landed
+        const unsigned char* hr = st + G.h_off + g * G.hs + sp * 256 + 32 * t;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) hx[i] = *reinterpret_cast<const uint4*>(hr + 16 * i);
-          }
+        for (int i = 0; i < 4; ++i) {
+          const bool live = slot_g >= 0 && 2 * sp + (i >> 1) < KB;  // k-block i / 2 of the span
+          hx[i] = live ? *reinterpret_cast<const uint4*>(hr + 128 * (i >> 1) + 16 * (i & 1)) : make_uint4(0, 0, 0, 0);
         }
         const int s0 = (2 * t < p.M) ? slotmap[u * kMaxM + 2 * t] : -1;
         const int s1 = (2 * t + 1 < p.M) ? slotmap[u * kMaxM + 2 * t + 1] : -1;
         const float wc0 = s0 >= 0 ? w_s[s0] : 0.f, wc1 = s1 >= 0 ? w_s[s1] : 0.f;
         float tmp[4] = {0.f, 0.f, 0.f, 0.f};
-        span_mma(lut_lane, r0, r1, a0, a1, hx, tmp);
+        span_mma(lut_lane, w0, w1, a0, a1, hx, tmp);
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
         acc[0] = fmaf(tmp[0], wc0, acc[0]);
