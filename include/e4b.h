@@ -40,6 +40,13 @@
  *     non-decreasing, indices out of range) cannot be checked on the host; the
  *     kernels clamp such values so that no access leaves the buffers, and the
  *     affected outputs are unspecified.
+ *   - Workspaces are 16-byte aligned like every other buffer.  The first 4
+ *     bytes of a workspace of e4b_grouped_nf4_gemm() or e4b_moe_expert_forward()
+ *     are an error word: a kernel whose bounded wait (2 s) gives up writes a
+ *     nonzero E4B_KERNEL_ERR_* code there (the first code wins) and returns,
+ *     and the output of that call is unspecified.  Nothing clears the word, so
+ *     allocate workspaces zeroed (or clear them with
+ *     e4b_workspace_clear_error()) and read it with e4b_workspace_error().
  */
 #ifndef E4B_H_
 #define E4B_H_
@@ -92,6 +99,21 @@ E4B_API const char* e4b_last_error(void);
 /* Name of the kernel path the last successful call on this host thread
  * launched, e.g. "quantize", "route.small", "gemm.tc", "forward.decode". */
 E4B_API const char* e4b_last_path(void);
+
+/* Error word codes (see the conventions above). */
+#define E4B_KERNEL_ERR_NONE 0
+#define E4B_KERNEL_ERR_WAIT_FULL 1  /* a consumer waited in vain for its input tile */
+#define E4B_KERNEL_ERR_WAIT_EMPTY 2 /* a producer waited in vain for a free stage */
+#define E4B_KERNEL_ERR_WAIT_DRAIN 3 /* a CTA gave up waiting for its own copies */
+
+/* Reads the error word of `workspace` into *code.  Synchronises the device
+ * first (a diagnostic call, not for the hot path or a graph capture).  This
+ * call and the next leave e4b_last_path() and e4b_last_launches() as the
+ * previous call set them. */
+E4B_API e4b_status e4b_workspace_error(const void* workspace, int32_t* code);
+
+/* Sets the error word of `workspace` to E4B_KERNEL_ERR_NONE, ordered on `stream`. */
+E4B_API e4b_status e4b_workspace_clear_error(void* workspace, e4b_stream stream);
 
 /* E4B_VERSION of the built library. */
 E4B_API int e4b_version(void);

@@ -2,7 +2,8 @@
 //
 // Every call validates its arguments on the host before launching anything
 // and reports failures through a status code plus a per-thread message; no
-// call allocates, frees or synchronises.  See include/e4b.h for the contract.
+// call allocates or frees, and none synchronises except the diagnostic read of
+// a workspace's error word.  See include/e4b.h for the contract.
 #include <algorithm>
 #include <cstdio>
 #include <cstring>
@@ -11,6 +12,7 @@
 #include <string>
 #include <vector>
 
+#include "async.cuh"
 #include "e4b_internal.h"
 
 namespace e4b {
@@ -92,6 +94,19 @@ e4b_status cuda_fail(cudaError_t err, const char* where) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Size, presence and alignment of a caller's workspace.
+e4b_status check_workspace(const char* what, size_t need, const void* workspace, size_t workspace_bytes) {
+  if (workspace_bytes < need || (need > 0 && !workspace))
+    return fail(E4B_ERR_WORKSPACE, std::string(what) + " workspace needs " + std::to_string(need) + " bytes");
+  if (workspace && !aligned16(workspace))
+    return fail(E4B_ERR_INVALID_ARGUMENT, std::string(what) + " workspace must be 16-byte aligned");
+  return E4B_OK;
+}
+
+static_assert(kErrNone == E4B_KERNEL_ERR_NONE && kErrWaitFull == E4B_KERNEL_ERR_WAIT_FULL &&
+                  kErrWaitEmpty == E4B_KERNEL_ERR_WAIT_EMPTY && kErrWaitDrain == E4B_KERNEL_ERR_WAIT_DRAIN,
+              "device error codes match the header");
 
 e4b_status check_device() {
   DeviceInfo di;
@@ -198,6 +213,27 @@ const char* e4b_last_path(void) { return g_path; }
 int e4b_version(void) { return E4B_VERSION; }
 int e4b_last_launches(void) { return g_launches; }
 
+// The two error-word calls leave the last call's path and launch count alone.
+e4b_status e4b_workspace_error(const void* workspace, int32_t* code) {
+  if (!workspace || !code) return fail(E4B_ERR_INVALID_ARGUMENT, "null workspace or code");
+  if (!aligned16(workspace)) return fail(E4B_ERR_INVALID_ARGUMENT, "workspace must be 16-byte aligned");
+  if (e4b_status s = check_device(); s != E4B_OK) return s;
+  cudaError_t err = cudaDeviceSynchronize();
+  if (err != cudaSuccess) return cuda_fail(err, "synchronise before reading the error word");
+  err = cudaMemcpy(code, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost);
+  if (err != cudaSuccess) return cuda_fail(err, "read of the error word");
+  return E4B_OK;
+}
+
+e4b_status e4b_workspace_clear_error(void* workspace, e4b_stream stream) {
+  if (!workspace) return fail(E4B_ERR_INVALID_ARGUMENT, "null workspace");
+  if (!aligned16(workspace)) return fail(E4B_ERR_INVALID_ARGUMENT, "workspace must be 16-byte aligned");
+  if (e4b_status s = check_device(); s != E4B_OK) return s;
+  cudaError_t err = cudaMemsetAsync(workspace, 0, sizeof(int32_t), reinterpret_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "clear of the error word");
+  return E4B_OK;
+}
+
 e4b_status e4b_timing_enable(int on) {
   g_timing.on = on != 0;
   g_timing.recs.clear();
@@ -276,9 +312,9 @@ e4b_status e4b_moe_route_permute(const float* logits, int64_t M, int64_t E, int 
   if (!expert_offsets) return fail(E4B_ERR_INVALID_ARGUMENT, "null expert_offsets");
   if (M > 0 && (!logits || !topk_ids || !topk_w || !perm || !inv_perm))
     return fail(E4B_ERR_INVALID_ARGUMENT, "null pointer (logits, topk_ids, topk_w, perm or inv_perm)");
-  const size_t need = route_workspace_bytes(M, E, k);
-  if (workspace_bytes < need || (need > 0 && !workspace))
-    return fail(E4B_ERR_WORKSPACE, "route workspace needs " + std::to_string(need) + " bytes");
+  if (e4b_status s = check_workspace("route", route_workspace_bytes(M, E, k), workspace, workspace_bytes);
+      s != E4B_OK)
+    return s;
   if (e4b_status s = check_device(); s != E4B_OK) return s;
   RouteOut o{topk_ids, topk_w, expert_offsets, perm, inv_perm, nullptr};
   cudaError_t err = launch_route(logits, M, static_cast<int>(E), k, renormalize != 0, o, workspace, stream);
@@ -318,9 +354,9 @@ e4b_status e4b_grouped_nf4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda, 
     return fail(E4B_ERR_INVALID_ARGUMENT, "A, packed and out must be 16-byte aligned");
   if (lora_A && (!aligned16(lora_A) || !aligned16(lora_B)))
     return fail(E4B_ERR_INVALID_ARGUMENT, "lora_A and lora_B must be 16-byte aligned");
-  const size_t need = gemm_workspace_bytes(total_rows, K, r);
-  if (workspace_bytes < need || (need > 0 && !workspace))
-    return fail(E4B_ERR_WORKSPACE, "gemm workspace needs " + std::to_string(need) + " bytes");
+  if (e4b_status s = check_workspace("gemm", gemm_workspace_bytes(total_rows, K, r), workspace, workspace_bytes);
+      s != E4B_OK)
+    return s;
   if (e4b_status s = check_device(); s != E4B_OK) return s;
   if (total_rows == 0) {
     set_path("gemm.empty");
@@ -453,9 +489,10 @@ e4b_status e4b_moe_expert_forward_path(const uint16_t* x, int64_t M, const float
   if (M > 0 && (!aligned16(x) || !aligned16(out))) return fail(E4B_ERR_INVALID_ARGUMENT, "x and out must be 16-byte aligned");
   if (path != E4B_PATH_AUTO && path != E4B_PATH_DECODE && path != E4B_PATH_GROUPED)
     return fail(E4B_ERR_INVALID_ARGUMENT, "unknown path");
-  const size_t need = e4b_moe_expert_forward_workspace_size(M, w, k);
-  if (workspace_bytes < need || (need > 0 && !workspace))
-    return fail(E4B_ERR_WORKSPACE, "forward workspace needs " + std::to_string(need) + " bytes");
+  if (e4b_status s = check_workspace("forward", e4b_moe_expert_forward_workspace_size(M, w, k), workspace,
+                                     workspace_bytes);
+      s != E4B_OK)
+    return s;
   if (e4b_status s = check_device(); s != E4B_OK) return s;
   if (M == 0) {
     set_path("forward.empty");

@@ -667,13 +667,13 @@ struct DecodeWs {
   size_t h, meta, total;
 };
 
-// Workspace: h [M*k, I] bf16, then 4 + S * (2 + kMaxM) ints whose first is the
-// error word.
+// Workspace: the error word every workspace begins with (256-byte slot),
+// h [M*k, I] bf16, then 4 + S * (2 + kMaxM) ints (kept for the layout's size).
 DecodeWs decode_ws(int64_t M, int k, int64_t I) {
   DecodeWs w;
   const int64_t S = M * k;
-  w.h = 0;
-  w.meta = align_up(static_cast<size_t>(S * I * 2), 256);
+  w.h = 256;
+  w.meta = w.h + align_up(static_cast<size_t>(S * I * 2), 256);
   w.total = w.meta + align_up(static_cast<size_t>(4 + S * (2 + kMaxM)) * 4, 256);
   return w;
 }
@@ -738,7 +738,7 @@ cudaError_t launch_decode_forward(const DecodeArgs& a, cudaStream_t stream) {
   p.r = r;
   p.lora_scale = r ? w->lora_alpha / static_cast<float>(r) : 0.f;
   p.h = reinterpret_cast<uint16_t*>(static_cast<char*>(a.workspace) + ws.h);
-  p.err = reinterpret_cast<int*>(static_cast<char*>(a.workspace) + ws.meta);
+  p.err = static_cast<int*>(a.workspace);
   p.out = a.out;
   const Stages st = plan_stages(p.M, p.k, p.E, p.H, p.I, r, di.smem_optin - 1024);
   if (st.a < kMinStages || st.b < kMinStages) return cudaErrorInvalidConfiguration;

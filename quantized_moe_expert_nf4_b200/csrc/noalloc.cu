@@ -20,7 +20,7 @@ namespace {
 // h holds M*k*I bf16 values; the limit below allows e.g. M=8, k=8, I=4096.
 constexpr int64_t kNoAllocMaxHElems = 256 * 1024;
 constexpr size_t kNoAllocHBytes = static_cast<size_t>(kNoAllocMaxHElems) * 2;
-constexpr size_t kNoAllocBytes = kNoAllocHBytes + 16 * 1024;  // + the routing the two decode kernels share
+constexpr size_t kNoAllocBytes = kNoAllocHBytes + 16 * 1024;  // + the error word and the routing the kernels share
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 

@@ -30,6 +30,7 @@ E4B_PATH_AUTO, E4B_PATH_DECODE, E4B_PATH_GROUPED = 0, 1, 2
 # Every symbol include/e4b.h declares.
 EXPORTED = (
     "e4b_status_string", "e4b_last_error", "e4b_last_path", "e4b_version", "e4b_last_launches",
+    "e4b_workspace_error", "e4b_workspace_clear_error",
     "e4b_timing_enable", "e4b_timing_kernels", "e4b_timing_get",
     "e4b_nf4_quantize_stack",
     "e4b_moe_route_permute_workspace_size", "e4b_moe_route_permute",
@@ -102,6 +103,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.e4b_moe_expert_forward_decode_noalloc.restype = i32
     lib.e4b_moe_expert_forward_decode_noalloc.argtypes = [vp, i64, vp, i32, i32, ctypes.POINTER(ExpertStackC), vp,
                                                           vp]
+    lib.e4b_workspace_error.restype = i32
+    lib.e4b_workspace_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
+    lib.e4b_workspace_clear_error.restype = i32
+    lib.e4b_workspace_clear_error.argtypes = [vp, vp]
     lib.e4b_moe_expert_forward_path.restype = i32
     lib.e4b_moe_expert_forward_path.argtypes = [vp, i64, vp, i32, i32, ctypes.POINTER(ExpertStackC), vp, vp,
                                                 sz, i32, vp]
@@ -294,5 +299,21 @@ def e4b_moe_expert_forward_decode_noalloc(x: torch.Tensor, router_logits: torch.
 
 
 def workspace(nbytes: int, device="cuda") -> torch.Tensor:
-    """A device byte buffer of at least nbytes (at least 256 B, 256-B aligned by torch)."""
-    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    """A zeroed device byte buffer of at least nbytes (at least 256 B, 256-B aligned
+    by torch); its first 4 bytes are the error word the kernels report through."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+E4B_KERNEL_ERR_NONE, E4B_KERNEL_ERR_WAIT_FULL, E4B_KERNEL_ERR_WAIT_EMPTY, E4B_KERNEL_ERR_WAIT_DRAIN = 0, 1, 2, 3
+
+
+def workspace_error(ws: torch.Tensor) -> int:
+    """The error word of a workspace (0: no kernel gave up a bounded wait).
+    Synchronises the device."""
+    code = ctypes.c_int32(-1)
+    _check(load_library().e4b_workspace_error(_ptr(ws), ctypes.byref(code)), "e4b_workspace_error")
+    return int(code.value)
+
+
+def workspace_clear_error(ws: torch.Tensor, stream=None) -> None:
+    _check(load_library().e4b_workspace_clear_error(_ptr(ws), _stream(stream)), "e4b_workspace_clear_error")

@@ -115,3 +115,32 @@ def test_misaligned_lora_adapter_is_rejected_on_the_host(lib):
     stk = e4b.ExpertStackC(1 << 20, 1 << 20, 1 << 20, 1 << 20, (1 << 20) + 2, 1 << 20, 8, 16.0, 8, 256, 128)
     st = lib.e4b_moe_expert_forward(p, 4, p, 2, 1, ctypes.byref(stk), p, p, 1 << 30, None)
     assert st == 1 and b"lora_A and lora_B" in lib.e4b_last_error()
+
+
+def test_misaligned_workspace_is_rejected_on_the_host(lib):
+    """Workspaces feed bulk and tensor-map copies (16-byte rule): an unaligned
+    one is an argument error for every call that takes one, never a launch."""
+    p = ctypes.c_void_p(1 << 20)
+    bad = ctypes.c_void_p((1 << 20) + 8)
+    rows, N, K = 64, 128, 128
+    need = e4b.e4b_grouped_nf4_gemm_workspace_size(rows, N, K, 0)
+    st = lib.e4b_grouped_nf4_gemm(p, rows, K, None, p, 2, rows, p, p, N, K, None, None, 0, 0.0, 0,
+                                  p, 0, bad, need, None)
+    assert st == 1 and b"gemm workspace must be 16-byte aligned" in lib.e4b_last_error()
+    stk = e4b.ExpertStackC(1 << 20, 1 << 20, 1 << 20, 1 << 20, None, None, 0, 0.0, 8, 256, 128)
+    need = lib.e4b_moe_expert_forward_workspace_size(4, ctypes.byref(stk), 2)
+    st = lib.e4b_moe_expert_forward(p, 4, p, 2, 1, ctypes.byref(stk), p, bad, need, None)
+    assert st == 1 and b"forward workspace must be 16-byte aligned" in lib.e4b_last_error()
+    need = e4b.e4b_moe_route_permute_workspace_size(4096, 64, 8)
+    st = lib.e4b_moe_route_permute(p, 4096, 64, 8, 1, p, p, p, p, p, bad, need, None)
+    assert st == 1 and b"route workspace must be 16-byte aligned" in lib.e4b_last_error()
+
+
+def test_error_word_calls_check_their_arguments_on_the_host(lib):
+    code = ctypes.c_int32(7)
+    assert lib.e4b_workspace_error(None, ctypes.byref(code)) == 1
+    assert lib.e4b_workspace_error(ctypes.c_void_p((1 << 20) + 4), ctypes.byref(code)) == 1
+    assert b"16-byte aligned" in lib.e4b_last_error()
+    assert lib.e4b_workspace_clear_error(None, None) == 1
+    assert code.value == 7   # untouched on a rejected call
+

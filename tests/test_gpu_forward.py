@@ -23,7 +23,9 @@ def _forward(layer, x, logits, path=e4b.E4B_PATH_AUTO):
     ws = e4b.workspace(e4b.e4b_moe_expert_forward_workspace_size(M, layer.stack, cfg.k))
     e4b.e4b_moe_expert_forward(x, logits, cfg.k, True, layer.stack, out, ws, path=path)
     torch.cuda.synchronize()
-    return out, e4b.last_path()
+    p = e4b.last_path()
+    assert e4b.workspace_error(ws) == e4b.E4B_KERNEL_ERR_NONE, "a kernel gave up a bounded wait"
+    return out, p
 
 
 def _oracle_tokens(cfg, x, logits, tokens, check_gpu_layer=None):

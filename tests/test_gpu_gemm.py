@@ -41,6 +41,7 @@ def _run_gpu(c, epi, out_dtype, use_ridx=True, scale=2.0):
         torch.from_numpy(c["absmax"]).cuda(), c["N"], c["K"], out, epi,
         _t_bf16(c["la"]) if c["r"] else None, _t_bf16(c["lb"]) if c["r"] else None, scale, ws)
     torch.cuda.synchronize()
+    assert e4b.workspace_error(ws) == e4b.E4B_KERNEL_ERR_NONE, "a kernel gave up a bounded wait"
     res = out.float().cpu().numpy().astype(np.float64)
     assert np.all(np.isnan(res[c["rows"]])), "guard row written"
     return res[:c["rows"]], e4b.last_path()
