@@ -15,7 +15,8 @@ moe      the grouped NF4 GEMM, the SwiGLU expert MLP with its optional LoRA
          delta, the weighted combine; a brute-force per-token form and a
          permuted grouped form of the same layer
 backward the layer's gradients through the frozen NF4 experts (input,
-         router logits, LoRA A and B) with the routing ids held fixed
+         router logits, LoRA A and B) with the routing ids held fixed, per
+         token and in the grouped form built on the grouped dgrad product
 
 Parity status: every function here is pinned by a ``-m "not gpu"`` test
 against closed forms, brute force, invariants or a textbook routine, except

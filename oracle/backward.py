@@ -140,3 +140,105 @@ def layer_backward(x: np.ndarray, logits: np.ndarray, ids: np.ndarray, stack: Ex
                 dlogits[t] -= coef * p[t]
                 dlogits[t, e] += coef
     return dx, dlogits, dA, dB
+
+
+def grouped_nf4_gemm_dgrad(dY: np.ndarray, row_index, offsets: np.ndarray, packed: np.ndarray,
+                           absmax: np.ndarray, N: int, K: int, lora_A=None, lora_B=None,
+                           lora_scale: float = 0.0) -> np.ndarray:
+    """The input gradient of the grouped NF4 GEMM, in one call over all groups.
+
+    The forward row p is ``y_p = a_p . W_e^T (+ s (a_p . A_e^T) . B_e^T)``; for
+    an upstream gradient ``dY`` the result row p is
+
+        da_p = dY[row_index[p]] . W_e  (+ s (dY[row_index[p]] . B_e) . A_e)
+
+    with W_e the dequantised [N, K] expert of the group e holding p (the
+    frozen base is decoded again from the packed bytes, never kept), so the
+    result has K columns.  ``row_index=None`` means identity.  This is the
+    single grouped dgrad launch the pages put in place of a per-expert decode
+    loop (experts4bit-qlora 0.22.0, "Which training path?").
+    """
+    from . import nf4
+    dY = np.asarray(dY, dtype=np.float64)
+    offsets = np.asarray(offsets, dtype=np.int64)
+    E = offsets.size - 1
+    rows = offsets[-1]
+    idx = np.arange(rows) if row_index is None else np.asarray(row_index, dtype=np.int64)
+    packed = np.asarray(packed, dtype=np.uint8).reshape(E, -1)
+    absmax = np.asarray(absmax, dtype=np.float32).reshape(E, -1)
+    out = np.zeros((rows, K), dtype=np.float64)
+    for e in range(E):
+        lo, hi = offsets[e], offsets[e + 1]
+        if hi == lo:
+            continue
+        W = nf4.dequantize_expert(packed[e], absmax[e], (N, K))
+        G = dY[idx[lo:hi]]
+        d = G @ W
+        if lora_A is not None and lora_B is not None:
+            la = np.asarray(lora_A, dtype=np.float64)[e]
+            lb = np.asarray(lora_B, dtype=np.float64)[e]
+            d = d + lora_scale * ((G @ lb) @ la)
+        out[lo:hi] = d
+    return out
+
+
+def layer_backward_grouped(x: np.ndarray, logits: np.ndarray, ids: np.ndarray, stack: ExpertStack,
+                           dout: np.ndarray, renormalize: bool = True):
+    """``layer_backward`` restated in the permuted, grouped form a GPU runs:
+    gather by the permutation, recompute the gate_up output and z per group,
+    two grouped dgrad products (down, then gate_up with its LoRA term), the
+    SwiGLU derivative in between, and the per-token sum through the inverse
+    permutation.  Returns the same ``(dx, dlogits, dA, dB)``."""
+    from . import moe, routing
+    x = np.asarray(x, dtype=np.float64)
+    dout = np.asarray(dout, dtype=np.float64)
+    ids = np.asarray(ids, dtype=np.int64)
+    M, k = ids.shape
+    I, H = stack.I, stack.H
+    s = stack.lora_scale
+    lora = stack.has_lora()
+    w = route_weights64(logits, ids, renormalize)
+    offsets, perm, inv = routing.permute(ids.astype(np.int32), stack.E)
+    perm = np.asarray(perm, dtype=np.int64)
+    tok = perm // k
+    a = moe.grouped_nf4_gemm(x, tok, offsets, stack.gu_packed, stack.gu_absmax, 2 * I, H,
+                             stack.lora_A if lora else None, stack.lora_B if lora else None, s)
+    g, u = a[:, :I], a[:, I:]
+    h = silu(g) * u
+    z = moe.grouped_nf4_gemm(h, None, offsets, stack.dn_packed, stack.dn_absmax, H, I)
+    wp = w.reshape(-1)[perm]                       # routing weight of each grouped row
+    dz = wp[:, None] * dout[tok]
+    dh = grouped_nf4_gemm_dgrad(dz, None, offsets, stack.dn_packed, stack.dn_absmax, H, I)
+    da = np.concatenate([dh * u * silu_grad(g), dh * silu(g)], axis=1)
+    dxg = grouped_nf4_gemm_dgrad(da, None, offsets, stack.gu_packed, stack.gu_absmax, 2 * I, H,
+                                 stack.lora_A if lora else None, stack.lora_B if lora else None, s)
+    dx = dxg[np.asarray(inv, dtype=np.int64)].reshape(M, k, H).sum(axis=1)
+    dw = np.zeros(M * k, dtype=np.float64)
+    dw[perm] = np.sum(dout[tok] * z, axis=1)
+    dw = dw.reshape(M, k)
+    dA = dB = None
+    if lora:
+        dA = np.zeros_like(stack.lora_A)
+        dB = np.zeros_like(stack.lora_B)
+        off = np.asarray(offsets, dtype=np.int64)
+        for e in range(stack.E):
+            lo, hi = off[e], off[e + 1]
+            if hi == lo:
+                continue
+            xe = x[tok[lo:hi]]
+            dae = da[lo:hi]
+            dB[e] = s * dae.T @ (xe @ stack.lora_A[e].T)
+            dA[e] = s * (dae @ stack.lora_B[e]).T @ xe
+    l = np.asarray(logits, dtype=np.float64)
+    dlogits = np.zeros_like(l)
+    if renormalize:
+        inner = (w * dw).sum(axis=1, keepdims=True)
+        np.put_along_axis(dlogits, ids, w * (dw - inner), axis=1)
+    else:
+        p = np.exp(l - l.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        for j in range(k):
+            coef = dw[:, j] * p[np.arange(M), ids[:, j]]
+            dlogits -= coef[:, None] * p
+            dlogits[np.arange(M), ids[:, j]] += coef
+    return dx, dlogits, dA, dB

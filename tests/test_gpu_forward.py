@@ -16,23 +16,23 @@ from gpu_util import assert_close_layer, bf16_to_f64, require_gpu
 pytestmark = pytest.mark.gpu
 
 
-def _forward(layer, x, logits, path=e4b.E4B_PATH_AUTO):
+def _forward(layer, x, logits, path=e4b.E4B_PATH_AUTO, renormalize=True):
     cfg = layer.cfg
     M = x.shape[0]
     out = torch.full((M, cfg.H), float("nan"), dtype=torch.bfloat16, device="cuda")
     ws = e4b.workspace(e4b.e4b_moe_expert_forward_workspace_size(M, layer.stack, cfg.k))
-    e4b.e4b_moe_expert_forward(x, logits, cfg.k, True, layer.stack, out, ws, path=path)
+    e4b.e4b_moe_expert_forward(x, logits, cfg.k, renormalize, layer.stack, out, ws, path=path)
     torch.cuda.synchronize()
     p = e4b.last_path()
     assert e4b.workspace_error(ws) == e4b.E4B_KERNEL_ERR_NONE, "a kernel gave up a bounded wait"
     return out, p
 
 
-def _oracle_tokens(cfg, x, logits, tokens, check_gpu_layer=None):
+def _oracle_tokens(cfg, x, logits, tokens, check_gpu_layer=None, renormalize=True):
     """Oracle output rows for `tokens`, quantising only the experts they use."""
     lg = logits.cpu().numpy()
     ids = routing.topk(lg[tokens], cfg.k)
-    w = routing.route_weights(lg[tokens], ids)
+    w = routing.route_weights(lg[tokens], ids, renormalize)
     need = sorted(set(ids.reshape(-1).tolist()))
     E, H, I = cfg.E, cfg.H, cfg.I
     gp = np.zeros((E, I * H), np.uint8)
@@ -154,3 +154,36 @@ def test_forward_errors_and_empty():
     x0 = x[:0]
     e4b.e4b_moe_expert_forward(x0, logits[:0], cfg.k, True, layer.stack, out[:0], None)
     assert e4b.last_path() == "forward.empty"
+
+
+@pytest.mark.parametrize("path", [e4b.E4B_PATH_DECODE, e4b.E4B_PATH_GROUPED])
+def test_forward_without_renormalisation(path):
+    """renormalize = 0: each selected expert keeps its weight from the softmax
+    over all E logits (the k weights no longer sum to 1)."""
+    require_gpu()
+    cfg = workloads.small_config("fullsm", E=12, H=192, I=320, k=3)
+    M = 5 if path == e4b.E4B_PATH_DECODE else 40
+    layer = synthetic.make_device_layer(cfg)
+    x, logits = synthetic.inputs(cfg, M)
+    out, p = _forward(layer, x, logits, path, renormalize=False)
+    ref = _oracle_tokens(cfg, x, logits, np.arange(M), renormalize=False)
+    assert_close_layer(bf16_to_f64(out), ref, f"renormalize=0 M={M} {p}")
+    ref_renorm = _oracle_tokens(cfg, x, logits, np.arange(M))
+    from gpu_util import rel_errors
+    assert rel_errors(bf16_to_f64(out), ref_renorm)[0] > 1e-2   # the flag changes the result
+
+
+@pytest.mark.parametrize("E,k,M,path", [(8, 1, 6, e4b.E4B_PATH_DECODE), (8, 1, 700, e4b.E4B_PATH_GROUPED),
+                                        (4, 4, 300, e4b.E4B_PATH_GROUPED), (4, 4, 7, e4b.E4B_PATH_DECODE)])
+def test_forward_degenerate_routing(E, k, M, path):
+    """One expert takes every token (k = 1: one group holds all rows, the
+    others are empty), or every token takes every expert (k = E)."""
+    require_gpu()
+    cfg = workloads.small_config(f"degen{E}_{k}", E=E, H=256, I=192, k=k)
+    layer = synthetic.make_device_layer(cfg)
+    x, logits = synthetic.inputs(cfg, M)
+    if k == 1:
+        logits[:, 5] += 30.0
+    out, p = _forward(layer, x, logits, path)
+    ref = _oracle_tokens(cfg, x, logits, np.arange(M))
+    assert_close_layer(bf16_to_f64(out), ref, f"E={E} k={k} M={M} {p}")

@@ -136,3 +136,78 @@ def test_lora_gradient_closed_forms():
     _, _, dA0, dB0 = backward.layer_backward(x, logits, ids, zero_A, dout)
     assert np.all(dB0 == 0.0)
     assert np.any(dA0 != 0.0)
+
+
+def _gemm_case(E=3, N=64, K=128, counts=(5, 0, 7), r=4, seed=5):
+    rng = np.random.default_rng(seed)
+    W = (rng.standard_normal((E, N, K)) * 0.05).astype(np.float32)
+    packed, absmax = nf4.quantize_stack(W)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+    rows = int(offsets[-1])
+    la = rng.standard_normal((E, r, K)) * 0.1
+    lb = rng.standard_normal((E, N, r)) * 0.1
+    return packed, absmax, offsets, rows, la, lb, rng
+
+
+@pytest.mark.parametrize("lora", [False, True])
+def test_grouped_dgrad_is_the_adjoint_of_the_grouped_gemm(lora):
+    """<dY, gemm(A)> = <dgrad(dY), A> for every A and dY: the dgrad oracle is
+    pinned to the (separately pinned) forward GEMM oracle, so a transposed
+    operand or a missing LoRA term fails here."""
+    E, N, K = 3, 64, 128
+    packed, absmax, offsets, rows, la, lb, rng = _gemm_case(E, N, K)
+    A = rng.standard_normal((rows, K))
+    dY = rng.standard_normal((rows, N))
+    kw = dict(lora_A=la, lora_B=lb, lora_scale=2.5) if lora else {}
+    y = moe.grouped_nf4_gemm(A, None, offsets, packed, absmax, N, K, **kw)
+    d = backward.grouped_nf4_gemm_dgrad(dY, None, offsets, packed, absmax, N, K, **kw)
+    assert d.shape == (rows, K)
+    assert np.sum(dY * y) == pytest.approx(np.sum(d * A), rel=1e-12)
+
+
+def test_grouped_dgrad_brute_force_and_row_index():
+    """Element by element from the codes, the codebook and absmax (no
+    dequantised matrix), and the row index gathers dY rows."""
+    E, N, K = 3, 64, 128
+    packed, absmax, offsets, rows, _, _, rng = _gemm_case(E, N, K)
+    dY = rng.standard_normal((rows + 4, N))
+    idx = rng.permutation(rows + 4)[:rows]
+    d = backward.grouped_nf4_gemm_dgrad(dY, idx, offsets, packed, absmax, N, K)
+    cb = nf4.codebook_f64()
+    for p in (0, 4, rows - 1):
+        e = int(np.searchsorted(offsets, p, side="right") - 1)
+        q = nf4.unpack_codes(packed[e])
+        for kk in (0, 63, 64, K - 1):
+            ref = sum(dY[idx[p], n] * cb[q[n * K + kk]] * float(absmax[e][(n * K + kk) // 64]) for n in range(N))
+            assert d[p, kk] == pytest.approx(ref, rel=1e-12, abs=1e-12)
+    assert np.array_equal(d, backward.grouped_nf4_gemm_dgrad(dY[idx], None, offsets, packed, absmax, N, K))
+
+
+def test_adjoint_check_detects_a_transposed_operand():
+    # Positive control: the same check fails for dY . W^T on a square stack.
+    E, N, K = 2, 64, 64
+    packed, absmax, offsets, rows, _, _, rng = _gemm_case(E, N, K, counts=(4, 6))
+    A = rng.standard_normal((rows, K))
+    dY = rng.standard_normal((rows, N))
+    y = moe.grouped_nf4_gemm(A, None, offsets, packed, absmax, N, K)
+    wrong = np.zeros((rows, K))
+    for e in range(E):
+        W = nf4.dequantize_expert(packed[e], absmax[e], (N, K))
+        wrong[offsets[e]:offsets[e + 1]] = dY[offsets[e]:offsets[e + 1]] @ W.T
+    assert np.sum(dY * y) != pytest.approx(np.sum(wrong * A), rel=1e-6)
+
+
+@pytest.mark.parametrize("renorm", [True, False])
+@pytest.mark.parametrize("lora", [True, False])
+def test_grouped_backward_equals_the_per_token_backward(renorm, lora):
+    """The permuted grouped form (two grouped dgrad products around the SwiGLU
+    derivative, sums through the inverse permutation) gives the gradients of
+    the finite-difference-pinned per-token backward."""
+    stack, x, logits, ids, dout = _case(M=6, lora=lora)
+    a = backward.layer_backward(x, logits, ids, stack, dout, renorm)
+    b = backward.layer_backward_grouped(x, logits, ids, stack, dout, renorm)
+    for u, v in zip(a, b):
+        if u is None:
+            assert v is None
+            continue
+        assert np.allclose(u, v, rtol=0, atol=1e-12 * max(1.0, np.abs(u).max()))
