@@ -38,15 +38,16 @@ namespace e4b {
 namespace {
 
 constexpr int kMaxM = 8;
-constexpr int kMath = 16;                  // math warps: split K in spans of 128
-constexpr int kProducer = kMath;           // warp issuing the bulk copies
-constexpr int kEpilogue = kMath + 1;       // warp summing the math warps' partials
+constexpr int kMath = 16;                  // math warps of the down kernel (and at most of gate_up)
+constexpr int kProducer = kMath;           // down kernel: warp issuing the bulk copies
+constexpr int kEpilogue = kMath + 1;       // down kernel: warp summing the math warps' partials
 constexpr int kWarps = kMath + 2;
 constexpr int kThreads = kWarps * 32;
 constexpr int kMaxKBW = 2;                 // spans per math warp per row: K <= 128 * 16 * 2 = 4096
 constexpr int kMaxStages = 12;
 constexpr int kMinStages = 2;
-constexpr uint32_t kRedBytes = kMath * 32 * 16;  // one float4 per lane of every math warp
+constexpr uint32_t kRedLaneBytes = 32 * 16;  // one float4 per lane of a math warp
+constexpr uint32_t kRedBytes = kMath * kRedLaneBytes;
 
 struct DecodeParams {
   const uint16_t* x;
@@ -82,8 +83,9 @@ struct RingGeom {
   uint32_t bytes;    // stage size (128-byte multiple)
 };
 
-// K = row length of the streamed matrix; h_rows = token rows of h per stage.
-__host__ __device__ inline RingGeom ring_geom(int K, int h_rows, bool with_red) {
+// K = row length of the streamed matrix; h_rows = token rows of h per stage;
+// red_warps = math warps whose partials the stage holds (0: none).
+__host__ __device__ inline RingGeom ring_geom(int K, int h_rows, int red_warps) {
   RingGeom g;
   const int KB = K / 64;
   g.ps = static_cast<uint32_t>(K / 2 + 16);
@@ -97,7 +99,7 @@ __host__ __device__ inline RingGeom ring_geom(int K, int h_rows, bool with_red) 
   g.h_off = g.am_off + al(16 * g.sa * 4, 16);
   g.hs = static_cast<uint32_t>(2 * K + 16);
   g.red_off = g.h_off + static_cast<uint32_t>(h_rows) * g.hs;
-  g.bytes = al(g.red_off + (with_red ? kRedBytes : 0u), 128);
+  g.bytes = al(g.red_off + static_cast<uint32_t>(red_warps) * kRedLaneBytes, 128);
   return g;
 }
 
@@ -244,8 +246,9 @@ __device__ void route_prologue(const DecodeParams& p, uint32_t* lut, int* ids_s,
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int S = p.M * p.k;
   for (int e = tid; e < p.E; e += blockDim.x) uidx[e] = -1;
+  const int nwarps = static_cast<int>(blockDim.x >> 5);
   if (warp < p.M) route_one(p, warp, ids_s, w_s);
-  else fill_lut(lut, warp - p.M, kWarps - p.M);
+  else fill_lut(lut, warp - p.M, nwarps - p.M);
   __syncthreads();
   for (int s = tid; s < S; s += blockDim.x) uidx[ids_s[s]] = 0;  // flag
   __syncthreads();
@@ -302,12 +305,15 @@ __device__ __forceinline__ void drain_ring(uint64_t* full, int issued, int stage
 }
 
 // ---------------------------------------------------------------------------
-// Kernel A: gate_up + SwiGLU (+ LoRA delta) -> h.  KBW = spans per math warp.
-template <int KBW>
-__global__ void __launch_bounds__(kThreads, 1) decode_gate_up_kernel(DecodeParams p) {
+// Kernel A: gate_up + SwiGLU (+ LoRA delta) -> h.  MATH math warps with KBW
+// spans each (MATH * KBW >= the spans of a row), then the producer and the
+// epilogue warp.
+template <int KBW, int MATH>
+__global__ void __launch_bounds__((MATH + 2) * 32, 1) decode_gate_up_kernel(DecodeParams p) {
+  constexpr int kProducerA = MATH, kEpilogueA = MATH + 1;
   extern __shared__ __align__(128) unsigned char smem[];
   const int RS = p.stages_a;
-  const RingGeom G = ring_geom(p.H, 0, true);
+  const RingGeom G = ring_geom(p.H, 0, MATH);
   const Layout L = make_layout(true, p.M, p.k, p.E, p.r, G, RS);
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L.lut);
   int* ids_s = reinterpret_cast<int*>(smem + L.ids);
@@ -324,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gate_up_kernel(DecodeParam
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int H = p.H, I = p.I, KB = H / 64, NSP = (KB + 1) / 2;
-  const int nact = min(kMath, NSP);  // math warps with a span
+  const int nact = min(MATH, NSP);  // math warps with a span
   if (tid == 0) {
     for (int s = 0; s < RS; ++s) {
       mbar_init(&full[s], 1);
@@ -348,8 +354,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gate_up_kernel(DecodeParam
   const int S = p.M * p.k;
   if (p.r > 0) {
     // LoRA first factor per slot: xa[s, rho] = x[token(s)] . lora_A[e(s), rho]
-    if (warp < kMath) {
-      for (int qd = warp; qd < S * p.r; qd += kMath) {
+    if (warp < MATH) {
+      for (int qd = warp; qd < S * p.r; qd += MATH) {
         const int s = qd / p.r, rho = qd % p.r;
         const uint16_t* xr = p.x + static_cast<int64_t>(s / p.k) * H;
         const uint16_t* la = p.lora_A + (static_cast<int64_t>(ids_s[s]) * p.r + rho) * H;
@@ -372,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gate_up_kernel(DecodeParam
     __syncthreads();
   }
 
-  if (warp == kProducer) {
+  if (warp == kProducerA) {
     int issued = 0;
     for (int j = 0; j < n; ++j) {
       const int s = j % RS;
@@ -386,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gate_up_kernel(DecodeParam
       ++issued;
     }
     drain_ring(full, issued, RS);
-  } else if (warp == kEpilogue) {
+  } else if (warp == kEpilogueA) {
     for (int j = 0; j < n; ++j) {
       const int s = j % RS;
       if (!mbar_wait(&done[s], (j / RS) & 1)) {
@@ -439,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gate_up_kernel(DecodeParam
     uint4 xv[KBW][4];
 #pragma unroll
     for (int q2 = 0; q2 < KBW; ++q2) {
-      const int sp = warp + kMath * q2;
+      const int sp = warp + MATH * q2;
       const uint16_t* xr = p.x + static_cast<int64_t>(g) * H + sp * 128 + 16 * t;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -458,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gate_up_kernel(DecodeParam
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int q2 = 0; q2 < KBW; ++q2) {
-        const int sp = warp + kMath * q2;
+        const int sp = warp + MATH * q2;
         if (sp >= NSP) break;
         uint32_t w0[4], w1[4];
         float a0[2], a1[2];
@@ -482,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gate_up_kernel(DecodeParam
 __global__ void __launch_bounds__(kThreads, 1) decode_down_kernel(DecodeParams p) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int RS = p.stages_b;
-  const RingGeom G = ring_geom(p.I, p.M, false);
+  const RingGeom G = ring_geom(p.I, p.M, 0);
   const Layout L = make_layout(false, p.M, p.k, p.E, 0, G, RS);
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L.lut);
   int* ids_s = reinterpret_cast<int*>(smem + L.ids);
@@ -635,9 +641,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_down_kernel(DecodeParams p
   }
 }
 
-template <int KBW>
+template <int KBW, int MATH>
 cudaError_t launch_pair(const DecodeParams& p, int sm_count, size_t smem_a, size_t smem_b, cudaStream_t stream) {
-  cudaError_t err = ensure_smem_limit(reinterpret_cast<const void*>(decode_gate_up_kernel<KBW>), smem_a);
+  cudaError_t err = ensure_smem_limit(reinterpret_cast<const void*>(decode_gate_up_kernel<KBW, MATH>), smem_a);
   if (err != cudaSuccess) return err;
   err = ensure_smem_limit(reinterpret_cast<const void*>(decode_down_kernel), smem_b);
   if (err != cudaSuccess) return err;
@@ -645,7 +651,7 @@ cudaError_t launch_pair(const DecodeParams& p, int sm_count, size_t smem_a, size
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3((MATH + 2) * 32);
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
@@ -654,9 +660,10 @@ cudaError_t launch_pair(const DecodeParams& p, int sm_count, size_t smem_a, size
   cfg.dynamicSmemBytes = smem_a;
   {
     LaunchScope ls("decode.gate_up", stream);
-    err = cudaLaunchKernelEx(&cfg, decode_gate_up_kernel<KBW>, p);
+    err = cudaLaunchKernelEx(&cfg, decode_gate_up_kernel<KBW, MATH>, p);
     if (err != cudaSuccess) return err;
   }
+  cfg.blockDim = dim3(kThreads);
   cfg.gridDim = dim3(std::max(1, std::min(sm_count, p.H / 16)));
   cfg.dynamicSmemBytes = smem_b;
   LaunchScope ls("decode.down", stream);
@@ -678,6 +685,19 @@ DecodeWs decode_ws(int64_t M, int k, int64_t I) {
   return w;
 }
 
+// Math warps of the gate_up kernel and spans per warp for rows of H: the
+// fewest span slots (MATH * KBW) that cover the row's spans, so that no warp
+// of an item waits for another with more spans.
+struct MathSplit {
+  int kbw, math;
+};
+inline MathSplit math_split(int H) {
+  const int nsp = (H / 64 + 1) / 2;
+  if (nsp <= kMath) return {1, kMath};
+  if (nsp <= 24) return {2, 12};
+  return {2, kMath};
+}
+
 struct Stages {
   int a, b;
   size_t smem_a, smem_b;
@@ -685,7 +705,7 @@ struct Stages {
 
 Stages plan_stages(int M, int k, int E, int H, int I, int r, size_t limit) {
   Stages st{};
-  const RingGeom ga = ring_geom(H, 0, true), gb = ring_geom(I, M, false);
+  const RingGeom ga = ring_geom(H, 0, math_split(H).math), gb = ring_geom(I, M, 0);
   st.a = pick_stages(true, M, k, E, r, ga, limit);
   st.b = pick_stages(false, M, k, E, 0, gb, limit);
   if (st.a) st.smem_a = make_layout(true, M, k, E, r, ga, st.a).total;
@@ -744,9 +764,10 @@ cudaError_t launch_decode_forward(const DecodeArgs& a, cudaStream_t stream) {
   if (st.a < kMinStages || st.b < kMinStages) return cudaErrorInvalidConfiguration;
   p.stages_a = st.a;
   p.stages_b = st.b;
-  const int nsp = (p.H / 64 + 1) / 2;
-  if (nsp <= kMath) return launch_pair<1>(p, di.sm_count, st.smem_a, st.smem_b, stream);
-  return launch_pair<2>(p, di.sm_count, st.smem_a, st.smem_b, stream);
+  const MathSplit ms = math_split(p.H);
+  if (ms.kbw == 1) return launch_pair<1, kMath>(p, di.sm_count, st.smem_a, st.smem_b, stream);
+  if (ms.math == 12) return launch_pair<2, 12>(p, di.sm_count, st.smem_a, st.smem_b, stream);
+  return launch_pair<2, kMath>(p, di.sm_count, st.smem_a, st.smem_b, stream);
 }
 
 }  // namespace e4b
