@@ -104,7 +104,7 @@ __host__ __device__ inline RingGeom ring_geom(int K, int h_rows, int red_warps) 
 }
 
 struct Layout {
-  uint32_t lut, ids, w, uidx, touched, slotmap, xa, bars, red, ring, total;
+  uint32_t lut, ids, w, uidx, touched, slotmap, xa, bars, seq, red, ring, total;
 };
 
 // Shared-memory carve of kernel A (gate_up) or B (down) with `stages` ring stages.
@@ -129,6 +129,8 @@ __host__ __device__ inline Layout make_layout(bool is_a, int M, int k, int E, in
   if (is_a && r > 0) o = al(o + S * r * 4, 16);
   L.bars = o;
   o = al(o + (is_a ? 3 * stages : 2 * stages + 4) * 8, 16);
+  L.seq = o;
+  if (!is_a) o = al(o + stages * 4, 16);  // stage held by each ring slot
   L.red = o;
   if (!is_a) o += 2 * kRedBytes;  // partials of two row blocks
   L.ring = al(o, 128);
@@ -297,6 +299,22 @@ __device__ __forceinline__ void issue_rows(const RingGeom& G, unsigned char* st,
     const int i = lane - 16;
     bulk_g2s(st + G.am_off + i * 8 * G.sa * 4, absmax + (i == 0 ? row_a : row_b) * KB, 8 * KB * 4, full);
   }
+}
+
+// Waits (bounded) until ring slot s holds stage j and its copies have landed.
+// A warp that takes only some stages of the ring can reach stage j before the
+// slot's previous stage j - stages has even landed; the parity of the full
+// barrier alone would then look complete.  The producer publishes j in seq[s]
+// (release) after the slot's previous stage was consumed, so once seq[s] == j
+// is seen (acquire) the barrier is at the phase of j or just past it, where
+// the parity wait is exact.
+__device__ __forceinline__ bool wait_stage(uint64_t* full, const int* seq, int s, int j, int stages) {
+  auto ready = [&]() { return ld_acquire_shared(seq + s) == j && mbar_try_wait(&full[s], (j / stages) & 1); };
+  if (ready()) return true;
+  const unsigned long long t0 = global_ns();
+  while (!ready())
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+  return true;
 }
 
 // Drains the producer's copies in flight (bounded) before the CTA exits.
@@ -500,6 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_down_kernel(DecodeParams p
   uint64_t* empty = full + RS;                                   // every span of the stage consumed
   uint64_t* rdone = empty + RS;                                  // [2] partials of a row block written
   uint64_t* rfree = rdone + 2;                                   // [2] partials of a row block summed
+  int* seq = reinterpret_cast<int*>(smem + L.seq);              // stage held by each slot
   float4* red = reinterpret_cast<float4*>(smem + L.red);         // [2][kMath][32]
   unsigned char* ring = smem + L.ring;
   __shared__ int nU_s;
@@ -510,6 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_down_kernel(DecodeParams p
     for (int s = 0; s < RS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], NSP);
+      seq[s] = -1;
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&rdone[b], kMath);
@@ -531,6 +551,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_down_kernel(DecodeParams p
     const uint32_t hrow = static_cast<uint32_t>(I) * 2;
     auto issue_w = [&](int j) {
       const int s = j % RS, u = j % nU;
+      if (lane == 0) st_release_shared(&seq[s], j);  // the slot's previous stage is consumed
+      __syncwarp();
       const int rb = static_cast<int>(blockIdx.x) + (j / nU) * static_cast<int>(gridDim.x);
       const bool has = lane < p.M && slotmap[u * kMaxM + lane] >= 0;
       const int nh = __popc(__ballot_sync(0xffffffffu, has));
@@ -598,7 +620,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_down_kernel(DecodeParams p
       for (int qp = warp; qp < npr; qp += kMath) {
         const int u = qp / NSP, sp = qp % NSP;
         const int j = rbi * nU + u, s = j % RS;
-        if (!mbar_wait(&full[s], (j / RS) & 1)) {
+        if (!wait_stage(full, seq, s, j, RS)) {
           record_error(p.err, kErrWaitFull);
           ok = false;
           break;
