@@ -9,7 +9,8 @@
 //   kernel A  routing (every CTA, redundantly: M <= 8 tokens), then the gate
 //             and up rows of every touched expert in items of 8 gate + 8 up
 //             rows over all of K = H -> SiLU(gate) * up (+ LoRA delta) -> h
-//             (bf16, [M*k, I], slot order).
+//             (bf16, [M*k, I], slot order).  Once its ring is full, its
+//             producer prefetches the touched experts' down rows into L2.
 //   kernel B  the same routing, then for every block of 16 output rows of H
 //             the down rows of every touched expert, with the routing weights
 //             folded in, so the combine happens inside the CTA in a fixed
@@ -47,6 +48,8 @@ constexpr int kMaxKBW = 2;                 // spans per math warp per row: K <= 
 constexpr int kMaxStages = 12;
 constexpr int kMinStages = 2;
 constexpr uint32_t kRedLaneBytes = 32 * 16;  // one float4 per lane of a math warp
+constexpr unsigned long long kPrefetchLimit = 64ull << 20;  // L2 prefetch of the down rows, bytes
+constexpr uint32_t kPrefetchChunk = 32 * 1024;
 constexpr uint32_t kRedBytes = kMath * kRedLaneBytes;
 
 struct DecodeParams {
@@ -322,6 +325,35 @@ __device__ __forceinline__ void drain_ring(uint64_t* full, int issued, int stage
   for (int j = max(0, issued - stages); j < issued; ++j) mbar_wait(&full[j % stages], (j / stages) & 1);
 }
 
+// L2 prefetch of this CTA's share (by 32 KB chunks across the grid and the
+// calling warp's lanes) of the touched experts' down rows and absmax, at most
+// kPrefetchLimit bytes in all.
+__device__ __forceinline__ void prefetch_down_rows(const DecodeParams& p, const int* touched, int nU) {
+  const int lane = threadIdx.x & 31;
+  const uint64_t per_expert = static_cast<uint64_t>(p.H) * p.I / 2;
+  const uint64_t per_expert_am = static_cast<uint64_t>(p.H) * (p.I / 64) * 4;
+  const uint64_t chunks_pk = (per_expert + kPrefetchChunk - 1) / kPrefetchChunk;
+  const uint64_t chunks_am = (per_expert_am + kPrefetchChunk - 1) / kPrefetchChunk;
+  const uint64_t per_u = chunks_pk + chunks_am;
+  uint64_t total = static_cast<uint64_t>(nU) * per_u;
+  const uint64_t cap = kPrefetchLimit / kPrefetchChunk;
+  if (total > cap) total = cap;
+  for (uint64_t c = static_cast<uint64_t>(blockIdx.x) * 32 + lane; c < total; c += static_cast<uint64_t>(gridDim.x) * 32) {
+    const uint64_t u = c / per_u, qq = c % per_u;
+    const int64_t e = touched[u];
+    if (qq < chunks_pk) {
+      const uint64_t off = qq * kPrefetchChunk;
+      const uint64_t nb = min(static_cast<uint64_t>(kPrefetchChunk), per_expert - off);
+      prefetch_l2(p.dn_packed + e * per_expert + off, static_cast<uint32_t>(nb));
+    } else {
+      const uint64_t off = (qq - chunks_pk) * kPrefetchChunk;
+      const uint64_t nb = min(static_cast<uint64_t>(kPrefetchChunk), per_expert_am - off);
+      prefetch_l2(reinterpret_cast<const unsigned char*>(p.dn_absmax) + e * per_expert_am + off,
+                  static_cast<uint32_t>(nb));
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Kernel A: gate_up + SwiGLU (+ LoRA delta) -> h.  MATH math warps with KBW
 // spans each (MATH * KBW >= the spans of a row), then the producer and the
@@ -408,7 +440,12 @@ __global__ void __launch_bounds__((MATH + 2) * 32, 1) decode_gate_up_kernel(Deco
       const int64_t grow = static_cast<int64_t>(touched[u]) * 2 * I + rb * 8;
       issue_rows(G, ring + s * G.bytes, &full[s], p.gu_packed, p.gu_absmax, H, grow, grow + I, 0);
       ++issued;
+      // Once the ring is full: this CTA's share of the touched experts' down
+      // rows into L2.  The down kernel cannot share an SM with this one, so
+      // without it that kernel's stream would start only after this one ends.
+      if (issued == min(n, RS)) prefetch_down_rows(p, touched, nU);
     }
+    if (n == 0) prefetch_down_rows(p, touched, nU);
     drain_ring(full, issued, RS);
   } else if (warp == kEpilogueA) {
     for (int j = 0; j < n; ++j) {
