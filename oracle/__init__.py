@@ -14,6 +14,8 @@ routing  router top-k, the renormalised weights, the token/expert permutation
 moe      the grouped NF4 GEMM, the SwiGLU expert MLP with its optional LoRA
          delta, the weighted combine; a brute-force per-token form and a
          permuted grouped form of the same layer
+mxfp4    e2m1 codes with e8m0 block-32 scales (the OCP microscaling format of
+         released checkpoints) and their grouped GEMM
 backward the layer's gradients through the frozen NF4 experts (input,
          router logits, LoRA A and B) with the routing ids held fixed, per
          token and in the grouped form built on the grouped dgrad product

@@ -182,6 +182,36 @@ def grouped_nf4_gemm_dgrad(dY: np.ndarray, row_index, offsets: np.ndarray, packe
     return out
 
 
+def grouped_lora_grads(x: np.ndarray, row_index, offsets: np.ndarray, da: np.ndarray, lora_A: np.ndarray,
+                       lora_B: np.ndarray, lora_scale: float):
+    """The adapter gradients of one grouped projection, from the gradient ``da``
+    of its output rows (group order) and its input rows ``x[row_index[p]]``:
+
+        dB_e = s * sum_{p in e} da_p^T (x_p . A_e^T)        [N, r]
+        dA_e = s * sum_{p in e} (da_p . B_e)^T x_p          [r, K]
+
+    (the per-slot outer products of ``layer_backward`` summed over a group).
+    Experts without rows get zero gradients."""
+    x = np.asarray(x, dtype=np.float64)
+    da = np.asarray(da, dtype=np.float64)
+    lora_A = np.asarray(lora_A, dtype=np.float64)
+    lora_B = np.asarray(lora_B, dtype=np.float64)
+    off = np.asarray(offsets, dtype=np.int64)
+    rows = off[-1]
+    idx = np.arange(rows) if row_index is None else np.asarray(row_index, dtype=np.int64)
+    dA = np.zeros_like(lora_A)
+    dB = np.zeros_like(lora_B)
+    for e in range(off.size - 1):
+        lo, hi = off[e], off[e + 1]
+        if hi == lo:
+            continue
+        xe = x[idx[lo:hi]]
+        dae = da[lo:hi]
+        dB[e] = lora_scale * dae.T @ (xe @ lora_A[e].T)
+        dA[e] = lora_scale * (dae @ lora_B[e]).T @ xe
+    return dA, dB
+
+
 def layer_backward_grouped(x: np.ndarray, logits: np.ndarray, ids: np.ndarray, stack: ExpertStack,
                            dout: np.ndarray, renormalize: bool = True):
     """``layer_backward`` restated in the permuted, grouped form a GPU runs:
@@ -218,17 +248,7 @@ def layer_backward_grouped(x: np.ndarray, logits: np.ndarray, ids: np.ndarray, s
     dw = dw.reshape(M, k)
     dA = dB = None
     if lora:
-        dA = np.zeros_like(stack.lora_A)
-        dB = np.zeros_like(stack.lora_B)
-        off = np.asarray(offsets, dtype=np.int64)
-        for e in range(stack.E):
-            lo, hi = off[e], off[e + 1]
-            if hi == lo:
-                continue
-            xe = x[tok[lo:hi]]
-            dae = da[lo:hi]
-            dB[e] = s * dae.T @ (xe @ stack.lora_A[e].T)
-            dA[e] = s * (dae @ stack.lora_B[e]).T @ xe
+        dA, dB = grouped_lora_grads(x, tok, offsets, da, stack.lora_A, stack.lora_B, s)
     l = np.asarray(logits, dtype=np.float64)
     dlogits = np.zeros_like(l)
     if renormalize:

@@ -211,3 +211,27 @@ def test_grouped_backward_equals_the_per_token_backward(renorm, lora):
             assert v is None
             continue
         assert np.allclose(u, v, rtol=0, atol=1e-12 * max(1.0, np.abs(u).max()))
+
+
+def test_grouped_lora_grads_brute_force_and_empty_groups():
+    """Element by element over the rows of each group; an expert with no rows
+    gets zero gradients; the row index gathers the input rows."""
+    rng = np.random.default_rng(9)
+    E, N, K, r, s = 3, 6, 5, 2, 1.5
+    offsets = np.array([0, 4, 4, 7])
+    x = rng.standard_normal((9, K))
+    idx = np.array([8, 0, 3, 3, 1, 5, 2])
+    da = rng.standard_normal((7, N))
+    A = rng.standard_normal((E, r, K))
+    B = rng.standard_normal((E, N, r))
+    dA, dB = backward.grouped_lora_grads(x, idx, offsets, da, A, B, s)
+    assert np.all(dA[1] == 0) and np.all(dB[1] == 0)
+    for e, (lo, hi) in enumerate([(0, 4), (4, 4), (4, 7)]):
+        for i in range(N):
+            for rho in range(r):
+                ref = s * sum(da[p, i] * sum(x[idx[p], kk] * A[e, rho, kk] for kk in range(K)) for p in range(lo, hi))
+                assert dB[e, i, rho] == pytest.approx(ref, rel=1e-12, abs=1e-12)
+        for rho in range(r):
+            for kk in range(K):
+                ref = s * sum(sum(da[p, i] * B[e, i, rho] for i in range(N)) * x[idx[p], kk] for p in range(lo, hi))
+                assert dA[e, rho, kk] == pytest.approx(ref, rel=1e-12, abs=1e-12)
