@@ -533,6 +533,63 @@ def time_quantize(cfg, dev, reps=3):
             "GB_per_s": nbytes / (ms * 1e-3) / 1e9}
 
 
+BACKWARD_WORKLOAD = "qwen3_lora_m4096"   # the pages' training shape: Qwen3-MoE-shaped layer with per-expert LoRA
+
+
+def time_backward(name, dev, steps=10, warmup=3):
+    """The layer backward (e4b_moe_expert_backward: recompute, two grouped dgrad
+    products, router and adapter gradients), timed apart from the forward with
+    CUDA events on its stream.  Algorithmic FLOPs: the recompute 6*S*H*I plus the
+    two dgrad products 6*S*H*I (plus the adapter's terms)."""
+    import torch
+
+    from quantized_moe_expert_nf4_b200 import e4b, synthetic
+
+    cfgname, M = WORKLOADS[name]
+    cfg = workloads.CONFIGS[cfgname]
+    layer = synthetic.make_device_layer(cfg, device=dev)
+    x, logits = synthetic.inputs(cfg, M, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(7)
+    dout = torch.randn((M, cfg.H), generator=g, device=dev).bfloat16()
+    dx = torch.empty((M, cfg.H), dtype=torch.float32, device=dev)
+    dl = torch.empty((M, cfg.E), dtype=torch.float32, device=dev)
+    dA = dB = None
+    if cfg.lora_r:
+        dA = torch.empty((cfg.E, cfg.lora_r, cfg.H), dtype=torch.float32, device=dev)
+        dB = torch.empty((cfg.E, 2 * cfg.I, cfg.lora_r), dtype=torch.float32, device=dev)
+    ws = e4b.workspace(e4b.e4b_moe_expert_backward_workspace_size(M, layer.stack, cfg.k), dev)
+
+    def call():
+        e4b.e4b_moe_expert_backward(x, logits, cfg.k, True, layer.stack, dout, dx, dl, dA, dB, ws)
+
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        call()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    launches = e4b.last_launches()
+    e4b.timing_enable(True)
+    call()
+    kt = e4b.timing_read()
+    e4b.timing_enable(False)
+    S = M * cfg.k
+    flops = 12.0 * S * cfg.H * cfg.I
+    if cfg.lora_r:
+        flops += 6.0 * S * cfg.lora_r * (cfg.H + 2 * cfg.I)
+    res = {"workload": name, "ms": ms, "value": S / (ms * 1e-3), "unit": "routed_tokens/s",
+           "tflops": flops / (ms * 1e-3) / 1e12, "algorithmic_flops": flops, "launches": launches,
+           "path": e4b.last_path(), "kernels_us": {k: v[0] * 1e3 / max(v[1], 1) for k, v in kt.items()}}
+    del layer, x, logits, dout, dx, dl, dA, dB, ws
+    torch.cuda.empty_cache()
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -544,6 +601,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end host-buffer pass")
     ap.add_argument("--no-kernel-timing", action="store_true", help="skip the per-kernel event pass")
+    ap.add_argument("--no-backward", action="store_true", help="skip the layer-backward timing")
     ap.add_argument("--replicas", type=int, default=0, help="layer replicas (0: enough to exceed L2 4x)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -589,9 +647,13 @@ def main():
                           "step_roofline_frac": r["step_roofline"]["frac"],
                           "clocks": r["clocks"]})
     quant = None
+    bwd = None
     if rank == 0 and world == 1:
         quant = time_quantize(cfg, f"cuda:{local}")
         quant["frac_hbm"] = quant["GB_per_s"] / peaks["hbm_gbs"]
+        if not args.no_backward:
+            bwd = time_backward(BACKWARD_WORKLOAD, f"cuda:{local}")
+            bwd["frac_tensor"] = bwd["tflops"] / peaks["bf16_tflops"]
     if rank == 0:
         cb = None
         if world == 1 and not args.no_cpu_baseline:
@@ -615,6 +677,7 @@ def main():
             "cpu_baseline": cb, "e2e": main_res["e2e"], "clocks": main_res["clocks"],
             "gpu_launches": main_res["launches_per_step"] * args.steps,
             "quantize": quant,
+            "backward": bwd,
             "sweep": sweep,
         }
         print(json.dumps(line), flush=True)

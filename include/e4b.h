@@ -224,6 +224,65 @@ E4B_API e4b_status e4b_grouped_nf4_gemm(const uint16_t* A, int64_t a_rows, int64
                                 e4b_dtype out_dtype, void* workspace, size_t workspace_bytes,
                                 e4b_stream stream);
 
+/*
+ * Backward through the frozen base -- the input gradient of the grouped NF4
+ * GEMM above, in one launch over all groups.
+ * Source: experts4bit-qlora 0.22.0, "Which training path?" (the backward's
+ * dgrad runs as one launch instead of a per-expert decode loop; the frozen
+ * base is decoded again from the packed bytes, never kept dequantised).
+ *
+ * Row p (0 <= p < total_rows) of group e computes
+ *     dx[p, :] = dY[row_index[p], :] . W_e                       (K values)
+ *     dx[p, :] += lora_scale * (dY[row_index[p], :] . lora_B[e]) . lora_A[e]
+ * with W_e expert e's [N, K] NF4 matrix as in e4b_grouped_nf4_gemm(): for a
+ * forward y = a . W_e^T (+ adapter), dx is the gradient of <dY, y> by a.
+ *
+ * dY              [dy_rows, lddy] bf16 (lddy >= N, lddy % 8 == 0).
+ * row_index       [total_rows] int32 indices into dY, or NULL for p itself.
+ * expert_offsets, packed, absmax, lora_A, lora_B: as in e4b_grouped_nf4_gemm().
+ * out             [total_rows, K] of out_dtype.
+ * Requires K % 64 == 0, N % 64 == 0, 0 <= r <= 16, total_rows < 2^31.
+ * workspace       e4b_grouped_nf4_gemm_dgrad_workspace_size() bytes: an error
+ *                 word and the products dY . lora_B (total_rows x r fp32).
+ * Groups with no rows cost nothing and write nothing.
+ */
+E4B_API size_t e4b_grouped_nf4_gemm_dgrad_workspace_size(int64_t total_rows, int64_t N, int64_t K, int r);
+E4B_API e4b_status e4b_grouped_nf4_gemm_dgrad(const uint16_t* dY, int64_t dy_rows, int64_t lddy,
+                                      const int32_t* row_index, const int32_t* expert_offsets,
+                                      int64_t E, int64_t total_rows, const uint8_t* packed,
+                                      const float* absmax, int64_t N, int64_t K,
+                                      const uint16_t* lora_A, const uint16_t* lora_B, int r,
+                                      float lora_scale, void* out, e4b_dtype out_dtype,
+                                      void* workspace, size_t workspace_bytes, e4b_stream stream);
+
+/*
+ * The adapter's gradients of one grouped projection (backward of the
+ * per-expert LoRA delta over the frozen NF4 base).
+ * Source: Solutions -- one page per problem, the ExpertsLoRA row (a per-expert
+ * low-rank delta before each routed expert's activation, trained over the
+ * frozen stack); experts4bit-qlora 0.22.0, "Which training path?".
+ *
+ * For the forward y_p = x_p . W_e^T + s (x_p . A_e^T) . B_e^T of
+ * e4b_grouped_nf4_gemm() (x_p = x[row_index[p]]) and the gradient da of its
+ * output rows (group order, [total_rows, ldda]):
+ *     dB_e = s * sum_{p in e} da_p^T (x_p . A_e^T)          [N, r] fp32
+ *     dA_e = s * sum_{p in e} (da_p . B_e)^T x_p            [r, K] fp32
+ * summed over each group's rows in order (deterministic); experts without rows
+ * get zeros.  x [x_rows, ldx] bf16 (ldx >= K, ldx % 8 == 0), da bf16,
+ * lora_A [E, r, K], lora_B [E, N, r] bf16, dA [E, r, K], dB [E, N, r] fp32.
+ * Requires K % 64 == 0, N % 64 == 0, 1 <= r <= 16.
+ * workspace       e4b_grouped_lora_grads_workspace_size() bytes: an error
+ *                 word and the products x . A^T and da . B (total_rows x r fp32 each).
+ */
+E4B_API size_t e4b_grouped_lora_grads_workspace_size(int64_t total_rows, int r);
+E4B_API e4b_status e4b_grouped_lora_grads(const uint16_t* x, int64_t x_rows, int64_t ldx,
+                                  const int32_t* row_index, const int32_t* expert_offsets,
+                                  int64_t E, int64_t total_rows, const uint16_t* da, int64_t ldda,
+                                  int64_t N, int64_t K, const uint16_t* lora_A,
+                                  const uint16_t* lora_B, int r, float lora_scale, float* dA,
+                                  float* dB, void* workspace, size_t workspace_bytes,
+                                  e4b_stream stream);
+
 /* The two packed stacks of one MoE layer (device pointers), plus its adapter. */
 typedef struct {
   const uint8_t* gu_packed; /* [E, 2I*H/2]  gate_up_proj, NF4 */
@@ -260,6 +319,33 @@ E4B_API e4b_status e4b_moe_expert_forward_path(const uint16_t* x, int64_t M, con
                                        int k, int renormalize, const e4b_expert_stack* w,
                                        uint16_t* out, void* workspace, size_t workspace_bytes,
                                        e4b_path path, e4b_stream stream);
+
+/*
+ * Backward of the layer through the frozen NF4 experts, routing ids held fixed
+ * (top-k selection is piecewise constant in the logits).
+ * Source: experts4bit-qlora 0.22.0, "Which training path?" (per-expert LoRA
+ * over a frozen NF4 stack; the base is decoded again in backward, one dgrad
+ * launch per projection); Solutions -- one page per problem, the ExpertsLoRA row.
+ *
+ * For out = e4b_moe_expert_forward(x, router_logits, ...) and an upstream
+ * gradient dout [M, H] bf16, writes the gradients of sum(dout * out):
+ *   dx       [M, H] fp32    through gate_up and the adapter's delta
+ *   dlogits  [M, E] fp32    through the routing weights (zero on unselected
+ *                           experts with renormalisation)
+ *   dA, dB   [E, r, H], [E, 2I, r] fp32, the adapter's gradients (required
+ *            when the stack has an adapter, ignored otherwise)
+ * The frozen stacks get no gradient.  It routes again, recomputes the gate_up
+ * output (fp32) and the per-slot expert outputs (fp32), and runs the two
+ * grouped dgrad products of e4b_grouped_nf4_gemm_dgrad() with the SwiGLU
+ * derivative between them; every sum runs in a fixed order (deterministic).
+ * workspace  e4b_moe_expert_backward_workspace_size() bytes (error word first).
+ */
+E4B_API size_t e4b_moe_expert_backward_workspace_size(int64_t M, const e4b_expert_stack* w, int k);
+E4B_API e4b_status e4b_moe_expert_backward(const uint16_t* x, int64_t M, const float* router_logits,
+                                   int k, int renormalize, const e4b_expert_stack* w,
+                                   const uint16_t* dout, float* dx, float* dlogits, float* dA,
+                                   float* dB, void* workspace, size_t workspace_bytes,
+                                   e4b_stream stream);
 
 /*
  * Allocation-free small-batch forward.  The pages have no counterpart of this

@@ -78,6 +78,39 @@ GroupedLayout grouped_layout(int64_t M, int64_t E, int64_t H, int64_t I, int k, 
   return L;
 }
 
+// Workspace of the layer backward (grouped order throughout).
+struct BackwardLayout {
+  size_t err, ids, w, offsets, perm, inv, row_token, route_ws, xa, xg, a, h, z, dz, dw, dh, da, dxg, yb, lg_xa, total;
+};
+
+BackwardLayout backward_layout(int64_t M, int64_t E, int64_t H, int64_t I, int k, int r) {
+  const int64_t S = M * k;
+  Carve c;
+  BackwardLayout L;
+  L.err = c.take(sizeof(int32_t));
+  L.ids = c.take(S * sizeof(int32_t));
+  L.w = c.take(S * sizeof(float));
+  L.offsets = c.take((E + 1) * sizeof(int32_t));
+  L.perm = c.take(S * sizeof(int32_t));
+  L.inv = c.take(S * sizeof(int32_t));
+  L.row_token = c.take(S * sizeof(int32_t));
+  L.route_ws = c.take(route_workspace_bytes(M, E, k));
+  L.xa = c.take(r > 0 ? S * 128 : 0);
+  L.xg = c.take(S * H * sizeof(uint16_t));
+  L.a = c.take(S * 2 * I * sizeof(float));
+  L.h = c.take(S * I * sizeof(uint16_t));
+  L.z = c.take(S * H * sizeof(float));
+  L.dz = c.take(S * H * sizeof(uint16_t));
+  L.dw = c.take(S * sizeof(float));
+  L.dh = c.take(S * I * sizeof(float));
+  L.da = c.take(S * 2 * I * sizeof(uint16_t));
+  L.dxg = c.take(S * H * sizeof(float));
+  L.yb = c.take(r > 0 ? S * r * sizeof(float) : 0);
+  L.lg_xa = c.take(r > 0 ? S * r * sizeof(float) : 0);
+  L.total = c.off;
+  return L;
+}
+
 template <typename T>
 T* at(void* base, size_t off) {
   return reinterpret_cast<T*>(static_cast<char*>(base) + off);
@@ -393,6 +426,164 @@ e4b_status e4b_grouped_nf4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda, 
   return E4B_OK;
 }
 
+size_t e4b_grouped_nf4_gemm_dgrad_workspace_size(int64_t total_rows, int64_t N, int64_t K, int r) {
+  (void)N;
+  (void)K;
+  if (total_rows < 0 || r < 0 || N < 0) return 0;
+  return dgrad_workspace_bytes(total_rows, N, r);
+}
+
+e4b_status e4b_grouped_nf4_gemm_dgrad(const uint16_t* dY, int64_t dy_rows, int64_t lddy, const int32_t* row_index,
+                                      const int32_t* expert_offsets, int64_t E, int64_t total_rows,
+                                      const uint8_t* packed, const float* absmax, int64_t N, int64_t K,
+                                      const uint16_t* lora_A, const uint16_t* lora_B, int r, float lora_scale,
+                                      void* out, e4b_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                                      e4b_stream stream) {
+  begin_call();
+  if (E < 1 || E > 65536) return fail(E4B_ERR_INVALID_ARGUMENT, "E must be in [1, 65536]");
+  if (total_rows < 0 || dy_rows < 0) return fail(E4B_ERR_INVALID_ARGUMENT, "total_rows and dy_rows must be >= 0");
+  if (total_rows > 0 && dy_rows < 1) return fail(E4B_ERR_INVALID_ARGUMENT, "dy_rows must be >= 1 when rows exist");
+  if (K < 64 || K % 64 != 0) return fail(E4B_ERR_UNSUPPORTED, "K must be a positive multiple of 64");
+  if (N < 64 || N % 64 != 0) return fail(E4B_ERR_UNSUPPORTED, "N must be a positive multiple of 64");
+  if (lddy < N || lddy % 8 != 0) return fail(E4B_ERR_INVALID_ARGUMENT, "lddy must be >= N and a multiple of 8");
+  if (out_dtype != E4B_F32 && out_dtype != E4B_BF16) return fail(E4B_ERR_INVALID_ARGUMENT, "out_dtype must be F32 or BF16");
+  if ((lora_A == nullptr) != (lora_B == nullptr))
+    return fail(E4B_ERR_INVALID_ARGUMENT, "lora_A and lora_B must be both set or both NULL");
+  if (lora_A && (r < 1 || r > 16)) return fail(E4B_ERR_UNSUPPORTED, "LoRA rank must be in [1, 16]");
+  if (!lora_A) r = 0;
+  if (!expert_offsets || !packed || !absmax) return fail(E4B_ERR_INVALID_ARGUMENT, "null expert_offsets, packed or absmax");
+  if (total_rows > 0 && (!dY || !out)) return fail(E4B_ERR_INVALID_ARGUMENT, "null dY or out");
+  if (total_rows > INT32_MAX) return fail(E4B_ERR_UNSUPPORTED, "total_rows exceeds int32");
+  if ((dY && !aligned16(dY)) || !aligned16(packed) || !aligned16(absmax) || (out && !aligned16(out)))
+    return fail(E4B_ERR_INVALID_ARGUMENT, "dY, packed, absmax and out must be 16-byte aligned");
+  if (lora_A && (!aligned16(lora_A) || !aligned16(lora_B)))
+    return fail(E4B_ERR_INVALID_ARGUMENT, "lora_A and lora_B must be 16-byte aligned");
+  if (e4b_status s = check_workspace("dgrad", dgrad_workspace_bytes(total_rows, N, r), workspace, workspace_bytes);
+      s != E4B_OK)
+    return s;
+  if (e4b_status s = check_device(); s != E4B_OK) return s;
+  if (total_rows == 0) {
+    set_path("dgrad.empty");
+    return E4B_OK;
+  }
+  DgradArgs d{};
+  d.dY = dY;
+  d.dy_rows = dy_rows;
+  d.lddy = lddy;
+  d.row_index = row_index;
+  d.offsets = expert_offsets;
+  d.E = static_cast<int>(E);
+  d.total_rows = total_rows;
+  d.packed = packed;
+  d.absmax = absmax;
+  d.N = static_cast<int>(N);
+  d.K = static_cast<int>(K);
+  d.lora_A = r ? lora_A : nullptr;
+  d.lora_B = r ? lora_B : nullptr;
+  d.r = r;
+  d.lora_scale = lora_scale;
+  d.yb = r ? reinterpret_cast<float*>(static_cast<char*>(workspace) + dgrad_workspace_yb_offset()) : nullptr;
+  d.gathered = reinterpret_cast<uint16_t*>(static_cast<char*>(workspace) + dgrad_workspace_gather_offset(total_rows, r));
+  d.err = static_cast<int*>(workspace);
+  d.out = out;
+  d.out_bf16 = out_dtype == E4B_BF16;
+  const char* path = "";
+  cudaError_t err = launch_grouped_dgrad(d, reinterpret_cast<cudaStream_t>(stream), &path);
+  if (err != cudaSuccess) return cuda_fail(err, "grouped dgrad launch");
+  set_path(path);
+  return E4B_OK;
+}
+
+size_t e4b_grouped_lora_grads_workspace_size(int64_t total_rows, int r) {
+  if (total_rows < 0 || r < 1 || r > 16) return 0;
+  return lora_grads_workspace_bytes(total_rows, r);
+}
+
+e4b_status e4b_grouped_lora_grads(const uint16_t* x, int64_t x_rows, int64_t ldx, const int32_t* row_index,
+                                  const int32_t* expert_offsets, int64_t E, int64_t total_rows, const uint16_t* da,
+                                  int64_t ldda, int64_t N, int64_t K, const uint16_t* lora_A,
+                                  const uint16_t* lora_B, int r, float lora_scale, float* dA, float* dB,
+                                  void* workspace, size_t workspace_bytes, e4b_stream stream) {
+  begin_call();
+  if (E < 1 || E > 65536) return fail(E4B_ERR_INVALID_ARGUMENT, "E must be in [1, 65536]");
+  if (total_rows < 0 || x_rows < 0) return fail(E4B_ERR_INVALID_ARGUMENT, "total_rows and x_rows must be >= 0");
+  if (total_rows > 0 && x_rows < 1) return fail(E4B_ERR_INVALID_ARGUMENT, "x_rows must be >= 1 when rows exist");
+  if (K < 64 || K % 64 != 0) return fail(E4B_ERR_UNSUPPORTED, "K must be a positive multiple of 64");
+  if (N < 64 || N % 64 != 0) return fail(E4B_ERR_UNSUPPORTED, "N must be a positive multiple of 64");
+  if (r < 1 || r > 16) return fail(E4B_ERR_UNSUPPORTED, "LoRA rank must be in [1, 16]");
+  if (ldx < K || ldx % 8 != 0) return fail(E4B_ERR_INVALID_ARGUMENT, "ldx must be >= K and a multiple of 8");
+  if (ldda < N) return fail(E4B_ERR_INVALID_ARGUMENT, "ldda must be >= N");
+  if (!expert_offsets || !lora_A || !lora_B || !dA || !dB)
+    return fail(E4B_ERR_INVALID_ARGUMENT, "null expert_offsets, lora_A, lora_B, dA or dB");
+  if (total_rows > 0 && (!x || !da)) return fail(E4B_ERR_INVALID_ARGUMENT, "null x or da");
+  if (total_rows > INT32_MAX) return fail(E4B_ERR_UNSUPPORTED, "total_rows exceeds int32");
+  if ((x && !aligned16(x)) || !aligned16(lora_A) || !aligned16(lora_B) || !aligned16(dA) || !aligned16(dB) ||
+      (da && !aligned16(da)))
+    return fail(E4B_ERR_INVALID_ARGUMENT, "x, da, lora_A, lora_B, dA and dB must be 16-byte aligned");
+  if (e4b_status s = check_workspace("lora grads", lora_grads_workspace_bytes(total_rows, r), workspace,
+                                     workspace_bytes);
+      s != E4B_OK)
+    return s;
+  if (e4b_status s = check_device(); s != E4B_OK) return s;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  float* xa = reinterpret_cast<float*>(static_cast<char*>(workspace) + 256);
+  float* yb = reinterpret_cast<float*>(static_cast<char*>(workspace) + lora_grads_workspace_yb_offset(total_rows, r));
+  if (total_rows > 0) {
+    GemmArgs g{};
+    g.A = x;
+    g.a_rows = x_rows;
+    g.lda = ldx;
+    g.row_index = row_index;
+    g.offsets = expert_offsets;
+    g.E = static_cast<int>(E);
+    g.total_rows = total_rows;
+    g.N = static_cast<int>(N);
+    g.K = static_cast<int>(K);
+    g.lora_A = lora_A;
+    g.lora_B = lora_B;
+    g.r = r;
+    g.xa = xa;
+    cudaError_t err = launch_lora_xa(g, st);
+    if (err != cudaSuccess) return cuda_fail(err, "lora grads: x . A^T");
+    DgradArgs d{};
+    d.dY = da;
+    d.dy_rows = total_rows;
+    d.lddy = ldda;
+    d.offsets = expert_offsets;
+    d.E = static_cast<int>(E);
+    d.total_rows = total_rows;
+    d.N = static_cast<int>(N);
+    d.K = static_cast<int>(K);
+    d.lora_B = lora_B;
+    d.r = r;
+    d.yb = yb;
+    err = launch_dgrad_lora_yb(d, st);
+    if (err != cudaSuccess) return cuda_fail(err, "lora grads: da . B");
+  }
+  LoraGradArgs a{};
+  a.x = x;
+  a.x_rows = x_rows;
+  a.ldx = ldx;
+  a.row_index = row_index;
+  a.offsets = expert_offsets;
+  a.E = static_cast<int>(E);
+  a.total_rows = total_rows;
+  a.da = da;
+  a.ldda = ldda;
+  a.N = static_cast<int>(N);
+  a.K = static_cast<int>(K);
+  a.r = r;
+  a.lora_scale = lora_scale;
+  a.xa = xa;
+  a.yb = yb;
+  a.dA = dA;
+  a.dB = dB;
+  cudaError_t err = launch_lora_grads(a, st);
+  if (err != cudaSuccess) return cuda_fail(err, "lora grads launch");
+  set_path("lora_grads");
+  return E4B_OK;
+}
+
 static e4b_status check_stack(const e4b_expert_stack* w, int k) {
   if (!w) return fail(E4B_ERR_INVALID_ARGUMENT, "null expert stack");
   if (w->E < 1 || w->E > 1024) return fail(E4B_ERR_UNSUPPORTED, "E must be in [1, 1024]");
@@ -516,6 +707,173 @@ e4b_status e4b_moe_expert_forward(const uint16_t* x, int64_t M, const float* rou
                                   e4b_stream stream) {
   return e4b_moe_expert_forward_path(x, M, router_logits, k, renormalize, w, out, workspace, workspace_bytes,
                                      E4B_PATH_AUTO, stream);
+}
+
+size_t e4b_moe_expert_backward_workspace_size(int64_t M, const e4b_expert_stack* w, int k) {
+  if (!w || M <= 0 || k < 1 || w->E < 1 || w->H < 1 || w->I < 1) return 0;
+  return backward_layout(M, w->E, w->H, w->I, k, stack_r(w)).total;
+}
+
+e4b_status e4b_moe_expert_backward(const uint16_t* x, int64_t M, const float* router_logits, int k, int renormalize,
+                                   const e4b_expert_stack* w, const uint16_t* dout, float* dx, float* dlogits,
+                                   float* dA, float* dB, void* workspace, size_t workspace_bytes,
+                                   e4b_stream stream) {
+  begin_call();
+  if (e4b_status s = check_stack(w, k); s != E4B_OK) return s;
+  if (M < 0) return fail(E4B_ERR_INVALID_ARGUMENT, "M must be >= 0");
+  if (M * k > INT32_MAX) return fail(E4B_ERR_UNSUPPORTED, "M*k exceeds int32 slot indices");
+  if (M > 0 && (!x || !router_logits || !dout || !dx || !dlogits))
+    return fail(E4B_ERR_INVALID_ARGUMENT, "null x, router_logits, dout, dx or dlogits");
+  const int r = stack_r(w);
+  if (r > 0 && (!dA || !dB)) return fail(E4B_ERR_INVALID_ARGUMENT, "a stack with an adapter needs dA and dB");
+  if (M > 0 && (!aligned16(x) || !aligned16(dout) || !aligned16(dx) || !aligned16(dlogits) ||
+                (dA && !aligned16(dA)) || (dB && !aligned16(dB))))
+    return fail(E4B_ERR_INVALID_ARGUMENT, "x, dout, dx, dlogits, dA and dB must be 16-byte aligned");
+  if (e4b_status s = check_workspace("backward", e4b_moe_expert_backward_workspace_size(M, w, k), workspace,
+                                     workspace_bytes);
+      s != E4B_OK)
+    return s;
+  if (e4b_status s = check_device(); s != E4B_OK) return s;
+  const cudaStream_t stream_ = reinterpret_cast<cudaStream_t>(stream);
+  if (M == 0) {
+    if (r > 0) {  // no rows: the adapter gradients are zero
+      cudaError_t err = cudaMemsetAsync(dA, 0, static_cast<size_t>(w->E) * r * w->H * sizeof(float), stream_);
+      if (err == cudaSuccess)
+        err = cudaMemsetAsync(dB, 0, static_cast<size_t>(w->E) * 2 * w->I * r * sizeof(float), stream_);
+      if (err != cudaSuccess) return cuda_fail(err, "backward: zero adapter gradients");
+    }
+    set_path("backward.empty");
+    return E4B_OK;
+  }
+  void* ws = workspace;
+  const BackwardLayout L = backward_layout(M, w->E, w->H, w->I, k, r);
+  const int64_t S = M * k;
+  const int E = static_cast<int>(w->E), H = static_cast<int>(w->H), I = static_cast<int>(w->I);
+  const float scale = r ? w->lora_alpha / static_cast<float>(r) : 0.0f;
+  RouteOut o{at<int32_t>(ws, L.ids), at<float>(ws, L.w), at<int32_t>(ws, L.offsets),
+             at<int32_t>(ws, L.perm), at<int32_t>(ws, L.inv), at<int32_t>(ws, L.row_token)};
+  cudaError_t err = launch_route(router_logits, M, E, k, renormalize != 0, o, at<void>(ws, L.route_ws), stream_);
+  if (err != cudaSuccess) return cuda_fail(err, "backward: route");
+  // Recompute a = [g | u] (fp32) and z (fp32) per grouped row.
+  GemmArgs g{};
+  g.A = x;
+  g.a_rows = M;
+  g.lda = H;
+  g.row_index = o.row_token;
+  g.offsets = o.offsets;
+  g.E = E;
+  g.total_rows = S;
+  g.packed = w->gu_packed;
+  g.absmax = w->gu_absmax;
+  g.N = 2 * I;
+  g.K = H;
+  g.lora_A = r ? w->lora_A : nullptr;
+  g.lora_B = r ? w->lora_B : nullptr;
+  g.r = r;
+  g.lora_scale = scale;
+  g.xa = r ? at<float>(ws, L.xa) : nullptr;
+  g.a_gathered = at<uint16_t>(ws, L.xg);
+  g.err = at<int>(ws, L.err);
+  g.epi = E4B_EPI_NONE;
+  g.out = at<float>(ws, L.a);
+  g.out_bf16 = false;
+  const char* path = "";
+  if ((err = launch_grouped_gemm(g, stream_, &path)) != cudaSuccess) return cuda_fail(err, "backward: gate_up gemm");
+  if ((err = launch_swiglu_h(at<float>(ws, L.a), S, I, at<uint16_t>(ws, L.h), stream_)) != cudaSuccess)
+    return cuda_fail(err, "backward: swiglu");
+  GemmArgs d{};
+  d.A = at<uint16_t>(ws, L.h);
+  d.a_rows = S;
+  d.lda = I;
+  d.offsets = o.offsets;
+  d.E = E;
+  d.total_rows = S;
+  d.packed = w->dn_packed;
+  d.absmax = w->dn_absmax;
+  d.N = H;
+  d.K = I;
+  d.err = at<int>(ws, L.err);
+  d.epi = E4B_EPI_NONE;
+  d.out = at<float>(ws, L.z);
+  d.out_bf16 = false;
+  if ((err = launch_grouped_gemm(d, stream_, &path)) != cudaSuccess) return cuda_fail(err, "backward: down gemm");
+  // dz = w * dout per grouped row, dw = dout . z per slot
+  if ((err = launch_slot_grads(dout, at<float>(ws, L.z), o.perm, o.row_token, o.w, S, M, H, at<uint16_t>(ws, L.dz),
+                               at<float>(ws, L.dw), stream_)) != cudaSuccess)
+    return cuda_fail(err, "backward: slot gradients");
+  // dh = dz . Wd (dgrad through down), da by the SwiGLU derivative
+  DgradArgs dd{};
+  dd.dY = at<uint16_t>(ws, L.dz);
+  dd.dy_rows = S;
+  dd.lddy = H;
+  dd.offsets = o.offsets;
+  dd.E = E;
+  dd.total_rows = S;
+  dd.packed = w->dn_packed;
+  dd.absmax = w->dn_absmax;
+  dd.N = H;
+  dd.K = I;
+  dd.out = at<float>(ws, L.dh);
+  dd.out_bf16 = false;
+  dd.err = at<int>(ws, L.err);
+  if ((err = launch_grouped_dgrad(dd, stream_, &path)) != cudaSuccess) return cuda_fail(err, "backward: dgrad down");
+  if ((err = launch_swiglu_bwd(at<float>(ws, L.a), at<float>(ws, L.dh), S, I, at<uint16_t>(ws, L.da), stream_)) !=
+      cudaSuccess)
+    return cuda_fail(err, "backward: swiglu derivative");
+  // dx per grouped row through gate_up (with the adapter's share), then per token
+  DgradArgs dg{};
+  dg.dY = at<uint16_t>(ws, L.da);
+  dg.dy_rows = S;
+  dg.lddy = 2 * I;
+  dg.offsets = o.offsets;
+  dg.E = E;
+  dg.total_rows = S;
+  dg.packed = w->gu_packed;
+  dg.absmax = w->gu_absmax;
+  dg.N = 2 * I;
+  dg.K = H;
+  dg.lora_A = r ? w->lora_A : nullptr;
+  dg.lora_B = r ? w->lora_B : nullptr;
+  dg.r = r;
+  dg.lora_scale = scale;
+  dg.yb = r ? at<float>(ws, L.yb) : nullptr;
+  dg.out = at<float>(ws, L.dxg);
+  dg.out_bf16 = false;
+  dg.err = at<int>(ws, L.err);
+  if ((err = launch_grouped_dgrad(dg, stream_, &path)) != cudaSuccess) return cuda_fail(err, "backward: dgrad gate_up");
+  if ((err = launch_token_sum(at<float>(ws, L.dxg), o.inv, M, k, H, dx, stream_)) != cudaSuccess)
+    return cuda_fail(err, "backward: token sum");
+  if ((err = launch_router_grad(router_logits, o.ids, o.w, at<float>(ws, L.dw), M, E, k, renormalize != 0, dlogits,
+                                stream_)) != cudaSuccess)
+    return cuda_fail(err, "backward: router gradient");
+  if (r > 0) {
+    // adapter gradients of gate_up: xa = x . A^T here, yb = da . B from the
+    // gate_up dgrad above, then the per-group sums
+    GemmArgs gx = g;
+    gx.xa = at<float>(ws, L.lg_xa);
+    if ((err = launch_lora_xa(gx, stream_)) != cudaSuccess) return cuda_fail(err, "backward: x . A^T");
+    LoraGradArgs la{};
+    la.x = x;
+    la.x_rows = M;
+    la.ldx = H;
+    la.row_index = o.row_token;
+    la.offsets = o.offsets;
+    la.E = E;
+    la.total_rows = S;
+    la.da = at<uint16_t>(ws, L.da);
+    la.ldda = 2 * I;
+    la.N = 2 * I;
+    la.K = H;
+    la.r = r;
+    la.lora_scale = scale;
+    la.xa = at<float>(ws, L.lg_xa);
+    la.yb = at<float>(ws, L.yb);
+    la.dA = dA;
+    la.dB = dB;
+    if ((err = launch_lora_grads(la, stream_)) != cudaSuccess) return cuda_fail(err, "backward: adapter gradients");
+  }
+  set_path("backward.grouped");
+  return E4B_OK;
 }
 
 }  // extern "C"

@@ -97,6 +97,74 @@ cudaError_t launch_tc_lora_prep(const GemmArgs& a, cudaStream_t stream);
 // Picks the implementation; reports the path name through set_path.
 cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const char** path);
 
+// ---- grouped dgrad ---------------------------------------------------------
+struct DgradArgs {
+  const uint16_t* dY;
+  int64_t dy_rows, lddy;
+  const int32_t* row_index;  // nullable
+  const int32_t* offsets;    // [E+1]
+  int E;
+  int64_t total_rows;
+  const uint8_t* packed;
+  const float* absmax;
+  int N, K;
+  const uint16_t* lora_A;  // [E, r, K] or nullptr
+  const uint16_t* lora_B;  // [E, N, r] or nullptr
+  int r;
+  float lora_scale;
+  float* yb;  // workspace [total_rows, r] fp32: dY . lora_B
+  uint16_t* gathered;  // workspace [total_rows, N] bf16: dY rows in group order (tensor-core path)
+  int* err;            // workspace error word
+  void* out;  // [total_rows, K]
+  bool out_bf16;
+};
+// Workspace: [error word, 256 B][dY . lora_B, total_rows * r fp32][dY rows gathered,
+// total_rows * N bf16], parts 256-B aligned.
+size_t dgrad_workspace_bytes(int64_t total_rows, int64_t N, int r);
+size_t dgrad_workspace_yb_offset();
+size_t dgrad_workspace_gather_offset(int64_t total_rows, int r);
+// Warp-MMA kernel below 512 routed rows (and with an adapter and bf16 output),
+// the tensor-core kernel otherwise; E4B_DGRAD=mma|tc forces one.
+cudaError_t launch_grouped_dgrad(const DgradArgs& a, cudaStream_t stream, const char** path);
+bool dgrad_tc_supported(const DgradArgs& a, int64_t lddy);
+cudaError_t launch_grouped_dgrad_tc(const DgradArgs& a, const uint16_t* dy, int64_t dy_rows, int64_t lddy,
+                                    int* err_word, cudaStream_t stream);
+// yb = dY . lora_B per routed row (into a.yb); a.lora_B, a.r, a.N, a.dY, a.lddy used.
+cudaError_t launch_dgrad_lora_yb(const DgradArgs& a, cudaStream_t stream);
+
+// ---- grouped LoRA gradients ---------------------------------------------------
+struct LoraGradArgs {
+  const uint16_t* x;  // input rows of the projection (gathered by row_index)
+  int64_t x_rows, ldx;
+  const int32_t* row_index;  // nullable
+  const int32_t* offsets;    // [E+1]
+  int E;
+  int64_t total_rows;
+  const uint16_t* da;  // [total_rows, ldda] gradient of the projection's output rows
+  int64_t ldda;
+  int N, K, r;
+  float lora_scale;
+  const float* xa;  // [total_rows, r] x . A_e^T
+  const float* yb;  // [total_rows, r] da . B_e
+  float* dA;        // [E, r, K]
+  float* dB;        // [E, N, r]
+};
+// Workspace: [error word, 256 B][xa, total_rows * r fp32][yb, total_rows * r fp32], 256-B aligned parts.
+size_t lora_grads_workspace_bytes(int64_t total_rows, int r);
+size_t lora_grads_workspace_yb_offset(int64_t total_rows, int r);
+cudaError_t launch_lora_grads(const LoraGradArgs& a, cudaStream_t stream);
+
+// ---- layer backward steps (csrc/backward.cu) -------------------------------------
+cudaError_t launch_swiglu_h(const float* a, int64_t S, int I, uint16_t* h, cudaStream_t stream);
+cudaError_t launch_slot_grads(const uint16_t* dout, const float* z, const int32_t* perm, const int32_t* row_token,
+                              const float* w, int64_t S, int64_t M, int H, uint16_t* dz, float* dw,
+                              cudaStream_t stream);
+cudaError_t launch_swiglu_bwd(const float* a, const float* dh, int64_t S, int I, uint16_t* da, cudaStream_t stream);
+cudaError_t launch_token_sum(const float* dxg, const int32_t* inv, int64_t M, int k, int H, float* dx,
+                             cudaStream_t stream);
+cudaError_t launch_router_grad(const float* logits, const int32_t* ids, const float* w, const float* dw, int64_t M,
+                               int E, int k, bool renormalize, float* dlogits, cudaStream_t stream);
+
 // ---- combine ---------------------------------------------------------------
 cudaError_t launch_combine(const uint16_t* z, const int32_t* inv, const float* w, int64_t M, int k,
                            int H, uint16_t* out, cudaStream_t stream);

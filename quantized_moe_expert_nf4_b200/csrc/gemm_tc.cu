@@ -166,7 +166,91 @@ __device__ __forceinline__ bool locate(const TcParams& p, int64_t t, int* e, int
   return true;
 }
 
+// Decoders of the dgrad product.  Thread dt takes rows n in [8o, 8o + 8) of the
+// K step and columns k in [4q, 4q + 4) of the tile (q = 0..63: the tile's 256
+// columns, o = 0..7).  The nibbles of row pairs (n, n+1) are interleaved so
+// that one byte holds one column's codes of both rows; four such bytes decode
+// (byte permutes) to the bf16 pairs (W[n][k], W[n+1][k]) of four columns,
+// scaled by (absmax[n], absmax[n+1]) of their 64-column block.  Row k of the A
+// tile (K-major, 128-byte swizzle) takes the 8 rows n as one 16-byte chunk.
 template <class S>
+__device__ __forceinline__ void dgrad_decoders(const TcParams& p, unsigned char* smem, uint64_t* tma_full,
+                                               uint64_t* a_empty, uint64_t* a_full, int dt, int lane) {
+  static_assert(S::HALVES == 2, "the dgrad decoders cover 256 columns per tile");
+  constexpr int BN = S::BN, KS = S::kKS, AS = S::kAS;
+  constexpr int kRowBytes = S::HALVES * 64;  // packed bytes of one row n in the tile
+  const int q = (dt & 7) | (((dt >> 5) & 7) << 3);
+  const int o = ((dt >> 3) & 3) | ((dt >> 8) << 2);
+  const int KB = p.K / 64, kbw = p.N / 64;
+  const CodebookBytes cbt = codebook_bytes();
+  uint32_t kbg = 0;
+  bool ok = true;
+  for (int64_t t = blockIdx.x; ok; t += gridDim.x) {
+    int e, n_tile;
+    int64_t rb, re;
+    if (!locate<BN>(p, t, &e, &rb, &re, &n_tile)) break;
+    int r0, r1;
+    tile_rows<S::HALVES>(p, n_tile, &r0, &r1);
+    const int kcol = r0 + 4 * q;  // first of this thread's four columns
+    const bool valid = kcol < p.N;
+    const float* am = p.absmax + (static_cast<int64_t>(e) * p.K + 8 * o) * kbw + (valid ? kcol / 64 : 0);
+    float sc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) sc[i] = valid ? __ldg(am + static_cast<int64_t>(i) * kbw) : 0.0f;
+    for (int kb = 0; kb < KB && ok; ++kb) {
+      float nsc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        nsc[i] = (valid && kb + 1 < KB) ? __ldg(am + static_cast<int64_t>((kb + 1) * 64 + i) * kbw) : 0.0f;
+      const int s = kbg % KS, a = kbg % AS;
+      if (!mbar_wait(&tma_full[s], (kbg / KS) & 1) ||
+          (kbg >= AS && !mbar_wait(&a_empty[a], ((kbg / AS) - 1) & 1))) {
+        record_error(p.err, kErrWaitFull);
+        ok = false;
+        break;
+      }
+      const unsigned char* src = smem + S::kOffTma + s * S::kTmaStageBytes;
+      uint32_t col[4][4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int n = 8 * o + 2 * j;
+        const uint32_t x = *reinterpret_cast<const uint16_t*>(src + n * kRowBytes + 2 * q);
+        const uint32_t y = *reinterpret_cast<const uint16_t*>(src + (n + 1) * kRowBytes + 2 * q);
+        const uint32_t ev = (x & 0xF0F0u) | ((y >> 4) & 0x0F0Fu);  // columns 4q, 4q+2: (row n, row n+1) codes
+        const uint32_t od = ((x << 4) & 0xF0F0u) | (y & 0x0F0Fu);  // columns 4q+1, 4q+3
+        uint32_t v[4];
+        decode4(ev, cbt, &v[0], &v[2]);
+        decode4(od, cbt, &v[1], &v[3]);
+        const __nv_bfloat162 s2 = __floats2bfloat162_rn(sc[2 * j], sc[2 * j + 1]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          __nv_bfloat162 h2 = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&v[c]), s2);
+          col[c][j] = *reinterpret_cast<uint32_t*>(&h2);
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int kl = 4 * q + c;  // A row: column k of the tile
+        const int half = kl >> 7, ri = kl & 127;
+        unsigned char* arow =
+            smem + S::kOffA + a * S::kAStageBytes + half * kAHalfBytes + (ri >> 3) * 1024 + (ri & 7) * 128;
+        *reinterpret_cast<uint4*>(arow + ((o ^ (ri & 7)) << 4)) = make_uint4(col[c][0], col[c][1], col[c][2], col[c][3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&a_full[a]);
+      ++kbg;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) sc[i] = nsc[i];
+    }
+  }
+}
+
+// DG: the input-gradient product (dgrad).  The tile's "weight rows" are then
+// columns k of W (p.N = K of W), the K steps run over the rows n of W
+// (p.K = N of W), the packed tile is 64 rows n x (HALVES * 64) bytes, and the
+// decoders write W^T: row k of the A tile holds W[n][k] for the step's 64 n.
+template <class S, bool DG>
 __global__ void __launch_bounds__(kThreadsTc, 1)
     grouped_nf4_tc_kernel(const __grid_constant__ CUtensorMap tm_packed, const __grid_constant__ CUtensorMap tm_b,
                           const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ CUtensorMap tm_xa,
@@ -225,6 +309,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       int r0, r1;
       tile_rows<HALVES>(p, n_tile, &r0, &r1);
       const int32_t y0 = e * p.N + r0, y1 = e * p.N + r1;
+      (void)y0;
+      (void)y1;
       for (int kb = 0; kb < KB; ++kb, ++kbg) {
         const int s = kbg % KS;
         if (kbg >= KS && !mbar_wait(&tma_empty[s], ((kbg / KS) - 1) & 1)) {
@@ -235,8 +321,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         unsigned char* st = smem + S::kOffTma + s * S::kTmaStageBytes;
         if (lane == 0) {
           mbar_arrive_expect_tx(&tma_full[s], S::kTmaStageBytes);
-          tma_load_2d(st, &tm_packed, kb * 32, y0, &tma_full[s]);
-          if (HALVES == 2) tma_load_2d(st + kPackedHalfBytes, &tm_packed, kb * 32, y1, &tma_full[s]);
+          if constexpr (DG) {
+            tma_load_2d(st, &tm_packed, r0 / 2, static_cast<int32_t>(static_cast<int64_t>(e) * p.K + kb * 64),
+                        &tma_full[s]);
+          } else {
+            tma_load_2d(st, &tm_packed, kb * 32, y0, &tma_full[s]);
+            if (HALVES == 2) tma_load_2d(st + kPackedHalfBytes, &tm_packed, kb * 32, y1, &tma_full[s]);
+          }
           tma_load_2d(st + S::kPackedBytes, &tm_b, kb * 64, static_cast<int32_t>(rb), &tma_full[s]);
         }
         __syncwarp();
@@ -329,6 +420,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   } else if (warp >= kWarpDec && warp < kWarpDec + kNumDecWarps) {
     // ------------------------------------------------------------- decoders
     const int dt = tid - kWarpDec * 32;            // 0..511
+    if constexpr (DG) {
+      dgrad_decoders<S>(p, smem, tma_full, a_empty, a_full, dt, lane);
+    } else {
     const int r = dt / S::kTpr, kq = dt % S::kTpr;  // weight row of the tile, part of the k block
     const int half = r >> 7, ri = r & 127;
     const CodebookBytes cbt = codebook_bytes();
@@ -429,6 +523,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         if (lane == 0) mbar_arrive(&a_full[a]);
         ++kbg;
       }
+    }
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------- epilogue
@@ -548,7 +643,7 @@ cudaError_t launch_shape(const GemmArgs& a, int* err_word, cudaStream_t stream) 
   DeviceInfo di;
   cudaError_t err = device_info(&di);
   if (err != cudaSuccess) return err;
-  err = ensure_smem_limit(reinterpret_cast<const void*>(grouped_nf4_tc_kernel<S>), S::kSmemBytes);
+  err = ensure_smem_limit(reinterpret_cast<const void*>(grouped_nf4_tc_kernel<S, false>), S::kSmemBytes);
   if (err != cudaSuccess) return err;
   CUtensorMap tm_packed, tm_b;
   const uint64_t total_w_rows = static_cast<uint64_t>(a.E) * a.N;
@@ -591,7 +686,53 @@ cudaError_t launch_shape(const GemmArgs& a, int* err_word, cudaStream_t stream) 
       ((a.total_rows + S::BN - 1) / S::BN + (a.E < a.total_rows ? a.E : a.total_rows)) * p.n_tiles;
   const int grid = static_cast<int>(tiles < di.sm_count ? tiles : di.sm_count);
   LaunchScope ls(p.swiglu ? "gemm.tc.swiglu" : "gemm.tc", stream);
-  grouped_nf4_tc_kernel<S><<<grid, kThreadsTc, S::kSmemBytes, stream>>>(tm_packed, tm_b, tm_out, tm_xa, p);
+  grouped_nf4_tc_kernel<S, false><<<grid, kThreadsTc, S::kSmemBytes, stream>>>(tm_packed, tm_b, tm_out, tm_xa, p);
+  return cudaGetLastError();
+}
+
+// The dgrad product on the tensor cores: A tile = W^T (256 columns k per
+// tile), B = the dY rows (contiguous, in group order), K steps over the rows n.
+template <class S>
+cudaError_t launch_dgrad_shape(const DgradArgs& a, const uint16_t* dy, int64_t dy_rows, int64_t lddy, int* err_word,
+                               cudaStream_t stream) {
+  static_assert(S::HALVES == 2, "dgrad tiles cover 256 columns");
+  DeviceInfo di;
+  cudaError_t err = device_info(&di);
+  if (err != cudaSuccess) return err;
+  err = ensure_smem_limit(reinterpret_cast<const void*>(grouped_nf4_tc_kernel<S, true>), S::kSmemBytes);
+  if (err != cudaSuccess) return err;
+  CUtensorMap tm_packed, tm_b, tm_out;
+  const uint64_t total_w_rows = static_cast<uint64_t>(a.E) * a.N;  // rows n of every expert
+  if (!make_map_2d(&tm_packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.packed, a.K / 2, total_w_rows, a.K / 2,
+                   S::HALVES * 64, 64, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  if (!make_map_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dy, a.N, dy_rows, lddy * 2, 64, S::BN,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  const int esize = a.out_bf16 ? 2 : 4;
+  if (!make_map_2d(&tm_out, a.out_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.out,
+                   a.K, a.total_rows, static_cast<uint64_t>(a.K) * esize, kBM, kChunk, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  TcParams p{};
+  p.offsets = a.offsets;
+  p.E = a.E;
+  p.total_rows = a.total_rows;
+  p.absmax = a.absmax;
+  p.N = a.K;  // tile rows: columns k of W
+  p.K = a.N;  // K steps: rows n of W
+  p.swiglu = 0;
+  p.out = a.out;
+  p.out_bf16 = a.out_bf16;
+  p.out_cols = a.K;
+  p.lora_B = nullptr;
+  p.r = 0;
+  p.n_tiles = (a.K + S::HALVES * kBM - 1) / (S::HALVES * kBM);
+  p.err = err_word;
+  const int64_t tiles =
+      ((a.total_rows + S::BN - 1) / S::BN + (a.E < a.total_rows ? a.E : a.total_rows)) * p.n_tiles;
+  const int grid = static_cast<int>(tiles < di.sm_count ? tiles : di.sm_count);
+  LaunchScope ls("dgrad.tc", stream);
+  grouped_nf4_tc_kernel<S, true><<<grid, kThreadsTc, S::kSmemBytes, stream>>>(tm_packed, tm_b, tm_out, tm_b, p);
   return cudaGetLastError();
 }
 
@@ -756,6 +897,21 @@ cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int* err_word, cudaStream_
   if (s == 1) return launch_shape<ShapeWide>(a, err_word, stream);
   if (s == 2) return launch_shape<ShapeDouble>(a, err_word, stream);
   return launch_shape<ShapeNarrow>(a, err_word, stream);
+}
+
+bool dgrad_tc_supported(const DgradArgs& a, int64_t lddy) {
+  return tensor_maps_available() && lddy % 8 == 0 && (a.lora_A == nullptr || !a.out_bf16);
+}
+
+cudaError_t launch_grouped_dgrad_tc(const DgradArgs& a, const uint16_t* dy, int64_t dy_rows, int64_t lddy,
+                                    int* err_word, cudaStream_t stream) {
+  // Groups of 512 rows and more fill the 256-row tile; smaller ones waste less
+  // with 128 routed rows and two accumulator sets.
+  const int64_t rows_per_group = a.total_rows / (a.E > 0 ? a.E : 1);
+  int s = shape_override();
+  if (s != 1 && s != 2) s = rows_per_group >= 512 ? 1 : 2;
+  if (s == 1) return launch_dgrad_shape<ShapeWide>(a, dy, dy_rows, lddy, err_word, stream);
+  return launch_dgrad_shape<ShapeDouble>(a, dy, dy_rows, lddy, err_word, stream);
 }
 
 cudaError_t launch_tc_lora_prep(const GemmArgs& a, cudaStream_t stream) {

@@ -35,8 +35,11 @@ EXPORTED = (
     "e4b_nf4_quantize_stack",
     "e4b_moe_route_permute_workspace_size", "e4b_moe_route_permute",
     "e4b_grouped_nf4_gemm_workspace_size", "e4b_grouped_nf4_gemm",
+    "e4b_grouped_nf4_gemm_dgrad_workspace_size", "e4b_grouped_nf4_gemm_dgrad",
+    "e4b_grouped_lora_grads_workspace_size", "e4b_grouped_lora_grads",
     "e4b_moe_expert_forward_workspace_size", "e4b_moe_expert_forward",
     "e4b_moe_expert_forward_path", "e4b_moe_expert_forward_decode_noalloc",
+    "e4b_moe_expert_backward_workspace_size", "e4b_moe_expert_backward",
 )
 
 
@@ -96,6 +99,16 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.e4b_grouped_nf4_gemm.restype = i32
     lib.e4b_grouped_nf4_gemm.argtypes = [vp, i64, i64, vp, vp, i64, i64, vp, vp, i64, i64, vp, vp, i32,
                                          ctypes.c_float, i32, vp, i32, vp, sz, vp]
+    lib.e4b_grouped_nf4_gemm_dgrad_workspace_size.restype = sz
+    lib.e4b_grouped_nf4_gemm_dgrad_workspace_size.argtypes = [i64, i64, i64, i32]
+    lib.e4b_grouped_nf4_gemm_dgrad.restype = i32
+    lib.e4b_grouped_nf4_gemm_dgrad.argtypes = [vp, i64, i64, vp, vp, i64, i64, vp, vp, i64, i64, vp, vp, i32,
+                                               ctypes.c_float, vp, i32, vp, sz, vp]
+    lib.e4b_grouped_lora_grads_workspace_size.restype = sz
+    lib.e4b_grouped_lora_grads_workspace_size.argtypes = [i64, i32]
+    lib.e4b_grouped_lora_grads.restype = i32
+    lib.e4b_grouped_lora_grads.argtypes = [vp, i64, i64, vp, vp, i64, i64, vp, i64, i64, i64, vp, vp, i32,
+                                           ctypes.c_float, vp, vp, vp, sz, vp]
     lib.e4b_moe_expert_forward_workspace_size.restype = sz
     lib.e4b_moe_expert_forward_workspace_size.argtypes = [i64, ctypes.POINTER(ExpertStackC), i32]
     lib.e4b_moe_expert_forward.restype = i32
@@ -107,6 +120,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.e4b_workspace_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
     lib.e4b_workspace_clear_error.restype = i32
     lib.e4b_workspace_clear_error.argtypes = [vp, vp]
+    lib.e4b_moe_expert_backward_workspace_size.restype = sz
+    lib.e4b_moe_expert_backward_workspace_size.argtypes = [i64, ctypes.POINTER(ExpertStackC), i32]
+    lib.e4b_moe_expert_backward.restype = i32
+    lib.e4b_moe_expert_backward.argtypes = [vp, i64, vp, i32, i32, ctypes.POINTER(ExpertStackC), vp, vp, vp, vp,
+                                            vp, vp, sz, vp]
     lib.e4b_moe_expert_forward_path.restype = i32
     lib.e4b_moe_expert_forward_path.argtypes = [vp, i64, vp, i32, i32, ctypes.POINTER(ExpertStackC), vp, vp,
                                                 sz, i32, vp]
@@ -240,6 +258,72 @@ def e4b_grouped_nf4_gemm(A: torch.Tensor, row_index: Optional[torch.Tensor], exp
         out.data_ptr(), od, _ptr(workspace), ws, _stream(stream)), "e4b_grouped_nf4_gemm")
 
 
+def e4b_grouped_nf4_gemm_dgrad_workspace_size(total_rows: int, N: int, K: int, r: int = 0) -> int:
+    return int(load_library().e4b_grouped_nf4_gemm_dgrad_workspace_size(total_rows, N, K, r))
+
+
+def e4b_grouped_nf4_gemm_dgrad(dY: torch.Tensor, row_index: Optional[torch.Tensor], expert_offsets: torch.Tensor,
+                               total_rows: int, packed: torch.Tensor, absmax: torch.Tensor, N: int, K: int,
+                               out: torch.Tensor, lora_A: Optional[torch.Tensor] = None,
+                               lora_B: Optional[torch.Tensor] = None, lora_scale: float = 0.0,
+                               workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """out[p] = dY[row_index[p]] . W_e (+ lora_scale * (dY . lora_B[e]) . lora_A[e]), [total_rows, K]."""
+    if dY.dim() != 2 or dY.dtype != torch.bfloat16 or not dY.is_cuda or dY.stride(1) != 1:
+        raise ValueError("dY must be a 2-D bf16 CUDA tensor with unit column stride")
+    _dev(expert_offsets, "expert_offsets", torch.int32)
+    _dev(packed, "packed", torch.uint8)
+    _dev(absmax, "absmax", torch.float32)
+    _dev(out, "out")
+    if row_index is not None:
+        _dev(row_index, "row_index", torch.int32)
+    E = expert_offsets.numel() - 1
+    r = 0
+    if lora_A is not None:
+        _dev(lora_A, "lora_A", torch.bfloat16)
+        _dev(lora_B, "lora_B", torch.bfloat16)
+        r = lora_A.shape[1]
+    od = {torch.float32: E4B_F32, torch.bfloat16: E4B_BF16}.get(out.dtype)
+    if od is None:
+        raise ValueError("out must be float32 or bfloat16")
+    if out.numel() < total_rows * K:
+        raise ValueError("out too small")
+    ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load_library().e4b_grouped_nf4_gemm_dgrad(
+        dY.data_ptr(), dY.shape[0], dY.stride(0), _ptr(row_index), expert_offsets.data_ptr(), E, total_rows,
+        packed.data_ptr(), absmax.data_ptr(), N, K, _ptr(lora_A), _ptr(lora_B), r, float(lora_scale),
+        out.data_ptr(), od, _ptr(workspace), ws, _stream(stream)), "e4b_grouped_nf4_gemm_dgrad")
+
+
+def e4b_grouped_lora_grads_workspace_size(total_rows: int, r: int) -> int:
+    return int(load_library().e4b_grouped_lora_grads_workspace_size(total_rows, r))
+
+
+def e4b_grouped_lora_grads(x: torch.Tensor, row_index: Optional[torch.Tensor], expert_offsets: torch.Tensor,
+                           total_rows: int, da: torch.Tensor, N: int, K: int, lora_A: torch.Tensor,
+                           lora_B: torch.Tensor, lora_scale: float, dA: torch.Tensor, dB: torch.Tensor,
+                           workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """dA [E, r, K], dB [E, N, r] (fp32) of one grouped projection's adapter."""
+    for t, n in ((x, "x"), (da, "da")):
+        if t.dim() != 2 or t.dtype != torch.bfloat16 or not t.is_cuda or t.stride(1) != 1:
+            raise ValueError(f"{n} must be a 2-D bf16 CUDA tensor with unit column stride")
+    _dev(expert_offsets, "expert_offsets", torch.int32)
+    _dev(lora_A, "lora_A", torch.bfloat16)
+    _dev(lora_B, "lora_B", torch.bfloat16)
+    _dev(dA, "dA", torch.float32)
+    _dev(dB, "dB", torch.float32)
+    if row_index is not None:
+        _dev(row_index, "row_index", torch.int32)
+    E = expert_offsets.numel() - 1
+    r = lora_A.shape[1]
+    if dA.numel() < E * r * K or dB.numel() < E * N * r:
+        raise ValueError("dA/dB too small")
+    ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load_library().e4b_grouped_lora_grads(
+        x.data_ptr(), x.shape[0], x.stride(0), _ptr(row_index), expert_offsets.data_ptr(), E, total_rows,
+        da.data_ptr(), da.stride(0), N, K, lora_A.data_ptr(), lora_B.data_ptr(), r, float(lora_scale),
+        dA.data_ptr(), dB.data_ptr(), _ptr(workspace), ws, _stream(stream)), "e4b_grouped_lora_grads")
+
+
 class ExpertStack:
     """Device tensors of one MoE layer's packed stacks (and optional adapter)."""
 
@@ -282,6 +366,35 @@ def e4b_moe_expert_forward(x: torch.Tensor, router_logits: torch.Tensor, k: int,
     _check(load_library().e4b_moe_expert_forward_path(
         x.data_ptr(), M, router_logits.data_ptr(), k, int(bool(renormalize)), ctypes.byref(stack.c),
         out.data_ptr(), _ptr(workspace), ws, path, _stream(stream)), "e4b_moe_expert_forward")
+
+
+def e4b_moe_expert_backward_workspace_size(M: int, stack: "ExpertStack", k: int) -> int:
+    return int(load_library().e4b_moe_expert_backward_workspace_size(M, ctypes.byref(stack.c), k))
+
+
+def e4b_moe_expert_backward(x: torch.Tensor, router_logits: torch.Tensor, k: int, renormalize: bool,
+                            stack: "ExpertStack", dout: torch.Tensor, dx: torch.Tensor, dlogits: torch.Tensor,
+                            dA: Optional[torch.Tensor], dB: Optional[torch.Tensor], workspace: Optional[torch.Tensor],
+                            stream=None) -> None:
+    """Gradients of sum(dout * forward(x, router_logits)): dx [M, H], dlogits [M, E] and, with an
+    adapter, dA [E, r, H], dB [E, 2I, r] (all fp32); routing ids held fixed (see include/e4b.h)."""
+    _dev(x, "x", torch.bfloat16)
+    _dev(router_logits, "router_logits", torch.float32)
+    _dev(dout, "dout", torch.bfloat16)
+    _dev(dx, "dx", torch.float32)
+    _dev(dlogits, "dlogits", torch.float32)
+    M = x.shape[0]
+    if (x.shape[1] != stack.H or router_logits.shape != (M, stack.E) or dout.shape != (M, stack.H)
+            or dx.shape != (M, stack.H) or dlogits.shape != (M, stack.E)):
+        raise ValueError("x, dout, dx [M, H] and router_logits, dlogits [M, E] required")
+    for t, n in ((dA, "dA"), (dB, "dB")):
+        if t is not None:
+            _dev(t, n, torch.float32)
+    ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load_library().e4b_moe_expert_backward(
+        x.data_ptr(), M, router_logits.data_ptr(), k, int(bool(renormalize)), ctypes.byref(stack.c),
+        dout.data_ptr(), dx.data_ptr(), dlogits.data_ptr(), _ptr(dA), _ptr(dB), _ptr(workspace), ws,
+        _stream(stream)), "e4b_moe_expert_backward")
 
 
 def e4b_moe_expert_forward_decode_noalloc(x: torch.Tensor, router_logits: torch.Tensor, k: int, renormalize: bool,

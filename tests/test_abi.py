@@ -144,3 +144,73 @@ def test_error_word_calls_check_their_arguments_on_the_host(lib):
     assert lib.e4b_workspace_clear_error(None, None) == 1
     assert code.value == 7   # untouched on a rejected call
 
+
+
+def test_dgrad_host_side_rejections(lib):
+    """The grouped dgrad checks its arguments before any device query."""
+    p = ctypes.c_void_p(1 << 20)
+    rows, N, K = 64, 128, 192
+    need = e4b.e4b_grouped_nf4_gemm_dgrad_workspace_size(rows, N, K, 0)
+    # error word, then (with an adapter) dY . lora_B, then room for the dY rows gathered in group order
+    assert need == 256 + rows * N * 2
+    assert e4b.e4b_grouped_nf4_gemm_dgrad_workspace_size(rows, N, K, 8) == \
+        256 + (rows * 8 * 4 + 255) // 256 * 256 + rows * N * 2
+
+    def call(**kw):
+        a = dict(dY=p, dy_rows=rows, lddy=N, ridx=None, offs=p, E=2, rows=rows, packed=p, absmax=p, N=N, K=K,
+                 la=None, lb=None, r=0, scale=0.0, out=p, od=0, ws=p, wsb=need)
+        a.update(kw)
+        return lib.e4b_grouped_nf4_gemm_dgrad(a["dY"], a["dy_rows"], a["lddy"], a["ridx"], a["offs"], a["E"],
+                                              a["rows"], a["packed"], a["absmax"], a["N"], a["K"], a["la"],
+                                              a["lb"], a["r"], a["scale"], a["out"], a["od"], a["ws"], a["wsb"],
+                                              None)
+    assert call(K=96) == 2 and b"K must be" in lib.e4b_last_error()
+    assert call(N=100) == 2 and b"N must be" in lib.e4b_last_error()
+    assert call(lddy=N - 8) == 1 and b"lddy" in lib.e4b_last_error()
+    assert call(lddy=N + 4) == 1 and b"lddy" in lib.e4b_last_error()
+    assert call(la=p) == 1 and b"both set" in lib.e4b_last_error()
+    assert call(la=p, lb=p, r=17) == 2 and b"rank" in lib.e4b_last_error()
+    assert call(absmax=ctypes.c_void_p((1 << 20) + 4)) == 1 and b"16-byte aligned" in lib.e4b_last_error()
+    assert call(wsb=need - 1) == 3 and str(need).encode() in lib.e4b_last_error()
+    assert call(ws=ctypes.c_void_p((1 << 20) + 8)) == 1 and b"dgrad workspace must be" in lib.e4b_last_error()
+
+
+def test_lora_grads_host_side_rejections(lib):
+    p = ctypes.c_void_p(1 << 20)
+    rows, N, K, r = 64, 128, 192, 8
+    need = e4b.e4b_grouped_lora_grads_workspace_size(rows, r)
+    assert need == 256 + 2 * ((rows * r * 4 + 255) // 256 * 256)
+    assert e4b.e4b_grouped_lora_grads_workspace_size(rows, 0) == 0
+
+    def call(**kw):
+        a = dict(x=p, x_rows=rows, ldx=K, ridx=None, offs=p, E=2, rows=rows, da=p, ldda=N, N=N, K=K, la=p, lb=p,
+                 r=r, scale=1.0, dA=p, dB=p, ws=p, wsb=need)
+        a.update(kw)
+        return lib.e4b_grouped_lora_grads(a["x"], a["x_rows"], a["ldx"], a["ridx"], a["offs"], a["E"], a["rows"],
+                                          a["da"], a["ldda"], a["N"], a["K"], a["la"], a["lb"], a["r"], a["scale"],
+                                          a["dA"], a["dB"], a["ws"], a["wsb"], None)
+    assert call(r=0) == 2 and b"rank" in lib.e4b_last_error()
+    assert call(K=100) == 2 and b"K must be" in lib.e4b_last_error()
+    assert call(ldx=K + 4) == 1 and b"ldx" in lib.e4b_last_error()
+    assert call(ldda=N - 1) == 1 and b"ldda" in lib.e4b_last_error()
+    assert call(dB=None) == 1 and b"null" in lib.e4b_last_error()
+    assert call(wsb=need - 1) == 3 and str(need).encode() in lib.e4b_last_error()
+
+
+def test_backward_host_side_checks(lib):
+    p = 1 << 20
+    st = e4b.ExpertStackC(p, p, p, p, None, None, 0, 0.0, 8, 256, 128)
+    sizes = [lib.e4b_moe_expert_backward_workspace_size(M, ctypes.byref(st), 2) for M in (1, 64, 300)]
+    assert sizes[0] < sizes[1] < sizes[2]
+    # per routed row at least a (fp32 2I), z and dxg (fp32 H each), dz (bf16 H), dh (fp32 I), da (bf16 2I)
+    assert sizes[2] >= 600 * (8 * 128 + 4 * 256 * 2 + 2 * 256 + 4 * 128 + 4 * 128)
+    assert lib.e4b_moe_expert_backward_workspace_size(0, ctypes.byref(st), 2) == 0
+    vp = ctypes.c_void_p(p)
+    need = sizes[1]
+    status = lib.e4b_moe_expert_backward(vp, 64, vp, 2, 1, ctypes.byref(st), vp, vp, vp, None, None, vp, need - 1,
+                                         None)
+    assert status == 3 and str(need).encode() in lib.e4b_last_error()
+    stl = e4b.ExpertStackC(p, p, p, p, p, p, 8, 16.0, 8, 256, 128)
+    status = lib.e4b_moe_expert_backward(vp, 64, vp, 2, 1, ctypes.byref(stl), vp, vp, vp, None, None, vp, 1 << 40,
+                                         None)
+    assert status == 1 and b"needs dA and dB" in lib.e4b_last_error()
