@@ -71,7 +71,7 @@ struct TcShape {
   static constexpr bool ATMEM = ATMEM_;
   static constexpr int kRows = HALVES * kBM;        // weight rows per tile
   static constexpr int kTpr = kDecThreads / kRows;  // decoder threads per weight row
-  [[maybe_unused]] static constexpr int kChunks = 8 / kTpr;          // 16-byte decoded chunks per thread per k block
+  static constexpr int kChunks = 8 / kTpr;          // 16-byte decoded chunks per thread per k block
   static constexpr uint32_t kPackedBytes = HALVES * kPackedHalfBytes;
   static constexpr uint32_t kBBytes = BN * 128;
   static constexpr uint32_t kTmaStageBytes = kPackedBytes + kBBytes;
@@ -82,7 +82,7 @@ struct TcShape {
   static constexpr int kKS = kKSFit < 6 ? kKSFit : 6;
   static constexpr uint32_t kCols = HALVES * BN;    // TMEM columns of one accumulator set
   static constexpr uint32_t kACols = HALVES * 32;   // TMEM columns of one A stage (ATMEM): 64 k as bf16 pairs
-  [[maybe_unused]] static constexpr uint32_t kAColBase = kCols * NACC;
+  static constexpr uint32_t kAColBase = kCols * NACC;
   static constexpr uint32_t kOffTma = 0;
   static constexpr uint32_t kOffA = kOffTma + kKS * kTmaStageBytes;
   static constexpr uint32_t kOffOut = kOffA + kAS * kAStageBytes;
@@ -94,6 +94,7 @@ struct TcShape {
   static_assert(kKS >= 2, "ring depth");
   static_assert(kCols * NACC + (ATMEM ? kAS * kACols : 0) <= 512, "TMEM columns");
   static_assert(!ATMEM || HALVES == 2, "the TMEM decoders cover two halves");
+  static_assert(kChunks >= 1 && kAColBase <= 512, "decoder chunks, TMEM A base");
   static_assert(BN % 16 == 0 && BN <= 256, "MMA N");
   static_assert(kSmemBytes <= kSmemLimit, "shared memory");
 };
