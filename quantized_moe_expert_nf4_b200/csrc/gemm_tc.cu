@@ -62,9 +62,13 @@ constexpr uint32_t kSmemMisc = 1024 + 512;       // alignment slack, barriers, T
 constexpr int kLoraCols = 64;                    // width of a row of scale * x . lora_A^T (bf16, zero past r)
 constexpr size_t kLoraPrepSmemMax = 192 * 1024;  // lora_A[e] staged by the prep kernel
 
-template <int BN_, int HALVES_, int NACC_>
+// ATMEM: the decoders write the decoded weight tile into tensor memory
+// (tcgen05.st) and the MMA reads A from there, so the tile never passes
+// through shared memory; the A stages take TMEM columns after the accumulators.
+template <int BN_, int HALVES_, int NACC_, bool ATMEM_ = false>
 struct TcShape {
   static constexpr int BN = BN_, HALVES = HALVES_, NACC = NACC_;
+  static constexpr bool ATMEM = ATMEM_;
   static constexpr int kRows = HALVES * kBM;        // weight rows per tile
   static constexpr int kTpr = kDecThreads / kRows;  // decoder threads per weight row
   static constexpr int kChunks = 8 / kTpr;          // 16-byte decoded chunks per thread per k block
@@ -72,11 +76,13 @@ struct TcShape {
   static constexpr uint32_t kBBytes = BN * 128;
   static constexpr uint32_t kTmaStageBytes = kPackedBytes + kBBytes;
   static constexpr int kAS = 2;
-  static constexpr uint32_t kAStageBytes = HALVES * kAHalfBytes;
+  static constexpr uint32_t kAStageBytes = ATMEM ? 0 : HALVES * kAHalfBytes;
   static constexpr int kKSFit =
       static_cast<int>((kSmemLimit - kSmemMisc - kOutBytes - kAS * kAStageBytes) / kTmaStageBytes);
   static constexpr int kKS = kKSFit < 6 ? kKSFit : 6;
   static constexpr uint32_t kCols = HALVES * BN;    // TMEM columns of one accumulator set
+  static constexpr uint32_t kACols = HALVES * 32;   // TMEM columns of one A stage (ATMEM): 64 k as bf16 pairs
+  static constexpr uint32_t kAColBase = kCols * NACC;
   static constexpr uint32_t kOffTma = 0;
   static constexpr uint32_t kOffA = kOffTma + kKS * kTmaStageBytes;
   static constexpr uint32_t kOffOut = kOffA + kAS * kAStageBytes;
@@ -86,7 +92,9 @@ struct TcShape {
   static constexpr uint32_t kSmemBytes = kOffTmemSlot + 16 + 1024;
   static_assert(kTpr == 2 || kTpr == 4, "decoder split");
   static_assert(kKS >= 2, "ring depth");
-  static_assert(kCols * NACC <= 512, "TMEM columns");
+  static_assert(kCols * NACC + (ATMEM ? kAS * kACols : 0) <= 512, "TMEM columns");
+  static_assert(!ATMEM || HALVES == 2, "the TMEM decoders cover two halves");
+  static_assert(kChunks >= 1 && kAColBase <= 512, "decoder chunks, TMEM A base");
   static_assert(BN % 16 == 0 && BN <= 256, "MMA N");
   static_assert(kSmemBytes <= kSmemLimit, "shared memory");
 };
@@ -164,6 +172,77 @@ __device__ __forceinline__ bool locate(const TcParams& p, int64_t t, int* e, int
   *re = b1;
   *n_tile = static_cast<int>(t % p.n_tiles);
   return true;
+}
+
+// Decoders of the TMEM-operand shape.  A warp may only reach the 32 TMEM lanes
+// of its quadrant (warp % 4), so warp w takes weight rows 32 (w % 4) + lane of
+// one half, and the four warps of a quadrant split (half, 32-k part); a thread
+// decodes its row's 32 k of the step into 16 bf16 pairs and stores them as 16
+// consecutive TMEM columns of its lane.
+template <class S>
+__device__ __forceinline__ void tmem_decoders(const TcParams& p, unsigned char* smem, uint64_t* tma_full,
+                                              uint64_t* a_empty, uint64_t* a_full, uint32_t tmem_base, int warp,
+                                              int lane) {
+  constexpr int BN = S::BN, KS = S::kKS, AS = S::kAS;
+  const int qd = warp & 3, c = (warp - kWarpDec) >> 2;
+  const int half = c >> 1, kpart = c & 1;
+  const int ri = qd * 32 + lane;
+  const int KB = p.K / 64;
+  const CodebookBytes cbt = codebook_bytes();
+  uint32_t kbg = 0;
+  bool ok = true;
+  for (int64_t t = blockIdx.x; ok; t += gridDim.x) {
+    int e, n_tile;
+    int64_t rb, re;
+    if (!locate<BN>(p, t, &e, &rb, &re, &n_tile)) break;
+    int r0, r1;
+    tile_rows<S::HALVES>(p, n_tile, &r0, &r1);
+    const int n = (half ? r1 : r0) + ri;
+    const bool valid = n < p.N;
+    const float* am = p.absmax + (static_cast<int64_t>(e) * p.N + (valid ? n : 0)) * KB;
+    float sc_ring[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sc_ring[i] = (valid && i < KB) ? __ldg(am + i) : 0.0f;
+    for (int kb0 = 0; kb0 < KB && ok; kb0 += 4) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int kb = kb0 + i;
+        if (kb >= KB) break;
+        const float sc = sc_ring[i];
+        sc_ring[i] = (valid && kb + 4 < KB) ? __ldg(am + kb + 4) : 0.0f;
+        const int s = kbg % KS, a = kbg % AS;
+        if (!mbar_wait(&tma_full[s], (kbg / KS) & 1) ||
+            (kbg >= AS && !mbar_wait(&a_empty[a], ((kbg / AS) - 1) & 1))) {
+          record_error(p.err, kErrWaitFull);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint4 q = *reinterpret_cast<const uint4*>(smem + S::kOffTma + s * S::kTmaStageBytes +
+                                                        half * kPackedHalfBytes + ri * 32 + kpart * 16);
+        const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+        const __nv_bfloat162 s2 = __float2bfloat162_rn(sc);
+        uint32_t v[16];
+#pragma unroll
+        for (int cw = 0; cw < 4; ++cw) {
+          decode4(words[cw], cbt, &v[4 * cw], &v[4 * cw + 1]);
+          decode4(words[cw] >> 16, cbt, &v[4 * cw + 2], &v[4 * cw + 3]);
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          __nv_bfloat162 h2 = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&v[i]), s2);
+          v[i] = *reinterpret_cast<uint32_t*>(&h2);
+        }
+        tmem_st_32x32b_x16(
+            tmem_base + (static_cast<uint32_t>(qd * 32) << 16) + S::kAColBase + a * S::kACols + half * 32 + kpart * 16, v);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_full[a]);
+        ++kbg;
+      }
+    }
+  }
 }
 
 // Decoders of the dgrad product.  Thread dt takes rows n in [8o, 8o + 8) of the
@@ -384,8 +463,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             const uint32_t acc = (kb | kk) ? 1u : 0u;
             const uint64_t bd = smem_desc_sw128(b_addr + kk * 32);
 #pragma unroll
-            for (int h = 0; h < HALVES; ++h)
-              umma_bf16(d + h * BN, smem_desc_sw128(a_addr + h * kAHalfBytes + kk * 32), bd, idesc, acc);
+            for (int h = 0; h < HALVES; ++h) {
+              if constexpr (S::ATMEM)
+                umma_bf16_ts(d + h * BN, tmem_base + S::kAColBase + a * S::kACols + h * 32 + kk * 8, bd, idesc, acc);
+              else
+                umma_bf16(d + h * BN, smem_desc_sw128(a_addr + h * kAHalfBytes + kk * 32), bd, idesc, acc);
+            }
           }
           umma_commit(&tma_empty[s]);
           umma_commit(&a_empty[a]);
@@ -419,6 +502,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     }
   } else if (warp >= kWarpDec && warp < kWarpDec + kNumDecWarps) {
     // ------------------------------------------------------------- decoders
+    if constexpr (S::ATMEM) {
+      tmem_decoders<S>(p, smem, tma_full, a_empty, a_full, tmem_base, warp, lane);
+    } else {
     const int dt = tid - kWarpDec * 32;            // 0..511
     if constexpr (DG) {
       dgrad_decoders<S>(p, smem, tma_full, a_empty, a_full, dt, lane);
@@ -821,6 +907,7 @@ __global__ void __launch_bounds__(256) lora_prep_kernel(PrepParams q) {
 using ShapeWide = TcShape<256, 2, 1>;    // 2 x 128 weight rows x 256 routed rows, one accumulator set
 using ShapeDouble = TcShape<128, 2, 2>;  // 2 x 128 x 128, two accumulator sets
 using ShapeNarrow = TcShape<256, 1, 2>;  // 128 x 256, two accumulator sets (no SwiGLU)
+using ShapeTmem = TcShape<192, 2, 1, true>;  // 2 x 128 x 192, A in TMEM (no LoRA step)
 
 int shape_override() {
   const char* v = getenv("E4B_TC_SHAPE");
@@ -828,6 +915,7 @@ int shape_override() {
   if (!strcmp(v, "wide")) return 1;
   if (!strcmp(v, "double")) return 2;
   if (!strcmp(v, "narrow")) return 3;
+  if (!strcmp(v, "tmem")) return 4;
   return 0;
 }
 
@@ -894,6 +982,8 @@ cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int* err_word, cudaStream_
     const int64_t rows_per_group = a.total_rows / (a.E > 0 ? a.E : 1);
     s = swiglu ? 1 : (rows_per_group >= 512 ? 1 : 3);
   }
+  if (s == 4 && !(a.lora_B && a.r > 0)) return launch_shape<ShapeTmem>(a, err_word, stream);
+  if (s == 4) s = swiglu ? 1 : 3;
   if (s == 1) return launch_shape<ShapeWide>(a, err_word, stream);
   if (s == 2) return launch_shape<ShapeDouble>(a, err_word, stream);
   return launch_shape<ShapeNarrow>(a, err_word, stream);

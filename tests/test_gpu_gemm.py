@@ -145,7 +145,7 @@ def test_grouped_gemm_positive_control_flipped_nibble():
 # wide = 2 x 128 weight rows x 256 routed rows, double = 2 x 128 x 128 with two
 # accumulator sets, narrow = 128 x 256 with two accumulator sets (plain
 # epilogue only; a SwiGLU call takes the wide shape).
-TC_SHAPES = ["wide", "double", "narrow"]
+TC_SHAPES = ["wide", "double", "narrow", "tmem"]
 TC_CASES = CASES + [
     # several 256-row token tiles per group and a one-row group
     (3, 256, 512, [700, 1, 300], 500),
