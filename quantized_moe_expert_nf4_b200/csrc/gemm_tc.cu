@@ -611,6 +611,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       }
     }
     }
+    }
   } else if (warp < 4) {
     // ------------------------------------------------------------- epilogue
     const int q = warp;  // TMEM lane quadrant = output columns 32q .. 32q + 31 of a part
