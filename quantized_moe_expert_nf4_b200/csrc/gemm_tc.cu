@@ -824,10 +824,10 @@ cudaError_t launch_dgrad_shape(const DgradArgs& a, const uint16_t* dy, int64_t d
 }
 
 // LoRA prep for the tensor-core kernel: one CTA per (group, 64-row tile),
-// lora_A[e] (r x K bf16) staged in shared memory, one warp per routed row.
-// The warp copies the row into `gathered` (when a row index is given) and
-// writes xa[p, 0:64] = bf16(scale * A_row . lora_A[e, j]) for j < r, zeros
-// after -- the B operand of the kernel's extra K=16 MMA step.
+// lora_A[e] staged in shared memory.  It copies the tile's routed rows into
+// `gathered` (when a row index is given) and writes xa[p, 0:64] =
+// bf16(scale * A_row . lora_A[e, j]) for j < r, zeros after -- the B operand
+// of the GEMM kernel's extra K=16 MMA step.
 struct PrepParams {
   const uint16_t* A;
   int64_t a_rows, lda;
@@ -844,17 +844,35 @@ struct PrepParams {
 };
 
 constexpr int kPrepRows = 64;
+constexpr int kPrepUnroll = 4;  // 32-k chunks of the two rows' loads in flight per lane
 
-__global__ void __launch_bounds__(256) lora_prep_kernel(PrepParams q) {
-  extern __shared__ __align__(16) uint16_t la_s[];  // [r, K]
+__device__ __forceinline__ void mma_bf16_16816(float c[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Warp w takes routed rows 16w .. 16w + 15 of the tile as the rows of an
+// m16n8k16 MMA and the adapter rows (16, zero past r) as its columns; lane
+// (g, t) loads physical k [8t, 8t + 8) of each 32-k chunk of rows g and g + 8
+// as one 16-byte vector -- the A fragments of two MMAs, with K permuted the
+// same way for lora_A (rows g and g + 8 of its staged copy) -- and stores the
+// same vectors into `gathered`.  The loads are HBM-bound; the products cost a
+// few MMAs per 1 KB read.
+__global__ void __launch_bounds__(128) lora_prep_kernel(PrepParams q) {
+  extern __shared__ __align__(16) uint16_t la_s[];  // [16, K + 8]: lora_A[e], rows past r zero
   __shared__ int64_t tile_s[3];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
   if (warp == 0) {
-    int g;
+    int ge;
     int64_t b0, b1;
-    const bool found = find_group_tile(q.offsets, q.E, q.total_rows, kPrepRows, blockIdx.x, &g, &b0, &b1);
+    const bool found = find_group_tile(q.offsets, q.E, q.total_rows, kPrepRows, blockIdx.x, &ge, &b0, &b1);
     if (lane == 0) {
-      tile_s[0] = found ? g : -1;
+      tile_s[0] = found ? ge : -1;
       tile_s[1] = b0;
       tile_s[2] = b1;
     }
@@ -863,45 +881,66 @@ __global__ void __launch_bounds__(256) lora_prep_kernel(PrepParams q) {
   const int e = static_cast<int>(tile_s[0]);
   if (e < 0) return;
   const int64_t rb = tile_s[1], re = tile_s[2];
-  const int K = q.K, kv = K / 8;
+  const int K = q.K, kv = K / 8, ls = K + 8;  // shared row stride (bf16): 16 bytes of padding per row
   const uint4* src_a = reinterpret_cast<const uint4*>(q.lora_A + static_cast<int64_t>(e) * q.r * K);
-  for (int i = threadIdx.x; i < q.r * kv; i += blockDim.x) reinterpret_cast<uint4*>(la_s)[i] = src_a[i];
+  for (int i = threadIdx.x; i < 16 * kv; i += blockDim.x) {
+    const int row = i / kv, c = i % kv;
+    reinterpret_cast<uint4*>(la_s + row * ls)[c] = row < q.r ? src_a[row * kv + c] : make_uint4(0, 0, 0, 0);
+  }
   __syncthreads();
-  for (int64_t pr = rb + warp; pr < re; pr += blockDim.x / 32) {
-    int64_t src = q.row_index ? q.row_index[pr] : pr;
-    src = clampv<int64_t>(src, 0, q.a_rows - 1);
-    const uint4* xrow = reinterpret_cast<const uint4*>(q.A + src * q.lda);
-    uint4* grow = q.gathered ? reinterpret_cast<uint4*>(q.gathered + pr * K) : nullptr;
-    float acc[16];
+  const int64_t p0 = rb + 16 * warp + g, p1 = p0 + 8;
+  const bool v0 = p0 < re, v1 = p1 < re;
+  int64_t s0 = v0 ? (q.row_index ? q.row_index[p0] : p0) : 0;
+  int64_t s1 = v1 ? (q.row_index ? q.row_index[p1] : p1) : 0;
+  s0 = clampv<int64_t>(s0, 0, q.a_rows - 1);
+  s1 = clampv<int64_t>(s1, 0, q.a_rows - 1);
+  const uint4* x0 = reinterpret_cast<const uint4*>(q.A + s0 * q.lda);
+  const uint4* x1 = reinterpret_cast<const uint4*>(q.A + s1 * q.lda);
+  uint4* g0 = (q.gathered && v0) ? reinterpret_cast<uint4*>(q.gathered + p0 * K) : nullptr;
+  uint4* g1 = (q.gathered && v1) ? reinterpret_cast<uint4*>(q.gathered + p1 * K) : nullptr;
+  const bool two = q.r > 8;  // adapter rows 8..15 need the second n tile
+  float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+  const int nchunks = K / 32;
+  for (int ch0 = 0; ch0 < nchunks; ch0 += kPrepUnroll) {
+    uint4 xa0[kPrepUnroll], xa1[kPrepUnroll];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) acc[j] = 0.f;
-    for (int c = lane; c < kv; c += 32) {
-      const uint4 xv = __ldg(xrow + c);
-      if (grow) grow[c] = xv;
-      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+    for (int u = 0; u < kPrepUnroll; ++u) {
+      const int c = (ch0 + u) * 4 + t;  // 16-byte vector index within the row
+      const bool in = ch0 + u < nchunks;
+      xa0[u] = (in && v0) ? __ldg(x0 + c) : make_uint4(0, 0, 0, 0);
+      xa1[u] = (in && v1) ? __ldg(x1 + c) : make_uint4(0, 0, 0, 0);
+    }
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        if (j >= q.r) break;
-        const uint4 av = reinterpret_cast<const uint4*>(la_s + j * K)[c];
-        const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          acc[j] = fmaf(__uint_as_float(xw[i] << 16), __uint_as_float(aw[i] << 16), acc[j]);
-          acc[j] = fmaf(__uint_as_float(xw[i] & 0xffff0000u), __uint_as_float(aw[i] & 0xffff0000u), acc[j]);
-        }
+    for (int u = 0; u < kPrepUnroll; ++u) {
+      if (ch0 + u >= nchunks) break;
+      const int c = (ch0 + u) * 4 + t;
+      if (g0) g0[c] = xa0[u];
+      if (g1) g1[c] = xa1[u];
+      const uint4 b = reinterpret_cast<const uint4*>(la_s + g * ls)[c];
+      mma_bf16_16816(c0, xa0[u].x, xa1[u].x, xa0[u].y, xa1[u].y, b.x, b.y);
+      mma_bf16_16816(c0, xa0[u].z, xa1[u].z, xa0[u].w, xa1[u].w, b.z, b.w);
+      if (two) {
+        const uint4 b2 = reinterpret_cast<const uint4*>(la_s + (g + 8) * ls)[c];
+        mma_bf16_16816(c1, xa0[u].x, xa1[u].x, xa0[u].y, xa1[u].y, b2.x, b2.y);
+        mma_bf16_16816(c1, xa0[u].z, xa1[u].z, xa0[u].w, xa1[u].w, b2.z, b2.w);
       }
     }
-    float v0 = 0.f, v1 = 0.f;
+  }
+  // c0[0..1]: row g, adapter columns 2t, 2t + 1; c0[2..3]: row g + 8; c1: columns 8 + 2t, 8 + 2t + 1.
+  // Columns 16..63 of an xa row are zero: lane t writes words 8 + 6t .. 8 + 6t + 5.
+  if (v0) {
+    uint32_t* row = reinterpret_cast<uint32_t*>(q.xa + p0 * kLoraCols);
+    row[t] = pack_bf16x2(q.scale * c0[0], q.scale * c0[1]);
+    row[4 + t] = pack_bf16x2(q.scale * c1[0], q.scale * c1[1]);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      if (j >= q.r) break;
-      float v = acc[j];
+    for (int i = 0; i < 6; ++i) row[8 + 6 * t + i] = 0u;
+  }
+  if (v1) {
+    uint32_t* row = reinterpret_cast<uint32_t*>(q.xa + p1 * kLoraCols);
+    row[t] = pack_bf16x2(q.scale * c0[2], q.scale * c0[3]);
+    row[4 + t] = pack_bf16x2(q.scale * c1[2], q.scale * c1[3]);
 #pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (j == 2 * lane) v0 = v;
-      if (j == 2 * lane + 1) v1 = v;
-    }
-    reinterpret_cast<uint32_t*>(q.xa + pr * kLoraCols)[lane] = pack_bf16x2(q.scale * v0, q.scale * v1);
+    for (int i = 0; i < 6; ++i) row[8 + 6 * t + i] = 0u;
   }
 }
 
@@ -967,7 +1006,7 @@ bool tc_supported(const GemmArgs& a) {
   // kernel's shared memory and the products need their workspace rows.
   if (a.row_index != nullptr || a.lda % 8 != 0 || !tensor_maps_available()) return false;
   if (a.lora_B && a.r > 0)
-    return a.r <= 16 && a.xa != nullptr && static_cast<size_t>(a.r) * a.K * 2 <= kLoraPrepSmemMax &&
+    return a.r <= 16 && a.xa != nullptr && static_cast<size_t>(16) * (a.K + 8) * 2 <= kLoraPrepSmemMax &&
            (reinterpret_cast<uintptr_t>(a.lora_A) & 15u) == 0;
   return true;
 }
@@ -1021,12 +1060,12 @@ cudaError_t launch_tc_lora_prep(const GemmArgs& a, cudaStream_t stream) {
   q.r = a.r;
   q.scale = a.lora_scale;
   q.xa = reinterpret_cast<uint16_t*>(a.xa);
-  const size_t smem = static_cast<size_t>(a.r) * a.K * 2;
+  const size_t smem = static_cast<size_t>(16) * (a.K + 8) * 2;
   cudaError_t err = ensure_smem_limit(reinterpret_cast<const void*>(lora_prep_kernel), smem);
   if (err != cudaSuccess) return err;
   const int64_t tiles = (a.total_rows + kPrepRows - 1) / kPrepRows + (a.E < a.total_rows ? a.E : a.total_rows);
   LaunchScope ls("gemm.tc.lora_prep", stream);
-  lora_prep_kernel<<<static_cast<unsigned>(tiles), 256, smem, stream>>>(q);
+  lora_prep_kernel<<<static_cast<unsigned>(tiles), 128, smem, stream>>>(q);
   return cudaGetLastError();
 }
 
