@@ -283,6 +283,28 @@ E4B_API e4b_status e4b_grouped_lora_grads(const uint16_t* x, int64_t x_rows, int
                                   float* dB, void* workspace, size_t workspace_bytes,
                                   e4b_stream stream);
 
+/*
+ * One grouped GEMM over E expert groups straight from MXFP4 expert bytes.
+ * Source: Solutions -- one page per problem, the grouped-nf4-gemm row on
+ * gemm_mxfp4_grouped (released e2m1 blocks and e8m0 scales multiplied as they
+ * are, no requantisation, no bf16 weight copy).
+ *
+ * As e4b_grouped_nf4_gemm() (row p of group e: y[p, :] = A[row_index[p], :] .
+ * W_e^T, the same epilogues, no adapter), with W_e in the OCP microscaling
+ * format: element (n, k) = e2m1(code) * 2^(scale - 127), where
+ *   blocks  [E, N*K/2] uint8: row n of expert e holds K/2 bytes, element 2i
+ *           of the row in the low nibble of byte i (the released layout);
+ *           e2m1 = sign (bit 3), exponent (bits 2-1, bias 1), mantissa (bit 0);
+ *   scales  [E, N*K/32] uint8: one e8m0 byte per 32 consecutive elements of a
+ *           row; 255 is NaN and makes its block NaN.
+ * Requires K % 64 == 0, N % 64 == 0.  No workspace (nothing waits).
+ */
+E4B_API e4b_status e4b_grouped_mxfp4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda,
+                                  const int32_t* row_index, const int32_t* expert_offsets,
+                                  int64_t E, int64_t total_rows, const uint8_t* blocks,
+                                  const uint8_t* scales, int64_t N, int64_t K, e4b_epilogue epi,
+                                  void* out, e4b_dtype out_dtype, e4b_stream stream);
+
 /* The two packed stacks of one MoE layer (device pointers), plus its adapter. */
 typedef struct {
   const uint8_t* gu_packed; /* [E, 2I*H/2]  gate_up_proj, NF4 */

@@ -584,6 +584,50 @@ e4b_status e4b_grouped_lora_grads(const uint16_t* x, int64_t x_rows, int64_t ldx
   return E4B_OK;
 }
 
+e4b_status e4b_grouped_mxfp4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda, const int32_t* row_index,
+                                  const int32_t* expert_offsets, int64_t E, int64_t total_rows,
+                                  const uint8_t* blocks, const uint8_t* scales, int64_t N, int64_t K,
+                                  e4b_epilogue epi, void* out, e4b_dtype out_dtype, e4b_stream stream) {
+  begin_call();
+  if (E < 1 || E > 65536) return fail(E4B_ERR_INVALID_ARGUMENT, "E must be in [1, 65536]");
+  if (total_rows < 0 || a_rows < 0) return fail(E4B_ERR_INVALID_ARGUMENT, "total_rows and a_rows must be >= 0");
+  if (total_rows > 0 && a_rows < 1) return fail(E4B_ERR_INVALID_ARGUMENT, "a_rows must be >= 1 when rows exist");
+  if (K < 64 || K % 64 != 0) return fail(E4B_ERR_UNSUPPORTED, "K must be a positive multiple of 64");
+  if (N < 64 || N % 64 != 0) return fail(E4B_ERR_UNSUPPORTED, "N must be a positive multiple of 64");
+  if (lda < K || lda % 8 != 0) return fail(E4B_ERR_INVALID_ARGUMENT, "lda must be >= K and a multiple of 8");
+  if (epi != E4B_EPI_NONE && epi != E4B_EPI_SWIGLU) return fail(E4B_ERR_INVALID_ARGUMENT, "unknown epilogue");
+  if (out_dtype != E4B_F32 && out_dtype != E4B_BF16) return fail(E4B_ERR_INVALID_ARGUMENT, "out_dtype must be F32 or BF16");
+  if (!expert_offsets || !blocks || !scales) return fail(E4B_ERR_INVALID_ARGUMENT, "null expert_offsets, blocks or scales");
+  if (total_rows > 0 && (!A || !out)) return fail(E4B_ERR_INVALID_ARGUMENT, "null A or out");
+  if (total_rows > INT32_MAX) return fail(E4B_ERR_UNSUPPORTED, "total_rows exceeds int32");
+  if ((A && !aligned16(A)) || !aligned16(blocks) || (out && !aligned16(out)))
+    return fail(E4B_ERR_INVALID_ARGUMENT, "A, blocks and out must be 16-byte aligned");
+  if (e4b_status s = check_device(); s != E4B_OK) return s;
+  if (total_rows == 0) {
+    set_path("mxfp4.empty");
+    return E4B_OK;
+  }
+  Mxfp4Args m{};
+  m.A = A;
+  m.a_rows = a_rows;
+  m.lda = lda;
+  m.row_index = row_index;
+  m.offsets = expert_offsets;
+  m.E = static_cast<int>(E);
+  m.total_rows = total_rows;
+  m.blocks = blocks;
+  m.scales = scales;
+  m.N = static_cast<int>(N);
+  m.K = static_cast<int>(K);
+  m.epi = epi;
+  m.out = out;
+  m.out_bf16 = out_dtype == E4B_BF16;
+  cudaError_t err = launch_grouped_mxfp4_gemm(m, reinterpret_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "grouped mxfp4 gemm launch");
+  set_path(epi == E4B_EPI_SWIGLU ? "mxfp4.mma.swiglu" : "mxfp4.mma");
+  return E4B_OK;
+}
+
 static e4b_status check_stack(const e4b_expert_stack* w, int k) {
   if (!w) return fail(E4B_ERR_INVALID_ARGUMENT, "null expert stack");
   if (w->E < 1 || w->E > 1024) return fail(E4B_ERR_UNSUPPORTED, "E must be in [1, 1024]");

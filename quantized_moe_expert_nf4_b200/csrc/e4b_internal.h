@@ -165,6 +165,23 @@ cudaError_t launch_token_sum(const float* dxg, const int32_t* inv, int64_t M, in
 cudaError_t launch_router_grad(const float* logits, const int32_t* ids, const float* w, const float* dw, int64_t M,
                                int E, int k, bool renormalize, float* dlogits, cudaStream_t stream);
 
+// ---- grouped MXFP4 GEMM -------------------------------------------------------
+struct Mxfp4Args {
+  const uint16_t* A;
+  int64_t a_rows, lda;
+  const int32_t* row_index;  // nullable
+  const int32_t* offsets;    // [E+1]
+  int E;
+  int64_t total_rows;
+  const uint8_t* blocks;  // [E, N*K/2] e2m1 codes, element 2i in the low nibble
+  const uint8_t* scales;  // [E, N*K/32] e8m0
+  int N, K;
+  int epi;
+  void* out;
+  bool out_bf16;
+};
+cudaError_t launch_grouped_mxfp4_gemm(const Mxfp4Args& a, cudaStream_t stream);
+
 // ---- combine ---------------------------------------------------------------
 cudaError_t launch_combine(const uint16_t* z, const int32_t* inv, const float* w, int64_t M, int k,
                            int H, uint16_t* out, cudaStream_t stream);

@@ -37,6 +37,7 @@ EXPORTED = (
     "e4b_grouped_nf4_gemm_workspace_size", "e4b_grouped_nf4_gemm",
     "e4b_grouped_nf4_gemm_dgrad_workspace_size", "e4b_grouped_nf4_gemm_dgrad",
     "e4b_grouped_lora_grads_workspace_size", "e4b_grouped_lora_grads",
+    "e4b_grouped_mxfp4_gemm",
     "e4b_moe_expert_forward_workspace_size", "e4b_moe_expert_forward",
     "e4b_moe_expert_forward_path", "e4b_moe_expert_forward_decode_noalloc",
     "e4b_moe_expert_backward_workspace_size", "e4b_moe_expert_backward",
@@ -109,6 +110,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.e4b_grouped_lora_grads.restype = i32
     lib.e4b_grouped_lora_grads.argtypes = [vp, i64, i64, vp, vp, i64, i64, vp, i64, i64, i64, vp, vp, i32,
                                            ctypes.c_float, vp, vp, vp, sz, vp]
+    lib.e4b_grouped_mxfp4_gemm.restype = i32
+    lib.e4b_grouped_mxfp4_gemm.argtypes = [vp, i64, i64, vp, vp, i64, i64, vp, vp, i64, i64, i32, vp, i32, vp]
     lib.e4b_moe_expert_forward_workspace_size.restype = sz
     lib.e4b_moe_expert_forward_workspace_size.argtypes = [i64, ctypes.POINTER(ExpertStackC), i32]
     lib.e4b_moe_expert_forward.restype = i32
@@ -322,6 +325,31 @@ def e4b_grouped_lora_grads(x: torch.Tensor, row_index: Optional[torch.Tensor], e
         x.data_ptr(), x.shape[0], x.stride(0), _ptr(row_index), expert_offsets.data_ptr(), E, total_rows,
         da.data_ptr(), da.stride(0), N, K, lora_A.data_ptr(), lora_B.data_ptr(), r, float(lora_scale),
         dA.data_ptr(), dB.data_ptr(), _ptr(workspace), ws, _stream(stream)), "e4b_grouped_lora_grads")
+
+
+def e4b_grouped_mxfp4_gemm(A: torch.Tensor, row_index: Optional[torch.Tensor], expert_offsets: torch.Tensor,
+                           total_rows: int, blocks: torch.Tensor, scales: torch.Tensor, N: int, K: int,
+                           out: torch.Tensor, epi: int = E4B_EPI_NONE, stream=None) -> None:
+    """y[p] = A[row_index[p]] . W_e^T with W_e given as MXFP4 code bytes and e8m0 scales."""
+    if A.dim() != 2 or A.dtype != torch.bfloat16 or not A.is_cuda or A.stride(1) != 1:
+        raise ValueError("A must be a 2-D bf16 CUDA tensor with unit column stride")
+    _dev(expert_offsets, "expert_offsets", torch.int32)
+    _dev(blocks, "blocks", torch.uint8)
+    _dev(scales, "scales", torch.uint8)
+    _dev(out, "out")
+    if row_index is not None:
+        _dev(row_index, "row_index", torch.int32)
+    E = expert_offsets.numel() - 1
+    od = {torch.float32: E4B_F32, torch.bfloat16: E4B_BF16}.get(out.dtype)
+    if od is None:
+        raise ValueError("out must be float32 or bfloat16")
+    ncols = N // 2 if epi == E4B_EPI_SWIGLU else N
+    if out.numel() < total_rows * ncols:
+        raise ValueError("out too small")
+    _check(load_library().e4b_grouped_mxfp4_gemm(
+        A.data_ptr(), A.shape[0], A.stride(0), _ptr(row_index), expert_offsets.data_ptr(), E, total_rows,
+        blocks.data_ptr(), scales.data_ptr(), N, K, epi, out.data_ptr(), od, _stream(stream)),
+        "e4b_grouped_mxfp4_gemm")
 
 
 class ExpertStack:

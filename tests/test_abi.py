@@ -214,3 +214,20 @@ def test_backward_host_side_checks(lib):
     status = lib.e4b_moe_expert_backward(vp, 64, vp, 2, 1, ctypes.byref(stl), vp, vp, vp, None, None, vp, 1 << 40,
                                          None)
     assert status == 1 and b"needs dA and dB" in lib.e4b_last_error()
+
+
+def test_mxfp4_host_side_rejections(lib):
+    p = ctypes.c_void_p(1 << 20)
+
+    def call(**kw):
+        a = dict(A=p, a_rows=4, lda=128, ridx=None, offs=p, E=2, rows=4, blocks=p, scales=p, N=128, K=128, epi=0,
+                 out=p, od=0)
+        a.update(kw)
+        return lib.e4b_grouped_mxfp4_gemm(a["A"], a["a_rows"], a["lda"], a["ridx"], a["offs"], a["E"], a["rows"],
+                                          a["blocks"], a["scales"], a["N"], a["K"], a["epi"], a["out"], a["od"], None)
+    assert call(K=96) == 2 and b"K must be" in lib.e4b_last_error()
+    assert call(N=32) == 2 and b"N must be" in lib.e4b_last_error()
+    assert call(lda=100) == 1 and b"lda" in lib.e4b_last_error()
+    assert call(epi=7) == 1 and b"epilogue" in lib.e4b_last_error()
+    assert call(scales=None) == 1 and b"null" in lib.e4b_last_error()
+    assert call(blocks=ctypes.c_void_p((1 << 20) + 4)) == 1 and b"16-byte aligned" in lib.e4b_last_error()
