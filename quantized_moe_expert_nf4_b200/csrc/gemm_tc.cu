@@ -748,6 +748,8 @@ cudaError_t launch_shape(const GemmArgs& a, int* err_word, cudaStream_t stream) 
                    CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   const bool lora = a.lora_B != nullptr && a.r > 0;
+  // The TMEM decoders have no LoRA step: their barrier phases would drift from the MMA issuer's.
+  if (S::ATMEM && lora) return cudaErrorInvalidValue;
   CUtensorMap tm_xa = tm_b;  // unused without LoRA
   if (lora && !make_map_2d(&tm_xa, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.xa, kLoraCols, a.total_rows, kLoraCols * 2, 64,
                            S::BN, CU_TENSOR_MAP_SWIZZLE_128B))
