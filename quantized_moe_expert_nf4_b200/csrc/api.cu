@@ -127,6 +127,7 @@ e4b_status cuda_fail(cudaError_t err, const char* where) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool quant_type_ok(int q) { return q == E4B_QUANT_NF4 || q == E4B_QUANT_FP4; }
 
 // Size, presence and alignment of a caller's workspace.
 e4b_status check_workspace(const char* what, size_t need, const void* workspace, size_t workspace_bytes) {
@@ -311,7 +312,13 @@ e4b_status e4b_timing_get(int i, const char** name, double* total_ms, int* launc
 
 e4b_status e4b_nf4_quantize_stack(const void* W, e4b_dtype w_dtype, int64_t E, int64_t N, int64_t K,
                                   int blocksize, uint8_t* packed, float* absmax, e4b_stream stream) {
+  return e4b_quantize_stack(W, w_dtype, E, N, K, blocksize, E4B_QUANT_NF4, packed, absmax, stream);
+}
+
+e4b_status e4b_quantize_stack(const void* W, e4b_dtype w_dtype, int64_t E, int64_t N, int64_t K, int blocksize,
+                              e4b_quant_type quant_type, uint8_t* packed, float* absmax, e4b_stream stream) {
   begin_call();
+  if (!quant_type_ok(quant_type)) return fail(E4B_ERR_INVALID_ARGUMENT, "quant_type must be NF4 or FP4");
   if (blocksize != 64) return fail(E4B_ERR_UNSUPPORTED, "blocksize must be 64, got " + std::to_string(blocksize));
   if (w_dtype != E4B_F32 && w_dtype != E4B_BF16) return fail(E4B_ERR_INVALID_ARGUMENT, "w_dtype must be F32 or BF16");
   if (E < 1 || N < 1 || K < 1)
@@ -323,7 +330,7 @@ e4b_status e4b_nf4_quantize_stack(const void* W, e4b_dtype w_dtype, int64_t E, i
     return fail(E4B_ERR_INVALID_ARGUMENT, "W, packed and absmax must be 16-byte aligned");
   if (e4b_status s = check_device(); s != E4B_OK) return s;
   const int64_t nblocks = E * N * K / 64;
-  cudaError_t err = launch_quantize(W, w_dtype == E4B_BF16, nblocks, packed, absmax, stream);
+  cudaError_t err = launch_quantize(W, w_dtype == E4B_BF16, nblocks, static_cast<int>(quant_type), packed, absmax, stream);
   if (err != cudaSuccess) return cuda_fail(err, "quantize launch");
   set_path("quantize");
   return E4B_OK;
@@ -367,7 +374,19 @@ e4b_status e4b_grouped_nf4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda, 
                                 const float* absmax, int64_t N, int64_t K, const uint16_t* lora_A,
                                 const uint16_t* lora_B, int r, float lora_scale, e4b_epilogue epi, void* out,
                                 e4b_dtype out_dtype, void* workspace, size_t workspace_bytes, e4b_stream stream) {
+  return e4b_grouped_4bit_gemm(A, a_rows, lda, row_index, expert_offsets, E, total_rows, packed, absmax,
+                               E4B_QUANT_NF4, N, K, lora_A, lora_B, r, lora_scale, epi, out, out_dtype, workspace,
+                               workspace_bytes, stream);
+}
+
+e4b_status e4b_grouped_4bit_gemm(const uint16_t* A, int64_t a_rows, int64_t lda, const int32_t* row_index,
+                                 const int32_t* expert_offsets, int64_t E, int64_t total_rows, const uint8_t* packed,
+                                 const float* absmax, e4b_quant_type quant_type, int64_t N, int64_t K,
+                                 const uint16_t* lora_A, const uint16_t* lora_B, int r, float lora_scale,
+                                 e4b_epilogue epi, void* out, e4b_dtype out_dtype, void* workspace,
+                                 size_t workspace_bytes, e4b_stream stream) {
   begin_call();
+  if (!quant_type_ok(quant_type)) return fail(E4B_ERR_INVALID_ARGUMENT, "quant_type must be NF4 or FP4");
   if (E < 1 || E > 65536) return fail(E4B_ERR_INVALID_ARGUMENT, "E must be in [1, 65536]");
   if (total_rows < 0 || a_rows < 0) return fail(E4B_ERR_INVALID_ARGUMENT, "total_rows and a_rows must be >= 0");
   if (total_rows > 0 && a_rows < 1) return fail(E4B_ERR_INVALID_ARGUMENT, "a_rows must be >= 1 when rows exist");
@@ -405,6 +424,7 @@ e4b_status e4b_grouped_nf4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda, 
   g.total_rows = total_rows;
   g.packed = packed;
   g.absmax = absmax;
+  g.quant = quant_type;
   g.N = static_cast<int>(N);
   g.K = static_cast<int>(K);
   g.lora_A = lora_A;
@@ -439,7 +459,19 @@ e4b_status e4b_grouped_nf4_gemm_dgrad(const uint16_t* dY, int64_t dy_rows, int64
                                       const uint16_t* lora_A, const uint16_t* lora_B, int r, float lora_scale,
                                       void* out, e4b_dtype out_dtype, void* workspace, size_t workspace_bytes,
                                       e4b_stream stream) {
+  return e4b_grouped_4bit_gemm_dgrad(dY, dy_rows, lddy, row_index, expert_offsets, E, total_rows, packed, absmax,
+                                     E4B_QUANT_NF4, N, K, lora_A, lora_B, r, lora_scale, out, out_dtype, workspace,
+                                     workspace_bytes, stream);
+}
+
+e4b_status e4b_grouped_4bit_gemm_dgrad(const uint16_t* dY, int64_t dy_rows, int64_t lddy, const int32_t* row_index,
+                                       const int32_t* expert_offsets, int64_t E, int64_t total_rows,
+                                       const uint8_t* packed, const float* absmax, e4b_quant_type quant_type,
+                                       int64_t N, int64_t K, const uint16_t* lora_A, const uint16_t* lora_B, int r,
+                                       float lora_scale, void* out, e4b_dtype out_dtype, void* workspace,
+                                       size_t workspace_bytes, e4b_stream stream) {
   begin_call();
+  if (!quant_type_ok(quant_type)) return fail(E4B_ERR_INVALID_ARGUMENT, "quant_type must be NF4 or FP4");
   if (E < 1 || E > 65536) return fail(E4B_ERR_INVALID_ARGUMENT, "E must be in [1, 65536]");
   if (total_rows < 0 || dy_rows < 0) return fail(E4B_ERR_INVALID_ARGUMENT, "total_rows and dy_rows must be >= 0");
   if (total_rows > 0 && dy_rows < 1) return fail(E4B_ERR_INVALID_ARGUMENT, "dy_rows must be >= 1 when rows exist");
@@ -476,6 +508,7 @@ e4b_status e4b_grouped_nf4_gemm_dgrad(const uint16_t* dY, int64_t dy_rows, int64
   d.total_rows = total_rows;
   d.packed = packed;
   d.absmax = absmax;
+  d.quant = quant_type;
   d.N = static_cast<int>(N);
   d.K = static_cast<int>(K);
   d.lora_A = r ? lora_A : nullptr;
@@ -636,6 +669,7 @@ static e4b_status check_stack(const e4b_expert_stack* w, int k) {
   if (k < 1 || k > w->E || k > 32) return fail(E4B_ERR_INVALID_ARGUMENT, "k must be in [1, min(E, 32)]");
   if (!w->gu_packed || !w->gu_absmax || !w->dn_packed || !w->dn_absmax)
     return fail(E4B_ERR_INVALID_ARGUMENT, "null packed stack pointer");
+  if (!quant_type_ok(w->quant_type)) return fail(E4B_ERR_INVALID_ARGUMENT, "quant_type must be NF4 or FP4");
   if ((w->lora_A == nullptr) != (w->lora_B == nullptr))
     return fail(E4B_ERR_INVALID_ARGUMENT, "lora_A and lora_B must be both set or both NULL");
   if (w->lora_A && (w->lora_r < 1 || w->lora_r > 16)) return fail(E4B_ERR_UNSUPPORTED, "LoRA rank must be in [1, 16]");
@@ -675,6 +709,7 @@ static e4b_status forward_grouped(const uint16_t* x, int64_t M, const float* log
   g.total_rows = S;
   g.packed = w->gu_packed;
   g.absmax = w->gu_absmax;
+  g.quant = w->quant_type;
   g.N = static_cast<int>(2 * w->I);
   g.K = static_cast<int>(w->H);
   g.lora_A = r ? w->lora_A : nullptr;
@@ -699,6 +734,7 @@ static e4b_status forward_grouped(const uint16_t* x, int64_t M, const float* log
   d.total_rows = S;
   d.packed = w->dn_packed;
   d.absmax = w->dn_absmax;
+  d.quant = w->quant_type;
   d.N = static_cast<int>(w->H);
   d.K = static_cast<int>(w->I);
   d.err = at<int>(ws, L.err);
@@ -809,6 +845,7 @@ e4b_status e4b_moe_expert_backward(const uint16_t* x, int64_t M, const float* ro
   g.total_rows = S;
   g.packed = w->gu_packed;
   g.absmax = w->gu_absmax;
+  g.quant = w->quant_type;
   g.N = 2 * I;
   g.K = H;
   g.lora_A = r ? w->lora_A : nullptr;
@@ -834,6 +871,7 @@ e4b_status e4b_moe_expert_backward(const uint16_t* x, int64_t M, const float* ro
   d.total_rows = S;
   d.packed = w->dn_packed;
   d.absmax = w->dn_absmax;
+  d.quant = w->quant_type;
   d.N = H;
   d.K = I;
   d.err = at<int>(ws, L.err);
@@ -855,6 +893,7 @@ e4b_status e4b_moe_expert_backward(const uint16_t* x, int64_t M, const float* ro
   dd.total_rows = S;
   dd.packed = w->dn_packed;
   dd.absmax = w->dn_absmax;
+  dd.quant = w->quant_type;
   dd.N = H;
   dd.K = I;
   dd.out = at<float>(ws, L.dh);
@@ -874,6 +913,7 @@ e4b_status e4b_moe_expert_backward(const uint16_t* x, int64_t M, const float* ro
   dg.total_rows = S;
   dg.packed = w->gu_packed;
   dg.absmax = w->gu_absmax;
+  dg.quant = w->quant_type;
   dg.N = 2 * I;
   dg.K = H;
   dg.lora_A = r ? w->lora_A : nullptr;

@@ -14,9 +14,21 @@
       0.33791524171829224f, 0.44070982933044434f, 0.5626170039176941f, 0.7229568362236023f, \
       1.0f
 
+// The FP4 codebook: code c is the e2m1 element (sign bit 3, exponent bits 2-1
+// with bias 1, mantissa bit 0; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6) divided by
+// 6, each entry the float nearest to that ratio (the divisions below are
+// correctly rounded).  Codes 0 and 8 are both zero.
+#define E4B_FP4_CODEBOOK_VALUES                                                                          \
+  0.0f, 0.5f / 6.0f, 1.0f / 6.0f, 1.5f / 6.0f, 2.0f / 6.0f, 3.0f / 6.0f, 4.0f / 6.0f, 1.0f, -0.0f,      \
+      -0.5f / 6.0f, -1.0f / 6.0f, -1.5f / 6.0f, -2.0f / 6.0f, -3.0f / 6.0f, -4.0f / 6.0f, -1.0f
+
 namespace e4b {
 
-static __device__ __constant__ float kNf4CodebookDev[16] = {E4B_NF4_CODEBOOK_VALUES};
+// Indexed by e4b_quant_type: [0] NF4, [1] FP4.
+static __device__ __constant__ float kCodebooksDev[2][16] = {{E4B_NF4_CODEBOOK_VALUES}, {E4B_FP4_CODEBOOK_VALUES}};
+
+// Entry c (0..15) of the codebook of storage type `quant` (0 NF4, any other value FP4).
+__device__ __forceinline__ float codebook_entry(int quant, int c) { return kCodebooksDev[quant != 0 ? 1 : 0][c & 15]; }
 
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
   return __uint_as_float(static_cast<uint32_t>(b) << 16);

@@ -61,6 +61,7 @@ struct DecodeParams {
   const float* gu_absmax;
   const uint8_t* dn_packed;
   const float* dn_absmax;
+  int quant;  // e4b_quant_type of both stacks
   const uint16_t* lora_A;
   const uint16_t* lora_B;
   int r;
@@ -232,9 +233,9 @@ __device__ __forceinline__ void route_one(const DecodeParams& p, int t, int* ids
 
 // Byte -> bf16x2 codebook pairs, replicated per lane (entry b of lane l at
 // b * 32 + l), entries first, first + step, ... written by the calling warp.
-__device__ __forceinline__ void fill_lut(uint32_t* lut, int first, int step) {
+__device__ __forceinline__ void fill_lut(uint32_t* lut, int quant, int first, int step) {
   const int lane = threadIdx.x & 31;
-  const float cbl = kNf4CodebookDev[lane & 15];
+  const float cbl = codebook_entry(quant, lane & 15);
   for (int b = first; b < 256; b += step) {
     const float hi = __shfl_sync(0xffffffffu, cbl, b >> 4);
     const float lo = __shfl_sync(0xffffffffu, cbl, b & 15);
@@ -253,7 +254,7 @@ __device__ void route_prologue(const DecodeParams& p, uint32_t* lut, int* ids_s,
   for (int e = tid; e < p.E; e += blockDim.x) uidx[e] = -1;
   const int nwarps = static_cast<int>(blockDim.x >> 5);
   if (warp < p.M) route_one(p, warp, ids_s, w_s);
-  else fill_lut(lut, warp - p.M, nwarps - p.M);
+  else fill_lut(lut, p.quant, warp - p.M, nwarps - p.M);
   __syncthreads();
   for (int s = tid; s < S; s += blockDim.x) uidx[ids_s[s]] = 0;  // flag
   __syncthreads();
@@ -812,6 +813,7 @@ cudaError_t launch_decode_forward(const DecodeArgs& a, cudaStream_t stream) {
   p.gu_absmax = w->gu_absmax;
   p.dn_packed = w->dn_packed;
   p.dn_absmax = w->dn_absmax;
+  p.quant = w->quant_type;
   p.lora_A = r ? w->lora_A : nullptr;
   p.lora_B = r ? w->lora_B : nullptr;
   p.r = r;

@@ -31,18 +31,25 @@ class LaunchScope {
 };
 void begin_call();  // resets the per-call launch counter
 
-// The NF4 codebook as the library holds it (QLoRA table, ascending).
-extern const float kNf4Codebook[16];
+// The codebooks as the library holds them, indexed by e4b_quant_type: NF4
+// (QLoRA table, ascending) and FP4 (e2m1 / 6, in code order).
+extern const float kCodebooks[2][16];
 
-// Quantiser decision thresholds: T[c] is the smallest float strictly above
-// the exact midpoint (cb[c] + cb[c+1]) / 2, so that for any float s,
-// s > midpoint  <=>  s >= T[c].  T[15] = +inf.
-struct Nf4Thresholds {
+// Quantiser tables of one storage type.  The distinct codebook values in
+// ascending order are the levels; T[l] is the smallest float strictly above
+// the exact midpoint of levels l and l+1, so that for any float s,
+// s > midpoint  <=>  s >= T[l]; the unused tail of T is +inf.  The level of s
+// is the number of thresholds <= s; code[level] is the code written for it
+// (the lowest code holding that value); zero_code is written for an all-zero
+// block.
+struct QuantTables {
   float t[16];
+  uint32_t code[16];
+  uint32_t zero_code;
 };
-Nf4Thresholds nf4_thresholds();
+QuantTables quant_tables(int quant);
 
-cudaError_t launch_quantize(const void* W, bool bf16, int64_t nblocks, uint8_t* packed,
+cudaError_t launch_quantize(const void* W, bool bf16, int64_t nblocks, int quant, uint8_t* packed,
                             float* absmax, cudaStream_t stream);
 
 // ---- routing -------------------------------------------------------------
@@ -71,6 +78,7 @@ struct GemmArgs {
   int64_t total_rows;
   const uint8_t* packed;
   const float* absmax;
+  int quant;  // e4b_quant_type of packed
   int N, K;
   const uint16_t* lora_A;  // [E, r, K] or nullptr
   const uint16_t* lora_B;  // [E, N, r] or nullptr
@@ -107,6 +115,7 @@ struct DgradArgs {
   int64_t total_rows;
   const uint8_t* packed;
   const float* absmax;
+  int quant;  // e4b_quant_type of packed
   int N, K;
   const uint16_t* lora_A;  // [E, r, K] or nullptr
   const uint16_t* lora_B;  // [E, N, r] or nullptr

@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(kThreads) grouped_nf4_mma_kernel(GemmArgs a) {
   if (!find_group_tile(a.offsets, a.E, a.total_rows, kTileT, blockIdx.x, &e, &row_begin, &row_end)) return;
 
   // byte b = (code of the even element << 4) | code of the odd element
-  for (int b = tid; b < 256; b += kThreads) lut[b] = pack_bf16x2(kNf4CodebookDev[b >> 4], kNf4CodebookDev[b & 15]);
+  for (int b = tid; b < 256; b += kThreads) lut[b] = pack_bf16x2(codebook_entry(a.quant, b >> 4), codebook_entry(a.quant, b & 15));
   const int nrows = static_cast<int>(row_end - row_begin);
   for (int i = tid; i < kTileT; i += kThreads) {
     int64_t src = row_begin + i;

@@ -113,6 +113,7 @@ struct TcParams {
   int* err;
   const uint16_t* lora_B;  // [E, N, r] bf16, or null (no LoRA step)
   int r;
+  int quant;  // e4b_quant_type of the packed codes
 };
 
 // The codebook's bf16 patterns split into low and high bytes, four entries per
@@ -121,11 +122,11 @@ struct CodebookBytes {
   uint32_t lo[4], hi[4];
 };
 
-__device__ __forceinline__ CodebookBytes codebook_bytes() {
+__device__ __forceinline__ CodebookBytes codebook_bytes(int quant) {
   CodebookBytes t{};
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
-    const uint32_t b = float_to_bf16_bits(kNf4CodebookDev[j]);
+    const uint32_t b = float_to_bf16_bits(codebook_entry(quant, j));
     t.lo[j >> 2] |= (b & 0xffu) << (8 * (j & 3));
     t.hi[j >> 2] |= (b >> 8) << (8 * (j & 3));
   }
@@ -188,7 +189,7 @@ __device__ __forceinline__ void tmem_decoders(const TcParams& p, unsigned char* 
   const int half = c >> 1, kpart = c & 1;
   const int ri = qd * 32 + lane;
   const int KB = p.K / 64;
-  const CodebookBytes cbt = codebook_bytes();
+  const CodebookBytes cbt = codebook_bytes(p.quant);
   uint32_t kbg = 0;
   bool ok = true;
   for (int64_t t = blockIdx.x; ok; t += gridDim.x) {
@@ -261,7 +262,7 @@ __device__ __forceinline__ void dgrad_decoders(const TcParams& p, unsigned char*
   const int q = (dt & 7) | (((dt >> 5) & 7) << 3);
   const int o = ((dt >> 3) & 3) | ((dt >> 8) << 2);
   const int KB = p.K / 64, kbw = p.N / 64;
-  const CodebookBytes cbt = codebook_bytes();
+  const CodebookBytes cbt = codebook_bytes(p.quant);
   uint32_t kbg = 0;
   bool ok = true;
   for (int64_t t = blockIdx.x; ok; t += gridDim.x) {
@@ -511,7 +512,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     } else {
     const int r = dt / S::kTpr, kq = dt % S::kTpr;  // weight row of the tile, part of the k block
     const int half = r >> 7, ri = r & 127;
-    const CodebookBytes cbt = codebook_bytes();
+    const CodebookBytes cbt = codebook_bytes(p.quant);
     uint32_t kbg = 0;
     bool ok = true;
     for (int64_t t = blockIdx.x; ok; t += gridDim.x) {
@@ -759,6 +760,7 @@ cudaError_t launch_shape(const GemmArgs& a, int* err_word, cudaStream_t stream) 
   p.E = a.E;
   p.total_rows = a.total_rows;
   p.absmax = a.absmax;
+  p.quant = a.quant;
   p.N = a.N;
   p.K = a.K;
   p.swiglu = a.epi == E4B_EPI_SWIGLU;
@@ -807,6 +809,7 @@ cudaError_t launch_dgrad_shape(const DgradArgs& a, const uint16_t* dy, int64_t d
   p.E = a.E;
   p.total_rows = a.total_rows;
   p.absmax = a.absmax;
+  p.quant = a.quant;
   p.N = a.K;  // tile rows: columns k of W
   p.K = a.N;  // K steps: rows n of W
   p.swiglu = 0;

@@ -74,6 +74,8 @@ extern "C" e4b_status e4b_moe_expert_forward_decode_noalloc(const uint16_t* x, i
   if ((w->lora_A == nullptr) != (w->lora_B == nullptr))
     return nofail(E4B_ERR_INVALID_ARGUMENT, "lora_A and lora_B must be both set or both NULL");
   if (w->lora_A && (w->lora_r < 1 || w->lora_r > 16)) return nofail(E4B_ERR_UNSUPPORTED, "LoRA rank must be in [1, 16]");
+  if (w->quant_type != E4B_QUANT_NF4 && w->quant_type != E4B_QUANT_FP4)
+    return nofail(E4B_ERR_INVALID_ARGUMENT, "quant_type must be NF4 or FP4");
   auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
   if (!a16(x) || !a16(out) || !a16(w->gu_packed) || !a16(w->dn_packed) || !a16(w->gu_absmax) || !a16(w->dn_absmax))
     return nofail(E4B_ERR_INVALID_ARGUMENT, "x, out, packed stacks and absmax must be 16-byte aligned");

@@ -48,7 +48,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.e4b_version() == 1
+    assert lib.e4b_version() == e4b.ABI_VERSION == 2
     assert lib.e4b_status_string(0) == b"E4B_OK"
     assert lib.e4b_status_string(3) == b"E4B_ERR_WORKSPACE"
 
@@ -231,3 +231,37 @@ def test_mxfp4_host_side_rejections(lib):
     assert call(epi=7) == 1 and b"epilogue" in lib.e4b_last_error()
     assert call(scales=None) == 1 and b"null" in lib.e4b_last_error()
     assert call(blocks=ctypes.c_void_p((1 << 20) + 4)) == 1 and b"16-byte aligned" in lib.e4b_last_error()
+
+
+def test_storage_type_is_checked_on_the_host(lib):
+    """An e4b_quant_type other than NF4 and FP4 is an argument error from every
+    call that takes one, before any device work; FP4 itself passes the host
+    checks."""
+    p = ctypes.c_void_p(1 << 20)
+    assert lib.e4b_quantize_stack(p, 0, 1, 1, 64, 64, 2, p, p, None) == 1
+    assert b"quant_type" in lib.e4b_last_error()
+    assert lib.e4b_quantize_stack(p, 0, 1, 1, 64, 64, e4b.E4B_QUANT_FP4, p, p, None) != 1
+    assert b"quant_type" not in lib.e4b_last_error()
+    rows, N, K = 64, 128, 128
+    need = e4b.e4b_grouped_nf4_gemm_workspace_size(rows, N, K, 0)
+    st = lib.e4b_grouped_4bit_gemm(p, rows, K, None, p, 2, rows, p, p, 5, N, K, None, None, 0, 0.0, 0, p, 0, p, need,
+                                   None)
+    assert st == 1 and b"quant_type" in lib.e4b_last_error()
+    st = lib.e4b_grouped_4bit_gemm_dgrad(p, rows, N, None, p, 2, rows, p, p, -1, N, K, None, None, 0, 0.0, p, 0, p,
+                                         1 << 30, None)
+    assert st == 1 and b"quant_type" in lib.e4b_last_error()
+    stk = e4b.ExpertStackC(1 << 20, 1 << 20, 1 << 20, 1 << 20, None, None, 0, 0.0, 8, 256, 128, 3)
+    st = lib.e4b_moe_expert_forward(p, 4, p, 2, 1, ctypes.byref(stk), p, p, 1 << 30, None)
+    assert st == 1 and b"quant_type" in lib.e4b_last_error()
+    st = lib.e4b_moe_expert_forward_decode_noalloc(p, 4, p, 2, 1, ctypes.byref(stk), p, None)
+    assert st == 1 and b"quant_type" in lib.e4b_last_error()
+
+
+def test_expert_stack_layout_matches_the_header():
+    """ctypes mirror of e4b_expert_stack: the storage type follows I."""
+    names = [f[0] for f in e4b.ExpertStackC._fields_]
+    assert names[-4:] == ["E", "H", "I", "quant_type"]
+    assert e4b.ExpertStackC.quant_type.offset == e4b.ExpertStackC.I.offset + 8
+    hdr = open(os.path.join(os.path.dirname(__file__), "..", "include", "e4b.h")).read()
+    body = hdr[hdr.index("typedef struct {\n  const uint8_t* gu_packed"):hdr.index("} e4b_expert_stack;")]
+    assert body.index("int64_t E, H, I;") < body.index("int32_t quant_type;")

@@ -115,3 +115,47 @@ def test_tensor_core_decoders_fill_the_swizzled_k_major_tile(halves, tpr):
         for k in range(64):
             addr = half * 128 * 64 + (ri >> 3) * 512 + (ri & 7) * 64 + (((k // 8) ^ (ri & 7)) << 3) + (k % 8)
             assert tile[addr] == W[r, k]
+
+
+def _byte_perm(x: int, y: int, s: int) -> int:
+    """PTX prmt (default mode): result byte i = byte (selector nibble i & 7) of
+    the 8-byte value y:x, or that byte's sign replicated when the nibble's bit 3 is set."""
+    src = (x & 0xFFFFFFFF) | ((y & 0xFFFFFFFF) << 32)
+    out = 0
+    for i in range(4):
+        n = (s >> (4 * i)) & 0xF
+        b = (src >> (8 * (n & 7))) & 0xFF
+        if n & 8:
+            b = 0xFF if b & 0x80 else 0x00
+        out |= b << (8 * i)
+    return out
+
+
+@pytest.mark.parametrize("table", ["nf4", "fp4"])
+def test_tensor_core_byte_permute_decoder_is_a_table_lookup(table):
+    """csrc/gemm_tc.cu decode4 for every 16-bit input: the codebook's bf16
+    patterns split into low and high bytes (four entries per word), two
+    permutes look up entries 0-7 and 8-15 by the nibbles' low three bits, a
+    third keeps the half each nibble's top bit names, two more interleave the
+    bytes -> (element 2i, 2i+1) and (2i+2, 2i+3), the high nibble of a byte
+    being the lower-index element.  Checked against direct lookup for the NF4
+    and the FP4 (e2m1 / 6, with -0 at code 8) tables."""
+    from oracle import fp4
+    from quantized_moe_expert_nf4_b200 import workloads
+    cb32 = nf4.NF4_CODEBOOK if table == "nf4" else fp4.codebook_f64().astype(np.float32)
+    bits = [int(b) for b in workloads.to_bf16_bits(np.asarray(cb32, np.float32))]
+    lo = [0, 0, 0, 0]
+    hi = [0, 0, 0, 0]
+    for j, b in enumerate(bits):
+        lo[j >> 2] |= (b & 0xFF) << (8 * (j & 3))
+        hi[j >> 2] |= (b >> 8) << (8 * (j & 3))
+    for g in range(1 << 16):
+        s = g & 0x7777
+        pick = ((g >> 1) & 0x4444) | 0x3210
+        L = _byte_perm(_byte_perm(lo[0], lo[1], s), _byte_perm(lo[2], lo[3], s), pick)
+        Hh = _byte_perm(_byte_perm(hi[0], hi[1], s), _byte_perm(hi[2], hi[3], s), pick)
+        w0 = _byte_perm(L, Hh, 0x4051)
+        w1 = _byte_perm(L, Hh, 0x6273)
+        n = [g & 15, (g >> 4) & 15, (g >> 8) & 15, (g >> 12) & 15]
+        assert w0 == bits[n[1]] | (bits[n[0]] << 16), hex(g)
+        assert w1 == bits[n[3]] | (bits[n[2]] << 16), hex(g)
