@@ -187,3 +187,30 @@ def test_forward_degenerate_routing(E, k, M, path):
     out, p = _forward(layer, x, logits, path)
     ref = _oracle_tokens(cfg, x, logits, np.arange(M))
     assert_close_layer(bf16_to_f64(out), ref, f"E={E} k={k} M={M} {p}")
+
+
+@pytest.mark.parametrize("M", [3, 300])
+def test_forward_replays_bit_identically_from_a_cuda_graph(M):
+    """The header promises graph-capturable calls (no host sync, no device data
+    read back): a captured forward replays to the same bits as an eager call,
+    on the decode path (M = 3) and the grouped tensor-core path (M = 300)."""
+    require_gpu()
+    cfg = workloads.CONFIGS["tiny"]
+    layer = synthetic.make_device_layer(cfg)
+    x, logits = synthetic.inputs(cfg, M)
+    eager, _ = _forward(layer, x, logits)
+    out = torch.empty_like(eager)
+    ws = e4b.workspace(e4b.e4b_moe_expert_forward_workspace_size(M, layer.stack, cfg.k))
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):   # warm the library's per-device state outside the capture
+        e4b.e4b_moe_expert_forward(x, logits, cfg.k, True, layer.stack, out, ws)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        e4b.e4b_moe_expert_forward(x, logits, cfg.k, True, layer.stack, out, ws)
+    out.fill_(float("nan"))
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), eager.view(torch.int16))

@@ -1,0 +1,153 @@
+"""CPU models of the index maps of the GPU kernels (regression pins).
+
+Each model restates, in numpy and exact arithmetic, how a kernel's threads
+place data -- which packed bytes a thread decodes, where it stores them, which
+MMA fragment registers they feed (PTX m16n8k16 layout) -- and checks the
+result against the plain definition.  The GPU tests check the compiled
+kernels against the oracle; these pin the index arithmetic itself.
+"""
+import numpy as np
+import pytest
+
+from oracle import nf4
+
+CB = nf4.codebook_f64()
+
+
+def _mma(acc, A, B):
+    """One m16n8k16: A[lane] = 4 pairs (a0..a3), B[lane] = 2 pairs; acc[lane] += 4 outputs."""
+    Am = np.zeros((16, 16))
+    Bm = np.zeros((16, 8))
+    for lane in range(32):
+        g, t = lane >> 2, lane & 3
+        a0, a1, a2, a3 = A[lane]
+        b0, b1 = B[lane]
+        Am[g, 2 * t:2 * t + 2] = a0
+        Am[g + 8, 2 * t:2 * t + 2] = a1
+        Am[g, 2 * t + 8:2 * t + 10] = a2
+        Am[g + 8, 2 * t + 8:2 * t + 10] = a3
+        Bm[2 * t:2 * t + 2, g] = b0
+        Bm[2 * t + 8:2 * t + 10, g] = b1
+    D = Am @ Bm
+    for lane in range(32):
+        g, t = lane >> 2, lane & 3
+        acc[lane] += [D[g, 2 * t], D[g, 2 * t + 1], D[g + 8, 2 * t], D[g + 8, 2 * t + 1]]
+
+
+def _pair(byte):
+    """An NF4 byte as (element 2i, element 2i+1): the high nibble first."""
+    return CB[byte >> 4], CB[byte & 15]
+
+
+def _layer_rows(seed, rows, K):
+    rng = np.random.default_rng(seed)
+    packed = rng.integers(0, 256, size=(rows, K // 2), dtype=np.uint8)
+    absmax = rng.random((rows, K // 64)) + 0.5
+    # the definition, through the oracle's own unpacking (independent of _pair)
+    W = CB[nf4.unpack_codes(packed).reshape(rows, K)] * np.repeat(absmax, 64, axis=1)
+    return packed, absmax, W
+
+
+@pytest.mark.parametrize("K", [128, 192, 2880])
+def test_decode_span_fragment_mapping(K):
+    """csrc/decode.cu span_mma: thread (g, t) of a span (128 k) holds 16 packed
+    bytes of rows g and g+8 at byte 16t (all inside k-block 2 span + t/2), the
+    block's absmax multiplied into each decoded pair, MMA j taking bytes 2j and
+    2j+1 and x words 2j, 2j+1 of the thread's 32 k."""
+    packed, absmax, W = _layer_rows(1, 16, K)
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((8, K))
+    KB = K // 64
+    acc = np.zeros((32, 4))
+    for sp in range((KB + 1) // 2):
+        A = [[None] * 32 for _ in range(8)]
+        B = [[None] * 32 for _ in range(8)]
+        for lane in range(32):
+            g, t = lane >> 2, lane & 3
+            kb = 2 * sp + (t >> 1)
+            live = kb < KB
+            r0 = packed[g, sp * 64 + 16 * t: sp * 64 + 16 * t + 16] if live else np.zeros(16, np.uint8)
+            r1 = packed[g + 8, sp * 64 + 16 * t: sp * 64 + 16 * t + 16] if live else np.zeros(16, np.uint8)
+            a0 = absmax[g, kb] if live else 0.0
+            a1 = absmax[g + 8, kb] if live else 0.0
+            xs = x[g, sp * 128 + 32 * t: sp * 128 + 32 * t + 32] if live else np.zeros(32)
+            for j in range(8):
+                p = lambda r, i, a: tuple(v * a for v in _pair(r[i]))
+                A[j][lane] = (p(r0, 2 * j, a0), p(r1, 2 * j, a1), p(r0, 2 * j + 1, a0), p(r1, 2 * j + 1, a1))
+                B[j][lane] = ((xs[4 * j], xs[4 * j + 1]), (xs[4 * j + 2], xs[4 * j + 3]))
+        for j in range(8):
+            _mma(acc, A[j], B[j])
+    got = np.zeros((16, 8))
+    for lane in range(32):
+        g, t = lane >> 2, lane & 3
+        got[g, 2 * t], got[g, 2 * t + 1], got[g + 8, 2 * t], got[g + 8, 2 * t + 1] = acc[lane]
+    ref = W @ x.T
+    assert np.abs(got - ref).max() <= 1e-12 * np.abs(ref).max()
+
+
+def test_warp_mma_gemm_fragment_mapping():
+    """csrc/gemm_mma.cu: lane t owns physical k [8t, 8t+8) of each 32-k chunk --
+    one 32-bit word of packed nibbles per row and one 16-byte vector of x -- the
+    chunk's two MMAs accumulate unscaled codebook values, folded into the result
+    times the row's absmax once per 64-k block."""
+    K = 192
+    packed, absmax, W = _layer_rows(3, 16, K)
+    x = np.random.default_rng(4).standard_normal((8, K))
+    acc = np.zeros((32, 4))
+    for kb in range(K // 64):
+        tmp = np.zeros((32, 4))
+        for c in range(2):
+            A0, A1, B0, B1 = [], [], [], []
+            for lane in range(32):
+                g, t = lane >> 2, lane & 3
+                b0 = packed[g, kb * 32 + 16 * c + 4 * t: kb * 32 + 16 * c + 4 * t + 4]
+                b1 = packed[g + 8, kb * 32 + 16 * c + 4 * t: kb * 32 + 16 * c + 4 * t + 4]
+                A0.append((_pair(b0[0]), _pair(b1[0]), _pair(b0[1]), _pair(b1[1])))
+                A1.append((_pair(b0[2]), _pair(b1[2]), _pair(b0[3]), _pair(b1[3])))
+                kx = kb * 64 + 32 * c + 8 * t
+                B0.append(((x[g, kx], x[g, kx + 1]), (x[g, kx + 2], x[g, kx + 3])))
+                B1.append(((x[g, kx + 4], x[g, kx + 5]), (x[g, kx + 6], x[g, kx + 7])))
+            _mma(tmp, A0, B0)
+            _mma(tmp, A1, B1)
+        for lane in range(32):
+            g = lane >> 2
+            acc[lane] += tmp[lane] * [absmax[g, kb], absmax[g, kb], absmax[g + 8, kb], absmax[g + 8, kb]]
+    got = np.zeros((16, 8))
+    for lane in range(32):
+        g, t = lane >> 2, lane & 3
+        got[g, 2 * t], got[g, 2 * t + 1], got[g + 8, 2 * t], got[g + 8, 2 * t + 1] = acc[lane]
+    ref = W @ x.T
+    assert np.abs(got - ref).max() <= 1e-12 * np.abs(ref).max()
+
+
+@pytest.mark.parametrize("halves,tpr", [(2, 2), (1, 4)])
+def test_tensor_core_decoders_fill_the_swizzled_k_major_tile(halves, tpr):
+    """csrc/gemm_tc.cu decoders: thread dt decodes row dt / tpr of the tile (half
+    = row / 128) and its part dt % tpr of the 64-k block (32 / tpr packed bytes,
+    one 32-bit word = 8 elements = one 16-byte chunk), scales by the block's
+    absmax and stores chunk c of row ri at byte (ri / 8) * 1024 + (ri % 8) * 128
+    + ((c ^ (ri % 8)) * 16) of its half: read back through the same 128-byte
+    swizzle, the tile is the block's W rows."""
+    rows = 128 * halves
+    packed, absmax, W = _layer_rows(5, rows, 64)      # one 64-k block per row
+    tile = np.full(rows * 64, np.nan)                   # bf16 slots of the A stage
+    nchunks = 8 // tpr
+    for dt in range(512):
+        r, kq = dt // tpr, dt % tpr
+        half, ri = r >> 7, r & 127
+        src = packed[r, kq * (32 // tpr): (kq + 1) * (32 // tpr)]
+        for c in range(nchunks):
+            w = src[4 * c: 4 * c + 4]
+            vals = []
+            for byte in w:                               # decode4 on the low, then the high half-word
+                vals += [v * absmax[r, 0] for v in _pair(byte)]
+            chunk = kq * nchunks + c
+            base = half * 128 * 64 + (ri >> 3) * 512 + (ri & 7) * 64 + ((chunk ^ (ri & 7)) << 3)
+            assert np.isnan(tile[base:base + 8]).all(), "slot written twice"
+            tile[base:base + 8] = vals
+    assert not np.isnan(tile).any()
+    for r in range(rows):
+        half, ri = r >> 7, r & 127
+        for k in range(64):
+            addr = half * 128 * 64 + (ri >> 3) * 512 + (ri & 7) * 64 + (((k // 8) ^ (ri & 7)) << 3) + (k % 8)
+            assert tile[addr] == W[r, k]
