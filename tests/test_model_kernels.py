@@ -1,4 +1,5 @@
-"""CPU models of the index maps of the GPU kernels (regression pins).
+"""CPU models of the index maps of the GPU kernels (regression pins; the decode
+kernels' models are in test_model_decode_ring.py).
 
 Each model restates, in numpy and exact arithmetic, how a kernel's threads
 place data -- which packed bytes a thread decodes, where it stores them, which
@@ -46,43 +47,6 @@ def _layer_rows(seed, rows, K):
     # the definition, through the oracle's own unpacking (independent of _pair)
     W = CB[nf4.unpack_codes(packed).reshape(rows, K)] * np.repeat(absmax, 64, axis=1)
     return packed, absmax, W
-
-
-@pytest.mark.parametrize("K", [128, 192, 2880])
-def test_decode_span_fragment_mapping(K):
-    """csrc/decode.cu span_mma: thread (g, t) of a span (128 k) holds 16 packed
-    bytes of rows g and g+8 at byte 16t (all inside k-block 2 span + t/2), the
-    block's absmax multiplied into each decoded pair, MMA j taking bytes 2j and
-    2j+1 and x words 2j, 2j+1 of the thread's 32 k."""
-    packed, absmax, W = _layer_rows(1, 16, K)
-    rng = np.random.default_rng(2)
-    x = rng.standard_normal((8, K))
-    KB = K // 64
-    acc = np.zeros((32, 4))
-    for sp in range((KB + 1) // 2):
-        A = [[None] * 32 for _ in range(8)]
-        B = [[None] * 32 for _ in range(8)]
-        for lane in range(32):
-            g, t = lane >> 2, lane & 3
-            kb = 2 * sp + (t >> 1)
-            live = kb < KB
-            r0 = packed[g, sp * 64 + 16 * t: sp * 64 + 16 * t + 16] if live else np.zeros(16, np.uint8)
-            r1 = packed[g + 8, sp * 64 + 16 * t: sp * 64 + 16 * t + 16] if live else np.zeros(16, np.uint8)
-            a0 = absmax[g, kb] if live else 0.0
-            a1 = absmax[g + 8, kb] if live else 0.0
-            xs = x[g, sp * 128 + 32 * t: sp * 128 + 32 * t + 32] if live else np.zeros(32)
-            for j in range(8):
-                p = lambda r, i, a: tuple(v * a for v in _pair(r[i]))
-                A[j][lane] = (p(r0, 2 * j, a0), p(r1, 2 * j, a1), p(r0, 2 * j + 1, a0), p(r1, 2 * j + 1, a1))
-                B[j][lane] = ((xs[4 * j], xs[4 * j + 1]), (xs[4 * j + 2], xs[4 * j + 3]))
-        for j in range(8):
-            _mma(acc, A[j], B[j])
-    got = np.zeros((16, 8))
-    for lane in range(32):
-        g, t = lane >> 2, lane & 3
-        got[g, 2 * t], got[g, 2 * t + 1], got[g + 8, 2 * t], got[g + 8, 2 * t + 1] = acc[lane]
-    ref = W @ x.T
-    assert np.abs(got - ref).max() <= 1e-12 * np.abs(ref).max()
 
 
 def test_warp_mma_gemm_fragment_mapping():
