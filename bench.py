@@ -48,7 +48,11 @@ WORKLOADS = {
     "gptoss_m1": ("gptoss", 1), "gptoss_m8192": ("gptoss", 8192), "tiny_m64": ("tiny", 64),
 }
 DEFAULT_WORKLOAD = "olmoe_m1"
-DEFAULT_SWEEP = ("olmoe_m4", "olmoe_m8", "olmoe_m2048")
+# Every other workload of the table runs in the default sweep, so the JSON line
+# carries the prefill rows' (M >= 4096) tensor-core fractions and the gpt-oss
+# decode row beside the OLMoE ones.
+DEFAULT_SWEEP = ("olmoe_m4", "olmoe_m8", "olmoe_m2048", "qwen3_m4096", "qwen3_lora_m4096", "gptoss_m1",
+                 "gptoss_m8192")
 
 
 def load_peaks():
@@ -580,7 +584,12 @@ def main():
     sweep = []
     if not args.no_sweep and args.workload == DEFAULT_WORKLOAD:
         for name in DEFAULT_SWEEP:
-            r = measure(args, name, rank, world, dist, peaks, primary=False)
+            try:
+                r = measure(args, name, rank, world, dist, peaks, primary=False)
+            except Exception as exc:  # a failing sweep row is reported, the headline line still prints
+                sweep.append({"workload": name, "error": f"{type(exc).__name__}: {exc}"})
+                torch.cuda.empty_cache()
+                continue
             sweep.append({"workload": name, "value": r["value"], "ms_per_step": r["ms_per_step"],
                           "tflops": r["tflops"], "path": r["path"], "touched_experts_avg": r["touched_experts_avg"],
                           "roofline_frac": r["roofline"]["frac"] if r["roofline"] else None,
