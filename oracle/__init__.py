@@ -10,6 +10,8 @@ method fixes it: the scaled value ``w / absmax`` of the quantiser).
 Modules
 -------
 nf4      the 16-entry codebook, the blockwise stack quantiser, dequantisation
+fp4      the same blockwise storage with e2m1 codes scaled to [-1, 1] (the
+         pages' other 4-bit storage mode)
 routing  router top-k, the renormalised weights, the token/expert permutation
 moe      the grouped NF4 GEMM, the SwiGLU expert MLP with its optional LoRA
          delta, the weighted combine; a brute-force per-token form and a

@@ -144,7 +144,7 @@ def layer_backward(x: np.ndarray, logits: np.ndarray, ids: np.ndarray, stack: Ex
 
 def grouped_nf4_gemm_dgrad(dY: np.ndarray, row_index, offsets: np.ndarray, packed: np.ndarray,
                            absmax: np.ndarray, N: int, K: int, lora_A=None, lora_B=None,
-                           lora_scale: float = 0.0) -> np.ndarray:
+                           lora_scale: float = 0.0, quant: str = "nf4") -> np.ndarray:
     """The input gradient of the grouped NF4 GEMM, in one call over all groups.
 
     The forward row p is ``y_p = a_p . W_e^T (+ s (a_p . A_e^T) . B_e^T)``; for
@@ -154,11 +154,12 @@ def grouped_nf4_gemm_dgrad(dY: np.ndarray, row_index, offsets: np.ndarray, packe
 
     with W_e the dequantised [N, K] expert of the group e holding p (the
     frozen base is decoded again from the packed bytes, never kept), so the
-    result has K columns.  ``row_index=None`` means identity.  This is the
+    result has K columns.  ``row_index=None`` means identity; ``quant`` names
+    the storage of ``packed`` (``nf4`` or ``fp4``).  This is the
     single grouped dgrad launch the pages put in place of a per-expert decode
     loop (experts4bit-qlora 0.22.0, "Which training path?").
     """
-    from . import nf4
+    from . import moe
     dY = np.asarray(dY, dtype=np.float64)
     offsets = np.asarray(offsets, dtype=np.int64)
     E = offsets.size - 1
@@ -171,7 +172,7 @@ def grouped_nf4_gemm_dgrad(dY: np.ndarray, row_index, offsets: np.ndarray, packe
         lo, hi = offsets[e], offsets[e + 1]
         if hi == lo:
             continue
-        W = nf4.dequantize_expert(packed[e], absmax[e], (N, K))
+        W = moe.dequantize(quant, packed[e], absmax[e], (N, K))
         G = dY[idx[lo:hi]]
         d = G @ W
         if lora_A is not None and lora_B is not None:
@@ -232,16 +233,18 @@ def layer_backward_grouped(x: np.ndarray, logits: np.ndarray, ids: np.ndarray, s
     perm = np.asarray(perm, dtype=np.int64)
     tok = perm // k
     a = moe.grouped_nf4_gemm(x, tok, offsets, stack.gu_packed, stack.gu_absmax, 2 * I, H,
-                             stack.lora_A if lora else None, stack.lora_B if lora else None, s)
+                             stack.lora_A if lora else None, stack.lora_B if lora else None, s,
+                             quant=stack.quant)
     g, u = a[:, :I], a[:, I:]
     h = silu(g) * u
-    z = moe.grouped_nf4_gemm(h, None, offsets, stack.dn_packed, stack.dn_absmax, H, I)
+    z = moe.grouped_nf4_gemm(h, None, offsets, stack.dn_packed, stack.dn_absmax, H, I, quant=stack.quant)
     wp = w.reshape(-1)[perm]                       # routing weight of each grouped row
     dz = wp[:, None] * dout[tok]
-    dh = grouped_nf4_gemm_dgrad(dz, None, offsets, stack.dn_packed, stack.dn_absmax, H, I)
+    dh = grouped_nf4_gemm_dgrad(dz, None, offsets, stack.dn_packed, stack.dn_absmax, H, I, quant=stack.quant)
     da = np.concatenate([dh * u * silu_grad(g), dh * silu(g)], axis=1)
     dxg = grouped_nf4_gemm_dgrad(da, None, offsets, stack.gu_packed, stack.gu_absmax, 2 * I, H,
-                                 stack.lora_A if lora else None, stack.lora_B if lora else None, s)
+                                 stack.lora_A if lora else None, stack.lora_B if lora else None, s,
+                                 quant=stack.quant)
     dx = dxg[np.asarray(inv, dtype=np.int64)].reshape(M, k, H).sum(axis=1)
     dw = np.zeros(M * k, dtype=np.float64)
     dw[perm] = np.sum(dout[tok] * z, axis=1)

@@ -36,7 +36,14 @@ from typing import Optional
 
 import numpy as np
 
-from . import nf4
+from . import fp4, nf4
+
+QUANT_TYPES = {"nf4": nf4, "fp4": fp4}
+
+
+def dequantize(quant: str, packed_e, absmax_e, shape) -> np.ndarray:
+    """One expert's weights in float64 from its 4-bit storage (``nf4`` or ``fp4``)."""
+    return QUANT_TYPES[quant].dequantize_expert(packed_e, absmax_e, shape)
 
 
 def silu(z: np.ndarray) -> np.ndarray:
@@ -46,10 +53,11 @@ def silu(z: np.ndarray) -> np.ndarray:
 
 
 class ExpertStack:
-    """An NF4 fused stack pair with lazily dequantised float64 experts."""
+    """A 4-bit fused stack pair (NF4, or FP4 with ``quant="fp4"``) with lazily
+    dequantised float64 experts."""
 
     def __init__(self, gu_packed, gu_absmax, dn_packed, dn_absmax, E, H, I,
-                 lora_A=None, lora_B=None, lora_scale=0.0):
+                 lora_A=None, lora_B=None, lora_scale=0.0, quant="nf4"):
         self.gu_packed = np.asarray(gu_packed, dtype=np.uint8).reshape(E, -1)
         self.gu_absmax = np.asarray(gu_absmax, dtype=np.float32).reshape(E, -1)
         self.dn_packed = np.asarray(dn_packed, dtype=np.uint8).reshape(E, -1)
@@ -58,21 +66,24 @@ class ExpertStack:
         self.lora_A = None if lora_A is None else np.asarray(lora_A, dtype=np.float64)
         self.lora_B = None if lora_B is None else np.asarray(lora_B, dtype=np.float64)
         self.lora_scale = float(lora_scale)
+        if quant not in QUANT_TYPES:
+            raise ValueError(f"unknown storage type {quant!r}")
+        self.quant = quant
         self._gu = {}
         self._dn = {}
 
     def gate_up(self, e: int) -> np.ndarray:
         """Dequantised ``[2I, H]`` float64."""
         if e not in self._gu:
-            self._gu[e] = nf4.dequantize_expert(self.gu_packed[e], self.gu_absmax[e],
-                                                (2 * self.I, self.H))
+            self._gu[e] = dequantize(self.quant, self.gu_packed[e], self.gu_absmax[e],
+                                     (2 * self.I, self.H))
         return self._gu[e]
 
     def down(self, e: int) -> np.ndarray:
         """Dequantised ``[H, I]`` float64."""
         if e not in self._dn:
-            self._dn[e] = nf4.dequantize_expert(self.dn_packed[e], self.dn_absmax[e],
-                                                (self.H, self.I))
+            self._dn[e] = dequantize(self.quant, self.dn_packed[e], self.dn_absmax[e],
+                                     (self.H, self.I))
         return self._dn[e]
 
     def has_lora(self) -> bool:
@@ -111,12 +122,13 @@ def moe_forward_per_token(x: np.ndarray, ids: np.ndarray, w: np.ndarray,
 def grouped_nf4_gemm(A: np.ndarray, row_index: Optional[np.ndarray], offsets: np.ndarray,
                      packed: np.ndarray, absmax: np.ndarray, N: int, K: int,
                      lora_A=None, lora_B=None, lora_scale: float = 0.0,
-                     swiglu: bool = False) -> np.ndarray:
+                     swiglu: bool = False, quant: str = "nf4") -> np.ndarray:
     """One grouped GEMM over the groups ``[offsets[e], offsets[e+1])``.
 
     Row p of the result is ``A[row_index[p]] . W_e^T`` (plus the LoRA delta)
     for the group e holding p; with ``swiglu`` the result is
-    ``SiLU(y[:, :N/2]) * y[:, N/2:]``.  ``row_index=None`` means identity.
+    ``SiLU(y[:, :N/2]) * y[:, N/2:]``.  ``row_index=None`` means identity;
+    ``quant`` names the storage of ``packed`` (``nf4`` or ``fp4``).
     """
     A = np.asarray(A, dtype=np.float64)
     offsets = np.asarray(offsets, dtype=np.int64)
@@ -130,7 +142,7 @@ def grouped_nf4_gemm(A: np.ndarray, row_index: Optional[np.ndarray], offsets: np
         lo, hi = offsets[e], offsets[e + 1]
         if hi == lo:
             continue
-        W = nf4.dequantize_expert(packed[e], absmax[e], (N, K))
+        W = dequantize(quant, packed[e], absmax[e], (N, K))
         Xe = A[idx[lo:hi]]
         y = Xe @ W.T
         if lora_A is not None and lora_B is not None:
@@ -153,9 +165,9 @@ def moe_forward_grouped(x: np.ndarray, ids: np.ndarray, w: np.ndarray, offsets: 
                          2 * stack.I, stack.H,
                          stack.lora_A if stack.has_lora() else None,
                          stack.lora_B if stack.has_lora() else None,
-                         stack.lora_scale, swiglu=True)
+                         stack.lora_scale, swiglu=True, quant=stack.quant)
     z = grouped_nf4_gemm(h, None, offsets, stack.dn_packed, stack.dn_absmax,
-                         stack.H, stack.I)
+                         stack.H, stack.I, quant=stack.quant)
     zs = z[np.asarray(inv, dtype=np.int64)].reshape(M, k, stack.H)
     out = np.zeros((M, stack.H), dtype=np.float64)
     w = np.asarray(w, dtype=np.float64)
