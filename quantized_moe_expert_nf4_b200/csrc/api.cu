@@ -769,9 +769,9 @@ e4b_status e4b_moe_expert_forward_path(const uint16_t* x, int64_t M, const float
     set_path("forward.empty");
     return E4B_OK;
   }
-  const bool dec_ok = decode_supported(M, w->E, k, w->H, w->I);
-  if (path == E4B_PATH_DECODE && !dec_ok)
-    return fail(E4B_ERR_UNSUPPORTED, "the decode path takes at most 8 tokens (M=" + std::to_string(M) + ")");
+  const std::string dec_why = decode_unsupported_reason(M, w->E, k, w->H, w->I);
+  const bool dec_ok = dec_why.empty();
+  if (path == E4B_PATH_DECODE && !dec_ok) return fail(E4B_ERR_UNSUPPORTED, dec_why);
   if (path == E4B_PATH_DECODE || (path == E4B_PATH_AUTO && dec_ok)) {
     DecodeArgs a{x, M, router_logits, k, renormalize != 0, w, out, workspace};
     cudaError_t err = launch_decode_forward(a, stream);

@@ -29,6 +29,7 @@
 // are staged 16 bytes apart from the next row's bank so that the fragment loads
 // are conflict-free.
 #include <algorithm>
+#include <string>
 
 #include "async.cuh"
 #include "common.cuh"
@@ -775,14 +776,24 @@ Stages plan_stages(int M, int k, int E, int H, int I, int r, size_t limit) {
 
 }  // namespace
 
-bool decode_supported(int64_t M, int64_t E, int k, int64_t H, int64_t I) {
-  if (M < 1 || M > kMaxM || k > 32 || E > 512 || H > 128 * kMath * kMaxKBW) return false;
+std::string decode_unsupported_reason(int64_t M, int64_t E, int k, int64_t H, int64_t I) {
+  if (M < 1 || M > kMaxM) return "the decode path takes 1 to " + std::to_string(kMaxM) + " tokens (M=" + std::to_string(M) + ")";
+  if (k > 32) return "the decode path takes k <= 32 (k=" + std::to_string(k) + ")";
+  if (E > 512) return "the decode path takes at most 512 experts (E=" + std::to_string(E) + ")";
+  if (H > 128 * kMath * kMaxKBW)
+    return "the decode path takes H <= " + std::to_string(128 * kMath * kMaxKBW) + " (H=" + std::to_string(H) + ")";
   DeviceInfo di;
-  if (device_info(&di) != cudaSuccess) return false;
+  if (device_info(&di) != cudaSuccess) return "device query failed";
   const size_t lim = di.smem_optin - 1024;  // leave room for the kernels' static shared memory
   const Stages st = plan_stages(static_cast<int>(M), k, static_cast<int>(E), static_cast<int>(H),
                                 static_cast<int>(I), 16, lim);
-  return st.a >= kMinStages && st.b >= kMinStages;
+  if (st.a < kMinStages || st.b < kMinStages)
+    return "the decode kernels' shared-memory rings do not fit this shape";
+  return "";
+}
+
+bool decode_supported(int64_t M, int64_t E, int k, int64_t H, int64_t I) {
+  return decode_unsupported_reason(M, E, k, H, I).empty();
 }
 
 size_t decode_workspace_bytes(int64_t M, int64_t E, int k, int64_t H, int64_t I, int r) {

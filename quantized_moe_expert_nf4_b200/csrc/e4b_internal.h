@@ -207,6 +207,8 @@ struct DecodeArgs {
   void* workspace;
 };
 bool decode_supported(int64_t M, int64_t E, int k, int64_t H, int64_t I);
+// Why the decode kernels cannot take this shape ("" when they can).
+std::string decode_unsupported_reason(int64_t M, int64_t E, int k, int64_t H, int64_t I);
 size_t decode_workspace_bytes(int64_t M, int64_t E, int k, int64_t H, int64_t I, int r);
 cudaError_t launch_decode_forward(const DecodeArgs& a, cudaStream_t stream);
 

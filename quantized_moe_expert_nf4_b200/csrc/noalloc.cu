@@ -85,8 +85,8 @@ extern "C" e4b_status e4b_moe_expert_forward_decode_noalloc(const uint16_t* x, i
   cudaError_t err = device_info(&di);
   if (err != cudaSuccess) return nofail(E4B_ERR_CUDA, std::string("device query: ") + cudaGetErrorString(err));
   if (di.major != 10 || di.minor != 0) return nofail(E4B_ERR_UNSUPPORTED, "libe4b is built for sm_100a (B200)");
-  if (!decode_supported(M, w->E, k, w->H, w->I))
-    return nofail(E4B_ERR_UNSUPPORTED, "shape not supported by the decode kernels (shared-memory limit or E > 512)");
+  if (const std::string why = decode_unsupported_reason(M, w->E, k, w->H, w->I); !why.empty())
+    return nofail(E4B_ERR_UNSUPPORTED, why);
   if (decode_workspace_bytes(M, w->E, k, w->H, w->I, w->lora_A ? w->lora_r : 0) > kNoAllocBytes)
     return nofail(E4B_ERR_UNSUPPORTED, "decode scratch layout exceeds the static array");
   void* scratch = nullptr;

@@ -214,3 +214,39 @@ def test_forward_replays_bit_identically_from_a_cuda_graph(M):
     g.replay()
     torch.cuda.synchronize()
     assert torch.equal(out.view(torch.int16), eager.view(torch.int16))
+
+
+LIMITS = [
+    # the largest hidden size the decode kernels take (two spans of 128 k per warp)
+    ("h4096", workloads.small_config("h4096", E=8, H=4096, I=128, k=2), 8),
+    # the largest expert count they take, every token routed to 8 of 512
+    ("e512", workloads.small_config("e512", E=512, H=128, I=64, k=8, routing="zipf"), 8),
+]
+
+
+@pytest.mark.parametrize("name,cfg,M", LIMITS, ids=[c[0] for c in LIMITS])
+def test_forward_decode_at_its_size_limits(name, cfg, M):
+    require_gpu()
+    layer = synthetic.make_device_layer(cfg)
+    x, logits = synthetic.inputs(cfg, M)
+    out, p = _forward(layer, x, logits, e4b.E4B_PATH_DECODE)
+    assert p == "forward.decode"
+    ref = _oracle_tokens(cfg, x, logits, np.arange(M))
+    assert_close_layer(bf16_to_f64(out), ref, f"{name} M={M} {p}")
+
+
+@pytest.mark.parametrize("name,cfg,why", [
+    ("h4160", workloads.small_config("h4160", E=4, H=4160, I=64, k=2), "H <= 4096"),
+    ("e513", workloads.small_config("e513", E=513, H=64, I=64, k=2), "at most 512 experts"),
+], ids=["h4160", "e513"])
+def test_forward_past_the_decode_limits_runs_grouped(name, cfg, why):
+    """One step past a decode limit: a forced decode call is refused with the
+    limit named; the automatic choice runs the grouped path and matches the oracle."""
+    require_gpu()
+    layer = synthetic.make_device_layer(cfg)
+    x, logits = synthetic.inputs(cfg, 4)
+    with pytest.raises(e4b.E4BError, match=why):
+        _forward(layer, x, logits, e4b.E4B_PATH_DECODE)
+    out, p = _forward(layer, x, logits)
+    assert p == "forward.grouped"
+    assert_close_layer(bf16_to_f64(out), _oracle_tokens(cfg, x, logits, np.arange(4)), f"{name} {p}")
