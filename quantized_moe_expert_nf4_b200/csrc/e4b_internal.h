@@ -49,6 +49,20 @@ struct QuantTables {
 };
 QuantTables quant_tables(int quant);
 
+// The quantiser kernel's lookup of a level: 128 cells of width 1/64 over s in
+// [-1, 1], each widened by kQuantCellSlack on both sides.  Cell c holds the one
+// decision threshold inside it (+inf if none; both codebooks' thresholds are
+// at least 0.079 apart, wider than a cell) and the codes written below and at
+// or above it.  Any s in the widened cell gets its code from one comparison.
+constexpr int kQuantCells = 128;
+constexpr double kQuantCellSlack = 1e-5;
+struct QuantCellTable {
+  uint2 cell[kQuantCells];  // x: threshold (float bits), y: code below | code at or above << 4
+  uint32_t zero_code;
+  int ok;                   // 0 if some widened cell held two thresholds
+};
+QuantCellTable quant_cell_table(int quant);
+
 cudaError_t launch_quantize(const void* W, bool bf16, int64_t nblocks, int quant, uint8_t* packed,
                             float* absmax, cudaStream_t stream);
 

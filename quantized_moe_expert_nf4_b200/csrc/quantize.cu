@@ -16,11 +16,17 @@
 // the code written is the level's code (NF4: the level itself; FP4: the
 // sign-magnitude code, +0 for zero); a = 0 gives the code of 0.
 //
+// The kernel finds the level of s by one lookup in a table of 128 cells over
+// [-1, 1] (the threshold inside the cell and the codes on either side of it)
+// and decides most weights on w * fl32(1 / a), keeping the exact division for
+// the few that fall within 2^-22 of a threshold (see code_of).
+//
 // HBM-bound: 4 B (fp32) or 2 B (bf16) read + 0.5625 B written per weight.  One
 // warp handles 8 blocks (512 weights) per step with 16-byte loads; each block
 // is reduced by a 16-lane shuffle tree.
 #include <algorithm>
 #include <cmath>
+#include <cstring>
 #include <limits>
 
 #include "common.cuh"
@@ -69,16 +75,47 @@ QuantTables quant_tables(int quant) {
   return qt;
 }
 
+QuantCellTable quant_cell_table(int quant) {
+  const QuantTables qt = quant_tables(quant);
+  int nthr = 0;
+  while (nthr < 16 && std::isfinite(qt.t[nthr])) ++nthr;
+  QuantCellTable ct{};
+  ct.ok = 1;
+  for (int c = 0; c < kQuantCells; ++c) {
+    const double lo = c / 64.0 - 1.0 - kQuantCellSlack, hi = (c + 1) / 64.0 - 1.0 + kQuantCellSlack;
+    int base = 0;  // thresholds at or below every s of the cell
+    while (base < nthr && static_cast<double>(qt.t[base]) <= lo) ++base;
+    float t = std::numeric_limits<float>::infinity();
+    if (base < nthr && static_cast<double>(qt.t[base]) <= hi) {
+      t = qt.t[base];
+      if (base + 1 < nthr && static_cast<double>(qt.t[base + 1]) <= hi) ct.ok = 0;
+    }
+    uint32_t tb;
+    std::memcpy(&tb, &t, sizeof tb);
+    ct.cell[c] = make_uint2(tb, qt.code[base] | (qt.code[std::min(base + 1, nthr)] << 4));
+  }
+  ct.zero_code = qt.zero_code;
+  return ct;
+}
+
 namespace {
 
-// Level of s: count of thresholds <= s, by a 4-step branchless binary search
-// over the ascending table in shared memory (T[15] = +inf).
-__device__ __forceinline__ uint32_t level_of(float s, const float* t) {
-  uint32_t q = (s >= t[7]) ? 8u : 0u;
-  q += (s >= t[q + 3]) ? 4u : 0u;
-  q += (s >= t[q + 1]) ? 2u : 0u;
-  q += (s >= t[q]) ? 1u : 0u;
-  return q;
+// The code of weight w in a block with absmax a > 0.  The method's scaled value
+// is s = fl32(w / a) (one IEEE division).  For a in [2^-125, 2^125] the kernel
+// first forms s' = fl32(w * y) with y = fl32(1 / a) computed once per block:
+// |s' - w/a| <= 2^-23 |w/a| + 2^-48 and |s - w/a| <= 2^-25, so |s' - s| < 2^-22
+// for |w| <= a.  When s' lies farther than 2^-22 from the cell's threshold
+// (tested on the rounded difference, which only errs towards the exact path),
+// s and s' fall on the same side of it and s' decides the code; otherwise, and
+// for absmax outside that range, the code is decided on s itself.  The cell
+// index is only a hint: every s and s' of a cell lies inside its widened range.
+__device__ __forceinline__ uint32_t code_of(float w, float a, float y, bool fast, const uint2* cells) {
+  float s = fast ? __fmul_rn(w, y) : __fdiv_rn(w, a);
+  const int c = min(max(__float2int_rd((s + 1.0f) * 64.0f), 0), kQuantCells - 1);
+  const uint2 e = cells[c];
+  const float t = __uint_as_float(e.x);
+  if (fast && !(fabsf(__fsub_rn(s, t)) > 0x1p-22f)) s = __fdiv_rn(w, a);
+  return (s >= t ? e.y >> 4 : e.y) & 15u;
 }
 
 template <bool kBf16>
@@ -101,13 +138,9 @@ __device__ __forceinline__ void load4(const void* W, int64_t elem, float v[4]) {
 template <bool kBf16>
 __global__ void __launch_bounds__(256) nf4_quantize_kernel(const void* __restrict__ W, int64_t nblocks,
                                                            uint8_t* __restrict__ packed,
-                                                           float* __restrict__ absmax, QuantTables qt) {
-  __shared__ float t_s[16];
-  __shared__ uint32_t c_s[16];
-  if (threadIdx.x < 16) {
-    t_s[threadIdx.x] = qt.t[threadIdx.x];
-    c_s[threadIdx.x] = qt.code[threadIdx.x];
-  }
+                                                           float* __restrict__ absmax, QuantCellTable ct) {
+  __shared__ uint2 cells_s[kQuantCells];
+  for (int i = threadIdx.x; i < kQuantCells; i += blockDim.x) cells_s[i] = ct.cell[i];
   __syncthreads();
 
   const int lane = threadIdx.x & 31;
@@ -135,12 +168,11 @@ __global__ void __launch_bounds__(256) nf4_quantize_kernel(const void* __restric
       float m = fmaxf(fmaxf(fabsf(v[i][0]), fabsf(v[i][1])), fmaxf(fabsf(v[i][2]), fabsf(v[i][3])));
 #pragma unroll
       for (int o = 8; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      const bool fast = m >= 0x1p-125f && m <= 0x1p125f;
+      const float y = __frcp_rn(m);  // IEEE reciprocal, used on the fast path only
       uint32_t q[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        // IEEE division (no fast-math in this file): bit-exact fl32(w / a).
-        q[j] = (m > 0.0f) ? c_s[level_of(__fdiv_rn(v[i][j], m), t_s)] : qt.zero_code;
-      }
+      for (int j = 0; j < 4; ++j) q[j] = (m > 0.0f) ? code_of(v[i][j], m, y, fast, cells_s) : ct.zero_code;
       const int64_t blk = g * 8 + 2 * i + (lane >> 4);
       const int64_t elem = g * 512 + 128 * i + 4 * lane;
       if (valid[i]) {
@@ -165,12 +197,13 @@ cudaError_t launch_quantize(const void* W, bool bf16, int64_t nblocks, int quant
   const int64_t want = (ngroups + (threads / 32) - 1) / (threads / 32);
   const int64_t cap = static_cast<int64_t>(di.sm_count) * 8;
   const int grid = static_cast<int>(want < cap ? want : cap);
-  const QuantTables qt = quant_tables(quant);
+  const QuantCellTable ct = quant_cell_table(quant);
+  if (!ct.ok) return cudaErrorInvalidValue;
   LaunchScope ls("quantize", stream);
   if (bf16)
-    nf4_quantize_kernel<true><<<grid, threads, 0, stream>>>(W, nblocks, packed, absmax, qt);
+    nf4_quantize_kernel<true><<<grid, threads, 0, stream>>>(W, nblocks, packed, absmax, ct);
   else
-    nf4_quantize_kernel<false><<<grid, threads, 0, stream>>>(W, nblocks, packed, absmax, qt);
+    nf4_quantize_kernel<false><<<grid, threads, 0, stream>>>(W, nblocks, packed, absmax, ct);
   return cudaGetLastError();
 }
 

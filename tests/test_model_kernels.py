@@ -159,3 +159,91 @@ def test_tensor_core_byte_permute_decoder_is_a_table_lookup(table):
         n = [g & 15, (g >> 4) & 15, (g >> 8) & 15, (g >> 12) & 15]
         assert w0 == bits[n[1]] | (bits[n[0]] << 16), hex(g)
         assert w1 == bits[n[3]] | (bits[n[2]] << 16), hex(g)
+
+
+def _quant_cell_table(cb):
+    """csrc/quantize.cu quant_cell_table: levels = distinct codebook values
+    ascending (each with its lowest code), thresholds = smallest float above
+    each exact midpoint, and per cell c of [c/64 - 1, (c+1)/64 - 1] widened by
+    1e-5 the one threshold inside it (+inf if none) with the codes below and at
+    or above it."""
+    vals, codes = [], []
+    for c in range(16):
+        v = float(cb[c]) + 0.0
+        if v not in vals:
+            vals.append(v)
+            codes.append(c)
+    order = np.argsort(vals, kind="stable")
+    vals = [vals[i] for i in order]
+    codes = [codes[i] for i in order]
+    T = []
+    for lv in range(len(vals) - 1):
+        mid = (vals[lv] + vals[lv + 1]) / 2
+        f = np.float32(mid)
+        T.append(float(f if float(f) > mid else np.nextafter(f, np.float32(np.inf))))
+    cells = []
+    for c in range(128):
+        lo, hi = c / 64.0 - 1.0 - 1e-5, (c + 1) / 64.0 - 1.0 + 1e-5
+        base = sum(1 for t in T if t <= lo)
+        inside = [t for t in T if lo < t <= hi]
+        assert len(inside) <= 1, "two thresholds in one cell"
+        cells.append((inside[0] if inside else np.inf, codes[base], codes[min(base + 1, len(vals) - 1)]))
+    return cells
+
+
+def _kernel_codes(w, a, cells):
+    """csrc/quantize.cu code_of for every (w, a): s' = fl32(w * fl32(1/a)) for
+    absmax in [2^-125, 2^125], the cell of s', and the exact fl32(w / a) when
+    s' lies within 2^-22 of the cell's threshold (or the absmax is outside)."""
+    f32 = np.float32
+    t_tab = np.array([c[0] for c in cells], f32)
+    lo_tab = np.array([c[1] for c in cells])
+    hi_tab = np.array([c[2] for c in cells])
+    with np.errstate(all="ignore"):
+        fast = (a >= f32(2.0 ** -125)) & (a <= f32(2.0 ** 125))
+        exact = (w / a).astype(f32)
+        s = np.where(fast, (w * (f32(1) / a).astype(f32)).astype(f32), exact)
+        c = np.clip(np.floor((s + f32(1)).astype(f32) * f32(64)).astype(np.int64), 0, 127)
+        t = t_tab[c]
+        near = fast & ~(np.abs((s - t).astype(f32)) > f32(2.0 ** -22))
+        s = np.where(near, exact, s)
+    return np.where(s >= t, hi_tab[c], lo_tab[c]).astype(np.uint8), int(near.sum())
+
+
+@pytest.mark.parametrize("table", ["nf4", "fp4"])
+def test_quantiser_cell_lookup_and_reciprocal_path_match_the_oracle(table):
+    """The quantiser kernel's decision -- one cell lookup, the weight scaled by
+    the block's reciprocal unless it lands within 2^-22 of the cell's threshold
+    -- equals the oracle's code of fl32(w / a), on random weights, on every
+    decision point times random absmax (and 3 floats either side), and on
+    |w| = a, zeros and subnormal absmax."""
+    from oracle import fp4
+    mod = nf4 if table == "nf4" else fp4
+    cells = _quant_cell_table(mod.codebook_f64())
+    rng = np.random.default_rng(11)
+    f32 = np.float32
+    n = 200_000
+    fallbacks = 0
+    for kind in range(3):
+        a = (rng.uniform(1, 2, n) * 2.0 ** rng.integers(-40, 40, n)).astype(f32)
+        if kind == 0:
+            w = (rng.uniform(-1, 1, n) * a).astype(f32)
+        elif kind == 1:
+            w = (rng.choice(mod.midpoints(), n) * a.astype(np.float64)).astype(f32)
+            k = rng.integers(-3, 4, n)
+            for step in range(3):
+                w = np.where(k > step, np.nextafter(w, f32(np.inf)), w)
+                w = np.where(k < -step, np.nextafter(w, f32(-np.inf)), w)
+        else:
+            tiny = (rng.uniform(1, 2, n) * 2.0 ** rng.integers(-149, -120, n)).astype(f32)
+            a = np.where(rng.random(n) < 0.2, tiny, a).astype(f32)
+            a = np.where(a == 0, f32(1e-45), a).astype(f32)
+            r = rng.random(n)
+            w = np.where(r < 0.25, a, np.where(r < 0.5, -a, (rng.uniform(-1, 1, n) * a).astype(f32))).astype(f32)
+            w = np.where(rng.random(n) < 0.05, f32(0), w).astype(f32)
+        got, nf = _kernel_codes(w, a, cells)
+        fallbacks += nf
+        with np.errstate(all="ignore"):
+            want = mod.code_of_scaled((w / a).astype(f32))
+        assert np.array_equal(got, want), kind
+    assert fallbacks > 0   # the exact path was exercised
