@@ -523,8 +523,8 @@ def measure(args, name, rank, world, dist, peaks, primary):
 NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 
 
-def time_quantize(cfg, dev, reps=3):
-    """Load-time step, timed apart from the forward: e4b_nf4_quantize_stack on the
+def time_quantize(cfg, dev, reps=3, storage="nf4"):
+    """Load-time step, timed apart from the forward: e4b_quantize_stack on the
     layer's whole gate_up stack from fp32 ([E, 2I, H]); HBM-bound (4 B read +
     0.5 + 4/64 B written per weight)."""
     import torch
@@ -535,20 +535,75 @@ def time_quantize(cfg, dev, reps=3):
     n = W.numel()
     packed = torch.empty(n // 2, dtype=torch.uint8, device=dev)
     absmax = torch.empty(n // 64, dtype=torch.float32, device=dev)
-    e4b.e4b_nf4_quantize_stack(W, packed, absmax)
+    qt = STORAGE[storage]
+    e4b.e4b_quantize_stack(W, packed, absmax, qt)
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
     for _ in range(reps):
-        e4b.e4b_nf4_quantize_stack(W, packed, absmax)
+        e4b.e4b_quantize_stack(W, packed, absmax, qt)
     b.record()
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / reps
     nbytes = n * (4 + 0.5 + 4.0 / 64)
     del W, packed, absmax
     torch.cuda.empty_cache()
-    return {"stack": f"gate_up [{cfg.E}, {2 * cfg.I}, {cfg.H}] fp32", "ms": ms, "bytes": nbytes,
-            "GB_per_s": nbytes / (ms * 1e-3) / 1e9}
+    return {"stack": f"gate_up [{cfg.E}, {2 * cfg.I}, {cfg.H}] fp32", "storage": storage, "ms": ms,
+            "bytes": nbytes, "GB_per_s": nbytes / (ms * 1e-3) / 1e9}
+
+
+MXFP4_WORKLOAD = "gptoss_m8192"   # released MXFP4 experts: gpt-oss-shaped gate_up, prefill routing
+
+
+def time_mxfp4(name, dev, steps=5, warmup=2):
+    """The grouped GEMM straight from MXFP4 bytes (e4b_grouped_mxfp4_gemm) on the
+    gate_up projection of the workload's layer shape: the routed rows of the
+    workload's own routing (e4b_moe_route_permute), seeded random e2m1 codes and
+    e8m0 scales around 2^0, SwiGLU epilogue, bf16 out.  Algorithmic FLOPs
+    2*S*2I*H; timed apart from the forward with CUDA events on its stream."""
+    import torch
+
+    from quantized_moe_expert_nf4_b200 import e4b, synthetic
+
+    cfgname, M, _ = workload(name)
+    cfg = workloads.CONFIGS[cfgname]
+    E, H, I, k = cfg.E, cfg.H, cfg.I, cfg.k
+    S = M * k
+    x, logits = synthetic.inputs(cfg, M, device=dev)
+    ids = torch.empty((M, k), dtype=torch.int32, device=dev)
+    w = torch.empty((M, k), dtype=torch.float32, device=dev)
+    offs = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(S, dtype=torch.int32, device=dev)
+    inv = torch.empty(S, dtype=torch.int32, device=dev)
+    rws = e4b.workspace(e4b.e4b_moe_route_permute_workspace_size(M, E, k), dev)
+    e4b.e4b_moe_route_permute(logits, k, True, ids, w, offs, perm, inv, rws)
+    row_token = torch.div(perm, k, rounding_mode="floor").to(torch.int32)
+    g = torch.Generator(device=dev)
+    g.manual_seed(11)
+    N, K = 2 * I, H
+    blocks = torch.randint(0, 256, (E, N * K // 2), generator=g, device=dev, dtype=torch.uint8)
+    scales = torch.randint(124, 131, (E, N * K // 32), generator=g, device=dev, dtype=torch.uint8)
+    out = torch.empty((S, I), dtype=torch.bfloat16, device=dev)
+
+    def call():
+        e4b.e4b_grouped_mxfp4_gemm(x, row_token, offs, S, blocks, scales, N, K, out, e4b.E4B_EPI_SWIGLU)
+
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        call()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    flops = 2.0 * S * N * K
+    res = {"workload": name, "projection": f"gate_up [{E}, {N}, {K}] MXFP4", "routed_rows": S, "ms": ms,
+           "tflops": flops / (ms * 1e-3) / 1e12, "algorithmic_flops": flops, "path": e4b.last_path()}
+    del x, logits, ids, w, offs, perm, inv, rws, row_token, blocks, scales, out
+    torch.cuda.empty_cache()
+    return res
 
 
 BACKWARD_WORKLOAD = "qwen3_lora_m4096"   # the pages' training shape: Qwen3-MoE-shaped layer with per-expert LoRA
@@ -620,6 +675,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end host-buffer pass")
     ap.add_argument("--no-kernel-timing", action="store_true", help="skip the per-kernel event pass")
     ap.add_argument("--no-backward", action="store_true", help="skip the layer-backward timing")
+    ap.add_argument("--no-mxfp4", action="store_true", help="skip the MXFP4 grouped-GEMM timing")
     ap.add_argument("--replicas", type=int, default=0, help="layer replicas (0: enough to exceed L2 4x)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -672,9 +728,19 @@ def main():
                           "clocks": r["clocks"]})
     quant = None
     bwd = None
+    mx = None
     if rank == 0 and world == 1:
         quant = time_quantize(cfg, f"cuda:{local}")
         quant["frac_hbm"] = quant["GB_per_s"] / peaks["hbm_gbs"]
+        q4 = time_quantize(cfg, f"cuda:{local}", storage="fp4")
+        quant["fp4"] = {"GB_per_s": q4["GB_per_s"], "ms": q4["ms"], "frac_hbm": q4["GB_per_s"] / peaks["hbm_gbs"]}
+        if not args.no_mxfp4:
+            try:
+                mx = time_mxfp4(MXFP4_WORKLOAD, f"cuda:{local}")
+                mx["frac_tensor"] = mx["tflops"] / peaks["bf16_tflops"]
+            except Exception as exc:  # reported, the headline line still prints
+                mx = {"workload": MXFP4_WORKLOAD, "error": f"{type(exc).__name__}: {exc}"}
+                torch.cuda.empty_cache()
         if not args.no_backward:
             bwd = time_backward(BACKWARD_WORKLOAD, f"cuda:{local}")
             bwd["frac_tensor"] = bwd["tflops"] / peaks["bf16_tflops"]
@@ -702,6 +768,7 @@ def main():
             "gpu_launches": main_res["launches_per_step"] * args.steps,
             "quantize": quant,
             "backward": bwd,
+            "mxfp4_gemm": mx,
             "sweep": sweep,
         }
         print(json.dumps(line), flush=True)
