@@ -584,9 +584,10 @@ def time_mxfp4(name, dev, steps=5, warmup=2):
     blocks = torch.randint(0, 256, (E, N * K // 2), generator=g, device=dev, dtype=torch.uint8)
     scales = torch.randint(124, 131, (E, N * K // 32), generator=g, device=dev, dtype=torch.uint8)
     out = torch.empty((S, I), dtype=torch.bfloat16, device=dev)
+    ws = e4b.workspace(e4b.e4b_grouped_mxfp4_gemm_workspace_size(S, N, K), dev)
 
     def call():
-        e4b.e4b_grouped_mxfp4_gemm(x, row_token, offs, S, blocks, scales, N, K, out, e4b.E4B_EPI_SWIGLU)
+        e4b.e4b_grouped_mxfp4_gemm(x, row_token, offs, S, blocks, scales, N, K, out, e4b.E4B_EPI_SWIGLU, ws)
 
     for _ in range(warmup):
         call()
@@ -601,7 +602,7 @@ def time_mxfp4(name, dev, steps=5, warmup=2):
     flops = 2.0 * S * N * K
     res = {"workload": name, "projection": f"gate_up [{E}, {N}, {K}] MXFP4", "routed_rows": S, "ms": ms,
            "tflops": flops / (ms * 1e-3) / 1e12, "algorithmic_flops": flops, "path": e4b.last_path()}
-    del x, logits, ids, w, offs, perm, inv, rws, row_token, blocks, scales, out
+    del x, logits, ids, w, offs, perm, inv, rws, row_token, blocks, scales, out, ws
     torch.cuda.empty_cache()
     return res
 

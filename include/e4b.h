@@ -58,7 +58,7 @@
 extern "C" {
 #endif
 
-#define E4B_VERSION 2
+#define E4B_VERSION 3
 
 #if defined(__GNUC__)
 #define E4B_API __attribute__((visibility("default")))
@@ -345,13 +345,21 @@ E4B_API e4b_status e4b_grouped_lora_grads(const uint16_t* x, int64_t x_rows, int
  *           e2m1 = sign (bit 3), exponent (bits 2-1, bias 1), mantissa (bit 0);
  *   scales  [E, N*K/32] uint8: one e8m0 byte per 32 consecutive elements of a
  *           row; 255 is NaN and makes its block NaN.
- * Requires K % 64 == 0, N % 64 == 0.  No workspace (nothing waits).
+ * Requires K % 64 == 0, N % 64 == 0.
+ * workspace  e4b_grouped_mxfp4_gemm_workspace_size() bytes: an error word and
+ *            room for the routed rows gathered in order (total_rows x K bf16),
+ *            which the tensor-core kernel (512 routed rows and more) reads as
+ *            contiguous tiles; the warp-MMA kernel below uses neither.
+ * Each e2m1 value and each scale is exact in bf16, so the products with the
+ * bf16 operand rows are the GEMM's only roundings (fp32 accumulation).
  */
+E4B_API size_t e4b_grouped_mxfp4_gemm_workspace_size(int64_t total_rows, int64_t N, int64_t K);
 E4B_API e4b_status e4b_grouped_mxfp4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda,
                                   const int32_t* row_index, const int32_t* expert_offsets,
                                   int64_t E, int64_t total_rows, const uint8_t* blocks,
                                   const uint8_t* scales, int64_t N, int64_t K, e4b_epilogue epi,
-                                  void* out, e4b_dtype out_dtype, e4b_stream stream);
+                                  void* out, e4b_dtype out_dtype, void* workspace,
+                                  size_t workspace_bytes, e4b_stream stream);
 
 /* The two packed stacks of one MoE layer (device pointers), plus its adapter. */
 typedef struct {

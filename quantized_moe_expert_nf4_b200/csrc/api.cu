@@ -617,10 +617,17 @@ e4b_status e4b_grouped_lora_grads(const uint16_t* x, int64_t x_rows, int64_t ldx
   return E4B_OK;
 }
 
+size_t e4b_grouped_mxfp4_gemm_workspace_size(int64_t total_rows, int64_t N, int64_t K) {
+  (void)N;
+  if (total_rows < 0 || K < 0) return 0;
+  return gemm_workspace_bytes(total_rows, K, 0);
+}
+
 e4b_status e4b_grouped_mxfp4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda, const int32_t* row_index,
                                   const int32_t* expert_offsets, int64_t E, int64_t total_rows,
                                   const uint8_t* blocks, const uint8_t* scales, int64_t N, int64_t K,
-                                  e4b_epilogue epi, void* out, e4b_dtype out_dtype, e4b_stream stream) {
+                                  e4b_epilogue epi, void* out, e4b_dtype out_dtype, void* workspace,
+                                  size_t workspace_bytes, e4b_stream stream) {
   begin_call();
   if (E < 1 || E > 65536) return fail(E4B_ERR_INVALID_ARGUMENT, "E must be in [1, 65536]");
   if (total_rows < 0 || a_rows < 0) return fail(E4B_ERR_INVALID_ARGUMENT, "total_rows and a_rows must be >= 0");
@@ -635,6 +642,9 @@ e4b_status e4b_grouped_mxfp4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda
   if (total_rows > INT32_MAX) return fail(E4B_ERR_UNSUPPORTED, "total_rows exceeds int32");
   if ((A && !aligned16(A)) || !aligned16(blocks) || (out && !aligned16(out)))
     return fail(E4B_ERR_INVALID_ARGUMENT, "A, blocks and out must be 16-byte aligned");
+  if (e4b_status s = check_workspace("mxfp4 gemm", gemm_workspace_bytes(total_rows, K, 0), workspace, workspace_bytes);
+      s != E4B_OK)
+    return s;
   if (e4b_status s = check_device(); s != E4B_OK) return s;
   if (total_rows == 0) {
     set_path("mxfp4.empty");
@@ -655,9 +665,30 @@ e4b_status e4b_grouped_mxfp4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda
   m.epi = epi;
   m.out = out;
   m.out_bf16 = out_dtype == E4B_BF16;
-  cudaError_t err = launch_grouped_mxfp4_gemm(m, reinterpret_cast<cudaStream_t>(stream));
+  GemmArgs g{};
+  g.A = A;
+  g.a_rows = a_rows;
+  g.lda = lda;
+  g.row_index = row_index;
+  g.offsets = expert_offsets;
+  g.E = static_cast<int>(E);
+  g.total_rows = total_rows;
+  g.packed = blocks;
+  g.mx_scales = scales;
+  g.quant = kQuantMxfp4;
+  g.N = static_cast<int>(N);
+  g.K = static_cast<int>(K);
+  g.err = static_cast<int*>(workspace);
+  g.a_gathered = row_index ? reinterpret_cast<uint16_t*>(static_cast<char*>(workspace) +
+                                                         gemm_workspace_gather_offset(total_rows, 0))
+                           : nullptr;
+  g.epi = epi;
+  g.out = out;
+  g.out_bf16 = out_dtype == E4B_BF16;
+  const char* path = "";
+  cudaError_t err = launch_grouped_mxfp4(g, m, reinterpret_cast<cudaStream_t>(stream), &path);
   if (err != cudaSuccess) return cuda_fail(err, "grouped mxfp4 gemm launch");
-  set_path(epi == E4B_EPI_SWIGLU ? "mxfp4.mma.swiglu" : "mxfp4.mma");
+  set_path(path);
   return E4B_OK;
 }
 

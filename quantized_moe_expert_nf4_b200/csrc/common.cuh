@@ -24,11 +24,18 @@
 
 namespace e4b {
 
-// Indexed by e4b_quant_type: [0] NF4, [1] FP4.
-static __device__ __constant__ float kCodebooksDev[2][16] = {{E4B_NF4_CODEBOOK_VALUES}, {E4B_FP4_CODEBOOK_VALUES}};
+// The e2m1 element values themselves (MXFP4 codes, before their e8m0 block scale).
+#define E4B_E2M1_VALUES \
+  0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f, -0.0f, -0.5f, -1.0f, -1.5f, -2.0f, -3.0f, -4.0f, -6.0f
 
-// Entry c (0..15) of the codebook of storage type `quant` (0 NF4, any other value FP4).
-__device__ __forceinline__ float codebook_entry(int quant, int c) { return kCodebooksDev[quant != 0 ? 1 : 0][c & 15]; }
+// Indexed by storage: [0] NF4, [1] FP4 (the e4b_quant_type values), [2] MXFP4 e2m1.
+static __device__ __constant__ float kCodebooksDev[3][16] = {
+    {E4B_NF4_CODEBOOK_VALUES}, {E4B_FP4_CODEBOOK_VALUES}, {E4B_E2M1_VALUES}};
+
+// Entry c (0..15) of the table of storage `quant` (0 NF4, 1 FP4, 2 MXFP4; others NF4).
+__device__ __forceinline__ float codebook_entry(int quant, int c) {
+  return kCodebooksDev[(quant == 1 || quant == 2) ? quant : 0][c & 15];
+}
 
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
   return __uint_as_float(static_cast<uint32_t>(b) << 16);

@@ -83,6 +83,11 @@ cudaError_t launch_gather_rows(const uint16_t* A, int64_t a_rows, int64_t lda, c
                                int K, uint16_t* out, cudaStream_t stream);
 
 // ---- grouped GEMM --------------------------------------------------------
+// Internal storage index of MXFP4 weights on the tensor-core kernel: e2m1 codes
+// (element 2i in the low nibble) with one e8m0 scale byte per 32 elements of a
+// row instead of an fp32 absmax per 64 (not an e4b_quant_type).
+constexpr int kQuantMxfp4 = 2;
+
 struct GemmArgs {
   const uint16_t* A;
   int64_t a_rows, lda;
@@ -91,8 +96,9 @@ struct GemmArgs {
   int E;
   int64_t total_rows;
   const uint8_t* packed;
-  const float* absmax;
-  int quant;  // e4b_quant_type of packed
+  const float* absmax;       // [E, N*K/64] (NF4, FP4)
+  const uint8_t* mx_scales;  // [E, N*K/32] e8m0 (quant == kQuantMxfp4; tensor-core kernel only)
+  int quant;  // e4b_quant_type of packed, or kQuantMxfp4
   int N, K;
   const uint16_t* lora_A;  // [E, r, K] or nullptr
   const uint16_t* lora_B;  // [E, N, r] or nullptr
@@ -204,6 +210,11 @@ struct Mxfp4Args {
   bool out_bf16;
 };
 cudaError_t launch_grouped_mxfp4_gemm(const Mxfp4Args& a, cudaStream_t stream);
+// Picks the kernel for an MXFP4 call as launch_grouped_gemm does for NF4 (the
+// tensor-core kernel from 512 routed rows, E4B_GEMM=mma|tc forces one): `a`
+// describes it for the tensor-core kernel (quant kQuantMxfp4, mx_scales, error
+// word and gather room in the workspace), `m` for the warp-MMA kernel.
+cudaError_t launch_grouped_mxfp4(const GemmArgs& a, const Mxfp4Args& m, cudaStream_t stream, const char** path);
 
 // ---- combine ---------------------------------------------------------------
 cudaError_t launch_combine(const uint16_t* z, const int32_t* inv, const float* w, int64_t M, int k,

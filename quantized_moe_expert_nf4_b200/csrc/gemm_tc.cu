@@ -113,7 +113,8 @@ struct TcParams {
   int* err;
   const uint16_t* lora_B;  // [E, N, r] bf16, or null (no LoRA step)
   int r;
-  int quant;  // e4b_quant_type of the packed codes
+  int quant;                 // e4b_quant_type of the packed codes, or kQuantMxfp4
+  const uint8_t* mx_scales;  // kQuantMxfp4: [E*N, K/32] e8m0 scale bytes (absmax unused)
 };
 
 // The codebook's bf16 patterns split into low and high bytes, four entries per
@@ -133,19 +134,32 @@ __device__ __forceinline__ CodebookBytes codebook_bytes(int quant) {
   return t;
 }
 
+// Final interleaves of decode4: the packed order of the two elements of a byte.
+constexpr uint32_t kSelHiFirst0 = 0x4051u, kSelHiFirst1 = 0x6273u;  // element 2i in the high nibble (NF4, FP4)
+constexpr uint32_t kSelLoFirst0 = 0x5140u, kSelLoFirst1 = 0x7362u;  // element 2i in the low nibble (MXFP4)
+
 // Four nibbles (bits 0-15 of g: the low then the high nibble of two packed
-// bytes, i.e. elements 2i+1, 2i, 2i+3, 2i+2) -> two bf16x2 words in element
-// order.  A byte permute looks up entries 0-7 and 8-15 for all four nibbles at
-// once (its selector takes the nibbles' low three bits); a second permute
-// keeps, per nibble, the half its top bit names; a third interleaves the low
-// and high bytes.
-__device__ __forceinline__ void decode4(uint32_t g, const CodebookBytes& t, uint32_t* w0, uint32_t* w1) {
+// bytes) -> two bf16x2 words in element order.  A byte permute looks up
+// entries 0-7 and 8-15 for all four nibbles at once (its selector takes the
+// nibbles' low three bits); a second permute keeps, per nibble, the half its
+// top bit names; a third interleaves the low and high bytes, in the byte's
+// element order (sel0, sel1: kSelHiFirst* or kSelLoFirst*).
+__device__ __forceinline__ void decode4(uint32_t g, const CodebookBytes& t, uint32_t* w0, uint32_t* w1,
+                                        uint32_t sel0 = kSelHiFirst0, uint32_t sel1 = kSelHiFirst1) {
   const uint32_t s = g & 0x7777u;
   const uint32_t pick = ((g >> 1) & 0x4444u) | 0x3210u;  // field i: i, or i + 4 when nibble i >= 8
   const uint32_t lo = __byte_perm(__byte_perm(t.lo[0], t.lo[1], s), __byte_perm(t.lo[2], t.lo[3], s), pick);
   const uint32_t hi = __byte_perm(__byte_perm(t.hi[0], t.hi[1], s), __byte_perm(t.hi[2], t.hi[3], s), pick);
-  *w0 = __byte_perm(lo, hi, 0x4051u);  // (element 2i, element 2i+1)
-  *w1 = __byte_perm(lo, hi, 0x6273u);  // (element 2i+2, element 2i+3)
+  *w0 = __byte_perm(lo, hi, sel0);  // (element 2i, element 2i+1)
+  *w1 = __byte_perm(lo, hi, sel1);  // (element 2i+2, element 2i+3)
+}
+
+// 2^(x - 127) for an e8m0 scale byte, as a float (x = 0: the subnormal 2^-127;
+// x = 255: NaN).  Exact, and exact again after rounding to bf16.
+__device__ __forceinline__ float e8m0_scale(uint32_t x) {
+  if (x == 255u) return __uint_as_float(0x7fc00000u);
+  if (x == 0u) return __uint_as_float(0x00400000u);
+  return __uint_as_float(x << 23);
 }
 
 // Weight rows of the tile's halves.
@@ -513,6 +527,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     const int r = dt / S::kTpr, kq = dt % S::kTpr;  // weight row of the tile, part of the k block
     const int half = r >> 7, ri = r & 127;
     const CodebookBytes cbt = codebook_bytes(p.quant);
+    // MXFP4: low nibble first, and one e8m0 scale per 32 k -- this thread's
+    // 64 / kTpr k of a block lie inside scale (2 kb + 2 kq / kTpr) of the row.
+    const bool mx = p.quant == kQuantMxfp4;
+    const uint32_t sel0 = mx ? kSelLoFirst0 : kSelHiFirst0, sel1 = mx ? kSelLoFirst1 : kSelHiFirst1;
+    const int mx_sub = (2 * kq) / S::kTpr;
     uint32_t kbg = 0;
     bool ok = true;
     for (int64_t t = blockIdx.x; ok; t += gridDim.x) {
@@ -523,18 +542,21 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       tile_rows<HALVES>(p, n_tile, &r0, &r1);
       const int n = (half ? r1 : r0) + ri;
       const bool valid = n < p.N;
-      const float* am = p.absmax + (static_cast<int64_t>(e) * p.N + (valid ? n : 0)) * KB;
-      // absmax of the next 4 k blocks in flight (an L2 round trip outlasts one k block)
+      const int64_t wrow = static_cast<int64_t>(e) * p.N + (valid ? n : 0);
+      const float* am = mx ? nullptr : p.absmax + wrow * KB;
+      const uint8_t* ms = mx ? p.mx_scales + wrow * (2 * KB) + mx_sub : nullptr;
+      auto scale_of = [&](int kb) { return mx ? e8m0_scale(__ldg(ms + 2 * kb)) : __ldg(am + kb); };
+      // scales of the next 4 k blocks in flight (an L2 round trip outlasts one k block)
       float sc_ring[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) sc_ring[i] = (valid && i < KB) ? __ldg(am + i) : 0.0f;
+      for (int i = 0; i < 4; ++i) sc_ring[i] = (valid && i < KB) ? scale_of(i) : 0.0f;
       for (int kb0 = 0; kb0 < KB && ok; kb0 += 4) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int kb = kb0 + i;
           if (kb >= KB) break;
           const float sc = sc_ring[i];
-          sc_ring[i] = (valid && kb + 4 < KB) ? __ldg(am + kb + 4) : 0.0f;
+          sc_ring[i] = (valid && kb + 4 < KB) ? scale_of(kb + 4) : 0.0f;
           const int s = kbg % KS, a = kbg % AS;
           if (!mbar_wait(&tma_full[s], (kbg / KS) & 1) ||
               (kbg >= AS && !mbar_wait(&a_empty[a], ((kbg / AS) - 1) & 1))) {
@@ -564,8 +586,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           for (int c = 0; c < S::kChunks; ++c) {
             const uint32_t w = words[c];
             uint32_t v[4];
-            decode4(w, cbt, &v[0], &v[1]);
-            decode4(w >> 16, cbt, &v[2], &v[3]);
+            decode4(w, cbt, &v[0], &v[1], sel0, sel1);
+            decode4(w >> 16, cbt, &v[2], &v[3], sel0, sel1);
 #pragma unroll
             for (int by = 0; by < 4; ++by) {
               __nv_bfloat162 h2 = *reinterpret_cast<__nv_bfloat162*>(&v[by]);
@@ -761,6 +783,7 @@ cudaError_t launch_shape(const GemmArgs& a, int* err_word, cudaStream_t stream) 
   p.total_rows = a.total_rows;
   p.absmax = a.absmax;
   p.quant = a.quant;
+  p.mx_scales = a.mx_scales;
   p.N = a.N;
   p.K = a.K;
   p.swiglu = a.epi == E4B_EPI_SWIGLU;
@@ -776,7 +799,9 @@ cudaError_t launch_shape(const GemmArgs& a, int* err_word, cudaStream_t stream) 
   const int64_t tiles =
       ((a.total_rows + S::BN - 1) / S::BN + (a.E < a.total_rows ? a.E : a.total_rows)) * p.n_tiles;
   const int grid = static_cast<int>(tiles < di.sm_count ? tiles : di.sm_count);
-  LaunchScope ls(p.swiglu ? "gemm.tc.swiglu" : "gemm.tc", stream);
+  const bool mx = a.quant == kQuantMxfp4;
+  if (mx && (S::ATMEM || lora || a.mx_scales == nullptr)) return cudaErrorInvalidValue;
+  LaunchScope ls(mx ? (p.swiglu ? "mxfp4.tc.swiglu" : "mxfp4.tc") : (p.swiglu ? "gemm.tc.swiglu" : "gemm.tc"), stream);
   grouped_nf4_tc_kernel<S, false><<<grid, kThreadsTc, S::kSmemBytes, stream>>>(tm_packed, tm_b, tm_out, tm_xa, p);
   return cudaGetLastError();
 }
@@ -1027,7 +1052,7 @@ cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int* err_word, cudaStream_
     const int64_t rows_per_group = a.total_rows / (a.E > 0 ? a.E : 1);
     s = swiglu ? 1 : (rows_per_group >= 512 ? 1 : 3);
   }
-  if (s == 4 && !(a.lora_B && a.r > 0)) return launch_shape<ShapeTmem>(a, err_word, stream);
+  if (s == 4 && !(a.lora_B && a.r > 0) && a.quant != kQuantMxfp4) return launch_shape<ShapeTmem>(a, err_word, stream);
   if (s == 4) s = swiglu ? 1 : 3;
   if (s == 1) return launch_shape<ShapeWide>(a, err_word, stream);
   if (s == 2) return launch_shape<ShapeDouble>(a, err_word, stream);

@@ -28,7 +28,7 @@ E4B_EPI_NONE, E4B_EPI_SWIGLU = 0, 1
 E4B_PATH_AUTO, E4B_PATH_DECODE, E4B_PATH_GROUPED = 0, 1, 2
 E4B_QUANT_NF4, E4B_QUANT_FP4 = 0, 1
 # The E4B_VERSION this binding marshals for (e4b_expert_stack's layout among others).
-ABI_VERSION = 2
+ABI_VERSION = 3
 
 # Every symbol include/e4b.h declares.
 EXPORTED = (
@@ -40,7 +40,7 @@ EXPORTED = (
     "e4b_grouped_nf4_gemm_workspace_size", "e4b_grouped_nf4_gemm", "e4b_grouped_4bit_gemm",
     "e4b_grouped_nf4_gemm_dgrad_workspace_size", "e4b_grouped_nf4_gemm_dgrad", "e4b_grouped_4bit_gemm_dgrad",
     "e4b_grouped_lora_grads_workspace_size", "e4b_grouped_lora_grads",
-    "e4b_grouped_mxfp4_gemm",
+    "e4b_grouped_mxfp4_gemm_workspace_size", "e4b_grouped_mxfp4_gemm",
     "e4b_moe_expert_forward_workspace_size", "e4b_moe_expert_forward",
     "e4b_moe_expert_forward_path", "e4b_moe_expert_forward_decode_noalloc",
     "e4b_moe_expert_backward_workspace_size", "e4b_moe_expert_backward",
@@ -126,7 +126,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.e4b_grouped_lora_grads.argtypes = [vp, i64, i64, vp, vp, i64, i64, vp, i64, i64, i64, vp, vp, i32,
                                            ctypes.c_float, vp, vp, vp, sz, vp]
     lib.e4b_grouped_mxfp4_gemm.restype = i32
-    lib.e4b_grouped_mxfp4_gemm.argtypes = [vp, i64, i64, vp, vp, i64, i64, vp, vp, i64, i64, i32, vp, i32, vp]
+    lib.e4b_grouped_mxfp4_gemm_workspace_size.restype = sz
+    lib.e4b_grouped_mxfp4_gemm_workspace_size.argtypes = [i64, i64, i64]
+    lib.e4b_grouped_mxfp4_gemm.argtypes = [vp, i64, i64, vp, vp, i64, i64, vp, vp, i64, i64, i32, vp, i32, vp, sz,
+                                           vp]
     lib.e4b_moe_expert_forward_workspace_size.restype = sz
     lib.e4b_moe_expert_forward_workspace_size.argtypes = [i64, ctypes.POINTER(ExpertStackC), i32]
     lib.e4b_moe_expert_forward.restype = i32
@@ -391,9 +394,14 @@ def e4b_grouped_lora_grads(x: torch.Tensor, row_index: Optional[torch.Tensor], e
         dA.data_ptr(), dB.data_ptr(), _ptr(workspace), ws, _stream(stream)), "e4b_grouped_lora_grads")
 
 
+def e4b_grouped_mxfp4_gemm_workspace_size(total_rows: int, N: int, K: int) -> int:
+    return int(load_library().e4b_grouped_mxfp4_gemm_workspace_size(total_rows, N, K))
+
+
 def e4b_grouped_mxfp4_gemm(A: torch.Tensor, row_index: Optional[torch.Tensor], expert_offsets: torch.Tensor,
                            total_rows: int, blocks: torch.Tensor, scales: torch.Tensor, N: int, K: int,
-                           out: torch.Tensor, epi: int = E4B_EPI_NONE, stream=None) -> None:
+                           out: torch.Tensor, epi: int = E4B_EPI_NONE, workspace: Optional[torch.Tensor] = None,
+                           stream=None) -> None:
     """y[p] = A[row_index[p]] . W_e^T with W_e given as MXFP4 code bytes and e8m0 scales."""
     if A.dim() != 2 or A.dtype != torch.bfloat16 or not A.is_cuda or A.stride(1) != 1:
         raise ValueError("A must be a 2-D bf16 CUDA tensor with unit column stride")
@@ -410,9 +418,10 @@ def e4b_grouped_mxfp4_gemm(A: torch.Tensor, row_index: Optional[torch.Tensor], e
     ncols = N // 2 if epi == E4B_EPI_SWIGLU else N
     if out.numel() < total_rows * ncols:
         raise ValueError("out too small")
+    ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(load_library().e4b_grouped_mxfp4_gemm(
         A.data_ptr(), A.shape[0], A.stride(0), _ptr(row_index), expert_offsets.data_ptr(), E, total_rows,
-        blocks.data_ptr(), scales.data_ptr(), N, K, epi, out.data_ptr(), od, _stream(stream)),
+        blocks.data_ptr(), scales.data_ptr(), N, K, epi, out.data_ptr(), od, _ptr(workspace), ws, _stream(stream)),
         "e4b_grouped_mxfp4_gemm")
 
 

@@ -48,7 +48,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.e4b_version() == e4b.ABI_VERSION == 2
+    assert lib.e4b_version() == e4b.ABI_VERSION == 3
     assert lib.e4b_status_string(0) == b"E4B_OK"
     assert lib.e4b_status_string(3) == b"E4B_ERR_WORKSPACE"
 
@@ -221,10 +221,15 @@ def test_mxfp4_host_side_rejections(lib):
 
     def call(**kw):
         a = dict(A=p, a_rows=4, lda=128, ridx=None, offs=p, E=2, rows=4, blocks=p, scales=p, N=128, K=128, epi=0,
-                 out=p, od=0)
+                 out=p, od=0, ws=p, wsb=1 << 30)
         a.update(kw)
         return lib.e4b_grouped_mxfp4_gemm(a["A"], a["a_rows"], a["lda"], a["ridx"], a["offs"], a["E"], a["rows"],
-                                          a["blocks"], a["scales"], a["N"], a["K"], a["epi"], a["out"], a["od"], None)
+                                          a["blocks"], a["scales"], a["N"], a["K"], a["epi"], a["out"], a["od"],
+                                          a["ws"], a["wsb"], None)
+    need = lib.e4b_grouped_mxfp4_gemm_workspace_size(4, 128, 128)
+    assert need == e4b.e4b_grouped_nf4_gemm_workspace_size(4, 128, 128, 0) >= 256 + 4 * 128 * 2
+    assert call(wsb=need - 1) == 3 and str(need).encode() in lib.e4b_last_error()
+    assert call(ws=ctypes.c_void_p((1 << 20) + 8), wsb=need) == 1 and b"16-byte aligned" in lib.e4b_last_error()
     assert call(K=96) == 2 and b"K must be" in lib.e4b_last_error()
     assert call(N=32) == 2 and b"N must be" in lib.e4b_last_error()
     assert call(lda=100) == 1 and b"lda" in lib.e4b_last_error()

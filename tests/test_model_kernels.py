@@ -131,7 +131,7 @@ def _byte_perm(x: int, y: int, s: int) -> int:
     return out
 
 
-@pytest.mark.parametrize("table", ["nf4", "fp4"])
+@pytest.mark.parametrize("table", ["nf4", "fp4", "mxfp4"])
 def test_tensor_core_byte_permute_decoder_is_a_table_lookup(table):
     """csrc/gemm_tc.cu decode4 for every 16-bit input: the codebook's bf16
     patterns split into low and high bytes (four entries per word), two
@@ -139,10 +139,17 @@ def test_tensor_core_byte_permute_decoder_is_a_table_lookup(table):
     third keeps the half each nibble's top bit names, two more interleave the
     bytes -> (element 2i, 2i+1) and (2i+2, 2i+3), the high nibble of a byte
     being the lower-index element.  Checked against direct lookup for the NF4
-    and the FP4 (e2m1 / 6, with -0 at code 8) tables."""
-    from oracle import fp4
+    and the FP4 (e2m1 / 6, with -0 at code 8) tables, and for MXFP4 codes (the
+    e2m1 values, element 2i in the LOW nibble: the other final selectors)."""
+    from oracle import fp4, mxfp4
     from quantized_moe_expert_nf4_b200 import workloads
-    cb32 = nf4.NF4_CODEBOOK if table == "nf4" else fp4.codebook_f64().astype(np.float32)
+    if table == "nf4":
+        cb32 = nf4.NF4_CODEBOOK
+    elif table == "fp4":
+        cb32 = fp4.codebook_f64().astype(np.float32)
+    else:
+        cb32 = mxfp4.e2m1_table().astype(np.float32)
+    sel0, sel1 = (0x5140, 0x7362) if table == "mxfp4" else (0x4051, 0x6273)
     bits = [int(b) for b in workloads.to_bf16_bits(np.asarray(cb32, np.float32))]
     lo = [0, 0, 0, 0]
     hi = [0, 0, 0, 0]
@@ -154,11 +161,41 @@ def test_tensor_core_byte_permute_decoder_is_a_table_lookup(table):
         pick = ((g >> 1) & 0x4444) | 0x3210
         L = _byte_perm(_byte_perm(lo[0], lo[1], s), _byte_perm(lo[2], lo[3], s), pick)
         Hh = _byte_perm(_byte_perm(hi[0], hi[1], s), _byte_perm(hi[2], hi[3], s), pick)
-        w0 = _byte_perm(L, Hh, 0x4051)
-        w1 = _byte_perm(L, Hh, 0x6273)
+        w0 = _byte_perm(L, Hh, sel0)
+        w1 = _byte_perm(L, Hh, sel1)
         n = [g & 15, (g >> 4) & 15, (g >> 8) & 15, (g >> 12) & 15]
-        assert w0 == bits[n[1]] | (bits[n[0]] << 16), hex(g)
-        assert w1 == bits[n[3]] | (bits[n[2]] << 16), hex(g)
+        if table == "mxfp4":   # byte = (element 2i+1 << 4) | element 2i
+            assert w0 == bits[n[0]] | (bits[n[1]] << 16), hex(g)
+            assert w1 == bits[n[2]] | (bits[n[3]] << 16), hex(g)
+        else:                  # byte = (element 2i << 4) | element 2i+1
+            assert w0 == bits[n[1]] | (bits[n[0]] << 16), hex(g)
+            assert w1 == bits[n[3]] | (bits[n[2]] << 16), hex(g)
+
+
+@pytest.mark.parametrize("tpr", [2, 4])
+def test_tensor_core_mxfp4_decoders_take_their_scale_block(tpr):
+    """csrc/gemm_tc.cu MXFP4 decoders: thread part kq of a 64-k block (64 / tpr
+    k from 64 kq / tpr) multiplies by scale byte 2 kb + (2 kq) / tpr of its row,
+    the one e8m0 block of 32 that holds all of its k; with the e2m1 values and
+    2^(x - 127) this rebuilds the oracle's dequantised row."""
+    from oracle import mxfp4
+    rng = np.random.default_rng(21)
+    K = 320
+    row = rng.integers(0, 256, K // 2, dtype=np.uint8)
+    sc = rng.integers(120, 135, K // 32, dtype=np.uint8)
+    want = mxfp4.dequantize_expert(row[None, :], sc[None, :], 1, K)[0]
+    got = np.full(K, np.nan)
+    e2m1 = mxfp4.e2m1_table()
+    for kb in range(K // 64):
+        for kq in range(tpr):
+            k0 = kb * 64 + kq * (64 // tpr)
+            x = int(sc[2 * kb + (2 * kq) // tpr])
+            assert all((k0 + j) // 32 == 2 * kb + (2 * kq) // tpr for j in range(64 // tpr))
+            for j in range(0, 64 // tpr, 2):
+                byte = int(row[(k0 + j) // 2])
+                got[k0 + j] = e2m1[byte & 15] * 2.0 ** (x - 127)
+                got[k0 + j + 1] = e2m1[byte >> 4] * 2.0 ** (x - 127)
+    assert np.array_equal(got, want)
 
 
 def _quant_cell_table(cb):
