@@ -393,7 +393,11 @@ E4B_API e4b_status e4b_moe_expert_forward(const uint16_t* x, int64_t M, const fl
                                   int k, int renormalize, const e4b_expert_stack* w,
                                   uint16_t* out, void* workspace, size_t workspace_bytes,
                                   e4b_stream stream);
-/* Same, with the implementation chosen explicitly (tests and benchmarks). */
+/* Same, with the implementation chosen explicitly (tests and benchmarks).
+ * E4B_PATH_AUTO takes the decode kernels when they can run the shape -- 1 <= M <= 8,
+ * k <= 32, E <= 512, H <= 4096 and their shared-memory plan fits -- and the grouped
+ * path otherwise.  E4B_PATH_DECODE on any other shape returns E4B_ERR_UNSUPPORTED
+ * and e4b_last_error() names the limit. */
 E4B_API e4b_status e4b_moe_expert_forward_path(const uint16_t* x, int64_t M, const float* router_logits,
                                        int k, int renormalize, const e4b_expert_stack* w,
                                        uint16_t* out, void* workspace, size_t workspace_bytes,
