@@ -57,3 +57,27 @@ def test_grouped_roofline_uses_the_sustained_peak_in_a_long_region():
     flops = 2.0 * 4096 * 8 * 2 * 768 * 2048
     assert r["achieved"] == pytest.approx(flops / 0.40e-3 / 1e12)
     assert r["peak"] == 1374.1 and "sustained" in r["peak_source"]
+
+
+def test_reference_arm_prints_one_contract_line():
+    """`bench.py --impl reference` (the oracle on this host's cores) prints one
+    JSON line with the keys the benchmark contract names, its e2e and
+    cpu_baseline objects describing the same run."""
+    import json
+    import subprocess
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    res = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--workload",
+                          "tiny_m64", "--steps", "2", "--warmup", "3"], capture_output=True, text=True, timeout=300,
+                         cwd=root)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [l for l in res.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["steps"] == 2 and d["warmup"] == 3 and d["value"] > 0
+    assert d["config"]["workload"] == "tiny_m64"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
