@@ -325,7 +325,7 @@ e4b_status e4b_moe_route_permute(const float* logits, int64_t M, int64_t E, int 
 
 size_t e4b_grouped_nf4_gemm_workspace_size(int64_t total_rows, int64_t N, int64_t K, int r) {
   (void)N;
-  if (total_rows < 0 || r < 0 || K < 0) return 0;
+  if (total_rows <= 0 || r < 0 || K < 0) return 0;  // no rows: nothing launches, nothing waits
   return gemm_workspace_bytes(total_rows, K, r);
 }
 
@@ -354,7 +354,8 @@ e4b_status e4b_grouped_nf4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda, 
     return fail(E4B_ERR_INVALID_ARGUMENT, "A, packed and out must be 16-byte aligned");
   if (lora_A && (!aligned16(lora_A) || !aligned16(lora_B)))
     return fail(E4B_ERR_INVALID_ARGUMENT, "lora_A and lora_B must be 16-byte aligned");
-  if (e4b_status s = check_workspace("gemm", gemm_workspace_bytes(total_rows, K, r), workspace, workspace_bytes);
+  if (e4b_status s = check_workspace("gemm", total_rows > 0 ? gemm_workspace_bytes(total_rows, K, r) : 0, workspace,
+                                     workspace_bytes);
       s != E4B_OK)
     return s;
   if (e4b_status s = check_device(); s != E4B_OK) return s;

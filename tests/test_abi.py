@@ -144,3 +144,15 @@ def test_error_word_calls_check_their_arguments_on_the_host(lib):
     assert lib.e4b_workspace_clear_error(None, None) == 1
     assert code.value == 7   # untouched on a rejected call
 
+
+
+def test_zero_row_gemm_needs_no_workspace(lib):
+    """With no routed rows nothing launches or waits: the size query is 0 and a
+    NULL workspace passes the host checks (on a host without a GPU the call then
+    stops at the device check, not at the workspace)."""
+    p = ctypes.c_void_p(1 << 20)
+    assert e4b.e4b_grouped_nf4_gemm_workspace_size(0, 128, 128, 8) == 0
+    assert e4b.e4b_grouped_nf4_gemm_workspace_size(1, 128, 128, 0) >= 256 + 128 * 2
+    st = lib.e4b_grouped_nf4_gemm(p, 1, 128, None, p, 2, 0, p, p, 128, 128, None, None, 0, 0.0, 0, p, 0, None, 0,
+                                  None)
+    assert st != 3 and b"workspace" not in lib.e4b_last_error()
