@@ -237,7 +237,7 @@ E4B_API e4b_status e4b_moe_route_permute(const float* logits, int64_t M, int64_t
  *                 the LoRA products x . lora_A^T (total_rows x r fp32) and room
  *                 for the routed rows gathered in order (total_rows x K bf16),
  *                 which the tensor-core kernel reads as contiguous tiles when
- *                 row_index is given.
+ *                 row_index is given.  0 bytes (NULL allowed) when total_rows == 0.
  * Groups with no rows cost nothing and write nothing.
  */
 E4B_API size_t e4b_grouped_nf4_gemm_workspace_size(int64_t total_rows, int64_t N, int64_t K, int r);
@@ -282,6 +282,7 @@ E4B_API e4b_status e4b_grouped_4bit_gemm(const uint16_t* A, int64_t a_rows, int6
  * Requires K % 64 == 0, N % 64 == 0, 0 <= r <= 16, total_rows < 2^31.
  * workspace       e4b_grouped_nf4_gemm_dgrad_workspace_size() bytes: an error
  *                 word and the products dY . lora_B (total_rows x r fp32).
+ *                 0 bytes (NULL allowed) when total_rows == 0.
  * Groups with no rows cost nothing and write nothing.
  */
 E4B_API size_t e4b_grouped_nf4_gemm_dgrad_workspace_size(int64_t total_rows, int64_t N, int64_t K, int r);

@@ -365,7 +365,7 @@ e4b_status e4b_moe_route_permute(const float* logits, int64_t M, int64_t E, int 
 
 size_t e4b_grouped_nf4_gemm_workspace_size(int64_t total_rows, int64_t N, int64_t K, int r) {
   (void)N;
-  if (total_rows < 0 || r < 0 || K < 0) return 0;
+  if (total_rows <= 0 || r < 0 || K < 0) return 0;  // no rows: nothing launches, nothing waits
   return gemm_workspace_bytes(total_rows, K, r);
 }
 
@@ -406,7 +406,8 @@ e4b_status e4b_grouped_4bit_gemm(const uint16_t* A, int64_t a_rows, int64_t lda,
     return fail(E4B_ERR_INVALID_ARGUMENT, "A, packed and out must be 16-byte aligned");
   if (lora_A && (!aligned16(lora_A) || !aligned16(lora_B)))
     return fail(E4B_ERR_INVALID_ARGUMENT, "lora_A and lora_B must be 16-byte aligned");
-  if (e4b_status s = check_workspace("gemm", gemm_workspace_bytes(total_rows, K, r), workspace, workspace_bytes);
+  if (e4b_status s = check_workspace("gemm", total_rows > 0 ? gemm_workspace_bytes(total_rows, K, r) : 0, workspace,
+                                     workspace_bytes);
       s != E4B_OK)
     return s;
   if (e4b_status s = check_device(); s != E4B_OK) return s;
@@ -449,7 +450,7 @@ e4b_status e4b_grouped_4bit_gemm(const uint16_t* A, int64_t a_rows, int64_t lda,
 size_t e4b_grouped_nf4_gemm_dgrad_workspace_size(int64_t total_rows, int64_t N, int64_t K, int r) {
   (void)N;
   (void)K;
-  if (total_rows < 0 || r < 0 || N < 0) return 0;
+  if (total_rows <= 0 || r < 0 || N < 0) return 0;  // no rows: nothing launches, nothing waits
   return dgrad_workspace_bytes(total_rows, N, r);
 }
 
@@ -490,7 +491,8 @@ e4b_status e4b_grouped_4bit_gemm_dgrad(const uint16_t* dY, int64_t dy_rows, int6
     return fail(E4B_ERR_INVALID_ARGUMENT, "dY, packed, absmax and out must be 16-byte aligned");
   if (lora_A && (!aligned16(lora_A) || !aligned16(lora_B)))
     return fail(E4B_ERR_INVALID_ARGUMENT, "lora_A and lora_B must be 16-byte aligned");
-  if (e4b_status s = check_workspace("dgrad", dgrad_workspace_bytes(total_rows, N, r), workspace, workspace_bytes);
+  if (e4b_status s = check_workspace("dgrad", total_rows > 0 ? dgrad_workspace_bytes(total_rows, N, r) : 0, workspace,
+                                     workspace_bytes);
       s != E4B_OK)
     return s;
   if (e4b_status s = check_device(); s != E4B_OK) return s;

@@ -270,3 +270,23 @@ def test_expert_stack_layout_matches_the_header():
     hdr = open(os.path.join(os.path.dirname(__file__), "..", "include", "e4b.h")).read()
     body = hdr[hdr.index("typedef struct {\n  const uint8_t* gu_packed"):hdr.index("} e4b_expert_stack;")]
     assert body.index("int64_t E, H, I;") < body.index("int32_t quant_type;")
+
+
+def test_zero_row_gemm_needs_no_workspace(lib):
+    """With no routed rows nothing launches or waits: the size query is 0 and a
+    NULL workspace passes the host checks (on a host without a GPU the call then
+    stops at the device check, not at the workspace)."""
+    p = ctypes.c_void_p(1 << 20)
+    assert e4b.e4b_grouped_nf4_gemm_workspace_size(0, 128, 128, 8) == 0
+    assert e4b.e4b_grouped_nf4_gemm_workspace_size(1, 128, 128, 0) >= 256 + 128 * 2
+    st = lib.e4b_grouped_nf4_gemm(p, 1, 128, None, p, 2, 0, p, p, 128, 128, None, None, 0, 0.0, 0, p, 0, None, 0,
+                                  None)
+    assert st != 3 and b"workspace" not in lib.e4b_last_error()
+
+
+def test_zero_row_dgrad_needs_no_workspace(lib):
+    p = ctypes.c_void_p(1 << 20)
+    assert e4b.e4b_grouped_nf4_gemm_dgrad_workspace_size(0, 128, 128, 8) == 0
+    st = lib.e4b_grouped_nf4_gemm_dgrad(p, 1, 128, None, p, 2, 0, p, p, 128, 128, None, None, 0, 0.0, p, 0, None, 0,
+                                        None)
+    assert st != 3 and b"workspace" not in lib.e4b_last_error()
