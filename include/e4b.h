@@ -350,7 +350,8 @@ E4B_API e4b_status e4b_grouped_lora_grads(const uint16_t* x, int64_t x_rows, int
  * workspace  e4b_grouped_mxfp4_gemm_workspace_size() bytes: an error word and
  *            room for the routed rows gathered in order (total_rows x K bf16),
  *            which the tensor-core kernel (512 routed rows and more) reads as
- *            contiguous tiles; the warp-MMA kernel below uses neither.
+ *            contiguous tiles; the warp-MMA kernel below uses neither.  0 bytes
+ *            (NULL allowed) when total_rows == 0.
  * Each e2m1 value and each scale is exact in bf16, so the products with the
  * bf16 operand rows are the GEMM's only roundings (fp32 accumulation).
  */

@@ -621,7 +621,7 @@ e4b_status e4b_grouped_lora_grads(const uint16_t* x, int64_t x_rows, int64_t ldx
 
 size_t e4b_grouped_mxfp4_gemm_workspace_size(int64_t total_rows, int64_t N, int64_t K) {
   (void)N;
-  if (total_rows < 0 || K < 0) return 0;
+  if (total_rows <= 0 || K < 0) return 0;  // no rows: nothing launches, nothing waits
   return gemm_workspace_bytes(total_rows, K, 0);
 }
 
@@ -644,7 +644,8 @@ e4b_status e4b_grouped_mxfp4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda
   if (total_rows > INT32_MAX) return fail(E4B_ERR_UNSUPPORTED, "total_rows exceeds int32");
   if ((A && !aligned16(A)) || !aligned16(blocks) || (out && !aligned16(out)))
     return fail(E4B_ERR_INVALID_ARGUMENT, "A, blocks and out must be 16-byte aligned");
-  if (e4b_status s = check_workspace("mxfp4 gemm", gemm_workspace_bytes(total_rows, K, 0), workspace, workspace_bytes);
+  if (e4b_status s = check_workspace("mxfp4 gemm", total_rows > 0 ? gemm_workspace_bytes(total_rows, K, 0) : 0,
+                                     workspace, workspace_bytes);
       s != E4B_OK)
     return s;
   if (e4b_status s = check_device(); s != E4B_OK) return s;

@@ -290,3 +290,10 @@ def test_zero_row_dgrad_needs_no_workspace(lib):
     st = lib.e4b_grouped_nf4_gemm_dgrad(p, 1, 128, None, p, 2, 0, p, p, 128, 128, None, None, 0, 0.0, p, 0, None, 0,
                                         None)
     assert st != 3 and b"workspace" not in lib.e4b_last_error()
+
+
+def test_zero_row_mxfp4_gemm_needs_no_workspace(lib):
+    p = ctypes.c_void_p(1 << 20)
+    assert lib.e4b_grouped_mxfp4_gemm_workspace_size(0, 128, 128) == 0
+    st = lib.e4b_grouped_mxfp4_gemm(p, 1, 128, None, p, 2, 0, p, p, 128, 128, 0, p, 0, None, 0, None)
+    assert st != 3 and b"workspace" not in lib.e4b_last_error()
