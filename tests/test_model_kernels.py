@@ -284,3 +284,36 @@ def test_quantiser_cell_lookup_and_reciprocal_path_match_the_oracle(table):
             want = mod.code_of_scaled((w / a).astype(f32))
         assert np.array_equal(got, want), kind
     assert fallbacks > 0   # the exact path was exercised
+
+
+def test_tensor_memory_decoders_fill_the_a_operand_the_mma_reads():
+    """csrc/gemm_tc.cu TMEM-operand tile: decoder warp w (lane quadrant w % 4,
+    part c = (w - 4) / 4: half c / 2, 32-k part c % 2) takes weight row
+    32 (w % 4) + lane of its half, decodes its 32 k (4 words, decode4 on each
+    half-word: v[i] = elements 2i, 2i+1) and stores v[0..15] as 16 consecutive
+    32-bit columns of its TMEM lane from column A + half*32 + part*16.  The MMA
+    of k-step kk of half h reads columns A + h*32 + kk*8 .. +7 of lanes 0..127,
+    two bf16 per column, the lower k in the low half: that must be the half's
+    rows and k [16 kk, 16 kk + 16) of the 64-k block."""
+    packed, absmax, W = _layer_rows(9, 256, 64)
+    tmem = {}
+    for w in range(4, 20):
+        qd, c = w & 3, (w - 4) >> 2
+        half, part = c >> 1, c & 1
+        for lane in range(32):
+            ri = qd * 32 + lane
+            r = half * 128 + ri
+            src = packed[r, part * 16: part * 16 + 16]          # 16 bytes = this thread's 32 k
+            vals = []
+            for byte in src:
+                vals += [v * absmax[r, 0] for v in _pair(byte)]   # elements in k order
+            v = [(vals[2 * i], vals[2 * i + 1]) for i in range(16)]
+            for i in range(16):
+                key = (ri, half * 32 + part * 16 + i)
+                assert key not in tmem, "column written twice"
+                tmem[key] = v[i]                                  # (low half, high half)
+    for h in range(2):
+        for kk in range(4):
+            for lane in range(128):
+                row = [x for col in range(8) for x in tmem[(lane, h * 32 + kk * 8 + col)]]
+                assert row == list(W[h * 128 + lane, kk * 16: kk * 16 + 16]), (h, kk, lane)
