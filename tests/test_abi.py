@@ -285,3 +285,10 @@ def test_zero_row_dgrad_needs_no_workspace(lib):
     st = lib.e4b_grouped_nf4_gemm_dgrad(p, 1, 128, None, p, 2, 0, p, p, 128, 128, None, None, 0, 0.0, p, 0, None, 0,
                                         None)
     assert st != 3 and b"workspace" not in lib.e4b_last_error()
+
+
+def test_graft_entry_build_checks_the_abi_version():
+    """build() compiles (or reuses) the library, loads it and checks its ABI
+    version against the binding's."""
+    import __graft_entry__ as ge
+    ge.build()
