@@ -297,3 +297,10 @@ def test_zero_row_mxfp4_gemm_needs_no_workspace(lib):
     assert lib.e4b_grouped_mxfp4_gemm_workspace_size(0, 128, 128) == 0
     st = lib.e4b_grouped_mxfp4_gemm(p, 1, 128, None, p, 2, 0, p, p, 128, 128, 0, p, 0, None, 0, None)
     assert st != 3 and b"workspace" not in lib.e4b_last_error()
+
+
+def test_graft_entry_build_checks_the_abi_version():
+    """build() compiles (or reuses) the library, loads it and checks its ABI
+    version against the binding's."""
+    import __graft_entry__ as ge
+    ge.build()
