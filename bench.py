@@ -713,6 +713,27 @@ def time_backward(name, dev, steps=10, warmup=3):
     return res
 
 
+def repeat_forward(name, reps):
+    """Profiling driver for ncu captures: the workload's layer (seed 0) and its
+    first input batch, then `reps` calls of the public forward; nothing is
+    timed.  Prints the path of the last call."""
+    import torch
+
+    from quantized_moe_expert_nf4_b200 import e4b, synthetic
+
+    cfgname, M = WORKLOADS[name][:2]
+    cfg = workloads.CONFIGS[cfgname]
+    e4b.load_library()
+    layer = synthetic.make_device_layer(cfg)
+    x, logits = synthetic.inputs(cfg, M)
+    out = torch.empty((M, cfg.H), dtype=torch.bfloat16, device="cuda")
+    ws = e4b.workspace(e4b.e4b_moe_expert_forward_workspace_size(M, layer.stack, cfg.k))
+    for _ in range(reps):
+        e4b.e4b_moe_expert_forward(x, logits, cfg.k, True, layer.stack, out, ws)
+    torch.cuda.synchronize()
+    print("ok", e4b.last_path(), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -727,7 +748,12 @@ def main():
     ap.add_argument("--no-backward", action="store_true", help="skip the layer-backward timing")
     ap.add_argument("--no-mxfp4", action="store_true", help="skip the MXFP4 grouped-GEMM timing")
     ap.add_argument("--replicas", type=int, default=0, help="layer replicas (0: enough to exceed L2 4x)")
+    ap.add_argument("--repeat-forward", type=int, default=0, metavar="N",
+                    help="profiling driver: build the workload's layer and call the forward N times, untimed")
     args = ap.parse_args()
+    if args.repeat_forward > 0:
+        repeat_forward(args.workload, args.repeat_forward)
+        return
     if args.warmup < 3:
         args.warmup = 3
 
