@@ -42,17 +42,26 @@ from quantized_moe_expert_nf4_b200 import workloads  # noqa: E402
 L2_BYTES = 126 * 1024 * 1024
 METRIC = "routed tokens/s and TFLOP/s per MoE layer; fraction of HBM/bf16 roofline"
 
+# name -> (layer configuration, tokens M[, 4-bit storage: "nf4" unless named])
 WORKLOADS = {
     "olmoe_m1": ("olmoe", 1), "olmoe_m4": ("olmoe", 4), "olmoe_m8": ("olmoe", 8), "olmoe_m2048": ("olmoe", 2048),
     "qwen3_m4096": ("qwen3", 4096), "qwen3_lora_m4096": ("qwen3_lora", 4096),
     "gptoss_m1": ("gptoss", 1), "gptoss_m8192": ("gptoss", 8192), "tiny_m64": ("tiny", 64),
+    "olmoe_fp4_m8": ("olmoe", 8, "fp4"), "qwen3_fp4_m4096": ("qwen3", 4096, "fp4"),
 }
+STORAGE = {"nf4": 0, "fp4": 1}   # e4b_quant_type
+
+
+def workload(name):
+    """(layer configuration name, M, storage name) of a bench workload."""
+    w = WORKLOADS[name]
+    return w[0], w[1], (w[2] if len(w) > 2 else "nf4")
 DEFAULT_WORKLOAD = "olmoe_m1"
 # Every other workload of the table runs in the default sweep, so the JSON line
 # carries the prefill rows' (M >= 4096) tensor-core fractions and the gpt-oss
 # decode row beside the OLMoE ones.
 DEFAULT_SWEEP = ("olmoe_m4", "olmoe_m8", "olmoe_m2048", "qwen3_m4096", "qwen3_lora_m4096", "gptoss_m1",
-                 "gptoss_m8192")
+                 "gptoss_m8192", "olmoe_fp4_m8", "qwen3_fp4_m4096")
 
 
 def load_peaks():
@@ -160,10 +169,11 @@ class OracleSample:
     the packed bytes every step) and the per-token forward.
     """
 
-    def __init__(self, cfg, M, max_tokens=8, replicas=2):
-        from oracle import nf4, routing
+    def __init__(self, cfg, M, max_tokens=8, replicas=2, storage="nf4"):
+        from oracle import fp4, nf4, routing
 
-        self.cfg, self.M = cfg, M
+        quant = {"nf4": nf4, "fp4": fp4}[storage]
+        self.cfg, self.M, self.storage = cfg, M, storage
         self.ntok = min(M, max_tokens)
         E, H, I = cfg.E, cfg.H, cfg.I
         self.samples = []
@@ -176,8 +186,8 @@ class OracleSample:
             dp = np.zeros((E, H * I // 2), np.uint8)
             da = np.zeros((E, H * I // 64), np.float32)
             for e in sorted(set(ids.reshape(-1).tolist())):
-                gp[e], ga[e] = nf4.quantize_expert(workloads.gate_up_expert(cfg, e))
-                dp[e], da[e] = nf4.quantize_expert(workloads.down_expert(cfg, e))
+                gp[e], ga[e] = quant.quantize_expert(workloads.gate_up_expert(cfg, e))
+                dp[e], da[e] = quant.quantize_expert(workloads.down_expert(cfg, e))
             self.samples.append((logits, x, ids, gp, ga, dp, da))
         self.la = self.lb = None
         if cfg.lora_r:
@@ -190,7 +200,8 @@ class OracleSample:
         cfg = self.cfg
         logits, x, ids, gp, ga, dp, da = self.samples[i % len(self.samples)]
         t0 = time.perf_counter()
-        st = moe.ExpertStack(gp, ga, dp, da, cfg.E, cfg.H, cfg.I, self.la, self.lb, workloads.lora_scale(cfg))
+        st = moe.ExpertStack(gp, ga, dp, da, cfg.E, cfg.H, cfg.I, self.la, self.lb, workloads.lora_scale(cfg),
+                             quant=self.storage)
         w = routing.route_weights(logits, ids)
         moe.moe_forward_per_token(x, ids, w, st)
         return time.perf_counter() - t0
@@ -201,9 +212,9 @@ class OracleSample:
                 f"experts, per-token SwiGLU expert MLPs and combine")
 
 
-def oracle_rate(cfg, M, budget_s=12.0, max_tokens=8):
+def oracle_rate(cfg, M, budget_s=12.0, max_tokens=8, storage="nf4"):
     """(routed tokens/s, description, seconds) of the oracle on a bounded sample."""
-    smp = OracleSample(cfg, M, max_tokens=max_tokens, replicas=2)
+    smp = OracleSample(cfg, M, max_tokens=max_tokens, replicas=2, storage=storage)
     smp.step(0)  # warm-up
     spent, toks, i = 0.0, 0, 0
     while spent < budget_s and i < 1000:
@@ -218,7 +229,7 @@ def run_reference(args, cfg, M, rank, world):
     if rank != 0:
         return None
     cores = cpu_cores()
-    smp = OracleSample(cfg, M, max_tokens=8, replicas=2)
+    smp = OracleSample(cfg, M, max_tokens=8, replicas=2, storage=workload(args.workload)[2])
     for i in range(args.warmup):
         smp.step(i)
     t_total = 0.0
@@ -230,7 +241,8 @@ def run_reference(args, cfg, M, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": args.workload, "E": cfg.E, "H": cfg.H, "I": cfg.I, "k": cfg.k, "M": M,
-                   "routing": cfg.routing, "sample_tokens_per_step": smp.ntok},
+                   "routing": cfg.routing, "weights": f"{smp.storage.upper()}/64 fp32 absmax",
+                   "sample_tokens_per_step": smp.ntok},
         "cpu_baseline": {"value": value, "unit": "routed_tokens/s", "cores": cores, "kind": "oracle",
                          "sample": smp.describe()},
         "e2e": {"value": value, "unit": "routed_tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -241,15 +253,16 @@ def run_reference(args, cfg, M, rank, world):
 
 # ---------------------------------------------------------------------------
 class Bench:
-    def __init__(self, cfg, M, device, replicas, seed_base=0):
+    def __init__(self, cfg, M, device, replicas, seed_base=0, storage="nf4"):
         import torch
         from quantized_moe_expert_nf4_b200 import e4b, synthetic
 
         self.torch, self.e4b = torch, e4b
         self.cfg, self.M, self.device = cfg, M, device
+        self.quant_type = STORAGE[storage]
         self.layers, self.xs, self.logits = [], [], []
         # replica 0: the seeded workload weights; others: seeded GPU draws of the same law
-        self.layers.append(synthetic.make_device_layer(cfg, seed=seed_base, device=device))
+        self.layers.append(synthetic.make_device_layer(cfg, seed=seed_base, device=device, quant_type=self.quant_type))
         for r in range(1, replicas):
             self.layers.append(self._gpu_replica(seed_base * 1000 + r))
         for r in range(replicas):
@@ -273,7 +286,7 @@ class Bench:
             for e0 in range(0, cfg.E, 8):
                 e1 = min(cfg.E, e0 + 8)
                 W = torch.randn((e1 - e0, N, K), generator=g, device=self.device) * cfg.weight_std
-                e4b.e4b_nf4_quantize_stack(W, packed[e0:e1], absmax[e0:e1])
+                e4b.e4b_quantize_stack(W, packed[e0:e1], absmax[e0:e1], self.quant_type)
             return packed, absmax
 
         gp, ga = pack(2 * cfg.I, cfg.H)
@@ -282,7 +295,7 @@ class Bench:
         if cfg.lora_r:
             la = (torch.randn((cfg.E, cfg.lora_r, cfg.H), generator=g, device=self.device) * cfg.lora_std).bfloat16()
             lb = (torch.randn((cfg.E, 2 * cfg.I, cfg.lora_r), generator=g, device=self.device) * cfg.lora_std).bfloat16()
-        stack = e4b.ExpertStack(gp, ga, dp, da, cfg.E, cfg.H, cfg.I, la, lb, cfg.lora_alpha)
+        stack = e4b.ExpertStack(gp, ga, dp, da, cfg.E, cfg.H, cfg.I, la, lb, cfg.lora_alpha, self.quant_type)
         return synthetic.DeviceLayer(cfg, gp, ga, dp, da, la, lb, stack)
 
     def _touched(self, r):
@@ -502,11 +515,11 @@ def job_throughput(per_rank_units, steps, world, max_seconds):
 def measure(args, name, rank, world, dist, peaks, primary):
     import torch
 
-    cfgname, M = WORKLOADS[name]
+    cfgname, M, storage = workload(name)
     cfg = workloads.CONFIGS[cfgname]
     dev = f"cuda:{torch.cuda.current_device()}"
     R = args.replicas if args.replicas > 0 else replicas_for(cfg, M)
-    b = Bench(cfg, M, dev, R, seed_base=rank)
+    b = Bench(cfg, M, dev, R, seed_base=rank, storage=storage)
     b.capture()
     b.run_steps(args.warmup)
     torch.cuda.synchronize()
@@ -558,6 +571,7 @@ def measure(args, name, rank, world, dist, peaks, primary):
                    "read, captured per replica"}
     res["cfg"] = cfg
     res["M"] = M
+    res["storage"] = storage
     del b
     torch.cuda.empty_cache()
     return res
@@ -567,8 +581,8 @@ def measure(args, name, rank, world, dist, peaks, primary):
 NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 
 
-def time_quantize(cfg, dev, reps=3):
-    """Load-time step, timed apart from the forward: e4b_nf4_quantize_stack on the
+def time_quantize(cfg, dev, reps=3, storage="nf4"):
+    """Load-time step, timed apart from the forward: e4b_quantize_stack on the
     layer's whole gate_up stack from fp32 ([E, 2I, H]); HBM-bound (4 B read +
     0.5 + 4/64 B written per weight)."""
     import torch
@@ -579,20 +593,76 @@ def time_quantize(cfg, dev, reps=3):
     n = W.numel()
     packed = torch.empty(n // 2, dtype=torch.uint8, device=dev)
     absmax = torch.empty(n // 64, dtype=torch.float32, device=dev)
-    e4b.e4b_nf4_quantize_stack(W, packed, absmax)
+    qt = STORAGE[storage]
+    e4b.e4b_quantize_stack(W, packed, absmax, qt)
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
     for _ in range(reps):
-        e4b.e4b_nf4_quantize_stack(W, packed, absmax)
+        e4b.e4b_quantize_stack(W, packed, absmax, qt)
     b.record()
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / reps
     nbytes = n * (4 + 0.5 + 4.0 / 64)
     del W, packed, absmax
     torch.cuda.empty_cache()
-    return {"stack": f"gate_up [{cfg.E}, {2 * cfg.I}, {cfg.H}] fp32", "ms": ms, "bytes": nbytes,
-            "GB_per_s": nbytes / (ms * 1e-3) / 1e9}
+    return {"stack": f"gate_up [{cfg.E}, {2 * cfg.I}, {cfg.H}] fp32", "storage": storage, "ms": ms,
+            "bytes": nbytes, "GB_per_s": nbytes / (ms * 1e-3) / 1e9}
+
+
+MXFP4_WORKLOAD = "gptoss_m8192"   # released MXFP4 experts: gpt-oss-shaped gate_up, prefill routing
+
+
+def time_mxfp4(name, dev, steps=5, warmup=2):
+    """The grouped GEMM straight from MXFP4 bytes (e4b_grouped_mxfp4_gemm) on the
+    gate_up projection of the workload's layer shape: the routed rows of the
+    workload's own routing (e4b_moe_route_permute), seeded random e2m1 codes and
+    e8m0 scales around 2^0, SwiGLU epilogue, bf16 out.  Algorithmic FLOPs
+    2*S*2I*H; timed apart from the forward with CUDA events on its stream."""
+    import torch
+
+    from quantized_moe_expert_nf4_b200 import e4b, synthetic
+
+    cfgname, M, _ = workload(name)
+    cfg = workloads.CONFIGS[cfgname]
+    E, H, I, k = cfg.E, cfg.H, cfg.I, cfg.k
+    S = M * k
+    x, logits = synthetic.inputs(cfg, M, device=dev)
+    ids = torch.empty((M, k), dtype=torch.int32, device=dev)
+    w = torch.empty((M, k), dtype=torch.float32, device=dev)
+    offs = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(S, dtype=torch.int32, device=dev)
+    inv = torch.empty(S, dtype=torch.int32, device=dev)
+    rws = e4b.workspace(e4b.e4b_moe_route_permute_workspace_size(M, E, k), dev)
+    e4b.e4b_moe_route_permute(logits, k, True, ids, w, offs, perm, inv, rws)
+    row_token = torch.div(perm, k, rounding_mode="floor").to(torch.int32)
+    g = torch.Generator(device=dev)
+    g.manual_seed(11)
+    N, K = 2 * I, H
+    blocks = torch.randint(0, 256, (E, N * K // 2), generator=g, device=dev, dtype=torch.uint8)
+    scales = torch.randint(124, 131, (E, N * K // 32), generator=g, device=dev, dtype=torch.uint8)
+    out = torch.empty((S, I), dtype=torch.bfloat16, device=dev)
+    ws = e4b.workspace(e4b.e4b_grouped_mxfp4_gemm_workspace_size(S, N, K), dev)
+
+    def call():
+        e4b.e4b_grouped_mxfp4_gemm(x, row_token, offs, S, blocks, scales, N, K, out, e4b.E4B_EPI_SWIGLU, ws)
+
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        call()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    flops = 2.0 * S * N * K
+    res = {"workload": name, "projection": f"gate_up [{E}, {N}, {K}] MXFP4", "routed_rows": S, "ms": ms,
+           "tflops": flops / (ms * 1e-3) / 1e12, "algorithmic_flops": flops, "path": e4b.last_path()}
+    del x, logits, ids, w, offs, perm, inv, rws, row_token, blocks, scales, out, ws
+    torch.cuda.empty_cache()
+    return res
 
 
 def repeat_forward(name, reps):
@@ -628,7 +698,7 @@ def time_backward(name, dev, steps=10, warmup=3):
 
     from quantized_moe_expert_nf4_b200 import e4b, synthetic
 
-    cfgname, M = WORKLOADS[name][:2]
+    cfgname, M, _ = workload(name)
     cfg = workloads.CONFIGS[cfgname]
     layer = synthetic.make_device_layer(cfg, device=dev)
     x, logits = synthetic.inputs(cfg, M, device=dev)
@@ -685,6 +755,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end host-buffer pass")
     ap.add_argument("--no-kernel-timing", action="store_true", help="skip the per-kernel event pass")
     ap.add_argument("--no-backward", action="store_true", help="skip the layer-backward timing")
+    ap.add_argument("--no-mxfp4", action="store_true", help="skip the MXFP4 grouped-GEMM timing")
     ap.add_argument("--replicas", type=int, default=0, help="layer replicas (0: enough to exceed L2 4x)")
     ap.add_argument("--repeat-forward", type=int, default=0, metavar="N",
                     help="profiling driver: build the workload's layer and call the forward N times, untimed")
@@ -698,7 +769,7 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    cfgname, M = WORKLOADS[args.workload]
+    cfgname, M, storage = workload(args.workload)
     cfg = workloads.CONFIGS[cfgname]
 
     if args.impl == "reference":
@@ -732,7 +803,8 @@ def main():
                 sweep.append({"workload": name, "error": f"{type(exc).__name__}: {exc}"})
                 torch.cuda.empty_cache()
                 continue
-            sweep.append({"workload": name, "value": r["value"], "ms_per_step": r["ms_per_step"],
+            sweep.append({"workload": name, "storage": r["storage"], "value": r["value"],
+                          "ms_per_step": r["ms_per_step"],
                           "tflops": r["tflops"], "path": r["path"], "touched_experts_avg": r["touched_experts_avg"],
                           "roofline_frac": r["roofline"]["frac"] if r["roofline"] else None,
                           "roofline_bound": r["roofline"]["bound"] if r["roofline"] else None,
@@ -741,16 +813,26 @@ def main():
                           "clocks": r["clocks"]})
     quant = None
     bwd = None
+    mx = None
     if rank == 0 and world == 1:
         quant = time_quantize(cfg, f"cuda:{local}")
         quant["frac_hbm"] = quant["GB_per_s"] / peaks["hbm_gbs"]
+        q4 = time_quantize(cfg, f"cuda:{local}", storage="fp4")
+        quant["fp4"] = {"GB_per_s": q4["GB_per_s"], "ms": q4["ms"], "frac_hbm": q4["GB_per_s"] / peaks["hbm_gbs"]}
+        if not args.no_mxfp4:
+            try:
+                mx = time_mxfp4(MXFP4_WORKLOAD, f"cuda:{local}")
+                mx["frac_tensor"] = mx["tflops"] / peaks["bf16_tflops"]
+            except Exception as exc:  # reported, the headline line still prints
+                mx = {"workload": MXFP4_WORKLOAD, "error": f"{type(exc).__name__}: {exc}"}
+                torch.cuda.empty_cache()
         if not args.no_backward:
             bwd = time_backward(BACKWARD_WORKLOAD, f"cuda:{local}")
             bwd["frac_tensor"] = bwd["tflops"] / peaks["bf16_tflops"]
     if rank == 0:
         cb = None
         if world == 1 and not args.no_cpu_baseline:
-            rate, desc, spent = oracle_rate(cfg, M, budget_s=12.0, max_tokens=8)
+            rate, desc, spent = oracle_rate(cfg, M, budget_s=12.0, max_tokens=8, storage=storage)
             cb = {"value": rate, "unit": "routed_tokens/s", "cores": cpu_cores(), "kind": "oracle", "sample": desc,
                   "seconds": spent}
         line = {
@@ -759,7 +841,7 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
             "config": {"workload": args.workload, "model": f"{cfg.name}-shaped MoE layer", "E": cfg.E, "H": cfg.H,
-                       "I": cfg.I, "k": cfg.k, "M": M, "routing": cfg.routing, "weights": "NF4/64 fp32 absmax",
+                       "I": cfg.I, "k": cfg.k, "M": M, "routing": cfg.routing, "weights": f"{storage.upper()}/64 fp32 absmax",
                        "replicas": main_res["replicas"],
                        "l2": f"inputs larger than L2: {main_res['replicas']} layer replicas cycled",
                        "global_batch": M * world, "parallelism": f"replicas x{world}", "timing": "CUDA graphs"},
@@ -772,6 +854,7 @@ def main():
             "gpu_launches": main_res["launches_per_step"] * args.steps,
             "quantize": quant,
             "backward": bwd,
+            "mxfp4_gemm": mx,
             "sweep": sweep,
         }
         print(json.dumps(line), flush=True)

@@ -58,7 +58,7 @@
 extern "C" {
 #endif
 
-#define E4B_VERSION 1
+#define E4B_VERSION 3
 
 #if defined(__GNUC__)
 #define E4B_API __attribute__((visibility("default")))
@@ -80,6 +80,19 @@ typedef enum {
   E4B_EPI_NONE = 0,  /* out = A_rows . W^T                                  */
   E4B_EPI_SWIGLU = 1 /* y = A_rows . W^T (+ LoRA); out = SiLU(y[:, :N/2]) * y[:, N/2:] */
 } e4b_epilogue;
+
+/*
+ * The 4-bit storage of a packed stack: which 16-entry codebook its codes
+ * index.  Both share the layout of e4b_quantize_stack() (blocks of 64, fp32
+ * absmax, two codes per byte, the lower-index element in the high nibble).
+ * Source: experts4bit-qlora 0.22.0, opening section and "Scope" (the storage
+ * modes nf4 and fp4 of one fused stack, with NF4 the more accurate).
+ */
+typedef enum {
+  E4B_QUANT_NF4 = 0, /* the NF4 table of the QLoRA paper, ascending, entry 7 = 0 */
+  E4B_QUANT_FP4 = 1  /* e2m1 codes over 6: code c = (-1)^(c>>3) * m[c & 7] / 6 with
+                        m = 0, 0.5, 1, 1.5, 2, 3, 4, 6 (codes 0 and 8 are zero) */
+} e4b_quant_type;
 
 /* Which implementation e4b_moe_expert_forward_path() runs. */
 typedef enum {
@@ -158,6 +171,19 @@ E4B_API e4b_status e4b_nf4_quantize_stack(const void* W, e4b_dtype w_dtype, int6
                                   e4b_stream stream);
 
 /*
+ * The same quantiser for either 4-bit storage (e4b_quant_type).  With
+ * E4B_QUANT_NF4 it is e4b_nf4_quantize_stack().  With E4B_QUANT_FP4 each code
+ * is the one whose value is nearest to s = w / absmax (one IEEE fp32
+ * division) in exact arithmetic; a value exactly between two values takes the
+ * smaller; zero is code 0 (code 8 is never written); an all-zero block stores
+ * absmax 0 and code 0.  Bit-exact by construction.  Same requirements as
+ * above; a quant_type other than the two is E4B_ERR_INVALID_ARGUMENT.
+ */
+E4B_API e4b_status e4b_quantize_stack(const void* W, e4b_dtype w_dtype, int64_t E, int64_t N, int64_t K,
+                                      int blocksize, e4b_quant_type quant_type, uint8_t* packed,
+                                      float* absmax, e4b_stream stream);
+
+/*
  * a2 + a3 -- router top-k and the token/expert permutation.
  * Source: experts4bit-qlora 0.22.0, "Which training path?" (sort the
  * token/expert pairs, run the groups); routing "softmax top-k renormalised".
@@ -225,6 +251,18 @@ E4B_API e4b_status e4b_grouped_nf4_gemm(const uint16_t* A, int64_t a_rows, int64
                                 e4b_dtype out_dtype, void* workspace, size_t workspace_bytes,
                                 e4b_stream stream);
 
+/* e4b_grouped_nf4_gemm() on a stack of either 4-bit storage: W_e =
+ * codebook(quant_type)[q] * absmax.  Same arguments, workspace and
+ * requirements; e4b_grouped_nf4_gemm() is this call with E4B_QUANT_NF4. */
+E4B_API e4b_status e4b_grouped_4bit_gemm(const uint16_t* A, int64_t a_rows, int64_t lda,
+                                 const int32_t* row_index, const int32_t* expert_offsets,
+                                 int64_t E, int64_t total_rows, const uint8_t* packed,
+                                 const float* absmax, e4b_quant_type quant_type, int64_t N,
+                                 int64_t K, const uint16_t* lora_A, const uint16_t* lora_B, int r,
+                                 float lora_scale, e4b_epilogue epi, void* out,
+                                 e4b_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                                 e4b_stream stream);
+
 /*
  * Backward through the frozen base -- the input gradient of the grouped NF4
  * GEMM above, in one launch over all groups.
@@ -245,6 +283,7 @@ E4B_API e4b_status e4b_grouped_nf4_gemm(const uint16_t* A, int64_t a_rows, int64
  * Requires K % 64 == 0, N % 64 == 0, 0 <= r <= 16, total_rows < 2^31.
  * workspace       e4b_grouped_nf4_gemm_dgrad_workspace_size() bytes: an error
  *                 word and the products dY . lora_B (total_rows x r fp32).
+ *                 0 bytes (NULL allowed) when total_rows == 0.
  * Groups with no rows cost nothing and write nothing.
  */
 E4B_API size_t e4b_grouped_nf4_gemm_dgrad_workspace_size(int64_t total_rows, int64_t N, int64_t K, int r);
@@ -255,6 +294,16 @@ E4B_API e4b_status e4b_grouped_nf4_gemm_dgrad(const uint16_t* dY, int64_t dy_row
                                       const uint16_t* lora_A, const uint16_t* lora_B, int r,
                                       float lora_scale, void* out, e4b_dtype out_dtype,
                                       void* workspace, size_t workspace_bytes, e4b_stream stream);
+
+/* e4b_grouped_nf4_gemm_dgrad() on a stack of either 4-bit storage; same
+ * arguments, workspace and requirements. */
+E4B_API e4b_status e4b_grouped_4bit_gemm_dgrad(const uint16_t* dY, int64_t dy_rows, int64_t lddy,
+                                       const int32_t* row_index, const int32_t* expert_offsets,
+                                       int64_t E, int64_t total_rows, const uint8_t* packed,
+                                       const float* absmax, e4b_quant_type quant_type, int64_t N,
+                                       int64_t K, const uint16_t* lora_A, const uint16_t* lora_B,
+                                       int r, float lora_scale, void* out, e4b_dtype out_dtype,
+                                       void* workspace, size_t workspace_bytes, e4b_stream stream);
 
 /*
  * The adapter's gradients of one grouped projection (backward of the
@@ -284,17 +333,49 @@ E4B_API e4b_status e4b_grouped_lora_grads(const uint16_t* x, int64_t x_rows, int
                                   float* dB, void* workspace, size_t workspace_bytes,
                                   e4b_stream stream);
 
+/*
+ * One grouped GEMM over E expert groups straight from MXFP4 expert bytes.
+ * Source: Solutions -- one page per problem, the grouped-nf4-gemm row on
+ * gemm_mxfp4_grouped (released e2m1 blocks and e8m0 scales multiplied as they
+ * are, no requantisation, no bf16 weight copy).
+ *
+ * As e4b_grouped_nf4_gemm() (row p of group e: y[p, :] = A[row_index[p], :] .
+ * W_e^T, the same epilogues, no adapter), with W_e in the OCP microscaling
+ * format: element (n, k) = e2m1(code) * 2^(scale - 127), where
+ *   blocks  [E, N*K/2] uint8: row n of expert e holds K/2 bytes, element 2i
+ *           of the row in the low nibble of byte i (the released layout);
+ *           e2m1 = sign (bit 3), exponent (bits 2-1, bias 1), mantissa (bit 0);
+ *   scales  [E, N*K/32] uint8: one e8m0 byte per 32 consecutive elements of a
+ *           row; 255 is NaN and makes its block NaN.
+ * Requires K % 64 == 0, N % 64 == 0.
+ * workspace  e4b_grouped_mxfp4_gemm_workspace_size() bytes: an error word and
+ *            room for the routed rows gathered in order (total_rows x K bf16),
+ *            which the tensor-core kernel (512 routed rows and more) reads as
+ *            contiguous tiles; the warp-MMA kernel below uses neither.  0 bytes
+ *            (NULL allowed) when total_rows == 0.
+ * Each e2m1 value and each scale is exact in bf16, so the products with the
+ * bf16 operand rows are the GEMM's only roundings (fp32 accumulation).
+ */
+E4B_API size_t e4b_grouped_mxfp4_gemm_workspace_size(int64_t total_rows, int64_t N, int64_t K);
+E4B_API e4b_status e4b_grouped_mxfp4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda,
+                                  const int32_t* row_index, const int32_t* expert_offsets,
+                                  int64_t E, int64_t total_rows, const uint8_t* blocks,
+                                  const uint8_t* scales, int64_t N, int64_t K, e4b_epilogue epi,
+                                  void* out, e4b_dtype out_dtype, void* workspace,
+                                  size_t workspace_bytes, e4b_stream stream);
+
 /* The two packed stacks of one MoE layer (device pointers), plus its adapter. */
 typedef struct {
-  const uint8_t* gu_packed; /* [E, 2I*H/2]  gate_up_proj, NF4 */
+  const uint8_t* gu_packed; /* [E, 2I*H/2]  gate_up_proj, 4-bit codes */
   const float* gu_absmax;   /* [E, 2I*H/64] */
-  const uint8_t* dn_packed; /* [E, H*I/2]   down_proj, NF4 */
+  const uint8_t* dn_packed; /* [E, H*I/2]   down_proj, 4-bit codes */
   const float* dn_absmax;   /* [E, H*I/64] */
   const uint16_t* lora_A;   /* [E, r, H] bf16 or NULL */
   const uint16_t* lora_B;   /* [E, 2I, r] bf16 or NULL */
   int lora_r;               /* 0 without an adapter */
   float lora_alpha;         /* scale = lora_alpha / lora_r */
   int64_t E, H, I;
+  int32_t quant_type;       /* e4b_quant_type of both stacks; 0 (zero-initialised) = NF4 */
 } e4b_expert_stack;
 
 /*

@@ -127,6 +127,7 @@ e4b_status cuda_fail(cudaError_t err, const char* where) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool quant_type_ok(int q) { return q == E4B_QUANT_NF4 || q == E4B_QUANT_FP4; }
 
 // Size, presence and alignment of a caller's workspace.
 e4b_status check_workspace(const char* what, size_t need, const void* workspace, size_t workspace_bytes) {
@@ -233,6 +234,7 @@ e4b_status check_stack(const e4b_expert_stack* w, int k) {
   if (k < 1 || k > w->E || k > 32) return fail(E4B_ERR_INVALID_ARGUMENT, "k must be in [1, min(E, 32)]");
   if (!w->gu_packed || !w->gu_absmax || !w->dn_packed || !w->dn_absmax)
     return fail(E4B_ERR_INVALID_ARGUMENT, "null packed stack pointer");
+  if (!quant_type_ok(w->quant_type)) return fail(E4B_ERR_INVALID_ARGUMENT, "quant_type must be NF4 or FP4");
   if ((w->lora_A == nullptr) != (w->lora_B == nullptr))
     return fail(E4B_ERR_INVALID_ARGUMENT, "lora_A and lora_B must be both set or both NULL");
   if (w->lora_A && (w->lora_r < 1 || w->lora_r > 16)) return fail(E4B_ERR_UNSUPPORTED, "LoRA rank must be in [1, 16]");
@@ -332,7 +334,13 @@ e4b_status e4b_timing_get(int i, const char** name, double* total_ms, int* launc
 
 e4b_status e4b_nf4_quantize_stack(const void* W, e4b_dtype w_dtype, int64_t E, int64_t N, int64_t K,
                                   int blocksize, uint8_t* packed, float* absmax, e4b_stream stream) {
+  return e4b_quantize_stack(W, w_dtype, E, N, K, blocksize, E4B_QUANT_NF4, packed, absmax, stream);
+}
+
+e4b_status e4b_quantize_stack(const void* W, e4b_dtype w_dtype, int64_t E, int64_t N, int64_t K, int blocksize,
+                              e4b_quant_type quant_type, uint8_t* packed, float* absmax, e4b_stream stream) {
   begin_call();
+  if (!quant_type_ok(quant_type)) return fail(E4B_ERR_INVALID_ARGUMENT, "quant_type must be NF4 or FP4");
   if (blocksize != 64) return fail(E4B_ERR_UNSUPPORTED, "blocksize must be 64, got " + std::to_string(blocksize));
   if (w_dtype != E4B_F32 && w_dtype != E4B_BF16) return fail(E4B_ERR_INVALID_ARGUMENT, "w_dtype must be F32 or BF16");
   if (E < 1 || N < 1 || K < 1)
@@ -344,7 +352,7 @@ e4b_status e4b_nf4_quantize_stack(const void* W, e4b_dtype w_dtype, int64_t E, i
     return fail(E4B_ERR_INVALID_ARGUMENT, "W, packed and absmax must be 16-byte aligned");
   if (e4b_status s = check_device(); s != E4B_OK) return s;
   const int64_t nblocks = E * N * K / 64;
-  cudaError_t err = launch_quantize(W, w_dtype == E4B_BF16, nblocks, packed, absmax, stream);
+  cudaError_t err = launch_quantize(W, w_dtype == E4B_BF16, nblocks, static_cast<int>(quant_type), packed, absmax, stream);
   if (err != cudaSuccess) return cuda_fail(err, "quantize launch");
   set_path("quantize");
   return E4B_OK;
@@ -388,7 +396,19 @@ e4b_status e4b_grouped_nf4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda, 
                                 const float* absmax, int64_t N, int64_t K, const uint16_t* lora_A,
                                 const uint16_t* lora_B, int r, float lora_scale, e4b_epilogue epi, void* out,
                                 e4b_dtype out_dtype, void* workspace, size_t workspace_bytes, e4b_stream stream) {
+  return e4b_grouped_4bit_gemm(A, a_rows, lda, row_index, expert_offsets, E, total_rows, packed, absmax,
+                               E4B_QUANT_NF4, N, K, lora_A, lora_B, r, lora_scale, epi, out, out_dtype, workspace,
+                               workspace_bytes, stream);
+}
+
+e4b_status e4b_grouped_4bit_gemm(const uint16_t* A, int64_t a_rows, int64_t lda, const int32_t* row_index,
+                                 const int32_t* expert_offsets, int64_t E, int64_t total_rows, const uint8_t* packed,
+                                 const float* absmax, e4b_quant_type quant_type, int64_t N, int64_t K,
+                                 const uint16_t* lora_A, const uint16_t* lora_B, int r, float lora_scale,
+                                 e4b_epilogue epi, void* out, e4b_dtype out_dtype, void* workspace,
+                                 size_t workspace_bytes, e4b_stream stream) {
   begin_call();
+  if (!quant_type_ok(quant_type)) return fail(E4B_ERR_INVALID_ARGUMENT, "quant_type must be NF4 or FP4");
   if (E < 1 || E > 65536) return fail(E4B_ERR_INVALID_ARGUMENT, "E must be in [1, 65536]");
   if (total_rows < 0 || a_rows < 0) return fail(E4B_ERR_INVALID_ARGUMENT, "total_rows and a_rows must be >= 0");
   if (total_rows > 0 && a_rows < 1) return fail(E4B_ERR_INVALID_ARGUMENT, "a_rows must be >= 1 when rows exist");
@@ -427,6 +447,7 @@ e4b_status e4b_grouped_nf4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda, 
   g.total_rows = total_rows;
   g.packed = packed;
   g.absmax = absmax;
+  g.quant = quant_type;
   g.N = static_cast<int>(N);
   g.K = static_cast<int>(K);
   g.lora_A = lora_A;
@@ -451,7 +472,7 @@ e4b_status e4b_grouped_nf4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda, 
 size_t e4b_grouped_nf4_gemm_dgrad_workspace_size(int64_t total_rows, int64_t N, int64_t K, int r) {
   (void)N;
   (void)K;
-  if (total_rows < 0 || r < 0 || N < 0) return 0;
+  if (total_rows <= 0 || r < 0 || N < 0) return 0;  // no rows: nothing launches, nothing waits
   return dgrad_workspace_bytes(total_rows, N, r);
 }
 
@@ -461,7 +482,19 @@ e4b_status e4b_grouped_nf4_gemm_dgrad(const uint16_t* dY, int64_t dy_rows, int64
                                       const uint16_t* lora_A, const uint16_t* lora_B, int r, float lora_scale,
                                       void* out, e4b_dtype out_dtype, void* workspace, size_t workspace_bytes,
                                       e4b_stream stream) {
+  return e4b_grouped_4bit_gemm_dgrad(dY, dy_rows, lddy, row_index, expert_offsets, E, total_rows, packed, absmax,
+                                     E4B_QUANT_NF4, N, K, lora_A, lora_B, r, lora_scale, out, out_dtype, workspace,
+                                     workspace_bytes, stream);
+}
+
+e4b_status e4b_grouped_4bit_gemm_dgrad(const uint16_t* dY, int64_t dy_rows, int64_t lddy, const int32_t* row_index,
+                                       const int32_t* expert_offsets, int64_t E, int64_t total_rows,
+                                       const uint8_t* packed, const float* absmax, e4b_quant_type quant_type,
+                                       int64_t N, int64_t K, const uint16_t* lora_A, const uint16_t* lora_B, int r,
+                                       float lora_scale, void* out, e4b_dtype out_dtype, void* workspace,
+                                       size_t workspace_bytes, e4b_stream stream) {
   begin_call();
+  if (!quant_type_ok(quant_type)) return fail(E4B_ERR_INVALID_ARGUMENT, "quant_type must be NF4 or FP4");
   if (E < 1 || E > 65536) return fail(E4B_ERR_INVALID_ARGUMENT, "E must be in [1, 65536]");
   if (total_rows < 0 || dy_rows < 0) return fail(E4B_ERR_INVALID_ARGUMENT, "total_rows and dy_rows must be >= 0");
   if (total_rows > 0 && dy_rows < 1) return fail(E4B_ERR_INVALID_ARGUMENT, "dy_rows must be >= 1 when rows exist");
@@ -480,7 +513,8 @@ e4b_status e4b_grouped_nf4_gemm_dgrad(const uint16_t* dY, int64_t dy_rows, int64
     return fail(E4B_ERR_INVALID_ARGUMENT, "dY, packed, absmax and out must be 16-byte aligned");
   if (lora_A && (!aligned16(lora_A) || !aligned16(lora_B)))
     return fail(E4B_ERR_INVALID_ARGUMENT, "lora_A and lora_B must be 16-byte aligned");
-  if (e4b_status s = check_workspace("dgrad", dgrad_workspace_bytes(total_rows, N, r), workspace, workspace_bytes);
+  if (e4b_status s = check_workspace("dgrad", total_rows > 0 ? dgrad_workspace_bytes(total_rows, N, r) : 0, workspace,
+                                     workspace_bytes);
       s != E4B_OK)
     return s;
   if (e4b_status s = check_device(); s != E4B_OK) return s;
@@ -498,6 +532,7 @@ e4b_status e4b_grouped_nf4_gemm_dgrad(const uint16_t* dY, int64_t dy_rows, int64
   d.total_rows = total_rows;
   d.packed = packed;
   d.absmax = absmax;
+  d.quant = quant_type;
   d.N = static_cast<int>(N);
   d.K = static_cast<int>(K);
   d.lora_A = r ? lora_A : nullptr;
@@ -606,6 +641,82 @@ e4b_status e4b_grouped_lora_grads(const uint16_t* x, int64_t x_rows, int64_t ldx
   return E4B_OK;
 }
 
+size_t e4b_grouped_mxfp4_gemm_workspace_size(int64_t total_rows, int64_t N, int64_t K) {
+  (void)N;
+  if (total_rows <= 0 || K < 0) return 0;  // no rows: nothing launches, nothing waits
+  return gemm_workspace_bytes(total_rows, K, 0);
+}
+
+e4b_status e4b_grouped_mxfp4_gemm(const uint16_t* A, int64_t a_rows, int64_t lda, const int32_t* row_index,
+                                  const int32_t* expert_offsets, int64_t E, int64_t total_rows,
+                                  const uint8_t* blocks, const uint8_t* scales, int64_t N, int64_t K,
+                                  e4b_epilogue epi, void* out, e4b_dtype out_dtype, void* workspace,
+                                  size_t workspace_bytes, e4b_stream stream) {
+  begin_call();
+  if (E < 1 || E > 65536) return fail(E4B_ERR_INVALID_ARGUMENT, "E must be in [1, 65536]");
+  if (total_rows < 0 || a_rows < 0) return fail(E4B_ERR_INVALID_ARGUMENT, "total_rows and a_rows must be >= 0");
+  if (total_rows > 0 && a_rows < 1) return fail(E4B_ERR_INVALID_ARGUMENT, "a_rows must be >= 1 when rows exist");
+  if (K < 64 || K % 64 != 0) return fail(E4B_ERR_UNSUPPORTED, "K must be a positive multiple of 64");
+  if (N < 64 || N % 64 != 0) return fail(E4B_ERR_UNSUPPORTED, "N must be a positive multiple of 64");
+  if (lda < K || lda % 8 != 0) return fail(E4B_ERR_INVALID_ARGUMENT, "lda must be >= K and a multiple of 8");
+  if (epi != E4B_EPI_NONE && epi != E4B_EPI_SWIGLU) return fail(E4B_ERR_INVALID_ARGUMENT, "unknown epilogue");
+  if (out_dtype != E4B_F32 && out_dtype != E4B_BF16) return fail(E4B_ERR_INVALID_ARGUMENT, "out_dtype must be F32 or BF16");
+  if (!expert_offsets || !blocks || !scales) return fail(E4B_ERR_INVALID_ARGUMENT, "null expert_offsets, blocks or scales");
+  if (total_rows > 0 && (!A || !out)) return fail(E4B_ERR_INVALID_ARGUMENT, "null A or out");
+  if (total_rows > INT32_MAX) return fail(E4B_ERR_UNSUPPORTED, "total_rows exceeds int32");
+  if ((A && !aligned16(A)) || !aligned16(blocks) || (out && !aligned16(out)))
+    return fail(E4B_ERR_INVALID_ARGUMENT, "A, blocks and out must be 16-byte aligned");
+  if (e4b_status s = check_workspace("mxfp4 gemm", total_rows > 0 ? gemm_workspace_bytes(total_rows, K, 0) : 0,
+                                     workspace, workspace_bytes);
+      s != E4B_OK)
+    return s;
+  if (e4b_status s = check_device(); s != E4B_OK) return s;
+  if (total_rows == 0) {
+    set_path("mxfp4.empty");
+    return E4B_OK;
+  }
+  Mxfp4Args m{};
+  m.A = A;
+  m.a_rows = a_rows;
+  m.lda = lda;
+  m.row_index = row_index;
+  m.offsets = expert_offsets;
+  m.E = static_cast<int>(E);
+  m.total_rows = total_rows;
+  m.blocks = blocks;
+  m.scales = scales;
+  m.N = static_cast<int>(N);
+  m.K = static_cast<int>(K);
+  m.epi = epi;
+  m.out = out;
+  m.out_bf16 = out_dtype == E4B_BF16;
+  GemmArgs g{};
+  g.A = A;
+  g.a_rows = a_rows;
+  g.lda = lda;
+  g.row_index = row_index;
+  g.offsets = expert_offsets;
+  g.E = static_cast<int>(E);
+  g.total_rows = total_rows;
+  g.packed = blocks;
+  g.mx_scales = scales;
+  g.quant = kQuantMxfp4;
+  g.N = static_cast<int>(N);
+  g.K = static_cast<int>(K);
+  g.err = static_cast<int*>(workspace);
+  g.a_gathered = row_index ? reinterpret_cast<uint16_t*>(static_cast<char*>(workspace) +
+                                                         gemm_workspace_gather_offset(total_rows, 0))
+                           : nullptr;
+  g.epi = epi;
+  g.out = out;
+  g.out_bf16 = out_dtype == E4B_BF16;
+  const char* path = "";
+  cudaError_t err = launch_grouped_mxfp4(g, m, reinterpret_cast<cudaStream_t>(stream), &path);
+  if (err != cudaSuccess) return cuda_fail(err, "grouped mxfp4 gemm launch");
+  set_path(path);
+  return E4B_OK;
+}
+
 static int stack_r(const e4b_expert_stack* w) { return w->lora_A ? w->lora_r : 0; }
 
 size_t e4b_moe_expert_forward_workspace_size(int64_t M, const e4b_expert_stack* w, int k) {
@@ -635,6 +746,7 @@ static e4b_status forward_grouped(const uint16_t* x, int64_t M, const float* log
   g.total_rows = S;
   g.packed = w->gu_packed;
   g.absmax = w->gu_absmax;
+  g.quant = w->quant_type;
   g.N = static_cast<int>(2 * w->I);
   g.K = static_cast<int>(w->H);
   g.lora_A = r ? w->lora_A : nullptr;
@@ -659,6 +771,7 @@ static e4b_status forward_grouped(const uint16_t* x, int64_t M, const float* log
   d.total_rows = S;
   d.packed = w->dn_packed;
   d.absmax = w->dn_absmax;
+  d.quant = w->quant_type;
   d.N = static_cast<int>(w->H);
   d.K = static_cast<int>(w->I);
   d.err = at<int>(ws, L.err);
@@ -769,6 +882,7 @@ e4b_status e4b_moe_expert_backward(const uint16_t* x, int64_t M, const float* ro
   g.total_rows = S;
   g.packed = w->gu_packed;
   g.absmax = w->gu_absmax;
+  g.quant = w->quant_type;
   g.N = 2 * I;
   g.K = H;
   g.lora_A = r ? w->lora_A : nullptr;
@@ -794,6 +908,7 @@ e4b_status e4b_moe_expert_backward(const uint16_t* x, int64_t M, const float* ro
   d.total_rows = S;
   d.packed = w->dn_packed;
   d.absmax = w->dn_absmax;
+  d.quant = w->quant_type;
   d.N = H;
   d.K = I;
   d.err = at<int>(ws, L.err);
@@ -815,6 +930,7 @@ e4b_status e4b_moe_expert_backward(const uint16_t* x, int64_t M, const float* ro
   dd.total_rows = S;
   dd.packed = w->dn_packed;
   dd.absmax = w->dn_absmax;
+  dd.quant = w->quant_type;
   dd.N = H;
   dd.K = I;
   dd.out = at<float>(ws, L.dh);
@@ -834,6 +950,7 @@ e4b_status e4b_moe_expert_backward(const uint16_t* x, int64_t M, const float* ro
   dg.total_rows = S;
   dg.packed = w->gu_packed;
   dg.absmax = w->gu_absmax;
+  dg.quant = w->quant_type;
   dg.N = 2 * I;
   dg.K = H;
   dg.lora_A = r ? w->lora_A : nullptr;

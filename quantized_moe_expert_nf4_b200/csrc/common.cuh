@@ -14,9 +14,28 @@
       0.33791524171829224f, 0.44070982933044434f, 0.5626170039176941f, 0.7229568362236023f, \
       1.0f
 
+// The FP4 codebook: code c is the e2m1 element (sign bit 3, exponent bits 2-1
+// with bias 1, mantissa bit 0; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6) divided by
+// 6, each entry the float nearest to that ratio (the divisions below are
+// correctly rounded).  Codes 0 and 8 are both zero.
+#define E4B_FP4_CODEBOOK_VALUES                                                                          \
+  0.0f, 0.5f / 6.0f, 1.0f / 6.0f, 1.5f / 6.0f, 2.0f / 6.0f, 3.0f / 6.0f, 4.0f / 6.0f, 1.0f, -0.0f,      \
+      -0.5f / 6.0f, -1.0f / 6.0f, -1.5f / 6.0f, -2.0f / 6.0f, -3.0f / 6.0f, -4.0f / 6.0f, -1.0f
+
 namespace e4b {
 
-static __device__ __constant__ float kNf4CodebookDev[16] = {E4B_NF4_CODEBOOK_VALUES};
+// The e2m1 element values themselves (MXFP4 codes, before their e8m0 block scale).
+#define E4B_E2M1_VALUES \
+  0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f, -0.0f, -0.5f, -1.0f, -1.5f, -2.0f, -3.0f, -4.0f, -6.0f
+
+// Indexed by storage: [0] NF4, [1] FP4 (the e4b_quant_type values), [2] MXFP4 e2m1.
+static __device__ __constant__ float kCodebooksDev[3][16] = {
+    {E4B_NF4_CODEBOOK_VALUES}, {E4B_FP4_CODEBOOK_VALUES}, {E4B_E2M1_VALUES}};
+
+// Entry c (0..15) of the table of storage `quant` (0 NF4, 1 FP4, 2 MXFP4; others NF4).
+__device__ __forceinline__ float codebook_entry(int quant, int c) {
+  return kCodebooksDev[(quant == 1 || quant == 2) ? quant : 0][c & 15];
+}
 
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
   return __uint_as_float(static_cast<uint32_t>(b) << 16);

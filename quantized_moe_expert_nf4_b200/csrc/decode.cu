@@ -86,6 +86,7 @@ struct FusedParams {
   const float* gu_absmax;
   const uint8_t* dn_packed;
   const float* dn_absmax;
+  int quant;                   // e4b_quant_type of both stacks (the table the decoders build)
   const uint16_t* lora_A;
   const uint16_t* lora_B;
   int r;
@@ -254,7 +255,7 @@ __device__ __forceinline__ void route_one(const FusedParams& p, int t, int* ids_
 }
 
 // Prologue: warps < M route one token each while the other warps build the
-// byte -> bf16x2 codebook table (entry b of lane l at b * 32 + l: low half the
+// byte -> bf16x2 table of the stacks' codebook (NF4 or FP4) (entry b of lane l at b * 32 + l: low half the
 // high nibble's value, i.e. element 2i, high half element 2i+1).  Then the
 // touched experts (ascending id) and slotmap[u][t] = slot of token t in expert
 // touched[u] (or -1).
@@ -266,7 +267,7 @@ __device__ void prologue(const FusedParams& p, uint32_t* lut, int* ids_s, float*
   if (warp < p.M) {
     route_one(p, warp, ids_s, w_s);
   } else {
-    const float cbl = kNf4CodebookDev[lane & 15];
+    const float cbl = codebook_entry(p.quant, lane & 15);
     for (int b = warp - p.M; b < 256; b += kWarps - p.M) {
       const float hi = __shfl_sync(0xffffffffu, cbl, b >> 4);
       const float lo = __shfl_sync(0xffffffffu, cbl, b & 15);
@@ -815,6 +816,7 @@ cudaError_t launch_decode_forward(const DecodeArgs& a, cudaStream_t stream) {
   p.gu_absmax = w->gu_absmax;
   p.dn_packed = w->dn_packed;
   p.dn_absmax = w->dn_absmax;
+  p.quant = w->quant_type;
   p.lora_A = r ? w->lora_A : nullptr;
   p.lora_B = r ? w->lora_B : nullptr;
   p.r = r;

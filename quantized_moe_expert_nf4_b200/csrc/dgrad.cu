@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(kThreads) grouped_nf4_dgrad_kernel(DgradArgs a
   int64_t row_begin, row_end;
   if (!find_group_tile(a.offsets, a.E, a.total_rows, kTileT, blockIdx.x, &e, &row_begin, &row_end)) return;
 
-  for (int b = tid; b < 256; b += kThreads) lut[b] = pack_bf16x2(kNf4CodebookDev[b >> 4], kNf4CodebookDev[b & 15]);
+  for (int b = tid; b < 256; b += kThreads) lut[b] = pack_bf16x2(codebook_entry(a.quant, b >> 4), codebook_entry(a.quant, b & 15));
   const int nrows = static_cast<int>(row_end - row_begin);
   for (int i = tid; i < kTileT; i += kThreads) {
     int64_t src = row_begin + i;

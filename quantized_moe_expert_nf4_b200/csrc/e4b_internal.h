@@ -36,18 +36,39 @@ void begin_call();  // resets the per-call launch counter
 e4b_status check_stack(const e4b_expert_stack* w, int k);  // stack pointers, shapes, alignment, LoRA rank, k
 e4b_status check_sm100();                                 // the current device is sm_100
 
-// The NF4 codebook as the library holds it (QLoRA table, ascending).
-extern const float kNf4Codebook[16];
+// The codebooks as the library holds them, indexed by e4b_quant_type: NF4
+// (QLoRA table, ascending) and FP4 (e2m1 / 6, in code order).
+extern const float kCodebooks[2][16];
 
-// Quantiser decision thresholds: T[c] is the smallest float strictly above
-// the exact midpoint (cb[c] + cb[c+1]) / 2, so that for any float s,
-// s > midpoint  <=>  s >= T[c].  T[15] = +inf.
-struct Nf4Thresholds {
+// Quantiser tables of one storage type.  The distinct codebook values in
+// ascending order are the levels; T[l] is the smallest float strictly above
+// the exact midpoint of levels l and l+1, so that for any float s,
+// s > midpoint  <=>  s >= T[l]; the unused tail of T is +inf.  The level of s
+// is the number of thresholds <= s; code[level] is the code written for it
+// (the lowest code holding that value); zero_code is written for an all-zero
+// block.
+struct QuantTables {
   float t[16];
+  uint32_t code[16];
+  uint32_t zero_code;
 };
-Nf4Thresholds nf4_thresholds();
+QuantTables quant_tables(int quant);
 
-cudaError_t launch_quantize(const void* W, bool bf16, int64_t nblocks, uint8_t* packed,
+// The quantiser kernel's lookup of a level: 128 cells of width 1/64 over s in
+// [-1, 1], each widened by kQuantCellSlack on both sides.  Cell c holds the one
+// decision threshold inside it (+inf if none; both codebooks' thresholds are
+// at least 0.079 apart, wider than a cell) and the codes written below and at
+// or above it.  Any s in the widened cell gets its code from one comparison.
+constexpr int kQuantCells = 128;
+constexpr double kQuantCellSlack = 1e-5;
+struct QuantCellTable {
+  uint2 cell[kQuantCells];  // x: threshold (float bits), y: code below | code at or above << 4
+  uint32_t zero_code;
+  int ok;                   // 0 if some widened cell held two thresholds
+};
+QuantCellTable quant_cell_table(int quant);
+
+cudaError_t launch_quantize(const void* W, bool bf16, int64_t nblocks, int quant, uint8_t* packed,
                             float* absmax, cudaStream_t stream);
 
 // ---- routing -------------------------------------------------------------
@@ -67,6 +88,11 @@ cudaError_t launch_gather_rows(const uint16_t* A, int64_t a_rows, int64_t lda, c
                                int K, uint16_t* out, cudaStream_t stream);
 
 // ---- grouped GEMM --------------------------------------------------------
+// Internal storage index of MXFP4 weights on the tensor-core kernel: e2m1 codes
+// (element 2i in the low nibble) with one e8m0 scale byte per 32 elements of a
+// row instead of an fp32 absmax per 64 (not an e4b_quant_type).
+constexpr int kQuantMxfp4 = 2;
+
 struct GemmArgs {
   const uint16_t* A;
   int64_t a_rows, lda;
@@ -75,7 +101,9 @@ struct GemmArgs {
   int E;
   int64_t total_rows;
   const uint8_t* packed;
-  const float* absmax;
+  const float* absmax;       // [E, N*K/64] (NF4, FP4)
+  const uint8_t* mx_scales;  // [E, N*K/32] e8m0 (quant == kQuantMxfp4; tensor-core kernel only)
+  int quant;  // e4b_quant_type of packed, or kQuantMxfp4
   int N, K;
   const uint16_t* lora_A;  // [E, r, K] or nullptr
   const uint16_t* lora_B;  // [E, N, r] or nullptr
@@ -112,6 +140,7 @@ struct DgradArgs {
   int64_t total_rows;
   const uint8_t* packed;
   const float* absmax;
+  int quant;  // e4b_quant_type of packed
   int N, K;
   const uint16_t* lora_A;  // [E, r, K] or nullptr
   const uint16_t* lora_B;  // [E, N, r] or nullptr
@@ -169,6 +198,28 @@ cudaError_t launch_token_sum(const float* dxg, const int32_t* inv, int64_t M, in
                              cudaStream_t stream);
 cudaError_t launch_router_grad(const float* logits, const int32_t* ids, const float* w, const float* dw, int64_t M,
                                int E, int k, bool renormalize, float* dlogits, cudaStream_t stream);
+
+// ---- grouped MXFP4 GEMM -------------------------------------------------------
+struct Mxfp4Args {
+  const uint16_t* A;
+  int64_t a_rows, lda;
+  const int32_t* row_index;  // nullable
+  const int32_t* offsets;    // [E+1]
+  int E;
+  int64_t total_rows;
+  const uint8_t* blocks;  // [E, N*K/2] e2m1 codes, element 2i in the low nibble
+  const uint8_t* scales;  // [E, N*K/32] e8m0
+  int N, K;
+  int epi;
+  void* out;
+  bool out_bf16;
+};
+cudaError_t launch_grouped_mxfp4_gemm(const Mxfp4Args& a, cudaStream_t stream);
+// Picks the kernel for an MXFP4 call as launch_grouped_gemm does for NF4 (the
+// tensor-core kernel from 512 routed rows, E4B_GEMM=mma|tc forces one): `a`
+// describes it for the tensor-core kernel (quant kQuantMxfp4, mx_scales, error
+// word and gather room in the workspace), `m` for the warp-MMA kernel.
+cudaError_t launch_grouped_mxfp4(const GemmArgs& a, const Mxfp4Args& m, cudaStream_t stream, const char** path);
 
 // ---- combine ---------------------------------------------------------------
 cudaError_t launch_combine(const uint16_t* z, const int32_t* inv, const float* w, int64_t M, int k,

@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(kThreads) grouped_nf4_mma_kernel(GemmArgs a) {
   if (!find_group_tile(a.offsets, a.E, a.total_rows, kTileT, blockIdx.x, &e, &row_begin, &row_end)) return;
 
   // byte b = (code of the even element << 4) | code of the odd element
-  for (int b = tid; b < 256; b += kThreads) lut[b] = pack_bf16x2(kNf4CodebookDev[b >> 4], kNf4CodebookDev[b & 15]);
+  for (int b = tid; b < 256; b += kThreads) lut[b] = pack_bf16x2(codebook_entry(a.quant, b >> 4), codebook_entry(a.quant, b & 15));
   const int nrows = static_cast<int>(row_end - row_begin);
   for (int i = tid; i < kTileT; i += kThreads) {
     int64_t src = row_begin + i;
@@ -322,6 +322,31 @@ int gemm_override() {
 }
 constexpr int64_t kTcMinRows = 512;
 }  // namespace
+
+cudaError_t launch_grouped_mxfp4(const GemmArgs& a, const Mxfp4Args& m, cudaStream_t stream, const char** path) {
+  const int ov = gemm_override();
+  GemmArgs c = a;
+  if (c.row_index && c.a_gathered) {
+    c.A = c.a_gathered;
+    c.a_rows = c.total_rows;
+    c.lda = c.K;
+    c.row_index = nullptr;
+  }
+  const bool swiglu = a.epi == E4B_EPI_SWIGLU;
+  const bool tc_ok = a.quant == kQuantMxfp4 && a.mx_scales != nullptr && !a.lora_B && tc_supported(c);
+  const bool use_tc = ov == 2 || (ov == 0 && tc_ok && a.total_rows >= kTcMinRows);
+  if (use_tc) {
+    if (!tc_ok) return cudaErrorNotSupported;
+    if (a.row_index) {
+      cudaError_t err = launch_gather_rows(a.A, a.a_rows, a.lda, a.row_index, a.total_rows, a.K, a.a_gathered, stream);
+      if (err != cudaSuccess) return err;
+    }
+    *path = swiglu ? "mxfp4.tc.swiglu" : "mxfp4.tc";
+    return launch_grouped_gemm_tc(c, c.err, stream);
+  }
+  *path = swiglu ? "mxfp4.mma.swiglu" : "mxfp4.mma";
+  return launch_grouped_mxfp4_gemm(m, stream);
+}
 
 cudaError_t launch_grouped_gemm(const GemmArgs& a, cudaStream_t stream, const char** path) {
   const int ov = gemm_override();

@@ -62,9 +62,13 @@ constexpr uint32_t kSmemMisc = 1024 + 512;       // alignment slack, barriers, T
 constexpr int kLoraCols = 64;                    // width of a row of scale * x . lora_A^T (bf16, zero past r)
 constexpr size_t kLoraPrepSmemMax = 192 * 1024;  // lora_A[e] staged by the prep kernel
 
-template <int BN_, int HALVES_, int NACC_>
+// ATMEM: the decoders write the decoded weight tile into tensor memory
+// (tcgen05.st) and the MMA reads A from there, so the tile never passes
+// through shared memory; the A stages take TMEM columns after the accumulators.
+template <int BN_, int HALVES_, int NACC_, bool ATMEM_ = false>
 struct TcShape {
   static constexpr int BN = BN_, HALVES = HALVES_, NACC = NACC_;
+  static constexpr bool ATMEM = ATMEM_;
   static constexpr int kRows = HALVES * kBM;        // weight rows per tile
   static constexpr int kTpr = kDecThreads / kRows;  // decoder threads per weight row
   static constexpr int kChunks = 8 / kTpr;          // 16-byte decoded chunks per thread per k block
@@ -72,11 +76,13 @@ struct TcShape {
   static constexpr uint32_t kBBytes = BN * 128;
   static constexpr uint32_t kTmaStageBytes = kPackedBytes + kBBytes;
   static constexpr int kAS = 2;
-  static constexpr uint32_t kAStageBytes = HALVES * kAHalfBytes;
+  static constexpr uint32_t kAStageBytes = ATMEM ? 0 : HALVES * kAHalfBytes;
   static constexpr int kKSFit =
       static_cast<int>((kSmemLimit - kSmemMisc - kOutBytes - kAS * kAStageBytes) / kTmaStageBytes);
   static constexpr int kKS = kKSFit < 6 ? kKSFit : 6;
   static constexpr uint32_t kCols = HALVES * BN;    // TMEM columns of one accumulator set
+  static constexpr uint32_t kACols = HALVES * 32;   // TMEM columns of one A stage (ATMEM): 64 k as bf16 pairs
+  static constexpr uint32_t kAColBase = kCols * NACC;
   static constexpr uint32_t kOffTma = 0;
   static constexpr uint32_t kOffA = kOffTma + kKS * kTmaStageBytes;
   static constexpr uint32_t kOffOut = kOffA + kAS * kAStageBytes;
@@ -86,7 +92,9 @@ struct TcShape {
   static constexpr uint32_t kSmemBytes = kOffTmemSlot + 16 + 1024;
   static_assert(kTpr == 2 || kTpr == 4, "decoder split");
   static_assert(kKS >= 2, "ring depth");
-  static_assert(kCols * NACC <= 512, "TMEM columns");
+  static_assert(kCols * NACC + (ATMEM ? kAS * kACols : 0) <= 512, "TMEM columns");
+  static_assert(!ATMEM || HALVES == 2, "the TMEM decoders cover two halves");
+  static_assert(kChunks >= 1 && kAColBase <= 512, "decoder chunks, TMEM A base");
   static_assert(BN % 16 == 0 && BN <= 256, "MMA N");
   static_assert(kSmemBytes <= kSmemLimit, "shared memory");
 };
@@ -105,6 +113,8 @@ struct TcParams {
   int* err;
   const uint16_t* lora_B;  // [E, N, r] bf16, or null (no LoRA step)
   int r;
+  int quant;                 // e4b_quant_type of the packed codes, or kQuantMxfp4
+  const uint8_t* mx_scales;  // kQuantMxfp4: [E*N, K/32] e8m0 scale bytes (absmax unused)
 };
 
 // The codebook's bf16 patterns split into low and high bytes, four entries per
@@ -113,30 +123,43 @@ struct CodebookBytes {
   uint32_t lo[4], hi[4];
 };
 
-__device__ __forceinline__ CodebookBytes codebook_bytes() {
+__device__ __forceinline__ CodebookBytes codebook_bytes(int quant) {
   CodebookBytes t{};
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
-    const uint32_t b = float_to_bf16_bits(kNf4CodebookDev[j]);
+    const uint32_t b = float_to_bf16_bits(codebook_entry(quant, j));
     t.lo[j >> 2] |= (b & 0xffu) << (8 * (j & 3));
     t.hi[j >> 2] |= (b >> 8) << (8 * (j & 3));
   }
   return t;
 }
 
+// Final interleaves of decode4: the packed order of the two elements of a byte.
+constexpr uint32_t kSelHiFirst0 = 0x4051u, kSelHiFirst1 = 0x6273u;  // element 2i in the high nibble (NF4, FP4)
+constexpr uint32_t kSelLoFirst0 = 0x5140u, kSelLoFirst1 = 0x7362u;  // element 2i in the low nibble (MXFP4)
+
 // Four nibbles (bits 0-15 of g: the low then the high nibble of two packed
-// bytes, i.e. elements 2i+1, 2i, 2i+3, 2i+2) -> two bf16x2 words in element
-// order.  A byte permute looks up entries 0-7 and 8-15 for all four nibbles at
-// once (its selector takes the nibbles' low three bits); a second permute
-// keeps, per nibble, the half its top bit names; a third interleaves the low
-// and high bytes.
-__device__ __forceinline__ void decode4(uint32_t g, const CodebookBytes& t, uint32_t* w0, uint32_t* w1) {
+// bytes) -> two bf16x2 words in element order.  A byte permute looks up
+// entries 0-7 and 8-15 for all four nibbles at once (its selector takes the
+// nibbles' low three bits); a second permute keeps, per nibble, the half its
+// top bit names; a third interleaves the low and high bytes, in the byte's
+// element order (sel0, sel1: kSelHiFirst* or kSelLoFirst*).
+__device__ __forceinline__ void decode4(uint32_t g, const CodebookBytes& t, uint32_t* w0, uint32_t* w1,
+                                        uint32_t sel0 = kSelHiFirst0, uint32_t sel1 = kSelHiFirst1) {
   const uint32_t s = g & 0x7777u;
   const uint32_t pick = ((g >> 1) & 0x4444u) | 0x3210u;  // field i: i, or i + 4 when nibble i >= 8
   const uint32_t lo = __byte_perm(__byte_perm(t.lo[0], t.lo[1], s), __byte_perm(t.lo[2], t.lo[3], s), pick);
   const uint32_t hi = __byte_perm(__byte_perm(t.hi[0], t.hi[1], s), __byte_perm(t.hi[2], t.hi[3], s), pick);
-  *w0 = __byte_perm(lo, hi, 0x4051u);  // (element 2i, element 2i+1)
-  *w1 = __byte_perm(lo, hi, 0x6273u);  // (element 2i+2, element 2i+3)
+  *w0 = __byte_perm(lo, hi, sel0);  // (element 2i, element 2i+1)
+  *w1 = __byte_perm(lo, hi, sel1);  // (element 2i+2, element 2i+3)
+}
+
+// 2^(x - 127) for an e8m0 scale byte, as a float (x = 0: the subnormal 2^-127;
+// x = 255: NaN).  Exact, and exact again after rounding to bf16.
+__device__ __forceinline__ float e8m0_scale(uint32_t x) {
+  if (x == 255u) return __uint_as_float(0x7fc00000u);
+  if (x == 0u) return __uint_as_float(0x00400000u);
+  return __uint_as_float(x << 23);
 }
 
 // Weight rows of the tile's halves.
@@ -166,6 +189,77 @@ __device__ __forceinline__ bool locate(const TcParams& p, int64_t t, int* e, int
   return true;
 }
 
+// Decoders of the TMEM-operand shape.  A warp may only reach the 32 TMEM lanes
+// of its quadrant (warp % 4), so warp w takes weight rows 32 (w % 4) + lane of
+// one half, and the four warps of a quadrant split (half, 32-k part); a thread
+// decodes its row's 32 k of the step into 16 bf16 pairs and stores them as 16
+// consecutive TMEM columns of its lane.
+template <class S>
+__device__ __forceinline__ void tmem_decoders(const TcParams& p, unsigned char* smem, uint64_t* tma_full,
+                                              uint64_t* a_empty, uint64_t* a_full, uint32_t tmem_base, int warp,
+                                              int lane) {
+  constexpr int BN = S::BN, KS = S::kKS, AS = S::kAS;
+  const int qd = warp & 3, c = (warp - kWarpDec) >> 2;
+  const int half = c >> 1, kpart = c & 1;
+  const int ri = qd * 32 + lane;
+  const int KB = p.K / 64;
+  const CodebookBytes cbt = codebook_bytes(p.quant);
+  uint32_t kbg = 0;
+  bool ok = true;
+  for (int64_t t = blockIdx.x; ok; t += gridDim.x) {
+    int e, n_tile;
+    int64_t rb, re;
+    if (!locate<BN>(p, t, &e, &rb, &re, &n_tile)) break;
+    int r0, r1;
+    tile_rows<S::HALVES>(p, n_tile, &r0, &r1);
+    const int n = (half ? r1 : r0) + ri;
+    const bool valid = n < p.N;
+    const float* am = p.absmax + (static_cast<int64_t>(e) * p.N + (valid ? n : 0)) * KB;
+    float sc_ring[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sc_ring[i] = (valid && i < KB) ? __ldg(am + i) : 0.0f;
+    for (int kb0 = 0; kb0 < KB && ok; kb0 += 4) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int kb = kb0 + i;
+        if (kb >= KB) break;
+        const float sc = sc_ring[i];
+        sc_ring[i] = (valid && kb + 4 < KB) ? __ldg(am + kb + 4) : 0.0f;
+        const int s = kbg % KS, a = kbg % AS;
+        if (!mbar_wait(&tma_full[s], (kbg / KS) & 1) ||
+            (kbg >= AS && !mbar_wait(&a_empty[a], ((kbg / AS) - 1) & 1))) {
+          record_error(p.err, kErrWaitFull);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint4 q = *reinterpret_cast<const uint4*>(smem + S::kOffTma + s * S::kTmaStageBytes +
+                                                        half * kPackedHalfBytes + ri * 32 + kpart * 16);
+        const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+        const __nv_bfloat162 s2 = __float2bfloat162_rn(sc);
+        uint32_t v[16];
+#pragma unroll
+        for (int cw = 0; cw < 4; ++cw) {
+          decode4(words[cw], cbt, &v[4 * cw], &v[4 * cw + 1]);
+          decode4(words[cw] >> 16, cbt, &v[4 * cw + 2], &v[4 * cw + 3]);
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          __nv_bfloat162 h2 = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&v[i]), s2);
+          v[i] = *reinterpret_cast<uint32_t*>(&h2);
+        }
+        tmem_st_32x32b_x16(
+            tmem_base + (static_cast<uint32_t>(qd * 32) << 16) + S::kAColBase + a * S::kACols + half * 32 + kpart * 16, v);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_full[a]);
+        ++kbg;
+      }
+    }
+  }
+}
+
 // Decoders of the dgrad product.  Thread dt takes rows n in [8o, 8o + 8) of the
 // K step and columns k in [4q, 4q + 4) of the tile (q = 0..63: the tile's 256
 // columns, o = 0..7).  The nibbles of row pairs (n, n+1) are interleaved so
@@ -182,7 +276,7 @@ __device__ __forceinline__ void dgrad_decoders(const TcParams& p, unsigned char*
   const int q = (dt & 7) | (((dt >> 5) & 7) << 3);
   const int o = ((dt >> 3) & 3) | ((dt >> 8) << 2);
   const int KB = p.K / 64, kbw = p.N / 64;
-  const CodebookBytes cbt = codebook_bytes();
+  const CodebookBytes cbt = codebook_bytes(p.quant);
   uint32_t kbg = 0;
   bool ok = true;
   for (int64_t t = blockIdx.x; ok; t += gridDim.x) {
@@ -384,8 +478,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             const uint32_t acc = (kb | kk) ? 1u : 0u;
             const uint64_t bd = smem_desc_sw128(b_addr + kk * 32);
 #pragma unroll
-            for (int h = 0; h < HALVES; ++h)
-              umma_bf16(d + h * BN, smem_desc_sw128(a_addr + h * kAHalfBytes + kk * 32), bd, idesc, acc);
+            for (int h = 0; h < HALVES; ++h) {
+              if constexpr (S::ATMEM)
+                umma_bf16_ts(d + h * BN, tmem_base + S::kAColBase + a * S::kACols + h * 32 + kk * 8, bd, idesc, acc);
+              else
+                umma_bf16(d + h * BN, smem_desc_sw128(a_addr + h * kAHalfBytes + kk * 32), bd, idesc, acc);
+            }
           }
           umma_commit(&tma_empty[s]);
           umma_commit(&a_empty[a]);
@@ -419,13 +517,21 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     }
   } else if (warp >= kWarpDec && warp < kWarpDec + kNumDecWarps) {
     // ------------------------------------------------------------- decoders
+    if constexpr (S::ATMEM) {
+      tmem_decoders<S>(p, smem, tma_full, a_empty, a_full, tmem_base, warp, lane);
+    } else {
     const int dt = tid - kWarpDec * 32;            // 0..511
     if constexpr (DG) {
       dgrad_decoders<S>(p, smem, tma_full, a_empty, a_full, dt, lane);
     } else {
     const int r = dt / S::kTpr, kq = dt % S::kTpr;  // weight row of the tile, part of the k block
     const int half = r >> 7, ri = r & 127;
-    const CodebookBytes cbt = codebook_bytes();
+    const CodebookBytes cbt = codebook_bytes(p.quant);
+    // MXFP4: low nibble first, and one e8m0 scale per 32 k -- this thread's
+    // 64 / kTpr k of a block lie inside scale (2 kb + 2 kq / kTpr) of the row.
+    const bool mx = p.quant == kQuantMxfp4;
+    const uint32_t sel0 = mx ? kSelLoFirst0 : kSelHiFirst0, sel1 = mx ? kSelLoFirst1 : kSelHiFirst1;
+    const int mx_sub = (2 * kq) / S::kTpr;
     uint32_t kbg = 0;
     bool ok = true;
     for (int64_t t = blockIdx.x; ok; t += gridDim.x) {
@@ -436,18 +542,21 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       tile_rows<HALVES>(p, n_tile, &r0, &r1);
       const int n = (half ? r1 : r0) + ri;
       const bool valid = n < p.N;
-      const float* am = p.absmax + (static_cast<int64_t>(e) * p.N + (valid ? n : 0)) * KB;
-      // absmax of the next 4 k blocks in flight (an L2 round trip outlasts one k block)
+      const int64_t wrow = static_cast<int64_t>(e) * p.N + (valid ? n : 0);
+      const float* am = mx ? nullptr : p.absmax + wrow * KB;
+      const uint8_t* ms = mx ? p.mx_scales + wrow * (2 * KB) + mx_sub : nullptr;
+      auto scale_of = [&](int kb) { return mx ? e8m0_scale(__ldg(ms + 2 * kb)) : __ldg(am + kb); };
+      // scales of the next 4 k blocks in flight (an L2 round trip outlasts one k block)
       float sc_ring[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) sc_ring[i] = (valid && i < KB) ? __ldg(am + i) : 0.0f;
+      for (int i = 0; i < 4; ++i) sc_ring[i] = (valid && i < KB) ? scale_of(i) : 0.0f;
       for (int kb0 = 0; kb0 < KB && ok; kb0 += 4) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int kb = kb0 + i;
           if (kb >= KB) break;
           const float sc = sc_ring[i];
-          sc_ring[i] = (valid && kb + 4 < KB) ? __ldg(am + kb + 4) : 0.0f;
+          sc_ring[i] = (valid && kb + 4 < KB) ? scale_of(kb + 4) : 0.0f;
           const int s = kbg % KS, a = kbg % AS;
           if (!mbar_wait(&tma_full[s], (kbg / KS) & 1) ||
               (kbg >= AS && !mbar_wait(&a_empty[a], ((kbg / AS) - 1) & 1))) {
@@ -477,8 +586,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           for (int c = 0; c < S::kChunks; ++c) {
             const uint32_t w = words[c];
             uint32_t v[4];
-            decode4(w, cbt, &v[0], &v[1]);
-            decode4(w >> 16, cbt, &v[2], &v[3]);
+            decode4(w, cbt, &v[0], &v[1], sel0, sel1);
+            decode4(w >> 16, cbt, &v[2], &v[3], sel0, sel1);
 #pragma unroll
             for (int by = 0; by < 4; ++by) {
               __nv_bfloat162 h2 = *reinterpret_cast<__nv_bfloat162*>(&v[by]);
@@ -523,6 +632,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         if (lane == 0) mbar_arrive(&a_full[a]);
         ++kbg;
       }
+    }
     }
     }
   } else if (warp < 4) {
@@ -661,6 +771,8 @@ cudaError_t launch_shape(const GemmArgs& a, int* err_word, cudaStream_t stream) 
                    CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   const bool lora = a.lora_B != nullptr && a.r > 0;
+  // The TMEM decoders have no LoRA step: their barrier phases would drift from the MMA issuer's.
+  if (S::ATMEM && lora) return cudaErrorInvalidValue;
   CUtensorMap tm_xa = tm_b;  // unused without LoRA
   if (lora && !make_map_2d(&tm_xa, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.xa, kLoraCols, a.total_rows, kLoraCols * 2, 64,
                            S::BN, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -670,6 +782,8 @@ cudaError_t launch_shape(const GemmArgs& a, int* err_word, cudaStream_t stream) 
   p.E = a.E;
   p.total_rows = a.total_rows;
   p.absmax = a.absmax;
+  p.quant = a.quant;
+  p.mx_scales = a.mx_scales;
   p.N = a.N;
   p.K = a.K;
   p.swiglu = a.epi == E4B_EPI_SWIGLU;
@@ -685,7 +799,9 @@ cudaError_t launch_shape(const GemmArgs& a, int* err_word, cudaStream_t stream) 
   const int64_t tiles =
       ((a.total_rows + S::BN - 1) / S::BN + (a.E < a.total_rows ? a.E : a.total_rows)) * p.n_tiles;
   const int grid = static_cast<int>(tiles < di.sm_count ? tiles : di.sm_count);
-  LaunchScope ls(p.swiglu ? "gemm.tc.swiglu" : "gemm.tc", stream);
+  const bool mx = a.quant == kQuantMxfp4;
+  if (mx && (S::ATMEM || lora || a.mx_scales == nullptr)) return cudaErrorInvalidValue;
+  LaunchScope ls(mx ? (p.swiglu ? "mxfp4.tc.swiglu" : "mxfp4.tc") : (p.swiglu ? "gemm.tc.swiglu" : "gemm.tc"), stream);
   grouped_nf4_tc_kernel<S, false><<<grid, kThreadsTc, S::kSmemBytes, stream>>>(tm_packed, tm_b, tm_out, tm_xa, p);
   return cudaGetLastError();
 }
@@ -718,6 +834,7 @@ cudaError_t launch_dgrad_shape(const DgradArgs& a, const uint16_t* dy, int64_t d
   p.E = a.E;
   p.total_rows = a.total_rows;
   p.absmax = a.absmax;
+  p.quant = a.quant;
   p.N = a.K;  // tile rows: columns k of W
   p.K = a.N;  // K steps: rows n of W
   p.swiglu = 0;
@@ -737,10 +854,10 @@ cudaError_t launch_dgrad_shape(const DgradArgs& a, const uint16_t* dy, int64_t d
 }
 
 // LoRA prep for the tensor-core kernel: one CTA per (group, 64-row tile),
-// lora_A[e] (r x K bf16) staged in shared memory, one warp per routed row.
-// The warp copies the row into `gathered` (when a row index is given) and
-// writes xa[p, 0:64] = bf16(scale * A_row . lora_A[e, j]) for j < r, zeros
-// after -- the B operand of the kernel's extra K=16 MMA step.
+// lora_A[e] staged in shared memory.  It copies the tile's routed rows into
+// `gathered` (when a row index is given) and writes xa[p, 0:64] =
+// bf16(scale * A_row . lora_A[e, j]) for j < r, zeros after -- the B operand
+// of the GEMM kernel's extra K=16 MMA step.
 struct PrepParams {
   const uint16_t* A;
   int64_t a_rows, lda;
@@ -757,17 +874,35 @@ struct PrepParams {
 };
 
 constexpr int kPrepRows = 64;
+constexpr int kPrepUnroll = 4;  // 32-k chunks of the two rows' loads in flight per lane
 
-__global__ void __launch_bounds__(256) lora_prep_kernel(PrepParams q) {
-  extern __shared__ __align__(16) uint16_t la_s[];  // [r, K]
+__device__ __forceinline__ void mma_bf16_16816(float c[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Warp w takes routed rows 16w .. 16w + 15 of the tile as the rows of an
+// m16n8k16 MMA and the adapter rows (16, zero past r) as its columns; lane
+// (g, t) loads physical k [8t, 8t + 8) of each 32-k chunk of rows g and g + 8
+// as one 16-byte vector -- the A fragments of two MMAs, with K permuted the
+// same way for lora_A (rows g and g + 8 of its staged copy) -- and stores the
+// same vectors into `gathered`.  The loads are HBM-bound; the products cost a
+// few MMAs per 1 KB read.
+__global__ void __launch_bounds__(128) lora_prep_kernel(PrepParams q) {
+  extern __shared__ __align__(16) uint16_t la_s[];  // [16, K + 8]: lora_A[e], rows past r zero
   __shared__ int64_t tile_s[3];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
   if (warp == 0) {
-    int g;
+    int ge;
     int64_t b0, b1;
-    const bool found = find_group_tile(q.offsets, q.E, q.total_rows, kPrepRows, blockIdx.x, &g, &b0, &b1);
+    const bool found = find_group_tile(q.offsets, q.E, q.total_rows, kPrepRows, blockIdx.x, &ge, &b0, &b1);
     if (lane == 0) {
-      tile_s[0] = found ? g : -1;
+      tile_s[0] = found ? ge : -1;
       tile_s[1] = b0;
       tile_s[2] = b1;
     }
@@ -776,51 +911,73 @@ __global__ void __launch_bounds__(256) lora_prep_kernel(PrepParams q) {
   const int e = static_cast<int>(tile_s[0]);
   if (e < 0) return;
   const int64_t rb = tile_s[1], re = tile_s[2];
-  const int K = q.K, kv = K / 8;
+  const int K = q.K, kv = K / 8, ls = K + 8;  // shared row stride (bf16): 16 bytes of padding per row
   const uint4* src_a = reinterpret_cast<const uint4*>(q.lora_A + static_cast<int64_t>(e) * q.r * K);
-  for (int i = threadIdx.x; i < q.r * kv; i += blockDim.x) reinterpret_cast<uint4*>(la_s)[i] = src_a[i];
+  for (int i = threadIdx.x; i < 16 * kv; i += blockDim.x) {
+    const int row = i / kv, c = i % kv;
+    reinterpret_cast<uint4*>(la_s + row * ls)[c] = row < q.r ? src_a[row * kv + c] : make_uint4(0, 0, 0, 0);
+  }
   __syncthreads();
-  for (int64_t pr = rb + warp; pr < re; pr += blockDim.x / 32) {
-    int64_t src = q.row_index ? q.row_index[pr] : pr;
-    src = clampv<int64_t>(src, 0, q.a_rows - 1);
-    const uint4* xrow = reinterpret_cast<const uint4*>(q.A + src * q.lda);
-    uint4* grow = q.gathered ? reinterpret_cast<uint4*>(q.gathered + pr * K) : nullptr;
-    float acc[16];
+  const int64_t p0 = rb + 16 * warp + g, p1 = p0 + 8;
+  const bool v0 = p0 < re, v1 = p1 < re;
+  int64_t s0 = v0 ? (q.row_index ? q.row_index[p0] : p0) : 0;
+  int64_t s1 = v1 ? (q.row_index ? q.row_index[p1] : p1) : 0;
+  s0 = clampv<int64_t>(s0, 0, q.a_rows - 1);
+  s1 = clampv<int64_t>(s1, 0, q.a_rows - 1);
+  const uint4* x0 = reinterpret_cast<const uint4*>(q.A + s0 * q.lda);
+  const uint4* x1 = reinterpret_cast<const uint4*>(q.A + s1 * q.lda);
+  uint4* g0 = (q.gathered && v0) ? reinterpret_cast<uint4*>(q.gathered + p0 * K) : nullptr;
+  uint4* g1 = (q.gathered && v1) ? reinterpret_cast<uint4*>(q.gathered + p1 * K) : nullptr;
+  const bool two = q.r > 8;  // adapter rows 8..15 need the second n tile
+  float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+  const int nchunks = K / 32;
+  for (int ch0 = 0; ch0 < nchunks; ch0 += kPrepUnroll) {
+    uint4 xa0[kPrepUnroll], xa1[kPrepUnroll];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) acc[j] = 0.f;
-    for (int c = lane; c < kv; c += 32) {
-      const uint4 xv = __ldg(xrow + c);
-      if (grow) grow[c] = xv;
-      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+    for (int u = 0; u < kPrepUnroll; ++u) {
+      const int c = (ch0 + u) * 4 + t;  // 16-byte vector index within the row
+      const bool in = ch0 + u < nchunks;
+      xa0[u] = (in && v0) ? __ldg(x0 + c) : make_uint4(0, 0, 0, 0);
+      xa1[u] = (in && v1) ? __ldg(x1 + c) : make_uint4(0, 0, 0, 0);
+    }
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        if (j >= q.r) break;
-        const uint4 av = reinterpret_cast<const uint4*>(la_s + j * K)[c];
-        const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          acc[j] = fmaf(__uint_as_float(xw[i] << 16), __uint_as_float(aw[i] << 16), acc[j]);
-          acc[j] = fmaf(__uint_as_float(xw[i] & 0xffff0000u), __uint_as_float(aw[i] & 0xffff0000u), acc[j]);
-        }
+    for (int u = 0; u < kPrepUnroll; ++u) {
+      if (ch0 + u >= nchunks) break;
+      const int c = (ch0 + u) * 4 + t;
+      if (g0) g0[c] = xa0[u];
+      if (g1) g1[c] = xa1[u];
+      const uint4 b = reinterpret_cast<const uint4*>(la_s + g * ls)[c];
+      mma_bf16_16816(c0, xa0[u].x, xa1[u].x, xa0[u].y, xa1[u].y, b.x, b.y);
+      mma_bf16_16816(c0, xa0[u].z, xa1[u].z, xa0[u].w, xa1[u].w, b.z, b.w);
+      if (two) {
+        const uint4 b2 = reinterpret_cast<const uint4*>(la_s + (g + 8) * ls)[c];
+        mma_bf16_16816(c1, xa0[u].x, xa1[u].x, xa0[u].y, xa1[u].y, b2.x, b2.y);
+        mma_bf16_16816(c1, xa0[u].z, xa1[u].z, xa0[u].w, xa1[u].w, b2.z, b2.w);
       }
     }
-    float v0 = 0.f, v1 = 0.f;
+  }
+  // c0[0..1]: row g, adapter columns 2t, 2t + 1; c0[2..3]: row g + 8; c1: columns 8 + 2t, 8 + 2t + 1.
+  // Columns 16..63 of an xa row are zero: lane t writes words 8 + 6t .. 8 + 6t + 5.
+  if (v0) {
+    uint32_t* row = reinterpret_cast<uint32_t*>(q.xa + p0 * kLoraCols);
+    row[t] = pack_bf16x2(q.scale * c0[0], q.scale * c0[1]);
+    row[4 + t] = pack_bf16x2(q.scale * c1[0], q.scale * c1[1]);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      if (j >= q.r) break;
-      float v = acc[j];
+    for (int i = 0; i < 6; ++i) row[8 + 6 * t + i] = 0u;
+  }
+  if (v1) {
+    uint32_t* row = reinterpret_cast<uint32_t*>(q.xa + p1 * kLoraCols);
+    row[t] = pack_bf16x2(q.scale * c0[2], q.scale * c0[3]);
+    row[4 + t] = pack_bf16x2(q.scale * c1[2], q.scale * c1[3]);
 #pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (j == 2 * lane) v0 = v;
-      if (j == 2 * lane + 1) v1 = v;
-    }
-    reinterpret_cast<uint32_t*>(q.xa + pr * kLoraCols)[lane] = pack_bf16x2(q.scale * v0, q.scale * v1);
+    for (int i = 0; i < 6; ++i) row[8 + 6 * t + i] = 0u;
   }
 }
 
 using ShapeWide = TcShape<256, 2, 1>;    // 2 x 128 weight rows x 256 routed rows, one accumulator set
 using ShapeDouble = TcShape<128, 2, 2>;  // 2 x 128 x 128, two accumulator sets
 using ShapeNarrow = TcShape<256, 1, 2>;  // 128 x 256, two accumulator sets (no SwiGLU)
+using ShapeTmem = TcShape<192, 2, 1, true>;  // 2 x 128 x 192, A in TMEM (no LoRA step)
 
 int shape_override() {
   const char* v = getenv("E4B_TC_SHAPE");
@@ -828,6 +985,7 @@ int shape_override() {
   if (!strcmp(v, "wide")) return 1;
   if (!strcmp(v, "double")) return 2;
   if (!strcmp(v, "narrow")) return 3;
+  if (!strcmp(v, "tmem")) return 4;
   return 0;
 }
 
@@ -878,7 +1036,7 @@ bool tc_supported(const GemmArgs& a) {
   // kernel's shared memory and the products need their workspace rows.
   if (a.row_index != nullptr || a.lda % 8 != 0 || !tensor_maps_available()) return false;
   if (a.lora_B && a.r > 0)
-    return a.r <= 16 && a.xa != nullptr && static_cast<size_t>(a.r) * a.K * 2 <= kLoraPrepSmemMax &&
+    return a.r <= 16 && a.xa != nullptr && static_cast<size_t>(16) * (a.K + 8) * 2 <= kLoraPrepSmemMax &&
            (reinterpret_cast<uintptr_t>(a.lora_A) & 15u) == 0;
   return true;
 }
@@ -894,6 +1052,8 @@ cudaError_t launch_grouped_gemm_tc(const GemmArgs& a, int* err_word, cudaStream_
     const int64_t rows_per_group = a.total_rows / (a.E > 0 ? a.E : 1);
     s = swiglu ? 1 : (rows_per_group >= 512 ? 1 : 3);
   }
+  if (s == 4 && !(a.lora_B && a.r > 0) && a.quant != kQuantMxfp4) return launch_shape<ShapeTmem>(a, err_word, stream);
+  if (s == 4) s = swiglu ? 1 : 3;
   if (s == 1) return launch_shape<ShapeWide>(a, err_word, stream);
   if (s == 2) return launch_shape<ShapeDouble>(a, err_word, stream);
   return launch_shape<ShapeNarrow>(a, err_word, stream);
@@ -930,12 +1090,12 @@ cudaError_t launch_tc_lora_prep(const GemmArgs& a, cudaStream_t stream) {
   q.r = a.r;
   q.scale = a.lora_scale;
   q.xa = reinterpret_cast<uint16_t*>(a.xa);
-  const size_t smem = static_cast<size_t>(a.r) * a.K * 2;
+  const size_t smem = static_cast<size_t>(16) * (a.K + 8) * 2;
   cudaError_t err = ensure_smem_limit(reinterpret_cast<const void*>(lora_prep_kernel), smem);
   if (err != cudaSuccess) return err;
   const int64_t tiles = (a.total_rows + kPrepRows - 1) / kPrepRows + (a.E < a.total_rows ? a.E : a.total_rows);
   LaunchScope ls("gemm.tc.lora_prep", stream);
-  lora_prep_kernel<<<static_cast<unsigned>(tiles), 256, smem, stream>>>(q);
+  lora_prep_kernel<<<static_cast<unsigned>(tiles), 128, smem, stream>>>(q);
   return cudaGetLastError();
 }
 

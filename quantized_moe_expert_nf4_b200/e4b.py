@@ -26,17 +26,21 @@ STATUS_NAMES = {0: "E4B_OK", 1: "E4B_ERR_INVALID_ARGUMENT", 2: "E4B_ERR_UNSUPPOR
 E4B_F32, E4B_BF16 = 0, 1
 E4B_EPI_NONE, E4B_EPI_SWIGLU = 0, 1
 E4B_PATH_AUTO, E4B_PATH_DECODE, E4B_PATH_GROUPED = 0, 1, 2
+E4B_QUANT_NF4, E4B_QUANT_FP4 = 0, 1
+# The E4B_VERSION this binding marshals for (e4b_expert_stack's layout among others).
+ABI_VERSION = 3
 
 # Every symbol include/e4b.h declares.
 EXPORTED = (
     "e4b_status_string", "e4b_last_error", "e4b_last_path", "e4b_version", "e4b_last_launches",
     "e4b_workspace_error", "e4b_workspace_clear_error",
     "e4b_timing_enable", "e4b_timing_kernels", "e4b_timing_get",
-    "e4b_nf4_quantize_stack",
+    "e4b_nf4_quantize_stack", "e4b_quantize_stack",
     "e4b_moe_route_permute_workspace_size", "e4b_moe_route_permute",
-    "e4b_grouped_nf4_gemm_workspace_size", "e4b_grouped_nf4_gemm",
-    "e4b_grouped_nf4_gemm_dgrad_workspace_size", "e4b_grouped_nf4_gemm_dgrad",
+    "e4b_grouped_nf4_gemm_workspace_size", "e4b_grouped_nf4_gemm", "e4b_grouped_4bit_gemm",
+    "e4b_grouped_nf4_gemm_dgrad_workspace_size", "e4b_grouped_nf4_gemm_dgrad", "e4b_grouped_4bit_gemm_dgrad",
     "e4b_grouped_lora_grads_workspace_size", "e4b_grouped_lora_grads",
+    "e4b_grouped_mxfp4_gemm_workspace_size", "e4b_grouped_mxfp4_gemm",
     "e4b_moe_expert_forward_workspace_size", "e4b_moe_expert_forward",
     "e4b_moe_expert_forward_path", "e4b_moe_expert_forward_decode_noalloc",
     "e4b_moe_expert_backward_workspace_size", "e4b_moe_expert_backward",
@@ -56,6 +60,7 @@ class ExpertStackC(ctypes.Structure):
         ("lora_A", ctypes.c_void_p), ("lora_B", ctypes.c_void_p),
         ("lora_r", ctypes.c_int), ("lora_alpha", ctypes.c_float),
         ("E", ctypes.c_int64), ("H", ctypes.c_int64), ("I", ctypes.c_int64),
+        ("quant_type", ctypes.c_int32),
     ]
 
 
@@ -79,6 +84,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.e4b_last_path.argtypes = []
     lib.e4b_version.restype = i32
     lib.e4b_version.argtypes = []
+    if lib.e4b_version() != ABI_VERSION:
+        raise RuntimeError(f"{path} is ABI version {lib.e4b_version()}, this binding expects {ABI_VERSION}: "
+                           "rebuild it with __graft_entry__.build()")
     lib.e4b_last_launches.restype = i32
     lib.e4b_last_launches.argtypes = []
     lib.e4b_timing_enable.restype = i32
@@ -90,6 +98,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                    ctypes.POINTER(ctypes.c_int)]
     lib.e4b_nf4_quantize_stack.restype = i32
     lib.e4b_nf4_quantize_stack.argtypes = [vp, i32, i64, i64, i64, i32, vp, vp, vp]
+    lib.e4b_quantize_stack.restype = i32
+    lib.e4b_quantize_stack.argtypes = [vp, i32, i64, i64, i64, i32, i32, vp, vp, vp]
     lib.e4b_moe_route_permute_workspace_size.restype = sz
     lib.e4b_moe_route_permute_workspace_size.argtypes = [i64, i64, i32]
     lib.e4b_moe_route_permute.restype = i32
@@ -99,16 +109,27 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.e4b_grouped_nf4_gemm.restype = i32
     lib.e4b_grouped_nf4_gemm.argtypes = [vp, i64, i64, vp, vp, i64, i64, vp, vp, i64, i64, vp, vp, i32,
                                          ctypes.c_float, i32, vp, i32, vp, sz, vp]
+    lib.e4b_grouped_4bit_gemm.restype = i32
+    lib.e4b_grouped_4bit_gemm.argtypes = [vp, i64, i64, vp, vp, i64, i64, vp, vp, i32, i64, i64, vp, vp, i32,
+                                          ctypes.c_float, i32, vp, i32, vp, sz, vp]
     lib.e4b_grouped_nf4_gemm_dgrad_workspace_size.restype = sz
     lib.e4b_grouped_nf4_gemm_dgrad_workspace_size.argtypes = [i64, i64, i64, i32]
     lib.e4b_grouped_nf4_gemm_dgrad.restype = i32
     lib.e4b_grouped_nf4_gemm_dgrad.argtypes = [vp, i64, i64, vp, vp, i64, i64, vp, vp, i64, i64, vp, vp, i32,
                                                ctypes.c_float, vp, i32, vp, sz, vp]
+    lib.e4b_grouped_4bit_gemm_dgrad.restype = i32
+    lib.e4b_grouped_4bit_gemm_dgrad.argtypes = [vp, i64, i64, vp, vp, i64, i64, vp, vp, i32, i64, i64, vp, vp,
+                                                i32, ctypes.c_float, vp, i32, vp, sz, vp]
     lib.e4b_grouped_lora_grads_workspace_size.restype = sz
     lib.e4b_grouped_lora_grads_workspace_size.argtypes = [i64, i32]
     lib.e4b_grouped_lora_grads.restype = i32
     lib.e4b_grouped_lora_grads.argtypes = [vp, i64, i64, vp, vp, i64, i64, vp, i64, i64, i64, vp, vp, i32,
                                            ctypes.c_float, vp, vp, vp, sz, vp]
+    lib.e4b_grouped_mxfp4_gemm.restype = i32
+    lib.e4b_grouped_mxfp4_gemm_workspace_size.restype = sz
+    lib.e4b_grouped_mxfp4_gemm_workspace_size.argtypes = [i64, i64, i64]
+    lib.e4b_grouped_mxfp4_gemm.argtypes = [vp, i64, i64, vp, vp, i64, i64, vp, vp, i64, i64, i32, vp, i32, vp, sz,
+                                           vp]
     lib.e4b_moe_expert_forward_workspace_size.restype = sz
     lib.e4b_moe_expert_forward_workspace_size.argtypes = [i64, ctypes.POINTER(ExpertStackC), i32]
     lib.e4b_moe_expert_forward.restype = i32
@@ -179,9 +200,7 @@ def _stream(stream) -> Optional[int]:
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
-def e4b_nf4_quantize_stack(W: torch.Tensor, packed: torch.Tensor, absmax: torch.Tensor,
-                           blocksize: int = 64, stream=None) -> None:
-    """W [E, N, K] fp32/bf16 -> packed [E, N*K/2] uint8, absmax [E, N*K/64] fp32."""
+def _quantize_args(W, packed, absmax):
     _dev(W, "W")
     _dev(packed, "packed", torch.uint8)
     _dev(absmax, "absmax", torch.float32)
@@ -193,9 +212,25 @@ def e4b_nf4_quantize_stack(W: torch.Tensor, packed: torch.Tensor, absmax: torch.
         raise ValueError("W must be float32 or bfloat16")
     if packed.numel() < E * N * K // 2 or absmax.numel() < E * N * K // 64:
         raise ValueError("packed/absmax too small")
+    return dt, E, N, K
+
+
+def e4b_nf4_quantize_stack(W: torch.Tensor, packed: torch.Tensor, absmax: torch.Tensor,
+                           blocksize: int = 64, stream=None) -> None:
+    """W [E, N, K] fp32/bf16 -> packed [E, N*K/2] uint8, absmax [E, N*K/64] fp32."""
+    dt, E, N, K = _quantize_args(W, packed, absmax)
     _check(load_library().e4b_nf4_quantize_stack(W.data_ptr(), dt, E, N, K, blocksize, packed.data_ptr(),
                                                  absmax.data_ptr(), _stream(stream)),
            "e4b_nf4_quantize_stack")
+
+
+def e4b_quantize_stack(W: torch.Tensor, packed: torch.Tensor, absmax: torch.Tensor,
+                       quant_type: int = E4B_QUANT_NF4, blocksize: int = 64, stream=None) -> None:
+    """As e4b_nf4_quantize_stack, for either 4-bit storage (E4B_QUANT_NF4 or E4B_QUANT_FP4)."""
+    dt, E, N, K = _quantize_args(W, packed, absmax)
+    _check(load_library().e4b_quantize_stack(W.data_ptr(), dt, E, N, K, blocksize, int(quant_type),
+                                             packed.data_ptr(), absmax.data_ptr(), _stream(stream)),
+           "e4b_quantize_stack")
 
 
 def e4b_moe_route_permute_workspace_size(M: int, E: int, k: int) -> int:
@@ -226,11 +261,8 @@ def e4b_grouped_nf4_gemm_workspace_size(total_rows: int, N: int, K: int, r: int 
     return int(load_library().e4b_grouped_nf4_gemm_workspace_size(total_rows, N, K, r))
 
 
-def e4b_grouped_nf4_gemm(A: torch.Tensor, row_index: Optional[torch.Tensor], expert_offsets: torch.Tensor,
-                         total_rows: int, packed: torch.Tensor, absmax: torch.Tensor, N: int, K: int,
-                         out: torch.Tensor, epi: int = E4B_EPI_NONE, lora_A: Optional[torch.Tensor] = None,
-                         lora_B: Optional[torch.Tensor] = None, lora_scale: float = 0.0,
-                         workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+def _gemm(fn: str, quant_type: Optional[int], A, row_index, expert_offsets, total_rows, packed, absmax, N, K,
+          out, epi, lora_A, lora_B, lora_scale, workspace, stream) -> None:
     if A.dim() != 2 or A.dtype != torch.bfloat16 or not A.is_cuda or A.stride(1) != 1:
         raise ValueError("A must be a 2-D bf16 CUDA tensor with unit column stride")
     _dev(expert_offsets, "expert_offsets", torch.int32)
@@ -252,22 +284,38 @@ def e4b_grouped_nf4_gemm(A: torch.Tensor, row_index: Optional[torch.Tensor], exp
     if out.numel() < total_rows * ncols:
         raise ValueError("out too small")
     ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(load_library().e4b_grouped_nf4_gemm(
+    q = [] if quant_type is None else [int(quant_type)]
+    _check(getattr(load_library(), fn)(
         A.data_ptr(), A.shape[0], A.stride(0), _ptr(row_index), expert_offsets.data_ptr(), E, total_rows,
-        packed.data_ptr(), absmax.data_ptr(), N, K, _ptr(lora_A), _ptr(lora_B), r, float(lora_scale), epi,
-        out.data_ptr(), od, _ptr(workspace), ws, _stream(stream)), "e4b_grouped_nf4_gemm")
+        packed.data_ptr(), absmax.data_ptr(), *q, N, K, _ptr(lora_A), _ptr(lora_B), r, float(lora_scale), epi,
+        out.data_ptr(), od, _ptr(workspace), ws, _stream(stream)), fn)
+
+
+def e4b_grouped_nf4_gemm(A: torch.Tensor, row_index: Optional[torch.Tensor], expert_offsets: torch.Tensor,
+                         total_rows: int, packed: torch.Tensor, absmax: torch.Tensor, N: int, K: int,
+                         out: torch.Tensor, epi: int = E4B_EPI_NONE, lora_A: Optional[torch.Tensor] = None,
+                         lora_B: Optional[torch.Tensor] = None, lora_scale: float = 0.0,
+                         workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    _gemm("e4b_grouped_nf4_gemm", None, A, row_index, expert_offsets, total_rows, packed, absmax, N, K, out, epi,
+          lora_A, lora_B, lora_scale, workspace, stream)
+
+
+def e4b_grouped_4bit_gemm(A: torch.Tensor, row_index: Optional[torch.Tensor], expert_offsets: torch.Tensor,
+                          total_rows: int, packed: torch.Tensor, absmax: torch.Tensor, N: int, K: int,
+                          out: torch.Tensor, quant_type: int = E4B_QUANT_NF4, epi: int = E4B_EPI_NONE,
+                          lora_A: Optional[torch.Tensor] = None, lora_B: Optional[torch.Tensor] = None,
+                          lora_scale: float = 0.0, workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """e4b_grouped_nf4_gemm on a stack of either 4-bit storage (quant_type)."""
+    _gemm("e4b_grouped_4bit_gemm", quant_type, A, row_index, expert_offsets, total_rows, packed, absmax, N, K, out,
+          epi, lora_A, lora_B, lora_scale, workspace, stream)
 
 
 def e4b_grouped_nf4_gemm_dgrad_workspace_size(total_rows: int, N: int, K: int, r: int = 0) -> int:
     return int(load_library().e4b_grouped_nf4_gemm_dgrad_workspace_size(total_rows, N, K, r))
 
 
-def e4b_grouped_nf4_gemm_dgrad(dY: torch.Tensor, row_index: Optional[torch.Tensor], expert_offsets: torch.Tensor,
-                               total_rows: int, packed: torch.Tensor, absmax: torch.Tensor, N: int, K: int,
-                               out: torch.Tensor, lora_A: Optional[torch.Tensor] = None,
-                               lora_B: Optional[torch.Tensor] = None, lora_scale: float = 0.0,
-                               workspace: Optional[torch.Tensor] = None, stream=None) -> None:
-    """out[p] = dY[row_index[p]] . W_e (+ lora_scale * (dY . lora_B[e]) . lora_A[e]), [total_rows, K]."""
+def _dgrad(fn: str, quant_type: Optional[int], dY, row_index, expert_offsets, total_rows, packed, absmax, N, K,
+           out, lora_A, lora_B, lora_scale, workspace, stream) -> None:
     if dY.dim() != 2 or dY.dtype != torch.bfloat16 or not dY.is_cuda or dY.stride(1) != 1:
         raise ValueError("dY must be a 2-D bf16 CUDA tensor with unit column stride")
     _dev(expert_offsets, "expert_offsets", torch.int32)
@@ -288,10 +336,32 @@ def e4b_grouped_nf4_gemm_dgrad(dY: torch.Tensor, row_index: Optional[torch.Tenso
     if out.numel() < total_rows * K:
         raise ValueError("out too small")
     ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(load_library().e4b_grouped_nf4_gemm_dgrad(
+    q = [] if quant_type is None else [int(quant_type)]
+    _check(getattr(load_library(), fn)(
         dY.data_ptr(), dY.shape[0], dY.stride(0), _ptr(row_index), expert_offsets.data_ptr(), E, total_rows,
-        packed.data_ptr(), absmax.data_ptr(), N, K, _ptr(lora_A), _ptr(lora_B), r, float(lora_scale),
-        out.data_ptr(), od, _ptr(workspace), ws, _stream(stream)), "e4b_grouped_nf4_gemm_dgrad")
+        packed.data_ptr(), absmax.data_ptr(), *q, N, K, _ptr(lora_A), _ptr(lora_B), r, float(lora_scale),
+        out.data_ptr(), od, _ptr(workspace), ws, _stream(stream)), fn)
+
+
+def e4b_grouped_nf4_gemm_dgrad(dY: torch.Tensor, row_index: Optional[torch.Tensor], expert_offsets: torch.Tensor,
+                               total_rows: int, packed: torch.Tensor, absmax: torch.Tensor, N: int, K: int,
+                               out: torch.Tensor, lora_A: Optional[torch.Tensor] = None,
+                               lora_B: Optional[torch.Tensor] = None, lora_scale: float = 0.0,
+                               workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """out[p] = dY[row_index[p]] . W_e (+ lora_scale * (dY . lora_B[e]) . lora_A[e]), [total_rows, K]."""
+    _dgrad("e4b_grouped_nf4_gemm_dgrad", None, dY, row_index, expert_offsets, total_rows, packed, absmax, N, K, out,
+           lora_A, lora_B, lora_scale, workspace, stream)
+
+
+def e4b_grouped_4bit_gemm_dgrad(dY: torch.Tensor, row_index: Optional[torch.Tensor], expert_offsets: torch.Tensor,
+                                total_rows: int, packed: torch.Tensor, absmax: torch.Tensor, N: int, K: int,
+                                out: torch.Tensor, quant_type: int = E4B_QUANT_NF4,
+                                lora_A: Optional[torch.Tensor] = None, lora_B: Optional[torch.Tensor] = None,
+                                lora_scale: float = 0.0, workspace: Optional[torch.Tensor] = None,
+                                stream=None) -> None:
+    """e4b_grouped_nf4_gemm_dgrad on a stack of either 4-bit storage (quant_type)."""
+    _dgrad("e4b_grouped_4bit_gemm_dgrad", quant_type, dY, row_index, expert_offsets, total_rows, packed, absmax, N,
+           K, out, lora_A, lora_B, lora_scale, workspace, stream)
 
 
 def e4b_grouped_lora_grads_workspace_size(total_rows: int, r: int) -> int:
@@ -324,11 +394,42 @@ def e4b_grouped_lora_grads(x: torch.Tensor, row_index: Optional[torch.Tensor], e
         dA.data_ptr(), dB.data_ptr(), _ptr(workspace), ws, _stream(stream)), "e4b_grouped_lora_grads")
 
 
+def e4b_grouped_mxfp4_gemm_workspace_size(total_rows: int, N: int, K: int) -> int:
+    return int(load_library().e4b_grouped_mxfp4_gemm_workspace_size(total_rows, N, K))
+
+
+def e4b_grouped_mxfp4_gemm(A: torch.Tensor, row_index: Optional[torch.Tensor], expert_offsets: torch.Tensor,
+                           total_rows: int, blocks: torch.Tensor, scales: torch.Tensor, N: int, K: int,
+                           out: torch.Tensor, epi: int = E4B_EPI_NONE, workspace: Optional[torch.Tensor] = None,
+                           stream=None) -> None:
+    """y[p] = A[row_index[p]] . W_e^T with W_e given as MXFP4 code bytes and e8m0 scales."""
+    if A.dim() != 2 or A.dtype != torch.bfloat16 or not A.is_cuda or A.stride(1) != 1:
+        raise ValueError("A must be a 2-D bf16 CUDA tensor with unit column stride")
+    _dev(expert_offsets, "expert_offsets", torch.int32)
+    _dev(blocks, "blocks", torch.uint8)
+    _dev(scales, "scales", torch.uint8)
+    _dev(out, "out")
+    if row_index is not None:
+        _dev(row_index, "row_index", torch.int32)
+    E = expert_offsets.numel() - 1
+    od = {torch.float32: E4B_F32, torch.bfloat16: E4B_BF16}.get(out.dtype)
+    if od is None:
+        raise ValueError("out must be float32 or bfloat16")
+    ncols = N // 2 if epi == E4B_EPI_SWIGLU else N
+    if out.numel() < total_rows * ncols:
+        raise ValueError("out too small")
+    ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load_library().e4b_grouped_mxfp4_gemm(
+        A.data_ptr(), A.shape[0], A.stride(0), _ptr(row_index), expert_offsets.data_ptr(), E, total_rows,
+        blocks.data_ptr(), scales.data_ptr(), N, K, epi, out.data_ptr(), od, _ptr(workspace), ws, _stream(stream)),
+        "e4b_grouped_mxfp4_gemm")
+
+
 class ExpertStack:
     """Device tensors of one MoE layer's packed stacks (and optional adapter)."""
 
     def __init__(self, gu_packed, gu_absmax, dn_packed, dn_absmax, E, H, I,
-                 lora_A=None, lora_B=None, lora_alpha=0.0):
+                 lora_A=None, lora_B=None, lora_alpha=0.0, quant_type=E4B_QUANT_NF4):
         for t, n, d in ((gu_packed, "gu_packed", torch.uint8), (gu_absmax, "gu_absmax", torch.float32),
                         (dn_packed, "dn_packed", torch.uint8), (dn_absmax, "dn_absmax", torch.float32)):
             _dev(t, n, d)
@@ -345,8 +446,10 @@ class ExpertStack:
                 raise ValueError("lora_A must be [E, r, H] and lora_B [E, 2I, r]")
         self.tensors = (gu_packed, gu_absmax, dn_packed, dn_absmax, lora_A, lora_B)
         self.E, self.H, self.I, self.r = E, H, I, r
+        self.quant_type = int(quant_type)
         self.c = ExpertStackC(gu_packed.data_ptr(), gu_absmax.data_ptr(), dn_packed.data_ptr(),
-                              dn_absmax.data_ptr(), _ptr(lora_A), _ptr(lora_B), r, float(lora_alpha), E, H, I)
+                              dn_absmax.data_ptr(), _ptr(lora_A), _ptr(lora_B), r, float(lora_alpha), E, H, I,
+                              self.quant_type)
 
 
 def e4b_moe_expert_forward_workspace_size(M: int, stack: ExpertStack, k: int) -> int:

@@ -48,7 +48,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.e4b_version() == 1
+    assert lib.e4b_version() == e4b.ABI_VERSION == 3
     assert lib.e4b_status_string(0) == b"E4B_OK"
     assert lib.e4b_status_string(3) == b"E4B_ERR_WORKSPACE"
 
@@ -248,3 +248,93 @@ def test_backward_host_side_checks(lib):
     status = lib.e4b_moe_expert_backward(vp, 64, vp, 2, 1, ctypes.byref(stl), vp, vp, vp, None, None, vp, 1 << 40,
                                          None)
     assert status == 1 and b"needs dA and dB" in lib.e4b_last_error()
+
+
+def test_mxfp4_host_side_rejections(lib):
+    p = ctypes.c_void_p(1 << 20)
+
+    def call(**kw):
+        a = dict(A=p, a_rows=4, lda=128, ridx=None, offs=p, E=2, rows=4, blocks=p, scales=p, N=128, K=128, epi=0,
+                 out=p, od=0, ws=p, wsb=1 << 30)
+        a.update(kw)
+        return lib.e4b_grouped_mxfp4_gemm(a["A"], a["a_rows"], a["lda"], a["ridx"], a["offs"], a["E"], a["rows"],
+                                          a["blocks"], a["scales"], a["N"], a["K"], a["epi"], a["out"], a["od"],
+                                          a["ws"], a["wsb"], None)
+    need = lib.e4b_grouped_mxfp4_gemm_workspace_size(4, 128, 128)
+    assert need == e4b.e4b_grouped_nf4_gemm_workspace_size(4, 128, 128, 0) >= 256 + 4 * 128 * 2
+    assert call(wsb=need - 1) == 3 and str(need).encode() in lib.e4b_last_error()
+    assert call(ws=ctypes.c_void_p((1 << 20) + 8), wsb=need) == 1 and b"16-byte aligned" in lib.e4b_last_error()
+    assert call(K=96) == 2 and b"K must be" in lib.e4b_last_error()
+    assert call(N=32) == 2 and b"N must be" in lib.e4b_last_error()
+    assert call(lda=100) == 1 and b"lda" in lib.e4b_last_error()
+    assert call(epi=7) == 1 and b"epilogue" in lib.e4b_last_error()
+    assert call(scales=None) == 1 and b"null" in lib.e4b_last_error()
+    assert call(blocks=ctypes.c_void_p((1 << 20) + 4)) == 1 and b"16-byte aligned" in lib.e4b_last_error()
+
+
+def test_storage_type_is_checked_on_the_host(lib):
+    """An e4b_quant_type other than NF4 and FP4 is an argument error from every
+    call that takes one, before any device work; FP4 itself passes the host
+    checks."""
+    p = ctypes.c_void_p(1 << 20)
+    assert lib.e4b_quantize_stack(p, 0, 1, 1, 64, 64, 2, p, p, None) == 1
+    assert b"quant_type" in lib.e4b_last_error()
+    assert lib.e4b_quantize_stack(p, 0, 1, 1, 64, 64, e4b.E4B_QUANT_FP4, p, p, None) != 1
+    assert b"quant_type" not in lib.e4b_last_error()
+    rows, N, K = 64, 128, 128
+    need = e4b.e4b_grouped_nf4_gemm_workspace_size(rows, N, K, 0)
+    st = lib.e4b_grouped_4bit_gemm(p, rows, K, None, p, 2, rows, p, p, 5, N, K, None, None, 0, 0.0, 0, p, 0, p, need,
+                                   None)
+    assert st == 1 and b"quant_type" in lib.e4b_last_error()
+    st = lib.e4b_grouped_4bit_gemm_dgrad(p, rows, N, None, p, 2, rows, p, p, -1, N, K, None, None, 0, 0.0, p, 0, p,
+                                         1 << 30, None)
+    assert st == 1 and b"quant_type" in lib.e4b_last_error()
+    stk = e4b.ExpertStackC(1 << 20, 1 << 20, 1 << 20, 1 << 20, None, None, 0, 0.0, 8, 256, 128, 3)
+    st = lib.e4b_moe_expert_forward(p, 4, p, 2, 1, ctypes.byref(stk), p, p, 1 << 30, None)
+    assert st == 1 and b"quant_type" in lib.e4b_last_error()
+    st = lib.e4b_moe_expert_forward_decode_noalloc(p, 4, p, 2, 1, ctypes.byref(stk), p, None)
+    assert st == 1 and b"quant_type" in lib.e4b_last_error()
+
+
+def test_expert_stack_layout_matches_the_header():
+    """ctypes mirror of e4b_expert_stack: the storage type follows I."""
+    names = [f[0] for f in e4b.ExpertStackC._fields_]
+    assert names[-4:] == ["E", "H", "I", "quant_type"]
+    assert e4b.ExpertStackC.quant_type.offset == e4b.ExpertStackC.I.offset + 8
+    hdr = open(os.path.join(os.path.dirname(__file__), "..", "include", "e4b.h")).read()
+    body = hdr[hdr.index("typedef struct {\n  const uint8_t* gu_packed"):hdr.index("} e4b_expert_stack;")]
+    assert body.index("int64_t E, H, I;") < body.index("int32_t quant_type;")
+
+
+def test_zero_row_gemm_needs_no_workspace(lib):
+    """With no routed rows nothing launches or waits: the size query is 0 and a
+    NULL workspace passes the host checks (on a host without a GPU the call then
+    stops at the device check, not at the workspace)."""
+    p = ctypes.c_void_p(1 << 20)
+    assert e4b.e4b_grouped_nf4_gemm_workspace_size(0, 128, 128, 8) == 0
+    assert e4b.e4b_grouped_nf4_gemm_workspace_size(1, 128, 128, 0) >= 256 + 128 * 2
+    st = lib.e4b_grouped_nf4_gemm(p, 1, 128, None, p, 2, 0, p, p, 128, 128, None, None, 0, 0.0, 0, p, 0, None, 0,
+                                  None)
+    assert st != 3 and b"workspace" not in lib.e4b_last_error()
+
+
+def test_zero_row_dgrad_needs_no_workspace(lib):
+    p = ctypes.c_void_p(1 << 20)
+    assert e4b.e4b_grouped_nf4_gemm_dgrad_workspace_size(0, 128, 128, 8) == 0
+    st = lib.e4b_grouped_nf4_gemm_dgrad(p, 1, 128, None, p, 2, 0, p, p, 128, 128, None, None, 0, 0.0, p, 0, None, 0,
+                                        None)
+    assert st != 3 and b"workspace" not in lib.e4b_last_error()
+
+
+def test_zero_row_mxfp4_gemm_needs_no_workspace(lib):
+    p = ctypes.c_void_p(1 << 20)
+    assert lib.e4b_grouped_mxfp4_gemm_workspace_size(0, 128, 128) == 0
+    st = lib.e4b_grouped_mxfp4_gemm(p, 1, 128, None, p, 2, 0, p, p, 128, 128, 0, p, 0, None, 0, None)
+    assert st != 3 and b"workspace" not in lib.e4b_last_error()
+
+
+def test_graft_entry_build_checks_the_abi_version():
+    """build() compiles (or reuses) the library, loads it and checks its ABI
+    version against the binding's."""
+    import __graft_entry__ as ge
+    ge.build()

@@ -1,4 +1,5 @@
-"""CPU models of the index maps of the GPU kernels (regression pins).
+"""CPU models of the index maps of the GPU kernels (regression pins; the decode
+kernels' models are in test_model_decode_ring.py).
 
 Each model restates, in numpy and exact arithmetic, how a kernel's threads
 place data -- which packed bytes a thread decodes, where it stores them, which
@@ -312,3 +313,205 @@ def test_tensor_core_decoders_fill_the_swizzled_k_major_tile(halves, tpr):
         for k in range(64):
             addr = half * 128 * 64 + (ri >> 3) * 512 + (ri & 7) * 64 + (((k // 8) ^ (ri & 7)) << 3) + (k % 8)
             assert tile[addr] == W[r, k]
+
+
+def _byte_perm(x: int, y: int, s: int) -> int:
+    """PTX prmt (default mode): result byte i = byte (selector nibble i & 7) of
+    the 8-byte value y:x, or that byte's sign replicated when the nibble's bit 3 is set."""
+    src = (x & 0xFFFFFFFF) | ((y & 0xFFFFFFFF) << 32)
+    out = 0
+    for i in range(4):
+        n = (s >> (4 * i)) & 0xF
+        b = (src >> (8 * (n & 7))) & 0xFF
+        if n & 8:
+            b = 0xFF if b & 0x80 else 0x00
+        out |= b << (8 * i)
+    return out
+
+
+@pytest.mark.parametrize("table", ["nf4", "fp4", "mxfp4"])
+def test_tensor_core_byte_permute_decoder_is_a_table_lookup(table):
+    """csrc/gemm_tc.cu decode4 for every 16-bit input: the codebook's bf16
+    patterns split into low and high bytes (four entries per word), two
+    permutes look up entries 0-7 and 8-15 by the nibbles' low three bits, a
+    third keeps the half each nibble's top bit names, two more interleave the
+    bytes -> (element 2i, 2i+1) and (2i+2, 2i+3), the high nibble of a byte
+    being the lower-index element.  Checked against direct lookup for the NF4
+    and the FP4 (e2m1 / 6, with -0 at code 8) tables, and for MXFP4 codes (the
+    e2m1 values, element 2i in the LOW nibble: the other final selectors)."""
+    from oracle import fp4, mxfp4
+    from quantized_moe_expert_nf4_b200 import workloads
+    if table == "nf4":
+        cb32 = nf4.NF4_CODEBOOK
+    elif table == "fp4":
+        cb32 = fp4.codebook_f64().astype(np.float32)
+    else:
+        cb32 = mxfp4.e2m1_table().astype(np.float32)
+    sel0, sel1 = (0x5140, 0x7362) if table == "mxfp4" else (0x4051, 0x6273)
+    bits = [int(b) for b in workloads.to_bf16_bits(np.asarray(cb32, np.float32))]
+    lo = [0, 0, 0, 0]
+    hi = [0, 0, 0, 0]
+    for j, b in enumerate(bits):
+        lo[j >> 2] |= (b & 0xFF) << (8 * (j & 3))
+        hi[j >> 2] |= (b >> 8) << (8 * (j & 3))
+    for g in range(1 << 16):
+        s = g & 0x7777
+        pick = ((g >> 1) & 0x4444) | 0x3210
+        L = _byte_perm(_byte_perm(lo[0], lo[1], s), _byte_perm(lo[2], lo[3], s), pick)
+        Hh = _byte_perm(_byte_perm(hi[0], hi[1], s), _byte_perm(hi[2], hi[3], s), pick)
+        w0 = _byte_perm(L, Hh, sel0)
+        w1 = _byte_perm(L, Hh, sel1)
+        n = [g & 15, (g >> 4) & 15, (g >> 8) & 15, (g >> 12) & 15]
+        if table == "mxfp4":   # byte = (element 2i+1 << 4) | element 2i
+            assert w0 == bits[n[0]] | (bits[n[1]] << 16), hex(g)
+            assert w1 == bits[n[2]] | (bits[n[3]] << 16), hex(g)
+        else:                  # byte = (element 2i << 4) | element 2i+1
+            assert w0 == bits[n[1]] | (bits[n[0]] << 16), hex(g)
+            assert w1 == bits[n[3]] | (bits[n[2]] << 16), hex(g)
+
+
+@pytest.mark.parametrize("tpr", [2, 4])
+def test_tensor_core_mxfp4_decoders_take_their_scale_block(tpr):
+    """csrc/gemm_tc.cu MXFP4 decoders: thread part kq of a 64-k block (64 / tpr
+    k from 64 kq / tpr) multiplies by scale byte 2 kb + (2 kq) / tpr of its row,
+    the one e8m0 block of 32 that holds all of its k; with the e2m1 values and
+    2^(x - 127) this rebuilds the oracle's dequantised row."""
+    from oracle import mxfp4
+    rng = np.random.default_rng(21)
+    K = 320
+    row = rng.integers(0, 256, K // 2, dtype=np.uint8)
+    sc = rng.integers(120, 135, K // 32, dtype=np.uint8)
+    want = mxfp4.dequantize_expert(row[None, :], sc[None, :], 1, K)[0]
+    got = np.full(K, np.nan)
+    e2m1 = mxfp4.e2m1_table()
+    for kb in range(K // 64):
+        for kq in range(tpr):
+            k0 = kb * 64 + kq * (64 // tpr)
+            x = int(sc[2 * kb + (2 * kq) // tpr])
+            assert all((k0 + j) // 32 == 2 * kb + (2 * kq) // tpr for j in range(64 // tpr))
+            for j in range(0, 64 // tpr, 2):
+                byte = int(row[(k0 + j) // 2])
+                got[k0 + j] = e2m1[byte & 15] * 2.0 ** (x - 127)
+                got[k0 + j + 1] = e2m1[byte >> 4] * 2.0 ** (x - 127)
+    assert np.array_equal(got, want)
+
+
+def _quant_cell_table(cb):
+    """csrc/quantize.cu quant_cell_table: levels = distinct codebook values
+    ascending (each with its lowest code), thresholds = smallest float above
+    each exact midpoint, and per cell c of [c/64 - 1, (c+1)/64 - 1] widened by
+    1e-5 the one threshold inside it (+inf if none) with the codes below and at
+    or above it."""
+    vals, codes = [], []
+    for c in range(16):
+        v = float(cb[c]) + 0.0
+        if v not in vals:
+            vals.append(v)
+            codes.append(c)
+    order = np.argsort(vals, kind="stable")
+    vals = [vals[i] for i in order]
+    codes = [codes[i] for i in order]
+    T = []
+    for lv in range(len(vals) - 1):
+        mid = (vals[lv] + vals[lv + 1]) / 2
+        f = np.float32(mid)
+        T.append(float(f if float(f) > mid else np.nextafter(f, np.float32(np.inf))))
+    cells = []
+    for c in range(128):
+        lo, hi = c / 64.0 - 1.0 - 1e-5, (c + 1) / 64.0 - 1.0 + 1e-5
+        base = sum(1 for t in T if t <= lo)
+        inside = [t for t in T if lo < t <= hi]
+        assert len(inside) <= 1, "two thresholds in one cell"
+        cells.append((inside[0] if inside else np.inf, codes[base], codes[min(base + 1, len(vals) - 1)]))
+    return cells
+
+
+def _kernel_codes(w, a, cells):
+    """csrc/quantize.cu code_of for every (w, a): s' = fl32(w * fl32(1/a)) for
+    absmax in [2^-125, 2^125], the cell of s', and the exact fl32(w / a) when
+    s' lies within 2^-22 of the cell's threshold (or the absmax is outside)."""
+    f32 = np.float32
+    t_tab = np.array([c[0] for c in cells], f32)
+    lo_tab = np.array([c[1] for c in cells])
+    hi_tab = np.array([c[2] for c in cells])
+    with np.errstate(all="ignore"):
+        fast = (a >= f32(2.0 ** -125)) & (a <= f32(2.0 ** 125))
+        exact = (w / a).astype(f32)
+        s = np.where(fast, (w * (f32(1) / a).astype(f32)).astype(f32), exact)
+        c = np.clip(np.floor((s + f32(1)).astype(f32) * f32(64)).astype(np.int64), 0, 127)
+        t = t_tab[c]
+        near = fast & ~(np.abs((s - t).astype(f32)) > f32(2.0 ** -22))
+        s = np.where(near, exact, s)
+    return np.where(s >= t, hi_tab[c], lo_tab[c]).astype(np.uint8), int(near.sum())
+
+
+@pytest.mark.parametrize("table", ["nf4", "fp4"])
+def test_quantiser_cell_lookup_and_reciprocal_path_match_the_oracle(table):
+    """The quantiser kernel's decision -- one cell lookup, the weight scaled by
+    the block's reciprocal unless it lands within 2^-22 of the cell's threshold
+    -- equals the oracle's code of fl32(w / a), on random weights, on every
+    decision point times random absmax (and 3 floats either side), and on
+    |w| = a, zeros and subnormal absmax."""
+    from oracle import fp4
+    mod = nf4 if table == "nf4" else fp4
+    cells = _quant_cell_table(mod.codebook_f64())
+    rng = np.random.default_rng(11)
+    f32 = np.float32
+    n = 200_000
+    fallbacks = 0
+    for kind in range(3):
+        a = (rng.uniform(1, 2, n) * 2.0 ** rng.integers(-40, 40, n)).astype(f32)
+        if kind == 0:
+            w = (rng.uniform(-1, 1, n) * a).astype(f32)
+        elif kind == 1:
+            w = (rng.choice(mod.midpoints(), n) * a.astype(np.float64)).astype(f32)
+            k = rng.integers(-3, 4, n)
+            for step in range(3):
+                w = np.where(k > step, np.nextafter(w, f32(np.inf)), w)
+                w = np.where(k < -step, np.nextafter(w, f32(-np.inf)), w)
+        else:
+            tiny = (rng.uniform(1, 2, n) * 2.0 ** rng.integers(-149, -120, n)).astype(f32)
+            a = np.where(rng.random(n) < 0.2, tiny, a).astype(f32)
+            a = np.where(a == 0, f32(1e-45), a).astype(f32)
+            r = rng.random(n)
+            w = np.where(r < 0.25, a, np.where(r < 0.5, -a, (rng.uniform(-1, 1, n) * a).astype(f32))).astype(f32)
+            w = np.where(rng.random(n) < 0.05, f32(0), w).astype(f32)
+        got, nf = _kernel_codes(w, a, cells)
+        fallbacks += nf
+        with np.errstate(all="ignore"):
+            want = mod.code_of_scaled((w / a).astype(f32))
+        assert np.array_equal(got, want), kind
+    assert fallbacks > 0   # the exact path was exercised
+
+
+def test_tensor_memory_decoders_fill_the_a_operand_the_mma_reads():
+    """csrc/gemm_tc.cu TMEM-operand tile: decoder warp w (lane quadrant w % 4,
+    part c = (w - 4) / 4: half c / 2, 32-k part c % 2) takes weight row
+    32 (w % 4) + lane of its half, decodes its 32 k (4 words, decode4 on each
+    half-word: v[i] = elements 2i, 2i+1) and stores v[0..15] as 16 consecutive
+    32-bit columns of its TMEM lane from column A + half*32 + part*16.  The MMA
+    of k-step kk of half h reads columns A + h*32 + kk*8 .. +7 of lanes 0..127,
+    two bf16 per column, the lower k in the low half: that must be the half's
+    rows and k [16 kk, 16 kk + 16) of the 64-k block."""
+    packed, absmax, W = _layer_rows(9, 256, 64)
+    tmem = {}
+    for w in range(4, 20):
+        qd, c = w & 3, (w - 4) >> 2
+        half, part = c >> 1, c & 1
+        for lane in range(32):
+            ri = qd * 32 + lane
+            r = half * 128 + ri
+            src = packed[r, part * 16: part * 16 + 16]          # 16 bytes = this thread's 32 k
+            vals = []
+            for byte in src:
+                vals += [v * absmax[r, 0] for v in _pair(byte)]   # elements in k order
+            v = [(vals[2 * i], vals[2 * i + 1]) for i in range(16)]
+            for i in range(16):
+                key = (ri, half * 32 + part * 16 + i)
+                assert key not in tmem, "column written twice"
+                tmem[key] = v[i]                                  # (low half, high half)
+    for h in range(2):
+        for kk in range(4):
+            for lane in range(128):
+                row = [x for col in range(8) for x in tmem[(lane, h * 32 + kk * 8 + col)]]
+                assert row == list(W[h * 128 + lane, kk * 16: kk * 16 + 16]), (h, kk, lane)
