@@ -116,8 +116,11 @@ __host__ __device__ inline uint32_t gu_stage_bytes(int H) { return 8 * copy_stri
 __host__ __device__ inline uint32_t dn_block_bytes(int I) { return 4 * copy_stride(I) + 4 * am_stride(I / 64); }
 
 // Bytes of h staged in shared memory for phase 2 (all of it when it fits the
-// budget, else 0: the fragments then come from L2 into registers).
-constexpr uint32_t kHStageMax = 32 * 1024;
+// budget, else 0: the fragments then come from L2 into registers).  The
+// staging area is the part of phase 1's reduction buffer that phase 2's
+// reduction (one float4 per lane of 16 warps, 8 KB) leaves free.
+constexpr uint32_t kRedDnBytes = kMath * 32 * 16;
+constexpr uint32_t kHStageMax = kRedBytes - kRedDnBytes;
 __host__ __device__ inline uint32_t h_stage_bytes(int M, int k, int I) {
   const uint32_t b = static_cast<uint32_t>(M * k) * static_cast<uint32_t>(I) * 2;
   return b <= kHStageMax ? b : 0;
@@ -147,8 +150,7 @@ __host__ __device__ inline Smem make_smem(int M, int k, int E, int r, int I, int
   o = al(o + S * kMaxM * 4, 16);
   L.xa = o;
   if (r > 0) o = al(o + S * r * 4, 16);
-  L.hs = o;
-  o = al(o + h_stage_bytes(M, k, I), 128);
+  L.hs = L.red + kRedDnBytes;
   L.bars = o;
   o = al(o + (2 * stages + 1) * 8, 16);
   L.ring = al(o, 128);
@@ -241,6 +243,28 @@ __device__ __forceinline__ void block_mma(const unsigned char* __restrict__ lut,
     const uint32_t wa = (j < 2) ? w0.x : w0.y, wb = (j < 2) ? w1.x : w1.y;
     const int b = 2 * (j & 1);
     mma_16816(d, pair(wa, b), pair(wb, b), pair(wa, b + 1), pair(wb, b + 1), xw[2 * j], xw[2 * j + 1]);
+  }
+}
+
+// Two independent blocks (a and b) at once, their MMAs interleaved: each
+// MMA of a chain waits for the previous one of the same chain, so two chains
+// keep the tensor pipe busy where one would leave it idle.
+__device__ __forceinline__ void block_mma2(const unsigned char* __restrict__ lut, uint32_t lane4, uint2 w0a,
+                                           uint2 w1a, const uint32_t* xa, uint2 w0b, uint2 w1b, const uint32_t* xb,
+                                           float da[4], float db[4]) {
+  auto pair = [&](uint32_t word, int byte) {
+    const uint32_t sh = byte == 0 ? (word << 7) : (word >> (8 * byte - 7));
+    return *reinterpret_cast<const uint32_t*>(lut + ((sh & 0x7f80u) | lane4));
+  };
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int b = 2 * (j & 1);
+    const uint32_t wa0 = (j < 2) ? w0a.x : w0a.y, wa1 = (j < 2) ? w1a.x : w1a.y;
+    const uint32_t wb0 = (j < 2) ? w0b.x : w0b.y, wb1 = (j < 2) ? w1b.x : w1b.y;
+    const uint32_t a0 = pair(wa0, b), a1 = pair(wa1, b), a2 = pair(wa0, b + 1), a3 = pair(wa1, b + 1);
+    const uint32_t b0 = pair(wb0, b), b1 = pair(wb1, b), b2 = pair(wb0, b + 1), b3 = pair(wb1, b + 1);
+    mma_16816(da, a0, a1, a2, a3, xa[2 * j], xa[2 * j + 1]);
+    mma_16816(db, b0, b1, b2, b3, xb[2 * j], xb[2 * j + 1]);
   }
 }
 
@@ -484,19 +508,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
         for (int hh = 0; hh < 2; ++hh) {
           const int kb = 2 * (wi + kGW * q) + hh;
           if (kb < KB) {
+            uint2 w0[2], w1[2];
+            float a0[2], a1[2];
 #pragma unroll
             for (int T = 0; T < 2; ++T) {
               const int r = 2 * T + (g >> 2), cg = g & 3;
               const uint32_t off = r * (H / 2) + kb * 32 + 8 * t;
-              const uint2 w0 = lds64(st + cg * cs_gu + off);
-              const uint2 w1 = lds64(st + (4 + cg) * cs_gu + off);
-              const float a0 = am[cg * as_gu + r * KB + kb], a1 = am[(4 + cg) * as_gu + r * KB + kb];
-              float d[4] = {0.f, 0.f, 0.f, 0.f};
-              block_mma(lut_b, lane4, w0, w1, xr[q][hh], d);
-              c[T][0] = fmaf(a0, d[0], c[T][0]);
-              c[T][1] = fmaf(a0, d[1], c[T][1]);
-              c[T][2] = fmaf(a1, d[2], c[T][2]);
-              c[T][3] = fmaf(a1, d[3], c[T][3]);
+              w0[T] = lds64(st + cg * cs_gu + off);
+              w1[T] = lds64(st + (4 + cg) * cs_gu + off);
+              a0[T] = am[cg * as_gu + r * KB + kb];
+              a1[T] = am[(4 + cg) * as_gu + r * KB + kb];
+            }
+            float d[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            block_mma2(lut_b, lane4, w0[0], w1[0], xr[q][hh], w0[1], w1[1], xr[q][hh], d[0], d[1]);
+#pragma unroll
+            for (int T = 0; T < 2; ++T) {
+              c[T][0] = fmaf(a0[T], d[T][0], c[T][0]);
+              c[T][1] = fmaf(a0[T], d[T][1], c[T][1]);
+              c[T][2] = fmaf(a1[T], d[T][2], c[T][2]);
+              c[T][3] = fmaf(a1[T], d[T][3], c[T][3]);
             }
           }
         }
@@ -641,42 +671,62 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
       ring_wait(&full[s], (j / RS) & 1, &abort_s, p.err, kErrWaitFull);
       const unsigned char* st = ring + static_cast<uint32_t>(s) * slot;
       const int ch = jd % nch, u0 = ch * DPE, np = min(DPE, nU - u0) * KBI;
-#pragma unroll
-      for (int q = 0; q < PPW; ++q) {
+      // The warp's pairs two at a time (independent MMA chains interleaved).
+      auto pair_in = [&](int q, uint2& w0, uint2& w1, float& s0, float& s1, float& s2, float& s3) {
         const int pi = warp + kMath * q;
-        if (pi < np) {
-          const int ei = pi / KBI, kb = pi % KBI, u = u0 + ei;
-          // MMA row g = block row 4 (g % 4) + g / 4, row g + 8 = that + 2.
-          const unsigned char* base = st + ei * exp_dn;
-          const float* am = reinterpret_cast<const float*>(base + am_dn);
-          const int cg = g & 3, r = g >> 2;
-          const uint32_t off = cg * cs_dn + r * (I / 2) + kb * 32 + 8 * t;
-          const uint2 w0 = lds64(base + off);
-          const uint2 w1 = lds64(base + off + I);  // two rows further
-          const float a0 = am[cg * as_dn + r * KBI + kb], a1 = am[cg * as_dn + (r + 2) * KBI + kb];
-          float d[4] = {0.f, 0.f, 0.f, 0.f};
-          block_mma(lut_b, lane4, w0, w1, reinterpret_cast<const uint32_t*>(hb[q]), d);
-          const int s0 = (2 * t < p.M) ? slotmap[u * kMaxM + 2 * t] : -1;
-          const int s1 = (2 * t + 1 < p.M) ? slotmap[u * kMaxM + 2 * t + 1] : -1;
-          const float wc0 = s0 >= 0 ? w_s[s0] : 0.f, wc1 = s1 >= 0 ? w_s[s1] : 0.f;
-          acc[0] = fmaf(a0 * wc0, d[0], acc[0]);
-          acc[1] = fmaf(a0 * wc1, d[1], acc[1]);
-          acc[2] = fmaf(a1 * wc0, d[2], acc[2]);
-          acc[3] = fmaf(a1 * wc1, d[3], acc[3]);
+        const int ei = pi / KBI, kb = pi % KBI, u = u0 + ei;
+        // MMA row g = block row 4 (g % 4) + g / 4, row g + 8 = that + 2.
+        const unsigned char* base = st + ei * exp_dn;
+        const float* am = reinterpret_cast<const float*>(base + am_dn);
+        const int cg = g & 3, r = g >> 2;
+        const uint32_t off = cg * cs_dn + r * (I / 2) + kb * 32 + 8 * t;
+        w0 = lds64(base + off);
+        w1 = lds64(base + off + I);  // two rows further
+        const float a0 = am[cg * as_dn + r * KBI + kb], a1 = am[cg * as_dn + (r + 2) * KBI + kb];
+        const int sl0 = (2 * t < p.M) ? slotmap[u * kMaxM + 2 * t] : -1;
+        const int sl1 = (2 * t + 1 < p.M) ? slotmap[u * kMaxM + 2 * t + 1] : -1;
+        const float wc0 = sl0 >= 0 ? w_s[sl0] : 0.f, wc1 = sl1 >= 0 ? w_s[sl1] : 0.f;
+        s0 = a0 * wc0;
+        s1 = a0 * wc1;
+        s2 = a1 * wc0;
+        s3 = a1 * wc1;
+      };
+#pragma unroll
+      for (int q = 0; q < PPW; q += 2) {
+        const bool va = warp + kMath * q < np, vb = q + 1 < PPW && warp + kMath * (q + 1) < np;
+        if (va && vb) {
+          uint2 w0a, w1a, w0b, w1b;
+          float sa[4], sb[4];
+          pair_in(q, w0a, w1a, sa[0], sa[1], sa[2], sa[3]);
+          pair_in(q + 1, w0b, w1b, sb[0], sb[1], sb[2], sb[3]);
+          float da[4] = {0.f, 0.f, 0.f, 0.f}, db[4] = {0.f, 0.f, 0.f, 0.f};
+          block_mma2(lut_b, lane4, w0a, w1a, reinterpret_cast<const uint32_t*>(hb[q]), w0b, w1b,
+                     reinterpret_cast<const uint32_t*>(hb[q + 1 < PPW ? q + 1 : q]), da, db);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[i] = fmaf(sb[i], db[i], fmaf(sa[i], da[i], acc[i]));
+        } else if (va) {
+          uint2 w0a, w1a;
+          float sa[4];
+          pair_in(q, w0a, w1a, sa[0], sa[1], sa[2], sa[3]);
+          float da[4] = {0.f, 0.f, 0.f, 0.f};
+          block_mma(lut_b, lane4, w0a, w1a, reinterpret_cast<const uint32_t*>(hb[q]), da);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[i] = fmaf(sa[i], da[i], acc[i]);
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
       if (ch == nch - 1) {
         // End of a row block: the 16 warps' sums in warp order -> out.
-        const int rbq = jd / nch, par = rbq & 1;
-        red[(par * kMath + warp) * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        const int rbq = jd / nch;
+        if (rbq > 0) named_bar(kBarMath, kMath * 32);  // the previous row block's sums are read
+        red[warp * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
         acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
         named_bar(kBarMath, kMath * 32);
         if (warp == rbq % kMath) {
           float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
           for (int w = 0; w < kMath; ++w) {
-            const float4 v = red[(par * kMath + w) * 32 + lane];
+            const float4 v = red[w * 32 + lane];
             sum.x += v.x;
             sum.y += v.y;
             sum.z += v.z;

@@ -123,8 +123,6 @@ def _plan(M, k, E, H, I, r):
         o = _al(o + n, 16)
     if r:
         o = _al(o + S * r * 4, 16)
-    hb = S * I * 2 if S * I * 2 <= 32 * 1024 else 0     # h staged in shared memory for phase 2
-    o = _al(o + hb, 128)
     fixed = _al(o, 128) + 2 * 32 * 8
     stages = min((SMEM_LIMIT - fixed) // slot, 32) & ~1
     ring = _al(_al(o + (2 * stages + 1) * 8, 16), 128)
