@@ -184,6 +184,24 @@ __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, u
                : "memory");
 }
 
+// L2 policy for data read exactly once per call (the packed weights): evict it
+// first, so the stream does not push out what the kernel reads again (its h,
+// barrier slots, x, and its own instructions).
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+__device__ __forceinline__ void bulk_g2s_stream(void* smem_dst, const void* gmem_src, uint32_t bytes, uint64_t* bar,
+                                                uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
+}
+
 __device__ __forceinline__ uint2 lds64(const unsigned char* p) { return *reinterpret_cast<const uint2*>(p); }
 
 __device__ __forceinline__ void st_release_gpu(unsigned long long* p, unsigned long long v) {
@@ -329,14 +347,14 @@ __device__ void prologue(const FusedParams& p, uint32_t* lut, int* ids_s, float*
 // (packed copies at dst + c * copy_stride, absmax copies at am_dst + c * am_stride).
 __device__ __forceinline__ void copy_block_part(int lane_c, unsigned char* dst, unsigned char* am_dst,
                                                 uint64_t* full, const uint8_t* packed, const float* absmax, int K,
-                                                int64_t row0) {
+                                                int64_t row0, uint64_t pol) {
   const int KB = K / 64;
   const int c = lane_c & 3;
   const int64_t row = row0 + 4 * c;
   if (lane_c < 4)
-    bulk_g2s(dst + c * copy_stride(K), packed + row * (K / 2), static_cast<uint32_t>(2 * K), full);
+    bulk_g2s_stream(dst + c * copy_stride(K), packed + row * (K / 2), static_cast<uint32_t>(2 * K), full, pol);
   else
-    bulk_g2s(am_dst + c * am_stride(KB), absmax + row * KB, static_cast<uint32_t>(16 * KB), full);
+    bulk_g2s_stream(am_dst + c * am_stride(KB), absmax + row * KB, static_cast<uint32_t>(16 * KB), full, pol);
 }
 
 // ---------------------------------------------------------------------------
@@ -401,6 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
 
   if (warp == kProducer) {
     // ------------------------------------------------------------ producer
+    const uint64_t pol = l2_evict_first_policy();
     int issued = 0;
     for (int j = 0; j < T; ++j) {
       const int s = j % RS;
@@ -416,7 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
         if (lane < 16) {
           const int blk = lane >> 3;
           copy_block_part(lane & 7, st + blk * 4 * cs_gu, st + am_gu + blk * 16 * as_gu, &full[s], p.gu_packed,
-                          p.gu_absmax, H, grow + blk * I);
+                          p.gu_absmax, H, grow + blk * I, pol);
         }
       } else {
         // One block of 16 down rows per expert: lane 8 ei + c issues copy c of expert ei.
@@ -428,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
           const int ei = lane >> 3;
           const int64_t row0 = static_cast<int64_t>(touched[u0 + ei]) * H + rb * 16;
           copy_block_part(lane & 7, st + ei * exp_dn, st + ei * exp_dn + am_dn, &full[s], p.dn_packed, p.dn_absmax, I,
-                          row0);
+                          row0, pol);
         }
       }
       ++issued;
@@ -744,12 +763,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
       }
     };
     load_h(0, hA);
-    for (int jd = 0; jd < n_dn; jd += 2) {
+#pragma unroll 1
+    for (int jd = 0; jd < n_dn; ++jd) {
       load_h(jd + 1, hB);
       compute(jd, hA);
-      if (jd + 1 < n_dn) {
-        load_h(jd + 2, hA);
-        compute(jd + 1, hB);
+#pragma unroll
+      for (int q = 0; q < PPW; ++q) {
+        hA[q][0] = hB[q][0];
+        hA[q][1] = hB[q][1];
       }
     }
   }
