@@ -74,8 +74,7 @@ constexpr int kMaxGrid = 1024;          // barrier slots in the workspace
 constexpr int kMaxStages = 32;
 constexpr uint32_t kLutBytes = 256 * 32 * 4;
 constexpr uint32_t kRedBytes = kGroups * 2 * kGW * 2 * 32 * 16;  // phase 1: [group][parity][warp][tile][lane] float4
-constexpr int kBarGroup0 = 1;           // named barriers: 1, 2 (groups), 3 (all math warps)
-constexpr int kBarMath = 3;
+constexpr int kBarMath = 3;             // named barrier of the 16 math warps
 
 struct FusedParams {
   const uint16_t* x;
@@ -152,7 +151,7 @@ __host__ __device__ inline Smem make_smem(int M, int k, int E, int r, int I, int
   if (r > 0) o = al(o + S * r * 4, 16);
   L.hs = L.red + kRedDnBytes;
   L.bars = o;
-  o = al(o + (2 * stages + 1) * 8, 16);
+  o = al(o + (2 * stages + 1 + 2 * kGroups) * 8, 16);
   L.ring = al(o, 128);
   L.total = L.ring + static_cast<uint32_t>(stages) * slot;
   return L;
@@ -381,10 +380,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);  // stage landed
   uint64_t* empty = full + RS;                                   // stage consumed (16 arrivals)
   uint64_t* hbar = empty + RS;                                   // h staged for phase 2
+  uint64_t* rfree = hbar + 1;                                    // [group][parity] partials read by the finisher
   const uint32_t HSB = h_stage_bytes(p.M, p.k, I);
   unsigned char* ring = smem + L.ring;
   __shared__ int nU_s;
   __shared__ volatile int abort_s;
+  __shared__ int fin_cnt[kGroups][2];  // warps of a group that have deposited an item's partials
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
@@ -398,6 +399,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
       mbar_init(&empty[s], kMath);
     }
     mbar_init(hbar, 1);
+    for (int i = 0; i < 2 * kGroups; ++i) {
+      mbar_init(&rfree[i], 1);
+      fin_cnt[i >> 1][i & 1] = 0;
+    }
     fence_mbar_init();
   }
   prologue(p, lut, ids_s, w_s, uidx, touched, slotmap, &nU_s);
@@ -552,12 +557,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
       }
       __syncwarp();
       if (lane == 0) mbar_arrive_cnt(&empty[s], kMath / kGW);
-      const int par = (jj / kGroups) & 1;
+      // Deposit the partials; the last warp of the group to do so finishes
+      // the item while the others go on to their next one.  Items iq and
+      // iq + 2 of the group share a buffer: wait until the finisher of iq - 2
+      // has read it.
+      const int iq = jj / kGroups, par = iq & 1;
+      if (iq >= 2) ring_wait(&rfree[gi * 2 + par], ((iq >> 1) - 1) & 1, &abort_s, p.err, kErrWaitFull);
       float4* rp = red + (((gi * 2 + par) * kGW + wi) * 2) * 32 + lane;
       rp[0] = make_float4(c[0][0], c[0][1], c[0][2], c[0][3]);
       rp[32] = make_float4(c[1][0], c[1][1], c[1][2], c[1][3]);
-      named_bar(kBarGroup0 + gi, kGW * 32);
-      if (wi == (jj / kGroups) % kGW) {
+      __syncwarp();
+      int last = 0;
+      if (lane == 0) {
+        __threadfence_block();
+        last = atomicAdd(&fin_cnt[gi][par], 1) == kGW - 1;
+      }
+      if (__shfl_sync(0xffffffffu, last, 0)) {
+        __threadfence_block();  // the other warps' partials, deposited before their increments
         // This warp finishes the item: the group's partials in warp order,
         // then SwiGLU (+ LoRA delta) for the tokens routed to the expert.
         const int it = i0 + jj, u = it / ipe, rb = it % ipe;
@@ -595,6 +611,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
             }
             p.h[static_cast<int64_t>(sl) * I + col] = float_to_bf16_bits(silu_f32(gv) * uv);
           }
+        }
+        __syncwarp();
+        if (lane == 0) {
+          fin_cnt[gi][par] = 0;
+          mbar_arrive(&rfree[gi * 2 + par]);  // the buffer may take item iq + 2's partials
         }
       }
     }

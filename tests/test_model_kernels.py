@@ -125,7 +125,7 @@ def _plan(M, k, E, H, I, r):
         o = _al(o + S * r * 4, 16)
     fixed = _al(o, 128) + 2 * 32 * 8
     stages = min((SMEM_LIMIT - fixed) // slot, 32) & ~1
-    ring = _al(_al(o + (2 * stages + 1) * 8, 16), 128)
+    ring = _al(_al(o + (2 * stages + 1 + 4) * 8, 16), 128)
     return dict(spw=spw, ppw=ppw, dpe=dpe, slot=slot, stages=stages, ring=ring, total=ring + stages * slot)
 
 
