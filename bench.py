@@ -56,7 +56,11 @@ def workload(name):
     """(layer configuration name, M, storage name) of a bench workload."""
     w = WORKLOADS[name]
     return w[0], w[1], (w[2] if len(w) > 2 else "nf4")
+
+
 DEFAULT_WORKLOAD = "olmoe_m1"
+# Sweep rows that also carry the end-to-end measurement and a CPU-oracle sample.
+E2E_SWEEP = ("qwen3_m4096", "gptoss_m8192")
 # Every other workload of the table runs in the default sweep, so the JSON line
 # carries the prefill rows' (M >= 4096) tensor-core fractions and the gpt-oss
 # decode row beside the OLMoE ones.
@@ -159,6 +163,19 @@ def cpu_cores():
         return os.cpu_count() or 1
 
 
+def cpu_model():
+    """The host CPU's model name (first /proc/cpuinfo entry), or the platform string."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or platform.machine()
+
+
 class OracleSample:
     """A bounded sample of the workload, prepared for the float64 oracle.
 
@@ -243,8 +260,8 @@ def run_reference(args, cfg, M, rank, world):
         "config": {"workload": args.workload, "E": cfg.E, "H": cfg.H, "I": cfg.I, "k": cfg.k, "M": M,
                    "routing": cfg.routing, "weights": f"{smp.storage.upper()}/64 fp32 absmax",
                    "sample_tokens_per_step": smp.ntok},
-        "cpu_baseline": {"value": value, "unit": "routed_tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": smp.describe()},
+        "cpu_baseline": {"value": value, "unit": "routed_tokens/s", "cores": cores, "cpu": cpu_model(),
+                         "kind": "oracle", "sample": smp.describe()},
         "e2e": {"value": value, "unit": "routed_tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -512,7 +529,7 @@ def job_throughput(per_rank_units, steps, world, max_seconds):
     return world * per_rank_units * steps / max_seconds
 
 
-def measure(args, name, rank, world, dist, peaks, primary):
+def measure(args, name, rank, world, dist, peaks, primary, e2e_steps=None):
     import torch
 
     cfgname, M, storage = workload(name)
@@ -555,13 +572,14 @@ def measure(args, name, rank, world, dist, peaks, primary):
     }
     res["e2e"] = None
     res["e2e_graph"] = None
-    if primary and not args.no_e2e:
-        ev, h2d, d2h = b.e2e(min(args.steps, 2000))
+    if (primary or e2e_steps) and not args.no_e2e:
+        K = e2e_steps or min(args.steps, 2000)
+        ev, h2d, d2h = b.e2e(K)
         ev = reduce_over_ranks(ev, dist, dev, "min") * world
         res["e2e"] = {"value": ev, "unit": "routed_tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
         gerr = None
         try:
-            gv, h2d, d2h = b.e2e_graph(min(args.steps, 2000))
+            gv, h2d, d2h = b.e2e_graph(K)
         except Exception as exc:  # reported, the headline line still prints
             gv, gerr = 0.0, f"{type(exc).__name__}: {exc}"
         gv = reduce_over_ranks(gv, dist, dev, "min") * world   # every rank takes this collective
@@ -798,7 +816,8 @@ def main():
     if not args.no_sweep and args.workload == DEFAULT_WORKLOAD:
         for name in DEFAULT_SWEEP:
             try:
-                r = measure(args, name, rank, world, dist, peaks, primary=False)
+                r = measure(args, name, rank, world, dist, peaks, primary=False,
+                            e2e_steps=min(args.steps, 200) if name in E2E_SWEEP else None)
             except Exception as exc:  # a failing sweep row is reported, the headline line still prints
                 sweep.append({"workload": name, "error": f"{type(exc).__name__}: {exc}"})
                 torch.cuda.empty_cache()
@@ -811,6 +830,16 @@ def main():
                           "roofline_kernel": r["roofline"]["kernel"] if r["roofline"] else None,
                           "step_roofline_frac": r["step_roofline"]["frac"],
                           "clocks": r["clocks"]})
+            if name in E2E_SWEEP:
+                sweep[-1]["e2e"] = r["e2e"]
+                sweep[-1]["e2e_graph"] = r["e2e_graph"]
+                if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                    rc, rstorage = workloads.CONFIGS[workload(name)[0]], workload(name)[2]
+                    rate, desc, spent = oracle_rate(rc, workload(name)[1], budget_s=3.0, max_tokens=2,
+                                                    storage=rstorage)
+                    sweep[-1]["cpu_baseline"] = {"value": rate, "unit": "routed_tokens/s", "cores": cpu_cores(),
+                                                 "cpu": cpu_model(), "kind": "oracle", "sample": desc,
+                                                 "seconds": spent}
     quant = None
     bwd = None
     mx = None
@@ -833,8 +862,8 @@ def main():
         cb = None
         if world == 1 and not args.no_cpu_baseline:
             rate, desc, spent = oracle_rate(cfg, M, budget_s=12.0, max_tokens=8, storage=storage)
-            cb = {"value": rate, "unit": "routed_tokens/s", "cores": cpu_cores(), "kind": "oracle", "sample": desc,
-                  "seconds": spent}
+            cb = {"value": rate, "unit": "routed_tokens/s", "cores": cpu_cores(), "cpu": cpu_model(), "kind": "oracle",
+                  "sample": desc, "seconds": spent}
         line = {
             "metric": METRIC, "value": main_res["value"], "unit": "routed_tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": main_res["ms_per_step"],
