@@ -475,7 +475,11 @@ def replicas_for(cfg, M):
 # DRAM bytes (read + write) per launch from one ncu capture of the kernel as it
 # is now, keyed by (layer config, M, kernel); a kernel changed since its capture
 # has no entry.
-MEASURED_TRAFFIC = {}
+MEASURED_TRAFFIC = {
+    ("olmoe", 1, "decode.fused"): 28436480 + 2048,
+    ("olmoe", 2048, "gemm.tc.swiglu"): 218631424 + 19088128,
+    ("olmoe", 2048, "gemm.tc"): 109154304 + 32880896,
+}
 
 
 def dominant_roofline(cfg, M, kt, touched_avg, peaks, long_region):

@@ -144,8 +144,9 @@ def test_grouped_gemm_positive_control_flipped_nibble():
 # E4B_GEMM / E4B_TC_SHAPE switches, which apply to every call of the process):
 # wide = 2 x 128 weight rows x 256 routed rows, double = 2 x 128 x 128 with two
 # accumulator sets, narrow = 128 x 256 with two accumulator sets (plain
-# epilogue only; a SwiGLU call takes the wide shape).
-TC_SHAPES = ["wide", "double", "narrow"]
+# epilogue only; a SwiGLU call takes the wide shape), tmem = 2 x 128 x 192 with
+# the decoded weights in tensor memory (a LoRA or MXFP4 call takes the default).
+TC_SHAPES = ["wide", "double", "narrow", "tmem"]
 TC_CASES = CASES + [
     # several 256-row token tiles per group and a one-row group
     (3, 256, 512, [700, 1, 300], 500),
