@@ -426,14 +426,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
     // ------------------------------------------------------------ producer
     const uint64_t pol = l2_evict_first_policy();
     int issued = 0;
+    // Ring slot s and its pass ph of stage j; item (u, rb) of stage j < n_gu;
+    // chunk ch and row-block round rq of stage j >= n_gu -- all advanced per
+    // stage instead of divided out.
+    int s = 0, ph = 0, u = i0 / ipe, rb = i0 % ipe, ch = 0, rq = 0;
     for (int j = 0; j < T; ++j) {
-      const int s = j % RS;
-      if (j >= RS && !ring_wait(&empty[s], ((j / RS) - 1) & 1, &abort_s, p.err, kErrWaitEmpty)) break;
+      if (j >= RS && !ring_wait(&empty[s], ph ^ 1, &abort_s, p.err, kErrWaitEmpty)) break;
       unsigned char* st = ring + static_cast<uint32_t>(s) * slot;
       if (j < n_gu) {
         // 16 gate rows (block 0) and the matching 16 up rows (block 1): lanes
         // 0-3 / 8-11 the gate / up packed copies, 4-7 / 12-15 their absmax.
-        const int it = i0 + j, u = it / ipe, rb = it % ipe;
         const int64_t grow = static_cast<int64_t>(touched[u]) * 2 * I + rb * 16;
         if (lane == 0) mbar_arrive_expect_tx(&full[s], 32u * (H / 2) + 32u * KB * 4);
         __syncwarp();
@@ -442,20 +444,32 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
           copy_block_part(lane & 7, st + blk * 4 * cs_gu, st + am_gu + blk * 16 * as_gu, &full[s], p.gu_packed,
                           p.gu_absmax, H, grow + blk * I, pol);
         }
+        if (++rb == ipe) {
+          rb = 0;
+          ++u;
+        }
       } else {
         // One block of 16 down rows per expert: lane 8 ei + c issues copy c of expert ei.
-        const int jd = j - n_gu, ch = jd % nch, rb = bid + (jd / nch) * G;
+        const int rbd = bid + rq * G;
         const int u0 = ch * DPE, ne = min(DPE, nU - u0);
         if (lane == 0) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(ne) * (16u * (I / 2) + 16u * KBI * 4));
         __syncwarp();
         if (lane < 8 * ne) {
           const int ei = lane >> 3;
-          const int64_t row0 = static_cast<int64_t>(touched[u0 + ei]) * H + rb * 16;
+          const int64_t row0 = static_cast<int64_t>(touched[u0 + ei]) * H + rbd * 16;
           copy_block_part(lane & 7, st + ei * exp_dn, st + ei * exp_dn + am_dn, &full[s], p.dn_packed, p.dn_absmax, I,
                           row0, pol);
         }
+        if (++ch == nch) {
+          ch = 0;
+          ++rq;
+        }
       }
       ++issued;
+      if (++s == RS) {
+        s = 0;
+        ph ^= 1;
+      }
     }
     // Every copy in flight lands before the CTA may exit.
     for (int j = max(0, issued - RS); j < issued; ++j)
@@ -517,9 +531,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
         xr[q][hh][4] = b.x; xr[q][hh][5] = b.y; xr[q][hh][6] = b.z; xr[q][hh][7] = b.w;
       }
     }
-    for (int jj = gi; jj < n_gu; jj += kGroups) {
-      const int s = jj % RS;
-      ring_wait(&full[s], (jj / RS) & 1, &abort_s, p.err, kErrWaitFull);
+    // Ring slot s and pass ph of item jj (the ring depth is even, so a group's
+    // items stay on slots of one parity of index).
+    int s = gi, ph = 0;
+    for (int jj = gi; jj < n_gu; jj += kGroups, s += kGroups) {
+      if (s >= RS) {
+        s -= RS;
+        ph ^= 1;
+      }
+      ring_wait(&full[s], ph, &abort_s, p.err, kErrWaitFull);
       const unsigned char* st = ring + static_cast<uint32_t>(s) * slot;
       const float* am = reinterpret_cast<const float*>(st + am_gu);
       // Tile T: MMA row g = gate column 4 (g % 4) + 2T + g / 4 of the item
@@ -682,16 +702,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
     // not route to the pair's expert), loaded one stage ahead of their use.
     if (HSB > 0 && n_dn > 0) ring_wait(hbar, 0, &abort_s, p.err, kErrWaitFull);
     const uint16_t* hsrc = HSB > 0 ? reinterpret_cast<const uint16_t*>(smem + L.hs) : p.h;
-    auto load_h = [&](int jd, uint4 (&hb)[PPW][2]) {
+    // The warp's pair q is (expert pe[q] of the stage's chunk, k-block pk[q])
+    // in every stage.
+    int pe[PPW], pk[PPW];
+#pragma unroll
+    for (int q = 0; q < PPW; ++q) {
+      pe[q] = (warp + kMath * q) / KBI;
+      pk[q] = (warp + kMath * q) - pe[q] * KBI;
+    }
+    // h fragments of a stage of chunk ch (nothing when `live` is false).
+    auto load_h = [&](int ch, bool live, uint4 (&hb)[PPW][2]) {
 #pragma unroll
       for (int q = 0; q < PPW; ++q) hb[q][0] = hb[q][1] = make_uint4(0, 0, 0, 0);
-      if (jd >= n_dn) return;
-      const int u0 = (jd % nch) * DPE, np = min(DPE, nU - u0) * KBI;
+      if (!live) return;
+      const int u0 = ch * DPE, np = min(DPE, nU - u0) * KBI;
 #pragma unroll
       for (int q = 0; q < PPW; ++q) {
         const int pi = warp + kMath * q;
         if (pi < np) {
-          const int u = u0 + pi / KBI, kb = pi % KBI;
+          const int u = u0 + pe[q], kb = pk[q];
           const int sg = g < p.M ? slotmap[u * kMaxM + g] : -1;
           if (sg >= 0) {
             const uint4* src = reinterpret_cast<const uint4*>(hsrc + static_cast<int64_t>(sg) * I + kb * 64 + 16 * t);
@@ -706,15 +735,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
         }
       }
     };
-    auto compute = [&](int jd, const uint4 (&hb)[PPW][2]) {
-      const int j = n_gu + jd, s = j % RS;
-      ring_wait(&full[s], (j / RS) & 1, &abort_s, p.err, kErrWaitFull);
+    // Stage of ring slot s (pass ph), chunk ch of row-block round rbq.
+    auto compute = [&](int s, int ph, int ch, int rbq, const uint4 (&hb)[PPW][2]) {
+      ring_wait(&full[s], ph, &abort_s, p.err, kErrWaitFull);
       const unsigned char* st = ring + static_cast<uint32_t>(s) * slot;
-      const int ch = jd % nch, u0 = ch * DPE, np = min(DPE, nU - u0) * KBI;
+      const int u0 = ch * DPE, np = min(DPE, nU - u0) * KBI;
       // The warp's pairs two at a time (independent MMA chains interleaved).
       auto pair_in = [&](int q, uint2& w0, uint2& w1, float& s0, float& s1, float& s2, float& s3) {
-        const int pi = warp + kMath * q;
-        const int ei = pi / KBI, kb = pi % KBI, u = u0 + ei;
+        const int ei = pe[q], kb = pk[q], u = u0 + ei;
         // MMA row g = block row 4 (g % 4) + g / 4, row g + 8 = that + 2.
         const unsigned char* base = st + ei * exp_dn;
         const float* am = reinterpret_cast<const float*>(base + am_dn);
@@ -758,7 +786,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
       if (lane == 0) mbar_arrive(&empty[s]);
       if (ch == nch - 1) {
         // End of a row block: the 16 warps' sums in warp order -> out.
-        const int rbq = jd / nch;
         if (rbq > 0) named_bar(kBarMath, kMath * 32);  // the previous row block's sums are read
         red[warp * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
         acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
@@ -783,16 +810,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
         }
       }
     };
-    load_h(0, hA);
+    // Stage jd is ring stage n_gu + jd: slot s, pass ph; chunk ch of round rbq.
+    int s = n_gu % RS, ph = (n_gu / RS) & 1, ch = 0, rbq = 0;
+    load_h(0, n_dn > 0, hA);
 #pragma unroll 1
     for (int jd = 0; jd < n_dn; ++jd) {
-      load_h(jd + 1, hB);
-      compute(jd, hA);
+      const int ch1 = ch + 1 == nch ? 0 : ch + 1;
+      load_h(ch1, jd + 1 < n_dn, hB);
+      compute(s, ph, ch, rbq, hA);
 #pragma unroll
       for (int q = 0; q < PPW; ++q) {
         hA[q][0] = hB[q][0];
         hA[q][1] = hB[q][1];
       }
+      if (++s == RS) {
+        s = 0;
+        ph ^= 1;
+      }
+      if (ch1 == 0) ++rbq;
+      ch = ch1;
     }
   }
 }
