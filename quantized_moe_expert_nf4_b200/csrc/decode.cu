@@ -31,7 +31,8 @@
 // fragment loads touch lie in four different copies, on four different bank
 // groups.  Sixteen math warps decode and multiply: nibbles become bf16 pairs
 // through a per-lane replicated byte -> bf16x2 codebook table (lane l reads
-// only bank l) and feed mma.sync m16n8k16 with the weight rows as MMA rows and
+// only bank l; one byte permute forms a lookup's address) and feed mma.sync
+// m16n8k16 with the weight rows as MMA rows and
 // the <= 8 tokens as the 8 MMA columns.  Each MMA stays inside one 64-element
 // absmax block, so the block's fp32 absmax scales the products (no rounding of
 // the scale).
@@ -72,8 +73,12 @@ constexpr int kMaxDPE = 4;              // down experts per stage (8 copies each
 constexpr int kMaxKBI = kMath * kMaxPPW;  // k-blocks of a down row: I <= 3072
 constexpr int kMaxGrid = 1024;          // barrier slots in the workspace
 constexpr int kMaxStages = 32;
-constexpr uint32_t kLutBytes = 256 * 32 * 4;
+// Byte -> bf16x2 table: entry b for lane l at byte 256 b + 4 l, so one byte
+// permute of the packed word and 4 l forms the address.  The upper 128 bytes of
+// every entry hold the partial sums of both phases (red_offset).
+constexpr uint32_t kLutBytes = 256 * 256;
 constexpr uint32_t kRedBytes = kGroups * 2 * kGW * 2 * 32 * 16;  // phase 1: [group][parity][warp][tile][lane] float4
+static_assert(kRedBytes <= 256 * 128, "the partial sums fit the table's upper halves");
 constexpr int kBarMath = 3;             // named barrier of the 16 math warps
 
 struct FusedParams {
@@ -114,19 +119,15 @@ __host__ __device__ inline uint32_t am_stride(int KB) {
 __host__ __device__ inline uint32_t gu_stage_bytes(int H) { return 8 * copy_stride(H) + 8 * am_stride(H / 64); }
 __host__ __device__ inline uint32_t dn_block_bytes(int I) { return 4 * copy_stride(I) + 4 * am_stride(I / 64); }
 
-// Bytes of h staged in shared memory for phase 2 (all of it when it fits the
-// budget, else 0: the fragments then come from L2 into registers).  The
-// staging area is the part of phase 1's reduction buffer that phase 2's
-// reduction (one float4 per lane of 16 warps, 8 KB) leaves free.
-constexpr uint32_t kRedDnBytes = kMath * 32 * 16;
-constexpr uint32_t kHStageMax = kRedBytes - kRedDnBytes;
-__host__ __device__ inline uint32_t h_stage_bytes(int M, int k, int I) {
-  const uint32_t b = static_cast<uint32_t>(M * k) * static_cast<uint32_t>(I) * 2;
-  return b <= kHStageMax ? b : 0;
+// Float4 slot i of the partial sums (phase 1: [group][parity][warp][tile][lane];
+// phase 2: [warp][lane]) in the upper half of table entry i / 8: a quarter
+// warp's float4 accesses fill one 128-byte row.
+__host__ __device__ inline uint32_t red_offset(int i) {
+  return (static_cast<uint32_t>(i >> 3) << 8) + 128u + (static_cast<uint32_t>(i & 7) << 4);
 }
 
 struct Smem {
-  uint32_t lut, red, ids, w, uidx, touched, slotmap, xa, hs, bars, ring, total;
+  uint32_t lut, ids, w, uidx, touched, slotmap, xa, bars, ring, total;
 };
 
 __host__ __device__ inline Smem make_smem(int M, int k, int E, int r, int I, int stages, uint32_t slot) {
@@ -135,8 +136,6 @@ __host__ __device__ inline Smem make_smem(int M, int k, int E, int r, int I, int
   uint32_t o = 0;
   L.lut = o;
   o += kLutBytes;
-  L.red = o;
-  o += kRedBytes;
   L.ids = o;
   o = al(o + S * 4, 16);
   L.w = o;
@@ -149,9 +148,8 @@ __host__ __device__ inline Smem make_smem(int M, int k, int E, int r, int I, int
   o = al(o + S * kMaxM * 4, 16);
   L.xa = o;
   if (r > 0) o = al(o + S * r * 4, 16);
-  L.hs = L.red + kRedDnBytes;
   L.bars = o;
-  o = al(o + (2 * stages + 1 + 2 * kGroups) * 8, 16);
+  o = al(o + (2 * stages + 2 * kGroups) * 8, 16);
   L.ring = al(o, 128);
   L.total = L.ring + static_cast<uint32_t>(stages) * slot;
   return L;
@@ -174,14 +172,6 @@ __device__ __forceinline__ void mbar_arrive_cnt(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }
 
-// Bulk asynchronous copy global -> this CTA's shared memory, completing on `bar`
-// (both addresses 16-byte aligned, bytes a multiple of 16).
-__device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   smem_u32(smem_dst)),
-               "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
-               : "memory");
-}
 
 // L2 policy for data read exactly once per call (the packed weights): evict it
 // first, so the stream does not push out what the kernel reads again (its h,
@@ -192,6 +182,8 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   return pol;
 }
 
+// Bulk asynchronous copy global -> this CTA's shared memory, completing on `bar`
+// (both addresses 16-byte aligned, bytes a multiple of 16), with an L2 policy.
 __device__ __forceinline__ void bulk_g2s_stream(void* smem_dst, const void* gmem_src, uint32_t bytes, uint64_t* bar,
                                                 uint64_t pol) {
   asm volatile(
@@ -213,11 +205,6 @@ __device__ __forceinline__ unsigned long long ld_relaxed_gpu(const unsigned long
   return v;
 }
 
-__device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
 
 // Bounded wait on a ring barrier.  Once any wait of the CTA has given up
 // (*abort set), every later wait returns false at once.
@@ -247,13 +234,13 @@ __device__ __forceinline__ bool ring_wait(uint64_t* bar, uint32_t parity, volati
 // bf16 pairs are the A fragment (row g / g+8, k slots 2t..2t+1 and 2t+8..2t+9)
 // and x words 2j, 2j+1 the B fragment, so both operands see the same physical
 // k for every slot.  The table entry of byte b for lane l is at byte
-// b * 128 + 4 l of the table, i.e. at (b << 7) | lane4: one shift and one
-// three-input logic op per lookup.
+// 256 b + 4 l of the table: one byte permute puts byte b of the packed word
+// above lane4 = 4 l (byte 0), so a lookup costs one ALU op and one load.
 __device__ __forceinline__ void block_mma(const unsigned char* __restrict__ lut, uint32_t lane4, uint2 w0, uint2 w1,
                                           const uint32_t* xw, float d[4]) {
   auto pair = [&](uint32_t word, int byte) {
-    const uint32_t sh = byte == 0 ? (word << 7) : (word >> (8 * byte - 7));
-    return *reinterpret_cast<const uint32_t*>(lut + ((sh & 0x7f80u) | lane4));
+    const uint32_t ad = __byte_perm(word, lane4, 0x5504u | (static_cast<uint32_t>(byte) << 4));
+    return *reinterpret_cast<const uint32_t*>(lut + ad);
   };
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
@@ -270,8 +257,8 @@ __device__ __forceinline__ void block_mma2(const unsigned char* __restrict__ lut
                                            uint2 w1a, const uint32_t* xa, uint2 w0b, uint2 w1b, const uint32_t* xb,
                                            float da[4], float db[4]) {
   auto pair = [&](uint32_t word, int byte) {
-    const uint32_t sh = byte == 0 ? (word << 7) : (word >> (8 * byte - 7));
-    return *reinterpret_cast<const uint32_t*>(lut + ((sh & 0x7f80u) | lane4));
+    const uint32_t ad = __byte_perm(word, lane4, 0x5504u | (static_cast<uint32_t>(byte) << 4));
+    return *reinterpret_cast<const uint32_t*>(lut + ad);
   };
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
@@ -296,8 +283,9 @@ __device__ __forceinline__ void route_one(const FusedParams& p, int t, int* ids_
 }
 
 // Prologue: warps < M route one token each while the other warps build the
-// byte -> bf16x2 table of the stacks' codebook (NF4 or FP4) (entry b of lane l at b * 32 + l: low half the
-// high nibble's value, i.e. element 2i, high half element 2i+1).  Then the
+// byte -> bf16x2 table of the stacks' codebook (NF4 or FP4) (entry b of lane l
+// at word 64 b + l: low half the high nibble's value, i.e. element 2i, high
+// half element 2i+1).  Then the
 // touched experts (ascending id) and slotmap[u][t] = slot of token t in expert
 // touched[u] (or -1).
 __device__ void prologue(const FusedParams& p, uint32_t* lut, int* ids_s, float* w_s, int* uidx, int* touched,
@@ -312,7 +300,7 @@ __device__ void prologue(const FusedParams& p, uint32_t* lut, int* ids_s, float*
     for (int b = warp - p.M; b < 256; b += kWarps - p.M) {
       const float hi = __shfl_sync(0xffffffffu, cbl, b >> 4);
       const float lo = __shfl_sync(0xffffffffu, cbl, b & 15);
-      lut[b * 32 + lane] = pack_bf16x2(hi, lo);
+      lut[b * 64 + lane] = pack_bf16x2(hi, lo);
     }
   }
   __syncthreads();
@@ -370,7 +358,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
   const uint32_t slot = al(max(gu_stage_bytes(H), static_cast<uint32_t>(DPE) * exp_dn), 128);
   const Smem L = make_smem(p.M, p.k, p.E, p.r, p.I, RS, slot);
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L.lut);
-  float4* red = reinterpret_cast<float4*>(smem + L.red);
+  unsigned char* lutb = smem + L.lut;
+  auto red_at = [&](int i) { return reinterpret_cast<float4*>(lutb + red_offset(i)); };
   int* ids_s = reinterpret_cast<int*>(smem + L.ids);
   float* w_s = reinterpret_cast<float*>(smem + L.w);
   int* uidx = reinterpret_cast<int*>(smem + L.uidx);
@@ -379,9 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
   float* xa = reinterpret_cast<float*>(smem + L.xa);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);  // stage landed
   uint64_t* empty = full + RS;                                   // stage consumed (16 arrivals)
-  uint64_t* hbar = empty + RS;                                   // h staged for phase 2
-  uint64_t* rfree = hbar + 1;                                    // [group][parity] partials read by the finisher
-  const uint32_t HSB = h_stage_bytes(p.M, p.k, I);
+  uint64_t* rfree = empty + RS;                                  // [group][parity] partials read by the finisher
   unsigned char* ring = smem + L.ring;
   __shared__ int nU_s;
   __shared__ volatile int abort_s;
@@ -398,7 +385,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kMath);
     }
-    mbar_init(hbar, 1);
     for (int i = 0; i < 2 * kGroups; ++i) {
       mbar_init(&rfree[i], 1);
       fin_cnt[i >> 1][i & 1] = 0;
@@ -583,9 +569,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
       // has read it.
       const int iq = jj / kGroups, par = iq & 1;
       if (iq >= 2) ring_wait(&rfree[gi * 2 + par], ((iq >> 1) - 1) & 1, &abort_s, p.err, kErrWaitFull);
-      float4* rp = red + (((gi * 2 + par) * kGW + wi) * 2) * 32 + lane;
-      rp[0] = make_float4(c[0][0], c[0][1], c[0][2], c[0][3]);
-      rp[32] = make_float4(c[1][0], c[1][1], c[1][2], c[1][3]);
+      const int ri = (((gi * 2 + par) * kGW + wi) * 2) * 32 + lane;
+      *red_at(ri) = make_float4(c[0][0], c[0][1], c[0][2], c[0][3]);
+      *red_at(ri + 32) = make_float4(c[1][0], c[1][1], c[1][2], c[1][3]);
       __syncwarp();
       int last = 0;
       if (lane == 0) {
@@ -602,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
         for (int T = 0; T < 2; ++T) {
           float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
           for (int w = 0; w < kGW; ++w) {
-            const float4 v = red[(((gi * 2 + par) * kGW + w) * 2 + T) * 32 + lane];
+            const float4 v = *red_at((((gi * 2 + par) * kGW + w) * 2 + T) * 32 + lane);
             sum.x += v.x;
             sum.y += v.y;
             sum.z += v.z;
@@ -684,13 +670,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
         }
       }
     }
-    if (HSB > 0 && n_dn > 0 && lane == 0) {
-      // Small h: all of it into shared memory with one bulk copy (the async
-      // proxy reads what the generic proxy of the other CTAs wrote).
-      asm volatile("fence.proxy.async;" ::: "memory");
-      mbar_arrive_expect_tx(hbar, HSB);
-      bulk_g2s(smem + L.hs, p.h, HSB, hbar);
-    }
   }
   named_bar(kBarMath, kMath * 32);
 
@@ -698,10 +677,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
   {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     uint4 hA[PPW][2], hB[PPW][2];
-    // h fragments of stage jd for this warp's pairs (zeros where token g does
-    // not route to the pair's expert), loaded one stage ahead of their use.
-    if (HSB > 0 && n_dn > 0) ring_wait(hbar, 0, &abort_s, p.err, kErrWaitFull);
-    const uint16_t* hsrc = HSB > 0 ? reinterpret_cast<const uint16_t*>(smem + L.hs) : p.h;
+    // h fragments of a stage for this warp's pairs (zeros where token g does
+    // not route to the pair's expert), read from L2 one stage ahead of their use.
     // The warp's pair q is (expert pe[q] of the stage's chunk, k-block pk[q])
     // in every stage.
     int pe[PPW], pk[PPW];
@@ -723,14 +700,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
           const int u = u0 + pe[q], kb = pk[q];
           const int sg = g < p.M ? slotmap[u * kMaxM + g] : -1;
           if (sg >= 0) {
-            const uint4* src = reinterpret_cast<const uint4*>(hsrc + static_cast<int64_t>(sg) * I + kb * 64 + 16 * t);
-            if (HSB > 0) {
-              hb[q][0] = src[0];
-              hb[q][1] = src[1];
-            } else {
-              hb[q][0] = __ldcg(src);
-              hb[q][1] = __ldcg(src + 1);
-            }
+            const uint4* src = reinterpret_cast<const uint4*>(p.h + static_cast<int64_t>(sg) * I + kb * 64 + 16 * t);
+            hb[q][0] = __ldcg(src);
+            hb[q][1] = __ldcg(src + 1);
           }
         }
       }
@@ -787,13 +759,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedParams p
       if (ch == nch - 1) {
         // End of a row block: the 16 warps' sums in warp order -> out.
         if (rbq > 0) named_bar(kBarMath, kMath * 32);  // the previous row block's sums are read
-        red[warp * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *red_at(warp * 32 + lane) = make_float4(acc[0], acc[1], acc[2], acc[3]);
         acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
         named_bar(kBarMath, kMath * 32);
         if (warp == rbq % kMath) {
           float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
           for (int w = 0; w < kMath; ++w) {
-            const float4 v = red[w * 32 + lane];
+            const float4 v = *red_at(w * 32 + lane);
             sum.x += v.x;
             sum.y += v.y;
             sum.z += v.z;

@@ -118,14 +118,14 @@ def _plan(M, k, E, H, I, r):
     ppw = -(-(dpe * KBI) // 16)
     slot = _al(max(gu, dpe * dn), 128)
     S = M * k
-    o = 256 * 32 * 4 + 2 * 2 * 8 * 2 * 32 * 16
+    o = 256 * 256  # the byte -> bf16x2 table, the partial sums in its entries' upper halves
     for n in (S * 4, S * 4, E * 4, S * 4, S * 8 * 4):
         o = _al(o + n, 16)
     if r:
         o = _al(o + S * r * 4, 16)
     fixed = _al(o, 128) + 2 * 32 * 8
     stages = min((SMEM_LIMIT - fixed) // slot, 32) & ~1
-    ring = _al(_al(o + (2 * stages + 1 + 4) * 8, 16), 128)
+    ring = _al(_al(o + (2 * stages + 4) * 8, 16), 128)
     return dict(spw=spw, ppw=ppw, dpe=dpe, slot=slot, stages=stages, ring=ring, total=ring + stages * slot)
 
 
@@ -218,6 +218,41 @@ def test_decode_fused_plan_copies_and_reads_stay_in_bounds(shape):
                         for row in (rr, rr + 2):
                             a = ei * exp + amd + cg * _am_stride(KBI) + (row * KBI + kb) * 4
                             assert set(range(a, a + 4)) <= written
+
+
+def _lut_address(word, byte, lane):
+    """csrc/decode.cu block_mma: __byte_perm(word, 4 lane, 0x5504 | byte << 4)."""
+    return _byte_perm(word, 4 * lane, 0x5504 | (byte << 4))
+
+
+def _red_offset(i):
+    return ((i >> 3) << 8) + 128 + ((i & 7) << 4)
+
+
+def test_decode_table_lookup_address_and_partial_sum_slots():
+    """The decode table: the byte permute of a packed word puts byte `byte` of
+    the word at bits 8-15 above 4 lane, i.e. entry b of lane l at 256 b + 4 l;
+    a warp's 32 lookups hit 32 distinct banks whatever the bytes; every address
+    lies in the lower half of its 256-byte entry.  The partial sums take the
+    upper halves: 2048 float4 slots (phase 1's [group][parity][warp][tile][lane]
+    and phase 2's [warp][lane]) inside the 64 KB table, disjoint from the
+    entries and from one another, each quarter warp's slots one 128-byte row."""
+    rng = np.random.default_rng(5)
+    for _ in range(200):
+        words = rng.integers(0, 2**32, size=32, dtype=np.uint64)
+        for byte in range(4):
+            addrs = [_lut_address(int(w), byte, lane) for lane, w in enumerate(words)]
+            for lane, (w, a) in enumerate(zip(words, addrs)):
+                b = (int(w) >> (8 * byte)) & 255
+                assert a == 256 * b + 4 * lane
+            assert len({(a // 4) % 32 for a in addrs}) == 32
+            assert all(a % 256 < 128 and a < 256 * 256 for a in addrs)
+    slots = [_red_offset(i) for i in range(2 * 2 * 8 * 2 * 32)]
+    assert all(o % 256 >= 128 and o + 16 <= 256 * 256 for o in slots)
+    assert len(set(slots)) == len(slots)
+    for q in range(0, len(slots), 8):
+        row = slots[q:q + 8]
+        assert row == list(range(row[0], row[0] + 128, 16))
 
 
 @pytest.mark.parametrize("K", [128, 192, 320, 448, 704, 768, 1024, 2048, 2880, 3072, 4096])
