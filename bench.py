@@ -476,6 +476,7 @@ def replicas_for(cfg, M):
 # is now, keyed by (layer config, M, kernel); a kernel changed since its capture
 # has no entry.
 MEASURED_TRAFFIC = {
+    ("olmoe", 1, "decode.fused"): 28421888 + 0,
     ("olmoe", 2048, "gemm.tc.swiglu"): 218631424 + 19088128,
     ("olmoe", 2048, "gemm.tc"): 109154304 + 32880896,
 }
