@@ -1,5 +1,6 @@
-"""CPU models of the index maps of the GPU kernels (regression pins; the decode
-kernels' models are in test_model_decode_ring.py).
+"""CPU models of the index maps of the GPU kernels (regression pins): the fused
+decode kernel's fragment mapping, shared-memory plan, copies and table lookups,
+and the tensor-core decoders.
 
 Each model restates, in numpy and exact arithmetic, how a kernel's threads
 place data -- which packed bytes a thread decodes, where it stores them, which
