@@ -396,25 +396,31 @@ class Bench:
         return {n: (ms / max(c, 1), c) for n, (ms, c) in res.items()}
 
     def e2e(self, K):
-        """Public call with host buffers, per step: H2D copies of the step's inputs
+        """Public call with host buffers, per step: H2D copy of the step's inputs
         from pinned memory, the forward, and a D2H copy of its output into pinned
         memory.  At decode sizes (M <= 8) the host's per-call work sets the pace, so
-        the copies are issued in the forward's own stream with nothing else per
-        step; above, the copies run on their own streams and overlap the forwards
-        (e2e_pipelined)."""
+        x and the router logits travel in one copy (one pinned staging buffer per
+        replica holding both, the forward reading views of one device buffer) in
+        the forward's own stream, with nothing else per step; above, the copies run
+        on their own streams and overlap the forwards (e2e_pipelined)."""
         if self.M > 8:
             return self.e2e_pipelined(K)
         torch, cfg, M = self.torch, self.cfg, self.M
         R = len(self.layers)
-        hx = [x.cpu().pin_memory() for x in self.xs]
-        hl = [l.cpu().pin_memory() for l in self.logits]
+        nx, nl = M * cfg.H * 2, M * cfg.E * 4              # bytes of x (bf16) and logits (fp32); nx % 16 == 0
+        hin = []
+        for x, l in zip(self.xs, self.logits):
+            buf = torch.empty(nx + nl, dtype=torch.uint8).pin_memory()
+            buf[:nx].copy_(x.cpu().view(torch.uint8).reshape(-1))
+            buf[nx:].copy_(l.cpu().view(torch.uint8).reshape(-1))
+            hin.append(buf)
         ho = [torch.empty((M, cfg.H), dtype=torch.bfloat16).pin_memory() for _ in range(R)]
-        dx = torch.empty_like(self.xs[0])
-        dl = torch.empty_like(self.logits[0])
+        din = torch.empty(nx + nl, dtype=torch.uint8, device=self.xs[0].device)
+        dx = din[:nx].view(torch.bfloat16).view(M, cfg.H)
+        dl = din[nx:].view(torch.float32).view(M, cfg.E)
         do = torch.empty_like(self.outs[0])
         for i in range(min(3, K)):
-            dx.copy_(hx[i % R], non_blocking=True)
-            dl.copy_(hl[i % R], non_blocking=True)
+            din.copy_(hin[i % R], non_blocking=True)
             self.e4b.e4b_moe_expert_forward(dx, dl, cfg.k, True, self.layers[i % R].stack, do, self.ws)
             ho[i % R].copy_(do, non_blocking=True)
         torch.cuda.synchronize()
@@ -422,16 +428,13 @@ class Bench:
         a.record()
         for i in range(K):
             r = i % R
-            dx.copy_(hx[r], non_blocking=True)
-            dl.copy_(hl[r], non_blocking=True)
+            din.copy_(hin[r], non_blocking=True)
             self.e4b.e4b_moe_expert_forward(dx, dl, cfg.k, True, self.layers[r].stack, do, self.ws)
             ho[r].copy_(do, non_blocking=True)
         b.record()
         torch.cuda.synchronize()
         t = a.elapsed_time(b) / 1e3
-        h2d = M * cfg.H * 2 + M * cfg.E * 4
-        d2h = M * cfg.H * 2
-        return M * cfg.k * K / t, h2d, d2h
+        return M * cfg.k * K / t, nx + nl, M * cfg.H * 2
 
     def e2e_pipelined(self, K):
         """Public call with host buffers, per step: H2D copies of the step's inputs
@@ -644,8 +647,9 @@ def measure(args, name, rank, world, dist, peaks, primary, e2e_steps=None):
         ev, h2d, d2h = b.e2e(K)
         ev = reduce_over_ranks(ev, dist, dev, "min") * world
         res["e2e"] = {"value": ev, "unit": "routed_tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                      "how": ("per step: H2D of the inputs from pinned memory, the public forward call, D2H of "
-                              "the output into pinned memory, all in the forward's stream" if b.M <= 8 else
+                      "how": ("per step: one H2D copy of x and the logits from one pinned buffer, the public "
+                              "forward call on views of one device buffer, D2H of the output into pinned memory, "
+                              "all in the forward's stream" if b.M <= 8 else
                               "per step: H2D of the inputs from pinned memory on a copy stream (double-buffered), "
                               "the public forward call, D2H of the output into pinned memory on a second copy "
                               "stream; copies of neighbouring steps overlap the forward")}
