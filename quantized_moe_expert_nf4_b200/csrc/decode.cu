@@ -32,10 +32,9 @@
 // groups.  Sixteen math warps decode and multiply: nibbles become bf16 pairs
 // through a per-lane replicated byte -> bf16x2 codebook table (lane l reads
 // only bank l; one byte permute forms a lookup's address) and feed mma.sync
-// m16n8k16 with the weight rows as MMA rows and
-// the <= 8 tokens as the 8 MMA columns.  Each MMA stays inside one 64-element
-// absmax block, so the block's fp32 absmax scales the products (no rounding of
-// the scale).
+// m16n8k16 with the weight rows as MMA rows and the <= 8 tokens as the 8 MMA
+// columns.  Each MMA stays inside one 64-element absmax block, so the block's
+// fp32 absmax scales the products (no rounding of the scale).
 //
 // The grid barrier needs no initialised workspace: a 64-bit epoch word sits
 // beside one slot per CTA.  Every CTA reads the epoch e at its start, publishes
