@@ -549,3 +549,58 @@ def test_tensor_memory_decoders_fill_the_a_operand_the_mma_reads():
             for lane in range(128):
                 row = [x for col in range(8) for x in tmem[(lane, h * 32 + kk * 8 + col)]]
                 assert row == list(W[h * 128 + lane, kk * 16: kk * 16 + 16]), (h, kk, lane)
+
+
+@pytest.mark.parametrize("RS", [2, 4, 6, 32])
+def test_decode_stage_indices_advance_like_their_definitions(RS):
+    """csrc/decode.cu advances ring slots, passes, items and chunks per stage
+    instead of dividing: the copy-issuing warp's (s, ph, u, rb, ch, rq), each
+    group's (s, ph) over its items jj = gi, gi + 2, ..., and the down loop's
+    (s, ph, ch, rbq) must equal j % RS, (j / RS) & 1, (i0 + j) / ipe and
+    % ipe, jd % nch and jd / nch of every stage."""
+    rng = np.random.default_rng(RS)
+    for _ in range(300):
+        ipe = int(rng.integers(1, 200))
+        i0 = int(rng.integers(0, 5000))
+        n_gu = int(rng.integers(0, 40))
+        nch = int(rng.integers(1, 9))
+        n_dn = nch * int(rng.integers(0, 6))
+        # producer
+        s = ph = ch = rq = 0
+        u, rb = i0 // ipe, i0 % ipe
+        for j in range(n_gu + n_dn):
+            assert (s, ph) == (j % RS, (j // RS) & 1)
+            if j < n_gu:
+                assert (u, rb) == ((i0 + j) // ipe, (i0 + j) % ipe)
+                rb += 1
+                if rb == ipe:
+                    rb, u = 0, u + 1
+            else:
+                jd = j - n_gu
+                assert (ch, rq) == (jd % nch, jd // nch)
+                ch += 1
+                if ch == nch:
+                    ch, rq = 0, rq + 1
+            s += 1
+            if s == RS:
+                s, ph = 0, ph ^ 1
+        # phase 1: group gi takes items gi, gi + 2, ...
+        for gi in range(2):
+            s, ph = gi, 0
+            for jj in range(gi, n_gu, 2):
+                if s >= RS:
+                    s, ph = s - RS, ph ^ 1
+                assert (s, ph) == (jj % RS, (jj // RS) & 1)
+                s += 2
+        # phase 2: stage jd is ring stage n_gu + jd
+        s, ph, ch, rbq = n_gu % RS, (n_gu // RS) & 1, 0, 0
+        for jd in range(n_dn):
+            j = n_gu + jd
+            assert (s, ph, ch, rbq) == (j % RS, (j // RS) & 1, jd % nch, jd // nch)
+            ch1 = 0 if ch + 1 == nch else ch + 1
+            s += 1
+            if s == RS:
+                s, ph = 0, ph ^ 1
+            if ch1 == 0:
+                rbq += 1
+            ch = ch1
